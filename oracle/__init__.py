@@ -1,0 +1,31 @@
+"""Reference oracle for the GPTQ-family per-layer solve: TEST INFRASTRUCTURE ONLY.
+
+Plain, slow, fp64 CPU code that states what the solve computes, step by step, in
+the notation of the source pages. Only the test suite, the smoke check and the
+benchmark's CPU-baseline leg may import it; the library path never does, and the
+two share no code.
+
+Pins (tests/test_oracle_pins.py) tie every function here to something other than
+itself: the worked examples printed on the pages, closed forms, special cases,
+brute force and independent least-squares solves. One reading is only partly
+pinned and says so where it is defined: which weight value multiplies the
+GPTAQ residual row (``gptaq`` arguments below).
+"""
+
+from .gptq_oracle import (  # noqa: F401
+    gram,
+    cross_gram,
+    dead_and_damp,
+    is_positive_definite,
+    symmetric_scale,
+    quantize_codes,
+    dequantize,
+    obq_sweep,
+    upper_factor,
+    gptaq_p1,
+    row_form_sweep,
+    replay_row_form,
+    layer_error,
+    solve_layer,
+    brute_force_best,
+)

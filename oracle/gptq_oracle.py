@@ -1,0 +1,403 @@
+"""fp64 reference of the GPTQ per-layer solve and its GPTAQ / grouped extensions.
+
+TEST INFRASTRUCTURE ONLY: imported by the tests, the smoke check and the
+benchmark's CPU-baseline leg, never by the library.
+
+Sources (cited by title and section):
+  [GPTQ blog]  "GPTQ：量化一个权重之后怎样补偿输出误差" (charlestar.github.io),
+               sections "Calibration 让量化看见输入方向", "两个权重怎样互相补偿",
+               "一次约束补偿的公式从哪里来", "为什么 Cholesky Factor 不能当作原始逆矩阵",
+               "GPTQ 怎样把逐个补偿变成可扩展算法", "Damping 与两个不同的分组参数",
+               "局部连续最优为什么不保证最终优于 RTN", "落在格点上与真正存成低位权重是两步".
+  [ResComp]    "Rethinking Residual Errors in Compensation-based LLM Quantization"
+               (papernotes.org), "关键设计" items 1-3 (column objective, residual split,
+               neuron decomposition with P1/P2).
+  [GPTAQ]      "GPTAQ: Efficient Finetuning-Free Quantization for Asymmetric
+               Calibration" (Paper-Notes), "关键设计" (asymmetric objective, OBC
+               closed form, channel parallelism).
+  [G2PTQ]      "G²PTQ: Improving LLM Post-Training Quantization with Generalized
+               Gradient Compensation" (agihunt.info summary): output-channel groups
+               sharing one Hessian per group.
+
+Layout. The blog writes X (M tokens x K inputs), W (K x N), Y = XW. Here weights are
+stored as nn.Linear does, W[n][k] (N x K): row n is the blog's column w of output
+channel n. Every function takes and returns float64 numpy arrays.
+"""
+
+from __future__ import annotations
+
+import itertools
+
+import numpy as np
+
+
+# --------------------------------------------------------------------------------------
+# Statistics: Gram / Hessian
+# --------------------------------------------------------------------------------------
+
+def gram(X, s=None):
+    """H = 2 X^T diag(s) X.
+
+    [GPTQ blog] "Calibration 让量化看见输入方向": the layer objective ||X(w_hat - w)||^2 has
+    Hessian 2X^T X, one K x K matrix shared by every output channel and accumulated
+    batch by batch. The factor 2 is fixed by the two-weight example of
+    "两个权重怎样互相补偿" (X = [[1, .5], [0, sqrt(3)/2]] gives H = [[2, 1], [1, 2]]).
+    [G2PTQ] groups of output channels each carry their own Hessian; with a per-token
+    weight s_m the group Hessian is 2 sum_m s_m x_m x_m^T.
+    """
+    X = np.asarray(X, dtype=np.float64)
+    if s is None:
+        return 2.0 * (X.T @ X)
+    s = np.asarray(s, dtype=np.float64)
+    return 2.0 * (X.T @ (X * s[:, None]))
+
+
+def cross_gram(X_quant, X_fp):
+    """C = 2 dX^T X with dX = X_fp - X_quant (tokens x inputs).
+
+    [ResComp] item 2 splits the residual as r1 = w (X~ - X) with X~ the
+    full-precision stream and X the quantised stream; item 3 precomputes the
+    cross statistic dX X^T (their row convention) from dX = X~ - X. In the K x N
+    convention that statistic is dX^T X; it carries the same factor 2 as H so that
+    the GPTAQ update below needs no extra constant.
+    """
+    Xq = np.asarray(X_quant, dtype=np.float64)
+    dX = np.asarray(X_fp, dtype=np.float64) - Xq
+    return 2.0 * (dX.T @ Xq)
+
+
+# --------------------------------------------------------------------------------------
+# Dead coordinates and damping
+# --------------------------------------------------------------------------------------
+
+def dead_and_damp(H, percdamp):
+    """Dead-coordinate fix, then damping. Returns (H_d, dead mask).
+
+    [GPTQ blog] "Damping 与两个不同的分组参数": a coordinate whose Hessian diagonal is
+    zero is "dead": its diagonal is adjusted and its weights are zeroed. Then the
+    diagonal increment percdamp * mean(diag H) (default ratio 0.01) is added.
+    Reading: the dead diagonal is set to 1 and the fix comes before the damping, so
+    the mean includes those 1s. (With a Gram H the dead row and column are zero, so
+    the value chosen does not change the solve.)
+    """
+    H = np.array(H, dtype=np.float64, copy=True)
+    K = H.shape[0]
+    dead = np.diag(H) == 0.0
+    idx = np.arange(K)
+    H[idx[dead], idx[dead]] = 1.0
+    damp = percdamp * np.mean(np.diag(H))
+    H[idx, idx] += damp
+    return H, dead
+
+
+def is_positive_definite(H):
+    """True when every Cholesky pivot of H is clearly positive.
+
+    [GPTQ blog] "Damping 与两个不同的分组参数": with only the input [1, 1] observed,
+    X^T X has rank 1 and cannot be inverted; the damping term makes it PD. The
+    blog's self-check ("用标准库核对二维补偿") refuses a non-PD Hessian instead of
+    repairing it. Reading: a pivot d_j is "clearly positive" when it exceeds the
+    Cholesky backward-error size K * eps * H_jj (eps = 2^-52 here); an exactly
+    singular H whose rounded pivot lands at +1e-16 is then refused too.
+    """
+    H = np.asarray(H, dtype=np.float64)
+    K = H.shape[0]
+    try:
+        L = np.linalg.cholesky(H)
+    except np.linalg.LinAlgError:
+        return False
+    pivots = np.diag(L) ** 2
+    return bool(np.all(pivots > K * np.finfo(np.float64).eps * np.diag(H)))
+
+
+# --------------------------------------------------------------------------------------
+# Quantisation grid
+# --------------------------------------------------------------------------------------
+
+def symmetric_scale(W, bits):
+    """Per-output-channel symmetric scale s_n and the zero point z.
+
+    [G2PTQ] weights use symmetric per-channel quantisation; [GPTQ blog]
+    "两个权重怎样互相补偿" fixes, for 4 bits, the grid {-8..7} written as unsigned codes
+    0..15 with zero point 8. Reading (the formula is not printed): the min-max
+    symmetric scale s = 2 * max_k |W[n, k]| / (2^b - 1), zero point z = 2^(b-1), so
+    the representable set is s * {-2^(b-1) .. 2^(b-1) - 1}. An all-zero channel takes
+    s = 1 (any positive value reconstructs it exactly).
+    """
+    W = np.asarray(W, dtype=np.float64)
+    amax = np.max(np.abs(W), axis=1)
+    s = 2.0 * amax / (2 ** bits - 1)
+    s[amax == 0.0] = 1.0
+    return s, 2 ** (bits - 1)
+
+
+def quantize_codes(w, s, bits):
+    """Integer codes c = clamp(round_half_even(w / s) + z, 0, 2^b - 1).
+
+    [GPTQ blog] "两个权重怎样互相补偿": nearest grid point with ties to even ("最近偶数舍入");
+    codes are unsigned 0..2^b-1 around the zero point z = 2^(b-1).
+    """
+    z = 2 ** (bits - 1)
+    c = np.rint(np.asarray(w, dtype=np.float64) / s) + z
+    return np.clip(c, 0, 2 ** bits - 1)
+
+
+def dequantize(c, s, bits):
+    """Reconstruction s (c - z).
+
+    [GPTQ blog] "落在格点上与真正存成低位权重是两步": the quantiser returns the
+    reconstructed value s(q - z) in floating point; codes are a separate artefact.
+    """
+    return np.asarray(s, dtype=np.float64) * (np.asarray(c, dtype=np.float64) - 2 ** (bits - 1))
+
+
+# --------------------------------------------------------------------------------------
+# The sweep in explicit OBQ form (no Cholesky, no lazy batching)
+# --------------------------------------------------------------------------------------
+
+def obq_sweep(H_d, W, s, bits, mode="schur", C=None, return_trace=False):
+    """Quantise coordinates 0..K-1 in order, compensating the free set each step.
+
+    [GPTQ blog] "一次约束补偿的公式从哪里来": with free set F and P_F = (H[F, F])^-1, fixing
+    coordinate q at its grid value Q(w_q) with r = w_q - Q(w_q) moves the free
+    coordinates by delta_F = -r P_F[:, q] / (P_F)_qq (this includes q itself, which
+    lands exactly on Q(w_q)); the objective rises by r^2 / (2 (P_F)_qq).
+    "为什么 Cholesky Factor 不能当作原始逆矩阵": after q is fixed the next free-set
+    inverse is the Schur update P_F - P_F[:, q] P_F[q, :] / (P_F)_qq, not a
+    sub-block of the original inverse.
+    "GPTQ 怎样把逐个补偿变成可扩展算法": all output channels use the same order.
+
+    mode "schur" carries P by the Schur update; mode "direct" re-inverts H_d[F, F]
+    at every step (small K only).
+
+    C (optional) adds the GPTAQ residual term ([GPTAQ] "非对称校准目标" and
+    "基于最优脑压缩的闭式解"; [ResComp] item 2, Δw = ... + r X^T H^-1_{-q} with
+    r1 = w^(q)(X~ - X)). By the neuron decomposition of [ResComp] item 3 the part of
+    r1 owed to coordinate q is applied at q's step, restricted to the coordinates
+    still free after q (F' = F minus q):
+        w_F' += w_q^pre * C[q, F'] (H_d[F', F'])^-1,
+    with w_q^pre the value of coordinate q at its step, before rounding (reading;
+    r1 is written with the current weights w^(q)). The single-step form is pinned by
+    an independent least-squares solve on the token matrices; which w multiplies
+    the row is a reading no printed value pins.
+
+    Returns (codes, W_hat, loss) with loss[n] = sum_q r^2 / (2 (P_F)_qq), and the
+    per-step weights when return_trace.
+    """
+    H_d = np.asarray(H_d, dtype=np.float64)
+    W = np.array(W, dtype=np.float64, copy=True)
+    N, K = W.shape
+    s = np.asarray(s, dtype=np.float64)
+    codes = np.zeros((N, K))
+    loss = np.zeros(N)
+    trace = []
+    P = np.linalg.inv(H_d) if mode == "schur" else None
+    for q in range(K):
+        if mode == "direct":
+            P = np.linalg.inv(H_d[q:, q:])
+        # P is the inverse over F = {q, ..., K-1}; local index 0 is coordinate q.
+        w_pre = W[:, q].copy()
+        c = quantize_codes(w_pre, s, bits)
+        target = dequantize(c, s, bits)
+        r = w_pre - target
+        p_qq = P[0, 0]
+        W[:, q:] -= np.outer(r / p_qq, P[:, 0])
+        W[:, q] = target                      # fixed exactly, not compensated twice
+        loss += r * r / (2.0 * p_qq)
+        codes[:, q] = c
+        if q + 1 < K:
+            P_next = P[1:, 1:] - np.outer(P[1:, 0], P[0, 1:]) / p_qq
+            if C is not None:
+                W[:, q + 1:] += np.outer(w_pre, C[q, q + 1:] @ P_next)
+            P = P_next
+        if return_trace:
+            trace.append(W.copy())
+    if return_trace:
+        return codes, W, loss, trace
+    return codes, W, loss
+
+
+# --------------------------------------------------------------------------------------
+# Cholesky row form (used for comparison with the GPU's factor and for replay)
+# --------------------------------------------------------------------------------------
+
+def upper_factor(H_d):
+    """U upper triangular with U^T U = H_d^-1.
+
+    [GPTQ blog] "为什么 Cholesky Factor 不能当作原始逆矩阵": GPTQ reads the inverse through
+    an upper triangular U with U^T U = H^-1; row q of U carries the free-set
+    inverse at q's step, (P_F)_qq = U_qq^2. Built here from the library inverse and
+    Cholesky routines.
+    """
+    P = np.linalg.inv(np.asarray(H_d, dtype=np.float64))
+    P = 0.5 * (P + P.T)
+    return np.linalg.cholesky(P).T
+
+
+def gptaq_p1(C, U):
+    """P1 = [(C U^T) ⊙ M] U with M the strict upper mask (column index > row index).
+
+    [ResComp] item 3: P1 = [(dX X^T L) ⊙ M_U] L^T with H^-1 = L L^T. In the K x N
+    convention L = U^T. Reading: M_U is strict. Row q then equals
+    C[q, F'] (H[F', F'])^-1 over the coordinates after q, the explicit GPTAQ term of
+    obq_sweep (pinned by comparing the two).
+    """
+    C = np.asarray(C, dtype=np.float64)
+    U = np.asarray(U, dtype=np.float64)
+    T = C @ U.T
+    T = np.triu(T, k=1)
+    return T @ U
+
+
+def row_form_sweep(U, W, s, bits, blocksize, P1=None):
+    """GPTQ sweep with U rows and lazy blocks of `blocksize` coordinates.
+
+    [GPTQ blog] "为什么 Cholesky Factor 不能当作原始逆矩阵" and "GPTQ 怎样把逐个补偿变成可扩展算法":
+    inside a block, E_j = (w_j - Q(w_j)) / U_jj and W_k -= U_jk E_j for the block's
+    later k at once; at the block end the far coordinates get the bulk update
+    W_far -= U[blk, far]^T E_blk. The blocking changes only the order of the work.
+    With P1, [ResComp] item 3's extra row term w_j^pre * P1[j, k] is added the same
+    way (immediately inside the block, in bulk for the far coordinates).
+
+    Returns (codes, W_hat, E) with E[n, j] the normalised errors.
+    """
+    U = np.asarray(U, dtype=np.float64)
+    W = np.array(W, dtype=np.float64, copy=True)
+    N, K = W.shape
+    codes = np.zeros((N, K))
+    E = np.zeros((N, K))
+    for i0 in range(0, K, blocksize):
+        i1 = min(i0 + blocksize, K)
+        W_pre = np.zeros((N, i1 - i0))
+        for j in range(i0, i1):
+            w = W[:, j].copy()
+            W_pre[:, j - i0] = w
+            c = quantize_codes(w, s, bits)
+            target = dequantize(c, s, bits)
+            e = (w - target) / U[j, j]
+            W[:, j:i1] -= np.outer(e, U[j, j:i1])
+            if P1 is not None:
+                W[:, j + 1:i1] += np.outer(w, P1[j, j + 1:i1])
+            W[:, j] = target
+            codes[:, j] = c
+            E[:, j] = e
+        if i1 < K:
+            W[:, i1:] -= E[:, i0:i1] @ U[i0:i1, i1:]
+            if P1 is not None:
+                W[:, i1:] += W_pre @ P1[i0:i1, i1:]
+    return codes, W, E
+
+
+def replay_row_form(U, W, s, bits, codes_gpu, P1=None, band=1e-4):
+    """Tie-follow replay of the unbatched row-form sweep against another run's codes.
+
+    At each (j, n) the oracle takes its own fp64 decision. Where the other run's
+    code differs, the step counts as a tie flip when the codes differ by one and
+    |frac(w / s) - 0.5| < band, else as a mismatch; in both cases the oracle then
+    continues with the other run's code, so one decision never cascades. A
+    negative entry in codes_gpu means "no decision given": the oracle keeps its own.
+
+    Returns dict(codes, W_hat, tie_flips, mismatches, worst_tie_distance).
+    """
+    U = np.asarray(U, dtype=np.float64)
+    W = np.array(W, dtype=np.float64, copy=True)
+    s = np.asarray(s, dtype=np.float64)
+    G = np.asarray(codes_gpu, dtype=np.float64)
+    N, K = W.shape
+    z = 2 ** (bits - 1)
+    codes = np.zeros((N, K))
+    tie_flips = 0
+    mismatches = 0
+    worst = 0.0
+    for j in range(K):
+        w = W[:, j].copy()
+        c = quantize_codes(w, s, bits)
+        diff = (c != G[:, j]) & (G[:, j] >= 0)
+        if np.any(diff):
+            ratio = w[diff] / s[diff]
+            frac_dist = np.abs(np.abs(ratio - np.floor(ratio)) - 0.5)
+            one_apart = np.abs(c[diff] - G[diff, j]) == 1
+            # clamped codes at the grid edge are never near a tie
+            tie = one_apart & (frac_dist < band)
+            tie_flips += int(np.count_nonzero(tie))
+            mismatches += int(np.count_nonzero(~tie))
+            if np.any(tie):
+                worst = max(worst, float(np.max(frac_dist[tie])))
+            c = np.where(diff, G[:, j], c)
+        target = s * (c - z)
+        e = (w - target) / U[j, j]
+        W[:, j:] -= np.outer(e, U[j, j:])
+        if P1 is not None and j + 1 < K:
+            W[:, j + 1:] += np.outer(w, P1[j, j + 1:])
+        W[:, j] = target
+        codes[:, j] = c
+    return dict(codes=codes, W_hat=W, tie_flips=tie_flips, mismatches=mismatches,
+                worst_tie_distance=worst)
+
+
+# --------------------------------------------------------------------------------------
+# Objective and whole-layer driver
+# --------------------------------------------------------------------------------------
+
+def layer_error(H, W, W_hat):
+    """sum_n 1/2 (w_hat_n - w_n)^T H (w_hat_n - w_n) = ||X (W_hat - W)^T||_F^2 for H = 2X^T X.
+
+    [GPTQ blog] "Calibration 让量化看见输入方向": the layer reconstruction objective; with
+    H = 2X^T X one half of the quadratic form is the squared output error.
+    """
+    D = np.asarray(W_hat, dtype=np.float64) - np.asarray(W, dtype=np.float64)
+    return 0.5 * float(np.sum((D @ np.asarray(H, dtype=np.float64)) * D))
+
+
+def solve_layer(H, W, bits, percdamp=0.01, groups=1, C=None, scales=None, mode="schur"):
+    """Whole per-layer solve: dead fix, damping, scale, dead zeroing, sweep.
+
+    H is (K, K) for groups == 1 or (g, K, K); output channels are split into g
+    contiguous groups of N / g, group i solved with H[i] ([G2PTQ] GuidedQuant-style
+    groups with one shared Hessian per group). The scale comes from W as given,
+    before dead coordinates are zeroed (reading). Returns dict(codes, W_hat, scales,
+    loss, dead).
+    """
+    W = np.asarray(W, dtype=np.float64)
+    N, K = W.shape
+    Hs = np.asarray(H, dtype=np.float64).reshape(groups, K, K)
+    if scales is None:
+        s, _ = symmetric_scale(W, bits)
+    else:
+        s = np.asarray(scales, dtype=np.float64)
+    per = N // groups
+    codes = np.zeros((N, K))
+    W_hat = np.zeros((N, K))
+    loss = np.zeros(N)
+    deads = np.zeros((groups, K), dtype=bool)
+    for g in range(groups):
+        H_d, dead = dead_and_damp(Hs[g], percdamp)
+        if not is_positive_definite(H_d):
+            raise np.linalg.LinAlgError("damped Hessian is not positive definite")
+        rows = slice(g * per, (g + 1) * per)
+        Wg = W[rows].copy()
+        Wg[:, dead] = 0.0
+        c, wh, l = obq_sweep(H_d, Wg, s[rows], bits, mode=mode, C=C)
+        codes[rows], W_hat[rows], loss[rows] = c, wh, l
+        deads[g] = dead
+    return dict(codes=codes, W_hat=W_hat, scales=s, loss=loss, dead=deads)
+
+
+def brute_force_best(H, w, grid):
+    """Exhaustive minimiser of 1/2 (v - w)^T H (v - w) over v in grid^K (tiny K only).
+
+    [GPTQ blog] "局部连续最优为什么不保证最终优于 RTN": the sequential result is compared with
+    the best of all 16^3 grid vectors. Returns (best value, list of minimisers).
+    """
+    H = np.asarray(H, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    best = np.inf
+    arg = []
+    for v in itertools.product(grid, repeat=len(w)):
+        d = np.asarray(v, dtype=np.float64) - w
+        val = 0.5 * float(d @ H @ d)
+        if val < best - 1e-12:
+            best, arg = val, [tuple(v)]
+        elif abs(val - best) <= 1e-12:
+            arg.append(tuple(v))
+    return best, arg

@@ -1,0 +1,38 @@
+import os
+import sys
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+GOLDEN = os.path.join(ROOT, "tests", "golden")
+
+
+def pytest_configure(config):
+    config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+    config.addinivalue_line("markers", "slow: full-size workloads")
+
+
+def load_golden(name):
+    """Parse a `key = values` fixture; `;` separates matrix rows."""
+    out = {}
+    with open(os.path.join(GOLDEN, name), encoding="utf-8") as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, val = (p.strip() for p in line.split("=", 1))
+            rows = [r.split() for r in val.split(";")]
+            arr = np.array([[float(x) for x in r] for r in rows])
+            out[key] = arr[0] if arr.shape[0] == 1 else arr
+            if out[key].size == 1:
+                out[key] = float(out[key].reshape(-1)[0])
+    return out
+
+
+@pytest.fixture
+def golden():
+    return load_golden

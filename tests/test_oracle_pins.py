@@ -1,0 +1,364 @@
+"""Pins of the fp64 oracle to what the pages and the mathematics fix (CPU only).
+
+Every function of the oracle is checked against something other than itself:
+printed worked examples (tests/golden), closed forms, special cases that reduce to
+round-to-nearest, brute force, and independent least-squares solves on the token
+matrices.
+"""
+
+import numpy as np
+import pytest
+
+import oracle as O
+
+
+def sse(X, cand, w):
+    """||X (cand - w)||^2 summed over samples, as in the pages' two self-checks."""
+    d = np.asarray(cand, float) - np.asarray(w, float)
+    return float(np.sum((np.asarray(X) @ d) ** 2))
+
+
+# ------------------------------------------------------------------ two-weight example
+
+def test_two_weight_example_gram_and_inverse(golden):
+    g = golden("two_weight_example.txt")
+    H = O.gram(g["X"])
+    np.testing.assert_allclose(H, g["H"], atol=1e-12)
+    np.testing.assert_allclose(np.linalg.inv(H), g["P"], atol=1e-12)
+
+
+def test_two_weight_example_first_step_and_final(golden):
+    g = golden("two_weight_example.txt")
+    H, w = g["H"], g["w"]
+    s = np.array([g["scale"]])
+    bits = int(g["bits"])
+    codes, W_hat, loss, trace = O.obq_sweep(H, w[None, :], s, bits, return_trace=True)
+    np.testing.assert_allclose(trace[0][0] - w, g["first_step_delta"], atol=1e-12)
+    np.testing.assert_allclose(trace[0][0], g["trace_after_step0"], atol=1e-12)
+    assert sse(g["X"], trace[0][0], w) == pytest.approx(g["sse_after_step0"], abs=1e-12)
+    np.testing.assert_array_equal(W_hat[0], g["final"])
+    np.testing.assert_array_equal(codes[0], g["final_codes"])
+    assert sse(g["X"], W_hat[0], w) == pytest.approx(g["sse_final"], abs=1e-12)
+    rtn = O.dequantize(O.quantize_codes(w, s[0], bits), s[0], bits)
+    np.testing.assert_array_equal(rtn, g["rtn"])
+    assert sse(g["X"], rtn, w) == pytest.approx(g["sse_rtn"], abs=1e-12)
+    assert np.mean((rtn - w) ** 2) == pytest.approx(g["weight_mse_rtn"], abs=1e-12)
+    assert np.mean((W_hat[0] - w) ** 2) == pytest.approx(g["weight_mse_final"], abs=1e-12)
+    # the per-step increase r^2 / (2 P_qq) sums to the final output error
+    assert loss[0] == pytest.approx(g["sse_final"], abs=1e-12)
+
+
+def test_two_weight_example_row_form(golden):
+    g = golden("two_weight_example.txt")
+    U = O.upper_factor(g["H"])
+    np.testing.assert_allclose(U.T @ U, g["P"], atol=1e-12)
+    assert U[1, 1] ** 2 == pytest.approx(g["U11_squared"], abs=1e-12)
+    assert abs(U[1, 1] ** 2 - g["P"][1, 1]) > 0.1
+    codes, W_hat, _ = O.row_form_sweep(U, g["w"][None, :], np.array([g["scale"]]),
+                                       int(g["bits"]), blocksize=2)
+    np.testing.assert_allclose(W_hat[0], g["final"], atol=1e-12)
+
+
+# ------------------------------------------------------------------ three-weight example
+
+def test_three_weight_counterexample(golden):
+    g = golden("three_weight_counterexample.txt")
+    H = O.gram(g["X"])
+    np.testing.assert_allclose(H, g["H"], atol=1e-12)
+    np.testing.assert_allclose(np.linalg.inv(H), g["P"], atol=1e-12)
+    np.testing.assert_allclose(O.upper_factor(H), g["U"], atol=1e-12)
+    w, s, bits = g["w"], np.array([g["scale"]]), int(g["bits"])
+    for mode in ("schur", "direct"):
+        codes, W_hat, loss, trace = O.obq_sweep(H, w[None, :], s, bits, mode=mode,
+                                                return_trace=True)
+        np.testing.assert_allclose(trace[0][0], g["trace_after_step0"], atol=1e-12)
+        np.testing.assert_allclose(trace[1][0], g["trace_after_step1"], atol=1e-12)
+        np.testing.assert_allclose(W_hat[0], g["final"], atol=1e-12)
+        assert sse(g["X"], W_hat[0], w) == pytest.approx(g["sse_sequential"], abs=1e-12)
+    for B in (1, 2, 3):
+        _, W_row, _ = O.row_form_sweep(g["U"], w[None, :], s, bits, blocksize=B)
+        np.testing.assert_allclose(W_row[0], g["final"], atol=1e-12)
+    rtn = O.dequantize(O.quantize_codes(w, s[0], bits), s[0], bits)
+    assert sse(g["X"], rtn, w) == pytest.approx(g["sse_rtn"], abs=1e-12)
+    best, arg = O.brute_force_best(H, w, range(-8, 8))
+    assert best == pytest.approx(g["sse_global_best"], abs=1e-12)
+    assert arg == [tuple(g["global_best"])]
+    assert len(list(range(-8, 8))) ** 3 == g["grid_points"]
+
+
+# ------------------------------------------------------------------ damping
+
+def test_rank_one_needs_damping(golden):
+    g = golden("rank_one_damping.txt")
+    H = O.gram(np.atleast_2d(g["X"]))
+    assert np.linalg.matrix_rank(H) == 1
+    H0, dead0 = O.dead_and_damp(H, g["percdamp_singular"])
+    assert not dead0.any()
+    assert not O.is_positive_definite(H0)
+    H1, _ = O.dead_and_damp(H, g["percdamp_default"])
+    assert O.is_positive_definite(H1)
+    # the increment is percdamp * mean(diag H)
+    np.testing.assert_allclose(np.diag(H1) - np.diag(H), 0.01 * np.mean(np.diag(H)))
+    with pytest.raises(np.linalg.LinAlgError):
+        O.solve_layer(H, np.array([[0.3, -0.2]]), 4, percdamp=0.0)
+
+
+def test_damping_scales_with_H_and_dead_fix():
+    rng = np.random.default_rng(0)
+    X = rng.standard_normal((50, 6))
+    X[:, 2] = 0.0                                  # coordinate 2 never excited
+    H = O.gram(X)
+    Hd, dead = O.dead_and_damp(H, 0.01)
+    assert dead.tolist() == [False, False, True, False, False, False]
+    H_fix = H.copy()
+    H_fix[2, 2] = 1.0
+    np.testing.assert_allclose(np.diag(Hd), np.diag(H_fix) + 0.01 * np.mean(np.diag(H_fix)))
+    # a positive scale of H scales the damped live diagonal by the same factor
+    Hd3, _ = O.dead_and_damp(3.0 * H, 0.01)
+    live = ~dead
+    H_fix3 = 3.0 * H
+    H_fix3[2, 2] = 1.0
+    np.testing.assert_allclose(np.diag(Hd3)[live],
+                               3.0 * np.diag(H)[live] + 0.01 * np.mean(np.diag(H_fix3)))
+    # dead weights are zeroed and end on code z (value 0)
+    W = rng.standard_normal((4, 6)) * 0.02
+    out = O.solve_layer(H, W, 3, percdamp=0.01)
+    assert np.all(out["W_hat"][:, 2] == 0.0)
+    assert np.all(out["codes"][:, 2] == 4)
+
+
+# ------------------------------------------------------------------ grid and rounding
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_symmetric_grid(bits):
+    rng = np.random.default_rng(bits)
+    W = rng.standard_normal((16, 40))
+    s, z = O.symmetric_scale(W, bits)
+    assert z == 2 ** (bits - 1)
+    c = O.quantize_codes(W, s[:, None], bits)
+    assert c.min() >= 0 and c.max() <= 2 ** bits - 1
+    q = O.dequantize(c, s[:, None], bits)
+    lv = q / s[:, None]
+    np.testing.assert_allclose(lv, np.round(lv), atol=1e-12)
+    lv = np.round(lv)
+    assert lv.min() >= -2 ** (bits - 1) and lv.max() <= 2 ** (bits - 1) - 1
+    # a channel whose scale is exact puts -amax and +amax on the grid edges:
+    # -amax / s = -(2^b - 1) / 2 is a tie that goes to the even level -2^(b-1)
+    amax = (2 ** bits - 1) / 2.0
+    s1, _ = O.symmetric_scale(np.array([[-amax, 0.25, amax]]), bits)
+    assert s1[0] == 1.0
+    edge = O.quantize_codes(np.array([-amax, amax]), s1[0], bits)
+    np.testing.assert_array_equal(edge, [0, 2 ** bits - 1])
+
+
+def test_round_half_to_even():
+    # ties go to the even neighbour ("最近偶数舍入")
+    w = np.array([0.5, 1.5, 2.5, -0.5, -1.5, 0.49, 0.51])
+    c = O.quantize_codes(w, 1.0, 4) - 8
+    np.testing.assert_array_equal(c, [0, 2, 2, 0, -2, 0, 1])
+    assert O.symmetric_scale(np.zeros((1, 3)), 4)[0][0] == 1.0
+
+
+# ------------------------------------------------------------------ forms agree
+
+def _random_problem(K, N, seed, M=None):
+    rng = np.random.default_rng(seed)
+    M = M or 3 * K
+    X = rng.standard_normal((M, K)) @ rng.standard_normal((K, K)) / np.sqrt(K)
+    H = O.gram(X)
+    Hd, _ = O.dead_and_damp(H, 0.01)
+    W = rng.standard_normal((N, K)) * 0.02
+    return X, H, Hd, W
+
+
+@pytest.mark.parametrize("K,seed", [(3, 1), (7, 2), (12, 3), (16, 4)])
+def test_direct_schur_and_row_forms_agree(K, seed):
+    X, H, Hd, W = _random_problem(K, 9, seed)
+    s, _ = O.symmetric_scale(W, 3)
+    c_dir, w_dir, l_dir = O.obq_sweep(Hd, W, s, 3, mode="direct")
+    c_sch, w_sch, l_sch = O.obq_sweep(Hd, W, s, 3, mode="schur")
+    np.testing.assert_array_equal(c_dir, c_sch)
+    np.testing.assert_allclose(w_dir, w_sch, atol=1e-12)
+    np.testing.assert_allclose(l_dir, l_sch, rtol=1e-10)
+    U = O.upper_factor(Hd)
+    for B in (1, 2, 4, 8, K):
+        c_row, w_row, E = O.row_form_sweep(U, W, s, 3, B)
+        np.testing.assert_array_equal(c_row, c_sch)
+        np.testing.assert_allclose(w_row, w_sch, atol=1e-12)
+        # per-channel loss: sum r^2/(2 P_qq) = 1/2 sum E^2
+        np.testing.assert_allclose(0.5 * np.sum(E ** 2, axis=1), l_sch, rtol=1e-9)
+
+
+@pytest.mark.parametrize("K", [4, 9, 16])
+def test_U_diagonal_is_free_set_pivot(K):
+    _, _, Hd, _ = _random_problem(K, 1, 10 + K)
+    U = O.upper_factor(Hd)
+    assert np.allclose(np.tril(U, -1), 0.0)
+    for j in range(K):
+        P_F = np.linalg.inv(Hd[j:, j:])
+        assert U[j, j] ** 2 == pytest.approx(P_F[0, 0], rel=1e-10)
+
+
+def test_objective_identities():
+    X, H, Hd, W = _random_problem(10, 5, 7, M=200)
+    s, _ = O.symmetric_scale(W, 2)
+    # undamped: the increase per step sums to the output error ||X Δ||^2
+    codes, W_hat, loss = O.obq_sweep(H, W, s, 2)
+    out_err = np.sum((X @ (W_hat - W).T) ** 2, axis=0)
+    np.testing.assert_allclose(loss, out_err, rtol=1e-9)
+    assert O.layer_error(H, W, W_hat) == pytest.approx(out_err.sum(), rel=1e-10)
+    # damped: 1/2 Δ^T H_d Δ = 1/2 sum E^2
+    U = O.upper_factor(Hd)
+    _, W_d, E = O.row_form_sweep(U, W, s, 2, 4)
+    D = W_d - W
+    np.testing.assert_allclose(0.5 * np.sum((D @ Hd) * D, axis=1),
+                               0.5 * np.sum(E ** 2, axis=1), rtol=1e-9)
+
+
+# ------------------------------------------------------------------ special cases
+
+def test_identity_hessian_is_rtn():
+    rng = np.random.default_rng(3)
+    W = rng.standard_normal((6, 20)) * 0.02
+    s, _ = O.symmetric_scale(W, 3)
+    codes, W_hat, _ = O.obq_sweep(2.0 * np.eye(20), W, s, 3)
+    np.testing.assert_array_equal(codes, O.quantize_codes(W, s[:, None], 3))
+    c1, _, _ = O.obq_sweep(np.array([[3.7]]), W[:, :1], s, 3)
+    np.testing.assert_array_equal(c1, O.quantize_codes(W[:, :1], s[:, None], 3))
+
+
+def test_scaled_hessian_same_codes_and_permutation_equivariance():
+    X, H, Hd, W = _random_problem(12, 8, 11)
+    s, _ = O.symmetric_scale(W, 4)
+    c0, w0, _ = O.obq_sweep(Hd, W, s, 4)
+    c1, w1, _ = O.obq_sweep(37.0 * Hd, W, s, 4)
+    np.testing.assert_array_equal(c0, c1)
+    np.testing.assert_allclose(w0, w1, atol=1e-12)
+    perm = np.random.default_rng(1).permutation(8)
+    c2, w2, _ = O.obq_sweep(Hd, W[perm], s[perm], 4)
+    np.testing.assert_array_equal(c2, c0[perm])
+
+
+def test_sequential_never_beats_brute_force():
+    for seed in range(5):
+        X, H, Hd, W = _random_problem(3, 1, 100 + seed)
+        w = W[0] / 0.02 * 1.3
+        codes, W_hat, _ = O.obq_sweep(H, w[None, :], np.array([1.0]), 4)
+        best, _ = O.brute_force_best(H, w, range(-8, 8))
+        assert O.layer_error(H, w[None, :], W_hat) >= best - 1e-12
+
+
+# ------------------------------------------------------------------ weighted / grouped Gram
+
+def test_weighted_gram_equals_repeated_tokens():
+    rng = np.random.default_rng(5)
+    X = rng.standard_normal((30, 7))
+    reps = rng.integers(0, 4, size=30)
+    np.testing.assert_allclose(O.gram(X, reps.astype(float)), O.gram(np.repeat(X, reps, 0)),
+                               atol=1e-10)
+    np.testing.assert_allclose(O.gram(X, np.ones(30)), O.gram(X), atol=1e-12)
+
+
+def test_grouped_solve_is_independent_groups():
+    rng = np.random.default_rng(8)
+    X = rng.standard_normal((120, 10))
+    W = rng.standard_normal((8, 10)) * 0.02
+    Hs = np.stack([O.gram(X, rng.random(120) * 2) for _ in range(4)])
+    out = O.solve_layer(Hs, W, 3, groups=4)
+    for g in range(4):
+        ref = O.solve_layer(Hs[g], W[2 * g:2 * g + 2], 3, scales=out["scales"][2 * g:2 * g + 2])
+        np.testing.assert_array_equal(out["codes"][2 * g:2 * g + 2], ref["codes"])
+    same = O.solve_layer(np.stack([O.gram(X)] * 2), W, 3, groups=2)
+    plain = O.solve_layer(O.gram(X), W, 3)
+    np.testing.assert_array_equal(same["codes"], plain["codes"])
+
+
+# ------------------------------------------------------------------ GPTAQ
+
+def _gptaq_problem(K, M, seed, noise=0.1):
+    rng = np.random.default_rng(seed)
+    X_fp = rng.standard_normal((M, K)) @ (np.eye(K) + 0.3 * rng.standard_normal((K, K)) / np.sqrt(K))
+    X_q = X_fp + noise * rng.standard_normal((M, K))
+    return X_fp, X_q
+
+
+def test_gptaq_first_step_is_least_squares_on_tokens():
+    """Step 0's residual term equals the least-squares fit of the free columns of the
+    quantised stream to neuron 0's share of r1 = w (X~ - X), solved on the token
+    matrices directly (no H, no C)."""
+    K, M = 6, 80
+    X_fp, X_q = _gptaq_problem(K, M, 21)
+    H = O.gram(X_q)
+    C = O.cross_gram(X_q, X_fp)
+    w = np.array([[0.31, -0.12, 0.05, 0.2, -0.07, 0.11]])
+    s = np.array([1.0])
+    _, _, _, tr_aq = O.obq_sweep(H, w, s, 4, C=C, return_trace=True)
+    _, _, _, tr_q = O.obq_sweep(H, w, s, 4, return_trace=True)
+    extra = tr_aq[0][0, 1:] - tr_q[0][0, 1:]
+    dX = X_fp - X_q
+    v, *_ = np.linalg.lstsq(X_q[:, 1:], dX[:, 0] * w[0, 0], rcond=None)
+    np.testing.assert_allclose(extra, v, rtol=1e-9, atol=1e-12)
+
+
+def test_gptaq_zero_residual_is_gptq_and_p1_matches_explicit():
+    K, M = 14, 90
+    X_fp, X_q = _gptaq_problem(K, M, 5)
+    H = O.gram(X_q)
+    Hd, _ = O.dead_and_damp(H, 0.01)
+    W = np.random.default_rng(2).standard_normal((7, K)) * 0.02
+    s, _ = O.symmetric_scale(W, 2)
+    c_q, w_q, _ = O.obq_sweep(Hd, W, s, 2)
+    c0, w0, _ = O.obq_sweep(Hd, W, s, 2, C=O.cross_gram(X_q, X_q))
+    np.testing.assert_array_equal(c0, c_q)
+    np.testing.assert_allclose(w0, w_q, atol=1e-12)
+    C = O.cross_gram(X_q, X_fp)
+    c_aq, w_aq, _ = O.obq_sweep(Hd, W, s, 2, C=C)
+    U = O.upper_factor(Hd)
+    P1 = O.gptaq_p1(C, U)
+    assert np.allclose(np.tril(P1), 0.0)
+    for q in range(K - 1):
+        row = C[q, q + 1:] @ np.linalg.inv(Hd[q + 1:, q + 1:])
+        np.testing.assert_allclose(P1[q, q + 1:], row, rtol=1e-8, atol=1e-12)
+    for B in (1, 3, 8, K):
+        c_row, w_row, _ = O.row_form_sweep(U, W, s, 2, B, P1=P1)
+        np.testing.assert_array_equal(c_row, c_aq)
+        np.testing.assert_allclose(w_row, w_aq, atol=1e-12)
+    # the asymmetric term moves the free weights for a non-trivial residual
+    _, _, _, tr_aq = O.obq_sweep(Hd, W, s, 2, C=C, return_trace=True)
+    _, _, _, tr_q = O.obq_sweep(Hd, W, s, 2, return_trace=True)
+    assert not np.allclose(tr_aq[0], tr_q[0])
+
+
+def test_gptaq_inclusive_mask_would_differ():
+    """An inclusive mask adds a diagonal term; the strict reading is the only one
+    equal to the explicit free-set update."""
+    K = 8
+    X_fp, X_q = _gptaq_problem(K, 40, 9)
+    Hd, _ = O.dead_and_damp(O.gram(X_q), 0.01)
+    C = O.cross_gram(X_q, X_fp)
+    U = O.upper_factor(Hd)
+    inclusive = np.triu(C @ U.T) @ U
+    assert not np.allclose(inclusive, O.gptaq_p1(C, U))
+
+
+# ------------------------------------------------------------------ replay protocol
+
+def test_replay_counts_flips_without_cascade():
+    X, H, Hd, W = _random_problem(16, 6, 31)
+    s, _ = O.symmetric_scale(W, 3)
+    U = O.upper_factor(Hd)
+    codes, W_hat, _ = O.row_form_sweep(U, W, s, 3, 16)
+    rep = O.replay_row_form(U, W, s, 3, codes)
+    assert rep["tie_flips"] == 0 and rep["mismatches"] == 0
+    np.testing.assert_array_equal(rep["codes"], codes)
+    # plant one wrong decision in an oracle run; the run continues consistently
+    # from it (as another implementation would), and the replay of that run counts
+    # exactly one mismatch
+    bad = codes.copy()
+    bad[2, 5] = bad[2, 5] + 1 if bad[2, 5] < 7 else bad[2, 5] - 1
+    planted = O.replay_row_form(U, W, s, 3, np.where(np.arange(16) == 5, bad, -1))
+    other = planted["codes"]
+    assert other[2, 5] == bad[2, 5]
+    rep = O.replay_row_form(U, W, s, 3, other)
+    assert rep["mismatches"] == 1 and rep["tie_flips"] == 0
+    np.testing.assert_array_equal(rep["codes"], other)
