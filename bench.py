@@ -1,0 +1,457 @@
+#!/usr/bin/env python3
+"""Benchmark of the GPTQ per-layer solve on B200.
+
+One step = the whole per-layer path on one layer's calibration batch, inputs
+resident in HBM:
+  Gram over the full token stream (32 x 65,536-token chunks of
+  gptq_accumulate_hessian) -> gptq_prepare -> gptq_quantize_layer.
+Workload (default): LLaMA-3-8B up_proj shapes, K=4096 inputs, N=14336 outputs,
+2,097,152 Student-t bf16 tokens, 3-bit symmetric per-channel, blocksize 128,
+percdamp 0.01. value = weights quantized per second of the whole step (K*N per
+step); the breakdown reports the layer solve (prepare + quantize) and the Gram.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+For N > 1 each rank solves its own independent layer (weak scaling, no
+collective on the data path); timing is the max over ranks.
+--impl reference times the fp64 CPU oracle on a bounded sample of the same job.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GPTQ layer-solve ms & weights quantized/s (4096×14336, W3); % of TC/HBM roofline"
+UNIT = "weights/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mlp_up_w3")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-seconds", type=float, default=12.0)
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override the stream length (small profiling cases only)")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- clocks
+
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms while the timed region runs."""
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.lines = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={CLOCK_FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.gpu_id)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def gpu_smi_id(torch, dev):
+    try:
+        p = torch.cuda.get_device_properties(dev)
+        return f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+    except Exception:
+        return dev.index or 0
+
+
+# ----------------------------------------------------------------------------- CPU oracle sample
+
+def oracle_sample(wl, budget_s):
+    """Time the fp64 oracle on a bounded sample of the job; scale to the full job.
+
+    Sample: the Gram of 4,096 tokens (scaled by tokens), the damping + PD check +
+    inverse at full K, and the explicit-OBQ sweep over a prefix of the coordinates
+    for 8 and 64 channels (scaled by operation counts: the Schur update costs
+    (K-j)^2 per step, the channel update N (K-j) per step)."""
+    import numpy as np
+    import torch
+
+    import oracle as O
+    from post_weight_quantization_solve_b200 import synth
+
+    K, N, M = wl.K, wl.N, wl.M
+    m_s = 4096
+    X = synth.tokens_chunk(wl, 0, "cpu", rows=m_s).double().numpy()
+    W = synth.weights(wl, "cpu").double().numpy()
+    t = time.perf_counter()
+    H = O.gram(X)
+    t_gram = (time.perf_counter() - t) * (M / m_s)
+    t = time.perf_counter()
+    Hd, _ = O.dead_and_damp(H, wl.percdamp)
+    O.is_positive_definite(Hd)
+    t_prep = time.perf_counter() - t
+    t = time.perf_counter()
+    np.linalg.inv(Hd)                      # the sweep's one-off inverse (counted in prepare)
+    t_inv = time.perf_counter() - t
+    t_prep += t_inv
+    s, _ = O.symmetric_scale(W, wl.bits)
+
+    def prefix(nch, q):
+        t0 = time.perf_counter()
+        O.obq_sweep(Hd, W[:nch], s[:nch], wl.bits, steps=q)
+        return max(time.perf_counter() - t0 - t_inv, 1e-6)
+
+    probe = 32
+    t_probe = prefix(64, probe)
+    q = int(max(probe, min(K, probe * (0.4 * budget_s) / t_probe)))
+    t_a = prefix(8, q)
+    t_b = prefix(64, q)
+    j = np.arange(K, dtype=np.float64)
+    S_all, S_pre = np.sum((K - j) ** 2), np.sum((K - j[:q]) ** 2)
+    L_all, L_pre = np.sum(K - j), np.sum(K - j[:q])
+    c_ch = max(t_b - t_a, 0.0) / 56.0
+    t_schur = max(t_a - 8 * c_ch, 1e-9)
+    t_sweep = t_schur * S_all / S_pre + c_ch * N * L_all / L_pre
+    total = t_gram + t_prep + t_sweep
+    cores = torch.get_num_threads()
+    return {
+        "seconds_per_step": total,
+        "value": K * N / total,
+        "cores": cores,
+        "sample": (f"oracle fp64: Gram of {m_s} tokens x{M // m_s} by tokens; damping+PD check+"
+                   f"inverse at K={K}; explicit-OBQ sweep, first {q} of {K} coordinates for 8 and "
+                   f"64 channels, scaled by (K-j)^2 Schur and N(K-j) channel operation counts "
+                   f"(extrapolated)"),
+        "parts_s": {"gram": t_gram, "prepare": t_prep, "sweep": t_sweep},
+        "measured_s": time_sum(t_gram * m_s / M, t_prep, t_probe, t_a, t_b, 3 * t_inv),
+    }
+
+
+def time_sum(*a):
+    return round(sum(a), 2)
+
+
+# ----------------------------------------------------------------------------- ours
+
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import post_weight_quantization_solve_b200 as gq
+    from post_weight_quantization_solve_b200 import synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    gq.load_library()
+    base = synth.WORKLOADS[args.workload]
+    wl = base.scaled(name=base.name, seed=base.seed + 1000 * rank)   # one layer per rank
+    if args.tokens:
+        wl = wl.scaled(name=base.name + f"_tokens{args.tokens}", M=args.tokens)
+    K, N, M, ch = wl.K, wl.N, wl.M, wl.chunk
+    nch = synth.num_chunks(wl)
+
+    X = torch.empty(M, K, dtype=wl.xdtype, device=dev)
+    for c in range(nch):
+        X[c * ch:(c + 1) * ch] = synth.tokens_chunk(wl, c, dev)
+    W = synth.weights(wl, dev).contiguous()
+    H = torch.empty(K, K, device=dev)
+    codes = torch.empty(N, K, dtype=torch.uint8, device=dev)
+    scales = torch.empty(N, device=dev)
+    status = gq.new_status(dev)
+    ws_p = torch.empty(gq.gptq_workspace_size(gq.GPTQ_OP_PREPARE, K, 0, 1, 0), dtype=torch.uint8,
+                       device=dev)
+    ws_q = torch.empty(gq.gptq_workspace_size(gq.GPTQ_OP_QUANTIZE, K, N, 1, wl.blocksize),
+                       dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    gram_ev = []
+
+    def step(record=None):
+        H.zero_()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev[0].record(stream)
+        for c in range(nch):
+            if record is not None:
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+            gq.gptq_accumulate_hessian(H, X[c * ch:(c + 1) * ch], stream=stream)
+            if record is not None:
+                b.record(stream)
+                record.append((a, b))
+        ev[1].record(stream)
+        gq.gptq_prepare(H, wl.percdamp, workspace=ws_p, status=status, stream=stream)
+        ev[2].record(stream)
+        gq.gptq_quantize_layer(W, H, wl.bits, wl.blocksize, scales_out=scales, codes=codes,
+                               workspace=ws_q, status=status, stream=stream)
+        ev[3].record(stream)
+        return ev
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    gq.raise_on_status(status, "warmup")
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+    launches0 = gq.gptq_kernel_launches()
+    evs = []
+    with ClockSampler(gpu_smi_id(torch, dev)) as clk:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            evs.append(step(gram_ev))
+        t1.record(stream)
+        torch.cuda.synchronize()
+    launches = gq.gptq_kernel_launches() - launches0
+    if world > 1:
+        dist.barrier()
+    gq.raise_on_status(status, "timed steps")
+    total_ms = t0.elapsed_time(t1)
+    parts = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])]
+                      for e in evs])
+    gram_launch_ms = float(np.mean([a.elapsed_time(b) for a, b in gram_ev]))
+
+    stats = torch.tensor([total_ms, *parts.mean(0).tolist(), gram_launch_ms], dtype=torch.float64,
+                         device=dev)
+    if world > 1:
+        dist.all_reduce(stats, op=dist.ReduceOp.MAX)
+    total_ms, gram_ms, prep_ms, quant_ms, gram_launch_ms = stats.tolist()
+    ms_per_step = total_ms / args.steps
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, wl, X, W, dev, gq, torch, dist, world)
+
+    if rank != 0:
+        return None
+    clocks = clk.summary()
+    flops_launch = float(ch) * K * (K + 1)          # symmetric Gram work per 65,536-token chunk
+    sm_clock = (clocks["sm_mhz"] or 1965.0) * 1e6
+    peaks = load_peaks()
+    # the SIMT Gram is bound by fp32 FMA issue: 148 SMs x 128 lanes x 2 FLOP x clock
+    alu_peak = 148 * 128 * 2 * 1965e6 / 1e12
+    achieved = flops_launch / (gram_launch_ms * 1e-3) / 1e12
+    roofline = {"kernel": "gemm_simt_kernel (Gram, gptq_accumulate_hessian)", "bound": "alu",
+                "achieved": round(achieved, 2), "peak": round(alu_peak, 1), "unit": "TFLOP/s",
+                "frac": round(achieved / alu_peak, 4), "traffic": None,
+                "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz",
+                "per_launch": f"{ch} tokens x K(K+1) = {flops_launch:.3e} FLOP"}
+    weights = K * N * world
+    line = {
+        "metric": METRIC, "value": weights / (ms_per_step * 1e-3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16->f32",
+        "data": "synthetic (seeded Student-t(4)/sqrt2 bf16 tokens, N(0,0.02^2) bf16 weights)",
+        "config": {"workload": f"{wl.name}: K={K} N={N} tokens={M} (chunks {nch}x{ch}) W{wl.bits} "
+                               f"blocksize {wl.blocksize} percdamp {wl.percdamp}",
+                   "l2": f"inputs larger than L2 (X {M * K * 2 / 1e9:.1f} GB)", "parallelism": f"{world} independent layers"},
+        "breakdown": {"gram_ms": gram_ms, "prepare_ms": prep_ms, "quantize_ms": quant_ms,
+                      "layer_solve_ms": prep_ms + quant_ms,
+                      "solve_weights_per_s": K * N / ((prep_ms + quant_ms) * 1e-3),
+                      "gram_tflops_symmetric": M * K * (K + 1) / (gram_ms * 1e-3) / 1e12},
+        "roofline": roofline,
+        "gpu_launches": int(launches),
+        "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
+                   "reasons": clocks["reasons"]},
+        "measured_peaks": {k: peaks.get(k) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")},
+    }
+    if e2e:
+        line["e2e"] = e2e
+    if world == 1 and not args.no_cpu_baseline:
+        cb = oracle_sample(wl, args.cpu_sample_seconds)
+        line["cpu_baseline"] = {"value": cb["value"], "unit": UNIT, "cores": cb["cores"],
+                                "kind": "oracle", "sample": cb["sample"]}
+    return line
+
+
+def run_e2e(args, wl, X, W, dev, gq, torch, dist, world):
+    """Same step through the public API with host buffers: every step copies the
+    token stream and W from pinned host memory and reads codes + scales back."""
+    K, N, M, ch = wl.K, wl.N, wl.M, wl.chunk
+    nch = (M + ch - 1) // ch
+    Xh = torch.empty(M, K, dtype=X.dtype, pin_memory=True)
+    Xh.copy_(X)
+    Wh = W.cpu().pin_memory()
+    codes_h = torch.empty(N, K, dtype=torch.uint8, pin_memory=True)
+    scales_h = torch.empty(N, dtype=torch.float32, pin_memory=True)
+    bufs = [torch.empty(ch, K, dtype=X.dtype, device=dev) for _ in range(2)]
+    Wd = torch.empty_like(W)
+    H = torch.empty(K, K, device=dev)
+    codes = torch.empty(N, K, dtype=torch.uint8, device=dev)
+    scales = torch.empty(N, device=dev)
+    status = gq.new_status(dev)
+    ws_p = torch.empty(gq.gptq_workspace_size(gq.GPTQ_OP_PREPARE, K, 0, 1, 0), dtype=torch.uint8,
+                       device=dev)
+    ws_q = torch.empty(gq.gptq_workspace_size(gq.GPTQ_OP_QUANTIZE, K, N, 1, wl.blocksize),
+                       dtype=torch.uint8, device=dev)
+    comp = torch.cuda.current_stream(dev)
+    copy = torch.cuda.Stream(dev)
+
+    def step():
+        H.zero_()
+        done = [torch.cuda.Event() for _ in range(2)]
+        ready = [torch.cuda.Event() for _ in range(nch)]
+        copy.wait_stream(comp)
+        for c in range(nch):
+            b = bufs[c % 2]
+            if c >= 2:
+                copy.wait_event(done[c % 2])
+            rows = min(ch, M - c * ch)
+            with torch.cuda.stream(copy):
+                b[:rows].copy_(Xh[c * ch:c * ch + rows], non_blocking=True)
+                if c == 0:
+                    Wd.copy_(Wh, non_blocking=True)
+            ready[c].record(copy)
+            comp.wait_event(ready[c])
+            gq.gptq_accumulate_hessian(H, b[:rows], stream=comp)
+            done[c % 2].record(comp)
+        gq.gptq_prepare(H, wl.percdamp, workspace=ws_p, status=status, stream=comp)
+        gq.gptq_quantize_layer(Wd, H, wl.bits, wl.blocksize, scales_out=scales, codes=codes,
+                               workspace=ws_q, status=status, stream=comp)
+        codes_h.copy_(codes, non_blocking=True)
+        scales_h.copy_(scales, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(comp)
+    for _ in range(args.e2e_steps):
+        step()
+    t1.record(comp)
+    torch.cuda.synchronize()
+    gq.raise_on_status(status, "e2e")
+    ms = torch.tensor([t0.elapsed_time(t1) / args.e2e_steps], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
+    ms = float(ms.item())
+    h2d = Xh.numel() * Xh.element_size() + Wh.numel() * Wh.element_size()
+    d2h = codes_h.numel() + scales_h.numel() * 4
+    return {"value": K * N * world / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "note": "token stream + W from pinned host each step (copy stream, double-buffered), "
+                    "codes + scales back"}
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f)
+    except OSError:
+        return {}
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args, rank, world):
+    from post_weight_quantization_solve_b200 import synth
+
+    if rank != 0:
+        return None
+    wl = synth.WORKLOADS[args.workload]
+    budget = max(2.0, min(args.cpu_sample_seconds, 150.0 / max(args.steps + args.warmup, 1)))
+    for _ in range(args.warmup):
+        oracle_sample(wl, budget)
+    runs = [oracle_sample(wl, budget) for _ in range(args.steps)]
+    sec = statistics.mean(r["seconds_per_step"] for r in runs)
+    value = wl.K * wl.N / sec
+    cb = runs[-1]
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (same recipe, CPU generator)",
+        "config": {"workload": f"{wl.name}: K={wl.K} N={wl.N} tokens={wl.M} W{wl.bits} "
+                               f"blocksize {wl.blocksize} percdamp {wl.percdamp}"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cb["cores"], "kind": "oracle",
+                         "sample": cb["sample"]},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", args.gpus if args.gpus == 1 else 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+    else:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        if world > 1:
+            torch.cuda.set_device(local_rank)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        try:
+            line = run_ours(args, rank, world, local_rank)
+        finally:
+            if world > 1:
+                dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

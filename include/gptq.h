@@ -1,0 +1,199 @@
+/*
+ * gptq.h -- C ABI of libgptq.so: the GPTQ-family per-layer compensation solve on
+ * NVIDIA B200 (sm_100a).
+ *
+ * Sources (cited by page title and section):
+ *   [GPTQ blog] "GPTQ：量化一个权重之后怎样补偿输出误差" (charlestar.github.io)
+ *   [ResComp]   "Rethinking Residual Errors in Compensation-based LLM Quantization"
+ *               (papernotes.org), "关键设计" items 1-3
+ *   [GPTAQ]     "GPTAQ: Efficient Finetuning-Free Quantization for Asymmetric
+ *               Calibration" (Paper-Notes), "关键设计"
+ *   [G2PTQ]     "G²PTQ: Improving LLM Post-Training Quantization with Generalized
+ *               Gradient Compensation" (agihunt.info summary)
+ *
+ * Conventions shared by every call
+ *   - All pointers named as device buffers are CUDA device memory owned by the
+ *     caller. The library allocates nothing; scratch comes from a caller
+ *     workspace of gptq_workspace_size() bytes (256-byte aligned).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL is the legacy default stream). No call synchronises the host.
+ *   - The return value reports argument errors (GPTQ_ERR_ARG, GPTQ_ERR_WORKSPACE)
+ *     and launch errors (GPTQ_ERR_CUDA) synchronously; nothing has been enqueued
+ *     when it is not GPTQ_OK.
+ *   - Numerical failures are found on the device and written to a caller-owned
+ *     device int32 `status` word: the first failing kernel stores its
+ *     gptq_status code there, later kernels of any call given the same word see
+ *     a non-zero value and skip their work. The caller zeroes the word before a
+ *     chain of calls and reads it after synchronising. This follows the blog's
+ *     self-check ("用标准库核对二维补偿"), which refuses non-finite or non-PD input
+ *     instead of repairing it.
+ *   - Layout: W is nn.Linear order W[N][K] row-major (N output channels, K input
+ *     coordinates): the blog's K x N weight matrix stored column-major, so row n
+ *     is output channel n ([GPTQ blog] "GPTQ 怎样把逐个补偿变成可扩展算法" on
+ *     N x K versus K x N). Token streams X are row-major [M][K].
+ *   - Matrices named K x K are fp32 row-major with leading dimension K; a stack of
+ *     g of them is contiguous, [g][K][K].
+ */
+#ifndef GPTQ_H
+#define GPTQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GPTQ_API __attribute__((visibility("default")))
+#else
+#define GPTQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GPTQ_OK = 0,
+    GPTQ_ERR_ARG = 1,        /* invalid argument (size, pointer, alignment, option) */
+    GPTQ_ERR_NOT_PD = 2,     /* a Cholesky pivot is not clearly positive after damping */
+    GPTQ_ERR_NONFINITE = 3,  /* NaN or Inf in an input or an intermediate */
+    GPTQ_ERR_CUDA = 4,       /* a CUDA launch or API call failed */
+    GPTQ_ERR_TIMEOUT = 5,    /* a bounded device wait ran out */
+    GPTQ_ERR_WORKSPACE = 6   /* workspace missing, misaligned or too small */
+} gptq_status;
+
+typedef enum { GPTQ_BF16 = 0, GPTQ_F32 = 1 } gptq_dtype;
+
+typedef enum {
+    GPTQ_OP_PREPARE = 0,
+    GPTQ_OP_RESIDUAL = 1,
+    GPTQ_OP_QUANTIZE = 2
+} gptq_op;
+
+/*
+ * gptq_accumulate_hessian -- H[g] += 2 * X^T diag(w[g]) X over one token chunk.
+ *
+ * [GPTQ blog] "Calibration 让量化看见输入方向": the layer objective's Hessian is
+ * 2 X^T X, shared by all output channels and accumulated batch by batch without
+ * keeping activations (factor 2 fixed by the two-weight example of "两个权重怎样互相补偿").
+ * [G2PTQ]: with output-channel groups each group g has its own Hessian; here a
+ * group's per-token weight w[g][m] scales token m's outer product.
+ *
+ *   H      device fp32 [g][K][K]; accumulated into (the caller zeroes it before the
+ *          first chunk). Full symmetric storage is written.
+ *   K      input coordinates, >= 1; bf16 streams need K % 8 == 0.
+ *   g      number of Hessians (>= 1). With w == NULL, g must be 1.
+ *   X      device [M][ldx] tokens, dtype xdtype. bf16: X and ldx 16-byte aligned
+ *          (ldx % 8 == 0). ldx >= K.
+ *   M      tokens in this chunk (>= 0; 0 is a no-op).
+ *   w      device fp32 [g][ldw] per-token weights, or NULL for unit weights.
+ *   Errors: GPTQ_ERR_ARG for bad sizes/alignment/dtype, GPTQ_ERR_CUDA on launch.
+ */
+GPTQ_API gptq_status gptq_accumulate_hessian(float *H, int K, int g, const void *X, int xdtype,
+                                    int64_t M, int64_t ldx, const float *w, int64_t ldw,
+                                    void *stream);
+
+/*
+ * gptaq_accumulate_cross -- C += 2 * (X_fp - X_q)^T X_q over one token chunk.
+ *
+ * [ResComp] item 2: r1 = w (X~ - X) with X~ the full-precision stream and X the
+ * quantised stream; item 3 precomputes the cross statistic dX X^T (their row
+ * convention; dX^T X here). The difference X_fp - X_q is formed exactly in fp32 on
+ * the device from the two inputs, so no rounded dX is ever stored.
+ *
+ *   C      device fp32 [K][K], accumulated into (caller zeroes it first). Not
+ *          symmetric: C[i][j] = 2 sum_m dX[m][i] X_q[m][j].
+ *   X_fp, X_q  device [M][ldx] each, same dtype and leading dimension; alignment
+ *          rules as gptq_accumulate_hessian.
+ */
+GPTQ_API gptq_status gptaq_accumulate_cross(float *C, int K, const void *X_fp, const void *X_q,
+                                   int xdtype, int64_t M, int64_t ldx, void *stream);
+
+/*
+ * gptq_prepare -- dead coordinates, damping and the upper factor U, in place.
+ *
+ * [GPTQ blog] "Damping 与两个不同的分组参数": coordinates with H_kk == 0 are dead
+ * (their diagonal is set to 1 here; their weights are zeroed by
+ * gptq_quantize_layer), then H += percdamp * mean(diag H) * I.
+ * "为什么 Cholesky Factor 不能当作原始逆矩阵": U is upper triangular with
+ * U^T U = H^-1; row q of U carries the free-set inverse at q's step.
+ * Computed as H = R R^T with R upper (Cholesky of the index-reversed matrix),
+ * U = R^-1 (triangular inversion): no explicit H^-1 is formed.
+ *
+ *   H        device fp32 [g][K][K] symmetric (the upper triangle is read). On
+ *            return it holds U per group: upper triangle U, strict lower zero.
+ *   percdamp >= 0 (0.01 is the pages' default).
+ *   dead_out device uint8 [g][K] (1 = dead), or NULL.
+ *   ws       device workspace of gptq_workspace_size(GPTQ_OP_PREPARE, K, 0, g, 0).
+ *   status   device int32 (see conventions). GPTQ_ERR_NONFINITE for NaN/Inf in H,
+ *            GPTQ_ERR_NOT_PD when a pivot p_j <= K * 2^-23 * Hd_jj (Hd the damped
+ *            matrix): the pivot is below the factorisation's rounding size.
+ */
+GPTQ_API gptq_status gptq_prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out,
+                         void *ws, size_t ws_bytes, int32_t *status, void *stream);
+
+/*
+ * gptaq_residual -- P1 = [(C U^T) ⊙ M] U with M the strict upper mask.
+ *
+ * [ResComp] item 3: P1 = [(dX X^T L) ⊙ M_U] L^T with H^-1 = L L^T, i.e. L = U^T in
+ * this layout; the strict mask makes row q equal C[q, F'] (H[F', F'])^-1 over the
+ * coordinates after q ([GPTAQ] "基于最优脑压缩的闭式解"), the residual term the
+ * sweep adds as w_q * P1[q, q+1:].
+ *
+ *   P1  device fp32 [K][K] output (strict upper; lower triangle and diagonal 0).
+ *   C   device fp32 [K][K] from gptaq_accumulate_cross.
+ *   U   device fp32 [K][K] from gptq_prepare (g = 1).
+ *   ws  gptq_workspace_size(GPTQ_OP_RESIDUAL, K, 0, 1, 0) bytes.
+ */
+GPTQ_API gptq_status gptaq_residual(float *P1, const float *C, const float *U, int K, void *ws,
+                           size_t ws_bytes, void *stream);
+
+/*
+ * gptq_quantize_layer -- the shared-order sweep with lazy blocks.
+ *
+ * [GPTQ blog] "GPTQ 怎样把逐个补偿变成可扩展算法": all channels take coordinates in
+ * the same order; for coordinate j, q = s (c - z) with
+ * c = clamp(round_half_even(w_j / s) + z, 0, 2^b - 1), E_j = (w_j - q) / U_jj, and
+ * W_k -= U_jk E_j for the block's later k at once; at the block end the far
+ * coordinates get W_far -= U[blk, far]^T E_blk. With P1 the GPTAQ row term
+ * w_j^pre * P1[j, k] is added the same way.
+ * Scale: per output channel s = 2 max_k |W[n][k]| / (2^b - 1) from W as given
+ * (before dead coordinates are zeroed), s = 1 for an all-zero channel; zero
+ * point z = 2^(b-1) ([G2PTQ] symmetric per-channel; [GPTQ blog] 4-bit grid
+ * {-8..7} as codes 0..15 with zero point 8).
+ *
+ *   W          device [N][K] weights, dtype wdtype. Read; overwritten with the
+ *              reconstruction s (c - z) when write_back != 0.
+ *   U          device fp32 [groups][K][K] from gptq_prepare; channel n uses
+ *              group n / (N / groups).
+ *   groups     >= 1, N % groups == 0.
+ *   bits       2, 3, 4 or 8.  blocksize 16, 32, 64 or 128.
+ *   P1         device fp32 [K][K] from gptaq_residual, or NULL (plain GPTQ).
+ *              Requires groups == 1.
+ *   dead       device uint8 [groups][K] from gptq_prepare, or NULL (none dead).
+ *   scales_in  device fp32 [N] fixed scales, or NULL (min-max as above).
+ *   scales_out device fp32 [N] the scales used, or NULL.
+ *   codes      device uint8 [N][K] codes c (required).
+ *   loss       device fp32 [N] with 1/2 sum_j E_j^2 per channel, or NULL.
+ *   ws         gptq_workspace_size(GPTQ_OP_QUANTIZE, K, N, groups, blocksize) bytes.
+ *   status     device int32: GPTQ_ERR_NONFINITE for NaN/Inf in W or scales.
+ */
+GPTQ_API gptq_status gptq_quantize_layer(void *W, int wdtype, int N, int K, const float *U, int groups,
+                                int bits, int blocksize, const float *P1, const uint8_t *dead,
+                                const float *scales_in, float *scales_out, uint8_t *codes,
+                                float *loss, int write_back, void *ws, size_t ws_bytes,
+                                int32_t *status, void *stream);
+
+/* Workspace bytes for an operation (gptq_op); 0 when none is needed. */
+GPTQ_API size_t gptq_workspace_size(int op, int K, int N, int g, int blocksize);
+
+/* Number of kernels this process has enqueued through the library so far
+ * (a host-side counter; for launch accounting in benchmarks). */
+GPTQ_API unsigned long long gptq_kernel_launches(void);
+
+/* Static, NUL-terminated description of a status code. */
+GPTQ_API const char *gptq_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPTQ_H */

@@ -155,7 +155,7 @@ def dequantize(c, s, bits):
 # The sweep in explicit OBQ form (no Cholesky, no lazy batching)
 # --------------------------------------------------------------------------------------
 
-def obq_sweep(H_d, W, s, bits, mode="schur", C=None, return_trace=False):
+def obq_sweep(H_d, W, s, bits, mode="schur", C=None, return_trace=False, steps=None):
     """Quantise coordinates 0..K-1 in order, compensating the free set each step.
 
     [GPTQ blog] "一次约束补偿的公式从哪里来": with free set F and P_F = (H[F, F])^-1, fixing
@@ -182,7 +182,8 @@ def obq_sweep(H_d, W, s, bits, mode="schur", C=None, return_trace=False):
     the row is a reading no printed value pins.
 
     Returns (codes, W_hat, loss) with loss[n] = sum_q r^2 / (2 (P_F)_qq), and the
-    per-step weights when return_trace.
+    per-step weights when return_trace. `steps` stops after the first `steps`
+    coordinates (a prefix of the same sweep; used to time a bounded sample).
     """
     H_d = np.asarray(H_d, dtype=np.float64)
     W = np.array(W, dtype=np.float64, copy=True)
@@ -192,7 +193,7 @@ def obq_sweep(H_d, W, s, bits, mode="schur", C=None, return_trace=False):
     loss = np.zeros(N)
     trace = []
     P = np.linalg.inv(H_d) if mode == "schur" else None
-    for q in range(K):
+    for q in range(K if steps is None else min(steps, K)):
         if mode == "direct":
             P = np.linalg.inv(H_d[q:, q:])
         # P is the inverse over F = {q, ..., K-1}; local index 0 is coordinate q.
@@ -297,7 +298,8 @@ def replay_row_form(U, W, s, bits, codes_gpu, P1=None, band=1e-4):
     continues with the other run's code, so one decision never cascades. A
     negative entry in codes_gpu means "no decision given": the oracle keeps its own.
 
-    Returns dict(codes, W_hat, tie_flips, mismatches, worst_tie_distance).
+    Returns dict(codes, W_hat, tie_flips, mismatches, worst_tie_distance, loss) with
+    loss[n] = 1/2 sum_j E_j^2 along the replayed trajectory.
     """
     U = np.asarray(U, dtype=np.float64)
     W = np.array(W, dtype=np.float64, copy=True)
@@ -309,6 +311,7 @@ def replay_row_form(U, W, s, bits, codes_gpu, P1=None, band=1e-4):
     tie_flips = 0
     mismatches = 0
     worst = 0.0
+    loss = np.zeros(N)
     for j in range(K):
         w = W[:, j].copy()
         c = quantize_codes(w, s, bits)
@@ -326,13 +329,14 @@ def replay_row_form(U, W, s, bits, codes_gpu, P1=None, band=1e-4):
             c = np.where(diff, G[:, j], c)
         target = s * (c - z)
         e = (w - target) / U[j, j]
+        loss += 0.5 * e * e
         W[:, j:] -= np.outer(e, U[j, j:])
         if P1 is not None and j + 1 < K:
             W[:, j + 1:] += np.outer(w, P1[j, j + 1:])
         W[:, j] = target
         codes[:, j] = c
     return dict(codes=codes, W_hat=W, tie_flips=tie_flips, mismatches=mismatches,
-                worst_tie_distance=worst)
+                worst_tie_distance=worst, loss=loss)
 
 
 # --------------------------------------------------------------------------------------

@@ -1,1 +1,184 @@
-"""GPTQ-family per-layer solve on B200 (sm_100a): thin binding over libgptq.so."""
+"""GPTQ-family per-layer solve on B200 (sm_100a): thin binding over libgptq.so.
+
+Each function here has the name of a C entry point of include/gptq.h and only
+marshals arguments: torch tensors supply device memory and the CUDA stream, every
+step of the solve runs in the library's kernels. There is no fallback: when the
+library is missing, every call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgptq.so")
+
+GPTQ_OK, GPTQ_ERR_ARG, GPTQ_ERR_NOT_PD, GPTQ_ERR_NONFINITE = 0, 1, 2, 3
+GPTQ_ERR_CUDA, GPTQ_ERR_TIMEOUT, GPTQ_ERR_WORKSPACE = 4, 5, 6
+GPTQ_BF16, GPTQ_F32 = 0, 1
+GPTQ_OP_PREPARE, GPTQ_OP_RESIDUAL, GPTQ_OP_QUANTIZE = 0, 1, 2
+
+EXPORTS = ("gptq_accumulate_hessian", "gptaq_accumulate_cross", "gptq_prepare",
+           "gptaq_residual", "gptq_quantize_layer", "gptq_workspace_size",
+           "gptq_kernel_launches", "gptq_status_string")
+
+_lib = None
+
+
+class GPTQError(RuntimeError):
+    def __init__(self, code, where=""):
+        self.code = int(code)
+        super().__init__(f"{where}: {gptq_status_string(code)} (status {self.code})")
+
+
+def load_library():
+    """Load libgptq.so from the package directory (raises if it was not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m post_weight_quantization_solve_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, I64, F, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    sig = {
+        "gptq_accumulate_hessian": [P, I, I, P, I, I64, I64, P, I64, P],
+        "gptaq_accumulate_cross": [P, I, P, P, I, I64, I64, P],
+        "gptq_prepare": [P, I, I, F, P, P, SZ, P, P],
+        "gptaq_residual": [P, P, P, I, P, SZ, P],
+        "gptq_quantize_layer": [P, I, I, I, P, I, I, I, P, P, P, P, P, P, I, P, SZ, P, P],
+        "gptq_workspace_size": [I, I, I, I, I],
+        "gptq_status_string": [I],
+        "gptq_kernel_launches": [],
+    }
+    for name, args in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int
+    lib.gptq_workspace_size.restype = ctypes.c_size_t
+    lib.gptq_status_string.restype = ctypes.c_char_p
+    lib.gptq_kernel_launches.restype = ctypes.c_ulonglong
+    _lib = lib
+    return lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return GPTQ_BF16
+    if t.dtype == torch.float32:
+        return GPTQ_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _check(code, where):
+    if code != GPTQ_OK:
+        raise GPTQError(code, where)
+
+
+def _workspace(nbytes, device, workspace):
+    if workspace is not None:
+        return workspace
+    return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+
+
+def new_status(device="cuda"):
+    """A zeroed device status word."""
+    return torch.zeros(1, dtype=torch.int32, device=device)
+
+
+def raise_on_status(status, where="gptq"):
+    """Synchronise with the status word's device and raise if a kernel failed."""
+    code = int(status.item())
+    _check(code, where)
+
+
+def gptq_status_string(code):
+    return load_library().gptq_status_string(int(code)).decode()
+
+
+def gptq_kernel_launches():
+    """Kernels enqueued through the library by this process so far."""
+    return int(load_library().gptq_kernel_launches())
+
+
+def gptq_workspace_size(op, K, N=0, g=1, blocksize=0):
+    return int(load_library().gptq_workspace_size(op, K, N, g, blocksize))
+
+
+def gptq_accumulate_hessian(H, X, w=None, stream=None):
+    """H[g] += 2 X^T diag(w[g]) X (see include/gptq.h). H: (K,K) or (g,K,K) fp32."""
+    lib = load_library()
+    K = H.shape[-1]
+    g = 1 if H.dim() == 2 else H.shape[0]
+    M = X.shape[0]
+    ldw = 0 if w is None else w.stride(0) if w.dim() == 2 else w.shape[-1]
+    code = lib.gptq_accumulate_hessian(_ptr(H), K, g, _ptr(X), _dtype_code(X), M, X.stride(0),
+                                       _ptr(w), ldw, _stream(stream))
+    _check(code, "gptq_accumulate_hessian")
+
+
+def gptaq_accumulate_cross(C, X_fp, X_q, stream=None):
+    """C += 2 (X_fp - X_q)^T X_q (see include/gptq.h)."""
+    lib = load_library()
+    if X_fp.stride(0) != X_q.stride(0) or X_fp.dtype != X_q.dtype or X_fp.shape != X_q.shape:
+        raise ValueError("X_fp and X_q must share shape, dtype and row stride")
+    code = lib.gptaq_accumulate_cross(_ptr(C), C.shape[-1], _ptr(X_fp), _ptr(X_q),
+                                      _dtype_code(X_q), X_q.shape[0], X_q.stride(0),
+                                      _stream(stream))
+    _check(code, "gptaq_accumulate_cross")
+
+
+def gptq_prepare(H, percdamp=0.01, dead_out=None, workspace=None, status=None, stream=None):
+    """In place: dead fix, damping, H -> U. Returns the status tensor (not synchronised)."""
+    lib = load_library()
+    K = H.shape[-1]
+    g = 1 if H.dim() == 2 else H.shape[0]
+    status = new_status(H.device) if status is None else status
+    ws = _workspace(gptq_workspace_size(GPTQ_OP_PREPARE, K, 0, g, 0), H.device, workspace)
+    code = lib.gptq_prepare(_ptr(H), K, g, float(percdamp), _ptr(dead_out), _ptr(ws),
+                            ws.numel() * ws.element_size(), _ptr(status), _stream(stream))
+    _check(code, "gptq_prepare")
+    return status
+
+
+def gptaq_residual(P1, C, U, workspace=None, stream=None):
+    """P1 = [(C U^T) ⊙ strict-upper] U (see include/gptq.h)."""
+    lib = load_library()
+    K = U.shape[-1]
+    ws = _workspace(gptq_workspace_size(GPTQ_OP_RESIDUAL, K, 0, 1, 0), U.device, workspace)
+    code = lib.gptaq_residual(_ptr(P1), _ptr(C), _ptr(U), K, _ptr(ws),
+                              ws.numel() * ws.element_size(), _stream(stream))
+    _check(code, "gptaq_residual")
+
+
+def gptq_quantize_layer(W, U, bits, blocksize=128, groups=1, P1=None, dead=None, scales_in=None,
+                        scales_out=None, codes=None, loss=None, write_back=False,
+                        workspace=None, status=None, stream=None):
+    """The shared-order sweep. Returns (codes, status); see include/gptq.h."""
+    lib = load_library()
+    N, K = W.shape
+    if codes is None:
+        codes = torch.empty(N, K, dtype=torch.uint8, device=W.device)
+    status = new_status(W.device) if status is None else status
+    ws = _workspace(gptq_workspace_size(GPTQ_OP_QUANTIZE, K, N, groups, blocksize), W.device,
+                    workspace)
+    code = lib.gptq_quantize_layer(_ptr(W), _dtype_code(W), N, K, _ptr(U), groups, bits,
+                                   blocksize, _ptr(P1), _ptr(dead), _ptr(scales_in),
+                                   _ptr(scales_out), _ptr(codes), _ptr(loss), int(write_back),
+                                   _ptr(ws), ws.numel() * ws.element_size(), _ptr(status),
+                                   _stream(stream))
+    _check(code, "gptq_quantize_layer")
+    return codes, status

@@ -1,0 +1,139 @@
+// C ABI entry points: argument checks, workspace sizing, dispatch. Every check
+// here runs on the host before anything is enqueued.
+#include "common.cuh"
+
+namespace gptq {
+gptq_status gram_simt(float *H, int K, int g, const void *X, int xdtype, int64_t M, int64_t ldx,
+                      const float *w, int64_t ldw, cudaStream_t st);
+gptq_status cross_simt(float *C, int K, const void *Xfp, const void *Xq, int xdtype, int64_t M,
+                       int64_t ldx, cudaStream_t st);
+gptq_status gram_tc(float *H, int K, int g, const void *X, int64_t M, int64_t ldx,
+                    const float *w, int64_t ldw, const void *X2, cudaStream_t st, bool *used);
+size_t prepare_workspace(int K, int g);
+gptq_status prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out, void *ws,
+                    int32_t *status, cudaStream_t st);
+size_t residual_workspace(int K);
+gptq_status residual(float *P1, const float *C, const float *U, int K, void *ws, cudaStream_t st);
+size_t quantize_workspace(int K, int N, int g, int blocksize);
+gptq_status quantize_layer(void *W, int wdtype, int N, int K, const float *U, int groups, int bits,
+                           int blocksize, const float *P1, const uint8_t *dead,
+                           const float *scales_in, float *scales_out, uint8_t *codes, float *loss,
+                           int write_back, void *ws, int32_t *status, cudaStream_t st);
+}  // namespace gptq
+
+namespace gptq {
+unsigned long long g_launches = 0;
+}
+
+using namespace gptq;
+
+static bool valid_dtype(int d) { return d == GPTQ_BF16 || d == GPTQ_F32; }
+
+static bool stream_ok(int xdtype, const void *X, int64_t ldx, int K) {
+    if (ldx < K) return false;
+    if (xdtype == GPTQ_BF16) return aligned(X, 16) && ldx % 8 == 0;
+    return aligned(X, 4);
+}
+
+extern "C" {
+
+gptq_status gptq_accumulate_hessian(float *H, int K, int g, const void *X, int xdtype, int64_t M,
+                                    int64_t ldx, const float *w, int64_t ldw, void *stream) {
+    if (K < 1 || g < 1 || M < 0 || !H || !valid_dtype(xdtype)) return GPTQ_ERR_ARG;
+    if (M > 0x7fffffff) return GPTQ_ERR_ARG;
+    if (w == nullptr && g != 1) return GPTQ_ERR_ARG;
+    if (w != nullptr && ldw < M) return GPTQ_ERR_ARG;
+    if (M == 0) return GPTQ_OK;
+    if (!X || !stream_ok(xdtype, X, ldx, K)) return GPTQ_ERR_ARG;
+    if (xdtype == GPTQ_BF16 && K % 8 != 0) return GPTQ_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (xdtype == GPTQ_BF16) {
+        bool used = false;
+        gptq_status s = gram_tc(H, K, g, X, M, ldx, w, ldw, nullptr, st, &used);
+        if (used || s != GPTQ_OK) return s;
+    }
+    return gram_simt(H, K, g, X, xdtype, M, ldx, w, ldw, st);
+}
+
+gptq_status gptaq_accumulate_cross(float *C, int K, const void *X_fp, const void *X_q, int xdtype,
+                                   int64_t M, int64_t ldx, void *stream) {
+    if (K < 1 || M < 0 || !C || !valid_dtype(xdtype)) return GPTQ_ERR_ARG;
+    if (M > 0x7fffffff) return GPTQ_ERR_ARG;
+    if (M == 0) return GPTQ_OK;
+    if (!X_fp || !X_q || !stream_ok(xdtype, X_fp, ldx, K) || !stream_ok(xdtype, X_q, ldx, K))
+        return GPTQ_ERR_ARG;
+    if (xdtype == GPTQ_BF16 && K % 8 != 0) return GPTQ_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (xdtype == GPTQ_BF16) {
+        bool used = false;
+        gptq_status s = gram_tc(C, K, 1, X_q, M, ldx, nullptr, 0, X_fp, st, &used);
+        if (used || s != GPTQ_OK) return s;
+    }
+    return cross_simt(C, K, X_fp, X_q, xdtype, M, ldx, st);
+}
+
+gptq_status gptq_prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out, void *ws,
+                         size_t ws_bytes, int32_t *status, void *stream) {
+    if (K < 1 || g < 1 || !H || !status || !(percdamp >= 0.f) || !aligned(H, 16))
+        return GPTQ_ERR_ARG;
+    if (!ws || !aligned(ws, 256) || ws_bytes < prepare_workspace(K, g)) return GPTQ_ERR_WORKSPACE;
+    return prepare(H, K, g, percdamp, dead_out, ws, status, static_cast<cudaStream_t>(stream));
+}
+
+gptq_status gptaq_residual(float *P1, const float *C, const float *U, int K, void *ws,
+                           size_t ws_bytes, void *stream) {
+    if (K < 1 || !P1 || !C || !U) return GPTQ_ERR_ARG;
+    if (!ws || !aligned(ws, 256) || ws_bytes < residual_workspace(K)) return GPTQ_ERR_WORKSPACE;
+    return residual(P1, C, U, K, ws, static_cast<cudaStream_t>(stream));
+}
+
+gptq_status gptq_quantize_layer(void *W, int wdtype, int N, int K, const float *U, int groups,
+                                int bits, int blocksize, const float *P1, const uint8_t *dead,
+                                const float *scales_in, float *scales_out, uint8_t *codes,
+                                float *loss, int write_back, void *ws, size_t ws_bytes,
+                                int32_t *status, void *stream) {
+    if (N < 1 || K < 1 || groups < 1 || N % groups != 0 || !W || !U || !codes || !status)
+        return GPTQ_ERR_ARG;
+    if (!valid_dtype(wdtype)) return GPTQ_ERR_ARG;
+    if (bits != 2 && bits != 3 && bits != 4 && bits != 8) return GPTQ_ERR_ARG;
+    if (blocksize != 16 && blocksize != 32 && blocksize != 64 && blocksize != 128)
+        return GPTQ_ERR_ARG;
+    if (P1 && groups != 1) return GPTQ_ERR_ARG;
+    if (!aligned(U, 16) || (P1 && !aligned(P1, 16))) return GPTQ_ERR_ARG;
+    if (!ws || !aligned(ws, 256) || ws_bytes < quantize_workspace(K, N, groups, blocksize))
+        return GPTQ_ERR_WORKSPACE;
+    return quantize_layer(W, wdtype, N, K, U, groups, bits, blocksize, P1, dead, scales_in,
+                          scales_out, codes, loss, write_back, ws, status,
+                          static_cast<cudaStream_t>(stream));
+}
+
+size_t gptq_workspace_size(int op, int K, int N, int g, int blocksize) {
+    if (K < 1 || g < 1) return 0;
+    switch (op) {
+        case GPTQ_OP_PREPARE: return prepare_workspace(K, g);
+        case GPTQ_OP_RESIDUAL: return residual_workspace(K);
+        case GPTQ_OP_QUANTIZE:
+            if (N < 1 || blocksize < 1) return 0;
+            return quantize_workspace(K, N, g, blocksize);
+        default: return 0;
+    }
+}
+
+unsigned long long gptq_kernel_launches(void) {
+    return __atomic_load_n(&g_launches, __ATOMIC_RELAXED);
+}
+
+const char *gptq_status_string(int status) {
+    switch (status) {
+        case GPTQ_OK: return "ok";
+        case GPTQ_ERR_ARG: return "invalid argument";
+        case GPTQ_ERR_NOT_PD: return "damped Hessian is not positive definite";
+        case GPTQ_ERR_NONFINITE: return "non-finite value in an input or intermediate";
+        case GPTQ_ERR_CUDA: return "CUDA launch or API error";
+        case GPTQ_ERR_TIMEOUT: return "bounded device wait ran out";
+        case GPTQ_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        default: return "unknown status";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,100 @@
+"""The C-ABI library loads on a machine without a GPU, exports every entry point
+that include/gptq.h declares, and rejects bad arguments on the host before any
+device work (no compute call is made here)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import post_weight_quantization_solve_b200 as gq
+from post_weight_quantization_solve_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return gq.load_library()
+
+
+def header_entry_points():
+    text = open(os.path.join(ROOT, "include", "gptq.h"), encoding="utf-8").read()
+    return re.findall(r"GPTQ_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+
+
+def test_exports_every_declared_symbol(lib):
+    names = header_entry_points()
+    assert set(names) == set(gq.EXPORTS)
+    for name in names:
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        assert gq.gptq_status_string(code) not in ("", "unknown status")
+    assert gq.gptq_status_string(99) == "unknown status"
+
+
+def test_workspace_sizes(lib):
+    p1 = gq.gptq_workspace_size(gq.GPTQ_OP_PREPARE, 4096, 0, 1, 0)
+    p4 = gq.gptq_workspace_size(gq.GPTQ_OP_PREPARE, 4096, 0, 4, 0)
+    assert p1 > 4096 * 4 and p4 > 3 * p1
+    q = gq.gptq_workspace_size(gq.GPTQ_OP_QUANTIZE, 4096, 14336, 1, 128)
+    assert q >= 4096 * 14336 * 4
+    assert gq.gptq_workspace_size(gq.GPTQ_OP_RESIDUAL, 512, 0, 1, 0) >= 512 * 512 * 4
+    assert gq.gptq_workspace_size(7, 128, 1, 1, 1) == 0
+    assert gq.gptq_workspace_size(gq.GPTQ_OP_PREPARE, 0, 0, 1, 0) == 0
+
+
+def test_host_argument_checks(lib):
+    P = ctypes.c_void_p
+    fake = P(1 << 20)   # never dereferenced: every call below fails its host checks
+    ws = P(1 << 21)
+    # quantize: bits, blocksize, groups, NULL pointers, GPTAQ with groups
+    assert lib.gptq_quantize_layer(fake, 0, 8, 16, fake, 1, 5, 128, None, None, None, None,
+                                   fake, None, 0, ws, 1 << 30, fake, None) == gq.GPTQ_ERR_ARG
+    assert lib.gptq_quantize_layer(fake, 0, 8, 16, fake, 1, 4, 256, None, None, None, None,
+                                   fake, None, 0, ws, 1 << 30, fake, None) == gq.GPTQ_ERR_ARG
+    assert lib.gptq_quantize_layer(fake, 0, 9, 16, fake, 2, 4, 128, None, None, None, None,
+                                   fake, None, 0, ws, 1 << 30, fake, None) == gq.GPTQ_ERR_ARG
+    assert lib.gptq_quantize_layer(fake, 0, 8, 16, fake, 2, 4, 128, fake, None, None, None,
+                                   fake, None, 0, ws, 1 << 30, fake, None) == gq.GPTQ_ERR_ARG
+    assert lib.gptq_quantize_layer(fake, 0, 8, 16, fake, 1, 4, 128, None, None, None, None,
+                                   None, None, 0, ws, 1 << 30, fake, None) == gq.GPTQ_ERR_ARG
+    assert lib.gptq_quantize_layer(fake, 0, 8, 16, fake, 1, 4, 128, None, None, None, None,
+                                   fake, None, 0, ws, 16, fake, None) == gq.GPTQ_ERR_WORKSPACE
+    assert lib.gptq_quantize_layer(fake, 0, 8, 16, fake, 1, 4, 128, None, None, None, None,
+                                   fake, None, 0, P((1 << 21) + 8), 1 << 30, fake,
+                                   None) == gq.GPTQ_ERR_WORKSPACE
+    # prepare: negative damping, missing status, small workspace
+    assert lib.gptq_prepare(fake, 16, 1, ctypes.c_float(-0.1), None, ws, 1 << 30, fake,
+                            None) == gq.GPTQ_ERR_ARG
+    assert lib.gptq_prepare(fake, 16, 1, ctypes.c_float(0.01), None, ws, 1 << 30, None,
+                            None) == gq.GPTQ_ERR_ARG
+    assert lib.gptq_prepare(fake, 4096, 1, ctypes.c_float(0.01), None, ws, 64, fake,
+                            None) == gq.GPTQ_ERR_WORKSPACE
+    # Hessian: bf16 needs K % 8 == 0 and 16-byte aligned rows; g > 1 needs weights
+    assert lib.gptq_accumulate_hessian(fake, 12, 1, fake, gq.GPTQ_BF16, 10, 12, None, 0,
+                                       None) == gq.GPTQ_ERR_ARG
+    assert lib.gptq_accumulate_hessian(fake, 16, 1, fake, gq.GPTQ_BF16, 10, 20, None, 0,
+                                       None) == gq.GPTQ_ERR_ARG
+    assert lib.gptq_accumulate_hessian(fake, 16, 2, fake, gq.GPTQ_BF16, 10, 16, None, 0,
+                                       None) == gq.GPTQ_ERR_ARG
+    assert lib.gptq_accumulate_hessian(fake, 16, 1, fake, 7, 10, 16, None, 0,
+                                       None) == gq.GPTQ_ERR_ARG
+    # M == 0 is a no-op that succeeds without touching the device
+    assert lib.gptq_accumulate_hessian(fake, 16, 1, fake, gq.GPTQ_BF16, 0, 16, None, 0,
+                                       None) == gq.GPTQ_OK
+    assert lib.gptaq_accumulate_cross(fake, 16, fake, fake, gq.GPTQ_BF16, 0, 16,
+                                      None) == gq.GPTQ_OK
+    assert lib.gptaq_residual(fake, fake, fake, 16, ws, 8, None) == gq.GPTQ_ERR_WORKSPACE
+
+
+def test_product_path_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(gq, "_lib", None)
+    monkeypatch.setattr(gq, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        gq.load_library()
