@@ -78,18 +78,18 @@ def test_host_argument_checks(lib):
                             None) == gq.GPTQ_ERR_WORKSPACE
     # Hessian: bf16 needs K % 8 == 0 and 16-byte aligned rows; g > 1 needs weights
     assert lib.gptq_accumulate_hessian(fake, 12, 1, fake, gq.GPTQ_BF16, 10, 12, None, 0,
-                                       None) == gq.GPTQ_ERR_ARG
+                                       None, None) == gq.GPTQ_ERR_ARG
     assert lib.gptq_accumulate_hessian(fake, 16, 1, fake, gq.GPTQ_BF16, 10, 20, None, 0,
-                                       None) == gq.GPTQ_ERR_ARG
+                                       None, None) == gq.GPTQ_ERR_ARG
     assert lib.gptq_accumulate_hessian(fake, 16, 2, fake, gq.GPTQ_BF16, 10, 16, None, 0,
-                                       None) == gq.GPTQ_ERR_ARG
+                                       None, None) == gq.GPTQ_ERR_ARG
     assert lib.gptq_accumulate_hessian(fake, 16, 1, fake, 7, 10, 16, None, 0,
-                                       None) == gq.GPTQ_ERR_ARG
+                                       None, None) == gq.GPTQ_ERR_ARG
     # M == 0 is a no-op that succeeds without touching the device
     assert lib.gptq_accumulate_hessian(fake, 16, 1, fake, gq.GPTQ_BF16, 0, 16, None, 0,
-                                       None) == gq.GPTQ_OK
+                                       None, None) == gq.GPTQ_OK
     assert lib.gptaq_accumulate_cross(fake, 16, fake, fake, gq.GPTQ_BF16, 0, 16,
-                                      None) == gq.GPTQ_OK
+                                      None, None) == gq.GPTQ_OK
     assert lib.gptaq_residual(fake, fake, fake, 16, ws, 8, None) == gq.GPTQ_ERR_WORKSPACE
 
 
