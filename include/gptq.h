@@ -85,11 +85,16 @@ typedef enum {
  *          (ldx % 8 == 0). ldx >= K.
  *   M      tokens in this chunk (>= 0; 0 is a no-op).
  *   w      device fp32 [g][ldw] per-token weights, or NULL for unit weights.
+ *   status device int32 or NULL (see conventions): GPTQ_ERR_TIMEOUT if a bounded
+ *          wait inside the tensor-core kernel ran out; the call is skipped when the
+ *          word is already non-zero.
  *   Errors: GPTQ_ERR_ARG for bad sizes/alignment/dtype, GPTQ_ERR_CUDA on launch.
+ *   Paths: bf16 with g == 1 and w == NULL runs on the tensor cores (tcgen05, TMA);
+ *   fp32 streams and weighted Hessians run the fp32 SIMT kernel.
  */
 GPTQ_API gptq_status gptq_accumulate_hessian(float *H, int K, int g, const void *X, int xdtype,
                                     int64_t M, int64_t ldx, const float *w, int64_t ldw,
-                                    void *stream);
+                                    int32_t *status, void *stream);
 
 /*
  * gptaq_accumulate_cross -- C += 2 * (X_fp - X_q)^T X_q over one token chunk.
@@ -103,9 +108,11 @@ GPTQ_API gptq_status gptq_accumulate_hessian(float *H, int K, int g, const void 
  *          symmetric: C[i][j] = 2 sum_m dX[m][i] X_q[m][j].
  *   X_fp, X_q  device [M][ldx] each, same dtype and leading dimension; alignment
  *          rules as gptq_accumulate_hessian.
+ *   status device int32 or NULL, as in gptq_accumulate_hessian.
  */
 GPTQ_API gptq_status gptaq_accumulate_cross(float *C, int K, const void *X_fp, const void *X_q,
-                                   int xdtype, int64_t M, int64_t ldx, void *stream);
+                                   int xdtype, int64_t M, int64_t ldx, int32_t *status,
+                                   void *stream);
 
 /*
  * gptq_prepare -- dead coordinates, damping and the upper factor U, in place.

@@ -45,8 +45,8 @@ def load_library():
     lib = ctypes.CDLL(LIB_PATH)
     P, I, I64, F, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
     sig = {
-        "gptq_accumulate_hessian": [P, I, I, P, I, I64, I64, P, I64, P],
-        "gptaq_accumulate_cross": [P, I, P, P, I, I64, I64, P],
+        "gptq_accumulate_hessian": [P, I, I, P, I, I64, I64, P, I64, P, P],
+        "gptaq_accumulate_cross": [P, I, P, P, I, I64, I64, P, P],
         "gptq_prepare": [P, I, I, F, P, P, SZ, P, P],
         "gptaq_residual": [P, P, P, I, P, SZ, P],
         "gptq_quantize_layer": [P, I, I, I, P, I, I, I, P, P, P, P, P, P, I, P, SZ, P, P],
@@ -118,7 +118,7 @@ def gptq_workspace_size(op, K, N=0, g=1, blocksize=0):
     return int(load_library().gptq_workspace_size(op, K, N, g, blocksize))
 
 
-def gptq_accumulate_hessian(H, X, w=None, stream=None):
+def gptq_accumulate_hessian(H, X, w=None, status=None, stream=None):
     """H[g] += 2 X^T diag(w[g]) X (see include/gptq.h). H: (K,K) or (g,K,K) fp32."""
     lib = load_library()
     K = H.shape[-1]
@@ -126,18 +126,18 @@ def gptq_accumulate_hessian(H, X, w=None, stream=None):
     M = X.shape[0]
     ldw = 0 if w is None else w.stride(0) if w.dim() == 2 else w.shape[-1]
     code = lib.gptq_accumulate_hessian(_ptr(H), K, g, _ptr(X), _dtype_code(X), M, X.stride(0),
-                                       _ptr(w), ldw, _stream(stream))
+                                       _ptr(w), ldw, _ptr(status), _stream(stream))
     _check(code, "gptq_accumulate_hessian")
 
 
-def gptaq_accumulate_cross(C, X_fp, X_q, stream=None):
+def gptaq_accumulate_cross(C, X_fp, X_q, status=None, stream=None):
     """C += 2 (X_fp - X_q)^T X_q (see include/gptq.h)."""
     lib = load_library()
     if X_fp.stride(0) != X_q.stride(0) or X_fp.dtype != X_q.dtype or X_fp.shape != X_q.shape:
         raise ValueError("X_fp and X_q must share shape, dtype and row stride")
     code = lib.gptaq_accumulate_cross(_ptr(C), C.shape[-1], _ptr(X_fp), _ptr(X_q),
                                       _dtype_code(X_q), X_q.shape[0], X_q.stride(0),
-                                      _stream(stream))
+                                      _ptr(status), _stream(stream))
     _check(code, "gptaq_accumulate_cross")
 
 

@@ -4,11 +4,12 @@
 
 namespace gptq {
 gptq_status gram_simt(float *H, int K, int g, const void *X, int xdtype, int64_t M, int64_t ldx,
-                      const float *w, int64_t ldw, cudaStream_t st);
+                      const float *w, int64_t ldw, const int32_t *status, cudaStream_t st);
 gptq_status cross_simt(float *C, int K, const void *Xfp, const void *Xq, int xdtype, int64_t M,
-                       int64_t ldx, cudaStream_t st);
+                       int64_t ldx, const int32_t *status, cudaStream_t st);
 gptq_status gram_tc(float *H, int K, int g, const void *X, int64_t M, int64_t ldx,
-                    const float *w, int64_t ldw, const void *X2, cudaStream_t st, bool *used);
+                    const float *w, int64_t ldw, const void *X2, cudaStream_t st, int32_t *status,
+                    bool *used);
 size_t prepare_workspace(int K, int g);
 gptq_status prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out, void *ws,
                     int32_t *status, cudaStream_t st);
@@ -38,7 +39,8 @@ static bool stream_ok(int xdtype, const void *X, int64_t ldx, int K) {
 extern "C" {
 
 gptq_status gptq_accumulate_hessian(float *H, int K, int g, const void *X, int xdtype, int64_t M,
-                                    int64_t ldx, const float *w, int64_t ldw, void *stream) {
+                                    int64_t ldx, const float *w, int64_t ldw, int32_t *status,
+                                    void *stream) {
     if (K < 1 || g < 1 || M < 0 || !H || !valid_dtype(xdtype)) return GPTQ_ERR_ARG;
     if (M > 0x7fffffff) return GPTQ_ERR_ARG;
     if (w == nullptr && g != 1) return GPTQ_ERR_ARG;
@@ -49,14 +51,14 @@ gptq_status gptq_accumulate_hessian(float *H, int K, int g, const void *X, int x
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (xdtype == GPTQ_BF16) {
         bool used = false;
-        gptq_status s = gram_tc(H, K, g, X, M, ldx, w, ldw, nullptr, st, &used);
+        gptq_status s = gram_tc(H, K, g, X, M, ldx, w, ldw, nullptr, st, status, &used);
         if (used || s != GPTQ_OK) return s;
     }
-    return gram_simt(H, K, g, X, xdtype, M, ldx, w, ldw, st);
+    return gram_simt(H, K, g, X, xdtype, M, ldx, w, ldw, status, st);
 }
 
 gptq_status gptaq_accumulate_cross(float *C, int K, const void *X_fp, const void *X_q, int xdtype,
-                                   int64_t M, int64_t ldx, void *stream) {
+                                   int64_t M, int64_t ldx, int32_t *status, void *stream) {
     if (K < 1 || M < 0 || !C || !valid_dtype(xdtype)) return GPTQ_ERR_ARG;
     if (M > 0x7fffffff) return GPTQ_ERR_ARG;
     if (M == 0) return GPTQ_OK;
@@ -64,12 +66,7 @@ gptq_status gptaq_accumulate_cross(float *C, int K, const void *X_fp, const void
         return GPTQ_ERR_ARG;
     if (xdtype == GPTQ_BF16 && K % 8 != 0) return GPTQ_ERR_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (xdtype == GPTQ_BF16) {
-        bool used = false;
-        gptq_status s = gram_tc(C, K, 1, X_q, M, ldx, nullptr, 0, X_fp, st, &used);
-        if (used || s != GPTQ_OK) return s;
-    }
-    return cross_simt(C, K, X_fp, X_q, xdtype, M, ldx, st);
+    return cross_simt(C, K, X_fp, X_q, xdtype, M, ldx, status, st);
 }
 
 gptq_status gptq_prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out, void *ws,

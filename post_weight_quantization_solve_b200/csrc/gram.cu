@@ -40,9 +40,10 @@ gptq_status mirror_upper(float *H, int K, int g, cudaStream_t st) {
 }
 
 gptq_status gram_simt(float *H, int K, int g, const void *X, int xdtype, int64_t M,
-                      int64_t ldx, const float *w, int64_t ldw, cudaStream_t st) {
+                      int64_t ldx, const float *w, int64_t ldw, const int32_t *status,
+                      cudaStream_t st) {
     // H(i,j) += 2 sum_m X[m][i] w[m] X[m][j]: A(i,m) = X[m*ldx + i] (transposed view)
-    GemmParams p = gemm_params(K, K, (int)M, X, ldx, X, ldx, H, K, 2.f, 1, nullptr);
+    GemmParams p = gemm_params(K, K, (int)M, X, ldx, X, ldx, H, K, 2.f, 1, status);
     p.upper_tiles = 1;
     p.kscale = w;
     p.sK = ldw;
@@ -55,8 +56,8 @@ gptq_status gram_simt(float *H, int K, int g, const void *X, int xdtype, int64_t
 }
 
 gptq_status cross_simt(float *C, int K, const void *Xfp, const void *Xq, int xdtype, int64_t M,
-                       int64_t ldx, cudaStream_t st) {
-    GemmParams p = gemm_params(K, K, (int)M, Xfp, ldx, Xq, ldx, C, K, 2.f, 1, nullptr);
+                       int64_t ldx, const int32_t *status, cudaStream_t st) {
+    GemmParams p = gemm_params(K, K, (int)M, Xfp, ldx, Xq, ldx, C, K, 2.f, 1, status);
     p.A2 = Xq;
     return (xdtype == GPTQ_F32) ? gemm_simt<float, float, true, false>(p, 1, st)
                                 : gemm_simt<__nv_bfloat16, __nv_bfloat16, true, false>(p, 1, st);
