@@ -138,6 +138,33 @@ GPTQ_API gptq_status gptq_prepare(float *H, int K, int g, float percdamp, uint8_
                          void *ws, size_t ws_bytes, int32_t *status, void *stream);
 
 /*
+ * gptq_prepare_noalloc -- gptq_prepare without a caller workspace.
+ *
+ * The pages have no counterpart of this call; it exists for callers that cannot
+ * allocate device memory when they need the factor, for example code running
+ * inside a host application that owns every device allocation through its own
+ * pool and hands plug-ins no workspace, or a latency-critical path that must not
+ * take the device-wide synchronisation of cudaMalloc / cudaFree. It computes
+ * exactly what gptq_prepare computes, with the same arguments minus the
+ * workspace, and allocates nothing: its scratch is a fixed 16 MiB + 64 KiB array
+ * in the library's device memory, which every GPU that loads the library holds
+ * until the process exits.
+ *
+ *   Limit: gptq_workspace_size(GPTQ_OP_PREPARE, K, 0, g, 0) must not exceed that
+ *   array (K <= 4096 with g = 1, K <= 2048 with g <= 4); larger sizes return
+ *   GPTQ_ERR_ARG before anything is enqueued.
+ *   Set-up: the first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call before
+ *   any stream capture.
+ *   Sharing: every call on a device uses the same array, and the array keeps the
+ *   last call's contents (nothing in it needs to start at zero). Calls whose
+ *   kernels overlap on the GPU (for example on two streams at once) race on the
+ *   array: serialise them.
+ */
+GPTQ_API gptq_status gptq_prepare_noalloc(float *H, int K, int g, float percdamp,
+                                          uint8_t *dead_out, int32_t *status, void *stream);
+
+/*
  * gptaq_residual -- P1 = [(C U^T) ⊙ M] U with M the strict upper mask.
  *
  * [ResComp] item 3: P1 = [(dX X^T L) ⊙ M_U] L^T with H^-1 = L L^T, i.e. L = U^T in

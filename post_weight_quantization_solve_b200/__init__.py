@@ -22,6 +22,7 @@ GPTQ_BF16, GPTQ_F32 = 0, 1
 GPTQ_OP_PREPARE, GPTQ_OP_RESIDUAL, GPTQ_OP_QUANTIZE = 0, 1, 2
 
 EXPORTS = ("gptq_accumulate_hessian", "gptaq_accumulate_cross", "gptq_prepare",
+           "gptq_prepare_noalloc",
            "gptaq_residual", "gptq_quantize_layer", "gptq_workspace_size",
            "gptq_kernel_launches", "gptq_status_string")
 
@@ -48,6 +49,7 @@ def load_library():
         "gptq_accumulate_hessian": [P, I, I, P, I, I64, I64, P, I64, P, P],
         "gptaq_accumulate_cross": [P, I, P, P, I, I64, I64, P, P],
         "gptq_prepare": [P, I, I, F, P, P, SZ, P, P],
+        "gptq_prepare_noalloc": [P, I, I, F, P, P, P],
         "gptaq_residual": [P, P, P, I, P, SZ, P],
         "gptq_quantize_layer": [P, I, I, I, P, I, I, I, P, P, P, P, P, P, I, P, SZ, P, P],
         "gptq_workspace_size": [I, I, I, I, I],
@@ -151,6 +153,20 @@ def gptq_prepare(H, percdamp=0.01, dead_out=None, workspace=None, status=None, s
     code = lib.gptq_prepare(_ptr(H), K, g, float(percdamp), _ptr(dead_out), _ptr(ws),
                             ws.numel() * ws.element_size(), _ptr(status), _stream(stream))
     _check(code, "gptq_prepare")
+    return status
+
+
+def gptq_prepare_noalloc(H, percdamp=0.01, dead_out=None, status=None, stream=None):
+    """gptq_prepare with the library's fixed device scratch instead of a workspace
+    (no allocation anywhere on this path). Returns the status tensor."""
+    lib = load_library()
+    K = H.shape[-1]
+    g = 1 if H.dim() == 2 else H.shape[0]
+    if status is None:
+        raise ValueError("gptq_prepare_noalloc needs a caller-provided status word")
+    code = lib.gptq_prepare_noalloc(_ptr(H), K, g, float(percdamp), _ptr(dead_out),
+                                    _ptr(status), _stream(stream))
+    _check(code, "gptq_prepare_noalloc")
     return status
 
 
