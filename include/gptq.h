@@ -62,6 +62,9 @@ typedef enum {
 
 typedef enum { GPTQ_BF16 = 0, GPTQ_F32 = 1 } gptq_dtype;
 
+/* Largest K (input coordinates) and N (output channels) any call accepts. */
+#define GPTQ_MAX_DIM 65535
+
 typedef enum {
     GPTQ_OP_PREPARE = 0,
     GPTQ_OP_RESIDUAL = 1,
@@ -198,7 +201,7 @@ GPTQ_API gptq_status gptaq_residual(float *P1, const float *C, const float *U, i
  *              reconstruction s (c - z) when write_back != 0.
  *   U          device fp32 [groups][K][K] from gptq_prepare; channel n uses
  *              group n / (N / groups).
- *   groups     >= 1, N % groups == 0.
+ *   groups     1..8, N % groups == 0.
  *   bits       2, 3, 4 or 8.  blocksize 16, 32, 64 or 128.
  *   P1         device fp32 [K][K] from gptaq_residual, or NULL (plain GPTQ).
  *              Requires groups == 1.

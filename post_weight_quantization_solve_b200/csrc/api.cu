@@ -41,7 +41,8 @@ extern "C" {
 gptq_status gptq_accumulate_hessian(float *H, int K, int g, const void *X, int xdtype, int64_t M,
                                     int64_t ldx, const float *w, int64_t ldw, int32_t *status,
                                     void *stream) {
-    if (K < 1 || g < 1 || M < 0 || !H || !valid_dtype(xdtype)) return GPTQ_ERR_ARG;
+    if (K < 1 || K > GPTQ_MAX_DIM || g < 1 || g > 65535 || M < 0 || !H || !valid_dtype(xdtype))
+        return GPTQ_ERR_ARG;
     if (M > 0x7fffffff) return GPTQ_ERR_ARG;
     if (w == nullptr && g != 1) return GPTQ_ERR_ARG;
     if (w != nullptr && ldw < M) return GPTQ_ERR_ARG;
@@ -59,7 +60,7 @@ gptq_status gptq_accumulate_hessian(float *H, int K, int g, const void *X, int x
 
 gptq_status gptaq_accumulate_cross(float *C, int K, const void *X_fp, const void *X_q, int xdtype,
                                    int64_t M, int64_t ldx, int32_t *status, void *stream) {
-    if (K < 1 || M < 0 || !C || !valid_dtype(xdtype)) return GPTQ_ERR_ARG;
+    if (K < 1 || K > GPTQ_MAX_DIM || M < 0 || !C || !valid_dtype(xdtype)) return GPTQ_ERR_ARG;
     if (M > 0x7fffffff) return GPTQ_ERR_ARG;
     if (M == 0) return GPTQ_OK;
     if (!X_fp || !X_q || !stream_ok(xdtype, X_fp, ldx, K) || !stream_ok(xdtype, X_q, ldx, K))
@@ -73,13 +74,14 @@ gptq_status gptq_prepare(float *H, int K, int g, float percdamp, uint8_t *dead_o
                          size_t ws_bytes, int32_t *status, void *stream) {
     if (K < 1 || g < 1 || !H || !status || !(percdamp >= 0.f) || !aligned(H, 16))
         return GPTQ_ERR_ARG;
+    if (K > GPTQ_MAX_DIM || g > 65535) return GPTQ_ERR_ARG;
     if (!ws || !aligned(ws, 256) || ws_bytes < prepare_workspace(K, g)) return GPTQ_ERR_WORKSPACE;
     return prepare(H, K, g, percdamp, dead_out, ws, status, static_cast<cudaStream_t>(stream));
 }
 
 gptq_status gptaq_residual(float *P1, const float *C, const float *U, int K, void *ws,
                            size_t ws_bytes, void *stream) {
-    if (K < 1 || !P1 || !C || !U) return GPTQ_ERR_ARG;
+    if (K < 1 || K > GPTQ_MAX_DIM || !P1 || !C || !U) return GPTQ_ERR_ARG;
     if (!ws || !aligned(ws, 256) || ws_bytes < residual_workspace(K)) return GPTQ_ERR_WORKSPACE;
     return residual(P1, C, U, K, ws, static_cast<cudaStream_t>(stream));
 }
@@ -91,6 +93,7 @@ gptq_status gptq_quantize_layer(void *W, int wdtype, int N, int K, const float *
                                 int32_t *status, void *stream) {
     if (N < 1 || K < 1 || groups < 1 || N % groups != 0 || !W || !U || !codes || !status)
         return GPTQ_ERR_ARG;
+    if (N > GPTQ_MAX_DIM || K > GPTQ_MAX_DIM || groups > 8) return GPTQ_ERR_ARG;
     if (!valid_dtype(wdtype)) return GPTQ_ERR_ARG;
     if (bits != 2 && bits != 3 && bits != 4 && bits != 8) return GPTQ_ERR_ARG;
     if (blocksize != 16 && blocksize != 32 && blocksize != 64 && blocksize != 128)

@@ -26,7 +26,7 @@
 namespace gptq {
 
 constexpr int CH_NB = 128;
-constexpr int CH_THREADS = 512;
+constexpr int CH_THREADS = 256;
 constexpr int CH_LD = CH_NB + 1;
 
 __global__ void k_check_finite(const float *A, int64_t count, int32_t *status) {
@@ -69,60 +69,239 @@ __global__ void k_dead_damp(float *H, int K, float percdamp, uint8_t *dead_out, 
     }
 }
 
-// Factor one diagonal block H[J,J] (J = [j0, j0+nb)) as R R^T (R upper), then
-// replace it by U_JJ = R^-1 (upper, strict lower zeroed). One CTA per group.
-__global__ void __launch_bounds__(CH_THREADS) k_chol_diag(float *H, int K, int j0, int nb,
-                                                          const float *diag_d, float tol,
-                                                          int32_t *status) {
+// Factor one diagonal block H[J,J] (J = [j0, j0+nb), nb <= 128) and replace it by
+// U_JJ. One CTA per group (256 threads), the block in shared memory, padded with
+// the identity beyond nb. H_JJ = L D L^T with L unit upper, built from the last
+// 32-wide sub-block Q to the first:
+//   - all threads factor C = S[Q,Q] = L_Q D_Q L_Q^T and invert V_Q = L_Q^-1, four
+//     register elements each, one published pivot column per barrier;
+//   - all threads: T = S[<Q, Q] V_Q^T, L[<Q, Q] = T D_Q^-1, and the trailing update
+//     S[<Q, <Q] -= L T^T (upper triangle).
+// Then V = L^-1 by block back-substitution, V_PQ = -V_PP sum_{P<R<=Q} L_PR V_RQ,
+// and U_JJ = R^-1 = D^-1/2 V with R = L D^1/2.
+constexpr int DG_T = 256;
+constexpr int DG_LD = CH_NB + 1;
+
+__global__ void __launch_bounds__(DG_T, 1) k_chol_diag(float *H, int K, int j0, int nb,
+                                                    const float *diag_d, float tol,
+                                                    int32_t *status) {
     if (failed(status)) return;
     const int g = blockIdx.x;
     H += (int64_t)g * K * K;
     diag_d += (int64_t)g * K;
-    extern __shared__ float S[];  // [CH_NB][CH_LD]
-    float *tmp = S + CH_NB * CH_LD;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = CH_THREADS / 32;
-    for (int idx = tid; idx < nb * nb; idx += CH_THREADS) {
-        const int r = idx / nb, c = idx % nb;
-        S[r * CH_LD + c] = (r <= c) ? H[(int64_t)(j0 + r) * K + j0 + c]
-                                    : H[(int64_t)(j0 + c) * K + j0 + r];
+    extern __shared__ float sm[];
+    float *S = sm;                          // [128][DG_LD]: L (strict upper), D (diagonal)
+    float *V = S + CH_NB * DG_LD;           // [128][DG_LD]: V = L^-1 (upper)
+    float *Ts = V + CH_NB * DG_LD;          // [96][33]: panel products
+    float *piv = Ts + 96 * 33;              // [128]
+    float *dref = piv + CH_NB;              // [128]
+    float *colb = dref + CH_NB;             // [2][32] published pivot column
+    float *rowb = colb + 64;                // [2][32] published row of V
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = DG_T / 32;
+
+    // stage whole rows (only the upper triangle is ever read); identity padding
+    const bool vec = (K % 4 == 0) && (nb == CH_NB);
+    if (vec) {
+#pragma unroll 8
+        for (int it = 0; it < CH_NB * CH_NB / 4 / DG_T; ++it) {
+            const int idx = it * DG_T + tid, r = idx >> 5, c4 = (idx & 31) * 4;
+            const float4 x = *reinterpret_cast<const float4 *>(H + (int64_t)(j0 + r) * K + j0 + c4);
+            float *dst = S + r * DG_LD + c4;
+            dst[0] = x.x; dst[1] = x.y; dst[2] = x.z; dst[3] = x.w;
+        }
+    } else {
+#pragma unroll 8
+        for (int it = 0; it < CH_NB * CH_NB / DG_T; ++it) {
+            const int idx = it * DG_T + tid, r = idx >> 7, c = idx & 127;
+            S[r * DG_LD + c] = (r < nb && c < nb) ? H[(int64_t)(j0 + r) * K + j0 + c]
+                                                  : (r == c ? 1.f : 0.f);
+        }
     }
+    for (int idx = tid; idx < CH_NB * CH_NB; idx += DG_T) V[(idx >> 7) * DG_LD + (idx & 127)] = 0.f;
+    if (tid < CH_NB) dref[tid] = tid < nb ? diag_d[j0 + tid] : 1.f;
     __syncthreads();
-    // R R^T factorisation, last column first (upper triangle of S holds R).
-    for (int j = nb - 1; j >= 0; --j) {
-        if (tid == 0) {
-            const float d = S[j * CH_LD + j];
-            if (!(d > tol * diag_d[j0 + j])) set_status(status, GPTQ_ERR_NOT_PD);
-            S[j * CH_LD + j] = sqrtf(fmaxf(d, FLT_MIN));
+
+    for (int q = 3; q >= 0; --q) {
+        const int o = 32 * q;
+        {
+            // all 256 threads: thread (ri, cg) holds row ri, columns 4cg .. 4cg+3 of the
+            // 32 x 32 sub-block; one pivot column is published per barrier
+            const int ri = tid >> 3, cg = tid & 7;
+            float c4[4], v4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) c4[e] = S[(o + ri) * DG_LD + o + 4 * cg + e];
+            int bb = 0;
+            for (int j = 31; j >= 0; --j) {
+                if ((j >> 2) == cg) {
+                    float x = c4[0];
+#pragma unroll
+                    for (int e = 1; e < 4; ++e) x = ((j & 3) == e) ? c4[e] : x;
+                    colb[bb * 32 + ri] = x;
+                }
+                __syncthreads();
+                const float d = colb[bb * 32 + j];
+                if (tid == 0) {
+                    piv[o + j] = d;
+                    if (o + j < nb && !(d > tol * dref[o + j])) set_status(status, GPTQ_ERR_NOT_PD);
+                }
+                const float aij = colb[bb * 32 + ri] / fmaxf(d, FLT_MIN);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int k = 4 * cg + e;
+                    if (ri <= k && k < j) c4[e] = fmaf(-aij, colb[bb * 32 + k], c4[e]);
+                }
+                bb ^= 1;
+            }
+            __syncthreads();
+            // unit upper L_Q, and V_Q = L_Q^-1 by column elimination on V = I
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int k = 4 * cg + e;
+                if (ri < k) c4[e] = c4[e] / fmaxf(piv[o + k], FLT_MIN);
+                v4[e] = (ri == k) ? 1.f : 0.f;
+            }
+            for (int k = 31; k >= 1; --k) {
+                if ((k >> 2) == cg) {
+                    float x = c4[0];
+#pragma unroll
+                    for (int e = 1; e < 4; ++e) x = ((k & 3) == e) ? c4[e] : x;
+                    colb[bb * 32 + ri] = x;
+                }
+                if (ri == k) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) rowb[bb * 32 + 4 * cg + e] = v4[e];
+                }
+                __syncthreads();
+                if (ri < k) {
+                    const float lik = colb[bb * 32 + ri];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) v4[e] = fmaf(-lik, rowb[bb * 32 + 4 * cg + e], v4[e]);
+                }
+                bb ^= 1;
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int k = 4 * cg + e;
+                S[(o + ri) * DG_LD + o + k] = (k >= ri) ? c4[e] : 0.f;   // L (strict upper), d
+                V[(o + ri) * DG_LD + o + k] = (k >= ri) ? v4[e] : 0.f;
+            }
         }
         __syncthreads();
-        const float r = S[j * CH_LD + j];
-        for (int i = tid; i < j; i += CH_THREADS) S[i * CH_LD + j] = S[i * CH_LD + j] / r;
+        if (q == 0) break;
+        // panel: T = B V_Q^T (B = S[0:o, Q] unscaled), L = T D_Q^-1. Thread (c, rs):
+        // column c = tid & 31, rows rs + 8r; V_Q is stored with zeros below its diagonal.
+        {
+            const int c = tid & 31, rs = tid >> 5, nr = o / 8;
+            float acc[12];
+#pragma unroll
+            for (int r = 0; r < 12; ++r) acc[r] = 0.f;
+#pragma unroll 4
+            for (int m = 0; m < 32; ++m) {
+                const float v = V[(o + c) * DG_LD + o + m];
+#pragma unroll
+                for (int r = 0; r < 12; ++r)
+                    if (r < nr) acc[r] = fmaf(S[(rs + 8 * r) * DG_LD + o + m], v, acc[r]);
+            }
+            __syncthreads();
+            const float rd = 1.f / fmaxf(piv[o + c], FLT_MIN);
+#pragma unroll
+            for (int r = 0; r < 12; ++r)
+                if (r < nr) {
+                    const int i = rs + 8 * r;
+                    Ts[i * 33 + c] = acc[r];
+                    S[i * DG_LD + o + c] = acc[r] * rd;
+                }
+        }
         __syncthreads();
-        for (int i = warp; i < j; i += nwarps) {
-            const float sij = S[i * CH_LD + j];
-            for (int k = i + lane; k < j; k += 32) S[i * CH_LD + k] -= sij * S[k * CH_LD + j];
+        // trailing update of the upper triangle: S[i][k] -= sum_c L[i][c] T[k][c];
+        // thread: k = (tid & 31) + 32 kk, i = (tid >> 5) + 8 r
+        {
+            const int kl = tid & 31, rs = tid >> 5, nr = o / 8, nk = o / 32;
+            float acc[12][3];
+#pragma unroll
+            for (int r = 0; r < 12; ++r)
+#pragma unroll
+                for (int kk = 0; kk < 3; ++kk) acc[r][kk] = 0.f;
+#pragma unroll 2
+            for (int c = 0; c < 32; ++c) {
+                float t[3];
+#pragma unroll
+                for (int kk = 0; kk < 3; ++kk) t[kk] = kk < nk ? Ts[(kl + 32 * kk) * 33 + c] : 0.f;
+#pragma unroll
+                for (int r = 0; r < 12; ++r) {
+                    if (r >= nr) continue;
+                    const float l = S[(rs + 8 * r) * DG_LD + o + c];
+#pragma unroll
+                    for (int kk = 0; kk < 3; ++kk) acc[r][kk] = fmaf(l, t[kk], acc[r][kk]);
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < 12; ++r)
+#pragma unroll
+                for (int kk = 0; kk < 3; ++kk) {
+                    const int i = rs + 8 * r, k = kl + 32 * kk;
+                    if (r < nr && kk < nk && i <= k) S[i * DG_LD + k] -= acc[r][kk];
+                }
         }
         __syncthreads();
     }
-    // In-place inverse of the upper triangular R, column by column:
-    // U_jj = 1/R_jj, U[0:j, j] = -U_jj * U[0:j, 0:j] R[0:j, j].
-    for (int j = 0; j < nb; ++j) {
-        for (int k = tid; k < j; k += CH_THREADS) tmp[k] = S[k * CH_LD + j];
+    // V = L^-1: for each block column Q, P = Q-1 .. 0; round s does every pair with
+    // Q - P = s. Thread: column c = tid & 31 of the pair, rows (tid >> 5) + 8 r.
+    for (int sr = 1; sr <= 3; ++sr) {
+        const int pairs = 4 - sr, c = tid & 31, rs = tid >> 5;
+        float x[3][4];
+#pragma unroll
+        for (int pr = 0; pr < 3; ++pr)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) x[pr][r] = 0.f;
+#pragma unroll
+        for (int pr = 0; pr < 3; ++pr) {
+            if (pr >= pairs) continue;
+            const int Q = sr + pr, P = Q - sr;
+#pragma unroll 4
+            for (int m = 32 * (P + 1); m < 32 * (Q + 1); ++m) {
+                const float v = V[m * DG_LD + 32 * Q + c];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) x[pr][r] = fmaf(S[(32 * P + rs + 8 * r) * DG_LD + m], v, x[pr][r]);
+            }
+        }
+#pragma unroll
+        for (int pr = 0; pr < 3; ++pr)
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+                if (pr < pairs) Ts[(32 * pr + rs + 8 * r) * 33 + c] = x[pr][r];
         __syncthreads();
-        const float ujj = 1.f / S[j * CH_LD + j];
-        for (int i = warp; i < j; i += nwarps) {
-            float acc = 0.f;
-            for (int k = i + lane; k < j; k += 32) acc += S[i * CH_LD + k] * tmp[k];
-            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-            if (lane == 0) S[i * CH_LD + j] = -ujj * acc;
+        float y[3][4];
+#pragma unroll
+        for (int pr = 0; pr < 3; ++pr)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) y[pr][r] = 0.f;
+#pragma unroll
+        for (int pr = 0; pr < 3; ++pr) {
+            if (pr >= pairs) continue;
+            const int P = sr + pr - sr;
+#pragma unroll 4
+            for (int m = 0; m < 32; ++m) {
+                const float t = Ts[(32 * pr + m) * 33 + c];
+#pragma unroll
+                for (int r = 0; r < 4; ++r)   // V_PP is upper: zero for m < row
+                    y[pr][r] = fmaf(V[(32 * P + rs + 8 * r) * DG_LD + 32 * P + m], t, y[pr][r]);
+            }
+        }
+#pragma unroll
+        for (int pr = 0; pr < 3; ++pr) {
+            if (pr >= pairs) continue;
+            const int Q = sr + pr, P = Q - sr;
+#pragma unroll
+            for (int r = 0; r < 4; ++r) V[(32 * P + rs + 8 * r) * DG_LD + 32 * Q + c] = -y[pr][r];
         }
         __syncthreads();
-        if (tid == 0) S[j * CH_LD + j] = ujj;
-        __syncthreads();
     }
-    for (int idx = tid; idx < nb * nb; idx += CH_THREADS) {
-        const int r = idx / nb, c = idx % nb;
-        H[(int64_t)(j0 + r) * K + j0 + c] = (r <= c) ? S[r * CH_LD + c] : 0.f;
+    // U = D^-1/2 V
+    for (int r = warp; r < nb; r += nwarps) {
+        const float sc = 1.f / sqrtf(fmaxf(piv[r], FLT_MIN));
+        for (int c = lane; c < nb; c += 32)
+            H[(int64_t)(j0 + r) * K + j0 + c] = (c >= r) ? V[r * DG_LD + c] * sc : 0.f;
     }
 }
 
@@ -195,15 +374,15 @@ gptq_status prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out, v
     k_dead_damp<<<g, 1024, 0, st>>>(H, K, percdamp, dead_out, diag_d, status);
     if ((s = launch_status()) != GPTQ_OK) return s;
 
-    const size_t smem = (size_t)(CH_NB * CH_LD + CH_NB) * sizeof(float);
-    cudaFuncSetAttribute(k_chol_diag, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     const float tol = (float)K * FLT_EPSILON;
+    const int chol_smem = (int)((2 * CH_NB * DG_LD + 96 * 33 + 2 * CH_NB + 128) * sizeof(float));
+    cudaFuncSetAttribute(k_chol_diag, cudaFuncAttributeMaxDynamicSharedMemorySize, chol_smem);
     Blocks bk{K, (K + CH_NB - 1) / CH_NB};
     for (int t = bk.T - 1; t >= 0; --t) {
         const int j0 = bk.start(t);
         const int j1 = (t == bk.T - 1) ? K : bk.start(t + 1);
         const int nb = j1 - j0;
-        k_chol_diag<<<g, CH_THREADS, smem, st>>>(H, K, j0, nb, diag_d, tol, status);
+        k_chol_diag<<<g, DG_T, chol_smem, st>>>(H, K, j0, nb, diag_d, tol, status);
         if ((s = launch_status()) != GPTQ_OK) return s;
         if (j0 == 0) break;
         // panel: R[0:j0, J] = H[0:j0, J] U_JJ^T  (in place: each CTA owns whole rows)

@@ -54,6 +54,7 @@ extern "C" gptq_status gptq_prepare_noalloc(float *H, int K, int g, float percda
                                             uint8_t *dead_out, int32_t *status, void *stream) {
     if (K < 1 || g < 1 || !H || !status || !(percdamp >= 0.f) || !aligned(H, 16))
         return GPTQ_ERR_ARG;
+    if (K > GPTQ_MAX_DIM) return GPTQ_ERR_ARG;
     if (prepare_workspace(K, g) > NOALLOC_SCRATCH_BYTES) return GPTQ_ERR_ARG;
     void *ws = nullptr;
     gptq_status s = scratch_for_current_device(&ws);

@@ -1,0 +1,39 @@
+// Shared declarations of the tensor-core lazy update (update_tc.cu).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+
+namespace gptq {
+
+constexpr int UT_MAX_TERMS = 6;
+
+struct UpdateMaps {
+    CUtensorMap a[4];   // A operands: [rows j][n], bf16
+    CUtensorMap b[4];   // B operands: [rows j][k], bf16
+};
+
+struct UpdateParams {
+    float *C;
+    int64_t ldc;
+    int M, Ncols, L;        // output rows, output columns, inner rows (multiple of 16)
+    int a_x0, a_y0;         // A: column (n) origin, row (j) origin
+    int b_x0, b_y0;         // B: column (k) origin, row (j) origin
+    int nterms;
+    int a_id[UT_MAX_TERMS], b_id[UT_MAX_TERMS], neg[UT_MAX_TERMS];
+    int vec4;               // C rows 16-byte aligned: float4 reductions
+    int32_t *status;
+};
+
+bool update_tc_available();
+gptq_status make_bf16_map(CUtensorMap *m, const void *base, int64_t cols, int64_t rows,
+                          int64_t ld, int box_rows);
+gptq_status launch_update_tc(const UpdateMaps &maps, const UpdateParams &p, int box_rows,
+                             cudaStream_t st);
+gptq_status split_bf16(const float *in, int64_t ld_in, int rows, int cols, __nv_bfloat16 *hi,
+                       __nv_bfloat16 *lo, int64_t ld_out, int batch, int64_t batch_in,
+                       int64_t batch_out, cudaStream_t st);
+
+}  // namespace gptq
