@@ -32,6 +32,11 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "GPTQ layer-solve ms & weights quantized/s (4096×14336, W3); % of TC/HBM roofline"
+
+# DRAM bytes (read + write) per launch of the dominant kernel, from the ncu capture
+# summarised in profiles/gram_tc_mlp_up_w3_chunk65536.md (same 65,536-token launch).
+# Set to None whenever k_gram_tc changes until it is captured again.
+GRAM_TRAFFIC_BYTES = 1.323837e9 + 0.234119e9
 UNIT = "weights/s"
 
 
@@ -291,7 +296,7 @@ def run_ours(args, rank, world, local_rank):
     achieved = flops_launch / (gram_launch_ms * 1e-3) / 1e12
     roofline = {"kernel": "k_gram_tc (gptq_accumulate_hessian, tcgen05)", "bound": "tensor",
                 "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "traffic": None,
+                "frac": round(achieved / peak, 4), "traffic": GRAM_TRAFFIC_BYTES,
                 "peak_source": ("MEASURED_PEAKS.json bf16_tflops_sustained (of measured)"
                                 if peaks.get("bf16_tflops_sustained") else "fallback 1.4 PFLOP/s"),
                 "per_launch": f"{ch} tokens x K(K+1) = {flops_launch:.3e} FLOP (symmetric count)",

@@ -143,14 +143,20 @@ def fp_tokens_chunk(wl: Workload, chunk: int, device="cpu", rows=None) -> torch.
     return torch.randn(rows, wl.K, generator=g, device=device).to(wl.xdtype)
 
 
+_RMS_CACHE: dict = {}
+
+
 def fp_stream_rms(wl: Workload, device="cpu") -> float:
     """Global scalar rms of X~ over the whole stream."""
-    acc, cnt = 0.0, 0
-    for c in range(num_chunks(wl)):
-        x = fp_tokens_chunk(wl, c, device).float()
-        acc += float((x * x).sum())
-        cnt += x.numel()
-    return (acc / cnt) ** 0.5
+    key = (wl.name, wl.seed, wl.M, wl.K, wl.chunk, str(device))
+    if key not in _RMS_CACHE:
+        acc, cnt = 0.0, 0
+        for c in range(num_chunks(wl)):
+            x = fp_tokens_chunk(wl, c, device).float()
+            acc += float((x * x).sum())
+            cnt += x.numel()
+        _RMS_CACHE[key] = (acc / cnt) ** 0.5
+    return _RMS_CACHE[key]
 
 
 def num_chunks(wl: Workload) -> int:

@@ -1,0 +1,117 @@
+"""Full-size parity: the workloads at their real sizes, in the launch configuration
+the benchmark times (65,536-token chunks streamed through gptq_accumulate_hessian,
+then gptq_prepare and gptq_quantize_layer on one GPU).
+
+The oracle cannot redo a 2M-token fp64 Gram or a 14k-channel explicit sweep, so it
+checks sampled outputs it can compute one by one:
+  - H on sampled (row, column) pairs, summed in fp64 over the whole stream;
+  - U in full (fp64 factor of the GPU's H);
+  - codes of sampled channels by tie-follow replay, and the output error of those
+    channels against the oracle's own solve.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import post_weight_quantization_solve_b200 as gq
+from post_weight_quantization_solve_b200 import synth
+from post_weight_quantization_solve_b200.build import build
+
+from gpu_util import CODE_SAME, TOL_H, TOL_RECON, TOL_U, dev, own_decisions_same, rel_max
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build()
+    gq.load_library()
+
+
+def _run_full(wl, n_rows=6, n_cols=48, n_ch=40, seed=123, gptaq=False):
+    d = dev()
+    K, N = wl.K, wl.N
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(K, n_rows, replace=False))
+    cols = np.sort(np.union1d(rng.choice(K, n_cols, replace=False), rows))
+    H = torch.zeros(K, K, device=d)
+    C = torch.zeros(K, K, device=d) if gptaq else None
+    H_ref = np.zeros((len(rows), len(cols)))
+    C_ref = np.zeros((len(rows), len(cols))) if gptaq else None
+    status = gq.new_status(d)
+    for c in range(synth.num_chunks(wl)):
+        X = synth.tokens_chunk(wl, c, d)
+        gq.gptq_accumulate_hessian(H, X, status=status)
+        xr = X[:, torch.as_tensor(rows, device=d)].double().cpu().numpy()
+        xc = X[:, torch.as_tensor(cols, device=d)].double().cpu().numpy()
+        H_ref += 2.0 * xr.T @ xc
+        if gptaq:
+            Xf = synth.fp_tokens_chunk(wl, c, d)
+            gq.gptaq_accumulate_cross(C, Xf, X, status=status)
+            dxr = (Xf[:, torch.as_tensor(rows, device=d)].double().cpu().numpy() - xr)
+            C_ref += 2.0 * dxr.T @ xc
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    H_gpu = H.double().cpu().numpy()
+    assert rel_max(H_gpu[np.ix_(rows, cols)], H_ref) <= TOL_H
+    np.testing.assert_array_equal(H_gpu, H_gpu.T)
+    if gptaq:
+        C_gpu = C.double().cpu().numpy()
+        assert rel_max(C_gpu[np.ix_(rows, cols)], C_ref) <= TOL_H
+
+    W = synth.weights(wl, d)
+    U = H.clone()
+    status = gq.gptq_prepare(U, wl.percdamp)
+    P1 = None
+    if gptaq:
+        P1 = torch.empty(K, K, device=d)
+        gq.gptaq_residual(P1, C, U)
+    Wq = W.clone()
+    scales = torch.empty(N, device=d)
+    codes, status = gq.gptq_quantize_layer(Wq, U, wl.bits, wl.blocksize, P1=P1, scales_out=scales,
+                                           write_back=True, status=status)
+    gq.raise_on_status(status, wl.name)
+    U_gpu = U.double().cpu().numpy()
+
+    Hd, dead = O.dead_and_damp(H_gpu, wl.percdamp)
+    assert not dead.any()
+    U_ora = O.upper_factor(Hd)
+    assert rel_max(U_gpu, U_ora) <= TOL_U
+    P1_ora = None
+    if gptaq:
+        P1_ora = O.gptaq_p1(C.double().cpu().numpy(), U_ora)
+        assert rel_max(P1.double().cpu().numpy(), P1_ora) <= TOL_U
+
+    ch = np.sort(rng.choice(N, n_ch, replace=False))
+    W64 = W.double().cpu().numpy()[ch]
+    s64 = scales.double().cpu().numpy()[ch]
+    s_ora, _ = O.symmetric_scale(W64, wl.bits)
+    np.testing.assert_allclose(s64, s_ora, rtol=2e-7)
+    c_gpu = codes[torch.as_tensor(ch, device=d)].cpu().numpy().astype(np.float64)
+    rep = O.replay_row_form(U_ora, W64, s64, wl.bits, c_gpu, P1=P1_ora)
+    assert rep["mismatches"] == 0, rep["mismatches"]
+    assert own_decisions_same(rep, c_gpu.size) >= CODE_SAME
+    # write-back is exactly s (c - z) in the weights' dtype
+    wq = Wq[torch.as_tensor(ch, device=d)].double().cpu().numpy()
+    expect = torch.tensor(s64[:, None].astype(np.float32) *
+                          (c_gpu - 2 ** (wl.bits - 1)).astype(np.float32)).to(W.dtype).double().numpy()
+    np.testing.assert_array_equal(wq, expect)
+    # output error of the sampled channels vs the oracle's own solve (same H)
+    _, W_ora, _ = O.row_form_sweep(U_ora, W64, s_ora, wl.bits, wl.blocksize, P1=P1_ora)
+    e_gpu = O.layer_error(H_gpu, W64, O.dequantize(c_gpu, s64[:, None], wl.bits))
+    e_ora = O.layer_error(H_gpu, W64, W_ora)
+    assert abs(e_gpu - e_ora) <= TOL_RECON * e_ora
+
+
+def test_headline_mlp_up_w3_fullsize():
+    _run_full(synth.WORKLOADS["mlp_up_w3"])
+
+
+def test_q_proj_fullsize():
+    _run_full(synth.WORKLOADS["q_proj"], seed=7)
+
+
+def test_gptaq_fullsize():
+    _run_full(synth.WORKLOADS["gptaq"], seed=11, gptaq=True)
