@@ -36,7 +36,7 @@ METRIC = "GPTQ layer-solve ms & weights quantized/s (4096×14336, W3); % of TC/H
 # DRAM bytes (read + write) per launch of the dominant kernel, from the ncu capture
 # summarised in profiles/gram_tc_mlp_up_w3_chunk65536.md (same 65,536-token launch).
 # Set to None whenever k_gram_tc changes until it is captured again.
-GRAM_TRAFFIC_BYTES = 1.323837e9 + 0.234119e9
+GRAM_TRAFFIC_BYTES = None   # k_gram_tc changed (bounded accumulation chains); recapture
 UNIT = "weights/s"
 
 

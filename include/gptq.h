@@ -92,8 +92,9 @@ typedef enum {
  *          wait inside the tensor-core kernel ran out; the call is skipped when the
  *          word is already non-zero.
  *   Errors: GPTQ_ERR_ARG for bad sizes/alignment/dtype, GPTQ_ERR_CUDA on launch.
- *   Paths: bf16 with g == 1 and w == NULL runs on the tensor cores (tcgen05, TMA);
- *   fp32 streams and weighted Hessians run the fp32 SIMT kernel.
+ *   Paths: bf16 streams with K >= 64 run on the tensor cores (tcgen05, TMA); with
+ *   weights, each token's s * x is formed in fp32 and split into a bf16 pair so the
+ *   product keeps ~16 bits. fp32 streams run the fp32 SIMT kernel.
  */
 GPTQ_API gptq_status gptq_accumulate_hessian(float *H, int K, int g, const void *X, int xdtype,
                                     int64_t M, int64_t ldx, const float *w, int64_t ldw,
@@ -112,6 +113,8 @@ GPTQ_API gptq_status gptq_accumulate_hessian(float *H, int K, int g, const void 
  *   X_fp, X_q  device [M][ldx] each, same dtype and leading dimension; alignment
  *          rules as gptq_accumulate_hessian.
  *   status device int32 or NULL, as in gptq_accumulate_hessian.
+ *   bf16 streams with K >= 64 run on the tensor cores (the difference is split into
+ *   a bf16 pair); fp32 streams run the fp32 SIMT kernel.
  */
 GPTQ_API gptq_status gptaq_accumulate_cross(float *C, int K, const void *X_fp, const void *X_q,
                                    int xdtype, int64_t M, int64_t ldx, int32_t *status,

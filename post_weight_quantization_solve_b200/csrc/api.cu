@@ -10,6 +10,9 @@ gptq_status cross_simt(float *C, int K, const void *Xfp, const void *Xq, int xdt
 gptq_status gram_tc(float *H, int K, int g, const void *X, int64_t M, int64_t ldx,
                     const float *w, int64_t ldw, const void *X2, cudaStream_t st, int32_t *status,
                     bool *used);
+gptq_status gram_x_tc(float *H, int K, int g, const void *X, const void *X2, int64_t M,
+                      int64_t ldx, const float *w, int64_t ldw, int32_t *status, cudaStream_t st,
+                      bool *used);
 size_t prepare_workspace(int K, int g);
 gptq_status prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out, void *ws,
                     int32_t *status, cudaStream_t st);
@@ -52,7 +55,9 @@ gptq_status gptq_accumulate_hessian(float *H, int K, int g, const void *X, int x
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (xdtype == GPTQ_BF16) {
         bool used = false;
-        gptq_status s = gram_tc(H, K, g, X, M, ldx, w, ldw, nullptr, st, status, &used);
+        gptq_status s = (w == nullptr)
+                            ? gram_tc(H, K, g, X, M, ldx, w, ldw, nullptr, st, status, &used)
+                            : gram_x_tc(H, K, g, X, nullptr, M, ldx, w, ldw, status, st, &used);
         if (used || s != GPTQ_OK) return s;
     }
     return gram_simt(H, K, g, X, xdtype, M, ldx, w, ldw, status, st);
@@ -67,6 +72,11 @@ gptq_status gptaq_accumulate_cross(float *C, int K, const void *X_fp, const void
         return GPTQ_ERR_ARG;
     if (xdtype == GPTQ_BF16 && K % 8 != 0) return GPTQ_ERR_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (xdtype == GPTQ_BF16) {
+        bool used = false;
+        gptq_status s = gram_x_tc(C, K, 1, X_fp, X_q, M, ldx, nullptr, 0, status, st, &used);
+        if (used || s != GPTQ_OK) return s;
+    }
     return cross_simt(C, K, X_fp, X_q, xdtype, M, ldx, status, st);
 }
 

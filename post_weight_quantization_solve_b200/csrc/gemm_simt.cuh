@@ -39,17 +39,12 @@ struct GemmParams {
 
 constexpr int GB_M = 128, GB_N = 128, GB_K = 8, G_THREADS = 256;
 
+// One 128 x 128 output tile (rows i0.., columns j0..) of the product described by p,
+// with A, A2, B, C, ks already offset to this product.
 template <typename TA, typename TB, bool AT, bool BT>
-__global__ void __launch_bounds__(G_THREADS) gemm_simt_kernel(GemmParams p) {
-    if (failed(p.status)) return;
-    const int bz = blockIdx.z;
-    const TA *A = static_cast<const TA *>(p.A) + bz * p.sA;
-    const TA *A2 = p.A2 ? static_cast<const TA *>(p.A2) + bz * p.sA2 : nullptr;
-    const TB *B = static_cast<const TB *>(p.B) + bz * p.sB;
-    float *C = p.C + bz * p.sC;
-    const float *ks = p.kscale ? p.kscale + bz * p.sK : nullptr;
-
-    const int i0 = blockIdx.y * GB_M, j0 = blockIdx.x * GB_N;
+__device__ __forceinline__ void gemm_tile(const GemmParams &p, const TA *A, const TA *A2,
+                                          const TB *B, float *C, const float *ks, int i0,
+                                          int j0) {
     if (p.upper_tiles && i0 > j0 + GB_N - 1) return;
     int kbeg = 0, kend = p.k;
     if (p.a_upper) kbeg = (i0 / GB_K) * GB_K;
@@ -152,10 +147,62 @@ __global__ void __launch_bounds__(G_THREADS) gemm_simt_kernel(GemmParams p) {
 }
 
 template <typename TA, typename TB, bool AT, bool BT>
+__global__ void __launch_bounds__(G_THREADS) gemm_simt_kernel(GemmParams p) {
+    if (failed(p.status)) return;
+    const int bz = blockIdx.z;
+    const TA *A = static_cast<const TA *>(p.A) + bz * p.sA;
+    const TA *A2 = p.A2 ? static_cast<const TA *>(p.A2) + bz * p.sA2 : nullptr;
+    const TB *B = static_cast<const TB *>(p.B) + bz * p.sB;
+    float *C = p.C + bz * p.sC;
+    const float *ks = p.kscale ? p.kscale + bz * p.sK : nullptr;
+    gemm_tile<TA, TB, AT, BT>(p, A, A2, B, C, ks, blockIdx.y * GB_M, blockIdx.x * GB_N);
+}
+
+// A group of independent products with their own sizes, offsets and leading
+// dimensions (one per blockIdx.z); the structural flags are shared.
+constexpr int GROUP_MAX = 128;
+struct GroupItem {
+    int m, n, k;
+    int lda, ldb, ldc;
+    int64_t offA, offB, offC;
+};
+struct GroupParams {
+    GemmParams base;
+    int nitems;
+    GroupItem item[GROUP_MAX];
+};
+
+template <typename TA, typename TB, bool AT, bool BT>
+__global__ void __launch_bounds__(G_THREADS) gemm_simt_grouped(const __grid_constant__ GroupParams gp) {
+    if (failed(gp.base.status)) return;
+    const GroupItem &it = gp.item[blockIdx.z];
+    const int i0 = blockIdx.y * GB_M, j0 = blockIdx.x * GB_N;
+    if (i0 >= it.m || j0 >= it.n) return;
+    GemmParams p = gp.base;
+    p.m = it.m; p.n = it.n; p.k = it.k;
+    p.lda = it.lda; p.ldb = it.ldb; p.ldc = it.ldc;
+    gemm_tile<TA, TB, AT, BT>(p, static_cast<const TA *>(p.A) + it.offA, nullptr,
+                              static_cast<const TB *>(p.B) + it.offB, p.C + it.offC, nullptr, i0, j0);
+}
+
+template <typename TA, typename TB, bool AT, bool BT>
 inline gptq_status gemm_simt(const GemmParams &p, int batch, cudaStream_t st) {
     if (p.m <= 0 || p.n <= 0) return GPTQ_OK;
     dim3 grid((p.n + GB_N - 1) / GB_N, (p.m + GB_M - 1) / GB_M, batch);
     gemm_simt_kernel<TA, TB, AT, BT><<<grid, G_THREADS, 0, st>>>(p);
+    return launch_status();
+}
+
+template <typename TA, typename TB, bool AT, bool BT>
+inline gptq_status gemm_simt_group(const GroupParams &gp, cudaStream_t st) {
+    int mm = 0, nn = 0;
+    for (int i = 0; i < gp.nitems; ++i) {
+        mm = mm > gp.item[i].m ? mm : gp.item[i].m;
+        nn = nn > gp.item[i].n ? nn : gp.item[i].n;
+    }
+    if (gp.nitems <= 0 || mm <= 0 || nn <= 0) return GPTQ_OK;
+    dim3 grid((nn + GB_N - 1) / GB_N, (mm + GB_M - 1) / GB_M, gp.nitems);
+    gemm_simt_grouped<TA, TB, AT, BT><<<grid, G_THREADS, 0, st>>>(gp);
     return launch_status();
 }
 

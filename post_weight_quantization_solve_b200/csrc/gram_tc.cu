@@ -249,13 +249,16 @@ static int sm_count() {
     return n > 0 ? n : 148;
 }
 
-// Token parts P: the first P whose units (T * P) fill the persistent grid to >= 97 %
-// in the last wave, keeping >= 16 k-steps per unit.
-static int pick_parts(int T, int S, int grid) {
+// Token parts P: at least enough parts that no TMEM accumulation chain exceeds
+// MAX_MMA_CHAIN MMAs, then the first P whose units (T * P) fill the persistent grid
+// to >= 97 % in the last wave, keeping >= 16 k-steps per unit.
+static int pick_parts(int T, int S, int grid, int mma_per_step) {
     int best = 1;
     double best_eff = 0.0;
-    const int pmax = std::max(1, std::min(64, S / 16));
-    for (int P = 1; P <= pmax; ++P) {
+    const int pmin = std::max(1, (S * mma_per_step + tc::MAX_MMA_CHAIN - 1) / tc::MAX_MMA_CHAIN);
+    const int pmax = std::max(pmin, std::min(std::max(64, pmin), S / 16));
+    best = pmin;
+    for (int P = pmin; P <= pmax; ++P) {
         const long units = (long)T * P;
         const long waves = (units + grid - 1) / grid;
         const double eff = (double)units / (double)(waves * grid);
@@ -294,7 +297,7 @@ gptq_status gram_tc(float *H, int K, int g, const void *X, int64_t M, int64_t ld
     p.T = 0;
     for (int j = 0; j < ntn; ++j) p.T += std::min(p.ntm, 2 * (j + 1));
     const int grid_max = sm_count();
-    p.P = pick_parts(p.T, p.S, grid_max);
+    p.P = pick_parts(p.T, p.S, grid_max, GT_BK / 16);
     if (p.P > p.S) p.P = p.S;
     p.alpha = 2.f;
     p.status = status;

@@ -20,14 +20,15 @@
 // over the same block boundaries, whose leaves U_JJ the diag kernel already wrote.
 #include <float.h>
 
+#include <algorithm>
+#include <vector>
+
 #include "common.cuh"
 #include "gemm_simt.cuh"
 
 namespace gptq {
 
 constexpr int CH_NB = 128;
-constexpr int CH_THREADS = 256;
-constexpr int CH_LD = CH_NB + 1;
 
 __global__ void k_check_finite(const float *A, int64_t count, int32_t *status) {
     int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
@@ -328,30 +329,67 @@ static size_t inverse_scratch_floats(int K) {
     return half * half;
 }
 
-// Off-diagonal blocks of U = R^-1 over blocks [bl, br).
-static gptq_status tri_inverse(float *H, int K, int g, const Blocks &bk, int bl, int br,
-                               float *T, const int32_t *status, cudaStream_t st) {
-    if (br - bl <= 1) return GPTQ_OK;
+// Off-diagonal blocks of U = R^-1. The recursion [A B; 0 D]^-1 =
+// [A^-1, -A^-1 B D^-1; 0, D^-1] over block ranges is laid out as a tree; all nodes
+// of one depth are independent and run as one grouped launch per product
+// (deepest first): T = R[a:m, m:b] U[m:b, m:b], then U[a:m, m:b] = -U[a:m, a:m] T.
+struct InvNode {
+    int a, m, b;
+};
+
+static void inv_nodes(const Blocks &bk, int K, int bl, int br, int depth,
+                      std::vector<std::vector<InvNode>> &levels) {
+    if (br - bl <= 1) return;
     const int mid = (bl + br) / 2;
-    gptq_status s = tri_inverse(H, K, g, bk, bl, mid, T, status, st);
-    if (s != GPTQ_OK) return s;
-    s = tri_inverse(H, K, g, bk, mid, br, T, status, st);
-    if (s != GPTQ_OK) return s;
-    const int a = bk.start(bl), m = bk.start(mid), b = (br == bk.T) ? K : bk.start(br);
+    if ((int)levels.size() <= depth) levels.resize(depth + 1);
+    levels[depth].push_back({bk.start(bl), bk.start(mid), br == bk.T ? K : bk.start(br)});
+    inv_nodes(bk, K, bl, mid, depth + 1, levels);
+    inv_nodes(bk, K, mid, br, depth + 1, levels);
+}
+
+static gptq_status tri_inverse(float *H, int K, int g, const Blocks &bk, float *T,
+                               const int32_t *status, cudaStream_t st) {
+    std::vector<std::vector<InvNode>> levels;
+    inv_nodes(bk, K, 0, bk.T, 0, levels);
     const int64_t KK = (int64_t)K * K;
     const int64_t tsz = (int64_t)inverse_scratch_floats(K);
-    // T = R[a:m, m:b] * U[m:b, m:b]   (U block upper triangular)
-    GemmParams p1 = gemm_params(m - a, b - m, b - m, H + (int64_t)a * K + m, K,
-                                H + (int64_t)m * K + m, K, T, b - m, 1.f, 0, status);
-    p1.b_upper = 1;
-    p1.sA = KK; p1.sB = KK; p1.sC = tsz;
-    if ((s = gemm_simt<float, float, false, false>(p1, g, st)) != GPTQ_OK) return s;
-    // U[a:m, m:b] = -U[a:m, a:m] * T
-    GemmParams p2 = gemm_params(m - a, b - m, m - a, H + (int64_t)a * K + a, K, T, b - m,
-                                H + (int64_t)a * K + m, K, -1.f, 0, status);
-    p2.a_upper = 1;
-    p2.sA = KK; p2.sB = tsz; p2.sC = KK;
-    return gemm_simt<float, float, false, false>(p2, g, st);
+    static thread_local GroupParams g1, g2;
+    for (int d = (int)levels.size() - 1; d >= 0; --d) {
+        const std::vector<InvNode> &lv = levels[d];
+        // (node, group) items, in launches of at most GROUP_MAX
+        std::vector<std::pair<int, int>> items;
+        for (int gi = 0; gi < g; ++gi)
+            for (int ni = 0; ni < (int)lv.size(); ++ni) items.push_back({gi, ni});
+        // scratch offsets of this depth's nodes (disjoint, within the scratch)
+        std::vector<int64_t> toff(lv.size());
+        int64_t acc = 0;
+        for (size_t ni = 0; ni < lv.size(); ++ni) {
+            toff[ni] = acc;
+            acc += (int64_t)(lv[ni].m - lv[ni].a) * (lv[ni].b - lv[ni].m);
+        }
+        for (size_t c0 = 0; c0 < items.size(); c0 += GROUP_MAX) {
+            const int cnt = (int)std::min<size_t>(GROUP_MAX, items.size() - c0);
+            g1.base = gemm_params(0, 0, 0, H, 0, H, 0, T, 0, 1.f, 0, status);
+            g1.base.b_upper = 1;
+            g2.base = gemm_params(0, 0, 0, H, 0, T, 0, H, 0, -1.f, 0, status);
+            g2.base.a_upper = 1;
+            g1.nitems = g2.nitems = cnt;
+            for (int i = 0; i < cnt; ++i) {
+                const int gi = items[c0 + i].first, ni = items[c0 + i].second;
+                const InvNode &nd = lv[ni];
+                const int rows = nd.m - nd.a, cols = nd.b - nd.m;
+                const int64_t hb = gi * KK, tb = gi * tsz + toff[ni];
+                g1.item[i] = {rows, cols, cols, K, K, cols, hb + (int64_t)nd.a * K + nd.m,
+                              hb + (int64_t)nd.m * K + nd.m, tb};
+                g2.item[i] = {rows, cols, rows, K, cols, K, hb + (int64_t)nd.a * K + nd.a, tb,
+                              hb + (int64_t)nd.a * K + nd.m};
+            }
+            gptq_status s = gemm_simt_group<float, float, false, false>(g1, st);
+            if (s != GPTQ_OK) return s;
+            if ((s = gemm_simt_group<float, float, false, false>(g2, st)) != GPTQ_OK) return s;
+        }
+    }
+    return GPTQ_OK;
 }
 
 size_t prepare_workspace(int K, int g) {
@@ -400,7 +438,7 @@ gptq_status prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out, v
     // inverse reads whole tiles of its triangular operands, so clear it first.
     k_zero_lower<<<dim3((K + 255) / 256 > 8 ? 8 : (K + 255) / 256, K, g), 256, 0, st>>>(H, K);
     if ((s = launch_status()) != GPTQ_OK) return s;
-    return tri_inverse(H, K, g, bk, 0, bk.T, T, status, st);
+    return tri_inverse(H, K, g, bk, T, status, st);
 }
 
 }  // namespace gptq

@@ -9,6 +9,13 @@
 namespace gptq {
 namespace tc {
 
+// Longest run of MMAs accumulated in one TMEM accumulator before it is flushed to
+// global memory with fp32 round-to-nearest atomics. The tensor core's fp32
+// accumulation drifts by about one ulp per accumulation step (measured as a
+// systematic relative bias of ~2^-24 per MMA), so chains are kept short enough that
+// the drift stays below ~3e-5 relative.
+constexpr int MAX_MMA_CHAIN = 512;
+
 // ~1 s at 2 GHz: far above any legitimate wait in these kernels.
 constexpr long long WAIT_BUDGET_CYCLES = 2000000000ll;
 

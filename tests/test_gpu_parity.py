@@ -139,6 +139,27 @@ def test_grouped_small():
     _full_check(wl, chunks, synth.weights(wl), groups=4, weights=wts, label="grouped")
 
 
+@pytest.mark.parametrize("K,M", [(64, 1000), (200, 333), (384, 4097)])
+def test_weighted_and_cross_gram_ragged(K, M):
+    """The tensor-core transform Gram on ragged shapes (partial tiles, token counts
+    that are not a multiple of the 32-token step)."""
+    d = dev()
+    g = 3
+    gen = torch.Generator(device="cpu").manual_seed(K + M)
+    Xf = torch.randn(M, K, generator=gen).bfloat16()
+    Xq = (Xf.float() + 0.05 * torch.randn(M, K, generator=gen)).bfloat16()
+    w = torch.rand(g, M, generator=gen) * 2
+    H = torch.zeros(g, K, K, device=d)
+    gq.gptq_accumulate_hessian(H, Xq.to(d), w.to(d))
+    C = torch.zeros(K, K, device=d)
+    gq.gptaq_accumulate_cross(C, Xf.to(d), Xq.to(d))
+    torch.cuda.synchronize()
+    Xq64, Xf64 = _np(Xq), _np(Xf)
+    for gi in range(g):
+        assert rel_max(_np(H[gi]), O.gram(Xq64, _np(w[gi]))) <= TOL_H
+    assert rel_max(_np(C), O.cross_gram(Xq64, Xf64)) <= TOL_H
+
+
 def test_dead_coordinates():
     wl = synth.WORKLOADS["mlp_up"].scaled(K=144, N=96, M=1000, blocksize=32, bits=3)
     X = synth.tokens_chunk(wl, 0).clone()
