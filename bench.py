@@ -36,7 +36,7 @@ METRIC = "GPTQ layer-solve ms & weights quantized/s (4096×14336, W3); % of TC/H
 # DRAM bytes (read + write) per launch of the dominant kernel, from the ncu capture
 # summarised in profiles/gram_tc_mlp_up_w3_chunk65536.md (same 65,536-token launch).
 # Set to None whenever k_gram_tc changes until it is captured again.
-GRAM_TRAFFIC_BYTES = None   # k_gram_tc changed (bounded accumulation chains); recapture
+GRAM_TRAFFIC_BYTES = 1.272892e9 + 0.264233e9
 UNIT = "weights/s"
 
 
@@ -212,38 +212,61 @@ def run_ours(args, rank, world, local_rank):
     K, N, M, ch = wl.K, wl.N, wl.M, wl.chunk
     nch = synth.num_chunks(wl)
 
+    g = wl.groups
     X = torch.empty(M, K, dtype=wl.xdtype, device=dev)
     for c in range(nch):
         X[c * ch:(c + 1) * ch] = synth.tokens_chunk(wl, c, dev)
+    Xf = None
+    if wl.gptaq:                       # full-precision stream of the asymmetric calibration
+        Xf = torch.empty(M, K, dtype=wl.xdtype, device=dev)
+        for c in range(nch):
+            Xf[c * ch:(c + 1) * ch] = synth.fp_tokens_chunk(wl, c, dev)
+    TW = None
+    if g > 1:                          # per-token group weights [g][M]
+        TW = torch.empty(g, M, device=dev)
+        for c in range(nch):
+            TW[:, c * ch:(c + 1) * ch] = synth.token_weights_chunk(wl, c, dev)
     W = synth.weights(wl, dev).contiguous()
-    H = torch.empty(K, K, device=dev)
+    H = torch.empty((g, K, K) if g > 1 else (K, K), device=dev)
+    C = torch.empty(K, K, device=dev) if wl.gptaq else None
+    P1 = torch.empty(K, K, device=dev) if wl.gptaq else None
     codes = torch.empty(N, K, dtype=torch.uint8, device=dev)
     scales = torch.empty(N, device=dev)
     status = gq.new_status(dev)
-    ws_p = torch.empty(gq.gptq_workspace_size(gq.GPTQ_OP_PREPARE, K, 0, 1, 0), dtype=torch.uint8,
+    ws_p = torch.empty(gq.gptq_workspace_size(gq.GPTQ_OP_PREPARE, K, 0, g, 0), dtype=torch.uint8,
                        device=dev)
-    ws_q = torch.empty(gq.gptq_workspace_size(gq.GPTQ_OP_QUANTIZE, K, N, 1, wl.blocksize),
+    ws_q = torch.empty(gq.gptq_workspace_size(gq.GPTQ_OP_QUANTIZE, K, N, g, wl.blocksize),
                        dtype=torch.uint8, device=dev)
+    ws_r = (torch.empty(gq.gptq_workspace_size(gq.GPTQ_OP_RESIDUAL, K, 0, 1, 0), dtype=torch.uint8,
+                        device=dev) if wl.gptaq else None)
     stream = torch.cuda.current_stream(dev)
     gram_ev = []
 
     def step(record=None):
         H.zero_()
+        if C is not None:
+            C.zero_()
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
         ev[0].record(stream)
         for c in range(nch):
             if record is not None:
                 a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a.record(stream)
-            gq.gptq_accumulate_hessian(H, X[c * ch:(c + 1) * ch], stream=stream)
+            w = None if TW is None else TW[:, c * ch:(c + 1) * ch]
+            gq.gptq_accumulate_hessian(H, X[c * ch:(c + 1) * ch], w, status=status, stream=stream)
             if record is not None:
                 b.record(stream)
                 record.append((a, b))
+            if C is not None:
+                gq.gptaq_accumulate_cross(C, Xf[c * ch:(c + 1) * ch], X[c * ch:(c + 1) * ch],
+                                          status=status, stream=stream)
         ev[1].record(stream)
         gq.gptq_prepare(H, wl.percdamp, workspace=ws_p, status=status, stream=stream)
+        if P1 is not None:
+            gq.gptaq_residual(P1, C, H, workspace=ws_r, stream=stream)
         ev[2].record(stream)
-        gq.gptq_quantize_layer(W, H, wl.bits, wl.blocksize, scales_out=scales, codes=codes,
-                               workspace=ws_q, status=status, stream=stream)
+        gq.gptq_quantize_layer(W, H, wl.bits, wl.blocksize, groups=g, P1=P1, scales_out=scales,
+                               codes=codes, workspace=ws_q, status=status, stream=stream)
         ev[3].record(stream)
         return ev
 
@@ -282,21 +305,24 @@ def run_ours(args, rank, world, local_rank):
     ms_per_step = total_ms / args.steps
 
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and g == 1 and not wl.gptaq:
         e2e = run_e2e(args, wl, X, W, dev, gq, torch, dist, world)
 
     if rank != 0:
         return None
     clocks = clk.summary()
-    flops_launch = float(ch) * K * (K + 1)          # symmetric Gram work per 65,536-token chunk
+    # symmetric Gram work per 65,536-token chunk (per group for weighted Hessians)
+    flops_launch = float(ch) * K * (K + 1) * g
     peaks = load_peaks()
     # the dominant kernel is the tcgen05 Gram; it is timed inside a seconds-long step, so it
     # is compared with the sustained bf16 peak (fallback 1400 TFLOP/s when no measurement)
     peak = peaks.get("bf16_tflops_sustained") or 1400.0
     achieved = flops_launch / (gram_launch_ms * 1e-3) / 1e12
-    roofline = {"kernel": "k_gram_tc (gptq_accumulate_hessian, tcgen05)", "bound": "tensor",
+    roofline = {"kernel": ("k_gram_tc" if g == 1 else "k_gram_x_tc (weighted)") +
+                          " (gptq_accumulate_hessian, tcgen05)", "bound": "tensor",
                 "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "traffic": GRAM_TRAFFIC_BYTES,
+                "frac": round(achieved / peak, 4),
+                "traffic": GRAM_TRAFFIC_BYTES if (g == 1 and args.workload == "mlp_up_w3") else None,
                 "peak_source": ("MEASURED_PEAKS.json bf16_tflops_sustained (of measured)"
                                 if peaks.get("bf16_tflops_sustained") else "fallback 1.4 PFLOP/s"),
                 "per_launch": f"{ch} tokens x K(K+1) = {flops_launch:.3e} FLOP (symmetric count)",
@@ -306,14 +332,17 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": weights / (ms_per_step * 1e-3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16->f32",
-        "data": "synthetic (seeded Student-t(4)/sqrt2 bf16 tokens, N(0,0.02^2) bf16 weights)",
+        "data": f"synthetic ({wl.stream} bf16 tokens, N(0,{wl.w_sigma}^2) bf16 weights)",
         "config": {"workload": f"{wl.name}: K={K} N={N} tokens={M} (chunks {nch}x{ch}) W{wl.bits} "
-                               f"blocksize {wl.blocksize} percdamp {wl.percdamp}",
+                               f"blocksize {wl.blocksize} percdamp {wl.percdamp} groups {g}"
+                               + (" gptaq" if wl.gptaq else ""),
                    "l2": f"inputs larger than L2 (X {M * K * 2 / 1e9:.1f} GB)", "parallelism": f"{world} independent layers"},
         "breakdown": {"gram_ms": gram_ms, "prepare_ms": prep_ms, "quantize_ms": quant_ms,
                       "layer_solve_ms": prep_ms + quant_ms,
                       "solve_weights_per_s": K * N / ((prep_ms + quant_ms) * 1e-3),
-                      "gram_tflops_symmetric": M * K * (K + 1) / (gram_ms * 1e-3) / 1e12},
+                      "gram_tflops_symmetric": M * K * (K + 1) * g / (gram_ms * 1e-3) / 1e12,
+                      "gram_includes_cross": bool(wl.gptaq),
+                      "prepare_includes_residual": bool(wl.gptaq)},
         "roofline": roofline,
         "gpu_launches": int(launches),
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
