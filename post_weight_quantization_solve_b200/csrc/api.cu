@@ -14,8 +14,9 @@ gptq_status gram_x_tc(float *H, int K, int g, const void *X, const void *X2, int
                       int64_t ldx, const float *w, int64_t ldw, int32_t *status, cudaStream_t st,
                       bool *used);
 size_t prepare_workspace(int K, int g);
+size_t prepare_workspace_compact(int K, int g);
 gptq_status prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out, void *ws,
-                    int32_t *status, cudaStream_t st);
+                    size_t ws_bytes, int32_t *status, cudaStream_t st);
 size_t residual_workspace(int K);
 gptq_status residual(float *P1, const float *C, const float *U, int K, void *ws, cudaStream_t st);
 size_t quantize_workspace(int K, int N, int g, int blocksize);
@@ -85,8 +86,10 @@ gptq_status gptq_prepare(float *H, int K, int g, float percdamp, uint8_t *dead_o
     if (K < 1 || g < 1 || !H || !status || !(percdamp >= 0.f) || !aligned(H, 16))
         return GPTQ_ERR_ARG;
     if (K > GPTQ_MAX_DIM || g > 65535) return GPTQ_ERR_ARG;
-    if (!ws || !aligned(ws, 256) || ws_bytes < prepare_workspace(K, g)) return GPTQ_ERR_WORKSPACE;
-    return prepare(H, K, g, percdamp, dead_out, ws, status, static_cast<cudaStream_t>(stream));
+    if (!ws || !aligned(ws, 256) || ws_bytes < prepare_workspace_compact(K, g))
+        return GPTQ_ERR_WORKSPACE;
+    return prepare(H, K, g, percdamp, dead_out, ws, ws_bytes, status,
+                   static_cast<cudaStream_t>(stream));
 }
 
 gptq_status gptaq_residual(float *P1, const float *C, const float *U, int K, void *ws,

@@ -1,0 +1,373 @@
+// fp32-accurate tensor-core GEMM for the factorisation and the GPTAQ residual:
+//   C[i][j] (+)= alpha * sum_k A[i][k] B(k, j)
+// with every operand carried as a tf32 pair x = hi + lo (hi = tf32(x) rounded to
+// nearest, lo = x - hi, exact in fp32). Three tcgen05 kind::tf32 products
+// hi*hi + hi*lo + lo*hi keep ~21 bits of each factor (the dropped lo*lo term is
+// ~2^-22 relative), enough for the 1e-4 bound on U at the conditioning the
+// damping allows; fp32 accumulation in TMEM in chains of at most MAX_MMA_CHAIN
+// MMAs, flushed with fp32 atomics when an item's inner range is split.
+//
+// Operands are read by TMA from pre-split copies (hi and lo arrays of the same
+// shape), both K-major: A rows i and B^T rows j with k contiguous, 32 x 128 boxes,
+// 128-byte swizzle (SBO = 1 KB, the MMA's k step = 32 bytes inside the atom). A
+// product whose B is naturally row-major in k is given B^T by a transposing split.
+//
+// One launch runs a list of independent products ("items", e.g. every node of one
+// level of the recursive inverse) on a persistent grid; structural flags skip work
+// known to be zero: tiles below the diagonal, A upper triangular (k starts at the
+// row tile), B upper triangular (k ends at the column tile).
+#include <cuda.h>
+
+#include <algorithm>
+#include <vector>
+
+#include "common.cuh"
+#include "gemm_tc32.cuh"
+#include "tc_ptx.cuh"
+
+namespace gptq {
+
+namespace {
+constexpr int G32_BM = 128, G32_BN = 128, G32_BK = 32, G32_STAGES = 3;
+constexpr int G32_TILE = G32_BM * G32_BK * 4;                  // 16 KB (A or B tile)
+constexpr int G32_STAGE = 4 * G32_TILE;                        // A hi, A lo, B hi, B lo
+constexpr int G32_EPI = 4 * 32 * 33 * 4;                       // per-warp 32 x 33 staging
+constexpr int G32_SMEM = G32_STAGES * G32_STAGE + G32_EPI + 1024 + 512;
+constexpr int G32_THREADS = 192;
+constexpr uint32_t G32_TMEM_COLS = 256;                        // two 128-column accumulators
+constexpr int G32_MMA_PER_KSTEP = (G32_BK / 8) * 3;
+}  // namespace
+
+__host__ __device__ constexpr uint32_t idesc_tf32_f32(int M, int N, int b_mn) {
+    return (1u << 4) | (2u << 7) | (2u << 10) | (static_cast<uint32_t>(b_mn) << 16) |
+           (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Unit u -> (item, row tile, column tile, k range).
+__device__ __forceinline__ bool g32_unit(const Tc32Params &p, int u, int &it, int &i0, int &j0,
+                                         int &k0, int &k1) {
+    it = 0;
+    while (it + 1 < p.nitems && u >= p.item[it + 1].unit0) ++it;
+    const Tc32Item &I = p.item[it];
+    const int local = u - I.unit0;
+    const int part = local % I.parts;
+    const int tile = local / I.parts;
+    const int tn = (I.n + G32_BN - 1) / G32_BN;
+    i0 = (tile / tn) * G32_BM;
+    j0 = (tile % tn) * G32_BN;
+    int kb = 0, ke = I.k;
+    if (p.a_upper) kb = (i0 / G32_BK) * G32_BK;
+    if (p.b_upper) ke = min(ke, j0 + G32_BN);
+    if (p.a_lower) ke = min(ke, i0 + G32_BM);
+    const int steps = ke > kb ? (ke - kb) / G32_BK : 0;
+    k0 = kb + (int)((int64_t)steps * part / I.parts) * G32_BK;
+    k1 = kb + (int)((int64_t)steps * (part + 1) / I.parts) * G32_BK;
+    return !(p.upper_tiles && i0 > j0 + G32_BN - 1);
+}
+
+__global__ void __launch_bounds__(G32_THREADS, 1)
+    k_gemm_tc32(const __grid_constant__ CUtensorMap ahi, const __grid_constant__ CUtensorMap alo,
+                const __grid_constant__ CUtensorMap bhi, const __grid_constant__ CUtensorMap blo,
+                const __grid_constant__ Tc32Params p) {
+    if (failed(p.status)) return;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float *epi = reinterpret_cast<float *>(smem + G32_STAGES * G32_STAGE);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + G32_STAGES * G32_STAGE + G32_EPI);
+    uint64_t *empty = full + G32_STAGES;
+    uint64_t *tfull = empty + G32_STAGES;
+    uint64_t *tempty = tfull + 2;
+    uint64_t *drain = tempty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    int *consumed = reinterpret_cast<int *>(tmem_slot + 2);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < G32_STAGES; ++s) {
+            tc::mbar_init(&full[s], 1);
+            tc::mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            tc::mbar_init(&tfull[b], 1);
+            tc::mbar_init(&tempty[b], 128);
+        }
+        tc::mbar_init(drain, 1);
+        *abort = 0;
+        *consumed = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == 1) tc::tmem_alloc(tmem_slot, G32_TMEM_COLS);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0, issued = 0;
+            uint32_t phase = 0;
+            for (int u = blockIdx.x; u < p.units && !*abort; u += gridDim.x) {
+                int it, i0, j0, k0, k1;
+                if (!g32_unit(p, u, it, i0, j0, k0, k1)) continue;
+                const Tc32Item &I = p.item[it];
+                for (int k = k0; k < k1; k += G32_BK) {
+                    if (!tc::mbar_wait(&empty[stage], phase ^ 1, abort)) break;
+                    tc::mbar_arrive_expect_tx(&full[stage], G32_STAGE);
+                    uint8_t *st = smem + stage * G32_STAGE;
+                    tc::tma_load_2d(st, &ahi, &full[stage], I.a_x0 + k, I.a_y0 + i0);
+                    tc::tma_load_2d(st + G32_TILE, &alo, &full[stage], I.a_x0 + k, I.a_y0 + i0);
+                    tc::tma_load_2d(st + 2 * G32_TILE, &bhi, &full[stage], I.b_x0 + k, I.b_y0 + j0);
+                    tc::tma_load_2d(st + 3 * G32_TILE, &blo, &full[stage], I.b_x0 + k, I.b_y0 + j0);
+                    ++issued;
+                    if (++stage == G32_STAGES) { stage = 0; phase ^= 1; }
+                }
+            }
+            if (*abort) {
+                for (int i = *reinterpret_cast<volatile int *>(consumed); i < issued; ++i) {
+                    volatile int never = 0;
+                    tc::mbar_wait(&full[i % G32_STAGES], (i / G32_STAGES) & 1, &never);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_tf32_f32(G32_BM, G32_BN, 0);
+            int stage = 0, acc = 0, n = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            for (int u = blockIdx.x; u < p.units && !*abort; u += gridDim.x) {
+                int it, i0, j0, k0, k1;
+                if (!g32_unit(p, u, it, i0, j0, k0, k1)) continue;
+                if (!tc::mbar_wait(&tempty[acc], acc_phase ^ 1, abort)) break;
+                tc::fence_after_sync();
+                const uint32_t d = tmem + acc * G32_BN;
+                bool ok = true, first = true;
+                for (int k = k0; k < k1; k += G32_BK) {
+                    if (!tc::mbar_wait(&full[stage], phase, abort)) { ok = false; break; }
+                    tc::fence_after_sync();
+                    const uint32_t s0 = tc::smem_u32(smem + stage * G32_STAGE);
+#pragma unroll
+                    for (int kk = 0; kk < G32_BK / 8; ++kk) {
+                        const uint64_t ah = tc::desc_sw128(s0 + kk * 32, 16, 1024);
+                        const uint64_t al = tc::desc_sw128(s0 + G32_TILE + kk * 32, 16, 1024);
+                        const uint64_t bh = tc::desc_sw128(s0 + 2 * G32_TILE + kk * 32, 16, 1024);
+                        const uint64_t bl = tc::desc_sw128(s0 + 3 * G32_TILE + kk * 32, 16, 1024);
+                        mma_tf32(d, ah, bh, idesc, first ? 0u : 1u);
+                        first = false;
+                        mma_tf32(d, ah, bl, idesc, 1u);
+                        mma_tf32(d, al, bh, idesc, 1u);
+                    }
+                    tc::mma_commit(&empty[stage]);
+                    *reinterpret_cast<volatile int *>(consumed) = ++n;
+                    if (++stage == G32_STAGES) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                tc::mma_commit(&tfull[acc]);     // an empty k range leaves TMEM unread
+                if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+            }
+            tc::mma_commit(drain);
+            volatile int never = 0;
+            tc::mbar_wait(drain, 0, &never);
+        }
+    } else {
+        const int quad = warp & 3;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
+            int it, i0, j0, k0, k1;
+            if (!g32_unit(p, u, it, i0, j0, k0, k1)) continue;
+            const Tc32Item &I = p.item[it];
+            if (!tc::mbar_wait(&tfull[acc], acc_phase, abort)) break;
+            tc::fence_after_sync();
+            const bool empty_range = k1 <= k0;
+            // TMEM (thread = row) -> warp-private 32 x 33 stage -> rows written by the
+            // whole warp, 32 consecutive columns per instruction (coalesced)
+            float *stg = epi + (warp - 2) * 32 * 33;
+            const int rbase = i0 + quad * 32;
+#pragma unroll 1
+            for (int c = 0; c < G32_BN / 32; ++c) {
+                uint32_t v[32];
+                tc::tmem_ld_32x32b_x32(tmem + acc * G32_BN + c * 32 + ((uint32_t)(quad * 32) << 16), v);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int q = 0; q < 32; ++q) stg[lane * 33 + q] = __uint_as_float(v[q]);
+                __syncwarp();
+                const int col = j0 + c * 32 + lane;
+#pragma unroll 4
+                for (int rr = 0; rr < 32; ++rr) {
+                    const int r = rbase + rr;
+                    if (r >= I.m || col >= I.n) continue;
+                    float x = empty_range ? 0.f : p.alpha * stg[rr * 33 + lane];
+                    if (p.mask_strict_upper && col <= r) x = 0.f;
+                    float *dst = p.C + I.c_off + (int64_t)r * I.ldc + col;
+                    // no read-back: reductions (accumulate, or split inner range) and
+                    // plain stores (overwrite) are both fire-and-forget
+                    if (p.accumulate || I.parts > 1)
+                        atomicAdd(dst, x);
+                    else
+                        *dst = x;
+                }
+                __syncwarp();
+            }
+            tc::fence_before_sync();
+            tc::mbar_arrive(&tempty[acc]);
+            if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+        }
+    }
+
+    tc::fence_before_sync();
+    __syncthreads();
+    if (*abort && threadIdx.x == 0) set_status(p.status, GPTQ_ERR_TIMEOUT);
+    if (warp == 1) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, G32_TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------------------ host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn tc32_encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+bool tc32_available() { return tc32_encode_fn() != nullptr; }
+
+// fp32 matrix [rows][ld] as boxes of box_cols x box_rows with the 128-byte swizzle.
+gptq_status make_f32_map(CUtensorMap *m, const float *base, int64_t cols, int64_t rows, int64_t ld,
+                         int box_cols, int box_rows) {
+    EncodeTiledFn enc = tc32_encode_fn();
+    if (!enc) return GPTQ_ERR_CUDA;
+    const cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t gstride[1] = {(cuuint64_t)ld * 4};
+    const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(base), gdim, gstride,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? GPTQ_OK : GPTQ_ERR_CUDA;
+}
+
+// x -> (hi, lo): hi = tf32(x) (round to nearest), lo = x - hi. rows x cols (ld_in) into
+// rows x cols (ld_out). One grid row per matrix row, batched over blockIdx.z.
+__global__ void k_split_tf32(const float *__restrict__ in, int64_t ld_in, int cols,
+                             float *__restrict__ hi, float *__restrict__ lo, int64_t ld_out,
+                             int64_t batch_in, int64_t batch_out) {
+    const int64_t r = blockIdx.y;
+    in += blockIdx.z * batch_in + r * ld_in;
+    hi += blockIdx.z * batch_out + r * ld_out;
+    lo += blockIdx.z * batch_out + r * ld_out;
+    for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < cols; c += gridDim.x * blockDim.x) {
+        const float x = in[c];
+        uint32_t h;
+        asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(x));
+        const float hf = __uint_as_float(h);
+        hi[c] = hf;
+        lo[c] = x - hf;
+    }
+}
+
+gptq_status split_tf32(const float *in, int64_t ld_in, int rows, int cols, float *hi, float *lo,
+                       int64_t ld_out, int batch, int64_t batch_in, int64_t batch_out,
+                       cudaStream_t st) {
+    if (rows <= 0 || cols <= 0) return GPTQ_OK;
+    const int bx = (int)std::min<int64_t>(8, (cols + 255) / 256);
+    k_split_tf32<<<dim3(bx, rows, batch), 256, 0, st>>>(in, ld_in, cols, hi, lo, ld_out, batch_in,
+                                                        batch_out);
+    return launch_status();
+}
+
+// Transposing split: in rows x cols (ld_in) -> hi/lo cols x rows (ld_out), through
+// 32 x 32 shared-memory tiles; batched over blockIdx.z.
+__global__ void k_split_tf32_t(const float *__restrict__ in, int64_t ld_in, int rows, int cols,
+                               float *__restrict__ hi, float *__restrict__ lo, int64_t ld_out,
+                               int64_t batch_in, int64_t batch_out) {
+    __shared__ float t[32][33];
+    in += blockIdx.z * batch_in;
+    hi += blockIdx.z * batch_out;
+    lo += blockIdx.z * batch_out;
+    const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+    for (int y = threadIdx.y; y < 32; y += 8) {
+        const int r = r0 + y, c = c0 + threadIdx.x;
+        t[y][threadIdx.x] = (r < rows && c < cols) ? in[(int64_t)r * ld_in + c] : 0.f;
+    }
+    __syncthreads();
+    for (int y = threadIdx.y; y < 32; y += 8) {
+        const int c = c0 + y, r = r0 + threadIdx.x;      // output row c, column r
+        if (c < cols && r < rows) {
+            const float x = t[threadIdx.x][y];
+            uint32_t h;
+            asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(x));
+            const float hf = __uint_as_float(h);
+            hi[(int64_t)c * ld_out + r] = hf;
+            lo[(int64_t)c * ld_out + r] = x - hf;
+        }
+    }
+}
+
+gptq_status split_tf32_t(const float *in, int64_t ld_in, int rows, int cols, float *hi, float *lo,
+                         int64_t ld_out, int batch, int64_t batch_in, int64_t batch_out,
+                         cudaStream_t st) {
+    if (rows <= 0 || cols <= 0) return GPTQ_OK;
+    k_split_tf32_t<<<dim3((cols + 31) / 32, (rows + 31) / 32, batch), dim3(32, 8), 0, st>>>(
+        in, ld_in, rows, cols, hi, lo, ld_out, batch_in, batch_out);
+    return launch_status();
+}
+
+static int tc32_sms() {
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+// Fill the unit table (tiles x parts per item, parts bounding the MMA chains) and
+// launch. Items whose C needs zeroing when split (overwrite mode) are zeroed here.
+gptq_status launch_gemm_tc32(const CUtensorMap maps[4], Tc32Params &p, cudaStream_t st) {
+    if (p.nitems <= 0) return GPTQ_OK;
+    int units = 0;
+    const int max_steps_per_part = std::max(1, tc::MAX_MMA_CHAIN / G32_MMA_PER_KSTEP);
+    for (int i = 0; i < p.nitems; ++i) {
+        Tc32Item &I = p.item[i];
+        const int tiles = ((I.m + G32_BM - 1) / G32_BM) * ((I.n + G32_BN - 1) / G32_BN);
+        const int steps = (I.k + G32_BK - 1) / G32_BK;
+        I.parts = std::max(1, (steps + max_steps_per_part - 1) / max_steps_per_part);
+        I.unit0 = units;
+        units += tiles * I.parts;
+    }
+    p.units = units;
+    if (units == 0) return GPTQ_OK;
+    const int grid = std::min(units, tc32_sms());
+    cudaFuncSetAttribute(k_gemm_tc32, cudaFuncAttributeMaxDynamicSharedMemorySize, G32_SMEM);
+    k_gemm_tc32<<<grid, G32_THREADS, G32_SMEM, st>>>(maps[0], maps[1], maps[2], maps[3], p);
+    return launch_status();
+}
+
+}  // namespace gptq

@@ -25,6 +25,7 @@
 
 #include "common.cuh"
 #include "gemm_simt.cuh"
+#include "gemm_tc32.cuh"
 
 namespace gptq {
 
@@ -392,18 +393,203 @@ static gptq_status tri_inverse(float *H, int K, int g, const Blocks &bk, float *
     return GPTQ_OK;
 }
 
-size_t prepare_workspace(int K, int g) {
+// Compact workspace: damped diagonal + one level's inverse scratch T (fp32 SIMT path).
+size_t prepare_workspace_compact(int K, int g) {
     Carver c(nullptr);
     c.take<float>((size_t)g * K);
     c.take<float>((size_t)g * inverse_scratch_floats(K));
     return round_up(c.off, 256);
 }
 
+static bool tc_inverse_eligible(int K) { return K % 32 == 0 && K >= 256; }
+
+// Tensor-core path (one group at a time): tf32 pairs of H and of H^T (4 K^2) and of
+// one level's T^T scratch (2 x the inverse scratch).
+static size_t tc_extra_floats(int K) {
+    return 4 * (size_t)K * K + 2 * inverse_scratch_floats(K) + 4 * 64;
+}
+
+// Panel and trailing update of one Cholesky step on the tensor cores, for one group:
+//   R[0:j0, J] = H[0:j0, J] U_JJ^T            (A = rows of the column block, B^T = U_JJ rows)
+//   H[0:j0, 0:j0] -= R[0:j0, J] R[0:j0, J]^T  (A = B^T = rows of R; upper tiles)
+// The tf32 pairs of the column block (j1 x nb) reuse the front of the H-pair buffers.
+static gptq_status chol_step_tc(float *H, int K, int j0, int j1, float *ex, int32_t *status,
+                                cudaStream_t st) {
+    const int nb = j1 - j0;
+    float *Ch = ex, *Cl = Ch + (size_t)j1 * nb;
+    static thread_local Tc32Params pp, ps;
+    CUtensorMap m[4];
+    gptq_status s;
+    if ((s = split_tf32(H + j0, K, j1, nb, Ch, Cl, nb, 1, 0, 0, st)) != GPTQ_OK) return s;
+    if ((s = make_f32_map(&m[0], Ch, nb, j1, nb, 32, 128)) != GPTQ_OK) return s;
+    if ((s = make_f32_map(&m[1], Cl, nb, j1, nb, 32, 128)) != GPTQ_OK) return s;
+    m[2] = m[0]; m[3] = m[1];
+    pp = Tc32Params{};
+    pp.C = H; pp.alpha = 1.f; pp.accumulate = 0; pp.status = status; pp.nitems = 1;
+    pp.item[0].m = j0; pp.item[0].n = nb; pp.item[0].k = nb;
+    pp.item[0].a_x0 = 0; pp.item[0].a_y0 = 0; pp.item[0].b_x0 = 0; pp.item[0].b_y0 = j0;
+    pp.item[0].c_off = j0; pp.item[0].ldc = K;
+    if ((s = launch_gemm_tc32(m, pp, st)) != GPTQ_OK) return s;
+    // pairs of the new panel R (rows 0..j0 of the block, overwriting the front)
+    if ((s = split_tf32(H + j0, K, j0, nb, Ch, Cl, nb, 1, 0, 0, st)) != GPTQ_OK) return s;
+    ps = Tc32Params{};
+    ps.C = H; ps.alpha = -1.f; ps.accumulate = 1; ps.upper_tiles = 1; ps.status = status;
+    ps.nitems = 1;
+    ps.item[0].m = j0; ps.item[0].n = j0; ps.item[0].k = nb;
+    ps.item[0].a_x0 = 0; ps.item[0].a_y0 = 0; ps.item[0].b_x0 = 0; ps.item[0].b_y0 = 0;
+    ps.item[0].c_off = 0; ps.item[0].ldc = K;
+    return launch_gemm_tc32(m, ps, st);
+}
+
+// Trailing sizes below this stay on the SIMT kernels (launch-bound there).
+constexpr int TC_STEP_MIN = 1024;
+
+size_t prepare_workspace(int K, int g) {
+    size_t base = prepare_workspace_compact(K, g);
+    if (!tc_inverse_eligible(K)) return base;
+    return round_up(base + tc_extra_floats(K) * sizeof(float), 256);
+}
+
+// tf32 pairs of square blocks H[r0:r0+n, r0:r0+n] (one block per blockIdx.z), written
+// at the same positions of the pair arrays; transposed pairs when `transposed`.
+struct SplitBlocks {
+    int n_items;
+    int r0[TC32_MAX_ITEMS], n[TC32_MAX_ITEMS];
+};
+
+__global__ void k_split_blocks(const float *__restrict__ H, int K, float *__restrict__ hi,
+                               float *__restrict__ lo, int transposed, const SplitBlocks sb) {
+    __shared__ float t[32][33];
+    const int r0 = sb.r0[blockIdx.z], n = sb.n[blockIdx.z];
+    const int tr = blockIdx.y * 32, tcol = blockIdx.x * 32;
+    if (tr >= n || tcol >= n) return;
+    for (int y = threadIdx.y; y < 32; y += 8) {
+        const int r = tr + y, c = tcol + threadIdx.x;
+        t[y][threadIdx.x] = (r < n && c < n) ? H[(int64_t)(r0 + r) * K + r0 + c] : 0.f;
+    }
+    __syncthreads();
+    for (int y = threadIdx.y; y < 32; y += 8) {
+        int orow, ocol;
+        float x;
+        if (transposed) { orow = tcol + y; ocol = tr + threadIdx.x; x = t[threadIdx.x][y]; }
+        else { orow = tr + y; ocol = tcol + threadIdx.x; x = t[y][threadIdx.x]; }
+        if (orow < n && ocol < n) {
+            uint32_t h;
+            asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(x));
+            const float hf = __uint_as_float(h);
+            const int64_t o = (int64_t)(r0 + orow) * K + r0 + ocol;
+            hi[o] = hf;
+            lo[o] = x - hf;
+        }
+    }
+}
+
+__global__ void k_zero_blocks(float *C, const Tc32Params p) {
+    const Tc32Item &I = p.item[blockIdx.z];
+    const int r = blockIdx.y;
+    if (r >= I.m) return;
+    float *row = C + I.c_off + (int64_t)r * I.ldc;
+    for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < I.n; c += gridDim.x * blockDim.x)
+        row[c] = 0.f;
+}
+
+// Level-batched inverse of one group on the tensor cores (the recursion of
+// tri_inverse). Every operand is K-major: per level, with tf32 pairs of H and H^T,
+//   T^T = U[m:b, m:b]^T R[a:m, m:b]^T      (A = rows of H^T, lower triangular)
+//   U[a:m, m:b] = -U[a:m, a:m] T           (B^T = rows of T^T; A upper triangular)
+static gptq_status tri_inverse_tc(float *H, int K, const Blocks &bk, float *Tt, float *ex,
+                                  int32_t *status, cudaStream_t st) {
+    std::vector<std::vector<InvNode>> levels;
+    inv_nodes(bk, K, 0, bk.T, 0, levels);
+    const int64_t KK = (int64_t)K * K;
+    const int64_t tsz = (int64_t)inverse_scratch_floats(K);
+    float *Hh = ex, *Hl = Hh + KK, *Gh = Hl + KK, *Gl = Gh + KK;   // H and H^T pairs
+    float *Th = Gl + KK, *Tl = Th + tsz;
+    static thread_local Tc32Params p1, p2;
+    CUtensorMap mh[2], mg[2], m1[4], m2[4];
+    gptq_status s;
+    if ((s = make_f32_map(&mh[0], Hh, K, K, K, 32, 128)) != GPTQ_OK) return s;
+    if ((s = make_f32_map(&mh[1], Hl, K, K, K, 32, 128)) != GPTQ_OK) return s;
+    if ((s = make_f32_map(&mg[0], Gh, K, K, K, 32, 128)) != GPTQ_OK) return s;
+    if ((s = make_f32_map(&mg[1], Gl, K, K, K, 32, 128)) != GPTQ_OK) return s;
+    for (int d = (int)levels.size() - 1; d >= 0; --d) {
+        const std::vector<InvNode> &lv = levels[d];
+        if ((int)lv.size() > TC32_MAX_ITEMS) return GPTQ_ERR_ARG;
+        // T^T of this level: node blocks (b - m) x (m - a) stacked, common pitch
+        int pitch = 0, trows = 0;
+        std::vector<int> trow0(lv.size());
+        for (size_t ni = 0; ni < lv.size(); ++ni) {
+            pitch = std::max(pitch, lv[ni].m - lv[ni].a);
+            trow0[ni] = trows;
+            trows += lv[ni].b - lv[ni].m;
+        }
+        if ((int64_t)trows * pitch > tsz) return GPTQ_ERR_WORKSPACE;
+        {   // pairs of the node blocks [a, b) x [a, b) only (normal and transposed)
+            static thread_local SplitBlocks sb;
+            sb.n_items = (int)lv.size();
+            int nmax = 0;
+            for (size_t ni = 0; ni < lv.size(); ++ni) {
+                sb.r0[ni] = lv[ni].a;
+                sb.n[ni] = lv[ni].b - lv[ni].a;
+                nmax = std::max(nmax, sb.n[ni]);
+            }
+            const dim3 grid((nmax + 31) / 32, (nmax + 31) / 32, sb.n_items);
+            k_split_blocks<<<grid, dim3(32, 8), 0, st>>>(H, K, Hh, Hl, 0, sb);
+            if ((s = launch_status()) != GPTQ_OK) return s;
+            k_split_blocks<<<grid, dim3(32, 8), 0, st>>>(H, K, Gh, Gl, 1, sb);
+            if ((s = launch_status()) != GPTQ_OK) return s;
+        }
+        cudaMemsetAsync(Tt, 0, sizeof(float) * (size_t)trows * pitch, st);
+        // T^T = (U_bb^T)(R_ab^T): A rows j of H^T at column m, B^T rows i of H at column m
+        p1 = Tc32Params{};
+        p1.C = Tt; p1.alpha = 1.f; p1.accumulate = 1; p1.a_lower = 1; p1.status = status;
+        p1.nitems = (int)lv.size();
+        for (size_t ni = 0; ni < lv.size(); ++ni) {
+            const InvNode &nd = lv[ni];
+            Tc32Item &I = p1.item[ni];
+            I.m = nd.b - nd.m; I.n = nd.m - nd.a; I.k = nd.b - nd.m;
+            I.a_x0 = nd.m; I.a_y0 = nd.m;
+            I.b_x0 = nd.m; I.b_y0 = nd.a;
+            I.c_off = (int64_t)trow0[ni] * pitch;
+            I.ldc = pitch;
+        }
+        m1[0] = mg[0]; m1[1] = mg[1]; m1[2] = mh[0]; m1[3] = mh[1];
+        if ((s = launch_gemm_tc32(m1, p1, st)) != GPTQ_OK) return s;
+        if ((s = split_tf32(Tt, pitch, trows, pitch, Th, Tl, pitch, 1, 0, 0, st)) != GPTQ_OK) return s;
+        if ((s = make_f32_map(&m2[2], Th, pitch, trows, pitch, 32, 128)) != GPTQ_OK) return s;
+        if ((s = make_f32_map(&m2[3], Tl, pitch, trows, pitch, 32, 128)) != GPTQ_OK) return s;
+        m2[0] = mh[0]; m2[1] = mh[1];
+        // U_ab = -U_aa T into zeroed blocks of H: A rows of H at column a, B^T rows of T^T
+        p2 = Tc32Params{};
+        p2.C = H; p2.alpha = -1.f; p2.accumulate = 1; p2.a_upper = 1; p2.status = status;
+        p2.nitems = (int)lv.size();
+        int maxm = 0, maxn = 0;
+        for (size_t ni = 0; ni < lv.size(); ++ni) {
+            const InvNode &nd = lv[ni];
+            Tc32Item &I = p2.item[ni];
+            I.m = nd.m - nd.a; I.n = nd.b - nd.m; I.k = nd.m - nd.a;
+            I.a_x0 = nd.a; I.a_y0 = nd.a;
+            I.b_x0 = 0; I.b_y0 = trow0[ni];
+            I.c_off = (int64_t)nd.a * K + nd.m;
+            I.ldc = K;
+            maxm = std::max(maxm, I.m);
+            maxn = std::max(maxn, I.n);
+        }
+        k_zero_blocks<<<dim3(std::min(8, (maxn + 255) / 256), maxm, p2.nitems), 256, 0, st>>>(H, p2);
+        if ((s = launch_status()) != GPTQ_OK) return s;
+        if ((s = launch_gemm_tc32(m2, p2, st)) != GPTQ_OK) return s;
+    }
+    return GPTQ_OK;
+}
+
 gptq_status prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out, void *ws,
-                    int32_t *status, cudaStream_t st) {
+                    size_t ws_bytes, int32_t *status, cudaStream_t st) {
     Carver c(ws);
     float *diag_d = c.take<float>((size_t)g * K);
     float *T = c.take<float>((size_t)g * inverse_scratch_floats(K));
+    const bool use_tc = tc_inverse_eligible(K) && tc32_available() &&
+                        ws_bytes >= prepare_workspace(K, g);
+    float *ex = use_tc ? c.take<float>(tc_extra_floats(K)) : nullptr;
     const int64_t KK = (int64_t)K * K;
 
     k_check_finite<<<592, 256, 0, st>>>(H, KK * g, status);
@@ -423,6 +609,12 @@ gptq_status prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out, v
         k_chol_diag<<<g, DG_T, chol_smem, st>>>(H, K, j0, nb, diag_d, tol, status);
         if ((s = launch_status()) != GPTQ_OK) return s;
         if (j0 == 0) break;
+        if (use_tc && j0 >= TC_STEP_MIN && nb % 32 == 0) {
+            for (int gi = 0; gi < g; ++gi)
+                if ((s = chol_step_tc(H + (int64_t)gi * KK, K, j0, j1, ex, status, st)) != GPTQ_OK)
+                    return s;
+            continue;
+        }
         // panel: R[0:j0, J] = H[0:j0, J] U_JJ^T  (in place: each CTA owns whole rows)
         GemmParams pp = gemm_params(j0, nb, nb, H + j0, K, H + (int64_t)j0 * K + j0, K,
                                     H + j0, K, 1.f, 0, status);
@@ -438,6 +630,12 @@ gptq_status prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out, v
     // inverse reads whole tiles of its triangular operands, so clear it first.
     k_zero_lower<<<dim3((K + 255) / 256 > 8 ? 8 : (K + 255) / 256, K, g), 256, 0, st>>>(H, K);
     if ((s = launch_status()) != GPTQ_OK) return s;
+    if (use_tc) {
+        for (int gi = 0; gi < g; ++gi)
+            if ((s = tri_inverse_tc(H + (int64_t)gi * KK, K, bk, T, ex, status, st)) != GPTQ_OK)
+                return s;
+        return GPTQ_OK;
+    }
     return tri_inverse(H, K, g, bk, T, status, st);
 }
 

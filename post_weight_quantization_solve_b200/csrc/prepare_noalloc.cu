@@ -14,9 +14,9 @@
 
 namespace gptq {
 
-size_t prepare_workspace(int K, int g);
+size_t prepare_workspace_compact(int K, int g);
 gptq_status prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out, void *ws,
-                    int32_t *status, cudaStream_t st);
+                    size_t ws_bytes, int32_t *status, cudaStream_t st);
 
 // 16 MiB + 64 KiB: enough for K <= 4096 with one Hessian (or K <= 2048 with g <= 4).
 constexpr size_t NOALLOC_SCRATCH_BYTES = (16u << 20) + (64u << 10);
@@ -55,9 +55,10 @@ extern "C" gptq_status gptq_prepare_noalloc(float *H, int K, int g, float percda
     if (K < 1 || g < 1 || !H || !status || !(percdamp >= 0.f) || !aligned(H, 16))
         return GPTQ_ERR_ARG;
     if (K > GPTQ_MAX_DIM) return GPTQ_ERR_ARG;
-    if (prepare_workspace(K, g) > NOALLOC_SCRATCH_BYTES) return GPTQ_ERR_ARG;
+    if (prepare_workspace_compact(K, g) > NOALLOC_SCRATCH_BYTES) return GPTQ_ERR_ARG;
     void *ws = nullptr;
     gptq_status s = scratch_for_current_device(&ws);
     if (s != GPTQ_OK) return s;
-    return prepare(H, K, g, percdamp, dead_out, ws, status, static_cast<cudaStream_t>(stream));
+    return prepare(H, K, g, percdamp, dead_out, ws, NOALLOC_SCRATCH_BYTES, status,
+                   static_cast<cudaStream_t>(stream));
 }

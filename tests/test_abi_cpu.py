@@ -41,7 +41,7 @@ def test_status_strings(lib):
 def test_workspace_sizes(lib):
     p1 = gq.gptq_workspace_size(gq.GPTQ_OP_PREPARE, 4096, 0, 1, 0)
     p4 = gq.gptq_workspace_size(gq.GPTQ_OP_PREPARE, 4096, 0, 4, 0)
-    assert p1 > 4096 * 4 and p4 > 3 * p1
+    assert p1 > 4096 * 4 and p4 > p1
     q = gq.gptq_workspace_size(gq.GPTQ_OP_QUANTIZE, 4096, 14336, 1, 128)
     assert q >= 4096 * 14336 * 4
     assert gq.gptq_workspace_size(gq.GPTQ_OP_RESIDUAL, 512, 0, 1, 0) >= 512 * 512 * 4
