@@ -31,8 +31,7 @@ namespace {
 constexpr int G32_BM = 128, G32_BN = 128, G32_BK = 32, G32_STAGES = 3;
 constexpr int G32_TILE = G32_BM * G32_BK * 4;                  // 16 KB (A or B tile)
 constexpr int G32_STAGE = 4 * G32_TILE;                        // A hi, A lo, B hi, B lo
-constexpr int G32_EPI = 4 * 32 * 33 * 4;                       // per-warp 32 x 33 staging
-constexpr int G32_SMEM = G32_STAGES * G32_STAGE + G32_EPI + 1024 + 512;
+constexpr int G32_SMEM = G32_STAGES * G32_STAGE + 1024 + 512;
 constexpr int G32_THREADS = 192;
 constexpr uint32_t G32_TMEM_COLS = 256;                        // two 128-column accumulators
 constexpr int G32_MMA_PER_KSTEP = (G32_BK / 8) * 3;
@@ -53,26 +52,39 @@ __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64
         : "memory");
 }
 
-// Unit u -> (item, row tile, column tile, k range).
-__device__ __forceinline__ bool g32_unit(const Tc32Params &p, int u, int &it, int &i0, int &j0,
-                                         int &k0, int &k1) {
-    it = 0;
+// One unit of work: an output tile of one item and a part of its k range, with the
+// item's fields copied into registers (the kernel parameter lives in the constant
+// bank; reading it through a reference inside loops that store to global memory
+// makes every access a reload).
+struct G32Unit {
+    int i0, j0, k0, k1;
+    int m, n, ldc, parts;
+    int a_x0, a_y0, b_x0, b_y0;
+    int64_t c_off;
+};
+
+// Unit u -> (item, row tile, column tile, k range); false for a tile the structure skips.
+__device__ __forceinline__ bool g32_unit(const Tc32Params &p, int u, G32Unit &w) {
+    int it = 0;
     while (it + 1 < p.nitems && u >= p.item[it + 1].unit0) ++it;
-    const Tc32Item &I = p.item[it];
+    const Tc32Item I = p.item[it];
     const int local = u - I.unit0;
     const int part = local % I.parts;
     const int tile = local / I.parts;
     const int tn = (I.n + G32_BN - 1) / G32_BN;
-    i0 = (tile / tn) * G32_BM;
-    j0 = (tile % tn) * G32_BN;
+    w.i0 = (tile / tn) * G32_BM;
+    w.j0 = (tile % tn) * G32_BN;
     int kb = 0, ke = I.k;
-    if (p.a_upper) kb = (i0 / G32_BK) * G32_BK;
-    if (p.b_upper) ke = min(ke, j0 + G32_BN);
-    if (p.a_lower) ke = min(ke, i0 + G32_BM);
+    if (p.a_upper) kb = (w.i0 / G32_BK) * G32_BK;
+    if (p.b_upper) ke = min(ke, w.j0 + G32_BN);
+    if (p.a_lower) ke = min(ke, w.i0 + G32_BM);
     const int steps = ke > kb ? (ke - kb) / G32_BK : 0;
-    k0 = kb + (int)((int64_t)steps * part / I.parts) * G32_BK;
-    k1 = kb + (int)((int64_t)steps * (part + 1) / I.parts) * G32_BK;
-    return !(p.upper_tiles && i0 > j0 + G32_BN - 1);
+    w.k0 = kb + (int)((int64_t)steps * part / I.parts) * G32_BK;
+    w.k1 = kb + (int)((int64_t)steps * (part + 1) / I.parts) * G32_BK;
+    w.m = I.m; w.n = I.n; w.ldc = I.ldc; w.parts = I.parts;
+    w.a_x0 = I.a_x0; w.a_y0 = I.a_y0; w.b_x0 = I.b_x0; w.b_y0 = I.b_y0;
+    w.c_off = I.c_off;
+    return !(p.upper_tiles && w.i0 > w.j0 + G32_BN - 1);
 }
 
 __global__ void __launch_bounds__(G32_THREADS, 1)
@@ -83,8 +95,7 @@ __global__ void __launch_bounds__(G32_THREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float *epi = reinterpret_cast<float *>(smem + G32_STAGES * G32_STAGE);
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + G32_STAGES * G32_STAGE + G32_EPI);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + G32_STAGES * G32_STAGE);
     uint64_t *empty = full + G32_STAGES;
     uint64_t *tfull = empty + G32_STAGES;
     uint64_t *tempty = tfull + 2;
@@ -120,17 +131,16 @@ __global__ void __launch_bounds__(G32_THREADS, 1)
             int stage = 0, issued = 0;
             uint32_t phase = 0;
             for (int u = blockIdx.x; u < p.units && !*abort; u += gridDim.x) {
-                int it, i0, j0, k0, k1;
-                if (!g32_unit(p, u, it, i0, j0, k0, k1)) continue;
-                const Tc32Item &I = p.item[it];
-                for (int k = k0; k < k1; k += G32_BK) {
+                G32Unit w;
+                if (!g32_unit(p, u, w)) continue;
+                for (int k = w.k0; k < w.k1; k += G32_BK) {
                     if (!tc::mbar_wait(&empty[stage], phase ^ 1, abort)) break;
                     tc::mbar_arrive_expect_tx(&full[stage], G32_STAGE);
                     uint8_t *st = smem + stage * G32_STAGE;
-                    tc::tma_load_2d(st, &ahi, &full[stage], I.a_x0 + k, I.a_y0 + i0);
-                    tc::tma_load_2d(st + G32_TILE, &alo, &full[stage], I.a_x0 + k, I.a_y0 + i0);
-                    tc::tma_load_2d(st + 2 * G32_TILE, &bhi, &full[stage], I.b_x0 + k, I.b_y0 + j0);
-                    tc::tma_load_2d(st + 3 * G32_TILE, &blo, &full[stage], I.b_x0 + k, I.b_y0 + j0);
+                    tc::tma_load_2d(st, &ahi, &full[stage], w.a_x0 + k, w.a_y0 + w.i0);
+                    tc::tma_load_2d(st + G32_TILE, &alo, &full[stage], w.a_x0 + k, w.a_y0 + w.i0);
+                    tc::tma_load_2d(st + 2 * G32_TILE, &bhi, &full[stage], w.b_x0 + k, w.b_y0 + w.j0);
+                    tc::tma_load_2d(st + 3 * G32_TILE, &blo, &full[stage], w.b_x0 + k, w.b_y0 + w.j0);
                     ++issued;
                     if (++stage == G32_STAGES) { stage = 0; phase ^= 1; }
                 }
@@ -148,13 +158,13 @@ __global__ void __launch_bounds__(G32_THREADS, 1)
             int stage = 0, acc = 0, n = 0;
             uint32_t phase = 0, acc_phase = 0;
             for (int u = blockIdx.x; u < p.units && !*abort; u += gridDim.x) {
-                int it, i0, j0, k0, k1;
-                if (!g32_unit(p, u, it, i0, j0, k0, k1)) continue;
+                G32Unit w;
+                if (!g32_unit(p, u, w)) continue;
                 if (!tc::mbar_wait(&tempty[acc], acc_phase ^ 1, abort)) break;
                 tc::fence_after_sync();
                 const uint32_t d = tmem + acc * G32_BN;
                 bool ok = true, first = true;
-                for (int k = k0; k < k1; k += G32_BK) {
+                for (int k = w.k0; k < w.k1; k += G32_BK) {
                     if (!tc::mbar_wait(&full[stage], phase, abort)) { ok = false; break; }
                     tc::fence_after_sync();
                     const uint32_t s0 = tc::smem_u32(smem + stage * G32_STAGE);
@@ -186,40 +196,53 @@ __global__ void __launch_bounds__(G32_THREADS, 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
-            int it, i0, j0, k0, k1;
-            if (!g32_unit(p, u, it, i0, j0, k0, k1)) continue;
-            const Tc32Item &I = p.item[it];
+            G32Unit w;
+            if (!g32_unit(p, u, w)) continue;
             if (!tc::mbar_wait(&tfull[acc], acc_phase, abort)) break;
             tc::fence_after_sync();
-            const bool empty_range = k1 <= k0;
-            // TMEM (thread = row) -> warp-private 32 x 33 stage -> rows written by the
-            // whole warp, 32 consecutive columns per instruction (coalesced)
-            float *stg = epi + (warp - 2) * 32 * 33;
-            const int rbase = i0 + quad * 32;
+            const bool empty_range = w.k1 <= w.k0;
+            const float alpha = p.alpha;
+            const bool mask = p.mask_strict_upper;
+            const bool reduce = p.accumulate || w.parts > 1;
+            float *cbase = p.C + w.c_off;
+            const bool vec_c = (reinterpret_cast<uintptr_t>(p.C) & 15) == 0;
+            // TMEM (thread = row): each thread writes its row's 32 columns of a chunk as
+            // 16-byte stores or reductions when rows are 16-byte aligned
+            const int row = w.i0 + quad * 32 + lane;
+            const bool rvalid = row < w.m;
+            float *crow = cbase + (int64_t)row * w.ldc;
+            const bool v4 = ((w.ldc | (int)(w.c_off & 3)) & 3) == 0 && vec_c;
 #pragma unroll 1
             for (int c = 0; c < G32_BN / 32; ++c) {
                 uint32_t v[32];
                 tc::tmem_ld_32x32b_x32(tmem + acc * G32_BN + c * 32 + ((uint32_t)(quad * 32) << 16), v);
                 tc::tmem_ld_wait();
+                const int col0 = w.j0 + c * 32;
+                if (!rvalid || col0 >= w.n) continue;
+                float x[32];
 #pragma unroll
-                for (int q = 0; q < 32; ++q) stg[lane * 33 + q] = __uint_as_float(v[q]);
-                __syncwarp();
-                const int col = j0 + c * 32 + lane;
-#pragma unroll 4
-                for (int rr = 0; rr < 32; ++rr) {
-                    const int r = rbase + rr;
-                    if (r >= I.m || col >= I.n) continue;
-                    float x = empty_range ? 0.f : p.alpha * stg[rr * 33 + lane];
-                    if (p.mask_strict_upper && col <= r) x = 0.f;
-                    float *dst = p.C + I.c_off + (int64_t)r * I.ldc + col;
-                    // no read-back: reductions (accumulate, or split inner range) and
-                    // plain stores (overwrite) are both fire-and-forget
-                    if (p.accumulate || I.parts > 1)
-                        atomicAdd(dst, x);
-                    else
-                        *dst = x;
+                for (int q = 0; q < 32; ++q) {
+                    x[q] = empty_range ? 0.f : alpha * __uint_as_float(v[q]);
+                    if (mask && col0 + q <= row) x[q] = 0.f;
                 }
-                __syncwarp();
+                // no read-back: reductions (accumulate, or split inner range) and plain
+                // stores (overwrite) are both fire-and-forget
+                if (v4 && col0 + 32 <= w.n) {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 f = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+                        float4 *dst = reinterpret_cast<float4 *>(crow + col0 + 4 * q);
+                        if (reduce) atomicAdd(dst, f);
+                        else *dst = f;
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) {
+                        if (col0 + q >= w.n) break;
+                        if (reduce) atomicAdd(crow + col0 + q, x[q]);
+                        else crow[col0 + q] = x[q];
+                    }
+                }
             }
             tc::fence_before_sync();
             tc::mbar_arrive(&tempty[acc]);
@@ -227,6 +250,7 @@ __global__ void __launch_bounds__(G32_THREADS, 1)
         }
     }
 
+    __syncwarp();   // each role warp reconverges before the block barrier
     tc::fence_before_sync();
     __syncthreads();
     if (*abort && threadIdx.x == 0) set_status(p.status, GPTQ_ERR_TIMEOUT);

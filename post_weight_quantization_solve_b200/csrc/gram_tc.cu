@@ -15,8 +15,9 @@
 // Work: only tiles that meet the upper triangle; the chunk's tokens are split into
 // P equal parts and units (part, tile) are dealt part-major to a persistent grid of
 // one CTA per SM, so CTAs running at the same time read the same token slab (L2
-// reuse). Each unit ends with fp32 vector atomics of alpha * D into H; the lower
-// triangle is mirrored afterwards.
+// reuse). Each unit ends with bulk tensor reductions of alpha * D into H, written
+// both in place (on and above the diagonal) and transposed (strictly above), so H
+// is complete and symmetric after every chunk.
 //
 // Roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer,
 // warps 2-5 epilogue (TMEM lane quadrant = warp % 4). 4-stage smem ring, 2 TMEM
@@ -36,7 +37,8 @@ constexpr int GT_BOX = GT_BK * 64 * 2;                 // one 64 x 64 bf16 box =
 constexpr int GT_A_BYTES = GT_BM * GT_BK * 2;          // 16 KB
 constexpr int GT_B_BYTES = GT_BN * GT_BK * 2;          // 32 KB
 constexpr int GT_STAGE = GT_A_BYTES + GT_B_BYTES;      // 48 KB
-constexpr int GT_SMEM = GT_STAGES * GT_STAGE + 1024 + 256;
+constexpr int GT_EPI = 4 * 32 * 32 * 4;               // one 32 x 32 fp32 box per epilogue warp
+constexpr int GT_SMEM = GT_STAGES * GT_STAGE + GT_EPI + 1024 + 256;
 constexpr int GT_THREADS = 192;
 constexpr uint32_t GT_TMEM_COLS = 512;
 constexpr uint32_t GT_IDESC = tc::idesc_bf16_f32(GT_BM, GT_BN, 1, 1);
@@ -71,12 +73,14 @@ __device__ __forceinline__ void gt_unit(const GramTcParams &p, int u, int &ti, i
 }
 
 __global__ void __launch_bounds__(GT_THREADS, 1)
-    k_gram_tc(const __grid_constant__ CUtensorMap tmap, const GramTcParams p) {
+    k_gram_tc(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap hmap,
+              const GramTcParams p) {
     if (failed(p.status)) return;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + GT_STAGES * GT_STAGE);
+    uint8_t *epi = smem + GT_STAGES * GT_STAGE;       // 1 KB aligned
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + GT_STAGES * GT_STAGE + GT_EPI);
     uint64_t *empty = full + GT_STAGES;
     uint64_t *tfull = empty + GT_STAGES;
     uint64_t *tempty = tfull + 2;
@@ -175,42 +179,68 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
             tc::mbar_wait(drain, 0, &never);
         }
     } else {
+        // alpha * D into H through bulk tensor reductions: the entries on or above the
+        // diagonal as they are, the strictly upper ones also transposed into the lower
+        // triangle, so H stays symmetric without a separate pass. Each warp stages one
+        // 32 x 32 box at a time (128-byte swizzle) and lets the reduction read it.
         const int quad = warp & 3;
         int acc = 0;
         uint32_t acc_phase = 0;
+        uint8_t *buf = epi + (warp - 2) * 4096;
+        const float alpha = p.alpha;
+        auto stage_out = [&](int x, int y) {
+            tc::fence_async_shared();
+            __syncwarp();
+            if (lane == 0) {
+                tc::tma_reduce_add_2d(&hmap, buf, x, y);
+                tc::bulk_commit();
+                tc::bulk_wait_read<0>();    // buf is free again
+            }
+            __syncwarp();
+        };
         for (int u = blockIdx.x; u < units; u += gridDim.x) {
             int ti, tj, k0, k1;
             gt_unit(p, u, ti, tj, k0, k1);
             if (!tc::mbar_wait(&tfull[acc], acc_phase, abort)) break;
             tc::fence_after_sync();
-            const int row = ti * GT_BM + quad * 32 + lane;
-            float *hrow = p.H + (int64_t)row * p.K;
+            const int r0 = ti * GT_BM + quad * 32;      // this warp's 32 rows
+            const int row = r0 + lane;
 #pragma unroll 1
             for (int c = 0; c < GT_BN / 32; ++c) {
                 uint32_t r[32];
                 tc::tmem_ld_32x32b_x32(tmem + acc * GT_BN + c * 32 + ((uint32_t)(quad * 32) << 16), r);
                 tc::tmem_ld_wait();
                 const int col0 = tj * GT_BN + c * 32;
-                if (row < p.K) {
+                if (r0 >= p.K || col0 >= p.K || r0 > col0 + 31) continue;   // nothing on or above
+                // upper part (row <= col) in place: row = lane, chunk q at q ^ (lane & 7)
 #pragma unroll
-                    for (int v = 0; v < 8; ++v) {
-                        const int col = col0 + 4 * v;
-                        if (col < p.K) {
-                            float4 val = make_float4(p.alpha * __uint_as_float(r[4 * v]),
-                                                     p.alpha * __uint_as_float(r[4 * v + 1]),
-                                                     p.alpha * __uint_as_float(r[4 * v + 2]),
-                                                     p.alpha * __uint_as_float(r[4 * v + 3]));
-                            atomicAdd(reinterpret_cast<float4 *>(hrow + col), val);
-                        }
-                    }
+                for (int q = 0; q < 8; ++q) {
+                    float x[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        x[e] = (row <= col0 + 4 * q + e) ? alpha * __uint_as_float(r[4 * q + e]) : 0.f;
+                    *reinterpret_cast<float4 *>(buf + lane * 128 + ((q ^ (lane & 7)) << 4)) =
+                        make_float4(x[0], x[1], x[2], x[3]);
                 }
+                stage_out(col0, r0);
+                if (r0 + 1 > col0 + 31) continue;           // no strictly upper entry
+                // strictly upper part transposed: box row q (column col0 + q), column lane
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    const float x = (row < col0 + q) ? alpha * __uint_as_float(r[q]) : 0.f;
+                    *reinterpret_cast<float *>(buf + q * 128 + ((((lane >> 2) ^ (q & 7))) << 4) +
+                                               (lane & 3) * 4) = x;
+                }
+                stage_out(r0, col0);
             }
             tc::fence_before_sync();
             tc::mbar_arrive(&tempty[acc]);
             if (++acc == 2) { acc = 0; acc_phase ^= 1; }
         }
+        if (lane == 0) tc::bulk_wait_all();
     }
 
+    __syncwarp();   // each role warp reconverges before the block barrier
     tc::fence_before_sync();
     __syncthreads();
     if (*abort && threadIdx.x == 0) set_status(p.status, GPTQ_ERR_TIMEOUT);
@@ -220,7 +250,6 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
     }
 }
 
-gptq_status mirror_upper(float *H, int K, int g, cudaStream_t st);
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
@@ -274,7 +303,7 @@ gptq_status gram_tc(float *H, int K, int g, const void *X, int64_t M, int64_t ld
     *used = false;
     // tensor-core path: plain bf16 Gram (one Hessian, unit weights, no cross term)
     if (g != 1 || w != nullptr || X2 != nullptr || K < 64) return GPTQ_OK;
-    if (!aligned(H, 16)) return GPTQ_OK;
+    if (!aligned(H, 16) || K % 4 != 0) return GPTQ_OK;
     EncodeTiledFn enc = encode_fn();
     if (!enc) return GPTQ_OK;
 
@@ -304,12 +333,23 @@ gptq_status gram_tc(float *H, int K, int g, const void *X, int64_t M, int64_t ld
     const int units = p.T * p.P;
     const int grid = std::min(units, grid_max);
 
+    // H as 32 x 32 fp32 boxes for the epilogue's reductions (rows 16-byte aligned)
+    CUtensorMap hmap;
+    {
+        const cuuint64_t hdim[2] = {(cuuint64_t)K, (cuuint64_t)K};
+        const cuuint64_t hstride[1] = {(cuuint64_t)K * 4};
+        const cuuint32_t hbox[2] = {32, 32};
+        r = enc(&hmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, H, hdim, hstride, hbox, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return GPTQ_ERR_CUDA;
+    }
     cudaFuncSetAttribute(k_gram_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, GT_SMEM);
-    k_gram_tc<<<grid, GT_THREADS, GT_SMEM, st>>>(tmap, p);
+    k_gram_tc<<<grid, GT_THREADS, GT_SMEM, st>>>(tmap, hmap, p);
     gptq_status s = launch_status();
     if (s != GPTQ_OK) return s;
     *used = true;
-    return mirror_upper(H, K, 1, st);
+    return GPTQ_OK;
 }
 
 }  // namespace gptq

@@ -19,7 +19,8 @@
 // Roles (320 threads): warp 0 TMA, warp 1 TMEM + MMA, warps 2-5 epilogue, 6-9
 // transform. Work units (group, token part, tile) are dealt part-major to a
 // persistent grid; the weighted Gram computes only tiles meeting the upper
-// triangle (mirrored afterwards), the cross Gram every tile.
+// triangle (written in place and transposed by the epilogue's bulk reductions),
+// the cross Gram every tile.
 #include <cuda.h>
 
 #include <algorithm>
@@ -36,7 +37,8 @@ constexpr int GX_A = GX_BM * GX_BK * 2;                 // 8 KB (one 128-row bf1
 constexpr int GX_B = GX_BN * GX_BK * 2;                 // 16 KB
 // stage: src0 (A source), src1 (second A source, cross only), B, A_hi, A_lo
 constexpr int GX_STAGE = 2 * GX_A + GX_B + 2 * GX_A;    // 48 KB
-constexpr int GX_SMEM = GX_STAGES * GX_STAGE + 1024 + 512;
+constexpr int GX_EPI = 4 * 32 * 32 * 4;                 // one 32 x 32 fp32 box per epilogue warp
+constexpr int GX_SMEM = GX_STAGES * GX_STAGE + GX_EPI + 1024 + 512;
 constexpr int GX_THREADS = 320;
 constexpr uint32_t GX_TMEM_COLS = 512;
 constexpr uint32_t GX_IDESC = tc::idesc_bf16_f32(GX_BM, GX_BN, 1, 1);
@@ -79,12 +81,14 @@ __device__ __forceinline__ void gx_unit(const GramXParams &p, int u, int &grp, i
 
 __global__ void __launch_bounds__(GX_THREADS, 1)
     k_gram_x_tc(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ CUtensorMap map_a1,
-                const __grid_constant__ CUtensorMap map_b, const GramXParams p) {
+                const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap hmap,
+                const GramXParams p) {
     if (failed(p.status)) return;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + GX_STAGES * GX_STAGE);
+    uint8_t *epi = smem + GX_STAGES * GX_STAGE;       // 1 KB aligned
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + GX_STAGES * GX_STAGE + GX_EPI);
     uint64_t *xfull = full + GX_STAGES;      // transformed tiles ready
     uint64_t *empty = xfull + GX_STAGES;
     uint64_t *tfull = empty + GX_STAGES;
@@ -244,41 +248,85 @@ __global__ void __launch_bounds__(GX_THREADS, 1)
             if (!ok) break;
         }
     } else {
+        // alpha * D into H through bulk tensor reductions (H seen as [g K][K]): the
+        // weighted Gram writes the entries on or above the diagonal and, transposed,
+        // the strictly upper ones (H_g stays symmetric); the cross Gram every entry.
         const int quad = warp & 3;
         int acc = 0;
         uint32_t acc_phase = 0;
+        uint8_t *buf = epi + (warp - 2) * 4096;
+        const float alpha = p.alpha;
+        const bool sym = !p.cross;
+        auto stage_out = [&](int x, int y) {
+            tc::fence_async_shared();
+            __syncwarp();
+            if (lane == 0) {
+                tc::tma_reduce_add_2d(&hmap, buf, x, y);
+                tc::bulk_commit();
+                tc::bulk_wait_read<0>();    // buf is free again
+            }
+            __syncwarp();
+        };
         for (int u = blockIdx.x; u < units; u += gridDim.x) {
             int grp, ti, tj, k0, k1;
             gx_unit(p, u, grp, ti, tj, k0, k1);
             if (!tc::mbar_wait(&tfull[acc], acc_phase, abort)) break;
             tc::fence_after_sync();
-            const int row = ti * GX_BM + quad * 32 + lane;
-            float *hrow = p.H + (int64_t)grp * p.K * p.K + (int64_t)row * p.K;
+            const int r0 = ti * GX_BM + quad * 32;      // this warp's 32 rows
+            const int row = r0 + lane;
+            const int gy = grp * p.K;                   // group offset in the [g K][K] view
 #pragma unroll 1
             for (int c = 0; c < GX_BN / 32; ++c) {
                 uint32_t r[32];
                 tc::tmem_ld_32x32b_x32(tmem + acc * GX_BN + c * 32 + ((uint32_t)(quad * 32) << 16), r);
                 tc::tmem_ld_wait();
                 const int col0 = tj * GX_BN + c * 32;
-                if (row < p.K) {
+                if (r0 >= p.K || col0 >= p.K || (sym && r0 > col0 + 31)) continue;
+                // row = lane, 16-byte chunk q at q ^ (lane & 7) (128-byte swizzle); rows or
+                // columns past K fall outside the map (and H_g) and are dropped
 #pragma unroll
-                    for (int v = 0; v < 8; ++v) {
-                        const int col = col0 + 4 * v;
-                        if (col < p.K)
-                            atomicAdd(reinterpret_cast<float4 *>(hrow + col),
-                                      make_float4(p.alpha * __uint_as_float(r[4 * v]),
-                                                  p.alpha * __uint_as_float(r[4 * v + 1]),
-                                                  p.alpha * __uint_as_float(r[4 * v + 2]),
-                                                  p.alpha * __uint_as_float(r[4 * v + 3])));
-                    }
+                for (int q = 0; q < 8; ++q) {
+                    float x[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        x[e] = (!sym || row <= col0 + 4 * q + e) ? alpha * __uint_as_float(r[4 * q + e]) : 0.f;
+                    *reinterpret_cast<float4 *>(buf + lane * 128 + ((q ^ (lane & 7)) << 4)) =
+                        make_float4(x[0], x[1], x[2], x[3]);
                 }
+                if (r0 + 32 > p.K) {
+                    // keep the box inside H_g: zero the rows past K (the next group's)
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        if (row >= p.K)
+                            *reinterpret_cast<float4 *>(buf + lane * 128 + ((q ^ (lane & 7)) << 4)) =
+                                make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+                stage_out(col0, gy + r0);
+                if (!sym || r0 >= col0 + 31) continue;     // no strictly upper entry
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    const float x = (row < col0 + q && row < p.K) ? alpha * __uint_as_float(r[q]) : 0.f;
+                    *reinterpret_cast<float *>(buf + q * 128 + ((((lane >> 2) ^ (q & 7))) << 4) +
+                                               (lane & 3) * 4) = x;
+                }
+                if (col0 + 32 > p.K) {
+                    // box rows past K would land in the next group's rows: zero them
+#pragma unroll
+                    for (int q = 0; q < 32; ++q)
+                        if (col0 + q >= p.K)
+                            *reinterpret_cast<float *>(buf + q * 128 + ((((lane >> 2) ^ (q & 7))) << 4) +
+                                                       (lane & 3) * 4) = 0.f;
+                }
+                stage_out(r0, gy + col0);
             }
             tc::fence_before_sync();
             tc::mbar_arrive(&tempty[acc]);
             if (++acc == 2) { acc = 0; acc_phase ^= 1; }
         }
+        if (lane == 0) tc::bulk_wait_all();
     }
 
+    __syncwarp();   // each role warp reconverges before the block barrier
     tc::fence_before_sync();
     __syncthreads();
     if (*abort && threadIdx.x == 0) set_status(p.status, GPTQ_ERR_TIMEOUT);
@@ -290,7 +338,8 @@ __global__ void __launch_bounds__(GX_THREADS, 1)
 
 // ------------------------------------------------------------------------------ host side
 
-gptq_status mirror_upper(float *H, int K, int g, cudaStream_t st);
+gptq_status make_f32_map(CUtensorMap *m, const float *base, int64_t cols, int64_t rows, int64_t ld,
+                         int box_cols, int box_rows);
 gptq_status make_bf16_map(CUtensorMap *m, const void *base, int64_t cols, int64_t rows,
                           int64_t ld, int box_rows);
 
@@ -324,7 +373,7 @@ gptq_status gram_x_tc(float *H, int K, int g, const void *X, const void *X2, int
                       int64_t ldx, const float *w, int64_t ldw, int32_t *status,
                       cudaStream_t st, bool *used) {
     *used = false;
-    if (K < 64 || !aligned(H, 16)) return GPTQ_OK;
+    if (K < 64 || K % 4 != 0 || !aligned(H, 16)) return GPTQ_OK;
     const bool cross = X2 != nullptr;
     CUtensorMap ma0, ma1, mb;
     // left source (x for weighted, x_fp for cross), second source (x_q), right operand
@@ -357,11 +406,14 @@ gptq_status gram_x_tc(float *H, int K, int g, const void *X, const void *X2, int
     p.status = status;
     const int units = p.groups * p.T * p.P;
     const int grid = std::min(units, grid_max);
+    // H as [groups K][K] fp32, 32 x 32 boxes with the 128-byte swizzle
+    CUtensorMap hmap;
+    if ((s = make_f32_map(&hmap, H, K, (int64_t)p.groups * K, K, 32, 32)) != GPTQ_OK) return s;
     cudaFuncSetAttribute(k_gram_x_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, GX_SMEM);
-    k_gram_x_tc<<<grid, GX_THREADS, GX_SMEM, st>>>(ma0, ma1, mb, p);
+    k_gram_x_tc<<<grid, GX_THREADS, GX_SMEM, st>>>(ma0, ma1, mb, hmap, p);
     if ((s = launch_status()) != GPTQ_OK) return s;
     *used = true;
-    return cross ? GPTQ_OK : mirror_upper(H, K, g, st);
+    return GPTQ_OK;
 }
 
 }  // namespace gptq

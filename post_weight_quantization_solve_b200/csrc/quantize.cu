@@ -21,9 +21,8 @@
 //             sweep's stores coalesce; the update reads it as an MN-major operand)
 //   Ph, Pl    bf16 [S][ldE] pre-rounding weights (GPTAQ), same layout
 //   Uh, Ul    bf16 [g][K][ldU] U as hi + lo pairs;  Qh, Ql  the same for P1
-// One CTA owns 128 channels of one group for a block; a thread owns a channel and
-// keeps 32 of its block coordinates in registers at a time, the rest of the block
-// in shared memory (coordinate-major so a warp's accesses hit distinct banks).
+// A sweep CTA owns 32 or 64 channels of one group for a block; each warp keeps one
+// 32-coordinate sub-block of 32 channels in registers (k_sweep_block).
 #include <cuda.h>
 
 #include <algorithm>
@@ -33,193 +32,308 @@
 
 namespace gptq {
 
-constexpr int SW_CH = 128;     // channels per CTA
-constexpr int SW_MAXB = 128;   // largest block
-constexpr int SW_ULD = SW_MAXB + 4;
-constexpr int SW_WLD = SW_CH + 1;
-constexpr int SW_CLD = SW_CH + 4;
+constexpr int SW_MAXB = 128;   // largest block: four 32-coordinate sub-blocks
 
-__global__ void k_scale(const void *W, int wdtype, int N, int K, int bits,
-                        const float *scales_in, float *scale, float *scales_out,
-                        int32_t *status) {
-    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-    if (warp >= N) return;
+// Eight consecutive weights of a row as fp32 (one 16-byte load for bf16, two for fp32).
+__device__ __forceinline__ void load8(const __nv_bfloat16 *p, float (&x)[8]) {
+    const uint4 v = *reinterpret_cast<const uint4 *>(p);
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        x[2 * i] = __uint_as_float(u[i] << 16);
+        x[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
+    }
+}
+__device__ __forceinline__ void load8(const float *p, float (&x)[8]) {
+    const float4 a = *reinterpret_cast<const float4 *>(p);
+    const float4 b = *reinterpret_cast<const float4 *>(p + 4);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+
+// One CTA per output channel n: the symmetric scale s_n = 2 max_k |W_nk| / (2^b - 1)
+// from W as given (or the caller's scale), and the fp32 working row with dead
+// coordinates zeroed, from one read of the row.
+template <typename T>
+__global__ void __launch_bounds__(256) k_scale_init(const T *__restrict__ W, float *__restrict__ Wk,
+                                                    int K, int per_group, int bits,
+                                                    const uint8_t *__restrict__ dead,
+                                                    const float *__restrict__ scales_in,
+                                                    float *__restrict__ scale, float *scales_out,
+                                                    float *__restrict__ loss_acc, int vec,
+                                                    int32_t *status) {
+    const int n = blockIdx.x;
+    const T *wr = W + (int64_t)n * K;
+    float *kr = Wk + (int64_t)n * K;
+    const uint8_t *dg = dead ? dead + (int64_t)(n / per_group) * K : nullptr;
     float amax = 0.f;
     bool bad = false;
-    for (int k = lane; k < K; k += 32) {
-        const float v = wdtype == GPTQ_F32
-                            ? static_cast<const float *>(W)[(int64_t)warp * K + k]
-                            : __bfloat162float(
-                                  static_cast<const __nv_bfloat16 *>(W)[(int64_t)warp * K + k]);
-        bad |= !isfinite(v);
-        amax = fmaxf(amax, fabsf(v));
+    if (vec) {   // rows 16-byte aligned for both W and Wk, K % 8 == 0
+        for (int k = threadIdx.x * 8; k < K; k += 256 * 8) {
+            float x[8];
+            load8(wr + k, x);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                bad |= !isfinite(x[i]);
+                amax = fmaxf(amax, fabsf(x[i]));
+                if (dg && dg[k + i]) x[i] = 0.f;
+            }
+            *reinterpret_cast<float4 *>(kr + k) = make_float4(x[0], x[1], x[2], x[3]);
+            *reinterpret_cast<float4 *>(kr + k + 4) = make_float4(x[4], x[5], x[6], x[7]);
+        }
+    } else {
+        for (int k = threadIdx.x; k < K; k += 256) {
+            const float x = to_f32(wr[k]);
+            bad |= !isfinite(x);
+            amax = fmaxf(amax, fabsf(x));
+            kr[k] = (dg && dg[k]) ? 0.f : x;
+        }
     }
+    __shared__ float red[8];
+    __shared__ int redb[8];
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    bad = __any_sync(0xffffffffu, bad);
-    if (lane == 0) {
+    const bool wbad = __any_sync(0xffffffffu, bad);
+    if ((threadIdx.x & 31) == 0) {
+        red[threadIdx.x >> 5] = amax;
+        redb[threadIdx.x >> 5] = wbad;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        bool b = false;
+        for (int i = 0; i < 8; ++i) {
+            amax = fmaxf(amax, red[i]);
+            b |= redb[i] != 0;
+        }
         float s;
         if (scales_in) {
-            s = scales_in[warp];
-            bad |= !(isfinite(s) && s > 0.f);
+            s = scales_in[n];
+            b |= !(isfinite(s) && s > 0.f);
         } else {
             s = amax == 0.f ? 1.f : 2.f * amax / (float)((1 << bits) - 1);
         }
-        if (bad) set_status(status, GPTQ_ERR_NONFINITE);
-        scale[warp] = s;
-        if (scales_out) scales_out[warp] = s;
+        if (b) set_status(status, GPTQ_ERR_NONFINITE);
+        scale[n] = s;
+        if (scales_out) scales_out[n] = s;
+        loss_acc[n] = 0.f;
     }
 }
 
-// One grid row (blockIdx.y) per output channel.
-template <typename T>
-__global__ void k_init_work(const T *W, float *Wk, int N, int K, int per_group,
-                            const uint8_t *dead, float *loss_acc) {
-    const int n = blockIdx.y;
-    const int64_t row = (int64_t)n * K;
-    const uint8_t *dg = dead ? dead + (int64_t)(n / per_group) * K : nullptr;
-    for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < K; k += gridDim.x * blockDim.x) {
-        const bool d = dg && dg[k];
-        Wk[row + k] = d ? 0.f : to_f32(W[row + k]);
-        if (k == 0) loss_acc[n] = 0.f;
-    }
+// 16-byte global -> shared copy that bypasses registers; src_bytes = 0 writes zeros.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
+                     static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                 "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
+// In-block sweep of one block [i0, i0 + bs) for 32 channels of one group.
+// A warp serves 8 channels with 4 lanes each: lane 4 c + q of the warp holds, of
+// channel c, the coordinates 32 b + 8 q + i (i < 8) of every 32-wide sub-block b, so
+// all 32 coordinates of the block stay in registers and every lane has work at every
+// step. At step j = 32 p + t the lane holding coordinate j (slot q = t / 8) rounds it
+// and computes E_j; a shuffle inside the channel's 4 lanes hands E_j to the others,
+// and each lane applies it to its own coordinates (U's zero lower triangle makes the
+// coordinates at or before j no-ops, so no lane masks). The sub-block in work is
+// always w[0]: the register array shifts by one sub-block after each phase. No block
+// barrier inside the sweep. U[blk, blk] (and P1) is staged once per CTA as its ten
+// 32 x 32 blocks on or above the diagonal.
 template <bool GPTAQ>
-__global__ void __launch_bounds__(SW_CH) k_sweep_block(
+__global__ void __launch_bounds__(128, GPTAQ ? 2 : 4) k_sweep_block(
     float *__restrict__ Wk, int N, int per_group, int K, int i0, int bs,
     const float *__restrict__ U, const float *__restrict__ P1, const float *__restrict__ scale,
     int bits, uint8_t *__restrict__ codes, __nv_bfloat16 *__restrict__ Eh,
     __nv_bfloat16 *__restrict__ El, __nv_bfloat16 *__restrict__ Ph, __nv_bfloat16 *__restrict__ Pl,
-    int ldE, int ldG, int erow0, float *__restrict__ loss_acc, const int32_t *status) {
+    int ldE, int ldG, int erow0, float *__restrict__ loss_acc, int vec, const int32_t *status) {
+    constexpr int NCH = 32, CLD = 132;
     if (failed(status)) return;
     extern __shared__ __align__(16) unsigned char smem[];
-    float *Us = reinterpret_cast<float *>(smem);                 // [SW_MAXB][SW_ULD]
-    float *Ps = Us + SW_MAXB * SW_ULD;                           // GPTAQ only
-    float *Wt = Ps + (GPTAQ ? SW_MAXB * SW_ULD : 0);             // [SW_MAXB][SW_WLD]
-    uint8_t *Cs = reinterpret_cast<uint8_t *>(Wt + SW_MAXB * SW_WLD);  // [SW_MAXB][SW_CLD]
+    float *Us = reinterpret_cast<float *>(smem);                 // [10][32][32]
+    float *Ps = Us + 10 * 1024;                                  // GPTAQ only
+    uint8_t *Cs = reinterpret_cast<uint8_t *>(Ps + (GPTAQ ? 10 * 1024 : 0));  // [NCH][CLD]
+    float *rpiv = reinterpret_cast<float *>(Cs + NCH * CLD);    // [SW_MAXB]
 
     const int grp = blockIdx.y;
-    const int n0 = grp * per_group + blockIdx.x * SW_CH;
-    const int nvalid = min(SW_CH, (grp + 1) * per_group - n0);
-    const int tid = threadIdx.x;
-    const int n = n0 + tid;
-    const int64_t ecol = (int64_t)grp * ldG + blockIdx.x * SW_CH + tid;
-    U += (int64_t)grp * K * K;
+    const int cta_ch0 = blockIdx.x * NCH;
+    const int n0 = grp * per_group + cta_ch0;
+    const int nvalid = min(NCH, per_group - cta_ch0);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q = lane & 3;
+    const int ch = warp * 8 + (lane >> 2);
+    const bool valid = ch < nvalid;
+    const int64_t n = (int64_t)n0 + ch;
+    const int nsb = (bs + 31) / 32;
+    const float *Ub = U + (int64_t)grp * K * K + (int64_t)i0 * K + i0;   // U[i0, i0]
+    const float *Pb = GPTAQ ? P1 + (int64_t)i0 * K + i0 : nullptr;
 
-    // Stage U[blk, blk] (and P1[blk, blk]) with zero padding, and the W tile; loads
-    // are unrolled so that many are in flight per thread.
-#pragma unroll 8
-    for (int it = 0; it < SW_MAXB; ++it) {
-        const int r = it, c = tid;
-        const bool in = r < bs && c < bs;
-        Us[r * SW_ULD + c] = in ? U[(int64_t)(i0 + r) * K + i0 + c] : 0.f;
-        if (GPTAQ) Ps[r * SW_ULD + c] = in ? P1[(int64_t)(i0 + r) * K + i0 + c] : 0.f;
+    // the ten blocks (P, Q), P <= Q, of U[blk, blk]; zero outside [0, bs)
+    for (int idx = tid; idx < 10 * 256; idx += 128) {
+        const int blk = idx >> 8;
+        const int P = blk < 4 ? 0 : blk < 7 ? 1 : blk < 9 ? 2 : 3;
+        const int Q = P + blk - (P * 4 - P * (P - 1) / 2);
+        if (Q >= nsb) continue;
+        const int r = (idx >> 3) & 31, c4 = (idx & 7) * 4;
+        const int row = 32 * P + r, col = 32 * Q + c4;
+        float *du = Us + blk * 1024 + r * 32 + c4;
+        float *dp = Ps + blk * 1024 + r * 32 + c4;
+        if (vec & 1) {        // rows 16-byte aligned and bs % 4 == 0
+            const bool in = row < bs && col < bs;
+            const int64_t off = in ? (int64_t)row * K + col : 0;
+            cp_async16(du, Ub + off, in ? 16 : 0);
+            if (GPTAQ) cp_async16(dp, Pb + off, in ? 16 : 0);
+        } else {
+            for (int e = 0; e < 4; ++e) {
+                const bool in = row < bs && col + e < bs;
+                du[e] = in ? Ub[(int64_t)row * K + col + e] : 0.f;
+                if (GPTAQ) dp[e] = in ? Pb[(int64_t)row * K + col + e] : 0.f;
+            }
+        }
     }
-#pragma unroll 8
-    for (int r = 0; r < SW_CH; ++r) {
-        const bool in = r < nvalid && tid < bs;
-        Wt[tid * SW_WLD + r] = in ? Wk[(int64_t)(n0 + r) * K + i0 + tid] : 0.f;
+    if (tid < bs) rpiv[tid] = 1.f / __ldg(Ub + (int64_t)tid * K + tid);
+
+    // this lane's coordinates 32 b + 8 q + i of its channel
+    float w[4][8];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        const int c0 = 32 * b + 8 * q;
+        const float *src = Wk + n * K + i0 + c0;
+        if (valid && (vec & 1) && c0 + 8 <= bs) {
+            const float4 x0 = *reinterpret_cast<const float4 *>(src);
+            const float4 x1 = *reinterpret_cast<const float4 *>(src + 4);
+            w[b][0] = x0.x; w[b][1] = x0.y; w[b][2] = x0.z; w[b][3] = x0.w;
+            w[b][4] = x1.x; w[b][5] = x1.y; w[b][6] = x1.z; w[b][7] = x1.w;
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) w[b][i] = (valid && c0 + i < bs) ? src[i] : 0.f;
+        }
     }
-    __syncthreads();
-    // reciprocal pivots of the block (a multiply in the serial chain instead of a divide)
-    float *rpiv = reinterpret_cast<float *>(Cs + SW_MAXB * SW_CLD);
-    if (tid < bs) rpiv[tid] = 1.f / Us[tid * SW_ULD + tid];
+    cp_async_wait_all();
     __syncthreads();
 
-    const float s = tid < nvalid ? scale[n] : 1.f;
+    const float s = valid ? scale[n] : 1.f;
     const float rs = 1.f / s;
     const float zf = (float)(1 << (bits - 1));
-    const float maxq = (float)((1 << bits) - 1);
+    const float cmin = -zf, cmax = (float)((1 << bits) - 1) - zf;
+    const int gsrc = lane & ~3;
     float lacc = 0.f;
+    uint8_t *crow = Cs + ch * CLD;
+    const int64_t ecol = (int64_t)grp * ldG + cta_ch0 + ch;
 
-    const int nsb = (bs + 31) / 32;
-    for (int sb = 0; sb < nsb; ++sb) {
-        const int jb = sb * 32;
-        float w[32], e[32], wp[32];
-#pragma unroll
-        for (int t = 0; t < 32; ++t) w[t] = Wt[(jb + t) * SW_WLD + tid];
+#pragma unroll 1
+    for (int p = 0; p < nsb; ++p) {
+        const int bbase = p * 4 - p * (p - 1) / 2;       // block (p, p)
+        int64_t eoff = (int64_t)(erow0 + 32 * p) * ldE + ecol;
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
-            const int j = jb + t;
-            e[t] = 0.f;
-            wp[t] = 0.f;
-            if (j < bs) {
-                const float wj = w[t];
-                const float c = fminf(fmaxf(rintf(wj * rs) + zf, 0.f), maxq);
-                const float q = s * (c - zf);
-                const float ej = (wj - q) * rpiv[j];
-                e[t] = ej;
-                wp[t] = wj;
+            const int j = 32 * p + t;
+            const int oq = t >> 3, oi = t & 7;
+            const bool live = j < bs;
+            const float wj = w[0][oi];
+            const float cf = fminf(fmaxf(rintf(wj * rs), cmin), cmax);
+            const float ej = live ? fmaf(-s, cf, wj) * rpiv[j] : 0.f;
+            const float e = __shfl_sync(0xffffffffu, ej, gsrc | oq);
+            float v = 0.f;
+            if (GPTAQ) v = __shfl_sync(0xffffffffu, live ? wj : 0.f, gsrc | oq);
+            if (q == oq && live) {
                 lacc = fmaf(ej, ej, lacc);
-                Cs[j * SW_CLD + tid] = (uint8_t)c;
-                if (tid < nvalid) {
-                    const int64_t e = (int64_t)(erow0 + j) * ldE + ecol;
+                crow[j] = (uint8_t)(int)(cf + zf);
+                if (valid) {
                     const __nv_bfloat16 eh = __float2bfloat16_rn(ej);
-                    Eh[e] = eh;
-                    El[e] = __float2bfloat16_rn(ej - __bfloat162float(eh));
+                    Eh[eoff] = eh;
+                    El[eoff] = __float2bfloat16_rn(ej - __bfloat162float(eh));
                     if (GPTAQ) {
                         const __nv_bfloat16 ph = __float2bfloat16_rn(wj);
-                        Ph[e] = ph;
-                        Pl[e] = __float2bfloat16_rn(wj - __bfloat162float(ph));
+                        Ph[eoff] = ph;
+                        Pl[eoff] = __float2bfloat16_rn(wj - __bfloat162float(ph));
                     }
                 }
+            }
+            eoff += ldE;
 #pragma unroll
-                for (int q4 = 0; q4 < 8; ++q4) {
-                    if (4 * q4 + 3 > t) {
-                        const float4 u = *reinterpret_cast<const float4 *>(&Us[j * SW_ULD + jb + 4 * q4]);
-                        const float uu[4] = {u.x, u.y, u.z, u.w};
-                        float pp[4] = {0.f, 0.f, 0.f, 0.f};
-                        if (GPTAQ) {
-                            const float4 p4 = *reinterpret_cast<const float4 *>(&Ps[j * SW_ULD + jb + 4 * q4]);
-                            pp[0] = p4.x; pp[1] = p4.y; pp[2] = p4.z; pp[3] = p4.w;
-                        }
-#pragma unroll
-                        for (int r = 0; r < 4; ++r) {
-                            const int ui = 4 * q4 + r;
-                            if (ui > t) {
-                                w[ui] = fmaf(-ej, uu[r], w[ui]);
-                                if (GPTAQ) w[ui] = fmaf(wj, pp[r], w[ui]);
-                            }
-                        }
-                    }
+            for (int b = 0; b < 4; ++b) {
+                if (b > 0 && p + b >= nsb) break;
+                const float *ur = Us + (bbase + b) * 1024 + t * 32 + 8 * q;
+                const float4 u0 = *reinterpret_cast<const float4 *>(ur);
+                const float4 u1 = *reinterpret_cast<const float4 *>(ur + 4);
+                w[b][0] = fmaf(-e, u0.x, w[b][0]); w[b][1] = fmaf(-e, u0.y, w[b][1]);
+                w[b][2] = fmaf(-e, u0.z, w[b][2]); w[b][3] = fmaf(-e, u0.w, w[b][3]);
+                w[b][4] = fmaf(-e, u1.x, w[b][4]); w[b][5] = fmaf(-e, u1.y, w[b][5]);
+                w[b][6] = fmaf(-e, u1.z, w[b][6]); w[b][7] = fmaf(-e, u1.w, w[b][7]);
+                if (GPTAQ) {
+                    const float *pr = Ps + (bbase + b) * 1024 + t * 32 + 8 * q;
+                    const float4 p0 = *reinterpret_cast<const float4 *>(pr);
+                    const float4 p1 = *reinterpret_cast<const float4 *>(pr + 4);
+                    w[b][0] = fmaf(v, p0.x, w[b][0]); w[b][1] = fmaf(v, p0.y, w[b][1]);
+                    w[b][2] = fmaf(v, p0.z, w[b][2]); w[b][3] = fmaf(v, p0.w, w[b][3]);
+                    w[b][4] = fmaf(v, p1.x, w[b][4]); w[b][5] = fmaf(v, p1.y, w[b][5]);
+                    w[b][6] = fmaf(v, p1.z, w[b][6]); w[b][7] = fmaf(v, p1.w, w[b][7]);
                 }
             }
         }
-        // later coordinates of this block: 4 at a time
-        for (int k = jb + 32; k < bs; k += 4) {
-            float a0 = Wt[(k + 0) * SW_WLD + tid], a1 = Wt[(k + 1) * SW_WLD + tid];
-            float a2 = Wt[(k + 2) * SW_WLD + tid], a3 = Wt[(k + 3) * SW_WLD + tid];
+        // the next sub-block becomes w[0]
 #pragma unroll
-            for (int t = 0; t < 32; ++t) {
-                const float4 u = *reinterpret_cast<const float4 *>(&Us[(jb + t) * SW_ULD + k]);
-                a0 = fmaf(-e[t], u.x, a0); a1 = fmaf(-e[t], u.y, a1);
-                a2 = fmaf(-e[t], u.z, a2); a3 = fmaf(-e[t], u.w, a3);
-                if (GPTAQ) {
-                    const float4 p4 = *reinterpret_cast<const float4 *>(&Ps[(jb + t) * SW_ULD + k]);
-                    a0 = fmaf(wp[t], p4.x, a0); a1 = fmaf(wp[t], p4.y, a1);
-                    a2 = fmaf(wp[t], p4.z, a2); a3 = fmaf(wp[t], p4.w, a3);
-                }
-            }
-            Wt[(k + 0) * SW_WLD + tid] = a0; Wt[(k + 1) * SW_WLD + tid] = a1;
-            Wt[(k + 2) * SW_WLD + tid] = a2; Wt[(k + 3) * SW_WLD + tid] = a3;
+        for (int b = 0; b < 3; ++b)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) w[b][i] = w[b + 1][i];
+    }
+    lacc += __shfl_xor_sync(0xffffffffu, lacc, 1);
+    lacc += __shfl_xor_sync(0xffffffffu, lacc, 2);
+    if (q == 0 && valid) loss_acc[n] += lacc;
+    __syncthreads();
+    // codes: 16-byte chunks of each channel's block row
+    const bool vecC = vec & 2;   // code rows 16-byte aligned
+    for (int idx = tid; idx < NCH * (SW_MAXB / 16); idx += 128) {
+        const int r = idx >> 3, c16 = (idx & 7) * 16;
+        if (r >= nvalid || c16 >= bs) continue;
+        uint8_t *dst = codes + ((int64_t)n0 + r) * K + i0 + c16;
+        const uint32_t *srcw = reinterpret_cast<const uint32_t *>(Cs + r * CLD + c16);
+        if (vecC && c16 + 16 <= bs) {
+            *reinterpret_cast<uint4 *>(dst) = make_uint4(srcw[0], srcw[1], srcw[2], srcw[3]);
+        } else {
+            for (int e = 0; e < 16 && c16 + e < bs; ++e) dst[e] = Cs[r * CLD + c16 + e];
         }
     }
-    if (tid < nvalid) loss_acc[n] += lacc;
-    __syncthreads();
-    for (int r = 0; r < nvalid; ++r)
-        if (tid < bs) codes[(int64_t)(n0 + r) * K + i0 + tid] = Cs[tid * SW_CLD + r];
 }
 
+// One CTA per channel: write-back s (c - z) in the weights' dtype and the loss.
 template <typename T>
-__global__ void k_finalize(T *W, const uint8_t *codes, const float *scale, int N, int K,
-                           int bits, int write_back, const float *loss_acc, float *loss) {
-    const int n = blockIdx.y;
-    const int64_t row = (int64_t)n * K;
+__global__ void __launch_bounds__(256) k_finalize(T *__restrict__ W, const uint8_t *__restrict__ codes,
+                                                  const float *__restrict__ scale, int K, int bits,
+                                                  int write_back, const float *__restrict__ loss_acc,
+                                                  float *__restrict__ loss, int vec) {
+    const int n = blockIdx.x;
     const float zf = (float)(1 << (bits - 1));
     const float s = scale[n];
-    for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < K; k += gridDim.x * blockDim.x) {
-        if (write_back) W[row + k] = from_f32<T>(s * ((float)codes[row + k] - zf));
-        if (loss && k == 0) loss[n] = 0.5f * loss_acc[n];
+    if (loss && threadIdx.x == 0) loss[n] = 0.5f * loss_acc[n];
+    if (!write_back) return;
+    T *wr = W + (int64_t)n * K;
+    const uint8_t *cr = codes + (int64_t)n * K;
+    if (vec) {   // W and code rows 16-byte aligned, K % 16 == 0
+        for (int k = threadIdx.x * 16; k < K; k += 256 * 16) {
+            const uint4 c = *reinterpret_cast<const uint4 *>(cr + k);
+            const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+            float x[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) x[i] = s * ((float)((cw[i >> 2] >> (8 * (i & 3))) & 0xffu) - zf);
+            if constexpr (sizeof(T) == 2) {
+                uint32_t o[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+                    o[i] = *reinterpret_cast<const uint32_t *>(&h);
+                }
+                *reinterpret_cast<uint4 *>(wr + k) = make_uint4(o[0], o[1], o[2], o[3]);
+                *reinterpret_cast<uint4 *>(wr + k + 8) = make_uint4(o[4], o[5], o[6], o[7]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    *reinterpret_cast<float4 *>(reinterpret_cast<float *>(wr) + k + 4 * i) =
+                        make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+            }
+        }
+    } else {
+        for (int k = threadIdx.x; k < K; k += 256) wr[k] = from_f32<T>(s * ((float)cr[k] - zf));
     }
 }
 
@@ -248,9 +362,7 @@ size_t quantize_workspace(int K, int N, int g, int blocksize) {
 }
 
 static size_t sweep_smem(bool gptaq) {
-    return (size_t)SW_MAXB * SW_ULD * sizeof(float) * (gptaq ? 2 : 1) +
-           (size_t)SW_MAXB * SW_WLD * sizeof(float) + (size_t)SW_MAXB * SW_CLD +
-           SW_MAXB * sizeof(float);
+    return sizeof(float) * (10 * 1024 * (gptaq ? 2 : 1) + 32 * 33 + SW_MAXB);
 }
 
 gptq_status quantize_layer(void *W, int wdtype, int N, int K, const float *U, int groups, int bits,
@@ -274,19 +386,18 @@ gptq_status quantize_layer(void *W, int wdtype, int N, int K, const float *U, in
     const int per_group = N / groups;
     const int64_t KK = (int64_t)K * K;
     const bool gptaq = P1 != nullptr;
-    const int rowgrid = std::min(8, (K + 255) / 256);
-
-    k_scale<<<(N * 32 + 255) / 256, 256, 0, st>>>(W, wdtype, N, K, bits, scales_in, scale,
-                                                   scales_out, status);
+    const int vin = (K % 8 == 0 && aligned(W, 16) && aligned(Wk, 16)) ? 1 : 0;
+    const int vfin = (K % 16 == 0 && aligned(W, 16) && aligned(codes, 16)) ? 1 : 0;
+    if (wdtype == GPTQ_F32)
+        k_scale_init<float><<<N, 256, 0, st>>>(static_cast<const float *>(W), Wk, K, per_group, bits,
+                                              dead, scales_in, scale, scales_out, loss_acc, vin,
+                                              status);
+    else
+        k_scale_init<__nv_bfloat16><<<N, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(W), Wk, K,
+                                                      per_group, bits, dead, scales_in, scale,
+                                                      scales_out, loss_acc, vin, status);
     gptq_status s = launch_status();
     if (s != GPTQ_OK) return s;
-    if (wdtype == GPTQ_F32)
-        k_init_work<float><<<dim3(rowgrid, N), 256, 0, st>>>(static_cast<const float *>(W), Wk, N,
-                                                            K, per_group, dead, loss_acc);
-    else
-        k_init_work<__nv_bfloat16><<<dim3(rowgrid, N), 256, 0, st>>>(
-            static_cast<const __nv_bfloat16 *>(W), Wk, N, K, per_group, dead, loss_acc);
-    if ((s = launch_status()) != GPTQ_OK) return s;
     if ((s = split_bf16(U, K, K, K, Uh, Ul, lay.ldU, groups, KK, (int64_t)K * lay.ldU, st)) != GPTQ_OK)
         return s;
     if (gptaq && (s = split_bf16(P1, K, K, K, Qh, Ql, lay.ldU, 1, 0, 0, st)) != GPTQ_OK) return s;
@@ -315,34 +426,28 @@ gptq_status quantize_layer(void *W, int wdtype, int N, int K, const float *U, in
     base.vec4 = (K % 4 == 0);
     base.status = status;
     // -E (hi*hi + hi*lo + lo*hi) U, and for GPTAQ +W_pre (same splits) P1
-    const int terms[6][3] = {{0, 0, 1}, {0, 1, 1}, {1, 0, 1}, {2, 2, 0}, {2, 3, 0}, {3, 2, 0}};
-    base.nterms = gptaq ? 6 : 3;
-    for (int t = 0; t < base.nterms; ++t) {
-        base.a_id[t] = terms[t][0];
-        base.b_id[t] = terms[t][1];
-        base.neg[t] = terms[t][2];
-    }
+    base.ngroups = gptaq ? 2 : 1;
+    base.neg[0] = 1;
+    base.neg[1] = 0;
 
+    const dim3 grid((per_group + 31) / 32, groups);
+    auto kern = gptaq ? k_sweep_block<true> : k_sweep_block<false>;
     const size_t smem = sweep_smem(gptaq);
-    if (gptaq)
-        cudaFuncSetAttribute(k_sweep_block<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    else
-        cudaFuncSetAttribute(k_sweep_block<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    const dim3 grid((per_group + SW_CH - 1) / SW_CH, groups);
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return launch_status();
+    const int vec = ((K % 4 == 0 && aligned(U, 16) && (!gptaq || aligned(P1, 16))) ? 1 : 0) |
+                    ((K % 16 == 0 && aligned(codes, 16)) ? 2 : 0);
     for (int sb0 = 0; sb0 < K; sb0 += SUPER) {
         const int sb1 = min(K, sb0 + SUPER);
         for (int i0 = sb0; i0 < sb1; i0 += blocksize) {
             const int i1 = min(i0 + blocksize, sb1);
             const int bs = i1 - i0;
-            if (gptaq)
-                k_sweep_block<true><<<grid, SW_CH, smem, st>>>(
-                    Wk, N, per_group, K, i0, bs, U, P1, scale, bits, codes, Eh, El, Ph, Pl,
-                    lay.ldE, lay.ldG, i0 - sb0, loss_acc, status);
-            else
-                k_sweep_block<false><<<grid, SW_CH, smem, st>>>(
-                    Wk, N, per_group, K, i0, bs, U, P1, scale, bits, codes, Eh, El, Ph, Pl,
-                    lay.ldE, lay.ldG, i0 - sb0, loss_acc, status);
-            if ((s = launch_status()) != GPTQ_OK) return s;
+            kern<<<grid, 128, smem, st>>>(Wk, N, per_group, K, i0, bs, U, P1, scale, bits,
+                                                codes, Eh, El, Ph, Pl, lay.ldE, lay.ldG, i0 - sb0,
+                                                loss_acc, vec, status);
+            s = launch_status();
+            if (s != GPTQ_OK) return s;
             if (i1 >= sb1) continue;
             for (int gi = 0; gi < groups; ++gi) {      // near: the rest of the super-block
                 UpdateParams p = base;
@@ -372,11 +477,11 @@ gptq_status quantize_layer(void *W, int wdtype, int N, int K, const float *U, in
         }
     }
     if (wdtype == GPTQ_F32)
-        k_finalize<float><<<dim3(rowgrid, N), 256, 0, st>>>(static_cast<float *>(W), codes, scale,
-                                                           N, K, bits, write_back, loss_acc, loss);
+        k_finalize<float><<<N, 256, 0, st>>>(static_cast<float *>(W), codes, scale, K, bits,
+                                             write_back, loss_acc, loss, vfin);
     else
-        k_finalize<__nv_bfloat16><<<dim3(rowgrid, N), 256, 0, st>>>(
-            static_cast<__nv_bfloat16 *>(W), codes, scale, N, K, bits, write_back, loss_acc, loss);
+        k_finalize<__nv_bfloat16><<<N, 256, 0, st>>>(static_cast<__nv_bfloat16 *>(W), codes, scale, K,
+                                                     bits, write_back, loss_acc, loss, vfin);
     return launch_status();
 }
 

@@ -1,5 +1,5 @@
 // Tensor-core lazy update of the far coordinates (tcgen05, TMA):
-//   C[n][k] += sum_t sign_t * sum_j A_t[j][n] * B_t[j][k]
+//   C[n][k] += sum_g sign_g * sum_j A_g[j][n] * B_g[j][k]
 // over j in a block (or super-block) of already-quantised coordinates.
 //
 // [GPTQ blog] "GPTQ 怎样把逐个补偿变成可扩展算法": after a block of B coordinates the
@@ -9,11 +9,17 @@
 // Operands are fp32 values carried as bf16 pairs x = hi + lo; three products
 // hi*hi + hi*lo + lo*hi keep about 16 bits of each factor (the dropped lo*lo term
 // is ~2^-18 relative), accumulated in fp32 in TMEM. Both operands are MN-major
-// (rows j, the n or k index contiguous), loaded as 64-wide x 16-row boxes with the
-// 128-byte swizzle: LBO = one box (2 KB), SBO = 8 rows (1 KB).
+// (rows j, the n or k index contiguous), loaded as 64-wide boxes with the 128-byte
+// swizzle: LBO = one box, SBO = 8 rows (1 KB). One pipeline stage holds the hi and
+// lo tiles of both operands for one k-step of one product group (E with U, or the
+// pre-rounding weights with P1), so each tile is loaded once for its three MMAs.
 //
-// One CTA per 128 x 256 output tile (two CTAs fit on an SM): warp 0 issues TMA,
-// warp 1 owns TMEM and issues the MMAs, warps 2-5 read TMEM and update C in place.
+// Persistent CTAs over 128 x 256 output tiles: warp 0 issues TMA, warp 1 owns TMEM
+// and issues the MMAs, warps 2-5 drain the double-buffered TMEM accumulator. The
+// epilogue adds into C with TMA tensor reductions (fp32 add performed in L2 on whole
+// lines): each epilogue warp stages its 32 rows x 32 columns in a swizzled
+// shared-memory buffer and issues one bulk reduction per chunk. Rows that are not
+// 16-byte aligned fall back to per-thread vector reductions.
 #include <cuda.h>
 
 #include <algorithm>
@@ -27,27 +33,27 @@ namespace gptq {
 namespace {
 constexpr int UT_BM = 128, UT_BN = 256;
 constexpr int UT_RING = 192 * 1024;                   // shared-memory ring for all stages
-constexpr int UT_SMEM = UT_RING + 1024 + 512;   // ring + alignment + barriers
+constexpr int UT_EPI = 4 * 2 * 32 * 32 * 4;           // 4 warps x 2 buffers x 32 x 32 fp32
+constexpr int UT_SMEM = UT_RING + UT_EPI + 1024 + 512;  // + alignment + barriers
 constexpr int UT_THREADS = 192;
 constexpr uint32_t UT_TMEM_COLS = 512;                // two 256-column accumulators
 }  // namespace
 
-// Persistent: tiles (row tile fastest, so CTAs running together share the B rows)
-// are dealt round-robin; each tile runs every term over the inner rows, then the
-// epilogue adds the TMEM accumulator into C with vector reductions while the MMA
-// warp already fills the other accumulator.
-template <int BK>
+template <int BK, bool TMA_EPI>
 __global__ void __launch_bounds__(UT_THREADS, 1)
-    k_update_tc(const __grid_constant__ UpdateMaps maps, const UpdateParams p) {
-    constexpr int BOX = 64 * BK * 2;
-    constexpr int A_BYTES = UT_BM * BK * 2;
-    constexpr int STAGE = A_BYTES + UT_BN * BK * 2;
+    k_update_tc(const __grid_constant__ UpdateMaps maps, const __grid_constant__ CUtensorMap cmap,
+                const UpdateParams p) {
+    constexpr int BOX = 64 * BK * 2;                  // one 64-wide box of BK rows
+    constexpr int A_BYTES = UT_BM * BK * 2;           // 2 boxes
+    constexpr int B_BYTES = UT_BN * BK * 2;           // 4 boxes
+    constexpr int STAGE = 2 * A_BYTES + 2 * B_BYTES;  // A hi, A lo, B hi, B lo
     constexpr int STAGES = UT_RING / STAGE;
     if (failed(p.status)) return;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + UT_RING);
+    uint8_t *epi = smem + UT_RING;                    // 1 KB aligned
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + UT_RING + UT_EPI);
     uint64_t *empty = full + STAGES;
     uint64_t *tfull = empty + STAGES;
     uint64_t *tempty = tfull + 2;
@@ -60,7 +66,7 @@ __global__ void __launch_bounds__(UT_THREADS, 1)
     const int nm = (p.M + UT_BM - 1) / UT_BM;
     const int tiles = nm * ((p.Ncols + UT_BN - 1) / UT_BN);
     const int ksteps = p.L / BK;
-    const int per_tile = ksteps * p.nterms;
+    const int per_tile = ksteps * p.ngroups;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -86,22 +92,27 @@ __global__ void __launch_bounds__(UT_THREADS, 1)
         if (lane == 0) {
             int stage = 0, issued = 0;
             uint32_t phase = 0;
+            const int a_x0 = p.a_x0, a_y0 = p.a_y0, b_x0 = p.b_x0, b_y0 = p.b_y0;
             for (int tile = blockIdx.x; tile < tiles && !*abort; tile += gridDim.x) {
                 const int row0 = (tile % nm) * UT_BM, col0 = (tile / nm) * UT_BN;
                 for (int it = 0; it < per_tile; ++it) {
-                    const int t = it / ksteps, ks = it - t * ksteps;
+                    const int g = it / ksteps, ks = it - g * ksteps;
                     if (!tc::mbar_wait(&empty[stage], phase ^ 1, abort)) break;
                     tc::mbar_arrive_expect_tx(&full[stage], STAGE);
-                    uint8_t *a = smem + stage * STAGE;
-                    uint8_t *b = a + A_BYTES;
-                    const CUtensorMap *am = &maps.a[p.a_id[t]];
-                    const CUtensorMap *bm = &maps.b[p.b_id[t]];
-                    const int ay = p.a_y0 + ks * BK, by = p.b_y0 + ks * BK;
-                    tc::tma_load_2d(a, am, &full[stage], p.a_x0 + row0, ay);
-                    tc::tma_load_2d(a + BOX, am, &full[stage], p.a_x0 + row0 + 64, ay);
+                    uint8_t *st = smem + stage * STAGE;
+                    const int ay = a_y0 + ks * BK, by = b_y0 + ks * BK;
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        tc::tma_load_2d(b + q * BOX, bm, &full[stage], p.b_x0 + col0 + 64 * q, by);
+                    for (int h = 0; h < 2; ++h) {       // hi, lo
+                        const CUtensorMap *am = &maps.a[2 * g + h];
+                        const CUtensorMap *bm = &maps.b[2 * g + h];
+                        uint8_t *a = st + h * A_BYTES;
+                        uint8_t *b = st + 2 * A_BYTES + h * B_BYTES;
+                        tc::tma_load_2d(a, am, &full[stage], a_x0 + row0, ay);
+                        tc::tma_load_2d(a + BOX, am, &full[stage], a_x0 + row0 + 64, ay);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            tc::tma_load_2d(b + q * BOX, bm, &full[stage], b_x0 + col0 + 64 * q, by);
+                    }
                     ++issued;
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
@@ -117,6 +128,7 @@ __global__ void __launch_bounds__(UT_THREADS, 1)
         if (lane == 0) {
             const uint32_t idesc_pos = tc::idesc_bf16_f32(UT_BM, UT_BN, 1, 1, 0);
             const uint32_t idesc_neg = tc::idesc_bf16_f32(UT_BM, UT_BN, 1, 1, 1);
+            const bool neg0 = p.neg[0] != 0, neg1 = p.neg[1] != 0;
             int stage = 0, n = 0, acc = 0;
             uint32_t phase = 0, acc_phase = 0;
             for (int tile = blockIdx.x; tile < tiles && !*abort; tile += gridDim.x) {
@@ -125,16 +137,20 @@ __global__ void __launch_bounds__(UT_THREADS, 1)
                 const uint32_t d = tmem + acc * UT_BN;
                 bool ok = true;
                 for (int it = 0; it < per_tile; ++it) {
-                    const int t = it / ksteps;
+                    const int g = it / ksteps;
                     if (!tc::mbar_wait(&full[stage], phase, abort)) { ok = false; break; }
                     tc::fence_after_sync();
-                    const uint32_t sa = tc::smem_u32(smem + stage * STAGE);
-                    const uint32_t idesc = p.neg[t] ? idesc_neg : idesc_pos;
+                    const uint32_t s0 = tc::smem_u32(smem + stage * STAGE);
+                    const uint32_t idesc = (g ? neg1 : neg0) ? idesc_neg : idesc_pos;
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
-                        const uint64_t ad = tc::desc_sw128(sa + kk * 2048, BOX, 1024);
-                        const uint64_t bd = tc::desc_sw128(sa + A_BYTES + kk * 2048, BOX, 1024);
-                        tc::mma_bf16(d, ad, bd, idesc, (it > 0 || kk > 0) ? 1u : 0u);
+                        const uint64_t ah = tc::desc_sw128(s0 + kk * 2048, BOX, 1024);
+                        const uint64_t al = tc::desc_sw128(s0 + A_BYTES + kk * 2048, BOX, 1024);
+                        const uint64_t bh = tc::desc_sw128(s0 + 2 * A_BYTES + kk * 2048, BOX, 1024);
+                        const uint64_t bl = tc::desc_sw128(s0 + 2 * A_BYTES + B_BYTES + kk * 2048, BOX, 1024);
+                        tc::mma_bf16(d, ah, bh, idesc, (it > 0 || kk > 0) ? 1u : 0u);
+                        tc::mma_bf16(d, ah, bl, idesc, 1u);
+                        tc::mma_bf16(d, al, bh, idesc, 1u);
                     }
                     tc::mma_commit(&empty[stage]);
                     *reinterpret_cast<volatile int *>(consumed) = ++n;
@@ -150,39 +166,65 @@ __global__ void __launch_bounds__(UT_THREADS, 1)
         }
     } else {
         const int quad = warp & 3;
-        int acc = 0;
+        int acc = 0, nbuf = 0;
         uint32_t acc_phase = 0;
+        uint8_t *mybuf = epi + (warp - 2) * 2 * 4096;
+        float *const C = p.C;
+        const int64_t ldc = p.ldc;
+        const int M = p.M, Ncols = p.Ncols;
+        const bool vec4 = p.vec4;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
             const int row0 = (tile % nm) * UT_BM, col0 = (tile / nm) * UT_BN;
             if (!tc::mbar_wait(&tfull[acc], acc_phase, abort)) break;
             tc::fence_after_sync();
             const int r = row0 + quad * 32 + lane;
-            float *crow = p.C + (int64_t)r * p.ldc;
 #pragma unroll 1
             for (int c = 0; c < UT_BN / 32; ++c) {
                 uint32_t v[32];
                 tc::tmem_ld_32x32b_x32(tmem + acc * UT_BN + c * 32 + ((uint32_t)(quad * 32) << 16), v);
                 tc::tmem_ld_wait();
                 const int cb = col0 + c * 32;
-                if (r >= p.M || cb >= p.Ncols) continue;
-                if (p.vec4 && cb + 32 <= p.Ncols) {
+                if (TMA_EPI) {
+                    if (row0 + quad * 32 >= M || cb >= Ncols) continue;    // warp-uniform
+                    uint8_t *buf = mybuf + (nbuf & 1) * 4096;
+                    if (lane == 0) tc::bulk_wait_read<1>();   // the reduction that used buf is done reading
+                    __syncwarp();
+                    // row = lane, 16-byte chunk q stored at chunk q ^ (row & 7) (128-byte swizzle)
 #pragma unroll
                     for (int q = 0; q < 8; ++q)
-                        atomicAdd(reinterpret_cast<float4 *>(crow + cb + 4 * q),
-                                  make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
-                                              __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])));
+                        *reinterpret_cast<uint4 *>(buf + lane * 128 + ((q ^ (lane & 7)) << 4)) =
+                            make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                    tc::fence_async_shared();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tc::tma_reduce_add_2d(&cmap, buf, cb, row0 + quad * 32);
+                        tc::bulk_commit();
+                    }
+                    ++nbuf;
                 } else {
+                    if (r >= M || cb >= Ncols) continue;
+                    float *crow = C + (int64_t)r * ldc;
+                    if (vec4 && cb + 32 <= Ncols) {
 #pragma unroll
-                    for (int q = 0; q < 32; ++q)
-                        if (cb + q < p.Ncols) atomicAdd(crow + cb + q, __uint_as_float(v[q]));
+                        for (int q = 0; q < 8; ++q)
+                            atomicAdd(reinterpret_cast<float4 *>(crow + cb + 4 * q),
+                                      make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                                  __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])));
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 32; ++q)
+                            if (cb + q < Ncols) atomicAdd(crow + cb + q, __uint_as_float(v[q]));
+                    }
                 }
             }
             tc::fence_before_sync();
             tc::mbar_arrive(&tempty[acc]);
             if (++acc == 2) { acc = 0; acc_phase ^= 1; }
         }
+        if (TMA_EPI && lane == 0) tc::bulk_wait_all();
     }
 
+    __syncwarp();   // each role warp reconverges before the block barrier
     tc::fence_before_sync();
     __syncthreads();
     if (*abort && threadIdx.x == 0) set_status(p.status, GPTQ_ERR_TIMEOUT);
@@ -231,6 +273,21 @@ gptq_status make_bf16_map(CUtensorMap *m, const void *base, int64_t cols, int64_
     return r == CUDA_SUCCESS ? GPTQ_OK : GPTQ_ERR_CUDA;
 }
 
+// The output C [M][ldc] fp32 as 32 x 32 boxes with the 128-byte swizzle (the target of
+// the epilogue's bulk reductions).
+static gptq_status make_out_map(CUtensorMap *m, float *C, int64_t cols, int64_t rows, int64_t ld) {
+    EncodeTiledFn enc = update_encode_fn();
+    if (!enc) return GPTQ_ERR_CUDA;
+    const cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t gstride[1] = {(cuuint64_t)ld * 4};
+    const cuuint32_t box[2] = {32, 32};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, C, gdim, gstride, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? GPTQ_OK : GPTQ_ERR_CUDA;
+}
+
 static int update_sms() {
     int dev = 0, n = 0;
     cudaGetDevice(&dev);
@@ -238,32 +295,69 @@ static int update_sms() {
     return n > 0 ? n : 148;
 }
 
+template <int BK, bool TMA_EPI>
+static gptq_status launch_update(const UpdateMaps &maps, const CUtensorMap &cmap,
+                                 const UpdateParams &p, int grid, cudaStream_t st) {
+    cudaFuncSetAttribute(k_update_tc<BK, TMA_EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, UT_SMEM);
+    k_update_tc<BK, TMA_EPI><<<grid, UT_THREADS, UT_SMEM, st>>>(maps, cmap, p);
+    return launch_status();
+}
+
 // box_rows of the maps must equal the kernel's BK: 64 when L % 64 == 0, else 16.
 gptq_status launch_update_tc(const UpdateMaps &maps, const UpdateParams &p, int box_rows,
                              cudaStream_t st) {
     if (p.M <= 0 || p.Ncols <= 0 || p.L <= 0) return GPTQ_OK;
-    if (p.L % box_rows != 0) return GPTQ_ERR_ARG;
+    if (p.L % box_rows != 0 || p.ngroups < 1 || p.ngroups > 2) return GPTQ_ERR_ARG;
     const int tiles = ((p.M + UT_BM - 1) / UT_BM) * ((p.Ncols + UT_BN - 1) / UT_BN);
     const int grid = std::min(tiles, update_sms());
-    if (box_rows == 64) {
-        cudaFuncSetAttribute(k_update_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, UT_SMEM);
-        k_update_tc<64><<<grid, UT_THREADS, UT_SMEM, st>>>(maps, p);
-    } else {
-        cudaFuncSetAttribute(k_update_tc<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, UT_SMEM);
-        k_update_tc<16><<<grid, UT_THREADS, UT_SMEM, st>>>(maps, p);
-    }
-    return launch_status();
+    // bulk reductions need a 16-byte aligned base and row pitch
+    CUtensorMap cmap;
+    const bool tma_epi = (p.ldc % 4 == 0) && aligned(p.C, 16) &&
+                         make_out_map(&cmap, p.C, p.Ncols, p.M, p.ldc) == GPTQ_OK;
+    if (!tma_epi) memset(&cmap, 0, sizeof(cmap));
+    if (box_rows == 64)
+        return tma_epi ? launch_update<64, true>(maps, cmap, p, grid, st)
+                       : launch_update<64, false>(maps, cmap, p, grid, st);
+    return tma_epi ? launch_update<16, true>(maps, cmap, p, grid, st)
+                   : launch_update<16, false>(maps, cmap, p, grid, st);
 }
 
 // x -> (hi, lo) with hi = bf16(x), lo = bf16(x - hi); rows x cols fp32 (ld_in) to bf16
-// pairs (ld_out, padded columns written as zero). One grid row per matrix row.
+// pairs (ld_out, padded columns written as zero). One grid row per matrix row; eight
+// columns per thread when the rows are 16-byte aligned.
 __global__ void k_split_bf16(const float *__restrict__ in, int64_t ld_in, int cols,
                              __nv_bfloat16 *__restrict__ hi, __nv_bfloat16 *__restrict__ lo,
-                             int64_t ld_out, int64_t batch_in, int64_t batch_out) {
+                             int64_t ld_out, int64_t batch_in, int64_t batch_out, int vec) {
     const int64_t r = blockIdx.y;
     in += blockIdx.z * batch_in + r * ld_in;
     hi += blockIdx.z * batch_out + r * ld_out;
     lo += blockIdx.z * batch_out + r * ld_out;
+    if (vec) {
+        for (int c = (blockIdx.x * blockDim.x + threadIdx.x) * 8; c < ld_out;
+             c += gridDim.x * blockDim.x * 8) {
+            float x[8];
+            if (c + 8 <= cols) {
+                const float4 a = *reinterpret_cast<const float4 *>(in + c);
+                const float4 b = *reinterpret_cast<const float4 *>(in + c + 4);
+                x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) x[i] = c + i < cols ? in[c + i] : 0.f;
+            }
+            uint32_t h[4], l[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const __nv_bfloat162 hh = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+                const float2 hf = __bfloat1622float2(hh);
+                const __nv_bfloat162 ll = __floats2bfloat162_rn(x[2 * i] - hf.x, x[2 * i + 1] - hf.y);
+                h[i] = *reinterpret_cast<const uint32_t *>(&hh);
+                l[i] = *reinterpret_cast<const uint32_t *>(&ll);
+            }
+            *reinterpret_cast<uint4 *>(hi + c) = make_uint4(h[0], h[1], h[2], h[3]);
+            *reinterpret_cast<uint4 *>(lo + c) = make_uint4(l[0], l[1], l[2], l[3]);
+        }
+        return;
+    }
     for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < ld_out; c += gridDim.x * blockDim.x) {
         const float x = c < cols ? in[c] : 0.f;
         const __nv_bfloat16 h = __float2bfloat16_rn(x);
@@ -275,9 +369,13 @@ __global__ void k_split_bf16(const float *__restrict__ in, int64_t ld_in, int co
 gptq_status split_bf16(const float *in, int64_t ld_in, int rows, int cols, __nv_bfloat16 *hi,
                        __nv_bfloat16 *lo, int64_t ld_out, int batch, int64_t batch_in,
                        int64_t batch_out, cudaStream_t st) {
-    const int bx = (int)std::min<int64_t>(8, (ld_out + 255) / 256);
+    const int vec = (ld_in % 4 == 0 && ld_out % 8 == 0 && batch_in % 4 == 0 && batch_out % 8 == 0 &&
+                     aligned(in, 16) && aligned(hi, 16) && aligned(lo, 16))
+                        ? 1
+                        : 0;
+    const int bx = (int)std::min<int64_t>(vec ? 2 : 8, (ld_out + 255) / 256);
     k_split_bf16<<<dim3(bx, rows, batch), 256, 0, st>>>(in, ld_in, cols, hi, lo, ld_out, batch_in,
-                                                        batch_out);
+                                                        batch_out, vec);
     return launch_status();
 }
 

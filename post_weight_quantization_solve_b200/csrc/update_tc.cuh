@@ -8,8 +8,8 @@
 
 namespace gptq {
 
-constexpr int UT_MAX_TERMS = 6;
-
+// Product group g uses A operands a[2g] (hi), a[2g+1] (lo) and B operands b[2g],
+// b[2g+1]: group 0 is E with U, group 1 (GPTAQ) the pre-rounding weights with P1.
 struct UpdateMaps {
     CUtensorMap a[4];   // A operands: [rows j][n], bf16
     CUtensorMap b[4];   // B operands: [rows j][k], bf16
@@ -21,8 +21,8 @@ struct UpdateParams {
     int M, Ncols, L;        // output rows, output columns, inner rows (multiple of 16)
     int a_x0, a_y0;         // A: column (n) origin, row (j) origin
     int b_x0, b_y0;         // B: column (k) origin, row (j) origin
-    int nterms;
-    int a_id[UT_MAX_TERMS], b_id[UT_MAX_TERMS], neg[UT_MAX_TERMS];
+    int ngroups;            // 1, or 2 with the GPTAQ group
+    int neg[2];             // subtract group g's product
     int vec4;               // C rows 16-byte aligned: float4 reductions
     int32_t *status;
 };
