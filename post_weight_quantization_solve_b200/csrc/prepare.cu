@@ -21,11 +21,13 @@
 #include <float.h>
 
 #include <algorithm>
+#include <mutex>
 #include <vector>
 
 #include "common.cuh"
 #include "gemm_simt.cuh"
 #include "gemm_tc32.cuh"
+#include "tc_ptx.cuh"
 
 namespace gptq {
 
@@ -72,17 +74,20 @@ __global__ void k_dead_damp(float *H, int K, float percdamp, uint8_t *dead_out, 
 }
 
 // Factor one diagonal block H[J,J] (J = [j0, j0+nb), nb <= 128) and replace it by
-// U_JJ. One CTA per group (256 threads), the block in shared memory, padded with
-// the identity beyond nb. H_JJ = L D L^T with L unit upper, built from the last
-// 32-wide sub-block Q to the first:
-//   - all threads factor C = S[Q,Q] = L_Q D_Q L_Q^T and invert V_Q = L_Q^-1, four
-//     register elements each, one published pivot column per barrier;
-//   - all threads: T = S[<Q, Q] V_Q^T, L[<Q, Q] = T D_Q^-1, and the trailing update
-//     S[<Q, <Q] -= L T^T (upper triangle).
-// Then V = L^-1 by block back-substitution, V_PQ = -V_PP sum_{P<R<=Q} L_PR V_RQ,
-// and U_JJ = R^-1 = D^-1/2 V with R = L D^1/2.
-constexpr int DG_T = 256;
-constexpr int DG_LD = CH_NB + 1;
+// U_JJ. One CTA per group; the block is padded with the identity beyond nb.
+// H_JJ = L D L^T with L unit upper, eliminated from the last pivot to the first,
+// and V = L^-1 built in the same pass: once pivot j is eliminated, column j of L
+// is final and so is row j of V (every later row has been applied to it), so
+//   S[i][k] -= S[i][j] S[k][j] / d_j        (i, k < j)
+//   V[i][c] -= (S[i][j] / d_j) V[j][c]      (i < j)
+// share one published column. Then U_JJ = R^-1 = D^-1/2 V with R = L D^1/2.
+// Each thread keeps a 4 x 8 tile of S and the same tile of V in registers; the 272
+// tiles that meet the upper triangle are dealt row-major, so a warp whose rows all
+// lie at or below pivot j skips the update. Column j of S, row j of V and d_j are
+// published into buffers of their own (no reuse), one barrier per pivot.
+constexpr int DG_TILES = 272;
+constexpr int DG_T = 288;
+constexpr int DG_N = CH_NB;
 
 __global__ void __launch_bounds__(DG_T, 1) k_chol_diag(float *H, int K, int j0, int nb,
                                                     const float *diag_d, float tol,
@@ -91,219 +96,127 @@ __global__ void __launch_bounds__(DG_T, 1) k_chol_diag(float *H, int K, int j0, 
     const int g = blockIdx.x;
     H += (int64_t)g * K * K;
     diag_d += (int64_t)g * K;
-    extern __shared__ float sm[];
-    float *S = sm;                          // [128][DG_LD]: L (strict upper), D (diagonal)
-    float *V = S + CH_NB * DG_LD;           // [128][DG_LD]: V = L^-1 (upper)
-    float *Ts = V + CH_NB * DG_LD;          // [96][33]: panel products
-    float *piv = Ts + 96 * 33;              // [128]
-    float *dref = piv + CH_NB;              // [128]
-    float *colb = dref + CH_NB;             // [2][32] published pivot column
-    float *rowb = colb + 64;                // [2][32] published row of V
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = DG_T / 32;
+    extern __shared__ __align__(16) float sm[];
+    float *colb = sm;                      // [128][128]: column j of S, rows < j
+    float *vrow = colb + DG_N * DG_N;      // [128][128]: row j of V
+    float *dpiv = vrow + DG_N * DG_N;      // [128]
+    float *rpiv = dpiv + DG_N;             // [128]
+    float *dref = rpiv + DG_N;             // [128]
+    const int tid = threadIdx.x;
 
-    // stage whole rows (only the upper triangle is ever read); identity padding
-    const bool vec = (K % 4 == 0) && (nb == CH_NB);
-    if (vec) {
-#pragma unroll 8
-        for (int it = 0; it < CH_NB * CH_NB / 4 / DG_T; ++it) {
-            const int idx = it * DG_T + tid, r = idx >> 5, c4 = (idx & 31) * 4;
-            const float4 x = *reinterpret_cast<const float4 *>(H + (int64_t)(j0 + r) * K + j0 + c4);
-            float *dst = S + r * DG_LD + c4;
-            dst[0] = x.x; dst[1] = x.y; dst[2] = x.z; dst[3] = x.w;
-        }
-    } else {
-#pragma unroll 8
-        for (int it = 0; it < CH_NB * CH_NB / DG_T; ++it) {
-            const int idx = it * DG_T + tid, r = idx >> 7, c = idx & 127;
-            S[r * DG_LD + c] = (r < nb && c < nb) ? H[(int64_t)(j0 + r) * K + j0 + c]
-                                                  : (r == c ? 1.f : 0.f);
+    // this thread's tile (ti, tk): rows 4 ti .. 4 ti + 3, columns 8 tk .. 8 tk + 7
+    int ti = 32, tk = 0;
+    if (tid < DG_TILES) {
+        int t = tid;
+        for (int r = 0; r < 32; ++r) {
+            const int cnt = 16 - (r >> 1);
+            if (t < cnt) { ti = r; tk = (r >> 1) + t; break; }
+            t -= cnt;
         }
     }
-    for (int idx = tid; idx < CH_NB * CH_NB; idx += DG_T) V[(idx >> 7) * DG_LD + (idx & 127)] = 0.f;
-    if (tid < CH_NB) dref[tid] = tid < nb ? diag_d[j0 + tid] : 1.f;
+    const int wrow0 = 4 * __shfl_sync(0xffffffffu, ti, 0);   // lowest row of this warp
+    const int i0 = 4 * ti, c0 = 8 * tk;
+
+    for (int idx = tid; idx < 2 * DG_N * DG_N / 4; idx += DG_T)
+        reinterpret_cast<float4 *>(colb)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (tid < DG_N) dref[tid] = tid < nb ? diag_d[j0 + tid] : 1.f;
+    // tiles entirely below the diagonal: zero in the output
+    for (int idx = tid; idx < DG_N * DG_N; idx += DG_T) {
+        const int r = idx >> 7, c = idx & 127;
+        if (r < nb && c < nb && (r >> 2) > 2 * (c >> 3) + 1) H[(int64_t)(j0 + r) * K + j0 + c] = 0.f;
+    }
+
+    float s[4][8], v[4][8];
+    const bool vec = (nb == DG_N) && (K % 4 == 0) && ((reinterpret_cast<uintptr_t>(H) & 15) == 0) &&
+                     (j0 % 4 == 0);
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const int i = i0 + r;
+        if (ti < 32 && vec) {
+            const float *src = H + (int64_t)(j0 + i) * K + j0 + c0;
+            const float4 x0 = *reinterpret_cast<const float4 *>(src);
+            const float4 x1 = *reinterpret_cast<const float4 *>(src + 4);
+            s[r][0] = x0.x; s[r][1] = x0.y; s[r][2] = x0.z; s[r][3] = x0.w;
+            s[r][4] = x1.x; s[r][5] = x1.y; s[r][6] = x1.z; s[r][7] = x1.w;
+        } else {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const int k = c0 + c;
+                s[r][c] = (i < nb && k < nb) ? H[(int64_t)(j0 + i) * K + j0 + k] : (i == k ? 1.f : 0.f);
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c) v[r][c] = (i == c0 + c) ? 1.f : 0.f;
+    }
     __syncthreads();
 
-    for (int q = 3; q >= 0; --q) {
-        const int o = 32 * q;
-        {
-            // all 256 threads: thread (ri, cg) holds row ri, columns 4cg .. 4cg+3 of the
-            // 32 x 32 sub-block; one pivot column is published per barrier
-            const int ri = tid >> 3, cg = tid & 7;
-            float c4[4], v4[4];
+    for (int jb = DG_N / 8 - 1; jb >= 0; --jb) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) c4[e] = S[(o + ri) * DG_LD + o + 4 * cg + e];
-            int bb = 0;
-            for (int j = 31; j >= 0; --j) {
-                if ((j >> 2) == cg) {
-                    float x = c4[0];
-#pragma unroll
-                    for (int e = 1; e < 4; ++e) x = ((j & 3) == e) ? c4[e] : x;
-                    colb[bb * 32 + ri] = x;
+        for (int jj = 7; jj >= 0; --jj) {
+            const int j = 8 * jb + jj;
+            // publish column j of S (rows < j), d_j and row j of V
+            if (tk == jb && i0 < j) {
+                float4 o;
+                o.x = (i0 + 0 < j) ? s[0][jj] : 0.f;
+                o.y = (i0 + 1 < j) ? s[1][jj] : 0.f;
+                o.z = (i0 + 2 < j) ? s[2][jj] : 0.f;
+                o.w = (i0 + 3 < j) ? s[3][jj] : 0.f;
+                *reinterpret_cast<float4 *>(colb + j * DG_N + i0) = o;
+            }
+            if (ti == (j >> 2)) {
+                const int r = jj & 3;
+                *reinterpret_cast<float4 *>(vrow + j * DG_N + c0) =
+                    make_float4(v[r][0], v[r][1], v[r][2], v[r][3]);
+                *reinterpret_cast<float4 *>(vrow + j * DG_N + c0 + 4) =
+                    make_float4(v[r][4], v[r][5], v[r][6], v[r][7]);
+                if (tk == jb) {
+                    const float d = s[r][jj];
+                    dpiv[j] = d;
+                    rpiv[j] = 1.f / fmaxf(d, FLT_MIN);
+                    if (j < nb && !(d > tol * dref[j])) set_status(status, GPTQ_ERR_NOT_PD);
                 }
-                __syncthreads();
-                const float d = colb[bb * 32 + j];
-                if (tid == 0) {
-                    piv[o + j] = d;
-                    if (o + j < nb && !(d > tol * dref[o + j])) set_status(status, GPTQ_ERR_NOT_PD);
-                }
-                const float aij = colb[bb * 32 + ri] / fmaxf(d, FLT_MIN);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int k = 4 * cg + e;
-                    if (ri <= k && k < j) c4[e] = fmaf(-aij, colb[bb * 32 + k], c4[e]);
-                }
-                bb ^= 1;
             }
             __syncthreads();
-            // unit upper L_Q, and V_Q = L_Q^-1 by column elimination on V = I
+            if (wrow0 < j) {
+                const float rd = rpiv[j];
+                const float4 a = *reinterpret_cast<const float4 *>(colb + j * DG_N + i0 % DG_N);
+                const float4 k0 = *reinterpret_cast<const float4 *>(colb + j * DG_N + c0);
+                const float4 k1 = *reinterpret_cast<const float4 *>(colb + j * DG_N + c0 + 4);
+                const float4 v0 = *reinterpret_cast<const float4 *>(vrow + j * DG_N + c0);
+                const float4 v1 = *reinterpret_cast<const float4 *>(vrow + j * DG_N + c0 + 4);
+                const float li[4] = {a.x * rd, a.y * rd, a.z * rd, a.w * rd};
+                const float ak[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+                const float vk[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int k = 4 * cg + e;
-                if (ri < k) c4[e] = c4[e] / fmaxf(piv[o + k], FLT_MIN);
-                v4[e] = (ri == k) ? 1.f : 0.f;
-            }
-            for (int k = 31; k >= 1; --k) {
-                if ((k >> 2) == cg) {
-                    float x = c4[0];
+                for (int r = 0; r < 4; ++r)
 #pragma unroll
-                    for (int e = 1; e < 4; ++e) x = ((k & 3) == e) ? c4[e] : x;
-                    colb[bb * 32 + ri] = x;
-                }
-                if (ri == k) {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) rowb[bb * 32 + 4 * cg + e] = v4[e];
-                }
-                __syncthreads();
-                if (ri < k) {
-                    const float lik = colb[bb * 32 + ri];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) v4[e] = fmaf(-lik, rowb[bb * 32 + 4 * cg + e], v4[e]);
-                }
-                bb ^= 1;
-            }
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int k = 4 * cg + e;
-                S[(o + ri) * DG_LD + o + k] = (k >= ri) ? c4[e] : 0.f;   // L (strict upper), d
-                V[(o + ri) * DG_LD + o + k] = (k >= ri) ? v4[e] : 0.f;
+                    for (int c = 0; c < 8; ++c) {
+                        s[r][c] = fmaf(-li[r], ak[c], s[r][c]);
+                        v[r][c] = fmaf(-li[r], vk[c], v[r][c]);
+                    }
             }
         }
-        __syncthreads();
-        if (q == 0) break;
-        // panel: T = B V_Q^T (B = S[0:o, Q] unscaled), L = T D_Q^-1. Thread (c, rs):
-        // column c = tid & 31, rows rs + 8r; V_Q is stored with zeros below its diagonal.
-        {
-            const int c = tid & 31, rs = tid >> 5, nr = o / 8;
-            float acc[12];
-#pragma unroll
-            for (int r = 0; r < 12; ++r) acc[r] = 0.f;
-#pragma unroll 4
-            for (int m = 0; m < 32; ++m) {
-                const float v = V[(o + c) * DG_LD + o + m];
-#pragma unroll
-                for (int r = 0; r < 12; ++r)
-                    if (r < nr) acc[r] = fmaf(S[(rs + 8 * r) * DG_LD + o + m], v, acc[r]);
-            }
-            __syncthreads();
-            const float rd = 1.f / fmaxf(piv[o + c], FLT_MIN);
-#pragma unroll
-            for (int r = 0; r < 12; ++r)
-                if (r < nr) {
-                    const int i = rs + 8 * r;
-                    Ts[i * 33 + c] = acc[r];
-                    S[i * DG_LD + o + c] = acc[r] * rd;
-                }
-        }
-        __syncthreads();
-        // trailing update of the upper triangle: S[i][k] -= sum_c L[i][c] T[k][c];
-        // thread: k = (tid & 31) + 32 kk, i = (tid >> 5) + 8 r
-        {
-            const int kl = tid & 31, rs = tid >> 5, nr = o / 8, nk = o / 32;
-            float acc[12][3];
-#pragma unroll
-            for (int r = 0; r < 12; ++r)
-#pragma unroll
-                for (int kk = 0; kk < 3; ++kk) acc[r][kk] = 0.f;
-#pragma unroll 2
-            for (int c = 0; c < 32; ++c) {
-                float t[3];
-#pragma unroll
-                for (int kk = 0; kk < 3; ++kk) t[kk] = kk < nk ? Ts[(kl + 32 * kk) * 33 + c] : 0.f;
-#pragma unroll
-                for (int r = 0; r < 12; ++r) {
-                    if (r >= nr) continue;
-                    const float l = S[(rs + 8 * r) * DG_LD + o + c];
-#pragma unroll
-                    for (int kk = 0; kk < 3; ++kk) acc[r][kk] = fmaf(l, t[kk], acc[r][kk]);
-                }
-            }
-#pragma unroll
-            for (int r = 0; r < 12; ++r)
-#pragma unroll
-                for (int kk = 0; kk < 3; ++kk) {
-                    const int i = rs + 8 * r, k = kl + 32 * kk;
-                    if (r < nr && kk < nk && i <= k) S[i * DG_LD + k] -= acc[r][kk];
-                }
-        }
-        __syncthreads();
     }
-    // V = L^-1: for each block column Q, P = Q-1 .. 0; round s does every pair with
-    // Q - P = s. Thread: column c = tid & 31 of the pair, rows (tid >> 5) + 8 r.
-    for (int sr = 1; sr <= 3; ++sr) {
-        const int pairs = 4 - sr, c = tid & 31, rs = tid >> 5;
-        float x[3][4];
+    // U = D^-1/2 V on the tiles (zero below the diagonal)
+    if (ti < 32) {
 #pragma unroll
-        for (int pr = 0; pr < 3; ++pr)
+        for (int r = 0; r < 4; ++r) {
+            const int i = i0 + r;
+            if (i >= nb) continue;
+            const float sc = 1.f / sqrtf(fmaxf(dpiv[i], FLT_MIN));
+            float o[8];
 #pragma unroll
-            for (int r = 0; r < 4; ++r) x[pr][r] = 0.f;
+            for (int c = 0; c < 8; ++c) o[c] = (c0 + c >= i) ? v[r][c] * sc : 0.f;
+            float *dst = H + (int64_t)(j0 + i) * K + j0 + c0;
+            if (vec) {
+                *reinterpret_cast<float4 *>(dst) = make_float4(o[0], o[1], o[2], o[3]);
+                *reinterpret_cast<float4 *>(dst + 4) = make_float4(o[4], o[5], o[6], o[7]);
+            } else {
 #pragma unroll
-        for (int pr = 0; pr < 3; ++pr) {
-            if (pr >= pairs) continue;
-            const int Q = sr + pr, P = Q - sr;
-#pragma unroll 4
-            for (int m = 32 * (P + 1); m < 32 * (Q + 1); ++m) {
-                const float v = V[m * DG_LD + 32 * Q + c];
-#pragma unroll
-                for (int r = 0; r < 4; ++r) x[pr][r] = fmaf(S[(32 * P + rs + 8 * r) * DG_LD + m], v, x[pr][r]);
+                for (int c = 0; c < 8; ++c)
+                    if (c0 + c < nb) dst[c] = o[c];
             }
         }
-#pragma unroll
-        for (int pr = 0; pr < 3; ++pr)
-#pragma unroll
-            for (int r = 0; r < 4; ++r)
-                if (pr < pairs) Ts[(32 * pr + rs + 8 * r) * 33 + c] = x[pr][r];
-        __syncthreads();
-        float y[3][4];
-#pragma unroll
-        for (int pr = 0; pr < 3; ++pr)
-#pragma unroll
-            for (int r = 0; r < 4; ++r) y[pr][r] = 0.f;
-#pragma unroll
-        for (int pr = 0; pr < 3; ++pr) {
-            if (pr >= pairs) continue;
-            const int P = sr + pr - sr;
-#pragma unroll 4
-            for (int m = 0; m < 32; ++m) {
-                const float t = Ts[(32 * pr + m) * 33 + c];
-#pragma unroll
-                for (int r = 0; r < 4; ++r)   // V_PP is upper: zero for m < row
-                    y[pr][r] = fmaf(V[(32 * P + rs + 8 * r) * DG_LD + 32 * P + m], t, y[pr][r]);
-            }
-        }
-#pragma unroll
-        for (int pr = 0; pr < 3; ++pr) {
-            if (pr >= pairs) continue;
-            const int Q = sr + pr, P = Q - sr;
-#pragma unroll
-            for (int r = 0; r < 4; ++r) V[(32 * P + rs + 8 * r) * DG_LD + 32 * Q + c] = -y[pr][r];
-        }
-        __syncthreads();
-    }
-    // U = D^-1/2 V
-    for (int r = warp; r < nb; r += nwarps) {
-        const float sc = 1.f / sqrtf(fmaxf(piv[r], FLT_MIN));
-        for (int c = lane; c < nb; c += 32)
-            H[(int64_t)(j0 + r) * K + j0 + c] = (c >= r) ? V[r * DG_LD + c] * sc : 0.f;
     }
 }
 
@@ -409,16 +322,22 @@ static size_t tc_extra_floats(int K) {
     return 4 * (size_t)K * K + 2 * inverse_scratch_floats(K) + 4 * 64;
 }
 
-// Panel and trailing update of one Cholesky step on the tensor cores, for one group:
-//   R[0:j0, J] = H[0:j0, J] U_JJ^T            (A = rows of the column block, B^T = U_JJ rows)
-//   H[0:j0, 0:j0] -= R[0:j0, J] R[0:j0, J]^T  (A = B^T = rows of R; upper tiles)
-// The tf32 pairs of the column block (j1 x nb) reuse the front of the H-pair buffers.
-static gptq_status chol_step_tc(float *H, int K, int j0, int j1, float *ex, int32_t *status,
-                                cudaStream_t st) {
+// One Cholesky step on the tensor cores, for one group, split for lookahead:
+//   panel : R[0:j0, J] = H[0:j0, J] U_JJ^T       (A = rows of the column block,
+//                                                 B^T = U_JJ rows)
+//   strip : H[0:j0, J'] -= R[0:j0, J] R[J', J]^T  (J' = the next diagonal block, the
+//                                                 columns the next step reads first)
+//   rest  : H[0:j0', 0:j0'] -= R R^T on the rows and columns before J' (upper tiles)
+// with j0' = start of J'. The panel and strip run on the caller's stream (the
+// critical path: next diagonal factor, next panel); the rest runs on a second
+// stream and overlaps the next steps. The tf32 pairs of the column block live in a
+// per-(group, step parity) buffer so that a rest still reading them is not
+// overwritten by the next step.
+static gptq_status chol_panel_strip_tc(float *H, int K, int j0, int j1, int j0n, float *buf,
+                                       int32_t *status, cudaStream_t st, CUtensorMap (&m)[4]) {
     const int nb = j1 - j0;
-    float *Ch = ex, *Cl = Ch + (size_t)j1 * nb;
+    float *Ch = buf, *Cl = Ch + (size_t)j1 * nb;
     static thread_local Tc32Params pp, ps;
-    CUtensorMap m[4];
     gptq_status s;
     if ((s = split_tf32(H + j0, K, j1, nb, Ch, Cl, nb, 1, 0, 0, st)) != GPTQ_OK) return s;
     if ((s = make_f32_map(&m[0], Ch, nb, j1, nb, 32, 128)) != GPTQ_OK) return s;
@@ -432,13 +351,59 @@ static gptq_status chol_step_tc(float *H, int K, int j0, int j1, float *ex, int3
     if ((s = launch_gemm_tc32(m, pp, st)) != GPTQ_OK) return s;
     // pairs of the new panel R (rows 0..j0 of the block, overwriting the front)
     if ((s = split_tf32(H + j0, K, j0, nb, Ch, Cl, nb, 1, 0, 0, st)) != GPTQ_OK) return s;
+    // strip: every row above j0 against the rows of J' (entries below the diagonal of
+    // H[J', J'] are updated too; nothing reads them)
     ps = Tc32Params{};
-    ps.C = H; ps.alpha = -1.f; ps.accumulate = 1; ps.upper_tiles = 1; ps.status = status;
-    ps.nitems = 1;
-    ps.item[0].m = j0; ps.item[0].n = j0; ps.item[0].k = nb;
-    ps.item[0].a_x0 = 0; ps.item[0].a_y0 = 0; ps.item[0].b_x0 = 0; ps.item[0].b_y0 = 0;
-    ps.item[0].c_off = 0; ps.item[0].ldc = K;
+    ps.C = H; ps.alpha = -1.f; ps.accumulate = 1; ps.status = status; ps.nitems = 1;
+    ps.item[0].m = j0; ps.item[0].n = j0 - j0n; ps.item[0].k = nb;
+    ps.item[0].a_x0 = 0; ps.item[0].a_y0 = 0; ps.item[0].b_x0 = 0; ps.item[0].b_y0 = j0n;
+    ps.item[0].c_off = j0n; ps.item[0].ldc = K;
     return launch_gemm_tc32(m, ps, st);
+}
+
+static gptq_status chol_rest_tc(float *H, int K, int j0n, const CUtensorMap (&m)[4],
+                                int32_t *status, cudaStream_t st, int nb) {
+    if (j0n <= 0) return GPTQ_OK;
+    static thread_local Tc32Params pr;
+    pr = Tc32Params{};
+    pr.C = H; pr.alpha = -1.f; pr.accumulate = 1; pr.upper_tiles = 1; pr.status = status;
+    pr.nitems = 1;
+    pr.item[0].m = j0n; pr.item[0].n = j0n; pr.item[0].k = nb;
+    pr.item[0].c_off = 0; pr.item[0].ldc = K;
+    return launch_gemm_tc32(m, pr, st);
+}
+
+// Per-device second stream and events for the lookahead (created once).
+constexpr int LA_MAX_GROUPS = 8;
+struct Lookahead {
+    cudaStream_t side = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+    cudaEvent_t panel[LA_MAX_GROUPS][2], rest[LA_MAX_GROUPS][2];
+    bool ok = false;
+};
+
+static Lookahead *lookahead_for_device() {
+    static std::mutex mu;
+    static Lookahead la[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    Lookahead &L = la[dev];
+    if (!L.ok) {
+        bool good = cudaStreamCreateWithFlags(&L.side, cudaStreamNonBlocking) == cudaSuccess;
+        good = good && cudaEventCreateWithFlags(&L.fork, cudaEventDisableTiming) == cudaSuccess;
+        good = good && cudaEventCreateWithFlags(&L.join, cudaEventDisableTiming) == cudaSuccess;
+        for (int gi = 0; gi < LA_MAX_GROUPS && good; ++gi)
+            for (int b = 0; b < 2 && good; ++b)
+                good = cudaEventCreateWithFlags(&L.panel[gi][b], cudaEventDisableTiming) == cudaSuccess &&
+                       cudaEventCreateWithFlags(&L.rest[gi][b], cudaEventDisableTiming) == cudaSuccess;
+        if (!good) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        L.ok = true;
+    }
+    return &L;
 }
 
 // Trailing sizes below this stay on the SIMT kernels (launch-bound there).
@@ -599,22 +564,75 @@ gptq_status prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out, v
     if ((s = launch_status()) != GPTQ_OK) return s;
 
     const float tol = (float)K * FLT_EPSILON;
-    const int chol_smem = (int)((2 * CH_NB * DG_LD + 96 * 33 + 2 * CH_NB + 128) * sizeof(float));
+    const int chol_smem = (int)((2 * DG_N * DG_N + 3 * DG_N) * sizeof(float));
     cudaFuncSetAttribute(k_chol_diag, cudaFuncAttributeMaxDynamicSharedMemorySize, chol_smem);
     Blocks bk{K, (K + CH_NB - 1) / CH_NB};
+    // lookahead on the tensor-core steps (a second stream runs the bulk trailing
+    // updates); without it every step runs in order on the caller's stream
+    const size_t pair_floats = (size_t)K * CH_NB * 2;
+    // the per-(group, parity) pair buffers use the front of the inverse's pair area
+    Lookahead *la = (use_tc && g <= LA_MAX_GROUPS && (size_t)g * 2 * pair_floats <= 4 * (size_t)KK)
+                        ? lookahead_for_device()
+                        : nullptr;
+    bool side_busy = false;         // work issued on the side stream not yet joined
+    int rest_of[2] = {-1, -1};      // step whose rest was last recorded in parity slot
+    auto join_side = [&]() -> gptq_status {
+        if (!side_busy) return GPTQ_OK;
+        if (cudaEventRecord(la->join, la->side) != cudaSuccess ||
+            cudaStreamWaitEvent(st, la->join, 0) != cudaSuccess)
+            return GPTQ_ERR_CUDA;
+        side_busy = false;
+        return GPTQ_OK;
+    };
     for (int t = bk.T - 1; t >= 0; --t) {
         const int j0 = bk.start(t);
         const int j1 = (t == bk.T - 1) ? K : bk.start(t + 1);
         const int nb = j1 - j0;
+        // the diagonal block's last updates: the rest of step t + 2 (the rest of step
+        // t + 1 does not reach it)
+        if (la && t + 2 < bk.T && rest_of[(t + 2) & 1] == t + 2)
+            for (int gi = 0; gi < g; ++gi)
+                if (cudaStreamWaitEvent(st, la->rest[gi][(t + 2) & 1], 0) != cudaSuccess)
+                    return GPTQ_ERR_CUDA;
         k_chol_diag<<<g, DG_T, chol_smem, st>>>(H, K, j0, nb, diag_d, tol, status);
         if ((s = launch_status()) != GPTQ_OK) return s;
         if (j0 == 0) break;
         if (use_tc && j0 >= TC_STEP_MIN && nb % 32 == 0) {
-            for (int gi = 0; gi < g; ++gi)
-                if ((s = chol_step_tc(H + (int64_t)gi * KK, K, j0, j1, ex, status, st)) != GPTQ_OK)
+            if (la) {
+                const int j0n = bk.start(t - 1);
+                if (!side_busy) {
+                    if (cudaEventRecord(la->fork, st) != cudaSuccess ||
+                        cudaStreamWaitEvent(la->side, la->fork, 0) != cudaSuccess)
+                        return GPTQ_ERR_CUDA;
+                    side_busy = true;
+                }
+                for (int gi = 0; gi < g; ++gi) {
+                    float *Hg = H + (int64_t)gi * KK;
+                    float *buf = ex + (size_t)(gi * 2 + (t & 1)) * pair_floats;
+                    CUtensorMap m[4];
+                    if ((s = chol_panel_strip_tc(Hg, K, j0, j1, j0n, buf, status, st, m)) != GPTQ_OK)
+                        return s;
+                    if (cudaEventRecord(la->panel[gi][t & 1], st) != cudaSuccess ||
+                        cudaStreamWaitEvent(la->side, la->panel[gi][t & 1], 0) != cudaSuccess)
+                        return GPTQ_ERR_CUDA;
+                    if ((s = chol_rest_tc(Hg, K, j0n, m, status, la->side, nb)) != GPTQ_OK) return s;
+                    if (cudaEventRecord(la->rest[gi][t & 1], la->side) != cudaSuccess)
+                        return GPTQ_ERR_CUDA;
+                }
+                rest_of[t & 1] = t;
+                continue;
+            }
+            for (int gi = 0; gi < g; ++gi) {
+                float *Hg = H + (int64_t)gi * KK;
+                CUtensorMap m[4];
+                const int j0n = bk.start(t - 1);
+                if ((s = chol_panel_strip_tc(Hg, K, j0, j1, j0n, ex, status, st, m)) != GPTQ_OK)
                     return s;
+                if ((s = chol_rest_tc(Hg, K, j0n, m, status, st, nb)) != GPTQ_OK) return s;
+            }
             continue;
         }
+        if ((s = join_side()) != GPTQ_OK) return s;
         // panel: R[0:j0, J] = H[0:j0, J] U_JJ^T  (in place: each CTA owns whole rows)
         GemmParams pp = gemm_params(j0, nb, nb, H + j0, K, H + (int64_t)j0 * K + j0, K,
                                     H + j0, K, 1.f, 0, status);
@@ -626,6 +644,7 @@ gptq_status prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out, v
         ps.sA = KK; ps.sB = KK; ps.sC = KK;
         if ((s = gemm_simt<float, float, false, true>(ps, g, st)) != GPTQ_OK) return s;
     }
+    if ((s = join_side()) != GPTQ_OK) return s;
     // The strict lower triangle still holds the input and update leftovers; the
     // inverse reads whole tiles of its triangular operands, so clear it first.
     k_zero_lower<<<dim3((K + 255) / 256 > 8 ? 8 : (K + 255) / 256, K, g), 256, 0, st>>>(H, K);
