@@ -47,6 +47,16 @@ inline gptq_status launch_status() {
     return e == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
 }
 
+// d = a * b + c on two fp32 lanes at once (sm_100 packed fp32 FMA, round to nearest).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;"
+        : "=l"(d)
+        : "l"(*reinterpret_cast<const uint64_t *>(&a)), "l"(*reinterpret_cast<const uint64_t *>(&b)),
+          "l"(*reinterpret_cast<const uint64_t *>(&c)));
+    return *reinterpret_cast<const float2 *>(&d);
+}
+
 inline bool aligned(const void *p, size_t a) {
     return (reinterpret_cast<uintptr_t>(p) % a) == 0;
 }

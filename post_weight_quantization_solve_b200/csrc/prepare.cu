@@ -126,7 +126,8 @@ __global__ void __launch_bounds__(DG_T, 1) k_chol_diag(float *H, int K, int j0, 
         if (r < nb && c < nb && (r >> 2) > 2 * (c >> 3) + 1) H[(int64_t)(j0 + r) * K + j0 + c] = 0.f;
     }
 
-    float s[4][8], v[4][8];
+    // tile rows as column pairs (c, c + 1): the updates run as packed fp32 FMAs
+    float2 s[4][4], v[4][4];
     const bool vec = (nb == DG_N) && (K % 4 == 0) && ((reinterpret_cast<uintptr_t>(H) & 15) == 0) &&
                      (j0 % 4 == 0);
 #pragma unroll
@@ -136,17 +137,21 @@ __global__ void __launch_bounds__(DG_T, 1) k_chol_diag(float *H, int K, int j0, 
             const float *src = H + (int64_t)(j0 + i) * K + j0 + c0;
             const float4 x0 = *reinterpret_cast<const float4 *>(src);
             const float4 x1 = *reinterpret_cast<const float4 *>(src + 4);
-            s[r][0] = x0.x; s[r][1] = x0.y; s[r][2] = x0.z; s[r][3] = x0.w;
-            s[r][4] = x1.x; s[r][5] = x1.y; s[r][6] = x1.z; s[r][7] = x1.w;
+            s[r][0] = make_float2(x0.x, x0.y); s[r][1] = make_float2(x0.z, x0.w);
+            s[r][2] = make_float2(x1.x, x1.y); s[r][3] = make_float2(x1.z, x1.w);
         } else {
+            float e[8];
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
                 const int k = c0 + c;
-                s[r][c] = (i < nb && k < nb) ? H[(int64_t)(j0 + i) * K + j0 + k] : (i == k ? 1.f : 0.f);
+                e[c] = (i < nb && k < nb) ? H[(int64_t)(j0 + i) * K + j0 + k] : (i == k ? 1.f : 0.f);
             }
+#pragma unroll
+            for (int c = 0; c < 4; ++c) s[r][c] = make_float2(e[2 * c], e[2 * c + 1]);
         }
 #pragma unroll
-        for (int c = 0; c < 8; ++c) v[r][c] = (i == c0 + c) ? 1.f : 0.f;
+        for (int c = 0; c < 4; ++c)
+            v[r][c] = make_float2((i == c0 + 2 * c) ? 1.f : 0.f, (i == c0 + 2 * c + 1) ? 1.f : 0.f);
     }
     __syncthreads();
 
@@ -157,20 +162,20 @@ __global__ void __launch_bounds__(DG_T, 1) k_chol_diag(float *H, int K, int j0, 
             // publish column j of S (rows < j), d_j and row j of V
             if (tk == jb && i0 < j) {
                 float4 o;
-                o.x = (i0 + 0 < j) ? s[0][jj] : 0.f;
-                o.y = (i0 + 1 < j) ? s[1][jj] : 0.f;
-                o.z = (i0 + 2 < j) ? s[2][jj] : 0.f;
-                o.w = (i0 + 3 < j) ? s[3][jj] : 0.f;
+                o.x = (i0 + 0 < j) ? ((jj & 1) ? s[0][jj >> 1].y : s[0][jj >> 1].x) : 0.f;
+                o.y = (i0 + 1 < j) ? ((jj & 1) ? s[1][jj >> 1].y : s[1][jj >> 1].x) : 0.f;
+                o.z = (i0 + 2 < j) ? ((jj & 1) ? s[2][jj >> 1].y : s[2][jj >> 1].x) : 0.f;
+                o.w = (i0 + 3 < j) ? ((jj & 1) ? s[3][jj >> 1].y : s[3][jj >> 1].x) : 0.f;
                 *reinterpret_cast<float4 *>(colb + j * DG_N + i0) = o;
             }
             if (ti == (j >> 2)) {
                 const int r = jj & 3;
                 *reinterpret_cast<float4 *>(vrow + j * DG_N + c0) =
-                    make_float4(v[r][0], v[r][1], v[r][2], v[r][3]);
+                    make_float4(v[r][0].x, v[r][0].y, v[r][1].x, v[r][1].y);
                 *reinterpret_cast<float4 *>(vrow + j * DG_N + c0 + 4) =
-                    make_float4(v[r][4], v[r][5], v[r][6], v[r][7]);
+                    make_float4(v[r][2].x, v[r][2].y, v[r][3].x, v[r][3].y);
                 if (tk == jb) {
-                    const float d = s[r][jj];
+                    const float d = (jj & 1) ? s[r][jj >> 1].y : s[r][jj >> 1].x;
                     dpiv[j] = d;
                     rpiv[j] = 1.f / fmaxf(d, FLT_MIN);
                     if (j < nb && !(d > tol * dref[j])) set_status(status, GPTQ_ERR_NOT_PD);
@@ -184,16 +189,20 @@ __global__ void __launch_bounds__(DG_T, 1) k_chol_diag(float *H, int K, int j0, 
                 const float4 k1 = *reinterpret_cast<const float4 *>(colb + j * DG_N + c0 + 4);
                 const float4 v0 = *reinterpret_cast<const float4 *>(vrow + j * DG_N + c0);
                 const float4 v1 = *reinterpret_cast<const float4 *>(vrow + j * DG_N + c0 + 4);
-                const float li[4] = {a.x * rd, a.y * rd, a.z * rd, a.w * rd};
-                const float ak[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-                const float vk[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                const float li[4] = {-a.x * rd, -a.y * rd, -a.z * rd, -a.w * rd};
+                const float2 ak[4] = {make_float2(k0.x, k0.y), make_float2(k0.z, k0.w),
+                                      make_float2(k1.x, k1.y), make_float2(k1.z, k1.w)};
+                const float2 vk[4] = {make_float2(v0.x, v0.y), make_float2(v0.z, v0.w),
+                                      make_float2(v1.x, v1.y), make_float2(v1.z, v1.w)};
 #pragma unroll
-                for (int r = 0; r < 4; ++r)
+                for (int r = 0; r < 4; ++r) {
+                    const float2 l2 = make_float2(li[r], li[r]);
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        s[r][c] = fmaf(-li[r], ak[c], s[r][c]);
-                        v[r][c] = fmaf(-li[r], vk[c], v[r][c]);
+                    for (int c = 0; c < 4; ++c) {
+                        s[r][c] = ffma2(l2, ak[c], s[r][c]);
+                        v[r][c] = ffma2(l2, vk[c], v[r][c]);
                     }
+                }
             }
         }
     }
@@ -206,7 +215,10 @@ __global__ void __launch_bounds__(DG_T, 1) k_chol_diag(float *H, int K, int j0, 
             const float sc = 1.f / sqrtf(fmaxf(dpiv[i], FLT_MIN));
             float o[8];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) o[c] = (c0 + c >= i) ? v[r][c] * sc : 0.f;
+            for (int c = 0; c < 8; ++c) {
+                const float vc = (c & 1) ? v[r][c >> 1].y : v[r][c >> 1].x;
+                o[c] = (c0 + c >= i) ? vc * sc : 0.f;
+            }
             float *dst = H + (int64_t)(j0 + i) * K + j0 + c0;
             if (vec) {
                 *reinterpret_cast<float4 *>(dst) = make_float4(o[0], o[1], o[2], o[3]);
@@ -406,8 +418,8 @@ static Lookahead *lookahead_for_device() {
     return &L;
 }
 
-// Trailing sizes below this stay on the SIMT kernels (launch-bound there).
-constexpr int TC_STEP_MIN = 1024;
+// Trailing sizes below this stay on the SIMT kernels.
+constexpr int TC_STEP_MIN = 128;
 
 size_t prepare_workspace(int K, int g) {
     size_t base = prepare_workspace_compact(K, g);
@@ -423,28 +435,38 @@ struct SplitBlocks {
 };
 
 __global__ void k_split_blocks(const float *__restrict__ H, int K, float *__restrict__ hi,
-                               float *__restrict__ lo, int transposed, const SplitBlocks sb) {
+                               float *__restrict__ lo, float *__restrict__ hit,
+                               float *__restrict__ lot, const SplitBlocks sb) {
+    // one read of each 32 x 32 tile; its pairs are written in place (hi, lo) and
+    // transposed (hit, lot)
     __shared__ float t[32][33];
     const int r0 = sb.r0[blockIdx.z], n = sb.n[blockIdx.z];
     const int tr = blockIdx.y * 32, tcol = blockIdx.x * 32;
     if (tr >= n || tcol >= n) return;
     for (int y = threadIdx.y; y < 32; y += 8) {
         const int r = tr + y, c = tcol + threadIdx.x;
-        t[y][threadIdx.x] = (r < n && c < n) ? H[(int64_t)(r0 + r) * K + r0 + c] : 0.f;
+        const float x = (r < n && c < n) ? H[(int64_t)(r0 + r) * K + r0 + c] : 0.f;
+        t[y][threadIdx.x] = x;
+        if (r < n && c < n) {
+            uint32_t h;
+            asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(x));
+            const float hf = __uint_as_float(h);
+            const int64_t o = (int64_t)(r0 + r) * K + r0 + c;
+            hi[o] = hf;
+            lo[o] = x - hf;
+        }
     }
     __syncthreads();
     for (int y = threadIdx.y; y < 32; y += 8) {
-        int orow, ocol;
-        float x;
-        if (transposed) { orow = tcol + y; ocol = tr + threadIdx.x; x = t[threadIdx.x][y]; }
-        else { orow = tr + y; ocol = tcol + threadIdx.x; x = t[y][threadIdx.x]; }
+        const int orow = tcol + y, ocol = tr + threadIdx.x;
         if (orow < n && ocol < n) {
+            const float x = t[threadIdx.x][y];
             uint32_t h;
             asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(x));
             const float hf = __uint_as_float(h);
             const int64_t o = (int64_t)(r0 + orow) * K + r0 + ocol;
-            hi[o] = hf;
-            lo[o] = x - hf;
+            hit[o] = hf;
+            lot[o] = x - hf;
         }
     }
 }
@@ -499,9 +521,7 @@ static gptq_status tri_inverse_tc(float *H, int K, const Blocks &bk, float *Tt, 
                 nmax = std::max(nmax, sb.n[ni]);
             }
             const dim3 grid((nmax + 31) / 32, (nmax + 31) / 32, sb.n_items);
-            k_split_blocks<<<grid, dim3(32, 8), 0, st>>>(H, K, Hh, Hl, 0, sb);
-            if ((s = launch_status()) != GPTQ_OK) return s;
-            k_split_blocks<<<grid, dim3(32, 8), 0, st>>>(H, K, Gh, Gl, 1, sb);
+            k_split_blocks<<<grid, dim3(32, 8), 0, st>>>(H, K, Hh, Hl, Gh, Gl, sb);
             if ((s = launch_status()) != GPTQ_OK) return s;
         }
         cudaMemsetAsync(Tt, 0, sizeof(float) * (size_t)trows * pitch, st);
