@@ -21,8 +21,9 @@
 //             sweep's stores coalesce; the update reads it as an MN-major operand)
 //   Ph, Pl    bf16 [S][ldE] pre-rounding weights (GPTAQ), same layout
 //   Uh, Ul    bf16 [g][K][ldU] U as hi + lo pairs;  Qh, Ql  the same for P1
-// A sweep CTA owns 32 or 64 channels of one group for a block; each warp keeps one
-// 32-coordinate sub-block of 32 channels in registers (k_sweep_block).
+// The sweep keeps each channel's block coordinates in registers: one thread per
+// channel for layers with many output channels (k_sweep_thread), four lanes per
+// channel otherwise (k_sweep_lanes).
 #include <cuda.h>
 
 #include <algorithm>
@@ -128,17 +129,187 @@ __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
-// In-block sweep of one block [i0, i0 + bs) for SW_T channels of one group, one
-// thread per channel with all of the block's coordinates in registers (as pairs).
+// In-block sweep, lane-group form (for layers with few output channels): one block
+// [i0, i0 + bs) for 32 channels of one group.
+// A warp serves 8 channels with 4 lanes each: lane 4 c + q of the warp holds, of
+// channel c, the coordinates 32 b + 8 q + i (i < 8) of every 32-wide sub-block b, so
+// all 32 coordinates of the block stay in registers and every lane has work at every
+// step. At step j = 32 p + t the lane holding coordinate j (slot q = t / 8) rounds it
+// and computes E_j; a shuffle inside the channel's 4 lanes hands E_j to the others,
+// and each lane applies it to its own coordinates (U's zero lower triangle makes the
+// coordinates at or before j no-ops, so no lane masks). The sub-block in work is
+// always w[0]: the register array shifts by one sub-block after each phase. No block
+// barrier inside the sweep. U[blk, blk] (and P1) is staged once per CTA as its ten
+// 32 x 32 blocks on or above the diagonal.
+template <bool GPTAQ>
+__global__ void __launch_bounds__(128, GPTAQ ? 2 : 4) k_sweep_lanes(
+    float *__restrict__ Wk, int N, int per_group, int K, int i0, int bs,
+    const float *__restrict__ U, const float *__restrict__ P1, const float *__restrict__ scale,
+    int bits, uint8_t *__restrict__ codes, __nv_bfloat16 *__restrict__ Eh,
+    __nv_bfloat16 *__restrict__ El, __nv_bfloat16 *__restrict__ Ph, __nv_bfloat16 *__restrict__ Pl,
+    int ldE, int ldG, int erow0, float *__restrict__ loss_acc, int vec, const int32_t *status) {
+    constexpr int NCH = 32, CLD = 132;
+    if (failed(status)) return;
+    extern __shared__ __align__(16) unsigned char smem[];
+    float *Us = reinterpret_cast<float *>(smem);                 // [10][32][32]
+    float *Ps = Us + 10 * 1024;                                  // GPTAQ only
+    uint8_t *Cs = reinterpret_cast<uint8_t *>(Ps + (GPTAQ ? 10 * 1024 : 0));  // [NCH][CLD]
+    float *rpiv = reinterpret_cast<float *>(Cs + NCH * CLD);    // [SW_MAXB]
+
+    const int grp = blockIdx.y;
+    const int cta_ch0 = blockIdx.x * NCH;
+    const int n0 = grp * per_group + cta_ch0;
+    const int nvalid = min(NCH, per_group - cta_ch0);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q = lane & 3;
+    const int ch = warp * 8 + (lane >> 2);
+    const bool valid = ch < nvalid;
+    const int64_t n = (int64_t)n0 + ch;
+    const int nsb = (bs + 31) / 32;
+    const float *Ub = U + (int64_t)grp * K * K + (int64_t)i0 * K + i0;   // U[i0, i0]
+    const float *Pb = GPTAQ ? P1 + (int64_t)i0 * K + i0 : nullptr;
+
+    // the ten blocks (P, Q), P <= Q, of U[blk, blk]; zero outside [0, bs)
+    for (int idx = tid; idx < 10 * 256; idx += 128) {
+        const int blk = idx >> 8;
+        const int P = blk < 4 ? 0 : blk < 7 ? 1 : blk < 9 ? 2 : 3;
+        const int Q = P + blk - (P * 4 - P * (P - 1) / 2);
+        if (Q >= nsb) continue;
+        const int r = (idx >> 3) & 31, c4 = (idx & 7) * 4;
+        const int row = 32 * P + r, col = 32 * Q + c4;
+        float *du = Us + blk * 1024 + r * 32 + c4;
+        float *dp = Ps + blk * 1024 + r * 32 + c4;
+        if (vec & 1) {        // rows 16-byte aligned and bs % 4 == 0
+            const bool in = row < bs && col < bs;
+            const int64_t off = in ? (int64_t)row * K + col : 0;
+            cp_async16(du, Ub + off, in ? 16 : 0);
+            if (GPTAQ) cp_async16(dp, Pb + off, in ? 16 : 0);
+        } else {
+            for (int e = 0; e < 4; ++e) {
+                const bool in = row < bs && col + e < bs;
+                du[e] = in ? Ub[(int64_t)row * K + col + e] : 0.f;
+                if (GPTAQ) dp[e] = in ? Pb[(int64_t)row * K + col + e] : 0.f;
+            }
+        }
+    }
+    if (tid < bs) rpiv[tid] = 1.f / __ldg(Ub + (int64_t)tid * K + tid);
+
+    // this lane's coordinates 32 b + 8 q + i of its channel
+    float w[4][8];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        const int c0 = 32 * b + 8 * q;
+        const float *src = Wk + n * K + i0 + c0;
+        if (valid && (vec & 1) && c0 + 8 <= bs) {
+            const float4 x0 = *reinterpret_cast<const float4 *>(src);
+            const float4 x1 = *reinterpret_cast<const float4 *>(src + 4);
+            w[b][0] = x0.x; w[b][1] = x0.y; w[b][2] = x0.z; w[b][3] = x0.w;
+            w[b][4] = x1.x; w[b][5] = x1.y; w[b][6] = x1.z; w[b][7] = x1.w;
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) w[b][i] = (valid && c0 + i < bs) ? src[i] : 0.f;
+        }
+    }
+    cp_async_wait_all();
+    __syncthreads();
+
+    const float s = valid ? scale[n] : 1.f;
+    const float rs = 1.f / s;
+    const float zf = (float)(1 << (bits - 1));
+    const float cmin = -zf, cmax = (float)((1 << bits) - 1) - zf;
+    const int gsrc = lane & ~3;
+    float lacc = 0.f;
+    uint8_t *crow = Cs + ch * CLD;
+    const int64_t ecol = (int64_t)grp * ldG + cta_ch0 + ch;
+
+#pragma unroll 1
+    for (int p = 0; p < nsb; ++p) {
+        const int bbase = p * 4 - p * (p - 1) / 2;       // block (p, p)
+        int64_t eoff = (int64_t)(erow0 + 32 * p) * ldE + ecol;
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+            const int j = 32 * p + t;
+            const int oq = t >> 3, oi = t & 7;
+            const bool live = j < bs;
+            const float wj = w[0][oi];
+            const float cf = fminf(fmaxf(rintf(wj * rs), cmin), cmax);
+            const float ej = live ? fmaf(-s, cf, wj) * rpiv[j] : 0.f;
+            const float e = __shfl_sync(0xffffffffu, ej, gsrc | oq);
+            float v = 0.f;
+            if (GPTAQ) v = __shfl_sync(0xffffffffu, live ? wj : 0.f, gsrc | oq);
+            if (q == oq && live) {
+                lacc = fmaf(ej, ej, lacc);
+                crow[j] = (uint8_t)(int)(cf + zf);
+                if (valid) {
+                    const __nv_bfloat16 eh = __float2bfloat16_rn(ej);
+                    Eh[eoff] = eh;
+                    El[eoff] = __float2bfloat16_rn(ej - __bfloat162float(eh));
+                    if (GPTAQ) {
+                        const __nv_bfloat16 ph = __float2bfloat16_rn(wj);
+                        Ph[eoff] = ph;
+                        Pl[eoff] = __float2bfloat16_rn(wj - __bfloat162float(ph));
+                    }
+                }
+            }
+            eoff += ldE;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                if (b > 0 && p + b >= nsb) break;
+                const float *ur = Us + (bbase + b) * 1024 + t * 32 + 8 * q;
+                const float4 u0 = *reinterpret_cast<const float4 *>(ur);
+                const float4 u1 = *reinterpret_cast<const float4 *>(ur + 4);
+                w[b][0] = fmaf(-e, u0.x, w[b][0]); w[b][1] = fmaf(-e, u0.y, w[b][1]);
+                w[b][2] = fmaf(-e, u0.z, w[b][2]); w[b][3] = fmaf(-e, u0.w, w[b][3]);
+                w[b][4] = fmaf(-e, u1.x, w[b][4]); w[b][5] = fmaf(-e, u1.y, w[b][5]);
+                w[b][6] = fmaf(-e, u1.z, w[b][6]); w[b][7] = fmaf(-e, u1.w, w[b][7]);
+                if (GPTAQ) {
+                    const float *pr = Ps + (bbase + b) * 1024 + t * 32 + 8 * q;
+                    const float4 p0 = *reinterpret_cast<const float4 *>(pr);
+                    const float4 p1 = *reinterpret_cast<const float4 *>(pr + 4);
+                    w[b][0] = fmaf(v, p0.x, w[b][0]); w[b][1] = fmaf(v, p0.y, w[b][1]);
+                    w[b][2] = fmaf(v, p0.z, w[b][2]); w[b][3] = fmaf(v, p0.w, w[b][3]);
+                    w[b][4] = fmaf(v, p1.x, w[b][4]); w[b][5] = fmaf(v, p1.y, w[b][5]);
+                    w[b][6] = fmaf(v, p1.z, w[b][6]); w[b][7] = fmaf(v, p1.w, w[b][7]);
+                }
+            }
+        }
+        // the next sub-block becomes w[0]
+#pragma unroll
+        for (int b = 0; b < 3; ++b)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) w[b][i] = w[b + 1][i];
+    }
+    lacc += __shfl_xor_sync(0xffffffffu, lacc, 1);
+    lacc += __shfl_xor_sync(0xffffffffu, lacc, 2);
+    if (q == 0 && valid) loss_acc[n] += lacc;
+    __syncthreads();
+    // codes: 16-byte chunks of each channel's block row
+    const bool vecC = vec & 2;   // code rows 16-byte aligned
+    for (int idx = tid; idx < NCH * (SW_MAXB / 16); idx += 128) {
+        const int r = idx >> 3, c16 = (idx & 7) * 16;
+        if (r >= nvalid || c16 >= bs) continue;
+        uint8_t *dst = codes + ((int64_t)n0 + r) * K + i0 + c16;
+        const uint32_t *srcw = reinterpret_cast<const uint32_t *>(Cs + r * CLD + c16);
+        if (vecC && c16 + 16 <= bs) {
+            *reinterpret_cast<uint4 *>(dst) = make_uint4(srcw[0], srcw[1], srcw[2], srcw[3]);
+        } else {
+            for (int e = 0; e < 16 && c16 + e < bs; ++e) dst[e] = Cs[r * CLD + c16 + e];
+        }
+    }
+}
+
+// In-block sweep, thread form (for layers with many output channels): one block
+// [i0, i0 + bs) for SW_T channels of one group, one thread per channel with all of the block's coordinates in registers (as pairs).
 // Phase p sweeps sub-block p (32 coordinates), always held in w[0]: step t rounds
-// coordinate 32 p + t, forms E_j, and applies it to the later coordinates of the
-// sub-block and to every later sub-block (packed fp32 FMAs against a broadcast row of
-// U); after the phase the register array shifts by one sub-block. U[blk, blk] (and P1)
+// coordinate 32 p + t, forms E_j and applies it to the later coordinates of the
+// sub-block (packed fp32 FMAs against a broadcast row of U); the phase's 32 errors then
+// go to every later sub-block in one compact loop, and the register array shifts by
+// one sub-block. U[blk, blk] (and P1)
 // is staged once per CTA as its ten 32 x 32 blocks on or above the diagonal.
 constexpr int SW_T = 64;
 
 template <bool GPTAQ>
-__global__ void __launch_bounds__(SW_T, 1) k_sweep_block(
+__global__ void __launch_bounds__(SW_T, 1) k_sweep_thread(
     float *__restrict__ Wk, int N, int per_group, int K, int i0, int bs,
     const float *__restrict__ U, const float *__restrict__ P1, const float *__restrict__ scale,
     int bits, uint8_t *__restrict__ codes, __nv_bfloat16 *__restrict__ Eh,
@@ -149,6 +320,8 @@ __global__ void __launch_bounds__(SW_T, 1) k_sweep_block(
     float *Us = reinterpret_cast<float *>(smem);                 // [10][32][32]
     float *Ps = Us + 10 * 1024;                                  // GPTAQ only
     float *rpiv = Ps + (GPTAQ ? 10 * 1024 : 0);                  // [SW_MAXB]
+    float *Es = rpiv + SW_MAXB;                                  // [32][SW_T] this phase's E
+    float *Vs = Es + 32 * SW_T;                                  // GPTAQ: pre-rounding weights
 
     const int grp = blockIdx.y;
     const int cta_ch0 = blockIdx.x * SW_T;
@@ -229,6 +402,8 @@ __global__ void __launch_bounds__(SW_T, 1) k_sweep_block(
         const float *Pp = Ps + bbase * 1024;
         int64_t eoff = (int64_t)(erow0 + 32 * p) * ldE + ecol;
         uint32_t cw[4] = {0u, 0u, 0u, 0u};
+        // the 32 steps inside sub-block p; each step's error is kept for the later
+        // sub-blocks, which take all 32 at once after the phase
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
             const int j = 32 * p + t;
@@ -237,6 +412,8 @@ __global__ void __launch_bounds__(SW_T, 1) k_sweep_block(
             const float cf = fminf(fmaxf(rintf(wj * rs), cmin), cmax);
             const float ej = live ? fmaf(-s, cf, wj) * rpiv[j] : 0.f;
             const float vj = (GPTAQ && live) ? wj : 0.f;
+            Es[t * SW_T + tid] = ej;
+            if (GPTAQ) Vs[t * SW_T + tid] = vj;
             cw[(t >> 2) & 3] |= (uint32_t)(int)(cf + zf) << (8 * (t & 3));
             if (live) {
                 lacc = fmaf(ej, ej, lacc);
@@ -264,24 +441,6 @@ __global__ void __launch_bounds__(SW_T, 1) k_sweep_block(
                     w[0][i] = ffma2(vv, pp, w[0][i]);
                 }
             }
-            // later sub-blocks
-#pragma unroll
-            for (int b = 1; b < 4; ++b) {
-                if (b >= nblk) break;
-                const float *ur = Up + b * 1024 + t * 32;
-                const float *pr = Pp + b * 1024 + t * 32;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float4 u = *reinterpret_cast<const float4 *>(ur + 4 * i);
-                    w[b][2 * i] = ffma2(ne, make_float2(u.x, u.y), w[b][2 * i]);
-                    w[b][2 * i + 1] = ffma2(ne, make_float2(u.z, u.w), w[b][2 * i + 1]);
-                    if (GPTAQ) {
-                        const float4 q = *reinterpret_cast<const float4 *>(pr + 4 * i);
-                        w[b][2 * i] = ffma2(vv, make_float2(q.x, q.y), w[b][2 * i]);
-                        w[b][2 * i + 1] = ffma2(vv, make_float2(q.z, q.w), w[b][2 * i + 1]);
-                    }
-                }
-            }
             if ((t & 15) == 15) {
                 // 16 codes of this channel
                 const int c16 = 32 * p + (t & 16);
@@ -294,6 +453,36 @@ __global__ void __launch_bounds__(SW_T, 1) k_sweep_block(
                     }
                 }
                 cw[0] = cw[1] = cw[2] = cw[3] = 0u;
+            }
+        }
+        // later sub-blocks: w_b -= sum_t E_t U[32 p + t, sub-block b] (+ GPTAQ term)
+        if (nblk > 1) {
+#pragma unroll 2
+            for (int t = 0; t < 32; ++t) {
+                const float et = Es[t * SW_T + tid];
+                const float2 ne = make_float2(-et, -et);
+                float2 vv = make_float2(0.f, 0.f);
+                if (GPTAQ) {
+                    const float vt = Vs[t * SW_T + tid];
+                    vv = make_float2(vt, vt);
+                }
+#pragma unroll
+                for (int b = 1; b < 4; ++b) {
+                    if (b >= nblk) break;
+                    const float *ur = Up + b * 1024 + t * 32;
+                    const float *pr = Pp + b * 1024 + t * 32;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float4 u = *reinterpret_cast<const float4 *>(ur + 4 * i);
+                        w[b][2 * i] = ffma2(ne, make_float2(u.x, u.y), w[b][2 * i]);
+                        w[b][2 * i + 1] = ffma2(ne, make_float2(u.z, u.w), w[b][2 * i + 1]);
+                        if (GPTAQ) {
+                            const float4 q = *reinterpret_cast<const float4 *>(pr + 4 * i);
+                            w[b][2 * i] = ffma2(vv, make_float2(q.x, q.y), w[b][2 * i]);
+                            w[b][2 * i + 1] = ffma2(vv, make_float2(q.z, q.w), w[b][2 * i + 1]);
+                        }
+                    }
+                }
             }
         }
         // the next sub-block becomes w[0]
@@ -370,8 +559,11 @@ size_t quantize_workspace(int K, int N, int g, int blocksize) {
     return round_up(c.off, 256);
 }
 
-static size_t sweep_smem(bool gptaq) {
-    return sizeof(float) * (10 * 1024 * (gptaq ? 2 : 1) + SW_MAXB);
+static size_t sweep_thread_smem(bool gptaq) {
+    return sizeof(float) * ((10 * 1024 + 32 * SW_T) * (gptaq ? 2 : 1) + SW_MAXB);
+}
+static size_t sweep_lanes_smem(bool gptaq) {
+    return sizeof(float) * (10 * 1024 * (gptaq ? 2 : 1) + 32 * 33 + SW_MAXB);
 }
 
 gptq_status quantize_layer(void *W, int wdtype, int N, int K, const float *U, int groups, int bits,
@@ -439,9 +631,14 @@ gptq_status quantize_layer(void *W, int wdtype, int N, int K, const float *U, in
     base.neg[0] = 1;
     base.neg[1] = 0;
 
-    const dim3 grid((per_group + SW_T - 1) / SW_T, groups);
-    auto kern = gptaq ? k_sweep_block<true> : k_sweep_block<false>;
-    const size_t smem = sweep_smem(gptaq);
+    // one thread per channel when that still gives every SM two warps; otherwise four
+    // lanes per channel
+    const bool per_thread = (int64_t)N >= 2LL * 148 * 32;
+    const int cta = per_thread ? SW_T : 128;
+    const dim3 grid((per_group + (per_thread ? SW_T : 32) - 1) / (per_thread ? SW_T : 32), groups);
+    auto kern = per_thread ? (gptaq ? k_sweep_thread<true> : k_sweep_thread<false>)
+                           : (gptaq ? k_sweep_lanes<true> : k_sweep_lanes<false>);
+    const size_t smem = per_thread ? sweep_thread_smem(gptaq) : sweep_lanes_smem(gptaq);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
         return launch_status();
@@ -452,7 +649,7 @@ gptq_status quantize_layer(void *W, int wdtype, int N, int K, const float *U, in
         for (int i0 = sb0; i0 < sb1; i0 += blocksize) {
             const int i1 = min(i0 + blocksize, sb1);
             const int bs = i1 - i0;
-            kern<<<grid, SW_T, smem, st>>>(Wk, N, per_group, K, i0, bs, U, P1, scale, bits,
+            kern<<<grid, cta, smem, st>>>(Wk, N, per_group, K, i0, bs, U, P1, scale, bits,
                                                 codes, Eh, El, Ph, Pl, lay.ldE, lay.ldG, i0 - sb0,
                                                 loss_acc, vec, status);
             s = launch_status();
