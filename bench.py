@@ -33,10 +33,10 @@ sys.path.insert(0, ROOT)
 
 METRIC = "GPTQ layer-solve ms & weights quantized/s (4096×14336, W3); % of TC/HBM roofline"
 
-# DRAM bytes (read + write) per launch of the dominant kernel, from the ncu capture
-# summarised in profiles/gram_tc_mlp_up_w3_chunk65536.md (same 65,536-token launch).
-# Set to None whenever k_gram_tc changes until it is captured again.
-GRAM_TRAFFIC_BYTES = 1.272892e9 + 0.264233e9
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the dominant
+# kernel, from an ncu capture of the same 65,536-token launch. Set to None whenever
+# k_gram_tc changes until it is captured again.
+GRAM_TRAFFIC_BYTES = 1.586335e9 + 0.500874e9
 UNIT = "weights/s"
 
 
