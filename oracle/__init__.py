@@ -28,4 +28,8 @@ from .gptq_oracle import (  # noqa: F401
     layer_error,
     solve_layer,
     brute_force_best,
+    act_order,
+    static_group_scales,
+    obq_sweep_grouped,
+    replay_row_form_grouped,
 )

@@ -405,3 +405,161 @@ def brute_force_best(H, w, grid):
         elif abs(val - best) <= 1e-12:
             arg.append(tuple(v))
     return best, arg
+
+
+# --------------------------------------------------------------------------------------
+# Input-dimension groups and act-order
+# --------------------------------------------------------------------------------------
+
+def act_order(H):
+    """Processing order of the input coordinates: decreasing Hessian diagonal.
+
+    [GPTQ blog] "Damping 与两个不同的分组参数": act-order reorders the input coordinates
+    by the Hessian diagonal from large to small; it is an ordering heuristic, and the
+    coordinates are restored afterwards. Reading: ties keep the lower index first;
+    the diagonal is the one given (the accumulated H, before the dead fix and the
+    damping, so dead coordinates come last).
+    """
+    d = np.diag(np.asarray(H, dtype=np.float64))
+    return np.array(sorted(range(len(d)), key=lambda k: (-d[k], k)), dtype=np.int64)
+
+
+def static_group_scales(W, bits, groupsize):
+    """Scales of fixed ("static") groups: for channel n and original group g, the
+    symmetric scale of W[n, gG:(g+1)G] as given.
+
+    [GPTQ blog] "Damping 与两个不同的分组参数": the group parameters can be re-estimated
+    during compensation or fixed beforehand as static groups. Reading: fixed groups
+    are the original columns [gG, (g+1)G) and take the min-max symmetric scale of
+    symmetric_scale on them.
+    """
+    W = np.asarray(W, dtype=np.float64)
+    N, K = W.shape
+    ng = (K + groupsize - 1) // groupsize
+    S = np.zeros((N, ng))
+    for g in range(ng):
+        S[:, g], _ = symmetric_scale(W[:, g * groupsize:(g + 1) * groupsize], bits)
+    return S
+
+
+def obq_sweep_grouped(H_d, W, bits, groupsize, static=False, perm=None, C=None):
+    """The explicit OBQ sweep of obq_sweep with input-dimension groups and an order.
+
+    [GPTQ blog] "Damping 与两个不同的分组参数": blocksize organises the computation,
+    groupsize changes the representation: each output channel has one scale per
+    group of input coordinates. Readings:
+      - processing order `perm` (identity when None): coordinate perm[q] is fixed at
+        step q, with H_d and W taken in that order;
+      - re-estimated groups (static=False): the groups are processing positions
+        [gG, (g+1)G); when the sweep enters group g, s[n, g] is the symmetric scale of
+        channel n's current (already compensated) weights on the group's coordinates;
+      - static groups (static=True): s from static_group_scales on W as given, and
+        coordinate k uses its original group k // G at whatever step it is fixed;
+      - afterwards codes and weights are restored to the original coordinate order,
+        with g_idx[k] the group whose scale reconstructs coordinate k.
+    C (optional) is the GPTAQ cross statistic in the original order.
+
+    Returns dict(codes, W_hat, scales, g_idx, loss), all in the original order.
+    """
+    H_d = np.asarray(H_d, dtype=np.float64)
+    W = np.asarray(W, dtype=np.float64)
+    N, K = W.shape
+    order = np.arange(K) if perm is None else np.asarray(perm)
+    G = groupsize
+    ng = (K + G - 1) // G
+    Hp = H_d[np.ix_(order, order)]
+    Wp = W[:, order].copy()
+    Cp = None if C is None else np.asarray(C, dtype=np.float64)[np.ix_(order, order)]
+    S_static = static_group_scales(W, bits, G) if static else None
+    scales = S_static.copy() if static else np.zeros((N, ng))
+    codes_p = np.zeros((N, K))
+    loss = np.zeros(N)
+    P = np.linalg.inv(Hp)
+    for q in range(K):
+        if static:
+            s = S_static[:, order[q] // G]
+        else:
+            if q % G == 0:
+                scales[:, q // G], _ = symmetric_scale(Wp[:, q:q + G], bits)
+            s = scales[:, q // G]
+        w_pre = Wp[:, q].copy()
+        c = quantize_codes(w_pre, s, bits)
+        target = dequantize(c, s, bits)
+        r = w_pre - target
+        p_qq = P[0, 0]
+        Wp[:, q:] -= np.outer(r / p_qq, P[:, 0])
+        Wp[:, q] = target
+        loss += r * r / (2.0 * p_qq)
+        codes_p[:, q] = c
+        if q + 1 < K:
+            P_next = P[1:, 1:] - np.outer(P[1:, 0], P[0, 1:]) / p_qq
+            if Cp is not None:
+                Wp[:, q + 1:] += np.outer(w_pre, Cp[q, q + 1:] @ P_next)
+            P = P_next
+    codes = np.zeros((N, K))
+    W_hat = np.zeros((N, K))
+    codes[:, order] = codes_p
+    W_hat[:, order] = Wp
+    inv = np.empty(K, dtype=np.int64)
+    inv[order] = np.arange(K)
+    g_idx = (np.arange(K) // G) if static else (inv // G)
+    return dict(codes=codes, W_hat=W_hat, scales=scales, g_idx=g_idx, loss=loss)
+
+
+def replay_row_form_grouped(U, W, bits, groupsize, codes_gpu, static=False, perm=None,
+                            static_scales=None, band=1e-4):
+    """Tie-follow replay (as replay_row_form) of the row-form sweep with groups and an
+    order, against another run's codes given in the original order.
+
+    U is the factor of H_d in processing order (U^T U = (H_d[perm][:, perm])^-1). The
+    scales follow obq_sweep_grouped's rules along the replayed trajectory (static
+    scales may be passed in, e.g. the other run's, to replay its decisions exactly).
+    Returns dict(codes, W_hat, scales, g_idx, tie_flips, mismatches) in the original
+    order.
+    """
+    U = np.asarray(U, dtype=np.float64)
+    W = np.asarray(W, dtype=np.float64)
+    N, K = W.shape
+    order = np.arange(K) if perm is None else np.asarray(perm)
+    G = groupsize
+    ng = (K + G - 1) // G
+    Wp = W[:, order].copy()
+    Gc = np.asarray(codes_gpu, dtype=np.float64)[:, order]
+    if static:
+        S = static_group_scales(W, bits, G) if static_scales is None else np.asarray(static_scales, dtype=np.float64)
+    else:
+        S = np.zeros((N, ng))
+    z = 2 ** (bits - 1)
+    codes_p = np.zeros((N, K))
+    tie_flips = mismatches = 0
+    for j in range(K):
+        if static:
+            s = S[:, order[j] // G]
+        else:
+            if j % G == 0:
+                S[:, j // G], _ = symmetric_scale(Wp[:, j:j + G], bits)
+            s = S[:, j // G]
+        w = Wp[:, j].copy()
+        c = quantize_codes(w, s, bits)
+        diff = c != Gc[:, j]
+        if np.any(diff):
+            ratio = w[diff] / s[diff]
+            frac_dist = np.abs(np.abs(ratio - np.floor(ratio)) - 0.5)
+            tie = (np.abs(c[diff] - Gc[diff, j]) == 1) & (frac_dist < band)
+            tie_flips += int(np.count_nonzero(tie))
+            mismatches += int(np.count_nonzero(~tie))
+            c = np.where(diff, Gc[:, j], c)
+        target = s * (c - z)
+        e = (w - target) / U[j, j]
+        Wp[:, j:] -= np.outer(e, U[j, j:])
+        Wp[:, j] = target
+        codes_p[:, j] = c
+    codes = np.zeros((N, K))
+    W_hat = np.zeros((N, K))
+    codes[:, order] = codes_p
+    W_hat[:, order] = Wp
+    inv = np.empty(K, dtype=np.int64)
+    inv[order] = np.arange(K)
+    g_idx = (np.arange(K) // G) if static else (inv // G)
+    return dict(codes=codes, W_hat=W_hat, scales=S, g_idx=g_idx, tie_flips=tie_flips,
+                mismatches=mismatches)

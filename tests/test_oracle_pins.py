@@ -362,3 +362,111 @@ def test_replay_counts_flips_without_cascade():
     rep = O.replay_row_form(U, W, s, 3, other)
     assert rep["mismatches"] == 1 and rep["tie_flips"] == 0
     np.testing.assert_array_equal(rep["codes"], other)
+
+
+# ------------------------------------------------------------ input groups and act-order
+
+def _problem(K, N, seed, M=None):
+    rng = np.random.default_rng(seed)
+    M = M or 4 * K
+    X = rng.standard_normal((M, K)) @ rng.standard_normal((K, K)) * 0.5
+    W = rng.standard_normal((N, K)) * 0.1
+    Hd, _ = O.dead_and_damp(O.gram(X), 0.01)
+    return Hd, W
+
+
+def test_act_order_example():
+    # diagonal (1, 3, 3, 2): 3 before 3 by index, then 2, then 1
+    H = np.diag([1.0, 3.0, 3.0, 2.0])
+    np.testing.assert_array_equal(O.act_order(H), [1, 2, 3, 0])
+    # a dead coordinate (zero diagonal) comes last
+    np.testing.assert_array_equal(O.act_order(np.diag([0.0, 5.0, 1.0])), [1, 2, 0])
+
+
+def test_one_group_is_per_channel_gptq():
+    # a single group spanning every coordinate, natural order: the per-channel sweep
+    Hd, W = _problem(12, 5, 1)
+    s, _ = O.symmetric_scale(W, 3)
+    c0, W0, l0 = O.obq_sweep(Hd, W, s, 3)
+    r = O.obq_sweep_grouped(Hd, W, 3, groupsize=12)
+    np.testing.assert_array_equal(r["codes"], c0)
+    np.testing.assert_allclose(r["W_hat"], W0, atol=1e-12)
+    np.testing.assert_allclose(r["scales"][:, 0], s, rtol=1e-15)
+    np.testing.assert_allclose(r["loss"], l0, rtol=1e-12)
+
+
+@pytest.mark.parametrize("static", [False, True])
+def test_diagonal_hessian_is_group_rtn(static):
+    # no coupling between coordinates: every coordinate is rounded with its group's
+    # scale taken from W as given (nothing is compensated before a group is entered)
+    rng = np.random.default_rng(2)
+    K, N, G, bits = 16, 6, 4, 2
+    Hd = np.diag(rng.uniform(0.5, 2.0, K))
+    W = rng.standard_normal((N, K))
+    perm = O.act_order(Hd)
+    r = O.obq_sweep_grouped(Hd, W, bits, G, static=static, perm=perm)
+    expect = np.zeros((N, K))
+    for g in range(K // G):
+        cols = (np.arange(g * G, (g + 1) * G) if static else perm[g * G:(g + 1) * G])
+        amax = np.max(np.abs(W[:, cols]), axis=1)
+        s = 2 * amax / (2 ** bits - 1)
+        expect[:, cols] = np.clip(np.rint(W[:, cols] / s[:, None]) + 2 ** (bits - 1), 0, 2 ** bits - 1)
+    np.testing.assert_array_equal(r["codes"], expect)
+    z = 2 ** (bits - 1)
+    np.testing.assert_allclose(r["W_hat"], r["scales"][np.arange(N)[:, None], r["g_idx"][None, :]]
+                               * (r["codes"] - z), atol=1e-15)
+
+
+def test_sorted_diagonal_act_order_is_natural_order():
+    Hd, W = _problem(10, 4, 3)
+    order = np.argsort(-np.diag(Hd), kind="stable")
+    Hs = Hd[np.ix_(order, order)]
+    Ws = W[:, order]
+    assert np.all(np.diff(np.diag(Hs)) <= 0)
+    a = O.obq_sweep_grouped(Hs, Ws, 3, 5, perm=O.act_order(Hs))
+    b = O.obq_sweep_grouped(Hs, Ws, 3, 5)
+    np.testing.assert_array_equal(a["codes"], b["codes"])
+    np.testing.assert_allclose(a["W_hat"], b["W_hat"], atol=1e-12)
+
+
+@pytest.mark.parametrize("static", [False])
+def test_act_order_is_permutation_equivariant(static):
+    # relabelling the input coordinates does not change what act-order computes with
+    # re-estimated groups (static groups are tied to the original column labels)
+    Hd, W = _problem(12, 5, 4)
+    rng = np.random.default_rng(5)
+    Q = rng.permutation(12)
+    Hq, Wq = Hd[np.ix_(Q, Q)], W[:, Q]
+    G = 4
+    a = O.obq_sweep_grouped(Hd, W, 3, G, static=static, perm=O.act_order(Hd))
+    b = O.obq_sweep_grouped(Hq, Wq, 3, G, static=static, perm=O.act_order(Hq))
+    np.testing.assert_array_equal(b["codes"], a["codes"][:, Q])
+    np.testing.assert_allclose(b["W_hat"], a["W_hat"][:, Q], atol=1e-12)
+    if not static:   # dynamic groups follow the processing order, itself equivariant
+        np.testing.assert_allclose(b["scales"], a["scales"], rtol=1e-12)
+
+
+@pytest.mark.parametrize("static", [False, True])
+def test_grouped_row_form_matches_explicit(static):
+    # the Cholesky row form with U of the reordered H_d reproduces the explicit
+    # Schur-updated sweep, group scales included
+    Hd, W = _problem(16, 6, 6)
+    perm = O.act_order(Hd)
+    G = 8
+    r = O.obq_sweep_grouped(Hd, W, 3, G, static=static, perm=perm)
+    U = O.upper_factor(Hd[np.ix_(perm, perm)])
+    rep = O.replay_row_form_grouped(U, W, 3, G, r["codes"], static=static, perm=perm)
+    assert rep["mismatches"] == 0 and rep["tie_flips"] == 0
+    np.testing.assert_allclose(rep["W_hat"], r["W_hat"], atol=1e-9)
+    np.testing.assert_allclose(rep["scales"], r["scales"], rtol=1e-9)
+    np.testing.assert_array_equal(rep["g_idx"], r["g_idx"])
+
+
+def test_reestimated_groups_see_compensation():
+    # the first group's scale is the same either way; a later group's re-estimated
+    # scale is taken from compensated weights and differs from the static one
+    Hd, W = _problem(12, 5, 7)
+    a = O.obq_sweep_grouped(Hd, W, 2, 4, static=False)
+    b = O.obq_sweep_grouped(Hd, W, 2, 4, static=True)
+    np.testing.assert_allclose(a["scales"][:, 0], b["scales"][:, 0], rtol=1e-15)
+    assert np.max(np.abs(a["scales"][:, 1:] - b["scales"][:, 1:])) > 1e-6
