@@ -231,11 +231,17 @@ def run_ours(args, rank, world, local_rank):
     C = torch.empty(K, K, device=dev) if wl.gptaq else None
     P1 = torch.empty(K, K, device=dev) if wl.gptaq else None
     codes = torch.empty(N, K, dtype=torch.uint8, device=dev)
-    scales = torch.empty(N, device=dev)
+    grouped = wl.groupsize > 0 or wl.act_order
+    scales = (torch.empty(N, (K + wl.groupsize - 1) // wl.groupsize, device=dev) if wl.groupsize
+              else torch.empty(N, device=dev))
+    g_idx = torch.empty(K, dtype=torch.int32, device=dev) if grouped else None
+    perm = torch.empty(K, dtype=torch.int32, device=dev) if wl.act_order else None
+    Hp = torch.empty(K, K, device=dev) if wl.act_order else None
     status = gq.new_status(dev)
     ws_p = torch.empty(gq.gptq_workspace_size(gq.GPTQ_OP_PREPARE, K, 0, g, 0), dtype=torch.uint8,
                        device=dev)
-    ws_q = torch.empty(gq.gptq_workspace_size(gq.GPTQ_OP_QUANTIZE, K, N, g, wl.blocksize),
+    ws_q = torch.empty(gq.gptq_workspace_size(gq.GPTQ_OP_QUANTIZE_GROUPED if grouped
+                                              else gq.GPTQ_OP_QUANTIZE, K, N, g, wl.blocksize),
                        dtype=torch.uint8, device=dev)
     ws_r = (torch.empty(gq.gptq_workspace_size(gq.GPTQ_OP_RESIDUAL, K, 0, 1, 0), dtype=torch.uint8,
                         device=dev) if wl.gptaq else None)
@@ -261,12 +267,23 @@ def run_ours(args, rank, world, local_rank):
                 gq.gptaq_accumulate_cross(C, Xf[c * ch:(c + 1) * ch], X[c * ch:(c + 1) * ch],
                                           status=status, stream=stream)
         ev[1].record(stream)
-        gq.gptq_prepare(H, wl.percdamp, workspace=ws_p, status=status, stream=stream)
+        Hs = H
+        if perm is not None:            # act-order: solve in the reordered coordinates
+            gq.gptq_act_order(H, perm=perm, stream=stream)
+            Hs = gq.gptq_permute_hessian(H, perm, out=Hp, stream=stream)
+        gq.gptq_prepare(Hs, wl.percdamp, workspace=ws_p, status=status, stream=stream)
         if P1 is not None:
-            gq.gptaq_residual(P1, C, H, workspace=ws_r, stream=stream)
+            gq.gptaq_residual(P1, C, Hs, workspace=ws_r, stream=stream)
         ev[2].record(stream)
-        gq.gptq_quantize_layer(W, H, wl.bits, wl.blocksize, groups=g, P1=P1, scales_out=scales,
-                               codes=codes, workspace=ws_q, status=status, stream=stream)
+        if grouped:
+            gq.gptq_quantize_layer_grouped(W, Hs, wl.bits, wl.blocksize, wl.groupsize,
+                                           static_groups=wl.static_groups, perm=perm, P1=P1,
+                                           scales_out=scales, g_idx=g_idx, codes=codes,
+                                           workspace=ws_q, status=status, stream=stream)
+        else:
+            gq.gptq_quantize_layer(W, Hs, wl.bits, wl.blocksize, groups=g, P1=P1,
+                                   scales_out=scales, codes=codes, workspace=ws_q, status=status,
+                                   stream=stream)
         ev[3].record(stream)
         return ev
 
@@ -372,7 +389,12 @@ def run_e2e(args, wl, X, W, dev, gq, torch, dist, world):
     Wd = torch.empty_like(W)
     H = torch.empty(K, K, device=dev)
     codes = torch.empty(N, K, dtype=torch.uint8, device=dev)
-    scales = torch.empty(N, device=dev)
+    grouped = wl.groupsize > 0 or wl.act_order
+    scales = (torch.empty(N, (K + wl.groupsize - 1) // wl.groupsize, device=dev) if wl.groupsize
+              else torch.empty(N, device=dev))
+    g_idx = torch.empty(K, dtype=torch.int32, device=dev) if grouped else None
+    perm = torch.empty(K, dtype=torch.int32, device=dev) if wl.act_order else None
+    Hp = torch.empty(K, K, device=dev) if wl.act_order else None
     status = gq.new_status(dev)
     ws_p = torch.empty(gq.gptq_workspace_size(gq.GPTQ_OP_PREPARE, K, 0, 1, 0), dtype=torch.uint8,
                        device=dev)

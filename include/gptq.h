@@ -68,7 +68,8 @@ typedef enum { GPTQ_BF16 = 0, GPTQ_F32 = 1 } gptq_dtype;
 typedef enum {
     GPTQ_OP_PREPARE = 0,
     GPTQ_OP_RESIDUAL = 1,
-    GPTQ_OP_QUANTIZE = 2
+    GPTQ_OP_QUANTIZE = 2,
+    GPTQ_OP_QUANTIZE_GROUPED = 3
 } gptq_op;
 
 /*
@@ -221,6 +222,72 @@ GPTQ_API gptq_status gptq_quantize_layer(void *W, int wdtype, int N, int K, cons
                                 const float *scales_in, float *scales_out, uint8_t *codes,
                                 float *loss, int write_back, void *ws, size_t ws_bytes,
                                 int32_t *status, void *stream);
+
+/*
+ * gptq_act_order -- the act-order processing order of the input coordinates.
+ *
+ * [GPTQ blog] "Damping 与两个不同的分组参数": act-order processes the input
+ * coordinates by the Hessian diagonal from large to small; they are restored after
+ * quantisation. perm[q] is the coordinate fixed at step q: decreasing H_kk, ties by
+ * lower index. Call it on the accumulated H (before gptq_prepare), so dead
+ * coordinates (H_kk = 0) come last.
+ *
+ *   H     device fp32 [K][K] (read).
+ *   perm  device int32 [K] (written).
+ *   Errors: GPTQ_ERR_ARG for K out of range or NULL pointers.
+ */
+GPTQ_API gptq_status gptq_act_order(const float *H, int K, int32_t *perm, void *stream);
+
+/*
+ * gptq_permute_hessian -- out[i][j] = H[perm[i]][perm[j]] (K x K fp32, out of place):
+ * the Hessian (or the GPTAQ cross statistic C) in the processing order, for
+ * gptq_prepare / gptaq_residual ahead of an ordered quantisation.
+ *
+ *   out, H  device fp32 [K][K], distinct buffers.  perm  device int32 [K].
+ */
+GPTQ_API gptq_status gptq_permute_hessian(float *out, const float *H, int K, const int32_t *perm,
+                                          void *stream);
+
+/*
+ * gptq_quantize_layer_grouped -- gptq_quantize_layer with input-dimension groups and
+ * an optional processing order (one Hessian, groups == 1).
+ *
+ * [GPTQ blog] "Damping 与两个不同的分组参数": blocksize organises the computation,
+ * groupsize changes the representation: each output channel takes one scale per
+ * group of input coordinates; the group parameters are either re-estimated during
+ * compensation or fixed beforehand (static groups); with act-order the coordinates,
+ * the group index and the permutation are restored consistently.
+ *   - static_groups == 0: groups are processing positions [gG, (g+1)G); when the
+ *     sweep enters group g, s[n][g] = 2 max |w| / (2^b - 1) over channel n's current
+ *     (already compensated) weights of the group.
+ *   - static_groups != 0: groups are the original columns [gG, (g+1)G) and s[n][g] is
+ *     taken from W as given before the sweep.
+ * Reconstruction: W_hat[n][k] = scales_out[n][g_idx[k]] * (codes[n][k] - z).
+ *
+ *   U          device fp32 [K][K] from gptq_prepare on the Hessian in processing
+ *              order (gptq_permute_hessian with perm), or on H itself when perm is
+ *              NULL.
+ *   groupsize  32, 64 or 128, dividing blocksize (blocksize 32, 64 or 128); or 0 for
+ *              one per-channel scale (gptq_quantize_layer's) with the order of perm.
+ *   perm       device int32 [K] processing order (gptq_act_order), or NULL (natural).
+ *   P1         device fp32 [K][K] from gptaq_residual in processing order, or NULL.
+ *   dead       device uint8 [K] in processing order (gptq_prepare's dead_out), or NULL.
+ *   scales_out device fp32 [N][ceil(K / groupsize)] ([N] when groupsize == 0), or NULL.
+ *   g_idx_out  device int32 [K] group of each original coordinate (0 when
+ *              groupsize == 0), or NULL.
+ *   codes      device uint8 [N][K] in the original coordinate order (required).
+ *   W, bits, loss, write_back, status: as gptq_quantize_layer (write-back in the
+ *              original order).
+ *   ws         gptq_workspace_size(GPTQ_OP_QUANTIZE_GROUPED, K, N, 1, blocksize) bytes.
+ */
+GPTQ_API gptq_status gptq_quantize_layer_grouped(void *W, int wdtype, int N, int K, const float *U,
+                                                 int bits, int blocksize, int groupsize,
+                                                 int static_groups, const int32_t *perm,
+                                                 const float *P1, const uint8_t *dead,
+                                                 float *scales_out, int32_t *g_idx_out,
+                                                 uint8_t *codes, float *loss, int write_back,
+                                                 void *ws, size_t ws_bytes, int32_t *status,
+                                                 void *stream);
 
 /* Workspace bytes for an operation (gptq_op); 0 when none is needed. */
 GPTQ_API size_t gptq_workspace_size(int op, int K, int N, int g, int blocksize);

@@ -19,11 +19,12 @@ LIB_PATH = os.path.join(_HERE, "libgptq.so")
 GPTQ_OK, GPTQ_ERR_ARG, GPTQ_ERR_NOT_PD, GPTQ_ERR_NONFINITE = 0, 1, 2, 3
 GPTQ_ERR_CUDA, GPTQ_ERR_TIMEOUT, GPTQ_ERR_WORKSPACE = 4, 5, 6
 GPTQ_BF16, GPTQ_F32 = 0, 1
-GPTQ_OP_PREPARE, GPTQ_OP_RESIDUAL, GPTQ_OP_QUANTIZE = 0, 1, 2
+GPTQ_OP_PREPARE, GPTQ_OP_RESIDUAL, GPTQ_OP_QUANTIZE, GPTQ_OP_QUANTIZE_GROUPED = 0, 1, 2, 3
 
 EXPORTS = ("gptq_accumulate_hessian", "gptaq_accumulate_cross", "gptq_prepare",
            "gptq_prepare_noalloc",
-           "gptaq_residual", "gptq_quantize_layer", "gptq_workspace_size",
+           "gptaq_residual", "gptq_quantize_layer", "gptq_act_order", "gptq_permute_hessian",
+           "gptq_quantize_layer_grouped", "gptq_workspace_size",
            "gptq_kernel_launches", "gptq_status_string")
 
 _lib = None
@@ -52,6 +53,10 @@ def load_library():
         "gptq_prepare_noalloc": [P, I, I, F, P, P, P],
         "gptaq_residual": [P, P, P, I, P, SZ, P],
         "gptq_quantize_layer": [P, I, I, I, P, I, I, I, P, P, P, P, P, P, I, P, SZ, P, P],
+        "gptq_act_order": [P, I, P, P],
+        "gptq_permute_hessian": [P, P, I, P, P],
+        "gptq_quantize_layer_grouped": [P, I, I, I, P, I, I, I, I, P, P, P, P, P, P, P, I, P, SZ,
+                                        P, P],
         "gptq_workspace_size": [I, I, I, I, I],
         "gptq_status_string": [I],
         "gptq_kernel_launches": [],
@@ -198,3 +203,52 @@ def gptq_quantize_layer(W, U, bits, blocksize=128, groups=1, P1=None, dead=None,
                                    _stream(stream))
     _check(code, "gptq_quantize_layer")
     return codes, status
+
+
+def gptq_act_order(H, perm=None, stream=None):
+    """The act-order processing order of H's input coordinates (int32 [K])."""
+    lib = load_library()
+    K = H.shape[-1]
+    if perm is None:
+        perm = torch.empty(K, dtype=torch.int32, device=H.device)
+    _check(lib.gptq_act_order(_ptr(H), K, _ptr(perm), _stream(stream)), "gptq_act_order")
+    return perm
+
+
+def gptq_permute_hessian(H, perm, out=None, stream=None):
+    """out = H[perm][:, perm] (a new K x K tensor unless `out` is given)."""
+    lib = load_library()
+    K = H.shape[-1]
+    if out is None:
+        out = torch.empty_like(H)
+    _check(lib.gptq_permute_hessian(_ptr(out), _ptr(H), K, _ptr(perm), _stream(stream)),
+           "gptq_permute_hessian")
+    return out
+
+
+def gptq_quantize_layer_grouped(W, U, bits, blocksize=128, groupsize=128, static_groups=False,
+                                perm=None, P1=None, dead=None, scales_out=None, g_idx=None,
+                                codes=None, loss=None, write_back=False, workspace=None,
+                                status=None, stream=None):
+    """The sweep with input-dimension groups and an optional processing order.
+    Returns (codes, scales [N][ceil(K / groupsize)], g_idx [K], status); see include/gptq.h."""
+    lib = load_library()
+    N, K = W.shape
+    if codes is None:
+        codes = torch.empty(N, K, dtype=torch.uint8, device=W.device)
+    if scales_out is None:
+        shape = (N, (K + groupsize - 1) // groupsize) if groupsize else (N,)
+        scales_out = torch.empty(shape, dtype=torch.float32, device=W.device)
+    if g_idx is None:
+        g_idx = torch.empty(K, dtype=torch.int32, device=W.device)
+    status = new_status(W.device) if status is None else status
+    ws = _workspace(gptq_workspace_size(GPTQ_OP_QUANTIZE_GROUPED, K, N, 1, blocksize), W.device,
+                    workspace)
+    code = lib.gptq_quantize_layer_grouped(_ptr(W), _dtype_code(W), N, K, _ptr(U), bits, blocksize,
+                                           groupsize, int(bool(static_groups)), _ptr(perm),
+                                           _ptr(P1), _ptr(dead), _ptr(scales_out), _ptr(g_idx),
+                                           _ptr(codes), _ptr(loss), int(write_back), _ptr(ws),
+                                           ws.numel() * ws.element_size(), _ptr(status),
+                                           _stream(stream))
+    _check(code, "gptq_quantize_layer_grouped")
+    return codes, scales_out, g_idx, status

@@ -24,6 +24,15 @@ gptq_status quantize_layer(void *W, int wdtype, int N, int K, const float *U, in
                            int blocksize, const float *P1, const uint8_t *dead,
                            const float *scales_in, float *scales_out, uint8_t *codes, float *loss,
                            int write_back, void *ws, int32_t *status, cudaStream_t st);
+size_t quantize_grouped_workspace(int K, int N, int blocksize);
+gptq_status quantize_layer_grouped(void *W, int wdtype, int N, int K, const float *U, int bits,
+                                   int blocksize, int groupsize, int static_groups,
+                                   const int32_t *perm, const float *P1, const uint8_t *dead,
+                                   float *scales_out, int32_t *g_idx, uint8_t *codes, float *loss,
+                                   int write_back, void *ws, int32_t *status, cudaStream_t st);
+gptq_status act_order(const float *H, int K, int32_t *perm, cudaStream_t st);
+gptq_status permute_square(float *out, const float *H, int K, const int32_t *perm,
+                           cudaStream_t st);
 }  // namespace gptq
 
 namespace gptq {
@@ -120,6 +129,37 @@ gptq_status gptq_quantize_layer(void *W, int wdtype, int N, int K, const float *
                           static_cast<cudaStream_t>(stream));
 }
 
+gptq_status gptq_act_order(const float *H, int K, int32_t *perm, void *stream) {
+    if (K < 1 || K > GPTQ_MAX_DIM || !H || !perm) return GPTQ_ERR_ARG;
+    return act_order(H, K, perm, static_cast<cudaStream_t>(stream));
+}
+
+gptq_status gptq_permute_hessian(float *out, const float *H, int K, const int32_t *perm,
+                                 void *stream) {
+    if (K < 1 || K > GPTQ_MAX_DIM || !out || !H || !perm || out == H) return GPTQ_ERR_ARG;
+    return permute_square(out, H, K, perm, static_cast<cudaStream_t>(stream));
+}
+
+gptq_status gptq_quantize_layer_grouped(void *W, int wdtype, int N, int K, const float *U,
+                                        int bits, int blocksize, int groupsize, int static_groups,
+                                        const int32_t *perm, const float *P1, const uint8_t *dead,
+                                        float *scales_out, int32_t *g_idx_out, uint8_t *codes,
+                                        float *loss, int write_back, void *ws, size_t ws_bytes,
+                                        int32_t *status, void *stream) {
+    if (N < 1 || K < 1 || !W || !U || !codes || !status) return GPTQ_ERR_ARG;
+    if (N > GPTQ_MAX_DIM || K > GPTQ_MAX_DIM || !valid_dtype(wdtype)) return GPTQ_ERR_ARG;
+    if (bits != 2 && bits != 3 && bits != 4 && bits != 8) return GPTQ_ERR_ARG;
+    if (groupsize != 0 && groupsize != 32 && groupsize != 64 && groupsize != 128) return GPTQ_ERR_ARG;
+    if (blocksize != 32 && blocksize != 64 && blocksize != 128) return GPTQ_ERR_ARG;
+    if (groupsize && blocksize % groupsize != 0) return GPTQ_ERR_ARG;
+    if (!aligned(U, 16) || (P1 && !aligned(P1, 16))) return GPTQ_ERR_ARG;
+    if (!ws || !aligned(ws, 256) || ws_bytes < quantize_grouped_workspace(K, N, blocksize))
+        return GPTQ_ERR_WORKSPACE;
+    return quantize_layer_grouped(W, wdtype, N, K, U, bits, blocksize, groupsize, static_groups,
+                                  perm, P1, dead, scales_out, g_idx_out, codes, loss, write_back,
+                                  ws, status, static_cast<cudaStream_t>(stream));
+}
+
 size_t gptq_workspace_size(int op, int K, int N, int g, int blocksize) {
     if (K < 1 || g < 1) return 0;
     switch (op) {
@@ -128,6 +168,9 @@ size_t gptq_workspace_size(int op, int K, int N, int g, int blocksize) {
         case GPTQ_OP_QUANTIZE:
             if (N < 1 || blocksize < 1) return 0;
             return quantize_workspace(K, N, g, blocksize);
+        case GPTQ_OP_QUANTIZE_GROUPED:
+            if (N < 1 || blocksize < 1) return 0;
+            return quantize_grouped_workspace(K, N, blocksize);
         default: return 0;
     }
 }

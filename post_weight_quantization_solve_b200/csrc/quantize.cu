@@ -61,14 +61,21 @@ __global__ void __launch_bounds__(256) k_scale_init(const T *__restrict__ W, flo
                                                     const float *__restrict__ scales_in,
                                                     float *__restrict__ scale, float *scales_out,
                                                     float *__restrict__ loss_acc, int vec,
-                                                    int32_t *status) {
+                                                    int32_t *status, const int32_t *perm) {
     const int n = blockIdx.x;
     const T *wr = W + (int64_t)n * K;
     float *kr = Wk + (int64_t)n * K;
     const uint8_t *dg = dead ? dead + (int64_t)(n / per_group) * K : nullptr;
     float amax = 0.f;
     bool bad = false;
-    if (vec) {   // rows 16-byte aligned for both W and Wk, K % 8 == 0
+    if (perm) {  // working copy in processing order: Wk[n][j] = W[n][perm[j]]
+        for (int k = threadIdx.x; k < K; k += 256) {
+            const float x = to_f32(wr[perm[k]]);
+            bad |= !isfinite(x);
+            amax = fmaxf(amax, fabsf(x));
+            kr[k] = (dg && dg[k]) ? 0.f : x;
+        }
+    } else if (vec) {   // rows 16-byte aligned for both W and Wk, K % 8 == 0
         for (int k = threadIdx.x * 8; k < K; k += 256 * 8) {
             float x[8];
             load8(wr + k, x);
@@ -118,6 +125,16 @@ __global__ void __launch_bounds__(256) k_scale_init(const T *__restrict__ W, flo
     }
 }
 
+// Input-dimension groups seen by the sweep: mode 0 per-channel scale, 1 re-estimated
+// at group entry (written to gsc), 2 static (read from gsc); gsc is [N][ldg], gsel[j]
+// the group of processing position j.
+struct SweepGroups {
+    int G;
+    float *gsc;
+    int ldg;
+    const int32_t *gsel;
+};
+
 // 16-byte global -> shared copy that bypasses registers; src_bytes = 0 writes zeros.
 __device__ __forceinline__ void cp_async16(void *dst, const void *src, int src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
@@ -141,13 +158,14 @@ __device__ __forceinline__ void cp_async_wait_all() {
 // always w[0]: the register array shifts by one sub-block after each phase. No block
 // barrier inside the sweep. U[blk, blk] (and P1) is staged once per CTA as its ten
 // 32 x 32 blocks on or above the diagonal.
-template <bool GPTAQ>
+template <bool GPTAQ, int GMODE>
 __global__ void __launch_bounds__(128, GPTAQ ? 2 : 4) k_sweep_lanes(
     float *__restrict__ Wk, int N, int per_group, int K, int i0, int bs,
     const float *__restrict__ U, const float *__restrict__ P1, const float *__restrict__ scale,
     int bits, uint8_t *__restrict__ codes, __nv_bfloat16 *__restrict__ Eh,
     __nv_bfloat16 *__restrict__ El, __nv_bfloat16 *__restrict__ Ph, __nv_bfloat16 *__restrict__ Pl,
-    int ldE, int ldG, int erow0, float *__restrict__ loss_acc, int vec, const int32_t *status) {
+    int ldE, int ldG, int erow0, float *__restrict__ loss_acc, int vec, const int32_t *status,
+    const SweepGroups sg) {
     constexpr int NCH = 32, CLD = 132;
     if (failed(status)) return;
     extern __shared__ __align__(16) unsigned char smem[];
@@ -155,6 +173,8 @@ __global__ void __launch_bounds__(128, GPTAQ ? 2 : 4) k_sweep_lanes(
     float *Ps = Us + 10 * 1024;                                  // GPTAQ only
     uint8_t *Cs = reinterpret_cast<uint8_t *>(Ps + (GPTAQ ? 10 * 1024 : 0));  // [NCH][CLD]
     float *rpiv = reinterpret_cast<float *>(Cs + NCH * CLD);    // [SW_MAXB]
+    float *sS = rpiv + SW_MAXB;                                  // static groups: [SW_MAXB][NCH]
+    float *sR = sS + SW_MAXB * NCH;                              // and 1 / s
 
     const int grp = blockIdx.y;
     const int cta_ch0 = blockIdx.x * NCH;
@@ -210,11 +230,18 @@ __global__ void __launch_bounds__(128, GPTAQ ? 2 : 4) k_sweep_lanes(
             for (int i = 0; i < 8; ++i) w[b][i] = (valid && c0 + i < bs) ? src[i] : 0.f;
         }
     }
+    if (GMODE == 2) {
+        for (int j = q; j < bs; j += 4) {
+            const float sj = valid ? sg.gsc[n * sg.ldg + sg.gsel[i0 + j]] : 1.f;
+            sS[j * NCH + ch] = sj;
+            sR[j * NCH + ch] = 1.f / sj;
+        }
+    }
     cp_async_wait_all();
     __syncthreads();
 
-    const float s = valid ? scale[n] : 1.f;
-    const float rs = 1.f / s;
+    float s = valid ? scale[n] : 1.f;
+    float rs = 1.f / s;
     const float zf = (float)(1 << (bits - 1));
     const float cmin = -zf, cmax = (float)((1 << bits) - 1) - zf;
     const int gsrc = lane & ~3;
@@ -226,14 +253,30 @@ __global__ void __launch_bounds__(128, GPTAQ ? 2 : 4) k_sweep_lanes(
     for (int p = 0; p < nsb; ++p) {
         const int bbase = p * 4 - p * (p - 1) / 2;       // block (p, p)
         int64_t eoff = (int64_t)(erow0 + 32 * p) * ldE + ecol;
+        if (GMODE == 1 && (i0 + 32 * p) % sg.G == 0) {
+            // entering a group: its scale from the channel's current weights
+            float a = 0.f;
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+                if (32 * b < sg.G)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(w[b][i]));
+            a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+            a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+            s = a == 0.f ? 1.f : 2.f * a / (cmax - cmin);
+            rs = 1.f / s;
+            if (valid && q == 0) sg.gsc[n * sg.ldg + (i0 + 32 * p) / sg.G] = s;
+        }
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
             const int j = 32 * p + t;
             const int oq = t >> 3, oi = t & 7;
             const bool live = j < bs;
+            const float sj = GMODE == 2 ? sS[j * NCH + ch] : s;
+            const float rsj = GMODE == 2 ? sR[j * NCH + ch] : rs;
             const float wj = w[0][oi];
-            const float cf = fminf(fmaxf(rintf(wj * rs), cmin), cmax);
-            const float ej = live ? fmaf(-s, cf, wj) * rpiv[j] : 0.f;
+            const float cf = fminf(fmaxf(rintf(wj * rsj), cmin), cmax);
+            const float ej = live ? fmaf(-sj, cf, wj) * rpiv[j] : 0.f;
             const float e = __shfl_sync(0xffffffffu, ej, gsrc | oq);
             float v = 0.f;
             if (GPTAQ) v = __shfl_sync(0xffffffffu, live ? wj : 0.f, gsrc | oq);
@@ -308,13 +351,14 @@ __global__ void __launch_bounds__(128, GPTAQ ? 2 : 4) k_sweep_lanes(
 // is staged once per CTA as its ten 32 x 32 blocks on or above the diagonal.
 constexpr int SW_T = 64;
 
-template <bool GPTAQ>
+template <bool GPTAQ, int GMODE>
 __global__ void __launch_bounds__(SW_T, 1) k_sweep_thread(
     float *__restrict__ Wk, int N, int per_group, int K, int i0, int bs,
     const float *__restrict__ U, const float *__restrict__ P1, const float *__restrict__ scale,
     int bits, uint8_t *__restrict__ codes, __nv_bfloat16 *__restrict__ Eh,
     __nv_bfloat16 *__restrict__ El, __nv_bfloat16 *__restrict__ Ph, __nv_bfloat16 *__restrict__ Pl,
-    int ldE, int ldG, int erow0, float *__restrict__ loss_acc, int vec, const int32_t *status) {
+    int ldE, int ldG, int erow0, float *__restrict__ loss_acc, int vec, const int32_t *status,
+    const SweepGroups sg) {
     if (failed(status)) return;
     extern __shared__ __align__(16) unsigned char smem[];
     float *Us = reinterpret_cast<float *>(smem);                 // [10][32][32]
@@ -322,6 +366,8 @@ __global__ void __launch_bounds__(SW_T, 1) k_sweep_thread(
     float *rpiv = Ps + (GPTAQ ? 10 * 1024 : 0);                  // [SW_MAXB]
     float *Es = rpiv + SW_MAXB;                                  // [32][SW_T] this phase's E
     float *Vs = Es + 32 * SW_T;                                  // GPTAQ: pre-rounding weights
+    float *sS = Vs + (GPTAQ ? 32 * SW_T : 0);                    // static groups: [SW_MAXB][SW_T]
+    float *sR = sS + SW_MAXB * SW_T;                             // and 1 / s
 
     const int grp = blockIdx.y;
     const int cta_ch0 = blockIdx.x * SW_T;
@@ -382,11 +428,18 @@ __global__ void __launch_bounds__(SW_T, 1) k_sweep_thread(
             }
         }
     }
+    if (GMODE == 2) {
+        for (int j = 0; j < bs; ++j) {
+            const float sj = valid ? sg.gsc[n * sg.ldg + sg.gsel[i0 + j]] : 1.f;
+            sS[j * SW_T + tid] = sj;
+            sR[j * SW_T + tid] = 1.f / sj;
+        }
+    }
     cp_async_wait_all();
     __syncthreads();
 
-    const float s = valid ? scale[n] : 1.f;
-    const float rs = 1.f / s;
+    float s = valid ? scale[n] : 1.f;
+    float rs = 1.f / s;
     const float zf = (float)(1 << (bits - 1));
     const float cmin = -zf, cmax = (float)((1 << bits) - 1) - zf;
     float lacc = 0.f;
@@ -402,15 +455,29 @@ __global__ void __launch_bounds__(SW_T, 1) k_sweep_thread(
         const float *Pp = Ps + bbase * 1024;
         int64_t eoff = (int64_t)(erow0 + 32 * p) * ldE + ecol;
         uint32_t cw[4] = {0u, 0u, 0u, 0u};
+        if (GMODE == 1 && (i0 + 32 * p) % sg.G == 0) {
+            // entering a group: its scale from the channel's current weights
+            float a = 0.f;
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+                if (32 * b < sg.G)
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) a = fmaxf(a, fmaxf(fabsf(w[b][i].x), fabsf(w[b][i].y)));
+            s = a == 0.f ? 1.f : 2.f * a / (cmax - cmin);
+            rs = 1.f / s;
+            if (valid) sg.gsc[n * sg.ldg + (i0 + 32 * p) / sg.G] = s;
+        }
         // the 32 steps inside sub-block p; each step's error is kept for the later
         // sub-blocks, which take all 32 at once after the phase
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
             const int j = 32 * p + t;
             const bool live = j < bs;
+            const float sj = GMODE == 2 ? sS[j * SW_T + tid] : s;
+            const float rsj = GMODE == 2 ? sR[j * SW_T + tid] : rs;
             const float wj = (t & 1) ? w[0][t >> 1].y : w[0][t >> 1].x;
-            const float cf = fminf(fmaxf(rintf(wj * rs), cmin), cmax);
-            const float ej = live ? fmaf(-s, cf, wj) * rpiv[j] : 0.f;
+            const float cf = fminf(fmaxf(rintf(wj * rsj), cmin), cmax);
+            const float ej = live ? fmaf(-sj, cf, wj) * rpiv[j] : 0.f;
             const float vj = (GPTAQ && live) ? wj : 0.f;
             Es[t * SW_T + tid] = ej;
             if (GPTAQ) Vs[t * SW_T + tid] = vj;
@@ -494,6 +561,57 @@ __global__ void __launch_bounds__(SW_T, 1) k_sweep_thread(
     if (valid) loss_acc[n] += lacc;
 }
 
+// Static groups: s[n][g] from W as given on the original columns [gG, (g+1)G), one
+// warp per (channel, group).
+template <typename T>
+__global__ void k_group_scales_static(const T *__restrict__ W, int N, int K, int G, int ng,
+                                      int bits, float *__restrict__ gsc) {
+    const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (wid >= (int64_t)N * ng) return;
+    const int n = (int)(wid / ng), g = (int)(wid % ng);
+    const T *wr = W + (int64_t)n * K;
+    float a = 0.f;
+    for (int k = g * G + lane; k < min(K, (g + 1) * G); k += 32) a = fmaxf(a, fabsf(to_f32(wr[k])));
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if (lane == 0) gsc[(int64_t)n * ng + g] = a == 0.f ? 1.f : 2.f * a / (float)((1 << bits) - 1);
+}
+
+// gsel[j]: the group whose scale serves processing position j (re-estimated groups:
+// j / G; static: the original group perm[j] / G); g_idx[original k] = that group.
+__global__ void k_group_select(int K, int G, int static_groups, const int32_t *__restrict__ perm,
+                               int32_t *__restrict__ gsel, int32_t *__restrict__ g_idx) {
+    const int j = blockIdx.x * blockDim.x + threadIdx.x;
+    if (j >= K) return;
+    const int k = perm ? perm[j] : j;
+    const int g = static_groups ? k / G : j / G;
+    gsel[j] = g;
+    if (g_idx) g_idx[k] = g;
+}
+
+// One CTA per channel: codes from processing order to the original order, and the
+// write-back s (c - z) with the group scale of each coordinate.
+template <typename T>
+__global__ void __launch_bounds__(256) k_finalize_grouped(
+    T *__restrict__ W, const uint8_t *__restrict__ cp, uint8_t *__restrict__ codes,
+    const int32_t *__restrict__ perm, const int32_t *__restrict__ gsel,
+    const float *__restrict__ gsc, int ldg, const float *__restrict__ scale, int K, int bits,
+    int write_back, const float *__restrict__ loss_acc, float *__restrict__ loss) {
+    const int n = blockIdx.x;
+    const float zf = (float)(1 << (bits - 1));
+    if (loss && threadIdx.x == 0) loss[n] = 0.5f * loss_acc[n];
+    const uint8_t *crow = cp + (int64_t)n * K;
+    for (int j = threadIdx.x; j < K; j += 256) {
+        const int k = perm ? perm[j] : j;
+        const uint8_t c = crow[j];
+        if (perm) codes[(int64_t)n * K + k] = c;
+        if (write_back) {
+            const float s = gsc ? gsc[(int64_t)n * ldg + gsel[j]] : scale[n];
+            W[(int64_t)n * K + k] = from_f32<T>(s * ((float)c - zf));
+        }
+    }
+}
+
 // One CTA per channel: write-back s (c - z) in the weights' dtype and the loss.
 template <typename T>
 __global__ void __launch_bounds__(256) k_finalize(T *__restrict__ W, const uint8_t *__restrict__ codes,
@@ -559,17 +677,53 @@ size_t quantize_workspace(int K, int N, int g, int blocksize) {
     return round_up(c.off, 256);
 }
 
-static size_t sweep_thread_smem(bool gptaq) {
-    return sizeof(float) * ((10 * 1024 + 32 * SW_T) * (gptaq ? 2 : 1) + SW_MAXB);
+static size_t sweep_thread_smem(bool gptaq, int gmode) {
+    return sizeof(float) * ((10 * 1024 + 32 * SW_T) * (gptaq ? 2 : 1) + SW_MAXB +
+                            (gmode == 2 ? 2 * SW_MAXB * SW_T : 0));
 }
-static size_t sweep_lanes_smem(bool gptaq) {
-    return sizeof(float) * (10 * 1024 * (gptaq ? 2 : 1) + 32 * 33 + SW_MAXB);
+static size_t sweep_lanes_smem(bool gptaq, int gmode) {
+    return sizeof(float) * (10 * 1024 * (gptaq ? 2 : 1) + 32 * 33 + SW_MAXB +
+                            (gmode == 2 ? 2 * SW_MAXB * 32 : 0));
 }
 
-gptq_status quantize_layer(void *W, int wdtype, int N, int K, const float *U, int groups, int bits,
-                           int blocksize, const float *P1, const uint8_t *dead,
-                           const float *scales_in, float *scales_out, uint8_t *codes, float *loss,
-                           int write_back, void *ws, int32_t *status, cudaStream_t st) {
+typedef void (*SweepKernel)(float *, int, int, int, int, int, const float *, const float *,
+                            const float *, int, uint8_t *, __nv_bfloat16 *, __nv_bfloat16 *,
+                            __nv_bfloat16 *, __nv_bfloat16 *, int, int, int, float *, int,
+                            const int32_t *, const SweepGroups);
+
+static SweepKernel sweep_kernel(bool per_thread, bool gptaq, int gmode) {
+    static const SweepKernel tab[2][2][3] = {
+        {{k_sweep_lanes<false, 0>, k_sweep_lanes<false, 1>, k_sweep_lanes<false, 2>},
+         {k_sweep_lanes<true, 0>, k_sweep_lanes<true, 1>, k_sweep_lanes<true, 2>}},
+        {{k_sweep_thread<false, 0>, k_sweep_thread<false, 1>, k_sweep_thread<false, 2>},
+         {k_sweep_thread<true, 0>, k_sweep_thread<true, 1>, k_sweep_thread<true, 2>}}};
+    return tab[per_thread][gptaq][gmode];
+}
+
+// Input-dimension groups and order of one quantisation (G == 0: per-channel scales,
+// natural order).
+struct QGroupOpts {
+    int G = 0;
+    int static_groups = 0;
+    const int32_t *perm = nullptr;
+    float *scales = nullptr;     // [N][ceil(K / G)] out, or NULL
+    int32_t *g_idx = nullptr;    // [K] out, or NULL
+};
+
+size_t quantize_grouped_workspace(int K, int N, int blocksize) {
+    Carver c(nullptr);
+    c.off = quantize_workspace(K, N, 1, blocksize);
+    c.take<float>((size_t)N * ((K + 31) / 32));   // group scales (smallest group: 32)
+    c.take<uint8_t>((size_t)N * K);               // codes in processing order
+    c.take<int32_t>((size_t)K);                   // group of each processing position
+    return round_up(c.off, 256);
+}
+
+static gptq_status quantize_impl(void *W, int wdtype, int N, int K, const float *U, int groups,
+                                 int bits, int blocksize, const float *P1, const uint8_t *dead,
+                                 const float *scales_in, float *scales_out, uint8_t *codes,
+                                 float *loss, int write_back, void *ws, int32_t *status,
+                                 cudaStream_t st, const QGroupOpts &go) {
     if (!update_tc_available()) return GPTQ_ERR_CUDA;
     const QLayout lay(K, N, groups);
     Carver cv(ws);
@@ -584,6 +738,22 @@ gptq_status quantize_layer(void *W, int wdtype, int N, int K, const float *U, in
     __nv_bfloat16 *Pl = cv.take<__nv_bfloat16>((size_t)SUPER * lay.ldE);
     float *scale = cv.take<float>((size_t)N);
     float *loss_acc = cv.take<float>((size_t)N);
+    const bool grouped = go.G > 0 || go.perm != nullptr;
+    const int G = go.G > 0 ? go.G : K;
+    const int ng = (K + G - 1) / G;
+    float *gsc = nullptr;
+    uint8_t *cp = codes;
+    int32_t *gsel = nullptr;
+    if (grouped) {
+        Carver gx(ws);
+        gx.off = quantize_workspace(K, N, 1, blocksize);
+        float *gws = gx.take<float>((size_t)N * ((K + 31) / 32));
+        uint8_t *cws = gx.take<uint8_t>((size_t)N * K);
+        gsel = gx.take<int32_t>((size_t)K);
+        if (go.G > 0) gsc = go.scales ? go.scales : gws;
+        if (go.perm) cp = cws;
+    }
+    const int gmode = go.G == 0 ? 0 : (go.static_groups ? 2 : 1);
     const int per_group = N / groups;
     const int64_t KK = (int64_t)K * K;
     const bool gptaq = P1 != nullptr;
@@ -592,13 +762,29 @@ gptq_status quantize_layer(void *W, int wdtype, int N, int K, const float *U, in
     if (wdtype == GPTQ_F32)
         k_scale_init<float><<<N, 256, 0, st>>>(static_cast<const float *>(W), Wk, K, per_group, bits,
                                               dead, scales_in, scale, scales_out, loss_acc, vin,
-                                              status);
+                                              status, go.perm);
     else
         k_scale_init<__nv_bfloat16><<<N, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(W), Wk, K,
                                                       per_group, bits, dead, scales_in, scale,
-                                                      scales_out, loss_acc, vin, status);
+                                                      scales_out, loss_acc, vin, status, go.perm);
     gptq_status s = launch_status();
     if (s != GPTQ_OK) return s;
+    if (grouped) {
+        k_group_select<<<(K + 255) / 256, 256, 0, st>>>(K, G, go.static_groups, go.perm, gsel,
+                                                        go.g_idx);
+        if ((s = launch_status()) != GPTQ_OK) return s;
+        if (gmode == 2) {
+            const int64_t warps = (int64_t)N * ng;
+            const int blocks = (int)((warps * 32 + 255) / 256);
+            if (wdtype == GPTQ_F32)
+                k_group_scales_static<float><<<blocks, 256, 0, st>>>(
+                    static_cast<const float *>(W), N, K, G, ng, bits, gsc);
+            else
+                k_group_scales_static<__nv_bfloat16><<<blocks, 256, 0, st>>>(
+                    static_cast<const __nv_bfloat16 *>(W), N, K, G, ng, bits, gsc);
+            if ((s = launch_status()) != GPTQ_OK) return s;
+        }
+    }
     if ((s = split_bf16(U, K, K, K, Uh, Ul, lay.ldU, groups, KK, (int64_t)K * lay.ldU, st)) != GPTQ_OK)
         return s;
     if (gptaq && (s = split_bf16(P1, K, K, K, Qh, Ql, lay.ldU, 1, 0, 0, st)) != GPTQ_OK) return s;
@@ -636,22 +822,22 @@ gptq_status quantize_layer(void *W, int wdtype, int N, int K, const float *U, in
     const bool per_thread = (int64_t)N >= 2LL * 148 * 32;
     const int cta = per_thread ? SW_T : 128;
     const dim3 grid((per_group + (per_thread ? SW_T : 32) - 1) / (per_thread ? SW_T : 32), groups);
-    auto kern = per_thread ? (gptaq ? k_sweep_thread<true> : k_sweep_thread<false>)
-                           : (gptaq ? k_sweep_lanes<true> : k_sweep_lanes<false>);
-    const size_t smem = per_thread ? sweep_thread_smem(gptaq) : sweep_lanes_smem(gptaq);
+    SweepKernel kern = sweep_kernel(per_thread, gptaq, gmode);
+    const size_t smem = per_thread ? sweep_thread_smem(gptaq, gmode) : sweep_lanes_smem(gptaq, gmode);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
         return launch_status();
     const int vec = ((K % 4 == 0 && aligned(U, 16) && (!gptaq || aligned(P1, 16))) ? 1 : 0) |
-                    ((K % 16 == 0 && aligned(codes, 16)) ? 2 : 0);
+                    ((K % 16 == 0 && aligned(cp, 16)) ? 2 : 0);
+    SweepGroups sg{G, gsc, ng, gsel};
     for (int sb0 = 0; sb0 < K; sb0 += SUPER) {
         const int sb1 = min(K, sb0 + SUPER);
         for (int i0 = sb0; i0 < sb1; i0 += blocksize) {
             const int i1 = min(i0 + blocksize, sb1);
             const int bs = i1 - i0;
-            kern<<<grid, cta, smem, st>>>(Wk, N, per_group, K, i0, bs, U, P1, scale, bits,
-                                                codes, Eh, El, Ph, Pl, lay.ldE, lay.ldG, i0 - sb0,
-                                                loss_acc, vec, status);
+            kern<<<grid, cta, smem, st>>>(Wk, N, per_group, K, i0, bs, U, P1, scale, bits, cp, Eh,
+                                          El, Ph, Pl, lay.ldE, lay.ldG, i0 - sb0, loss_acc, vec,
+                                          status, sg);
             s = launch_status();
             if (s != GPTQ_OK) return s;
             if (i1 >= sb1) continue;
@@ -682,6 +868,17 @@ gptq_status quantize_layer(void *W, int wdtype, int N, int K, const float *U, in
             if ((s = launch_update_tc(maps[box == 64][gi], p, box, st)) != GPTQ_OK) return s;
         }
     }
+    if (grouped) {
+        if (wdtype == GPTQ_F32)
+            k_finalize_grouped<float><<<N, 256, 0, st>>>(static_cast<float *>(W), cp, codes, go.perm,
+                                                         gsel, gsc, ng, scale, K, bits, write_back,
+                                                         loss_acc, loss);
+        else
+            k_finalize_grouped<__nv_bfloat16><<<N, 256, 0, st>>>(
+                static_cast<__nv_bfloat16 *>(W), cp, codes, go.perm, gsel, gsc, ng, scale, K, bits,
+                write_back, loss_acc, loss);
+        return launch_status();
+    }
     if (wdtype == GPTQ_F32)
         k_finalize<float><<<N, 256, 0, st>>>(static_cast<float *>(W), codes, scale, K, bits,
                                              write_back, loss_acc, loss, vfin);
@@ -689,6 +886,31 @@ gptq_status quantize_layer(void *W, int wdtype, int N, int K, const float *U, in
         k_finalize<__nv_bfloat16><<<N, 256, 0, st>>>(static_cast<__nv_bfloat16 *>(W), codes, scale, K,
                                                      bits, write_back, loss_acc, loss, vfin);
     return launch_status();
+}
+
+gptq_status quantize_layer(void *W, int wdtype, int N, int K, const float *U, int groups, int bits,
+                           int blocksize, const float *P1, const uint8_t *dead,
+                           const float *scales_in, float *scales_out, uint8_t *codes, float *loss,
+                           int write_back, void *ws, int32_t *status, cudaStream_t st) {
+    return quantize_impl(W, wdtype, N, K, U, groups, bits, blocksize, P1, dead, scales_in,
+                         scales_out, codes, loss, write_back, ws, status, st, QGroupOpts{});
+}
+
+gptq_status quantize_layer_grouped(void *W, int wdtype, int N, int K, const float *U, int bits,
+                                   int blocksize, int groupsize, int static_groups,
+                                   const int32_t *perm, const float *P1, const uint8_t *dead,
+                                   float *scales_out, int32_t *g_idx, uint8_t *codes, float *loss,
+                                   int write_back, void *ws, int32_t *status, cudaStream_t st) {
+    QGroupOpts go;
+    go.G = groupsize;
+    go.static_groups = static_groups;
+    go.perm = perm;
+    go.scales = scales_out;
+    go.g_idx = g_idx;
+    // without groups the per-channel scales go straight to scales_out
+    return quantize_impl(W, wdtype, N, K, U, 1, bits, blocksize, P1, dead, nullptr,
+                         groupsize ? nullptr : scales_out, codes, loss, write_back, ws, status, st,
+                         go);
 }
 
 }  // namespace gptq

@@ -55,6 +55,9 @@ class Workload:
     w_sigma: float = 0.02
     outliers: int = 0
     chunk: int = CHUNK_TOKENS
+    groupsize: int = 0            # input-dimension groups (0: per-channel scales)
+    act_order: bool = False
+    static_groups: bool = False
     extra: dict = field(default_factory=dict)
 
     def scaled(self, K=None, N=None, M=None, name=None, **kw):
@@ -80,6 +83,9 @@ WORKLOADS = {
 }
 # the headline solve: up_proj shapes at 3 bits
 WORKLOADS["mlp_up_w3"] = WORKLOADS["mlp_up"].scaled(name="mlp_up_w3", bits=3)
+# the same layer with 128-wide input groups (re-estimated) and act-order
+WORKLOADS["mlp_up_w3_g128"] = WORKLOADS["mlp_up"].scaled(name="mlp_up_w3_g128", bits=3,
+                                                         groupsize=128, act_order=True)
 
 
 def hadamard(K: int, device="cpu") -> torch.Tensor:
