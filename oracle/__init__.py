@@ -7,9 +7,10 @@ two share no code.
 
 Pins (tests/test_oracle_pins.py) tie every function here to something other than
 itself: the worked examples printed on the pages, closed forms, special cases,
-brute force and independent least-squares solves. One reading is only partly
-pinned and says so where it is defined: which weight value multiplies the
-GPTAQ residual row (``gptaq`` arguments below).
+brute force and independent least-squares solves. Two readings are only partly
+pinned and say so where they are defined: which weight value multiplies the
+GPTAQ residual row (``gptaq`` arguments below), and likewise which weight values
+enter the compensation-aware row (``cae`` arguments).
 """
 
 from .gptq_oracle import (  # noqa: F401
@@ -23,6 +24,7 @@ from .gptq_oracle import (  # noqa: F401
     obq_sweep,
     upper_factor,
     gptaq_p1,
+    cae_p2,
     row_form_sweep,
     replay_row_form,
     layer_error,

@@ -155,7 +155,8 @@ def dequantize(c, s, bits):
 # The sweep in explicit OBQ form (no Cholesky, no lazy batching)
 # --------------------------------------------------------------------------------------
 
-def obq_sweep(H_d, W, s, bits, mode="schur", C=None, return_trace=False, steps=None):
+def obq_sweep(H_d, W, s, bits, mode="schur", C=None, return_trace=False, steps=None,
+              cae_H=None):
     """Quantise coordinates 0..K-1 in order, compensating the free set each step.
 
     [GPTQ blog] "一次约束补偿的公式从哪里来": with free set F and P_F = (H[F, F])^-1, fixing
@@ -181,13 +182,26 @@ def obq_sweep(H_d, W, s, bits, mode="schur", C=None, return_trace=False, steps=N
     an independent least-squares solve on the token matrices; which w multiplies
     the row is a reading no printed value pins.
 
+    cae_H (optional) adds the compensation-aware error term of [ResComp] items 1-3:
+    the objective keeps the fixed target w^(0) X~, the residual gains
+    r2 = (w^(0) - w^(q)) X~, and by the same neuron decomposition the part owed to
+    coordinate q is applied at q's step:
+        w_F' += (w_q^(0) - w_q^pre) * (X~X^T)[q, F'] (H_d[F', F'])^-1,
+    with X~X^T = XX^T + dX X^T, i.e. cae_H + C in the factor-2 convention (cae_H the
+    undamped Gram 2 X^T X, C = 0 when absent). Readings: w^(0) is the weight vector
+    the sweep starts from (after dead coordinates are zeroed), and w_q^pre the value
+    of coordinate q at its step, before rounding.
+
     Returns (codes, W_hat, loss) with loss[n] = sum_q r^2 / (2 (P_F)_qq), and the
     per-step weights when return_trace. `steps` stops after the first `steps`
     coordinates (a prefix of the same sweep; used to time a bounded sample).
     """
     H_d = np.asarray(H_d, dtype=np.float64)
     W = np.array(W, dtype=np.float64, copy=True)
+    W0 = W.copy()
     N, K = W.shape
+    if cae_H is not None:
+        Xt = np.asarray(cae_H, dtype=np.float64) + (0.0 if C is None else np.asarray(C, dtype=np.float64))
     s = np.asarray(s, dtype=np.float64)
     codes = np.zeros((N, K))
     loss = np.zeros(N)
@@ -210,6 +224,8 @@ def obq_sweep(H_d, W, s, bits, mode="schur", C=None, return_trace=False, steps=N
             P_next = P[1:, 1:] - np.outer(P[1:, 0], P[0, 1:]) / p_qq
             if C is not None:
                 W[:, q + 1:] += np.outer(w_pre, C[q, q + 1:] @ P_next)
+            if cae_H is not None:
+                W[:, q + 1:] += np.outer(W0[:, q] - w_pre, Xt[q, q + 1:] @ P_next)
             P = P_next
         if return_trace:
             trace.append(W.copy())
@@ -250,7 +266,23 @@ def gptaq_p1(C, U):
     return T @ U
 
 
-def row_form_sweep(U, W, s, bits, blocksize, P1=None):
+def cae_p2(H, C, U):
+    """P2 = [((H + C) U^T) ⊙ M] U, M the strict upper mask as in gptaq_p1.
+
+    [ResComp] item 3: P2 = [(X~X^T L) ⊙ M_U] L^T with X~X^T = XX^T + dX X^T reused from
+    the quantities already at hand; in the factor-2 convention X~X^T is H + C with H
+    the undamped Gram and C the cross statistic (None: no asymmetric stream, X~ = X).
+    Row q is (H + C)[q, F'] (H_d[F', F'])^-1 over the coordinates after q, the
+    explicit compensation-aware term of obq_sweep.
+    """
+    A = np.asarray(H, dtype=np.float64)
+    if C is not None:
+        A = A + np.asarray(C, dtype=np.float64)
+    U = np.asarray(U, dtype=np.float64)
+    return np.triu(A @ U.T, k=1) @ U
+
+
+def row_form_sweep(U, W, s, bits, blocksize, P1=None, P2=None):
     """GPTQ sweep with U rows and lazy blocks of `blocksize` coordinates.
 
     [GPTQ blog] "为什么 Cholesky Factor 不能当作原始逆矩阵" and "GPTQ 怎样把逐个补偿变成可扩展算法":
@@ -258,12 +290,15 @@ def row_form_sweep(U, W, s, bits, blocksize, P1=None):
     later k at once; at the block end the far coordinates get the bulk update
     W_far -= U[blk, far]^T E_blk. The blocking changes only the order of the work.
     With P1, [ResComp] item 3's extra row term w_j^pre * P1[j, k] is added the same
-    way (immediately inside the block, in bulk for the far coordinates).
+    way (immediately inside the block, in bulk for the far coordinates); with P2, the
+    compensation-aware row term (w_j^(0) - w_j^pre) * P2[j, k] likewise, w^(0) being
+    the weights the sweep starts from.
 
     Returns (codes, W_hat, E) with E[n, j] the normalised errors.
     """
     U = np.asarray(U, dtype=np.float64)
     W = np.array(W, dtype=np.float64, copy=True)
+    W0 = W.copy()
     N, K = W.shape
     codes = np.zeros((N, K))
     E = np.zeros((N, K))
@@ -279,6 +314,8 @@ def row_form_sweep(U, W, s, bits, blocksize, P1=None):
             W[:, j:i1] -= np.outer(e, U[j, j:i1])
             if P1 is not None:
                 W[:, j + 1:i1] += np.outer(w, P1[j, j + 1:i1])
+            if P2 is not None:
+                W[:, j + 1:i1] += np.outer(W0[:, j] - w, P2[j, j + 1:i1])
             W[:, j] = target
             codes[:, j] = c
             E[:, j] = e
@@ -286,10 +323,12 @@ def row_form_sweep(U, W, s, bits, blocksize, P1=None):
             W[:, i1:] -= E[:, i0:i1] @ U[i0:i1, i1:]
             if P1 is not None:
                 W[:, i1:] += W_pre @ P1[i0:i1, i1:]
+            if P2 is not None:
+                W[:, i1:] += (W0[:, i0:i1] - W_pre) @ P2[i0:i1, i1:]
     return codes, W, E
 
 
-def replay_row_form(U, W, s, bits, codes_gpu, P1=None, band=1e-4):
+def replay_row_form(U, W, s, bits, codes_gpu, P1=None, band=1e-4, P2=None):
     """Tie-follow replay of the unbatched row-form sweep against another run's codes.
 
     At each (j, n) the oracle takes its own fp64 decision. Where the other run's
@@ -297,12 +336,14 @@ def replay_row_form(U, W, s, bits, codes_gpu, P1=None, band=1e-4):
     |frac(w / s) - 0.5| < band, else as a mismatch; in both cases the oracle then
     continues with the other run's code, so one decision never cascades. A
     negative entry in codes_gpu means "no decision given": the oracle keeps its own.
+    P1 and P2 add the row terms of row_form_sweep.
 
     Returns dict(codes, W_hat, tie_flips, mismatches, worst_tie_distance, loss) with
     loss[n] = 1/2 sum_j E_j^2 along the replayed trajectory.
     """
     U = np.asarray(U, dtype=np.float64)
     W = np.array(W, dtype=np.float64, copy=True)
+    W0 = W.copy()
     s = np.asarray(s, dtype=np.float64)
     G = np.asarray(codes_gpu, dtype=np.float64)
     N, K = W.shape
@@ -333,6 +374,8 @@ def replay_row_form(U, W, s, bits, codes_gpu, P1=None, band=1e-4):
         W[:, j:] -= np.outer(e, U[j, j:])
         if P1 is not None and j + 1 < K:
             W[:, j + 1:] += np.outer(w, P1[j, j + 1:])
+        if P2 is not None and j + 1 < K:
+            W[:, j + 1:] += np.outer(W0[:, j] - w, P2[j, j + 1:])
         W[:, j] = target
         codes[:, j] = c
     return dict(codes=codes, W_hat=W, tie_flips=tie_flips, mismatches=mismatches,
@@ -353,14 +396,16 @@ def layer_error(H, W, W_hat):
     return 0.5 * float(np.sum((D @ np.asarray(H, dtype=np.float64)) * D))
 
 
-def solve_layer(H, W, bits, percdamp=0.01, groups=1, C=None, scales=None, mode="schur"):
+def solve_layer(H, W, bits, percdamp=0.01, groups=1, C=None, scales=None, mode="schur",
+                cae=False):
     """Whole per-layer solve: dead fix, damping, scale, dead zeroing, sweep.
 
     H is (K, K) for groups == 1 or (g, K, K); output channels are split into g
     contiguous groups of N / g, group i solved with H[i] ([G2PTQ] GuidedQuant-style
     groups with one shared Hessian per group). The scale comes from W as given,
-    before dead coordinates are zeroed (reading). Returns dict(codes, W_hat, scales,
-    loss, dead).
+    before dead coordinates are zeroed (reading). cae adds the compensation-aware
+    term of obq_sweep with each group's H as given. Returns dict(codes, W_hat,
+    scales, loss, dead).
     """
     W = np.asarray(W, dtype=np.float64)
     N, K = W.shape
@@ -381,7 +426,8 @@ def solve_layer(H, W, bits, percdamp=0.01, groups=1, C=None, scales=None, mode="
         rows = slice(g * per, (g + 1) * per)
         Wg = W[rows].copy()
         Wg[:, dead] = 0.0
-        c, wh, l = obq_sweep(H_d, Wg, s[rows], bits, mode=mode, C=C)
+        c, wh, l = obq_sweep(H_d, Wg, s[rows], bits, mode=mode, C=C,
+                             cae_H=Hs[g] if cae else None)
         codes[rows], W_hat[rows], loss[rows] = c, wh, l
         deads[g] = dead
     return dict(codes=codes, W_hat=W_hat, scales=s, loss=loss, dead=deads)
@@ -442,7 +488,7 @@ def static_group_scales(W, bits, groupsize):
     return S
 
 
-def obq_sweep_grouped(H_d, W, bits, groupsize, static=False, perm=None, C=None):
+def obq_sweep_grouped(H_d, W, bits, groupsize, static=False, perm=None, C=None, cae_H=None):
     """The explicit OBQ sweep of obq_sweep with input-dimension groups and an order.
 
     [GPTQ blog] "Damping 与两个不同的分组参数": blocksize organises the computation,
@@ -457,7 +503,8 @@ def obq_sweep_grouped(H_d, W, bits, groupsize, static=False, perm=None, C=None):
         coordinate k uses its original group k // G at whatever step it is fixed;
       - afterwards codes and weights are restored to the original coordinate order,
         with g_idx[k] the group whose scale reconstructs coordinate k.
-    C (optional) is the GPTAQ cross statistic in the original order.
+    C (optional) is the GPTAQ cross statistic and cae_H (optional) the undamped Gram
+    of the compensation-aware term (both as in obq_sweep), in the original order.
 
     Returns dict(codes, W_hat, scales, g_idx, loss), all in the original order.
     """
@@ -470,6 +517,12 @@ def obq_sweep_grouped(H_d, W, bits, groupsize, static=False, perm=None, C=None):
     Hp = H_d[np.ix_(order, order)]
     Wp = W[:, order].copy()
     Cp = None if C is None else np.asarray(C, dtype=np.float64)[np.ix_(order, order)]
+    Xt = None
+    if cae_H is not None:
+        Xt = np.asarray(cae_H, dtype=np.float64)[np.ix_(order, order)]
+        if Cp is not None:
+            Xt = Xt + Cp
+    W0p = Wp.copy()
     S_static = static_group_scales(W, bits, G) if static else None
     scales = S_static.copy() if static else np.zeros((N, ng))
     codes_p = np.zeros((N, K))
@@ -495,6 +548,8 @@ def obq_sweep_grouped(H_d, W, bits, groupsize, static=False, perm=None, C=None):
             P_next = P[1:, 1:] - np.outer(P[1:, 0], P[0, 1:]) / p_qq
             if Cp is not None:
                 Wp[:, q + 1:] += np.outer(w_pre, Cp[q, q + 1:] @ P_next)
+            if Xt is not None:
+                Wp[:, q + 1:] += np.outer(W0p[:, q] - w_pre, Xt[q, q + 1:] @ P_next)
             P = P_next
     codes = np.zeros((N, K))
     W_hat = np.zeros((N, K))
@@ -507,13 +562,14 @@ def obq_sweep_grouped(H_d, W, bits, groupsize, static=False, perm=None, C=None):
 
 
 def replay_row_form_grouped(U, W, bits, groupsize, codes_gpu, static=False, perm=None,
-                            static_scales=None, band=1e-4):
+                            static_scales=None, band=1e-4, P1=None, P2=None):
     """Tie-follow replay (as replay_row_form) of the row-form sweep with groups and an
     order, against another run's codes given in the original order.
 
     U is the factor of H_d in processing order (U^T U = (H_d[perm][:, perm])^-1). The
     scales follow obq_sweep_grouped's rules along the replayed trajectory (static
     scales may be passed in, e.g. the other run's, to replay its decisions exactly).
+    P1 and P2, in processing order, add the row terms of row_form_sweep.
     Returns dict(codes, W_hat, scales, g_idx, tie_flips, mismatches) in the original
     order.
     """
@@ -524,6 +580,7 @@ def replay_row_form_grouped(U, W, bits, groupsize, codes_gpu, static=False, perm
     G = groupsize
     ng = (K + G - 1) // G
     Wp = W[:, order].copy()
+    W0p = Wp.copy()
     Gc = np.asarray(codes_gpu, dtype=np.float64)[:, order]
     if static:
         S = static_group_scales(W, bits, G) if static_scales is None else np.asarray(static_scales, dtype=np.float64)
@@ -552,6 +609,10 @@ def replay_row_form_grouped(U, W, bits, groupsize, codes_gpu, static=False, perm
         target = s * (c - z)
         e = (w - target) / U[j, j]
         Wp[:, j:] -= np.outer(e, U[j, j:])
+        if P1 is not None and j + 1 < K:
+            Wp[:, j + 1:] += np.outer(w, P1[j, j + 1:])
+        if P2 is not None and j + 1 < K:
+            Wp[:, j + 1:] += np.outer(W0p[:, j] - w, P2[j, j + 1:])
         Wp[:, j] = target
         codes_p[:, j] = c
     codes = np.zeros((N, K))

@@ -470,3 +470,157 @@ def test_reestimated_groups_see_compensation():
     b = O.obq_sweep_grouped(Hd, W, 2, 4, static=True)
     np.testing.assert_allclose(a["scales"][:, 0], b["scales"][:, 0], rtol=1e-15)
     assert np.max(np.abs(a["scales"][:, 1:] - b["scales"][:, 1:])) > 1e-6
+
+
+# ------------------------------------------------------------------ compensation-aware error
+
+def _collapsed(U):
+    """I - diag(U)^-1 U: what [(H U^T) ⊙ M] U reduces to when U^T U = (H + λI)^-1
+    (H U^T = U^-1 - λ U^T, and the strict upper part of U^T is zero), worked by hand."""
+    return np.eye(U.shape[0]) - U / np.diag(U)[:, None]
+
+
+def test_cae_p2_closed_form():
+    K, M = 12, 60
+    X_fp, X_q = _gptaq_problem(K, M, 31)
+    X_q[:, 4] = 0.0                        # a dead input coordinate
+    H = O.gram(X_q)
+    Hd, dead = O.dead_and_damp(H, 0.05)
+    assert dead[4]
+    C = O.cross_gram(X_q, X_fp)
+    assert np.abs(C[4]).max() > 0          # the dead row still carries cross terms
+    U = O.upper_factor(Hd)
+    np.testing.assert_allclose(O.cae_p2(H, C, U), O.gptaq_p1(C, U) + _collapsed(U), atol=1e-10)
+    np.testing.assert_allclose(O.cae_p2(H, None, U), _collapsed(U), atol=1e-10)
+    # the strict mask leaves a zero diagonal: coordinate q's own row term never moves q
+    assert np.allclose(np.tril(O.cae_p2(H, C, U)), 0.0)
+
+
+def test_cae_second_step_is_least_squares_on_tokens():
+    """Step 0 owes nothing to r2 (w^(0) and w^(0) agree); at step 1 the term equals
+    the least-squares fit of the quantised stream's free columns to coordinate 1's
+    share of r2 = (w^(0) - w^(1)) X~, solved on the token matrices (no H, no C)."""
+    K, M = 6, 80
+    X_fp, X_q = _gptaq_problem(K, M, 23)
+    H = O.gram(X_q)
+    C = O.cross_gram(X_q, X_fp)
+    w = np.array([[0.31, -0.12, 0.05, 0.2, -0.07, 0.11]])
+    s = np.array([1.0])
+    _, _, _, tr_cae = O.obq_sweep(H, w, s, 4, C=C, cae_H=H, return_trace=True)
+    _, _, _, tr_aq = O.obq_sweep(H, w, s, 4, C=C, return_trace=True)
+    np.testing.assert_array_equal(tr_cae[0], tr_aq[0])
+    drift = w[0, 1] - tr_aq[0][0, 1]
+    assert abs(drift) > 1e-3
+    extra = tr_cae[1][0, 2:] - tr_aq[1][0, 2:]
+    v, *_ = np.linalg.lstsq(X_q[:, 2:], X_fp[:, 1] * drift, rcond=None)
+    np.testing.assert_allclose(extra, v, rtol=1e-9, atol=1e-12)
+
+
+def test_cae_three_weight_hand_trace(golden):
+    """The printed three-weight problem with the compensation-aware term, worked by
+    hand: step 0 is unchanged, [0, -0.6, 0.2]; at step 1 coordinate 1 has drifted by
+    w^(0)_1 - w_1 = 0.2 and P2[1, 2] = H[1, 2] / H[2, 2] = 2/3 adds 2/15 to the 7/15
+    of plain GPTQ, giving [0, -1, 0.6]; step 2 rounds 0.6 to 1."""
+    g = golden("three_weight_counterexample.txt")
+    H = O.gram(g["X"])
+    w, s, bits = g["w"], np.array([g["scale"]]), int(g["bits"])
+    for mode in ("schur", "direct"):
+        _, W_hat, _, tr = O.obq_sweep(H, w[None, :], s, bits, mode=mode, cae_H=H,
+                                      return_trace=True)
+        np.testing.assert_allclose(tr[0][0], [0.0, -0.6, 0.2], atol=1e-12)
+        np.testing.assert_allclose(tr[1][0], [0.0, -1.0, 0.6], atol=1e-12)
+        np.testing.assert_allclose(W_hat[0], [0.0, -1.0, 1.0], atol=1e-12)
+    P2 = O.cae_p2(H, None, g["U"])
+    assert P2[1, 2] == pytest.approx(2.0 / 3.0, abs=1e-12)
+    for B in (1, 2, 3):
+        _, W_row, _ = O.row_form_sweep(g["U"], w[None, :], s, bits, B, P2=P2)
+        np.testing.assert_allclose(W_row[0], [0.0, -1.0, 1.0], atol=1e-12)
+
+
+@pytest.mark.parametrize("with_c", [False, True])
+def test_cae_row_form_matches_explicit(with_c):
+    K, M = 14, 90
+    X_fp, X_q = _gptaq_problem(K, M, 7)
+    H = O.gram(X_q)
+    Hd, _ = O.dead_and_damp(H, 0.01)
+    C = O.cross_gram(X_q, X_fp) if with_c else None
+    W = np.random.default_rng(3).standard_normal((7, K)) * 0.02
+    s, _ = O.symmetric_scale(W, 2)
+    c_ex, w_ex, _, tr = O.obq_sweep(Hd, W, s, 2, C=C, cae_H=H, return_trace=True)
+    c_dir, w_dir, _ = O.obq_sweep(Hd, W, s, 2, C=C, cae_H=H, mode="direct")
+    np.testing.assert_array_equal(c_dir, c_ex)
+    np.testing.assert_allclose(w_dir, w_ex, atol=1e-12)
+    U = O.upper_factor(Hd)
+    P1 = O.gptaq_p1(C, U) if with_c else None
+    P2 = O.cae_p2(H, C, U)
+    for B in (1, 3, 8, K):
+        c_row, w_row, _ = O.row_form_sweep(U, W, s, 2, B, P1=P1, P2=P2)
+        np.testing.assert_array_equal(c_row, c_ex)
+        np.testing.assert_allclose(w_row, w_ex, atol=1e-12)
+    rep = O.replay_row_form(U, W, s, 2, c_ex, P1=P1, P2=P2)
+    assert rep["mismatches"] == 0 and rep["tie_flips"] == 0
+    np.testing.assert_allclose(rep["W_hat"], w_ex, atol=1e-12)
+    # the term moves the free weights once compensation has moved a coordinate
+    _, _, _, tr_plain = O.obq_sweep(Hd, W, s, 2, C=C, return_trace=True)
+    assert not np.allclose(tr[1], tr_plain[1])
+
+
+def test_cae_collapsed_sweep_matches_row_form():
+    """With P2 = P1 + I - diag(U)^-1 U the two row terms merge with the GPTQ step into
+    one propagated error E'_j = (w^(0)_j - q_j) / U_jj and a P1 row scaled by w^(0)_j
+    (algebra; the form a lazy-block implementation can use without P2). Written out
+    here, separately from the oracle, and compared with its row form."""
+    K, M = 16, 100
+    X_fp, X_q = _gptaq_problem(K, M, 11)
+    H = O.gram(X_q)
+    Hd, _ = O.dead_and_damp(H, 0.01)
+    C = O.cross_gram(X_q, X_fp)
+    U = O.upper_factor(Hd)
+    P1 = O.gptaq_p1(C, U)
+    W0 = np.random.default_rng(5).standard_normal((5, K)) * 0.02
+    s, _ = O.symmetric_scale(W0, 3)
+    c_ref, w_ref, _ = O.row_form_sweep(U, W0, s, 3, 4, P1=P1, P2=O.cae_p2(H, C, U))
+    W = W0.copy()
+    z = 4
+    for j in range(K):
+        c = np.clip(np.rint(W[:, j] / s) + z, 0, 7)
+        q = s * (c - z)
+        e = (W0[:, j] - q) / U[j, j]
+        W[:, j + 1:] += -np.outer(e, U[j, j + 1:]) + np.outer(W0[:, j], P1[j, j + 1:])
+        W[:, j] = q
+        np.testing.assert_array_equal(c, c_ref[:, j])
+    np.testing.assert_allclose(W, w_ref, atol=1e-12)
+
+
+def test_cae_special_cases_reduce_to_rtn():
+    # a diagonal Hessian compensates nothing, so no coordinate drifts and the term is
+    # void; a single coordinate has nothing after it
+    rng = np.random.default_rng(9)
+    K = 10
+    H = np.diag(rng.uniform(0.5, 2.0, K))
+    W = rng.standard_normal((6, K)) * 0.02
+    s, _ = O.symmetric_scale(W, 3)
+    c, W_hat, _ = O.obq_sweep(H, W, s, 3, cae_H=H)
+    np.testing.assert_array_equal(c, O.quantize_codes(W, s[:, None], 3))
+    np.testing.assert_allclose(O.cae_p2(H, None, O.upper_factor(H)), 0.0, atol=1e-15)
+    c1, _, _ = O.obq_sweep(np.array([[2.0]]), W[:, :1], s, 3, cae_H=np.array([[2.0]]))
+    np.testing.assert_array_equal(c1, O.quantize_codes(W[:, :1], s[:, None], 3))
+
+
+def test_cae_grouped_row_form_matches_explicit():
+    K, M = 16, 90
+    X_fp, X_q = _gptaq_problem(K, M, 13)
+    H = O.gram(X_q)
+    Hd, _ = O.dead_and_damp(H, 0.01)
+    C = O.cross_gram(X_q, X_fp)
+    W = np.random.default_rng(4).standard_normal((6, K)) * 0.02
+    perm = O.act_order(H)
+    r = O.obq_sweep_grouped(Hd, W, 3, 8, perm=perm, C=C, cae_H=H)
+    ix = np.ix_(perm, perm)
+    U = O.upper_factor(Hd[ix])
+    rep = O.replay_row_form_grouped(U, W, 3, 8, r["codes"], perm=perm,
+                                    P1=O.gptaq_p1(C[ix], U), P2=O.cae_p2(H[ix], C[ix], U))
+    assert rep["mismatches"] == 0 and rep["tie_flips"] == 0
+    np.testing.assert_allclose(rep["W_hat"], r["W_hat"], atol=1e-9)
+    plain = O.obq_sweep_grouped(Hd, W, 3, 8, perm=perm, C=C)
+    assert not np.allclose(plain["W_hat"], r["W_hat"]) or not np.array_equal(plain["codes"], r["codes"])
