@@ -34,4 +34,6 @@ from .gptq_oracle import (  # noqa: F401
     static_group_scales,
     obq_sweep_grouped,
     replay_row_form_grouped,
+    pack_codes,
+    unpack_codes,
 )

@@ -624,3 +624,46 @@ def replay_row_form_grouped(U, W, bits, groupsize, codes_gpu, static=False, perm
     g_idx = (np.arange(K) // G) if static else (inv // G)
     return dict(codes=codes, W_hat=W_hat, scales=S, g_idx=g_idx, tie_flips=tie_flips,
                 mismatches=mismatches)
+
+
+# --------------------------------------------------------------------------------------
+# Storage: codes packed into 32-bit words
+# --------------------------------------------------------------------------------------
+
+def pack_codes(codes, bits):
+    """Each channel's codes as one little-endian bit stream in 32-bit words.
+
+    [GPTQ blog] "落在格点上与真正存成低位权重是两步": landing on the grid is not yet
+    low-bit storage; the integer codes must be packed into wider containers (the
+    3-bit codes into an integer buffer), with scale, zero point and layout kept
+    beside them. The pages fix no layout. Reading: per output channel n, code k takes
+    bits [b k, b k + b) of the channel's stream (least significant bit first), and
+    stream bit t is bit t mod 32 of word t // 32; a row has ceil(K b / 32) words and
+    the unused high bits of its last word are zero. For b = 2, 4, 8 this puts 32 / b
+    whole codes in each word; for b = 3, 32 codes fill 3 words and some straddle two.
+
+    codes: (N, K) integers in [0, 2^b). Returns (N, ceil(K b / 32)) uint32.
+    """
+    c = np.asarray(codes).astype(np.int64)
+    N, K = c.shape
+    nw = (K * bits + 31) // 32
+    words = np.zeros((N, nw), dtype=np.uint64)
+    for k in range(K):
+        for i in range(bits):
+            t = k * bits + i
+            bit = ((c[:, k] >> i) & 1).astype(np.uint64)
+            words[:, t // 32] |= bit << np.uint64(t % 32)
+    return words.astype(np.uint32)
+
+
+def unpack_codes(words, bits, K):
+    """Inverse of pack_codes: (N, ceil(K b / 32)) uint32 -> (N, K) codes."""
+    w = np.asarray(words).astype(np.uint64)
+    N = w.shape[0]
+    c = np.zeros((N, K), dtype=np.int64)
+    for k in range(K):
+        for i in range(bits):
+            t = k * bits + i
+            bit = (w[:, t // 32] >> np.uint64(t % 32)) & np.uint64(1)
+            c[:, k] |= bit.astype(np.int64) << i
+    return c

@@ -624,3 +624,50 @@ def test_cae_grouped_row_form_matches_explicit():
     np.testing.assert_allclose(rep["W_hat"], r["W_hat"], atol=1e-9)
     plain = O.obq_sweep_grouped(Hd, W, 3, 8, perm=perm, C=C)
     assert not np.allclose(plain["W_hat"], r["W_hat"]) or not np.array_equal(plain["codes"], r["codes"])
+
+
+# ------------------------------------------------------------------ packed storage
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+@pytest.mark.parametrize("K", [1, 31, 32, 33, 100])
+def test_pack_is_the_little_endian_bit_stream(bits, K):
+    # independent statement of the layout: the row's words read as one little-endian
+    # integer equal sum_k c_k 2^(b k) (Python integers, no bit loop over words)
+    rng = np.random.default_rng(bits * 100 + K)
+    c = rng.integers(0, 2 ** bits, size=(5, K))
+    words = O.pack_codes(c, bits)
+    assert words.dtype == np.uint32 and words.shape == (5, (K * bits + 31) // 32)
+    for n in range(5):
+        as_int = int.from_bytes(words[n].astype("<u4").tobytes(), "little")
+        assert as_int == sum(int(v) << (bits * k) for k, v in enumerate(c[n]))
+    np.testing.assert_array_equal(O.unpack_codes(words, bits, K), c)
+
+
+def test_pack_whole_code_widths_match_byte_views():
+    # 8-bit codes: the words' bytes are the codes; 4-bit: byte j = c[2j] | c[2j+1] << 4;
+    # 2-bit: byte j = c[4j] | c[4j+1] << 2 | c[4j+2] << 4 | c[4j+3] << 6
+    rng = np.random.default_rng(1)
+    c8 = rng.integers(0, 256, size=(3, 64))
+    np.testing.assert_array_equal(O.pack_codes(c8, 8).view(np.uint8), c8.astype(np.uint8))
+    c4 = rng.integers(0, 16, size=(3, 64))
+    np.testing.assert_array_equal(O.pack_codes(c4, 4).view(np.uint8),
+                                  (c4[:, 0::2] | (c4[:, 1::2] << 4)).astype(np.uint8))
+    c2 = rng.integers(0, 4, size=(3, 64))
+    np.testing.assert_array_equal(
+        O.pack_codes(c2, 2).view(np.uint8),
+        (c2[:, 0::4] | (c2[:, 1::4] << 2) | (c2[:, 2::4] << 4) | (c2[:, 3::4] << 6)).astype(np.uint8))
+
+
+def test_pack_three_bit_straddle_by_hand():
+    # 3-bit codes 0..7 repeated: code 10 (value 2 = 0b010) sits at bits 30..32, so
+    # word 0 ends with bits 30, 31 = 0, 1 and word 1 starts with bit 0 = 0; code 21
+    # (value 5 = 0b101) sits at bits 63..65: word 1's top bit 1, word 2's bits 0, 1 = 0, 1
+    c = (np.arange(32) % 8)[None, :]
+    w = O.pack_codes(c, 3)
+    assert w.shape == (1, 3)
+    assert (int(w[0, 0]) >> 30) == 0b10
+    assert int(w[0, 1]) & 1 == 0
+    assert (int(w[0, 1]) >> 31) == 1
+    assert int(w[0, 2]) & 0b11 == 0b10
+    # the first ten codes fill word 0's low 30 bits
+    assert int(w[0, 0]) & ((1 << 30) - 1) == sum(k % 8 << (3 * k) for k in range(10))
