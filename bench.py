@@ -240,9 +240,11 @@ def run_ours(args, rank, world, local_rank):
     status = gq.new_status(dev)
     ws_p = torch.empty(gq.gptq_workspace_size(gq.GPTQ_OP_PREPARE, K, 0, g, 0), dtype=torch.uint8,
                        device=dev)
-    ws_q = torch.empty(gq.gptq_workspace_size(gq.GPTQ_OP_QUANTIZE_GROUPED if grouped
-                                              else gq.GPTQ_OP_QUANTIZE, K, N, g, wl.blocksize),
-                       dtype=torch.uint8, device=dev)
+    op_q = ((gq.GPTQ_OP_QUANTIZE_GROUPED if grouped else gq.GPTQ_OP_QUANTIZE) |
+            (gq.GPTQ_WS_CAE if wl.cae else 0))
+    ws_q = torch.empty(gq.gptq_workspace_size(op_q, K, N, g, wl.blocksize), dtype=torch.uint8,
+                       device=dev)
+    Cp = torch.empty(K, K, device=dev) if (wl.act_order and wl.gptaq) else None
     ws_r = (torch.empty(gq.gptq_workspace_size(gq.GPTQ_OP_RESIDUAL, K, 0, 1, 0), dtype=torch.uint8,
                         device=dev) if wl.gptaq else None)
     stream = torch.cuda.current_stream(dev)
@@ -267,23 +269,26 @@ def run_ours(args, rank, world, local_rank):
                 gq.gptaq_accumulate_cross(C, Xf[c * ch:(c + 1) * ch], X[c * ch:(c + 1) * ch],
                                           status=status, stream=stream)
         ev[1].record(stream)
-        Hs = H
+        Hs, Cs = H, C
         if perm is not None:            # act-order: solve in the reordered coordinates
             gq.gptq_act_order(H, perm=perm, stream=stream)
             Hs = gq.gptq_permute_hessian(H, perm, out=Hp, stream=stream)
+            if C is not None:
+                Cs = gq.gptq_permute_hessian(C, perm, out=Cp, stream=stream)
         gq.gptq_prepare(Hs, wl.percdamp, workspace=ws_p, status=status, stream=stream)
         if P1 is not None:
-            gq.gptaq_residual(P1, C, Hs, workspace=ws_r, stream=stream)
+            gq.gptaq_residual(P1, Cs, Hs, workspace=ws_r, stream=stream)
         ev[2].record(stream)
         if grouped:
             gq.gptq_quantize_layer_grouped(W, Hs, wl.bits, wl.blocksize, wl.groupsize,
                                            static_groups=wl.static_groups, perm=perm, P1=P1,
                                            scales_out=scales, g_idx=g_idx, codes=codes,
-                                           workspace=ws_q, status=status, stream=stream)
+                                           workspace=ws_q, status=status, stream=stream,
+                                           cae=wl.cae)
         else:
             gq.gptq_quantize_layer(W, Hs, wl.bits, wl.blocksize, groups=g, P1=P1,
                                    scales_out=scales, codes=codes, workspace=ws_q, status=status,
-                                   stream=stream)
+                                   stream=stream, cae=wl.cae)
         ev[3].record(stream)
         return ev
 
@@ -321,6 +326,17 @@ def run_ours(args, rank, world, local_rank):
     total_ms, gram_ms, prep_ms, quant_ms, gram_launch_ms = stats.tolist()
     ms_per_step = total_ms / args.steps
 
+    # storage: the step's codes packed to low-bit words (outside the timed steps)
+    words = gq.gptq_pack_codes(codes, wl.bits, stream=stream)
+    pk0, pk1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    pk0.record(stream)
+    for _ in range(10):
+        gq.gptq_pack_codes(codes, wl.bits, words=words, stream=stream)
+    pk1.record(stream)
+    torch.cuda.synchronize()
+    pack_ms = pk0.elapsed_time(pk1) / 10
+    pack_bytes = N * K + words.numel() * 4
+
     e2e = None
     if not args.no_e2e and g == 1 and not wl.gptaq:
         e2e = run_e2e(args, wl, X, W, dev, gq, torch, dist, world)
@@ -352,7 +368,9 @@ def run_ours(args, rank, world, local_rank):
         "data": f"synthetic ({wl.stream} bf16 tokens, N(0,{wl.w_sigma}^2) bf16 weights)",
         "config": {"workload": f"{wl.name}: K={K} N={N} tokens={M} (chunks {nch}x{ch}) W{wl.bits} "
                                f"blocksize {wl.blocksize} percdamp {wl.percdamp} groups {g}"
-                               + (" gptaq" if wl.gptaq else ""),
+                               + (" gptaq" if wl.gptaq else "") + (" cae" if wl.cae else "")
+                               + (f" groupsize {wl.groupsize}" if wl.groupsize else "")
+                               + (" act-order" if wl.act_order else ""),
                    "l2": f"inputs larger than L2 (X {M * K * 2 / 1e9:.1f} GB)", "parallelism": f"{world} independent layers"},
         "breakdown": {"gram_ms": gram_ms, "prepare_ms": prep_ms, "quantize_ms": quant_ms,
                       "layer_solve_ms": prep_ms + quant_ms,
@@ -361,6 +379,12 @@ def run_ours(args, rank, world, local_rank):
                       "gram_includes_cross": bool(wl.gptaq),
                       "prepare_includes_residual": bool(wl.gptaq)},
         "roofline": roofline,
+        "pack": {"kernel": "k_pack (gptq_pack_codes)", "ms": round(pack_ms, 4),
+                 "bytes": pack_bytes, "gbs": round(pack_bytes / (pack_ms * 1e-3) / 1e9, 1),
+                 "frac_of_hbm": (round(pack_bytes / (pack_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)
+                                 if peaks.get("hbm_gbs") else None),
+                 "note": "codes N x K bytes in + packed words out, 10 launches after the timed "
+                         "steps, not part of the step"},
         "gpu_launches": int(launches),
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                    "reasons": clocks["reasons"]},

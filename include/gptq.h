@@ -72,6 +72,10 @@ typedef enum {
     GPTQ_OP_QUANTIZE_GROUPED = 3
 } gptq_op;
 
+/* OR-ed into GPTQ_OP_QUANTIZE or GPTQ_OP_QUANTIZE_GROUPED: the workspace of a call
+ * with cae != 0 (one more fp32 copy of W). */
+#define GPTQ_WS_CAE 0x100
+
 /*
  * gptq_accumulate_hessian -- H[g] += 2 * X^T diag(w[g]) X over one token chunk.
  *
@@ -196,6 +200,12 @@ GPTQ_API gptq_status gptaq_residual(float *P1, const float *C, const float *U, i
  * W_k -= U_jk E_j for the block's later k at once; at the block end the far
  * coordinates get W_far -= U[blk, far]^T E_blk. With P1 the GPTAQ row term
  * w_j^pre * P1[j, k] is added the same way.
+ * With cae != 0 the compensation-aware error term of [ResComp] "关键设计" items 1-3
+ * is added too: the row (w_j^(0) - w_j^pre) * P2[j, k], P2 = [((H + C) U^T) ⊙ M] U
+ * with H the undamped Gram and C the GPTAQ cross statistic (C = 0 without P1), and
+ * w^(0) the weights the sweep starts from (dead coordinates zeroed). P2 is not an
+ * argument: as U^T U is the inverse of H plus a diagonal, P2 = P1 + I - diag(U)^-1 U
+ * exactly, so the call needs only U (and P1).
  * Scale: per output channel s = 2 max_k |W[n][k]| / (2^b - 1) from W as given
  * (before dead coordinates are zeroed), s = 1 for an all-zero channel; zero
  * point z = 2^(b-1) ([G2PTQ] symmetric per-channel; [GPTQ blog] 4-bit grid
@@ -209,16 +219,21 @@ GPTQ_API gptq_status gptaq_residual(float *P1, const float *C, const float *U, i
  *   bits       2, 3, 4 or 8.  blocksize 16, 32, 64 or 128.
  *   P1         device fp32 [K][K] from gptaq_residual, or NULL (plain GPTQ).
  *              Requires groups == 1.
+ *   cae        0, or 1 for the compensation-aware error term (any groups).
  *   dead       device uint8 [groups][K] from gptq_prepare, or NULL (none dead).
  *   scales_in  device fp32 [N] fixed scales, or NULL (min-max as above).
  *   scales_out device fp32 [N] the scales used, or NULL.
  *   codes      device uint8 [N][K] codes c (required).
- *   loss       device fp32 [N] with 1/2 sum_j E_j^2 per channel, or NULL.
- *   ws         gptq_workspace_size(GPTQ_OP_QUANTIZE, K, N, groups, blocksize) bytes.
+ *   loss       device fp32 [N] with 1/2 sum_j E_j^2 per channel, or NULL; E_j is the
+ *              rounding error of the value quantised, (w_j^pre - q) / U_jj, with or
+ *              without cae.
+ *   ws         gptq_workspace_size(GPTQ_OP_QUANTIZE | (cae ? GPTQ_WS_CAE : 0), K, N,
+ *              groups, blocksize) bytes.
  *   status     device int32: GPTQ_ERR_NONFINITE for NaN/Inf in W or scales.
  */
 GPTQ_API gptq_status gptq_quantize_layer(void *W, int wdtype, int N, int K, const float *U, int groups,
-                                int bits, int blocksize, const float *P1, const uint8_t *dead,
+                                int bits, int blocksize, const float *P1, int cae,
+                                const uint8_t *dead,
                                 const float *scales_in, float *scales_out, uint8_t *codes,
                                 float *loss, int write_back, void *ws, size_t ws_bytes,
                                 int32_t *status, void *stream);
@@ -271,6 +286,7 @@ GPTQ_API gptq_status gptq_permute_hessian(float *out, const float *H, int K, con
  *              one per-channel scale (gptq_quantize_layer's) with the order of perm.
  *   perm       device int32 [K] processing order (gptq_act_order), or NULL (natural).
  *   P1         device fp32 [K][K] from gptaq_residual in processing order, or NULL.
+ *   cae        as gptq_quantize_layer; w^(0) is taken in processing order.
  *   dead       device uint8 [K] in processing order (gptq_prepare's dead_out), or NULL.
  *   scales_out device fp32 [N][ceil(K / groupsize)] ([N] when groupsize == 0), or NULL.
  *   g_idx_out  device int32 [K] group of each original coordinate (0 when
@@ -278,16 +294,44 @@ GPTQ_API gptq_status gptq_permute_hessian(float *out, const float *H, int K, con
  *   codes      device uint8 [N][K] in the original coordinate order (required).
  *   W, bits, loss, write_back, status: as gptq_quantize_layer (write-back in the
  *              original order).
- *   ws         gptq_workspace_size(GPTQ_OP_QUANTIZE_GROUPED, K, N, 1, blocksize) bytes.
+ *   ws         gptq_workspace_size(GPTQ_OP_QUANTIZE_GROUPED | (cae ? GPTQ_WS_CAE : 0), K,
+ *              N, 1, blocksize) bytes.
  */
 GPTQ_API gptq_status gptq_quantize_layer_grouped(void *W, int wdtype, int N, int K, const float *U,
                                                  int bits, int blocksize, int groupsize,
                                                  int static_groups, const int32_t *perm,
-                                                 const float *P1, const uint8_t *dead,
+                                                 const float *P1, int cae, const uint8_t *dead,
                                                  float *scales_out, int32_t *g_idx_out,
                                                  uint8_t *codes, float *loss, int write_back,
                                                  void *ws, size_t ws_bytes, int32_t *status,
                                                  void *stream);
+
+/*
+ * gptq_pack_codes -- codes [N][K] (uint8, < 2^bits) as low-bit words.
+ *
+ * [GPTQ blog] "落在格点上与真正存成低位权重是两步": codes on the grid are storage only
+ * once packed into wider integer containers, kept with scale, zero point and layout.
+ * Layout (the pages fix none): per output channel n, code k occupies bits
+ * [bits k, bits k + bits) of a little-endian bit stream whose bit t is bit t mod 32
+ * of words[n][t / 32]; 32 / bits whole codes per word for bits 2, 4, 8, and 32 codes
+ * per 3 words for bits 3 (some codes straddle two words). The row's last word has
+ * its unused high bits zero; words past ceil(K bits / 32) are not touched. The
+ * reconstruction is s (c - z) with z = 2^(bits-1) and the scales (and g_idx) of the
+ * quantisation call, in the original coordinate order.
+ *
+ *   codes     device uint8, row n at codes + n ld_codes (ld_codes >= K). Only the
+ *             low `bits` bits of each code are read.
+ *   words     device uint32, row n at words + n ld_words
+ *             (ld_words >= ceil(K bits / 32)).
+ *   N >= 0 (0: nothing to do), 1 <= K; bits 2, 3, 4 or 8.
+ *   Errors: GPTQ_ERR_ARG for sizes, strides or bits out of range, NULL pointers.
+ */
+GPTQ_API gptq_status gptq_pack_codes(const uint8_t *codes, int N, int K, int64_t ld_codes,
+                                     int bits, uint32_t *words, int64_t ld_words, void *stream);
+
+/* gptq_unpack_codes -- the inverse of gptq_pack_codes (same layout and arguments). */
+GPTQ_API gptq_status gptq_unpack_codes(const uint32_t *words, int N, int K, int64_t ld_words,
+                                       int bits, uint8_t *codes, int64_t ld_codes, void *stream);
 
 /* Workspace bytes for an operation (gptq_op); 0 when none is needed. */
 GPTQ_API size_t gptq_workspace_size(int op, int K, int N, int g, int blocksize);

@@ -20,11 +20,13 @@ GPTQ_OK, GPTQ_ERR_ARG, GPTQ_ERR_NOT_PD, GPTQ_ERR_NONFINITE = 0, 1, 2, 3
 GPTQ_ERR_CUDA, GPTQ_ERR_TIMEOUT, GPTQ_ERR_WORKSPACE = 4, 5, 6
 GPTQ_BF16, GPTQ_F32 = 0, 1
 GPTQ_OP_PREPARE, GPTQ_OP_RESIDUAL, GPTQ_OP_QUANTIZE, GPTQ_OP_QUANTIZE_GROUPED = 0, 1, 2, 3
+GPTQ_WS_CAE = 0x100
 
 EXPORTS = ("gptq_accumulate_hessian", "gptaq_accumulate_cross", "gptq_prepare",
            "gptq_prepare_noalloc",
            "gptaq_residual", "gptq_quantize_layer", "gptq_act_order", "gptq_permute_hessian",
-           "gptq_quantize_layer_grouped", "gptq_workspace_size",
+           "gptq_quantize_layer_grouped", "gptq_pack_codes", "gptq_unpack_codes",
+           "gptq_workspace_size",
            "gptq_kernel_launches", "gptq_status_string")
 
 _lib = None
@@ -52,11 +54,13 @@ def load_library():
         "gptq_prepare": [P, I, I, F, P, P, SZ, P, P],
         "gptq_prepare_noalloc": [P, I, I, F, P, P, P],
         "gptaq_residual": [P, P, P, I, P, SZ, P],
-        "gptq_quantize_layer": [P, I, I, I, P, I, I, I, P, P, P, P, P, P, I, P, SZ, P, P],
+        "gptq_quantize_layer": [P, I, I, I, P, I, I, I, P, I, P, P, P, P, P, I, P, SZ, P, P],
         "gptq_act_order": [P, I, P, P],
         "gptq_permute_hessian": [P, P, I, P, P],
-        "gptq_quantize_layer_grouped": [P, I, I, I, P, I, I, I, I, P, P, P, P, P, P, P, I, P, SZ,
-                                        P, P],
+        "gptq_quantize_layer_grouped": [P, I, I, I, P, I, I, I, I, P, P, I, P, P, P, P, P, I, P,
+                                        SZ, P, P],
+        "gptq_pack_codes": [P, I, I, I64, I, P, I64, P],
+        "gptq_unpack_codes": [P, I, I, I64, I, P, I64, P],
         "gptq_workspace_size": [I, I, I, I, I],
         "gptq_status_string": [I],
         "gptq_kernel_launches": [],
@@ -187,17 +191,18 @@ def gptaq_residual(P1, C, U, workspace=None, stream=None):
 
 def gptq_quantize_layer(W, U, bits, blocksize=128, groups=1, P1=None, dead=None, scales_in=None,
                         scales_out=None, codes=None, loss=None, write_back=False,
-                        workspace=None, status=None, stream=None):
-    """The shared-order sweep. Returns (codes, status); see include/gptq.h."""
+                        workspace=None, status=None, stream=None, cae=False):
+    """The shared-order sweep (cae: with the compensation-aware error term).
+    Returns (codes, status); see include/gptq.h."""
     lib = load_library()
     N, K = W.shape
     if codes is None:
         codes = torch.empty(N, K, dtype=torch.uint8, device=W.device)
     status = new_status(W.device) if status is None else status
-    ws = _workspace(gptq_workspace_size(GPTQ_OP_QUANTIZE, K, N, groups, blocksize), W.device,
-                    workspace)
+    op = GPTQ_OP_QUANTIZE | (GPTQ_WS_CAE if cae else 0)
+    ws = _workspace(gptq_workspace_size(op, K, N, groups, blocksize), W.device, workspace)
     code = lib.gptq_quantize_layer(_ptr(W), _dtype_code(W), N, K, _ptr(U), groups, bits,
-                                   blocksize, _ptr(P1), _ptr(dead), _ptr(scales_in),
+                                   blocksize, _ptr(P1), int(bool(cae)), _ptr(dead), _ptr(scales_in),
                                    _ptr(scales_out), _ptr(codes), _ptr(loss), int(write_back),
                                    _ptr(ws), ws.numel() * ws.element_size(), _ptr(status),
                                    _stream(stream))
@@ -229,7 +234,7 @@ def gptq_permute_hessian(H, perm, out=None, stream=None):
 def gptq_quantize_layer_grouped(W, U, bits, blocksize=128, groupsize=128, static_groups=False,
                                 perm=None, P1=None, dead=None, scales_out=None, g_idx=None,
                                 codes=None, loss=None, write_back=False, workspace=None,
-                                status=None, stream=None):
+                                status=None, stream=None, cae=False):
     """The sweep with input-dimension groups and an optional processing order.
     Returns (codes, scales [N][ceil(K / groupsize)], g_idx [K], status); see include/gptq.h."""
     lib = load_library()
@@ -242,13 +247,38 @@ def gptq_quantize_layer_grouped(W, U, bits, blocksize=128, groupsize=128, static
     if g_idx is None:
         g_idx = torch.empty(K, dtype=torch.int32, device=W.device)
     status = new_status(W.device) if status is None else status
-    ws = _workspace(gptq_workspace_size(GPTQ_OP_QUANTIZE_GROUPED, K, N, 1, blocksize), W.device,
-                    workspace)
+    op = GPTQ_OP_QUANTIZE_GROUPED | (GPTQ_WS_CAE if cae else 0)
+    ws = _workspace(gptq_workspace_size(op, K, N, 1, blocksize), W.device, workspace)
     code = lib.gptq_quantize_layer_grouped(_ptr(W), _dtype_code(W), N, K, _ptr(U), bits, blocksize,
                                            groupsize, int(bool(static_groups)), _ptr(perm),
-                                           _ptr(P1), _ptr(dead), _ptr(scales_out), _ptr(g_idx),
+                                           _ptr(P1), int(bool(cae)), _ptr(dead), _ptr(scales_out),
+                                           _ptr(g_idx),
                                            _ptr(codes), _ptr(loss), int(write_back), _ptr(ws),
                                            ws.numel() * ws.element_size(), _ptr(status),
                                            _stream(stream))
     _check(code, "gptq_quantize_layer_grouped")
     return codes, scales_out, g_idx, status
+
+
+def gptq_pack_codes(codes, bits, words=None, stream=None):
+    """codes uint8 [N][K] -> words int32 [N][ceil(K bits / 32)] holding the uint32 bit
+    patterns of include/gptq.h's layout (view them with .view(torch.uint32))."""
+    lib = load_library()
+    N, K = codes.shape
+    nw = (K * bits + 31) // 32
+    if words is None:
+        words = torch.empty(N, nw, dtype=torch.int32, device=codes.device)
+    _check(lib.gptq_pack_codes(_ptr(codes), N, K, codes.stride(0), bits, _ptr(words),
+                               words.stride(0), _stream(stream)), "gptq_pack_codes")
+    return words
+
+
+def gptq_unpack_codes(words, bits, K, codes=None, stream=None):
+    """The inverse of gptq_pack_codes: words [N][>= ceil(K bits / 32)] -> uint8 [N][K]."""
+    lib = load_library()
+    N = words.shape[0]
+    if codes is None:
+        codes = torch.empty(N, K, dtype=torch.uint8, device=words.device)
+    _check(lib.gptq_unpack_codes(_ptr(words), N, K, words.stride(0), bits, _ptr(codes),
+                                 codes.stride(0), _stream(stream)), "gptq_unpack_codes")
+    return codes

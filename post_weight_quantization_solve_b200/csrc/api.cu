@@ -21,16 +21,22 @@ size_t residual_workspace(int K);
 gptq_status residual(float *P1, const float *C, const float *U, int K, void *ws, cudaStream_t st);
 size_t quantize_workspace(int K, int N, int g, int blocksize);
 gptq_status quantize_layer(void *W, int wdtype, int N, int K, const float *U, int groups, int bits,
-                           int blocksize, const float *P1, const uint8_t *dead,
+                           int blocksize, const float *P1, int cae, const uint8_t *dead,
                            const float *scales_in, float *scales_out, uint8_t *codes, float *loss,
                            int write_back, void *ws, int32_t *status, cudaStream_t st);
 size_t quantize_grouped_workspace(int K, int N, int blocksize);
+size_t quantize_cae_extra(int K, int N);
 gptq_status quantize_layer_grouped(void *W, int wdtype, int N, int K, const float *U, int bits,
                                    int blocksize, int groupsize, int static_groups,
-                                   const int32_t *perm, const float *P1, const uint8_t *dead,
+                                   const int32_t *perm, const float *P1, int cae,
+                                   const uint8_t *dead,
                                    float *scales_out, int32_t *g_idx, uint8_t *codes, float *loss,
                                    int write_back, void *ws, int32_t *status, cudaStream_t st);
 gptq_status act_order(const float *H, int K, int32_t *perm, cudaStream_t st);
+gptq_status pack_codes(const uint8_t *codes, int N, int K, int64_t ldc, int bits, uint32_t *words,
+                       int64_t ldw, cudaStream_t st);
+gptq_status unpack_codes(const uint32_t *words, int N, int K, int64_t ldw, int bits,
+                         uint8_t *codes, int64_t ldc, cudaStream_t st);
 gptq_status permute_square(float *out, const float *H, int K, const int32_t *perm,
                            cudaStream_t st);
 }  // namespace gptq
@@ -109,10 +115,10 @@ gptq_status gptaq_residual(float *P1, const float *C, const float *U, int K, voi
 }
 
 gptq_status gptq_quantize_layer(void *W, int wdtype, int N, int K, const float *U, int groups,
-                                int bits, int blocksize, const float *P1, const uint8_t *dead,
-                                const float *scales_in, float *scales_out, uint8_t *codes,
-                                float *loss, int write_back, void *ws, size_t ws_bytes,
-                                int32_t *status, void *stream) {
+                                int bits, int blocksize, const float *P1, int cae,
+                                const uint8_t *dead, const float *scales_in, float *scales_out,
+                                uint8_t *codes, float *loss, int write_back, void *ws,
+                                size_t ws_bytes, int32_t *status, void *stream) {
     if (N < 1 || K < 1 || groups < 1 || N % groups != 0 || !W || !U || !codes || !status)
         return GPTQ_ERR_ARG;
     if (N > GPTQ_MAX_DIM || K > GPTQ_MAX_DIM || groups > 8) return GPTQ_ERR_ARG;
@@ -121,10 +127,12 @@ gptq_status gptq_quantize_layer(void *W, int wdtype, int N, int K, const float *
     if (blocksize != 16 && blocksize != 32 && blocksize != 64 && blocksize != 128)
         return GPTQ_ERR_ARG;
     if (P1 && groups != 1) return GPTQ_ERR_ARG;
+    if (cae != 0 && cae != 1) return GPTQ_ERR_ARG;
     if (!aligned(U, 16) || (P1 && !aligned(P1, 16))) return GPTQ_ERR_ARG;
-    if (!ws || !aligned(ws, 256) || ws_bytes < quantize_workspace(K, N, groups, blocksize))
+    if (!ws || !aligned(ws, 256) ||
+        ws_bytes < quantize_workspace(K, N, groups, blocksize) + (cae ? quantize_cae_extra(K, N) : 0))
         return GPTQ_ERR_WORKSPACE;
-    return quantize_layer(W, wdtype, N, K, U, groups, bits, blocksize, P1, dead, scales_in,
+    return quantize_layer(W, wdtype, N, K, U, groups, bits, blocksize, P1, cae, dead, scales_in,
                           scales_out, codes, loss, write_back, ws, status,
                           static_cast<cudaStream_t>(stream));
 }
@@ -142,8 +150,9 @@ gptq_status gptq_permute_hessian(float *out, const float *H, int K, const int32_
 
 gptq_status gptq_quantize_layer_grouped(void *W, int wdtype, int N, int K, const float *U,
                                         int bits, int blocksize, int groupsize, int static_groups,
-                                        const int32_t *perm, const float *P1, const uint8_t *dead,
-                                        float *scales_out, int32_t *g_idx_out, uint8_t *codes,
+                                        const int32_t *perm, const float *P1, int cae,
+                                        const uint8_t *dead, float *scales_out,
+                                        int32_t *g_idx_out, uint8_t *codes,
                                         float *loss, int write_back, void *ws, size_t ws_bytes,
                                         int32_t *status, void *stream) {
     if (N < 1 || K < 1 || !W || !U || !codes || !status) return GPTQ_ERR_ARG;
@@ -152,25 +161,54 @@ gptq_status gptq_quantize_layer_grouped(void *W, int wdtype, int N, int K, const
     if (groupsize != 0 && groupsize != 32 && groupsize != 64 && groupsize != 128) return GPTQ_ERR_ARG;
     if (blocksize != 32 && blocksize != 64 && blocksize != 128) return GPTQ_ERR_ARG;
     if (groupsize && blocksize % groupsize != 0) return GPTQ_ERR_ARG;
+    if (cae != 0 && cae != 1) return GPTQ_ERR_ARG;
     if (!aligned(U, 16) || (P1 && !aligned(P1, 16))) return GPTQ_ERR_ARG;
-    if (!ws || !aligned(ws, 256) || ws_bytes < quantize_grouped_workspace(K, N, blocksize))
+    if (!ws || !aligned(ws, 256) ||
+        ws_bytes < quantize_grouped_workspace(K, N, blocksize) + (cae ? quantize_cae_extra(K, N) : 0))
         return GPTQ_ERR_WORKSPACE;
     return quantize_layer_grouped(W, wdtype, N, K, U, bits, blocksize, groupsize, static_groups,
-                                  perm, P1, dead, scales_out, g_idx_out, codes, loss, write_back,
+                                  perm, P1, cae, dead, scales_out, g_idx_out, codes, loss, write_back,
                                   ws, status, static_cast<cudaStream_t>(stream));
+}
+
+static bool pack_args_ok(int N, int K, int bits, int64_t ldc, int64_t ldw) {
+    if (N < 0 || K < 1 || N > GPTQ_MAX_DIM || K > GPTQ_MAX_DIM) return false;
+    if (bits != 2 && bits != 3 && bits != 4 && bits != 8) return false;
+    return ldc >= K && ldw >= ((int64_t)K * bits + 31) / 32;
+}
+
+gptq_status gptq_pack_codes(const uint8_t *codes, int N, int K, int64_t ld_codes, int bits,
+                            uint32_t *words, int64_t ld_words, void *stream) {
+    if (!pack_args_ok(N, K, bits, ld_codes, ld_words)) return GPTQ_ERR_ARG;
+    if (N > 0 && (!codes || !words)) return GPTQ_ERR_ARG;
+    return pack_codes(codes, N, K, ld_codes, bits, words, ld_words,
+                      static_cast<cudaStream_t>(stream));
+}
+
+gptq_status gptq_unpack_codes(const uint32_t *words, int N, int K, int64_t ld_words, int bits,
+                              uint8_t *codes, int64_t ld_codes, void *stream) {
+    if (!pack_args_ok(N, K, bits, ld_codes, ld_words)) return GPTQ_ERR_ARG;
+    if (N > 0 && (!codes || !words)) return GPTQ_ERR_ARG;
+    return unpack_codes(words, N, K, ld_words, bits, codes, ld_codes,
+                        static_cast<cudaStream_t>(stream));
 }
 
 size_t gptq_workspace_size(int op, int K, int N, int g, int blocksize) {
     if (K < 1 || g < 1) return 0;
+    const bool cae = (op & GPTQ_WS_CAE) != 0;
+    op &= ~GPTQ_WS_CAE;
+    if (cae && op != GPTQ_OP_QUANTIZE && op != GPTQ_OP_QUANTIZE_GROUPED) return 0;
+    if (cae && N < 1) return 0;
+    const size_t extra = cae ? quantize_cae_extra(K, N) : 0;
     switch (op) {
         case GPTQ_OP_PREPARE: return prepare_workspace(K, g);
         case GPTQ_OP_RESIDUAL: return residual_workspace(K);
         case GPTQ_OP_QUANTIZE:
             if (N < 1 || blocksize < 1) return 0;
-            return quantize_workspace(K, N, g, blocksize);
+            return quantize_workspace(K, N, g, blocksize) + extra;
         case GPTQ_OP_QUANTIZE_GROUPED:
             if (N < 1 || blocksize < 1) return 0;
-            return quantize_grouped_workspace(K, N, blocksize);
+            return quantize_grouped_workspace(K, N, blocksize) + extra;
         default: return 0;
     }
 }

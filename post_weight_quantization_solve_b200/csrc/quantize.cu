@@ -7,6 +7,13 @@
 //   E_j = (w_j - q) / U_jj,   W_k -= U_jk E_j  (k later in the block),
 // and at the block end the far coordinates get W_far -= U[blk, far]^T E_blk.
 // [ResComp] item 3: GPTAQ adds w_j^pre * P1[j, k] the same way.
+// [ResComp] items 1-3, compensation-aware error (CAE): the row term
+// (w_j^(0) - w_j^pre) P2[j, k] with P2 = [((H + C) U^T) ⊙ M] U. Since U^T U = H_d^-1 and
+// H_d differs from H only on the diagonal, the H part of P2 is I - diag(U)^-1 U, and
+// the GPTQ step, the GPTAQ row and this row merge into one propagated error
+// E'_j = (w_j^(0) - q) / U_jj and a P1 row scaled by w_j^(0): P2 is never formed, the
+// sweep reads the starting weights w^(0) instead of the current ones for those two
+// terms, and the lazy updates are unchanged.
 //
 // Two-level lazy scheme: blocks of B coordinates inside super-blocks of S = 512.
 // After each block the rest of its super-block is updated ("near" update); after
@@ -19,7 +26,9 @@
 //   Eh, El    bf16 [S][ldE] normalised errors of the super-block as hi + lo pairs,
 //             row j - sb0, column grp * ldG + local channel (channel fastest, so the
 //             sweep's stores coalesce; the update reads it as an MN-major operand)
-//   Ph, Pl    bf16 [S][ldE] pre-rounding weights (GPTAQ), same layout
+//   Ph, Pl    bf16 [S][ldE] pre-rounding weights (GPTAQ; with CAE the starting
+//             weights), same layout
+//   W0k       fp32 [N][K] starting weights w^(0) (CAE only)
 //   Uh, Ul    bf16 [g][K][ldU] U as hi + lo pairs;  Qh, Ql  the same for P1
 // The sweep keeps each channel's block coordinates in registers: one thread per
 // channel for layers with many output channels (k_sweep_thread), four lanes per
@@ -61,10 +70,12 @@ __global__ void __launch_bounds__(256) k_scale_init(const T *__restrict__ W, flo
                                                     const float *__restrict__ scales_in,
                                                     float *__restrict__ scale, float *scales_out,
                                                     float *__restrict__ loss_acc, int vec,
-                                                    int32_t *status, const int32_t *perm) {
+                                                    int32_t *status, const int32_t *perm,
+                                                    float *__restrict__ W0k) {
     const int n = blockIdx.x;
     const T *wr = W + (int64_t)n * K;
     float *kr = Wk + (int64_t)n * K;
+    float *k0 = W0k ? W0k + (int64_t)n * K : nullptr;   // copy of the starting weights
     const uint8_t *dg = dead ? dead + (int64_t)(n / per_group) * K : nullptr;
     float amax = 0.f;
     bool bad = false;
@@ -74,6 +85,7 @@ __global__ void __launch_bounds__(256) k_scale_init(const T *__restrict__ W, flo
             bad |= !isfinite(x);
             amax = fmaxf(amax, fabsf(x));
             kr[k] = (dg && dg[k]) ? 0.f : x;
+            if (k0) k0[k] = kr[k];
         }
     } else if (vec) {   // rows 16-byte aligned for both W and Wk, K % 8 == 0
         for (int k = threadIdx.x * 8; k < K; k += 256 * 8) {
@@ -87,6 +99,10 @@ __global__ void __launch_bounds__(256) k_scale_init(const T *__restrict__ W, flo
             }
             *reinterpret_cast<float4 *>(kr + k) = make_float4(x[0], x[1], x[2], x[3]);
             *reinterpret_cast<float4 *>(kr + k + 4) = make_float4(x[4], x[5], x[6], x[7]);
+            if (k0) {
+                *reinterpret_cast<float4 *>(k0 + k) = make_float4(x[0], x[1], x[2], x[3]);
+                *reinterpret_cast<float4 *>(k0 + k + 4) = make_float4(x[4], x[5], x[6], x[7]);
+            }
         }
     } else {
         for (int k = threadIdx.x; k < K; k += 256) {
@@ -94,6 +110,7 @@ __global__ void __launch_bounds__(256) k_scale_init(const T *__restrict__ W, flo
             bad |= !isfinite(x);
             amax = fmaxf(amax, fabsf(x));
             kr[k] = (dg && dg[k]) ? 0.f : x;
+            if (k0) k0[k] = kr[k];
         }
     }
     __shared__ float red[8];
@@ -142,6 +159,13 @@ __device__ __forceinline__ void cp_async16(void *dst, const void *src, int src_b
                  "l"(src), "r"(src_bytes)
                  : "memory");
 }
+// 4-byte global -> shared copy; src_bytes = 0 writes a zero.
+__device__ __forceinline__ void cp_async4(void *dst, const void *src, int src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(
+                     static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                 "l"(src), "r"(src_bytes)
+                 : "memory");
+}
 __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.wait_all;" ::: "memory");
 }
@@ -158,14 +182,14 @@ __device__ __forceinline__ void cp_async_wait_all() {
 // always w[0]: the register array shifts by one sub-block after each phase. No block
 // barrier inside the sweep. U[blk, blk] (and P1) is staged once per CTA as its ten
 // 32 x 32 blocks on or above the diagonal.
-template <bool GPTAQ, int GMODE>
+template <bool GPTAQ, int GMODE, bool CAE>
 __global__ void __launch_bounds__(128, GPTAQ ? 2 : 4) k_sweep_lanes(
     float *__restrict__ Wk, int N, int per_group, int K, int i0, int bs,
     const float *__restrict__ U, const float *__restrict__ P1, const float *__restrict__ scale,
     int bits, uint8_t *__restrict__ codes, __nv_bfloat16 *__restrict__ Eh,
     __nv_bfloat16 *__restrict__ El, __nv_bfloat16 *__restrict__ Ph, __nv_bfloat16 *__restrict__ Pl,
     int ldE, int ldG, int erow0, float *__restrict__ loss_acc, int vec, const int32_t *status,
-    const SweepGroups sg) {
+    const SweepGroups sg, const float *__restrict__ W0k) {
     constexpr int NCH = 32, CLD = 132;
     if (failed(status)) return;
     extern __shared__ __align__(16) unsigned char smem[];
@@ -230,6 +254,22 @@ __global__ void __launch_bounds__(128, GPTAQ ? 2 : 4) k_sweep_lanes(
             for (int i = 0; i < 8; ++i) w[b][i] = (valid && c0 + i < bs) ? src[i] : 0.f;
         }
     }
+    // CAE: this lane's starting weights on the sub-block in work (w0c) and the next (w0n)
+    float w0c[8], w0n[8];
+    auto fetch_w0 = [&](int p, float (&d)[8]) {
+        const int c0 = 32 * p + 8 * q;
+        const float *src = W0k + n * K + i0 + c0;
+        if (valid && (vec & 1) && c0 + 8 <= bs) {
+            const float4 x0 = *reinterpret_cast<const float4 *>(src);
+            const float4 x1 = *reinterpret_cast<const float4 *>(src + 4);
+            d[0] = x0.x; d[1] = x0.y; d[2] = x0.z; d[3] = x0.w;
+            d[4] = x1.x; d[5] = x1.y; d[6] = x1.z; d[7] = x1.w;
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) d[i] = (valid && c0 + i < bs) ? src[i] : 0.f;
+        }
+    };
+    if (CAE) fetch_w0(0, w0c);
     if (GMODE == 2) {
         for (int j = q; j < bs; j += 4) {
             const float sj = valid ? sg.gsc[n * sg.ldg + sg.gsel[i0 + j]] : 1.f;
@@ -253,6 +293,7 @@ __global__ void __launch_bounds__(128, GPTAQ ? 2 : 4) k_sweep_lanes(
     for (int p = 0; p < nsb; ++p) {
         const int bbase = p * 4 - p * (p - 1) / 2;       // block (p, p)
         int64_t eoff = (int64_t)(erow0 + 32 * p) * ldE + ecol;
+        if (CAE && p + 1 < nsb) fetch_w0(p + 1, w0n);
         if (GMODE == 1 && (i0 + 32 * p) % sg.G == 0) {
             // entering a group: its scale from the channel's current weights
             float a = 0.f;
@@ -276,21 +317,25 @@ __global__ void __launch_bounds__(128, GPTAQ ? 2 : 4) k_sweep_lanes(
             const float rsj = GMODE == 2 ? sR[j * NCH + ch] : rs;
             const float wj = w[0][oi];
             const float cf = fminf(fmaxf(rintf(wj * rsj), cmin), cmax);
+            // ej: the rounding error of the value quantised (the loss); ep: the error
+            // propagated, which CAE measures from the starting weight
             const float ej = live ? fmaf(-sj, cf, wj) * rpiv[j] : 0.f;
-            const float e = __shfl_sync(0xffffffffu, ej, gsrc | oq);
+            const float w0j = CAE ? w0c[oi] : wj;
+            const float ep = CAE ? (live ? fmaf(-sj, cf, w0j) * rpiv[j] : 0.f) : ej;
+            const float e = __shfl_sync(0xffffffffu, ep, gsrc | oq);
             float v = 0.f;
-            if (GPTAQ) v = __shfl_sync(0xffffffffu, live ? wj : 0.f, gsrc | oq);
+            if (GPTAQ) v = __shfl_sync(0xffffffffu, live ? w0j : 0.f, gsrc | oq);
             if (q == oq && live) {
                 lacc = fmaf(ej, ej, lacc);
                 crow[j] = (uint8_t)(int)(cf + zf);
                 if (valid) {
-                    const __nv_bfloat16 eh = __float2bfloat16_rn(ej);
+                    const __nv_bfloat16 eh = __float2bfloat16_rn(ep);
                     Eh[eoff] = eh;
-                    El[eoff] = __float2bfloat16_rn(ej - __bfloat162float(eh));
+                    El[eoff] = __float2bfloat16_rn(ep - __bfloat162float(eh));
                     if (GPTAQ) {
-                        const __nv_bfloat16 ph = __float2bfloat16_rn(wj);
+                        const __nv_bfloat16 ph = __float2bfloat16_rn(w0j);
                         Ph[eoff] = ph;
-                        Pl[eoff] = __float2bfloat16_rn(wj - __bfloat162float(ph));
+                        Pl[eoff] = __float2bfloat16_rn(w0j - __bfloat162float(ph));
                     }
                 }
             }
@@ -321,6 +366,9 @@ __global__ void __launch_bounds__(128, GPTAQ ? 2 : 4) k_sweep_lanes(
         for (int b = 0; b < 3; ++b)
 #pragma unroll
             for (int i = 0; i < 8; ++i) w[b][i] = w[b + 1][i];
+        if (CAE)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) w0c[i] = w0n[i];
     }
     lacc += __shfl_xor_sync(0xffffffffu, lacc, 1);
     lacc += __shfl_xor_sync(0xffffffffu, lacc, 2);
@@ -351,14 +399,14 @@ __global__ void __launch_bounds__(128, GPTAQ ? 2 : 4) k_sweep_lanes(
 // is staged once per CTA as its ten 32 x 32 blocks on or above the diagonal.
 constexpr int SW_T = 64;
 
-template <bool GPTAQ, int GMODE>
+template <bool GPTAQ, int GMODE, bool CAE>
 __global__ void __launch_bounds__(SW_T, 1) k_sweep_thread(
     float *__restrict__ Wk, int N, int per_group, int K, int i0, int bs,
     const float *__restrict__ U, const float *__restrict__ P1, const float *__restrict__ scale,
     int bits, uint8_t *__restrict__ codes, __nv_bfloat16 *__restrict__ Eh,
     __nv_bfloat16 *__restrict__ El, __nv_bfloat16 *__restrict__ Ph, __nv_bfloat16 *__restrict__ Pl,
     int ldE, int ldG, int erow0, float *__restrict__ loss_acc, int vec, const int32_t *status,
-    const SweepGroups sg) {
+    const SweepGroups sg, const float *__restrict__ W0k) {
     if (failed(status)) return;
     extern __shared__ __align__(16) unsigned char smem[];
     float *Us = reinterpret_cast<float *>(smem);                 // [10][32][32]
@@ -368,6 +416,7 @@ __global__ void __launch_bounds__(SW_T, 1) k_sweep_thread(
     float *Vs = Es + 32 * SW_T;                                  // GPTAQ: pre-rounding weights
     float *sS = Vs + (GPTAQ ? 32 * SW_T : 0);                    // static groups: [SW_MAXB][SW_T]
     float *sR = sS + SW_MAXB * SW_T;                             // and 1 / s
+    float *W0s = sS + (GMODE == 2 ? 2 * SW_MAXB * SW_T : 0);     // CAE: [32][SW_T] w^(0)
 
     const int grp = blockIdx.y;
     const int cta_ch0 = blockIdx.x * SW_T;
@@ -404,6 +453,17 @@ __global__ void __launch_bounds__(SW_T, 1) k_sweep_thread(
         }
     }
     for (int j = tid; j < bs; j += SW_T) rpiv[j] = 1.f / __ldg(Ub + (int64_t)j * K + j);
+    // CAE: the channel's starting weights on sub-block p, into its own column of W0s
+    // (each thread reads only its column, so no barrier guards the refill)
+    auto fetch_w0 = [&](int p) {
+        const float *src = W0k + n * K + i0 + 32 * p;
+#pragma unroll 8
+        for (int t = 0; t < 32; ++t) {
+            const bool in = valid && 32 * p + t < bs;
+            cp_async4(W0s + t * SW_T + tid, in ? src + t : W0k, in ? 4 : 0);
+        }
+    };
+    if (CAE) fetch_w0(0);
 
     // the channel's block coordinates: sub-block b, pair i = coordinates (2 i, 2 i + 1)
     float2 w[4][16];
@@ -455,6 +515,7 @@ __global__ void __launch_bounds__(SW_T, 1) k_sweep_thread(
         const float *Pp = Ps + bbase * 1024;
         int64_t eoff = (int64_t)(erow0 + 32 * p) * ldE + ecol;
         uint32_t cw[4] = {0u, 0u, 0u, 0u};
+        if (CAE && p > 0) cp_async_wait_all();   // this phase's W0s, fetched during the last
         if (GMODE == 1 && (i0 + 32 * p) % sg.G == 0) {
             // entering a group: its scale from the channel's current weights
             float a = 0.f;
@@ -477,26 +538,30 @@ __global__ void __launch_bounds__(SW_T, 1) k_sweep_thread(
             const float rsj = GMODE == 2 ? sR[j * SW_T + tid] : rs;
             const float wj = (t & 1) ? w[0][t >> 1].y : w[0][t >> 1].x;
             const float cf = fminf(fmaxf(rintf(wj * rsj), cmin), cmax);
+            // ej: the rounding error of the value quantised (the loss); ep: the error
+            // propagated, which CAE measures from the starting weight
             const float ej = live ? fmaf(-sj, cf, wj) * rpiv[j] : 0.f;
-            const float vj = (GPTAQ && live) ? wj : 0.f;
-            Es[t * SW_T + tid] = ej;
+            const float w0j = CAE ? W0s[t * SW_T + tid] : wj;
+            const float ep = CAE ? (live ? fmaf(-sj, cf, w0j) * rpiv[j] : 0.f) : ej;
+            const float vj = (GPTAQ && live) ? w0j : 0.f;
+            Es[t * SW_T + tid] = ep;
             if (GPTAQ) Vs[t * SW_T + tid] = vj;
             cw[(t >> 2) & 3] |= (uint32_t)(int)(cf + zf) << (8 * (t & 3));
             if (live) {
                 lacc = fmaf(ej, ej, lacc);
                 if (valid) {
-                    const __nv_bfloat16 eh = __float2bfloat16_rn(ej);
+                    const __nv_bfloat16 eh = __float2bfloat16_rn(ep);
                     Eh[eoff] = eh;
-                    El[eoff] = __float2bfloat16_rn(ej - __bfloat162float(eh));
+                    El[eoff] = __float2bfloat16_rn(ep - __bfloat162float(eh));
                     if (GPTAQ) {
-                        const __nv_bfloat16 ph = __float2bfloat16_rn(wj);
+                        const __nv_bfloat16 ph = __float2bfloat16_rn(vj);
                         Ph[eoff] = ph;
-                        Pl[eoff] = __float2bfloat16_rn(wj - __bfloat162float(ph));
+                        Pl[eoff] = __float2bfloat16_rn(vj - __bfloat162float(ph));
                     }
                 }
             }
             eoff += ldE;
-            const float2 ne = make_float2(-ej, -ej);
+            const float2 ne = make_float2(-ep, -ep);
             const float2 vv = make_float2(vj, vj);
             // the rest of this sub-block: pairs from the one holding t + 1
 #pragma unroll
@@ -522,6 +587,9 @@ __global__ void __launch_bounds__(SW_T, 1) k_sweep_thread(
                 cw[0] = cw[1] = cw[2] = cw[3] = 0u;
             }
         }
+        // the phase is done with W0s: fetch the next sub-block's while the later
+        // sub-blocks are updated
+        if (CAE && p + 1 < nsb) fetch_w0(p + 1);
         // later sub-blocks: w_b -= sum_t E_t U[32 p + t, sub-block b] (+ GPTAQ term)
         if (nblk > 1) {
 #pragma unroll 2
@@ -677,9 +745,9 @@ size_t quantize_workspace(int K, int N, int g, int blocksize) {
     return round_up(c.off, 256);
 }
 
-static size_t sweep_thread_smem(bool gptaq, int gmode) {
+static size_t sweep_thread_smem(bool gptaq, int gmode, bool cae) {
     return sizeof(float) * ((10 * 1024 + 32 * SW_T) * (gptaq ? 2 : 1) + SW_MAXB +
-                            (gmode == 2 ? 2 * SW_MAXB * SW_T : 0));
+                            (gmode == 2 ? 2 * SW_MAXB * SW_T : 0) + (cae ? 32 * SW_T : 0));
 }
 static size_t sweep_lanes_smem(bool gptaq, int gmode) {
     return sizeof(float) * (10 * 1024 * (gptaq ? 2 : 1) + 32 * 33 + SW_MAXB +
@@ -689,16 +757,18 @@ static size_t sweep_lanes_smem(bool gptaq, int gmode) {
 typedef void (*SweepKernel)(float *, int, int, int, int, int, const float *, const float *,
                             const float *, int, uint8_t *, __nv_bfloat16 *, __nv_bfloat16 *,
                             __nv_bfloat16 *, __nv_bfloat16 *, int, int, int, float *, int,
-                            const int32_t *, const SweepGroups);
+                            const int32_t *, const SweepGroups, const float *);
 
-static SweepKernel sweep_kernel(bool per_thread, bool gptaq, int gmode) {
-    static const SweepKernel tab[2][2][3] = {
-        {{k_sweep_lanes<false, 0>, k_sweep_lanes<false, 1>, k_sweep_lanes<false, 2>},
-         {k_sweep_lanes<true, 0>, k_sweep_lanes<true, 1>, k_sweep_lanes<true, 2>}},
-        {{k_sweep_thread<false, 0>, k_sweep_thread<false, 1>, k_sweep_thread<false, 2>},
-         {k_sweep_thread<true, 0>, k_sweep_thread<true, 1>, k_sweep_thread<true, 2>}}};
-    return tab[per_thread][gptaq][gmode];
+#define GPTQ_SWEEP_MODES(K, A, C) {K<A, 0, C>, K<A, 1, C>, K<A, 2, C>}
+static SweepKernel sweep_kernel(bool per_thread, bool gptaq, int gmode, bool cae) {
+    static const SweepKernel tab[2][2][2][3] = {
+        {{GPTQ_SWEEP_MODES(k_sweep_lanes, false, false), GPTQ_SWEEP_MODES(k_sweep_lanes, false, true)},
+         {GPTQ_SWEEP_MODES(k_sweep_lanes, true, false), GPTQ_SWEEP_MODES(k_sweep_lanes, true, true)}},
+        {{GPTQ_SWEEP_MODES(k_sweep_thread, false, false), GPTQ_SWEEP_MODES(k_sweep_thread, false, true)},
+         {GPTQ_SWEEP_MODES(k_sweep_thread, true, false), GPTQ_SWEEP_MODES(k_sweep_thread, true, true)}}};
+    return tab[per_thread][gptaq][cae][gmode];
 }
+#undef GPTQ_SWEEP_MODES
 
 // Input-dimension groups and order of one quantisation (G == 0: per-channel scales,
 // natural order).
@@ -719,11 +789,14 @@ size_t quantize_grouped_workspace(int K, int N, int blocksize) {
     return round_up(c.off, 256);
 }
 
+// The compensation-aware term keeps the starting weights, after the rest.
+size_t quantize_cae_extra(int K, int N) { return round_up((size_t)N * K * sizeof(float), 256); }
+
 static gptq_status quantize_impl(void *W, int wdtype, int N, int K, const float *U, int groups,
                                  int bits, int blocksize, const float *P1, const uint8_t *dead,
                                  const float *scales_in, float *scales_out, uint8_t *codes,
                                  float *loss, int write_back, void *ws, int32_t *status,
-                                 cudaStream_t st, const QGroupOpts &go) {
+                                 cudaStream_t st, const QGroupOpts &go, int cae) {
     if (!update_tc_available()) return GPTQ_ERR_CUDA;
     const QLayout lay(K, N, groups);
     Carver cv(ws);
@@ -753,20 +826,29 @@ static gptq_status quantize_impl(void *W, int wdtype, int N, int K, const float 
         if (go.G > 0) gsc = go.scales ? go.scales : gws;
         if (go.perm) cp = cws;
     }
+    float *W0k = nullptr;
+    if (cae) {
+        Carver cx(ws);
+        cx.off = grouped ? quantize_grouped_workspace(K, N, blocksize)
+                         : quantize_workspace(K, N, groups, blocksize);
+        W0k = cx.take<float>((size_t)N * K);
+    }
     const int gmode = go.G == 0 ? 0 : (go.static_groups ? 2 : 1);
     const int per_group = N / groups;
     const int64_t KK = (int64_t)K * K;
     const bool gptaq = P1 != nullptr;
-    const int vin = (K % 8 == 0 && aligned(W, 16) && aligned(Wk, 16)) ? 1 : 0;
+    const int vin = (K % 8 == 0 && aligned(W, 16) && aligned(Wk, 16) && (!W0k || aligned(W0k, 16)))
+                        ? 1 : 0;
     const int vfin = (K % 16 == 0 && aligned(W, 16) && aligned(codes, 16)) ? 1 : 0;
     if (wdtype == GPTQ_F32)
         k_scale_init<float><<<N, 256, 0, st>>>(static_cast<const float *>(W), Wk, K, per_group, bits,
                                               dead, scales_in, scale, scales_out, loss_acc, vin,
-                                              status, go.perm);
+                                              status, go.perm, W0k);
     else
         k_scale_init<__nv_bfloat16><<<N, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(W), Wk, K,
                                                       per_group, bits, dead, scales_in, scale,
-                                                      scales_out, loss_acc, vin, status, go.perm);
+                                                      scales_out, loss_acc, vin, status, go.perm,
+                                                      W0k);
     gptq_status s = launch_status();
     if (s != GPTQ_OK) return s;
     if (grouped) {
@@ -822,8 +904,9 @@ static gptq_status quantize_impl(void *W, int wdtype, int N, int K, const float 
     const bool per_thread = (int64_t)N >= 2LL * 148 * 32;
     const int cta = per_thread ? SW_T : 128;
     const dim3 grid((per_group + (per_thread ? SW_T : 32) - 1) / (per_thread ? SW_T : 32), groups);
-    SweepKernel kern = sweep_kernel(per_thread, gptaq, gmode);
-    const size_t smem = per_thread ? sweep_thread_smem(gptaq, gmode) : sweep_lanes_smem(gptaq, gmode);
+    SweepKernel kern = sweep_kernel(per_thread, gptaq, gmode, cae != 0);
+    const size_t smem = per_thread ? sweep_thread_smem(gptaq, gmode, cae != 0)
+                                   : sweep_lanes_smem(gptaq, gmode);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
         return launch_status();
@@ -837,7 +920,7 @@ static gptq_status quantize_impl(void *W, int wdtype, int N, int K, const float 
             const int bs = i1 - i0;
             kern<<<grid, cta, smem, st>>>(Wk, N, per_group, K, i0, bs, U, P1, scale, bits, cp, Eh,
                                           El, Ph, Pl, lay.ldE, lay.ldG, i0 - sb0, loss_acc, vec,
-                                          status, sg);
+                                          status, sg, W0k);
             s = launch_status();
             if (s != GPTQ_OK) return s;
             if (i1 >= sb1) continue;
@@ -889,16 +972,17 @@ static gptq_status quantize_impl(void *W, int wdtype, int N, int K, const float 
 }
 
 gptq_status quantize_layer(void *W, int wdtype, int N, int K, const float *U, int groups, int bits,
-                           int blocksize, const float *P1, const uint8_t *dead,
+                           int blocksize, const float *P1, int cae, const uint8_t *dead,
                            const float *scales_in, float *scales_out, uint8_t *codes, float *loss,
                            int write_back, void *ws, int32_t *status, cudaStream_t st) {
     return quantize_impl(W, wdtype, N, K, U, groups, bits, blocksize, P1, dead, scales_in,
-                         scales_out, codes, loss, write_back, ws, status, st, QGroupOpts{});
+                         scales_out, codes, loss, write_back, ws, status, st, QGroupOpts{}, cae);
 }
 
 gptq_status quantize_layer_grouped(void *W, int wdtype, int N, int K, const float *U, int bits,
                                    int blocksize, int groupsize, int static_groups,
-                                   const int32_t *perm, const float *P1, const uint8_t *dead,
+                                   const int32_t *perm, const float *P1, int cae,
+                                   const uint8_t *dead,
                                    float *scales_out, int32_t *g_idx, uint8_t *codes, float *loss,
                                    int write_back, void *ws, int32_t *status, cudaStream_t st) {
     QGroupOpts go;
@@ -910,7 +994,7 @@ gptq_status quantize_layer_grouped(void *W, int wdtype, int N, int K, const floa
     // without groups the per-channel scales go straight to scales_out
     return quantize_impl(W, wdtype, N, K, U, 1, bits, blocksize, P1, dead, nullptr,
                          groupsize ? nullptr : scales_out, codes, loss, write_back, ws, status, st,
-                         go);
+                         go, cae);
 }
 
 }  // namespace gptq

@@ -58,6 +58,7 @@ class Workload:
     groupsize: int = 0            # input-dimension groups (0: per-channel scales)
     act_order: bool = False
     static_groups: bool = False
+    cae: bool = False             # compensation-aware error term
     extra: dict = field(default_factory=dict)
 
     def scaled(self, K=None, N=None, M=None, name=None, **kw):
@@ -86,6 +87,8 @@ WORKLOADS["mlp_up_w3"] = WORKLOADS["mlp_up"].scaled(name="mlp_up_w3", bits=3)
 # the same layer with 128-wide input groups (re-estimated) and act-order
 WORKLOADS["mlp_up_w3_g128"] = WORKLOADS["mlp_up"].scaled(name="mlp_up_w3_g128", bits=3,
                                                          groupsize=128, act_order=True)
+# the asymmetric-calibration layer with the compensation-aware error term as well
+WORKLOADS["gptaq_cae"] = WORKLOADS["gptaq"].scaled(name="gptaq_cae", cae=True)
 
 
 def hadamard(K: int, device="cpu") -> torch.Tensor:

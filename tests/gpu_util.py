@@ -40,7 +40,7 @@ def gpu_hessian(chunks, K, g=1, weights=None, device=None):
 
 
 def solve_on_gpu(H, W, bits, blocksize, percdamp, groups=1, P1_from_C=None, scales_in=None,
-                 write_back=True):
+                 write_back=True, cae=False):
     """prepare + (residual) + quantize on the device; returns host numpy results."""
     d = H.device
     K = H.shape[-1]
@@ -57,7 +57,7 @@ def solve_on_gpu(H, W, bits, blocksize, percdamp, groups=1, P1_from_C=None, scal
     loss = torch.empty(N, device=d)
     codes, status = gq.gptq_quantize_layer(
         Wd, U, bits, blocksize, groups=groups, P1=P1, dead=dead, scales_in=scales_in,
-        scales_out=scales, loss=loss, write_back=write_back, status=status)
+        scales_out=scales, loss=loss, write_back=write_back, status=status, cae=cae)
     gq.raise_on_status(status, "solve")
     torch.cuda.synchronize()
     return dict(U=U.double().cpu().numpy(), codes=codes.cpu().numpy().astype(np.float64),

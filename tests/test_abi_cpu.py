@@ -46,6 +46,13 @@ def test_workspace_sizes(lib):
     assert q >= 4096 * 14336 * 4
     assert gq.gptq_workspace_size(gq.GPTQ_OP_RESIDUAL, 512, 0, 1, 0) >= 512 * 512 * 4
     assert gq.gptq_workspace_size(7, 128, 1, 1, 1) == 0
+    # the compensation-aware term adds one fp32 copy of W; the flag fits only the sweeps
+    qc = gq.gptq_workspace_size(gq.GPTQ_OP_QUANTIZE | gq.GPTQ_WS_CAE, 4096, 14336, 1, 128)
+    assert qc >= q + 4096 * 14336 * 4
+    qg = gq.gptq_workspace_size(gq.GPTQ_OP_QUANTIZE_GROUPED, 4096, 14336, 1, 128)
+    assert gq.gptq_workspace_size(gq.GPTQ_OP_QUANTIZE_GROUPED | gq.GPTQ_WS_CAE, 4096, 14336, 1,
+                                  128) >= qg + 4096 * 14336 * 4
+    assert gq.gptq_workspace_size(gq.GPTQ_OP_PREPARE | gq.GPTQ_WS_CAE, 4096, 0, 1, 0) == 0
     assert gq.gptq_workspace_size(gq.GPTQ_OP_PREPARE, 0, 0, 1, 0) == 0
 
 
@@ -54,21 +61,38 @@ def test_host_argument_checks(lib):
     fake = P(1 << 20)   # never dereferenced: every call below fails its host checks
     ws = P(1 << 21)
     # quantize: bits, blocksize, groups, NULL pointers, GPTAQ with groups
-    assert lib.gptq_quantize_layer(fake, 0, 8, 16, fake, 1, 5, 128, None, None, None, None,
+    assert lib.gptq_quantize_layer(fake, 0, 8, 16, fake, 1, 5, 128, None, 0, None, None, None,
                                    fake, None, 0, ws, 1 << 30, fake, None) == gq.GPTQ_ERR_ARG
-    assert lib.gptq_quantize_layer(fake, 0, 8, 16, fake, 1, 4, 256, None, None, None, None,
+    assert lib.gptq_quantize_layer(fake, 0, 8, 16, fake, 1, 4, 256, None, 0, None, None, None,
                                    fake, None, 0, ws, 1 << 30, fake, None) == gq.GPTQ_ERR_ARG
-    assert lib.gptq_quantize_layer(fake, 0, 9, 16, fake, 2, 4, 128, None, None, None, None,
+    assert lib.gptq_quantize_layer(fake, 0, 9, 16, fake, 2, 4, 128, None, 0, None, None, None,
                                    fake, None, 0, ws, 1 << 30, fake, None) == gq.GPTQ_ERR_ARG
-    assert lib.gptq_quantize_layer(fake, 0, 8, 16, fake, 2, 4, 128, fake, None, None, None,
+    assert lib.gptq_quantize_layer(fake, 0, 8, 16, fake, 2, 4, 128, fake, 0, None, None, None,
                                    fake, None, 0, ws, 1 << 30, fake, None) == gq.GPTQ_ERR_ARG
-    assert lib.gptq_quantize_layer(fake, 0, 8, 16, fake, 1, 4, 128, None, None, None, None,
+    assert lib.gptq_quantize_layer(fake, 0, 8, 16, fake, 1, 4, 128, None, 0, None, None, None,
                                    None, None, 0, ws, 1 << 30, fake, None) == gq.GPTQ_ERR_ARG
-    assert lib.gptq_quantize_layer(fake, 0, 8, 16, fake, 1, 4, 128, None, None, None, None,
+    assert lib.gptq_quantize_layer(fake, 0, 8, 16, fake, 1, 4, 128, None, 0, None, None, None,
                                    fake, None, 0, ws, 16, fake, None) == gq.GPTQ_ERR_WORKSPACE
-    assert lib.gptq_quantize_layer(fake, 0, 8, 16, fake, 1, 4, 128, None, None, None, None,
+    assert lib.gptq_quantize_layer(fake, 0, 8, 16, fake, 1, 4, 128, None, 0, None, None, None,
                                    fake, None, 0, P((1 << 21) + 8), 1 << 30, fake,
                                    None) == gq.GPTQ_ERR_WORKSPACE
+    # cae: only 0 or 1, and its workspace includes the copy of W
+    assert lib.gptq_quantize_layer(fake, 0, 8, 16, fake, 1, 4, 128, None, 2, None, None, None,
+                                   fake, None, 0, ws, 1 << 30, fake, None) == gq.GPTQ_ERR_ARG
+    plain = gq.gptq_workspace_size(gq.GPTQ_OP_QUANTIZE, 16, 8, 1, 128)
+    assert lib.gptq_quantize_layer(fake, 0, 8, 16, fake, 1, 4, 128, None, 1, None, None, None,
+                                   fake, None, 0, ws, plain, fake, None) == gq.GPTQ_ERR_WORKSPACE
+    assert lib.gptq_quantize_layer_grouped(fake, 0, 8, 16, fake, 4, 128, 32, 0, None, None, 3,
+                                           None, None, None, fake, None, 0, ws, 1 << 30, fake,
+                                           None) == gq.GPTQ_ERR_ARG
+    # pack / unpack: bits, strides, NULL pointers; N == 0 does nothing
+    assert lib.gptq_pack_codes(fake, 4, 64, 64, 5, fake, 64, None) == gq.GPTQ_ERR_ARG
+    assert lib.gptq_pack_codes(fake, 4, 64, 63, 4, fake, 8, None) == gq.GPTQ_ERR_ARG
+    assert lib.gptq_pack_codes(fake, 4, 64, 64, 3, fake, 5, None) == gq.GPTQ_ERR_ARG
+    assert lib.gptq_pack_codes(None, 4, 64, 64, 3, fake, 6, None) == gq.GPTQ_ERR_ARG
+    assert lib.gptq_unpack_codes(fake, 4, 64, 1, 2, fake, 64, None) == gq.GPTQ_ERR_ARG
+    assert lib.gptq_pack_codes(fake, 0, 64, 64, 3, fake, 6, None) == gq.GPTQ_OK
+    assert lib.gptq_unpack_codes(fake, 0, 64, 6, 3, fake, 64, None) == gq.GPTQ_OK
     # prepare: negative damping, missing status, small workspace
     assert lib.gptq_prepare(fake, 16, 1, ctypes.c_float(-0.1), None, ws, 1 << 30, fake,
                             None) == gq.GPTQ_ERR_ARG
