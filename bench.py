@@ -35,8 +35,8 @@ METRIC = "GPTQ layer-solve ms & weights quantized/s (4096×14336, W3); % of TC/H
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the dominant
 # kernel, from an ncu capture of the same 65,536-token launch. Set to None whenever
-# k_gram_tc changes until it is captured again.
-GRAM_TRAFFIC_BYTES = 1.586335e9 + 0.500874e9
+# k_gram_tc2 changes until it is captured again.
+GRAM_TRAFFIC_BYTES = 1.588568e9 + 0.504924e9
 UNIT = "weights/s"
 
 
@@ -351,7 +351,8 @@ def run_ours(args, rank, world, local_rank):
     # is compared with the sustained bf16 peak (fallback 1400 TFLOP/s when no measurement)
     peak = peaks.get("bf16_tflops_sustained") or 1400.0
     achieved = flops_launch / (gram_launch_ms * 1e-3) / 1e12
-    roofline = {"kernel": ("k_gram_tc" if g == 1 else "k_gram_x_tc (weighted)") +
+    roofline = {"kernel": ("k_gram_tc2 (CTA pairs)" if g == 1 and K >= 256 else
+                           "k_gram_tc" if g == 1 else "k_gram_x_tc (weighted)") +
                           " (gptq_accumulate_hessian, tcgen05)", "bound": "tensor",
                 "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 4),

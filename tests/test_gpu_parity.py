@@ -243,3 +243,25 @@ def test_empty_chunk_is_noop():
     H = torch.ones(16, 16, device=d)
     gq.gptq_accumulate_hessian(H, torch.zeros(0, 16, dtype=torch.bfloat16, device=d))
     assert torch.all(H == 1)
+
+
+@pytest.mark.parametrize("K,M", [(256, 1000), (392, 3000), (1024, 70000)])
+def test_gram_cta_pair_matches_single_cta(K, M, monkeypatch):
+    # the CTA-pair Gram (256 x 256 tiles over two SMs) and the single-CTA Gram agree
+    # with each other and with the fp64 Gram, ragged tiles and token parts included
+    d = dev()
+    g = torch.Generator(device=d).manual_seed(K + M)
+    X = torch.randn(M, K, device=d, generator=g).to(torch.bfloat16)
+    out = {}
+    for pair in ("1", "0"):
+        monkeypatch.setenv("GPTQ_GRAM_PAIR", pair)
+        H = torch.zeros(K, K, device=d)
+        st = gq.new_status(d)
+        gq.gptq_accumulate_hessian(H, X, status=st)
+        gq.raise_on_status(st, "gram")
+        out[pair] = _np(H)
+    ref = O.gram(_np(X)) if K * M <= 400 * 3000 else 2.0 * _np((X.double().T @ X.double()))
+    for H in out.values():
+        assert rel_max(H, ref) <= TOL_H
+        assert np.abs(H - H.T).max() <= 1e-6 * np.abs(ref).max()
+    assert rel_max(out["1"], out["0"]) <= 1e-6
