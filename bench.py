@@ -13,7 +13,10 @@ step); the breakdown reports the layer solve (prepare + quantize) and the Gram.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
 For N > 1 each rank solves its own independent layer (weak scaling, no
-collective on the data path); timing is the max over ranks.
+collective on the data path); timing is the max over ranks. With --shard tokens the
+N ranks solve ONE layer instead (strong scaling): each accumulates its share of the
+token chunks, one NCCL all-reduce sums H (and C), every rank factors H, and each
+quantises its slice of the output channels.
 --impl reference times the fp64 CPU oracle on a bounded sample of the same job.
 """
 
@@ -51,6 +54,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-seconds", type=float, default=12.0)
+    ap.add_argument("--shard", choices=["layers", "tokens"], default="layers",
+                    help="N > 1: independent layers per rank, or one layer token-sharded")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the stream length (small profiling cases only)")
     return ap.parse_args()
@@ -200,40 +205,49 @@ def run_ours(args, rank, world, local_rank):
     import torch.distributed as dist
 
     import post_weight_quantization_solve_b200 as gq
-    from post_weight_quantization_solve_b200 import synth
+    from post_weight_quantization_solve_b200 import sharded, synth
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     gq.load_library()
     base = synth.WORKLOADS[args.workload]
-    wl = base.scaled(name=base.name, seed=base.seed + 1000 * rank)   # one layer per rank
+    tokens_sharded = args.shard == "tokens" and world > 1
+    # independent layers: one layer per rank; token-sharded: the same layer on every rank
+    wl = base.scaled(name=base.name, seed=base.seed + (0 if tokens_sharded else 1000 * rank))
     if args.tokens:
         wl = wl.scaled(name=base.name + f"_tokens{args.tokens}", M=args.tokens)
     K, N, M, ch = wl.K, wl.N, wl.M, wl.chunk
     nch = synth.num_chunks(wl)
+    # this rank's token chunks and output channels (everything when not token-sharded)
+    c0, c1 = sharded.chunk_range(nch, rank, world) if tokens_sharded else (0, nch)
+    n0, n1 = sharded.channel_range(N, rank, world) if tokens_sharded else (0, N)
+    Ml = min(M, c1 * ch) - c0 * ch     # tokens held by this rank
 
     g = wl.groups
-    X = torch.empty(M, K, dtype=wl.xdtype, device=dev)
-    for c in range(nch):
-        X[c * ch:(c + 1) * ch] = synth.tokens_chunk(wl, c, dev)
+    X = torch.empty(max(Ml, 0), K, dtype=wl.xdtype, device=dev)
+    for c in range(c0, c1):
+        X[(c - c0) * ch:(c - c0 + 1) * ch] = synth.tokens_chunk(wl, c, dev)
     Xf = None
     if wl.gptaq:                       # full-precision stream of the asymmetric calibration
-        Xf = torch.empty(M, K, dtype=wl.xdtype, device=dev)
-        for c in range(nch):
-            Xf[c * ch:(c + 1) * ch] = synth.fp_tokens_chunk(wl, c, dev)
+        Xf = torch.empty(max(Ml, 0), K, dtype=wl.xdtype, device=dev)
+        for c in range(c0, c1):
+            Xf[(c - c0) * ch:(c - c0 + 1) * ch] = synth.fp_tokens_chunk(wl, c, dev)
     TW = None
     if g > 1:                          # per-token group weights [g][M]
-        TW = torch.empty(g, M, device=dev)
-        for c in range(nch):
-            TW[:, c * ch:(c + 1) * ch] = synth.token_weights_chunk(wl, c, dev)
-    W = synth.weights(wl, dev).contiguous()
+        TW = torch.empty(g, max(Ml, 0), device=dev)
+        for c in range(c0, c1):
+            TW[:, (c - c0) * ch:(c - c0 + 1) * ch] = synth.token_weights_chunk(wl, c, dev)
+    W = synth.weights(wl, dev)[n0:n1].contiguous()
+    Nl = n1 - n0
     H = torch.empty((g, K, K) if g > 1 else (K, K), device=dev)
     C = torch.empty(K, K, device=dev) if wl.gptaq else None
     P1 = torch.empty(K, K, device=dev) if wl.gptaq else None
-    codes = torch.empty(N, K, dtype=torch.uint8, device=dev)
+    codes = torch.empty(Nl, K, dtype=torch.uint8, device=dev)
     grouped = wl.groupsize > 0 or wl.act_order
-    scales = (torch.empty(N, (K + wl.groupsize - 1) // wl.groupsize, device=dev) if wl.groupsize
-              else torch.empty(N, device=dev))
+    if grouped and g > 1:
+        raise SystemExit("input groups / act-order take one Hessian (groups == 1)")
+    scales = (torch.empty(Nl, (K + wl.groupsize - 1) // wl.groupsize, device=dev) if wl.groupsize
+              else torch.empty(Nl, device=dev))
     g_idx = torch.empty(K, dtype=torch.int32, device=dev) if grouped else None
     perm = torch.empty(K, dtype=torch.int32, device=dev) if wl.act_order else None
     Hp = torch.empty(K, K, device=dev) if wl.act_order else None
@@ -242,8 +256,9 @@ def run_ours(args, rank, world, local_rank):
                        device=dev)
     op_q = ((gq.GPTQ_OP_QUANTIZE_GROUPED if grouped else gq.GPTQ_OP_QUANTIZE) |
             (gq.GPTQ_WS_CAE if wl.cae else 0))
-    ws_q = torch.empty(gq.gptq_workspace_size(op_q, K, N, g, wl.blocksize), dtype=torch.uint8,
-                       device=dev)
+    ws_q = torch.empty(gq.gptq_workspace_size(op_q, K, max(Nl, 1), 1 if tokens_sharded else g,
+                                              wl.blocksize), dtype=torch.uint8, device=dev)
+    segments = sharded.channel_segments(n0, n1, N, g)
     Cp = torch.empty(K, K, device=dev) if (wl.act_order and wl.gptaq) else None
     ws_r = (torch.empty(gq.gptq_workspace_size(gq.GPTQ_OP_RESIDUAL, K, 0, 1, 0), dtype=torch.uint8,
                         device=dev) if wl.gptaq else None)
@@ -256,7 +271,7 @@ def run_ours(args, rank, world, local_rank):
             C.zero_()
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
         ev[0].record(stream)
-        for c in range(nch):
+        for c in range(c1 - c0):
             if record is not None:
                 a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a.record(stream)
@@ -268,6 +283,8 @@ def run_ours(args, rank, world, local_rank):
             if C is not None:
                 gq.gptaq_accumulate_cross(C, Xf[c * ch:(c + 1) * ch], X[c * ch:(c + 1) * ch],
                                           status=status, stream=stream)
+        if tokens_sharded:              # the solve's one exchange: sum the partial statistics
+            sharded.allreduce_statistics(H, C)
         ev[1].record(stream)
         Hs, Cs = H, C
         if perm is not None:            # act-order: solve in the reordered coordinates
@@ -279,16 +296,24 @@ def run_ours(args, rank, world, local_rank):
         if P1 is not None:
             gq.gptaq_residual(P1, Cs, Hs, workspace=ws_r, stream=stream)
         ev[2].record(stream)
-        if grouped:
+        if Nl == 0:
+            pass
+        elif grouped:
             gq.gptq_quantize_layer_grouped(W, Hs, wl.bits, wl.blocksize, wl.groupsize,
                                            static_groups=wl.static_groups, perm=perm, P1=P1,
                                            scales_out=scales, g_idx=g_idx, codes=codes,
                                            workspace=ws_q, status=status, stream=stream,
                                            cae=wl.cae)
-        else:
+        elif not tokens_sharded:
             gq.gptq_quantize_layer(W, Hs, wl.bits, wl.blocksize, groups=g, P1=P1,
                                    scales_out=scales, codes=codes, workspace=ws_q, status=status,
                                    stream=stream, cae=wl.cae)
+        else:                           # this rank's channels, segment by output group
+            for gi, a, b in segments:
+                gq.gptq_quantize_layer(W[a - n0:b - n0], Hs[gi] if g > 1 else Hs, wl.bits,
+                                       wl.blocksize, P1=P1, scales_out=scales[a - n0:b - n0],
+                                       codes=codes[a - n0:b - n0], workspace=ws_q,
+                                       status=status, stream=stream, cae=wl.cae)
         ev[3].record(stream)
         return ev
 
@@ -317,12 +342,12 @@ def run_ours(args, rank, world, local_rank):
     total_ms = t0.elapsed_time(t1)
     parts = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])]
                       for e in evs])
-    gram_launch_ms = float(np.mean([a.elapsed_time(b) for a, b in gram_ev]))
+    gram_launch_ms = (float(np.mean([a.elapsed_time(b) for a, b in gram_ev])) if gram_ev
+                      else 0.0)
 
     stats = torch.tensor([total_ms, *parts.mean(0).tolist(), gram_launch_ms], dtype=torch.float64,
                          device=dev)
-    if world > 1:
-        dist.all_reduce(stats, op=dist.ReduceOp.MAX)
+    sharded.max_over_ranks(stats)     # the slowest rank decides
     total_ms, gram_ms, prep_ms, quant_ms, gram_launch_ms = stats.tolist()
     ms_per_step = total_ms / args.steps
 
@@ -335,10 +360,10 @@ def run_ours(args, rank, world, local_rank):
     pk1.record(stream)
     torch.cuda.synchronize()
     pack_ms = pk0.elapsed_time(pk1) / 10
-    pack_bytes = N * K + words.numel() * 4
+    pack_bytes = Nl * K + words.numel() * 4
 
     e2e = None
-    if not args.no_e2e and g == 1 and not wl.gptaq:
+    if not args.no_e2e and g == 1 and not wl.gptaq and not tokens_sharded:
         e2e = run_e2e(args, wl, X, W, dev, gq, torch, dist, world)
 
     if rank != 0:
@@ -361,23 +386,28 @@ def run_ours(args, rank, world, local_rank):
                                 if peaks.get("bf16_tflops_sustained") else "fallback 1.4 PFLOP/s"),
                 "per_launch": f"{ch} tokens x K(K+1) = {flops_launch:.3e} FLOP (symmetric count)",
                 "ms_per_launch": round(gram_launch_ms, 4)}
-    weights = K * N * world
+    weights = K * N * (1 if tokens_sharded else world)
     line = {
         "metric": METRIC, "value": weights / (ms_per_step * 1e-3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16->f32",
+        "higher_is_better": True, "scaling": "strong" if tokens_sharded else "weak",
+        "vs_baseline": None, "dtype": "bf16->f32",
         "data": f"synthetic ({wl.stream} bf16 tokens, N(0,{wl.w_sigma}^2) bf16 weights)",
         "config": {"workload": f"{wl.name}: K={K} N={N} tokens={M} (chunks {nch}x{ch}) W{wl.bits} "
                                f"blocksize {wl.blocksize} percdamp {wl.percdamp} groups {g}"
                                + (" gptaq" if wl.gptaq else "") + (" cae" if wl.cae else "")
                                + (f" groupsize {wl.groupsize}" if wl.groupsize else "")
                                + (" act-order" if wl.act_order else ""),
-                   "l2": f"inputs larger than L2 (X {M * K * 2 / 1e9:.1f} GB)", "parallelism": f"{world} independent layers"},
+                   "l2": f"inputs larger than L2 (X {Ml * K * 2 / 1e9:.1f} GB per rank)",
+                   "parallelism": (f"{world} ranks on one layer: token-sharded Gram, NCCL "
+                                   "all-reduce of H, channel-sliced quantisation"
+                                   if tokens_sharded else f"{world} independent layers")},
         "breakdown": {"gram_ms": gram_ms, "prepare_ms": prep_ms, "quantize_ms": quant_ms,
                       "layer_solve_ms": prep_ms + quant_ms,
                       "solve_weights_per_s": K * N / ((prep_ms + quant_ms) * 1e-3),
                       "gram_tflops_symmetric": M * K * (K + 1) * g / (gram_ms * 1e-3) / 1e12,
                       "gram_includes_cross": bool(wl.gptaq),
+                      "gram_includes_allreduce": tokens_sharded,
                       "prepare_includes_residual": bool(wl.gptaq)},
         "roofline": roofline,
         "pack": {"kernel": "k_pack (gptq_pack_codes)", "ms": round(pack_ms, 4),
