@@ -186,7 +186,9 @@ def test_cae_grouped_act_order(G, static):
     assert rep["mismatches"] == 0, rep["mismatches"]
     assert 1.0 - rep["tie_flips"] / c_gpu.size >= CODE_SAME
     np.testing.assert_array_equal(g_idx.cpu().numpy(), rep["g_idx"])
-    np.testing.assert_allclose(_np(scales), rep["scales"], rtol=2e-5)
+    # re-estimated scales are maxima of compensated weights, so they carry the
+    # trajectory's error, which U's own tolerance bounds
+    np.testing.assert_allclose(_np(scales), rep["scales"], rtol=TOL_U)
     z = 2 ** (bits - 1)
     gi = g_idx.cpu().numpy()
     expect = torch.tensor((scales.cpu().numpy()[:, gi].astype(np.float32) *

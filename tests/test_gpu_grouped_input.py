@@ -93,7 +93,9 @@ def _run(K, N, bits, blocksize, G, static, act, seed, wdtype=torch.bfloat16, dea
     same = 1.0 - rep["tie_flips"] / c_gpu[rows].size
     assert same >= CODE_SAME
     np.testing.assert_array_equal(g_idx.cpu().numpy(), rep["g_idx"])
-    np.testing.assert_allclose(s_gpu[rows], rep["scales"], rtol=2e-5)
+    # re-estimated scales are maxima of compensated weights, so they carry the
+    # trajectory's error, which U's own tolerance bounds
+    np.testing.assert_allclose(s_gpu[rows], rep["scales"], rtol=TOL_U)
     # reconstruction on each coordinate's group grid, in the weights' dtype
     z = 2 ** (bits - 1)
     gi = g_idx.cpu().numpy()
