@@ -10,7 +10,9 @@ itself: the worked examples printed on the pages, closed forms, special cases,
 brute force and independent least-squares solves. Two readings are only partly
 pinned and say so where they are defined: which weight value multiplies the
 GPTAQ residual row (``gptaq`` arguments below), and likewise which weight values
-enter the compensation-aware row (``cae`` arguments).
+enter the compensation-aware row (``cae`` arguments). The first-order term
+(``first_order_*``) has no formula on the pages at all: its parity is unpinned
+against them and rests on internal pins only.
 """
 
 from .gptq_oracle import (  # noqa: F401
@@ -36,4 +38,7 @@ from .gptq_oracle import (  # noqa: F401
     replay_row_form_grouped,
     pack_codes,
     unpack_codes,
+    first_order_obq_sweep,
+    first_order_shift,
+    trust_region_beta,
 )

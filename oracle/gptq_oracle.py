@@ -667,3 +667,72 @@ def unpack_codes(words, bits, K):
             bit = (w[:, t // 32] >> np.uint64(t % 32)) & np.uint64(1)
             c[:, k] |= bit.astype(np.int64) << i
     return c
+
+
+# --------------------------------------------------------------------------------------
+# First-order (gradient) term with a trust-region step
+# --------------------------------------------------------------------------------------
+
+def first_order_obq_sweep(H_d, W, G, beta, bits):
+    """Sequential OBQ on the quadratic model with a first-order term, explicit form.
+
+    [G2PTQ] summary: the compensation keeps GPTQ's second-order update and adds the
+    first-order term from an exact gradient G of the block objective, scaled by a
+    trust-region factor beta in [0, 1]. The pages give no formula. Reading: per output
+    channel the objective around the given weights w0 is the quadratic model
+        L(w) = beta g^T (w - w0) + 1/2 (w - w0)^T H_d (w - w0),
+    and OBQ keeps every free coordinate at the model's minimiser given the fixed ones:
+    before step 0 all coordinates are free, so they start at w0 - beta H_d^-1 g; at
+    step q coordinate q is rounded on the grid of the weights being quantised (scale
+    from that starting point, as GPTQ takes it from the weights it is given) and fixed,
+    and the coordinates after q move to
+        x = w0_F - (H_d[F, F])^-1 (beta g_F + H_d[F, fixed] (w_fixed - w0_fixed)),
+    solved directly at every step (no Cholesky form, no lazy batching). With g = 0 this
+    is obq_sweep. PARITY UNPINNED against the pages: no formula or value is printed;
+    the pins are internal (reduction to GPTQ, the shifted-start identity, closed forms).
+
+    Returns (codes, W_hat, scales).
+    """
+    H_d = np.asarray(H_d, dtype=np.float64)
+    W0 = np.asarray(W, dtype=np.float64)
+    G = np.asarray(G, dtype=np.float64)
+    N, K = W0.shape
+    w = W0 - beta * np.linalg.solve(H_d, G.T).T
+    s, _ = symmetric_scale(w, bits)
+    codes = np.zeros((N, K))
+    for q in range(K):
+        c = quantize_codes(w[:, q], s, bits)
+        w[:, q] = dequantize(c, s, bits)
+        codes[:, q] = c
+        if q + 1 < K:
+            F = slice(q + 1, K)
+            fx = slice(0, q + 1)
+            rhs = beta * G[:, F].T + H_d[F, fx] @ (w[:, fx] - W0[:, fx]).T
+            w[:, F] = W0[:, F] - np.linalg.solve(H_d[F, F], rhs).T
+    return codes, w, s
+
+
+def first_order_shift(H_d, W, G, beta):
+    """w0 - beta H_d^-1 g per channel (the starting point of first_order_obq_sweep), and
+    gamma = sum_n g_n H_d^-1 g_n^T, the curvature-weighted size of the gradient: the
+    model's loss change along the step is -(beta - beta^2 / 2) gamma."""
+    H_d = np.asarray(H_d, dtype=np.float64)
+    G = np.asarray(G, dtype=np.float64)
+    Z = np.linalg.solve(H_d, G.T).T
+    return np.asarray(W, dtype=np.float64) - beta * Z, float(np.sum(G * Z))
+
+
+def trust_region_beta(alpha, loss_gptq, gamma):
+    """Largest beta in [0, 1] whose first-order loss change stays within alpha times the
+    GPTQ term's loss: (beta - beta^2 / 2) gamma <= alpha * loss_gptq.
+
+    [G2PTQ] summary: beta scales the first-order step so that the loss change it causes
+    does not exceed alpha times that of the GPTQ term (alpha searched per block on
+    [0, 3]). Reading: both changes are the quadratic model's, the first-order one along
+    the step -beta H^-1 g, the GPTQ one the sweep's loss (1/2 sum E^2)."""
+    if gamma <= 0.0:
+        return 1.0
+    x = alpha * loss_gptq / gamma
+    if x >= 0.5:
+        return 1.0
+    return 1.0 - np.sqrt(1.0 - 2.0 * x)

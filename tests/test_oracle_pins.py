@@ -671,3 +671,65 @@ def test_pack_three_bit_straddle_by_hand():
     assert int(w[0, 2]) & 0b11 == 0b10
     # the first ten codes fill word 0's low 30 bits
     assert int(w[0, 0]) & ((1 << 30) - 1) == sum(k % 8 << (3 * k) for k in range(10))
+
+
+# ------------------------------------------------------------------ first-order term (reading)
+
+def _fo_problem(K, N, seed):
+    rng = np.random.default_rng(seed)
+    X = rng.standard_normal((4 * K, K)) @ (np.eye(K) + 0.3 * rng.standard_normal((K, K)) / np.sqrt(K))
+    Hd, _ = O.dead_and_damp(O.gram(X), 0.01)
+    W = 0.02 * rng.standard_normal((N, K))
+    G = 0.5 * rng.standard_normal((N, K))
+    return Hd, W, G
+
+
+def test_first_order_zero_gradient_is_gptq():
+    Hd, W, _ = _fo_problem(12, 6, 1)
+    c, w, s = O.first_order_obq_sweep(Hd, W, np.zeros_like(W), 0.7, 3)
+    s0, _ = O.symmetric_scale(W, 3)
+    c0, w0, _ = O.obq_sweep(Hd, W, s0, 3)
+    np.testing.assert_array_equal(c, c0)
+    np.testing.assert_allclose(w, w0, atol=1e-12)
+
+
+def test_first_order_is_gptq_from_the_shifted_start():
+    # the quadratic model's sequential minimisers equal GPTQ's row form started at
+    # w0 - beta H^-1 g (solved per step vs Cholesky rows and lazy blocks)
+    Hd, W, G = _fo_problem(14, 7, 2)
+    for beta in (0.3, 1.0):
+        c, w, s = O.first_order_obq_sweep(Hd, W, G, beta, 3)
+        Ws, _ = O.first_order_shift(Hd, W, G, beta)
+        np.testing.assert_allclose(s, O.symmetric_scale(Ws, 3)[0], rtol=1e-12)
+        for B in (1, 4, 14):
+            c_row, w_row, _ = O.row_form_sweep(O.upper_factor(Hd), Ws, s, 3, B)
+            np.testing.assert_array_equal(c_row, c)
+            np.testing.assert_allclose(w_row, w, atol=1e-10)
+
+
+def test_first_order_diagonal_hessian_is_rtn_of_the_newton_point():
+    rng = np.random.default_rng(3)
+    K, N = 9, 5
+    h = rng.uniform(0.5, 2.0, K)
+    W = 0.02 * rng.standard_normal((N, K))
+    G = 0.01 * rng.standard_normal((N, K))
+    c, w, s = O.first_order_obq_sweep(np.diag(h), W, G, 0.6, 4)
+    target = W - 0.6 * G / h
+    np.testing.assert_array_equal(c, O.quantize_codes(target, s[:, None], 4))
+
+
+def test_first_order_gamma_and_trust_region():
+    Hd, W, G = _fo_problem(10, 4, 4)
+    _, gamma = O.first_order_shift(Hd, W, G, 1.0)
+    assert gamma == pytest.approx(sum(G[n] @ np.linalg.inv(Hd) @ G[n] for n in range(4)), rel=1e-12)
+    # the factor meets the bound with equality below 1, is 1 when the bound allows it,
+    # and 0 when alpha is 0
+    for alpha, lq in ((0.1, 0.05 * gamma), (2.0, 0.4 * gamma), (0.0, gamma)):
+        b = O.trust_region_beta(alpha, lq, gamma)
+        assert 0.0 <= b <= 1.0
+        lhs = (b - b * b / 2) * gamma
+        if b < 1.0:
+            assert lhs == pytest.approx(alpha * lq, rel=1e-12, abs=1e-300)
+        else:
+            assert lhs <= alpha * lq + 1e-15
+    assert O.trust_region_beta(1.0, 1.0, 0.0) == 1.0
