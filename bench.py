@@ -248,6 +248,16 @@ def run_ours(args, rank, world, local_rank):
         raise SystemExit("input groups / act-order take one Hessian (groups == 1)")
     scales = (torch.empty(Nl, (K + wl.groupsize - 1) // wl.groupsize, device=dev) if wl.groupsize
               else torch.empty(Nl, device=dev))
+    # first-order term: the sweep quantises an fp32 copy shifted by -beta G H^-1
+    Gd = W32 = gamma = ws_f = None
+    if wl.first_order:
+        if grouped or g > 1 or wl.gptaq or tokens_sharded:
+            raise SystemExit("the first-order workload is plain per-channel GPTQ on one layer")
+        Gd = synth.gradient(wl, dev)[n0:n1].contiguous()
+        W32 = torch.empty(Nl, K, device=dev)
+        gamma = torch.zeros(1, dtype=torch.float64, device=dev)
+        ws_f = torch.empty(gq.gptq_workspace_size(gq.GPTQ_OP_FIRST_ORDER, K, Nl, 1, 0),
+                           dtype=torch.uint8, device=dev)
     g_idx = torch.empty(K, dtype=torch.int32, device=dev) if grouped else None
     perm = torch.empty(K, dtype=torch.int32, device=dev) if wl.act_order else None
     Hp = torch.empty(K, K, device=dev) if wl.act_order else None
@@ -304,6 +314,12 @@ def run_ours(args, rank, world, local_rank):
                                            scales_out=scales, g_idx=g_idx, codes=codes,
                                            workspace=ws_q, status=status, stream=stream,
                                            cae=wl.cae)
+        elif wl.first_order:
+            W32.copy_(W)
+            gq.gptq_first_order_shift(W32, Hs, Gd, wl.first_order, gamma=gamma, workspace=ws_f,
+                                      status=status, stream=stream)
+            gq.gptq_quantize_layer(W32, Hs, wl.bits, wl.blocksize, scales_out=scales, codes=codes,
+                                   workspace=ws_q, status=status, stream=stream)
         elif not tokens_sharded:
             gq.gptq_quantize_layer(W, Hs, wl.bits, wl.blocksize, groups=g, P1=P1,
                                    scales_out=scales, codes=codes, workspace=ws_q, status=status,
@@ -397,7 +413,8 @@ def run_ours(args, rank, world, local_rank):
                                f"blocksize {wl.blocksize} percdamp {wl.percdamp} groups {g}"
                                + (" gptaq" if wl.gptaq else "") + (" cae" if wl.cae else "")
                                + (f" groupsize {wl.groupsize}" if wl.groupsize else "")
-                               + (" act-order" if wl.act_order else ""),
+                               + (" act-order" if wl.act_order else "")
+                               + (f" first-order beta {wl.first_order}" if wl.first_order else ""),
                    "l2": f"inputs larger than L2 (X {Ml * K * 2 / 1e9:.1f} GB per rank)",
                    "parallelism": (f"{world} ranks on one layer: token-sharded Gram, NCCL "
                                    "all-reduce of H, channel-sliced quantisation"
@@ -408,6 +425,7 @@ def run_ours(args, rank, world, local_rank):
                       "gram_tflops_symmetric": M * K * (K + 1) * g / (gram_ms * 1e-3) / 1e12,
                       "gram_includes_cross": bool(wl.gptaq),
                       "gram_includes_allreduce": tokens_sharded,
+                      "quantize_includes_first_order_shift": bool(wl.first_order),
                       "prepare_includes_residual": bool(wl.gptaq)},
         "roofline": roofline,
         "pack": {"kernel": "k_pack (gptq_pack_codes)", "ms": round(pack_ms, 4),

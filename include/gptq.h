@@ -69,7 +69,8 @@ typedef enum {
     GPTQ_OP_PREPARE = 0,
     GPTQ_OP_RESIDUAL = 1,
     GPTQ_OP_QUANTIZE = 2,
-    GPTQ_OP_QUANTIZE_GROUPED = 3
+    GPTQ_OP_QUANTIZE_GROUPED = 3,
+    GPTQ_OP_FIRST_ORDER = 4
 } gptq_op;
 
 /* OR-ed into GPTQ_OP_QUANTIZE or GPTQ_OP_QUANTIZE_GROUPED: the workspace of a call
@@ -332,6 +333,42 @@ GPTQ_API gptq_status gptq_pack_codes(const uint8_t *codes, int N, int K, int64_t
 /* gptq_unpack_codes -- the inverse of gptq_pack_codes (same layout and arguments). */
 GPTQ_API gptq_status gptq_unpack_codes(const uint32_t *words, int N, int K, int64_t ld_words,
                                        int bits, uint8_t *codes, int64_t ld_codes, void *stream);
+
+/*
+ * gptq_first_order_shift -- the first-order (gradient) term as a shifted start:
+ * W <- W - beta G H^-1 per output channel, with H^-1 = U^T U.
+ *
+ * [G2PTQ] summary: the compensation keeps GPTQ's second-order update and adds the
+ * first-order term of an exact gradient G of the block objective, scaled by a
+ * trust-region factor beta in [0, 1]. The pages print no formula. Reading: the
+ * objective per channel is the quadratic model beta g^T d + 1/2 d^T H d around the
+ * given weights; sequential OBQ on it is GPTQ started from the model's minimiser
+ * w - beta H^-1 g. So: shift an fp32 copy of W with this call, then quantise that
+ * copy with gptq_quantize_layer (its scales come from the shifted weights, as GPTQ
+ * takes them from the weights it is given).
+ *
+ *   W      device fp32 [N][K], shifted in place.
+ *   U      device fp32 [K][K] from gptq_prepare (g = 1).
+ *   G      device [N][K] gradient, dtype gdtype (GPTQ_BF16 or GPTQ_F32).
+ *   beta   in [0, 1] (gptq_trust_region_beta).
+ *   gamma  device double, or NULL: sum_n g_n H^-1 g_n^T; the model's loss change
+ *          along the step is -(beta - beta^2 / 2) gamma.
+ *   ws     gptq_workspace_size(GPTQ_OP_FIRST_ORDER, K, N, 1, 0) bytes.
+ *   Errors: GPTQ_ERR_ARG for sizes, dtype, beta outside [0, 1] or NULL pointers.
+ */
+GPTQ_API gptq_status gptq_first_order_shift(float *W, int N, int K, const float *U, const void *G,
+                                            int gdtype, float beta, double *gamma, void *ws,
+                                            size_t ws_bytes, int32_t *status, void *stream);
+
+/*
+ * gptq_trust_region_beta -- host: the largest beta in [0, 1] whose first-order loss
+ * change stays within alpha times the GPTQ term's: (beta - beta^2/2) gamma <=
+ * alpha loss_gptq ([G2PTQ] summary: beta bounds the first-order step by alpha times
+ * the GPTQ term's loss change; alpha is searched per block on [0, 3]). loss_gptq is
+ * the sweep's loss (sum of gptq_quantize_layer's loss output); gamma as above.
+ * gamma <= 0 gives 1; a negative or NaN ratio gives 0.
+ */
+GPTQ_API float gptq_trust_region_beta(float alpha, double loss_gptq, double gamma);
 
 /* Workspace bytes for an operation (gptq_op); 0 when none is needed. */
 GPTQ_API size_t gptq_workspace_size(int op, int K, int N, int g, int blocksize);

@@ -20,12 +20,14 @@ GPTQ_OK, GPTQ_ERR_ARG, GPTQ_ERR_NOT_PD, GPTQ_ERR_NONFINITE = 0, 1, 2, 3
 GPTQ_ERR_CUDA, GPTQ_ERR_TIMEOUT, GPTQ_ERR_WORKSPACE = 4, 5, 6
 GPTQ_BF16, GPTQ_F32 = 0, 1
 GPTQ_OP_PREPARE, GPTQ_OP_RESIDUAL, GPTQ_OP_QUANTIZE, GPTQ_OP_QUANTIZE_GROUPED = 0, 1, 2, 3
+GPTQ_OP_FIRST_ORDER = 4
 GPTQ_WS_CAE = 0x100
 
 EXPORTS = ("gptq_accumulate_hessian", "gptaq_accumulate_cross", "gptq_prepare",
            "gptq_prepare_noalloc",
            "gptaq_residual", "gptq_quantize_layer", "gptq_act_order", "gptq_permute_hessian",
            "gptq_quantize_layer_grouped", "gptq_pack_codes", "gptq_unpack_codes",
+           "gptq_first_order_shift", "gptq_trust_region_beta",
            "gptq_workspace_size",
            "gptq_kernel_launches", "gptq_status_string")
 
@@ -61,6 +63,8 @@ def load_library():
                                         SZ, P, P],
         "gptq_pack_codes": [P, I, I, I64, I, P, I64, P],
         "gptq_unpack_codes": [P, I, I, I64, I, P, I64, P],
+        "gptq_first_order_shift": [P, I, I, P, P, I, F, P, P, SZ, P, P],
+        "gptq_trust_region_beta": [F, ctypes.c_double, ctypes.c_double],
         "gptq_workspace_size": [I, I, I, I, I],
         "gptq_status_string": [I],
         "gptq_kernel_launches": [],
@@ -70,6 +74,7 @@ def load_library():
         fn.argtypes = args
         fn.restype = ctypes.c_int
     lib.gptq_workspace_size.restype = ctypes.c_size_t
+    lib.gptq_trust_region_beta.restype = ctypes.c_float
     lib.gptq_status_string.restype = ctypes.c_char_p
     lib.gptq_kernel_launches.restype = ctypes.c_ulonglong
     _lib = lib
@@ -282,3 +287,27 @@ def gptq_unpack_codes(words, bits, K, codes=None, stream=None):
     _check(lib.gptq_unpack_codes(_ptr(words), N, K, words.stride(0), bits, _ptr(codes),
                                  codes.stride(0), _stream(stream)), "gptq_unpack_codes")
     return codes
+
+
+def gptq_first_order_shift(W, U, G, beta, gamma=None, workspace=None, status=None, stream=None):
+    """W (fp32 [N][K]) <- W - beta G H^-1 in place; gamma (float64 [1]) gets
+    sum_n g_n H^-1 g_n^T when given. Returns status; see include/gptq.h."""
+    lib = load_library()
+    if W.dtype != torch.float32:
+        raise TypeError("gptq_first_order_shift shifts an fp32 copy of the weights")
+    N, K = W.shape
+    status = new_status(W.device) if status is None else status
+    ws = _workspace(gptq_workspace_size(GPTQ_OP_FIRST_ORDER, K, N, 1, 0), W.device, workspace)
+    code = lib.gptq_first_order_shift(_ptr(W), N, K, _ptr(U), _ptr(G), _dtype_code(G),
+                                      ctypes.c_float(beta), _ptr(gamma), _ptr(ws),
+                                      ws.numel() * ws.element_size(), _ptr(status),
+                                      _stream(stream))
+    _check(code, "gptq_first_order_shift")
+    return status
+
+
+def gptq_trust_region_beta(alpha, loss_gptq, gamma):
+    """Host: the largest beta in [0, 1] with (beta - beta^2/2) gamma <= alpha loss_gptq."""
+    return float(load_library().gptq_trust_region_beta(ctypes.c_float(alpha),
+                                                        ctypes.c_double(loss_gptq),
+                                                        ctypes.c_double(gamma)))

@@ -1,5 +1,7 @@
 // C ABI entry points: argument checks, workspace sizing, dispatch. Every check
 // here runs on the host before anything is enqueued.
+#include <cmath>
+
 #include "common.cuh"
 
 namespace gptq {
@@ -37,6 +39,10 @@ gptq_status pack_codes(const uint8_t *codes, int N, int K, int64_t ldc, int bits
                        int64_t ldw, cudaStream_t st);
 gptq_status unpack_codes(const uint32_t *words, int N, int K, int64_t ldw, int bits,
                          uint8_t *codes, int64_t ldc, cudaStream_t st);
+size_t first_order_workspace(int K, int N);
+gptq_status first_order_shift(float *W, int N, int K, const float *U, const void *G, int gdtype,
+                              float beta, double *gamma, void *ws, int32_t *status,
+                              cudaStream_t st);
 gptq_status permute_square(float *out, const float *H, int K, const int32_t *perm,
                            cudaStream_t st);
 }  // namespace gptq
@@ -193,6 +199,26 @@ gptq_status gptq_unpack_codes(const uint32_t *words, int N, int K, int64_t ld_wo
                         static_cast<cudaStream_t>(stream));
 }
 
+gptq_status gptq_first_order_shift(float *W, int N, int K, const float *U, const void *G,
+                                  int gdtype, float beta, double *gamma, void *ws,
+                                  size_t ws_bytes, int32_t *status, void *stream) {
+    if (N < 1 || K < 1 || N > GPTQ_MAX_DIM || K > GPTQ_MAX_DIM) return GPTQ_ERR_ARG;
+    if (!W || !U || !G || !status || !valid_dtype(gdtype)) return GPTQ_ERR_ARG;
+    if (!(beta >= 0.f && beta <= 1.f)) return GPTQ_ERR_ARG;
+    if (!ws || !aligned(ws, 256) || ws_bytes < first_order_workspace(K, N)) return GPTQ_ERR_WORKSPACE;
+    return first_order_shift(W, N, K, U, G, gdtype, beta, gamma, ws, status,
+                             static_cast<cudaStream_t>(stream));
+}
+
+float gptq_trust_region_beta(float alpha, double loss_gptq, double gamma) {
+    // largest beta in [0, 1] with (beta - beta^2 / 2) gamma <= alpha loss_gptq
+    if (!(gamma > 0.0)) return 1.f;
+    const double x = (double)alpha * loss_gptq / gamma;
+    if (!(x >= 0.0)) return 0.f;
+    if (x >= 0.5) return 1.f;
+    return (float)(1.0 - sqrt(1.0 - 2.0 * x));
+}
+
 size_t gptq_workspace_size(int op, int K, int N, int g, int blocksize) {
     if (K < 1 || g < 1) return 0;
     const bool cae = (op & GPTQ_WS_CAE) != 0;
@@ -209,6 +235,9 @@ size_t gptq_workspace_size(int op, int K, int N, int g, int blocksize) {
         case GPTQ_OP_QUANTIZE_GROUPED:
             if (N < 1 || blocksize < 1) return 0;
             return quantize_grouped_workspace(K, N, blocksize) + extra;
+        case GPTQ_OP_FIRST_ORDER:
+            if (N < 1) return 0;
+            return first_order_workspace(K, N);
         default: return 0;
     }
 }

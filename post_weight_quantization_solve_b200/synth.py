@@ -29,7 +29,7 @@ import torch
 CHUNK_TOKENS = 65536
 
 # tensor ids inside a workload
-T_X, T_W, T_MIX, T_OUTLIER, T_SIGNS, T_NOISE, T_TOKW, T_CHI = range(8)
+T_X, T_W, T_MIX, T_OUTLIER, T_SIGNS, T_NOISE, T_TOKW, T_CHI, T_GRAD = range(9)
 
 
 def generator(seed: int, tensor_id: int, chunk: int = 0, device="cpu") -> torch.Generator:
@@ -59,6 +59,7 @@ class Workload:
     act_order: bool = False
     static_groups: bool = False
     cae: bool = False             # compensation-aware error term
+    first_order: float = 0.0      # beta of the first-order (gradient) term; 0: none
     extra: dict = field(default_factory=dict)
 
     def scaled(self, K=None, N=None, M=None, name=None, **kw):
@@ -89,6 +90,9 @@ WORKLOADS["mlp_up_w3_g128"] = WORKLOADS["mlp_up"].scaled(name="mlp_up_w3_g128", 
                                                          groupsize=128, act_order=True)
 # the asymmetric-calibration layer with the compensation-aware error term as well
 WORKLOADS["gptaq_cae"] = WORKLOADS["gptaq"].scaled(name="gptaq_cae", cae=True)
+# the headline layer with a first-order term (synthetic gradient, beta 0.5)
+WORKLOADS["mlp_up_w3_fo"] = WORKLOADS["mlp_up"].scaled(name="mlp_up_w3_fo", bits=3,
+                                                       first_order=0.5)
 
 
 def hadamard(K: int, device="cpu") -> torch.Tensor:
@@ -207,3 +211,11 @@ def weights(wl: Workload, device="cpu") -> torch.Tensor:
     if wl.stream == "rotated":
         W = W @ _rotation(wl, device)
     return W.to(wl.xdtype)
+
+
+def gradient(wl: Workload, device="cpu") -> torch.Tensor:
+    """A synthetic gradient of the block objective w.r.t. W[N][K] for the first-order
+    term: N(0, (w_sigma / 10)^2), fp32 (the gradient comes from backprop, which the
+    solve does not run)."""
+    g = torch.randn(wl.N, wl.K, generator=generator(wl.seed, T_GRAD, 0, device), device=device)
+    return g * (wl.w_sigma / 10)

@@ -93,6 +93,13 @@ def test_host_argument_checks(lib):
     assert lib.gptq_unpack_codes(fake, 4, 64, 1, 2, fake, 64, None) == gq.GPTQ_ERR_ARG
     assert lib.gptq_pack_codes(fake, 0, 64, 64, 3, fake, 6, None) == gq.GPTQ_OK
     assert lib.gptq_unpack_codes(fake, 0, 64, 6, 3, fake, 64, None) == gq.GPTQ_OK
+    # first-order shift: beta in [0, 1], dtype, workspace
+    assert lib.gptq_first_order_shift(fake, 8, 16, fake, fake, 0, ctypes.c_float(1.5), None, ws,
+                                      1 << 30, fake, None) == gq.GPTQ_ERR_ARG
+    assert lib.gptq_first_order_shift(fake, 8, 16, fake, fake, 7, ctypes.c_float(0.5), None, ws,
+                                      1 << 30, fake, None) == gq.GPTQ_ERR_ARG
+    assert lib.gptq_first_order_shift(fake, 8, 16, fake, fake, 0, ctypes.c_float(0.5), None, ws,
+                                      64, fake, None) == gq.GPTQ_ERR_WORKSPACE
     # prepare: negative damping, missing status, small workspace
     assert lib.gptq_prepare(fake, 16, 1, ctypes.c_float(-0.1), None, ws, 1 << 30, fake,
                             None) == gq.GPTQ_ERR_ARG
@@ -122,3 +129,11 @@ def test_product_path_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(gq, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         gq.load_library()
+
+
+def test_trust_region_beta_matches_the_oracle(lib):
+    import oracle as O
+    for alpha, lq, gamma in ((0.1, 0.3, 2.0), (2.0, 1.0, 1.0), (0.0, 1.0, 5.0), (1.0, 1.0, 0.0),
+                             (0.7, 1e-3, 40.0)):
+        assert gq.gptq_trust_region_beta(alpha, lq, gamma) == pytest.approx(
+            O.trust_region_beta(alpha, lq, gamma), rel=1e-6, abs=1e-7)
