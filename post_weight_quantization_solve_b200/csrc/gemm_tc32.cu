@@ -78,6 +78,7 @@ __device__ __forceinline__ bool g32_unit(const Tc32Params &p, int u, G32Unit &w)
     if (p.a_upper) kb = (w.i0 / G32_BK) * G32_BK;
     if (p.b_upper) ke = min(ke, w.j0 + G32_BN);
     if (p.a_lower) ke = min(ke, w.i0 + G32_BM);
+    if (p.b_lower) kb = max(kb, (w.j0 / G32_BK) * G32_BK);
     const int steps = ke > kb ? (ke - kb) / G32_BK : 0;
     w.k0 = kb + (int)((int64_t)steps * part / I.parts) * G32_BK;
     w.k1 = kb + (int)((int64_t)steps * (part + 1) / I.parts) * G32_BK;

@@ -25,6 +25,7 @@ struct Tc32Params {
     int accumulate;         // C += alpha AB (else C = alpha AB; split items need C zeroed first)
     int upper_tiles, a_upper, b_upper, mask_strict_upper;
     int a_lower;            // A(i,k) == 0 for k > i: the k range ends at the row tile
+    int b_lower;            // B(k,j) == 0 for k < j: the k range starts at the column tile
     int nitems, units;
     int32_t *status;
     Tc32Item item[TC32_MAX_ITEMS];

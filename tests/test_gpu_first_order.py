@@ -1,6 +1,7 @@
 """First-order (gradient) term on the GPU vs the fp64 oracle (C ABI calls).
 
-The library applies the term as a shifted start W - beta G H^-1 (through U) and then
+The library applies the term as a shifted start W - beta G H^-1 (through U; tf32x3
+tensor-core products for K a multiple of 32 from 256, the fp32 SIMT GEMM otherwise) and then
 runs the ordinary sweep on the shifted fp32 weights; the oracle's explicit per-step
 form equals that reading by its CPU pins. Here: the shift and gamma against the fp64
 solve, then the sweep on the shifted weights by tie-follow replay. The reading itself
@@ -15,9 +16,13 @@ import oracle as O
 import post_weight_quantization_solve_b200 as gq
 from post_weight_quantization_solve_b200.build import build
 
-from gpu_util import CODE_SAME, TIE_BAND, TOL_U, dev, rel_max
+from gpu_util import CODE_SAME, TIE_BAND, TOL_P1, TOL_U, dev, rel_max
 
 pytestmark = pytest.mark.gpu
+
+# the two chained tf32x3 products against the same operands in fp64: the bound of P1,
+# which the residual computes by the same two-product route
+TOL_KERNEL = TOL_P1
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -47,7 +52,8 @@ def _setup(K, N, seed, gdtype):
 
 @pytest.mark.parametrize("K,N,gdtype,beta", [(392, 200, torch.float32, 0.6),
                                              (256, 96, torch.bfloat16, 1.0),
-                                             (136, 40, torch.float32, 0.0)])
+                                             (136, 40, torch.float32, 0.0),
+                                             (1024, 300, torch.bfloat16, 0.4)])
 def test_shift_and_gamma_match_oracle(K, N, gdtype, beta):
     H_in, U, W, G, st = _setup(K, N, K + N, gdtype)
     Ws = W.clone()
@@ -58,10 +64,16 @@ def test_shift_and_gamma_match_oracle(K, N, gdtype, beta):
     W_ora, gamma_ora = O.first_order_shift(Hd, _np(W), _np(G), beta)
     if beta == 0.0:
         assert torch.equal(Ws, W)
-    else:
-        # the step itself (not the weights it is added to) within U's tolerance
-        assert rel_max(_np(Ws) - _np(W), W_ora - _np(W)) <= TOL_U
-    assert gamma.item() == pytest.approx(gamma_ora, rel=TOL_U)
+        return
+    # the kernel: the step against the same factor in fp64, beta G (U^T U) and |G U^T|^2
+    U64, G64 = _np(U), _np(G)
+    T64 = G64 @ U64.T
+    assert rel_max(_np(Ws) - _np(W), -beta * T64 @ U64) <= TOL_KERNEL
+    assert gamma.item() == pytest.approx(float(np.sum(T64 * T64)), rel=TOL_KERNEL)
+    # end to end against the fp64 solve: the step applies U twice, so its bound is U's
+    # tolerance amplified by the conditioning of H (checked here with a 10x margin)
+    assert rel_max(_np(Ws) - _np(W), W_ora - _np(W)) <= 10 * TOL_U
+    assert gamma.item() == pytest.approx(gamma_ora, rel=10 * TOL_U)
 
 
 @pytest.mark.parametrize("K,N,sample", [(392, 200, None), (256, 9600, 64)])
