@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--cpu-sample-seconds", type=float, default=12.0)
     ap.add_argument("--shard", choices=["layers", "tokens"], default="layers",
                     help="N > 1: independent layers per rank, or one layer token-sharded")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch the step's kernels one by one instead of replaying CUDA graphs")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the stream length (small profiling cases only)")
     return ap.parse_args()
@@ -272,15 +274,18 @@ def run_ours(args, rank, world, local_rank):
     Cp = torch.empty(K, K, device=dev) if (wl.act_order and wl.gptaq) else None
     ws_r = (torch.empty(gq.gptq_workspace_size(gq.GPTQ_OP_RESIDUAL, K, 0, 1, 0), dtype=torch.uint8,
                         device=dev) if wl.gptaq else None)
-    stream = torch.cuda.current_stream(dev)
+    # the step runs on its own stream, so that its three phases can be captured as CUDA
+    # graphs (every kernel still runs at every replay; graphs only remove launch gaps)
+    stream = torch.cuda.Stream(dev)
+    use_graph = not args.no_graph and not tokens_sharded
     gram_ev = []
+    Hs = Hp if perm is not None else H
+    Cs = Cp if (perm is not None and C is not None) else C
 
-    def step(record=None):
+    def gram_part(record=None):
         H.zero_()
         if C is not None:
             C.zero_()
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-        ev[0].record(stream)
         for c in range(c1 - c0):
             if record is not None:
                 a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -295,17 +300,18 @@ def run_ours(args, rank, world, local_rank):
                                           status=status, stream=stream)
         if tokens_sharded:              # the solve's one exchange: sum the partial statistics
             sharded.allreduce_statistics(H, C)
-        ev[1].record(stream)
-        Hs, Cs = H, C
+
+    def prepare_part():
         if perm is not None:            # act-order: solve in the reordered coordinates
             gq.gptq_act_order(H, perm=perm, stream=stream)
-            Hs = gq.gptq_permute_hessian(H, perm, out=Hp, stream=stream)
+            gq.gptq_permute_hessian(H, perm, out=Hp, stream=stream)
             if C is not None:
-                Cs = gq.gptq_permute_hessian(C, perm, out=Cp, stream=stream)
+                gq.gptq_permute_hessian(C, perm, out=Cp, stream=stream)
         gq.gptq_prepare(Hs, wl.percdamp, workspace=ws_p, status=status, stream=stream)
         if P1 is not None:
             gq.gptaq_residual(P1, Cs, Hs, workspace=ws_r, stream=stream)
-        ev[2].record(stream)
+
+    def quantize_part():
         if Nl == 0:
             pass
         elif grouped:
@@ -330,13 +336,49 @@ def run_ours(args, rank, world, local_rank):
                                        wl.blocksize, P1=P1, scales_out=scales[a - n0:b - n0],
                                        codes=codes[a - n0:b - n0], workspace=ws_q,
                                        status=status, stream=stream, cae=wl.cae)
-        ev[3].record(stream)
+
+    parts = (gram_part, prepare_part, quantize_part)
+    graphs = None
+
+    def step(record=None):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        with torch.cuda.stream(stream):
+            ev[0].record(stream)
+            for i in range(3):
+                if graphs is not None:
+                    graphs[i].replay()
+                elif i == 0:
+                    gram_part(record)
+                else:
+                    parts[i]()
+                ev[i + 1].record(stream)
         return ev
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     gq.raise_on_status(status, "warmup")
+    graph_note = "off"
+    graph_launches = 0
+    if use_graph:
+        try:
+            l0 = gq.gptq_kernel_launches()
+            cap = []
+            for fn in parts:
+                gr = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gr, stream=stream):
+                    fn()
+                cap.append(gr)
+            graph_launches = gq.gptq_kernel_launches() - l0   # library kernels in one step
+            graphs = cap
+            step()                      # one replay before timing
+            torch.cuda.synchronize()
+            gq.raise_on_status(status, "graph replay")
+            graph_note = "on (Gram, prepare and quantize phases each replayed as a CUDA graph)"
+        except Exception as e:          # report it and time the eager launches instead
+            graphs = None
+            graph_note = f"capture failed, eager launches: {type(e).__name__}: {e}"[:200]
+            torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -351,18 +393,23 @@ def run_ours(args, rank, world, local_rank):
             evs.append(step(gram_ev))
         t1.record(stream)
         torch.cuda.synchronize()
-    launches = gq.gptq_kernel_launches() - launches0
+    # library kernels launched in the timed steps: counted at launch, or, for graph
+    # replays, the kernels captured into one step's graphs times the steps
+    launches = (gq.gptq_kernel_launches() - launches0) + (graph_launches * args.steps
+                                                          if graphs is not None else 0)
     if world > 1:
         dist.barrier()
     gq.raise_on_status(status, "timed steps")
     total_ms = t0.elapsed_time(t1)
-    parts = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])]
-                      for e in evs])
+    parts_ms = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]),
+                          e[2].elapsed_time(e[3])] for e in evs])
+    # per Gram launch: events around each launch when eager, the phase over its launches
+    # when replayed as a graph (inter-launch gaps included)
     gram_launch_ms = (float(np.mean([a.elapsed_time(b) for a, b in gram_ev])) if gram_ev
-                      else 0.0)
+                      else float(parts_ms[:, 0].mean()) / max(c1 - c0, 1))
 
-    stats = torch.tensor([total_ms, *parts.mean(0).tolist(), gram_launch_ms], dtype=torch.float64,
-                         device=dev)
+    stats = torch.tensor([total_ms, *parts_ms.mean(0).tolist(), gram_launch_ms],
+                         dtype=torch.float64, device=dev)
     sharded.max_over_ranks(stats)     # the slowest rank decides
     total_ms, gram_ms, prep_ms, quant_ms, gram_launch_ms = stats.tolist()
     ms_per_step = total_ms / args.steps
@@ -416,6 +463,7 @@ def run_ours(args, rank, world, local_rank):
                                + (" act-order" if wl.act_order else "")
                                + (f" first-order beta {wl.first_order}" if wl.first_order else ""),
                    "l2": f"inputs larger than L2 (X {Ml * K * 2 / 1e9:.1f} GB per rank)",
+                   "cuda_graphs": graph_note,
                    "parallelism": (f"{world} ranks on one layer: token-sharded Gram, NCCL "
                                    "all-reduce of H, channel-sliced quantisation"
                                    if tokens_sharded else f"{world} independent layers")},
