@@ -426,7 +426,9 @@ def run_ours(args, rank, world, local_rank):
     pack_bytes = Nl * K + words.numel() * 4
 
     e2e = None
-    if not args.no_e2e and g == 1 and not wl.gptaq and not tokens_sharded:
+    # through the public API with host buffers: the plain per-channel workloads
+    if (not args.no_e2e and g == 1 and not wl.gptaq and not tokens_sharded and not grouped
+            and not wl.cae and not wl.first_order):
         e2e = run_e2e(args, wl, X, W, dev, gq, torch, dist, world)
 
     if rank != 0:
@@ -510,12 +512,7 @@ def run_e2e(args, wl, X, W, dev, gq, torch, dist, world):
     Wd = torch.empty_like(W)
     H = torch.empty(K, K, device=dev)
     codes = torch.empty(N, K, dtype=torch.uint8, device=dev)
-    grouped = wl.groupsize > 0 or wl.act_order
-    scales = (torch.empty(N, (K + wl.groupsize - 1) // wl.groupsize, device=dev) if wl.groupsize
-              else torch.empty(N, device=dev))
-    g_idx = torch.empty(K, dtype=torch.int32, device=dev) if grouped else None
-    perm = torch.empty(K, dtype=torch.int32, device=dev) if wl.act_order else None
-    Hp = torch.empty(K, K, device=dev) if wl.act_order else None
+    scales = torch.empty(N, device=dev)
     status = gq.new_status(dev)
     ws_p = torch.empty(gq.gptq_workspace_size(gq.GPTQ_OP_PREPARE, K, 0, 1, 0), dtype=torch.uint8,
                        device=dev)
