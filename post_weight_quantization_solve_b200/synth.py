@@ -215,7 +215,9 @@ def weights(wl: Workload, device="cpu") -> torch.Tensor:
 
 def gradient(wl: Workload, device="cpu") -> torch.Tensor:
     """A synthetic gradient of the block objective w.r.t. W[N][K] for the first-order
-    term: N(0, (w_sigma / 10)^2), fp32 (the gradient comes from backprop, which the
-    solve does not run)."""
+    term, fp32 (the gradient comes from backprop, which the solve does not run). Like
+    H = 2 X^T X it grows with the token count: for unit-variance tokens H's diagonal is
+    about 2M, so g ~ N(0, (0.1 w_sigma 2M)^2) makes the Newton step H^-1 g about a tenth
+    of the weights' spread."""
     g = torch.randn(wl.N, wl.K, generator=generator(wl.seed, T_GRAD, 0, device), device=device)
-    return g * (wl.w_sigma / 10)
+    return g * (0.1 * wl.w_sigma * 2.0 * wl.M)
