@@ -87,7 +87,10 @@ typedef enum {
  * group's per-token weight w[g][m] scales token m's outer product.
  *
  *   H      device fp32 [g][K][K]; accumulated into (the caller zeroes it before the
- *          first chunk). Full symmetric storage is written.
+ *          first chunk). Full symmetric storage is written: each entry above the
+ *          diagonal and its mirror receive the same partial sums, in separate fp32
+ *          reductions, so the two triangles agree to fp32 rounding (gptq_prepare
+ *          reads the upper one).
  *   K      input coordinates, >= 1; bf16 streams need K % 8 == 0.
  *   g      number of Hessians (>= 1). With w == NULL, g must be 1.
  *   X      device [M][ldx] tokens, dtype xdtype. bf16: X and ldx 16-byte aligned
