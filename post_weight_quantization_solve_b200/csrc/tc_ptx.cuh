@@ -223,7 +223,7 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
 
 // 2-D tiled TMA load into this CTA's shared memory whose transaction bytes complete on
 // the pair's barrier `bar_cluster` (an address in the cluster window, normally the
-// even CTA's): the load half of a cta_group::2 operand stage. No multicast.
+// even CTA's): the load half of a cta_group::2 operand stage; one destination CTA.
 __device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *map,
                                                  uint32_t bar_cluster, int x, int y) {
     asm volatile(
