@@ -21,6 +21,7 @@
 #include <float.h>
 
 #include <algorithm>
+#include <cstdlib>
 #include <mutex>
 #include <vector>
 
@@ -201,6 +202,201 @@ __global__ void __launch_bounds__(DG_T, 1) k_chol_diag(float *H, int K, int j0, 
                     for (int c = 0; c < 4; ++c) {
                         s[r][c] = ffma2(l2, ak[c], s[r][c]);
                         v[r][c] = ffma2(l2, vk[c], v[r][c]);
+                    }
+                }
+            }
+        }
+    }
+    // U = D^-1/2 V on the tiles (zero below the diagonal)
+    if (ti < 32) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int i = i0 + r;
+            if (i >= nb) continue;
+            const float sc = 1.f / sqrtf(fmaxf(dpiv[i], FLT_MIN));
+            float o[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const float vc = (c & 1) ? v[r][c >> 1].y : v[r][c >> 1].x;
+                o[c] = (c0 + c >= i) ? vc * sc : 0.f;
+            }
+            float *dst = H + (int64_t)(j0 + i) * K + j0 + c0;
+            if (vec) {
+                *reinterpret_cast<float4 *>(dst) = make_float4(o[0], o[1], o[2], o[3]);
+                *reinterpret_cast<float4 *>(dst + 4) = make_float4(o[4], o[5], o[6], o[7]);
+            } else {
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    if (c0 + c < nb) dst[c] = o[c];
+            }
+        }
+    }
+}
+
+// The same factor with two pivots per block barrier: for the pair (ja, ja - 1) both
+// columns of S and both rows of V are published before pivot ja is applied, and every
+// thread forms column ja - 1, row ja - 1 and d_{ja - 1} after pivot ja itself, so the
+// 128 pivots of a block take 64 barriers.
+__global__ void __launch_bounds__(DG_T, 1) k_chol_diag2(float *H, int K, int j0, int nb,
+                                                    const float *diag_d, float tol,
+                                                    int32_t *status) {
+    if (failed(status)) return;
+    const int g = blockIdx.x;
+    H += (int64_t)g * K * K;
+    diag_d += (int64_t)g * K;
+    extern __shared__ __align__(16) float sm[];
+    float *colb = sm;                      // [128][128]: column j of S, rows < j
+    float *vrow = colb + DG_N * DG_N;      // [128][128]: row j of V
+    float *dpiv = vrow + DG_N * DG_N;      // [128]
+    float *rpiv = dpiv + DG_N;             // [128]
+    float *dref = rpiv + DG_N;             // [128]
+    const int tid = threadIdx.x;
+
+    // this thread's tile (ti, tk): rows 4 ti .. 4 ti + 3, columns 8 tk .. 8 tk + 7
+    int ti = 32, tk = 0;
+    if (tid < DG_TILES) {
+        int t = tid;
+        for (int r = 0; r < 32; ++r) {
+            const int cnt = 16 - (r >> 1);
+            if (t < cnt) { ti = r; tk = (r >> 1) + t; break; }
+            t -= cnt;
+        }
+    }
+    const int wrow0 = 4 * __shfl_sync(0xffffffffu, ti, 0);   // lowest row of this warp
+    const int i0 = 4 * ti, c0 = 8 * tk;
+
+    for (int idx = tid; idx < 2 * DG_N * DG_N / 4; idx += DG_T)
+        reinterpret_cast<float4 *>(colb)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (tid < DG_N) dref[tid] = tid < nb ? diag_d[j0 + tid] : 1.f;
+    // tiles entirely below the diagonal: zero in the output
+    for (int idx = tid; idx < DG_N * DG_N; idx += DG_T) {
+        const int r = idx >> 7, c = idx & 127;
+        if (r < nb && c < nb && (r >> 2) > 2 * (c >> 3) + 1) H[(int64_t)(j0 + r) * K + j0 + c] = 0.f;
+    }
+
+    // tile rows as column pairs (c, c + 1): the updates run as packed fp32 FMAs
+    float2 s[4][4], v[4][4];
+    const bool vec = (nb == DG_N) && (K % 4 == 0) && ((reinterpret_cast<uintptr_t>(H) & 15) == 0) &&
+                     (j0 % 4 == 0);
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const int i = i0 + r;
+        if (ti < 32 && vec) {
+            const float *src = H + (int64_t)(j0 + i) * K + j0 + c0;
+            const float4 x0 = *reinterpret_cast<const float4 *>(src);
+            const float4 x1 = *reinterpret_cast<const float4 *>(src + 4);
+            s[r][0] = make_float2(x0.x, x0.y); s[r][1] = make_float2(x0.z, x0.w);
+            s[r][2] = make_float2(x1.x, x1.y); s[r][3] = make_float2(x1.z, x1.w);
+        } else {
+            float e[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const int k = c0 + c;
+                e[c] = (i < nb && k < nb) ? H[(int64_t)(j0 + i) * K + j0 + k] : (i == k ? 1.f : 0.f);
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c) s[r][c] = make_float2(e[2 * c], e[2 * c + 1]);
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            v[r][c] = make_float2((i == c0 + 2 * c) ? 1.f : 0.f, (i == c0 + 2 * c + 1) ? 1.f : 0.f);
+    }
+    __syncthreads();
+
+    for (int jb = DG_N / 8 - 1; jb >= 0; --jb) {
+#pragma unroll
+        for (int jp = 3; jp >= 0; --jp) {
+            // pivots ja = 8 jb + 2 jp + 1 and jc = ja - 1 share a tile column pair, a
+            // four-row block and one barrier
+            const int ja = 8 * jb + 2 * jp + 1, jc = ja - 1;
+            if (tk == jb && i0 < ja) {
+                float4 o;
+                o.x = (i0 + 0 < ja) ? s[0][jp].y : 0.f;
+                o.y = (i0 + 1 < ja) ? s[1][jp].y : 0.f;
+                o.z = (i0 + 2 < ja) ? s[2][jp].y : 0.f;
+                o.w = (i0 + 3 < ja) ? s[3][jp].y : 0.f;
+                *reinterpret_cast<float4 *>(colb + ja * DG_N + i0) = o;
+                if (i0 < jc) {
+                    o.x = (i0 + 0 < jc) ? s[0][jp].x : 0.f;
+                    o.y = (i0 + 1 < jc) ? s[1][jp].x : 0.f;
+                    o.z = (i0 + 2 < jc) ? s[2][jp].x : 0.f;
+                    o.w = (i0 + 3 < jc) ? s[3][jp].x : 0.f;
+                    *reinterpret_cast<float4 *>(colb + jc * DG_N + i0) = o;
+                }
+            }
+            if (ti == (ja >> 2)) {
+                const int ra = ja & 3, rc = jc & 3;
+                *reinterpret_cast<float4 *>(vrow + ja * DG_N + c0) =
+                    make_float4(v[ra][0].x, v[ra][0].y, v[ra][1].x, v[ra][1].y);
+                *reinterpret_cast<float4 *>(vrow + ja * DG_N + c0 + 4) =
+                    make_float4(v[ra][2].x, v[ra][2].y, v[ra][3].x, v[ra][3].y);
+                *reinterpret_cast<float4 *>(vrow + jc * DG_N + c0) =
+                    make_float4(v[rc][0].x, v[rc][0].y, v[rc][1].x, v[rc][1].y);
+                *reinterpret_cast<float4 *>(vrow + jc * DG_N + c0 + 4) =
+                    make_float4(v[rc][2].x, v[rc][2].y, v[rc][3].x, v[rc][3].y);
+                if (tk == jb) {
+                    // d_ja, and d_jc after pivot ja (the same product as the tile update)
+                    const float da = s[ra][jp].y;
+                    const float rda = 1.f / fmaxf(da, FLT_MIN);
+                    const float sca = s[rc][jp].y;                 // S[jc][ja]
+                    const float dc = fmaf(-sca * rda, sca, s[rc][jp].x);
+                    dpiv[ja] = da;
+                    rpiv[ja] = rda;
+                    dpiv[jc] = dc;
+                    rpiv[jc] = 1.f / fmaxf(dc, FLT_MIN);
+                    if (ja < nb && !(da > tol * dref[ja])) set_status(status, GPTQ_ERR_NOT_PD);
+                    if (jc < nb && !(dc > tol * dref[jc])) set_status(status, GPTQ_ERR_NOT_PD);
+                }
+            }
+            __syncthreads();
+            if (wrow0 < ja) {
+                const float rda = rpiv[ja], rdc = rpiv[jc];
+                const float m = colb[ja * DG_N + jc] * rda;        // l of row jc on pivot ja
+                const float4 aa = *reinterpret_cast<const float4 *>(colb + ja * DG_N + i0 % DG_N);
+                const float4 ka0 = *reinterpret_cast<const float4 *>(colb + ja * DG_N + c0);
+                const float4 ka1 = *reinterpret_cast<const float4 *>(colb + ja * DG_N + c0 + 4);
+                const float4 va0 = *reinterpret_cast<const float4 *>(vrow + ja * DG_N + c0);
+                const float4 va1 = *reinterpret_cast<const float4 *>(vrow + ja * DG_N + c0 + 4);
+                const float4 ac = *reinterpret_cast<const float4 *>(colb + jc * DG_N + i0 % DG_N);
+                const float4 kc0 = *reinterpret_cast<const float4 *>(colb + jc * DG_N + c0);
+                const float4 kc1 = *reinterpret_cast<const float4 *>(colb + jc * DG_N + c0 + 4);
+                const float4 vc0 = *reinterpret_cast<const float4 *>(vrow + jc * DG_N + c0);
+                const float4 vc1 = *reinterpret_cast<const float4 *>(vrow + jc * DG_N + c0 + 4);
+                const float aav[4] = {aa.x, aa.y, aa.z, aa.w};
+                const float kav[8] = {ka0.x, ka0.y, ka0.z, ka0.w, ka1.x, ka1.y, ka1.z, ka1.w};
+                const float vav[8] = {va0.x, va0.y, va0.z, va0.w, va1.x, va1.y, va1.z, va1.w};
+                const float acv[4] = {ac.x, ac.y, ac.z, ac.w};
+                const float kcv[8] = {kc0.x, kc0.y, kc0.z, kc0.w, kc1.x, kc1.y, kc1.z, kc1.w};
+                const float vcv[8] = {vc0.x, vc0.y, vc0.z, vc0.w, vc1.x, vc1.y, vc1.z, vc1.w};
+                // column jc of S and row jc of V after pivot ja (entries at or past jc stay 0)
+                float la[4], lc[4];
+                float2 ka2[4], kc2[4], va2[4], vc2[4];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    la[r] = -aav[r] * rda;
+                    const float acn = (i0 + r < jc) ? fmaf(-aav[r], m, acv[r]) : 0.f;
+                    lc[r] = -acn * rdc;
+                }
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int k = c0 + 2 * c;
+                    ka2[c] = make_float2(kav[2 * c], kav[2 * c + 1]);
+                    va2[c] = make_float2(vav[2 * c], vav[2 * c + 1]);
+                    kc2[c] = make_float2((k < jc) ? fmaf(-kav[2 * c], m, kcv[2 * c]) : 0.f,
+                                         (k + 1 < jc) ? fmaf(-kav[2 * c + 1], m, kcv[2 * c + 1]) : 0.f);
+                    vc2[c] = make_float2(fmaf(-m, vav[2 * c], vcv[2 * c]),
+                                         fmaf(-m, vav[2 * c + 1], vcv[2 * c + 1]));
+                }
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const float2 l2a = make_float2(la[r], la[r]);
+                    const float2 l2c = make_float2(lc[r], lc[r]);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        s[r][c] = ffma2(l2a, ka2[c], s[r][c]);
+                        v[r][c] = ffma2(l2a, va2[c], v[r][c]);
+                        s[r][c] = ffma2(l2c, kc2[c], s[r][c]);
+                        v[r][c] = ffma2(l2c, vc2[c], v[r][c]);
                     }
                 }
             }
@@ -585,7 +781,11 @@ gptq_status prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out, v
 
     const float tol = (float)K * FLT_EPSILON;
     const int chol_smem = (int)((2 * DG_N * DG_N + 3 * DG_N) * sizeof(float));
-    cudaFuncSetAttribute(k_chol_diag, cudaFuncAttributeMaxDynamicSharedMemorySize, chol_smem);
+    // two pivots per barrier (GPTQ_DIAG_PAIRS=0 selects one pivot per barrier)
+    const char *pairs_env = getenv("GPTQ_DIAG_PAIRS");
+    const bool diag_pairs = !(pairs_env && pairs_env[0] == '0');
+    cudaFuncSetAttribute(diag_pairs ? k_chol_diag2 : k_chol_diag,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, chol_smem);
     Blocks bk{K, (K + CH_NB - 1) / CH_NB};
     // lookahead on the tensor-core steps (a second stream runs the bulk trailing
     // updates); without it every step runs in order on the caller's stream
@@ -614,7 +814,10 @@ gptq_status prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out, v
             for (int gi = 0; gi < g; ++gi)
                 if (cudaStreamWaitEvent(st, la->rest[gi][(t + 2) & 1], 0) != cudaSuccess)
                     return GPTQ_ERR_CUDA;
-        k_chol_diag<<<g, DG_T, chol_smem, st>>>(H, K, j0, nb, diag_d, tol, status);
+        if (diag_pairs)
+            k_chol_diag2<<<g, DG_T, chol_smem, st>>>(H, K, j0, nb, diag_d, tol, status);
+        else
+            k_chol_diag<<<g, DG_T, chol_smem, st>>>(H, K, j0, nb, diag_d, tol, status);
         if ((s = launch_status()) != GPTQ_OK) return s;
         if (j0 == 0) break;
         if (use_tc && j0 >= TC_STEP_MIN && nb % 32 == 0) {
