@@ -373,6 +373,16 @@ GPTQ_API gptq_status gptq_first_order_shift(float *W, int N, int K, const float 
  */
 GPTQ_API float gptq_trust_region_beta(float alpha, double loss_gptq, double gamma);
 
+/*
+ * gptq_selftest_timeout -- a diagnostic of the failure path every bounded device wait
+ * of the library shares: one kernel waits on a barrier that nothing arrives on; when
+ * the wait budget (about a second) runs out it sets GPTQ_ERR_TIMEOUT in *status and
+ * returns. Nothing faults or traps: the context stays usable afterwards.
+ *
+ *   status  device int32 (required).
+ */
+GPTQ_API gptq_status gptq_selftest_timeout(int32_t *status, void *stream);
+
 /* Workspace bytes for an operation (gptq_op); 0 when none is needed. */
 GPTQ_API size_t gptq_workspace_size(int op, int K, int N, int g, int blocksize);
 

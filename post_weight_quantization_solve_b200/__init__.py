@@ -27,7 +27,7 @@ EXPORTS = ("gptq_accumulate_hessian", "gptaq_accumulate_cross", "gptq_prepare",
            "gptq_prepare_noalloc",
            "gptaq_residual", "gptq_quantize_layer", "gptq_act_order", "gptq_permute_hessian",
            "gptq_quantize_layer_grouped", "gptq_pack_codes", "gptq_unpack_codes",
-           "gptq_first_order_shift", "gptq_trust_region_beta",
+           "gptq_first_order_shift", "gptq_trust_region_beta", "gptq_selftest_timeout",
            "gptq_workspace_size",
            "gptq_kernel_launches", "gptq_status_string")
 
@@ -65,6 +65,7 @@ def load_library():
         "gptq_unpack_codes": [P, I, I, I64, I, P, I64, P],
         "gptq_first_order_shift": [P, I, I, P, P, I, F, P, P, SZ, P, P],
         "gptq_trust_region_beta": [F, ctypes.c_double, ctypes.c_double],
+        "gptq_selftest_timeout": [P, P],
         "gptq_workspace_size": [I, I, I, I, I],
         "gptq_status_string": [I],
         "gptq_kernel_launches": [],
@@ -311,3 +312,13 @@ def gptq_trust_region_beta(alpha, loss_gptq, gamma):
     return float(load_library().gptq_trust_region_beta(ctypes.c_float(alpha),
                                                         ctypes.c_double(loss_gptq),
                                                         ctypes.c_double(gamma)))
+
+
+def gptq_selftest_timeout(status=None, stream=None):
+    """Run the library's bounded-wait failure path once (about a second): the returned
+    status word ends up holding GPTQ_ERR_TIMEOUT; see include/gptq.h."""
+    lib = load_library()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    status = new_status(dev) if status is None else status
+    _check(lib.gptq_selftest_timeout(_ptr(status), _stream(stream)), "gptq_selftest_timeout")
+    return status

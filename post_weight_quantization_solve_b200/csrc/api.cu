@@ -1,8 +1,11 @@
 // C ABI entry points: argument checks, workspace sizing, dispatch. Every check
 // here runs on the host before anything is enqueued.
+#include <nvtx3/nvToolsExt.h>
+
 #include <cmath>
 
 #include "common.cuh"
+#include "tc_ptx.cuh"
 
 namespace gptq {
 gptq_status gram_simt(float *H, int K, int g, const void *X, int xdtype, int64_t M, int64_t ldx,
@@ -55,6 +58,27 @@ using namespace gptq;
 
 static bool valid_dtype(int d) { return d == GPTQ_BF16 || d == GPTQ_F32; }
 
+// One NVTX range per entry point (a no-op unless a profiler collects NVTX).
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+};
+#define GPTQ_RANGE(name) NvtxRange gptq_nvtx_range_(name)
+
+// One bounded wait on a barrier that nothing arrives on: after the wait budget the
+// status word holds GPTQ_ERR_TIMEOUT and the kernel returns.
+__global__ void k_selftest_timeout(int32_t *status) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        tc::mbar_init(&bar, 1);
+        abort_flag = 0;
+        tc::fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !tc::mbar_wait(&bar, 0, &abort_flag)) set_status(status, GPTQ_ERR_TIMEOUT);
+}
+
 static bool stream_ok(int xdtype, const void *X, int64_t ldx, int K) {
     if (ldx < K) return false;
     if (xdtype == GPTQ_BF16) return aligned(X, 16) && ldx % 8 == 0;
@@ -66,6 +90,7 @@ extern "C" {
 gptq_status gptq_accumulate_hessian(float *H, int K, int g, const void *X, int xdtype, int64_t M,
                                     int64_t ldx, const float *w, int64_t ldw, int32_t *status,
                                     void *stream) {
+    GPTQ_RANGE("gptq_accumulate_hessian");
     if (K < 1 || K > GPTQ_MAX_DIM || g < 1 || g > 65535 || M < 0 || !H || !valid_dtype(xdtype))
         return GPTQ_ERR_ARG;
     if (M > 0x7fffffff) return GPTQ_ERR_ARG;
@@ -87,6 +112,7 @@ gptq_status gptq_accumulate_hessian(float *H, int K, int g, const void *X, int x
 
 gptq_status gptaq_accumulate_cross(float *C, int K, const void *X_fp, const void *X_q, int xdtype,
                                    int64_t M, int64_t ldx, int32_t *status, void *stream) {
+    GPTQ_RANGE("gptaq_accumulate_cross");
     if (K < 1 || K > GPTQ_MAX_DIM || M < 0 || !C || !valid_dtype(xdtype)) return GPTQ_ERR_ARG;
     if (M > 0x7fffffff) return GPTQ_ERR_ARG;
     if (M == 0) return GPTQ_OK;
@@ -104,6 +130,7 @@ gptq_status gptaq_accumulate_cross(float *C, int K, const void *X_fp, const void
 
 gptq_status gptq_prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out, void *ws,
                          size_t ws_bytes, int32_t *status, void *stream) {
+    GPTQ_RANGE("gptq_prepare");
     if (K < 1 || g < 1 || !H || !status || !(percdamp >= 0.f) || !aligned(H, 16))
         return GPTQ_ERR_ARG;
     if (K > GPTQ_MAX_DIM || g > 65535) return GPTQ_ERR_ARG;
@@ -115,6 +142,7 @@ gptq_status gptq_prepare(float *H, int K, int g, float percdamp, uint8_t *dead_o
 
 gptq_status gptaq_residual(float *P1, const float *C, const float *U, int K, void *ws,
                            size_t ws_bytes, void *stream) {
+    GPTQ_RANGE("gptaq_residual");
     if (K < 1 || K > GPTQ_MAX_DIM || !P1 || !C || !U) return GPTQ_ERR_ARG;
     if (!ws || !aligned(ws, 256) || ws_bytes < residual_workspace(K)) return GPTQ_ERR_WORKSPACE;
     return residual(P1, C, U, K, ws, static_cast<cudaStream_t>(stream));
@@ -125,6 +153,7 @@ gptq_status gptq_quantize_layer(void *W, int wdtype, int N, int K, const float *
                                 const uint8_t *dead, const float *scales_in, float *scales_out,
                                 uint8_t *codes, float *loss, int write_back, void *ws,
                                 size_t ws_bytes, int32_t *status, void *stream) {
+    GPTQ_RANGE("gptq_quantize_layer");
     if (N < 1 || K < 1 || groups < 1 || N % groups != 0 || !W || !U || !codes || !status)
         return GPTQ_ERR_ARG;
     if (N > GPTQ_MAX_DIM || K > GPTQ_MAX_DIM || groups > 8) return GPTQ_ERR_ARG;
@@ -144,12 +173,14 @@ gptq_status gptq_quantize_layer(void *W, int wdtype, int N, int K, const float *
 }
 
 gptq_status gptq_act_order(const float *H, int K, int32_t *perm, void *stream) {
+    GPTQ_RANGE("gptq_act_order");
     if (K < 1 || K > GPTQ_MAX_DIM || !H || !perm) return GPTQ_ERR_ARG;
     return act_order(H, K, perm, static_cast<cudaStream_t>(stream));
 }
 
 gptq_status gptq_permute_hessian(float *out, const float *H, int K, const int32_t *perm,
                                  void *stream) {
+    GPTQ_RANGE("gptq_permute_hessian");
     if (K < 1 || K > GPTQ_MAX_DIM || !out || !H || !perm || out == H) return GPTQ_ERR_ARG;
     return permute_square(out, H, K, perm, static_cast<cudaStream_t>(stream));
 }
@@ -161,6 +192,7 @@ gptq_status gptq_quantize_layer_grouped(void *W, int wdtype, int N, int K, const
                                         int32_t *g_idx_out, uint8_t *codes,
                                         float *loss, int write_back, void *ws, size_t ws_bytes,
                                         int32_t *status, void *stream) {
+    GPTQ_RANGE("gptq_quantize_layer_grouped");
     if (N < 1 || K < 1 || !W || !U || !codes || !status) return GPTQ_ERR_ARG;
     if (N > GPTQ_MAX_DIM || K > GPTQ_MAX_DIM || !valid_dtype(wdtype)) return GPTQ_ERR_ARG;
     if (bits != 2 && bits != 3 && bits != 4 && bits != 8) return GPTQ_ERR_ARG;
@@ -185,6 +217,7 @@ static bool pack_args_ok(int N, int K, int bits, int64_t ldc, int64_t ldw) {
 
 gptq_status gptq_pack_codes(const uint8_t *codes, int N, int K, int64_t ld_codes, int bits,
                             uint32_t *words, int64_t ld_words, void *stream) {
+    GPTQ_RANGE("gptq_pack_codes");
     if (!pack_args_ok(N, K, bits, ld_codes, ld_words)) return GPTQ_ERR_ARG;
     if (N > 0 && (!codes || !words)) return GPTQ_ERR_ARG;
     return pack_codes(codes, N, K, ld_codes, bits, words, ld_words,
@@ -193,6 +226,7 @@ gptq_status gptq_pack_codes(const uint8_t *codes, int N, int K, int64_t ld_codes
 
 gptq_status gptq_unpack_codes(const uint32_t *words, int N, int K, int64_t ld_words, int bits,
                               uint8_t *codes, int64_t ld_codes, void *stream) {
+    GPTQ_RANGE("gptq_unpack_codes");
     if (!pack_args_ok(N, K, bits, ld_codes, ld_words)) return GPTQ_ERR_ARG;
     if (N > 0 && (!codes || !words)) return GPTQ_ERR_ARG;
     return unpack_codes(words, N, K, ld_words, bits, codes, ld_codes,
@@ -202,6 +236,7 @@ gptq_status gptq_unpack_codes(const uint32_t *words, int N, int K, int64_t ld_wo
 gptq_status gptq_first_order_shift(float *W, int N, int K, const float *U, const void *G,
                                   int gdtype, float beta, double *gamma, void *ws,
                                   size_t ws_bytes, int32_t *status, void *stream) {
+    GPTQ_RANGE("gptq_first_order_shift");
     if (N < 1 || K < 1 || N > GPTQ_MAX_DIM || K > GPTQ_MAX_DIM) return GPTQ_ERR_ARG;
     if (!W || !U || !G || !status || !valid_dtype(gdtype)) return GPTQ_ERR_ARG;
     if (!(beta >= 0.f && beta <= 1.f)) return GPTQ_ERR_ARG;
@@ -217,6 +252,12 @@ float gptq_trust_region_beta(float alpha, double loss_gptq, double gamma) {
     if (!(x >= 0.0)) return 0.f;
     if (x >= 0.5) return 1.f;
     return (float)(1.0 - sqrt(1.0 - 2.0 * x));
+}
+
+gptq_status gptq_selftest_timeout(int32_t *status, void *stream) {
+    if (!status) return GPTQ_ERR_ARG;
+    k_selftest_timeout<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(status);
+    return launch_status();
 }
 
 size_t gptq_workspace_size(int op, int K, int N, int g, int blocksize) {

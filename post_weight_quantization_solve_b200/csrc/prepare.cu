@@ -428,7 +428,8 @@ __global__ void __launch_bounds__(DG_T, 1) k_chol_diag2(float *H, int K, int j0,
     }
 }
 
-__global__ void k_zero_lower(float *H, int K) {
+__global__ void k_zero_lower(float *H, int K, const int32_t *status) {
+    if (failed(status)) return;
     const int g = blockIdx.z;
     H += (int64_t)g * K * K;
     const int i = blockIdx.y;
@@ -668,6 +669,7 @@ __global__ void k_split_blocks(const float *__restrict__ H, int K, float *__rest
 }
 
 __global__ void k_zero_blocks(float *C, const Tc32Params p) {
+    if (failed(p.status)) return;
     const Tc32Item &I = p.item[blockIdx.z];
     const int r = blockIdx.y;
     if (r >= I.m) return;
@@ -870,7 +872,7 @@ gptq_status prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out, v
     if ((s = join_side()) != GPTQ_OK) return s;
     // The strict lower triangle still holds the input and update leftovers; the
     // inverse reads whole tiles of its triangular operands, so clear it first.
-    k_zero_lower<<<dim3((K + 255) / 256 > 8 ? 8 : (K + 255) / 256, K, g), 256, 0, st>>>(H, K);
+    k_zero_lower<<<dim3((K + 255) / 256 > 8 ? 8 : (K + 255) / 256, K, g), 256, 0, st>>>(H, K, status);
     if ((s = launch_status()) != GPTQ_OK) return s;
     if (use_tc) {
         for (int gi = 0; gi < g; ++gi)
