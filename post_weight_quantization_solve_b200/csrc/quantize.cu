@@ -31,11 +31,12 @@
 //   W0k       fp32 [N][K] starting weights w^(0) (CAE only)
 //   Uh, Ul    bf16 [g][K][ldU] U as hi + lo pairs;  Qh, Ql  the same for P1
 // The sweep keeps each channel's block coordinates in registers: one thread per
-// channel for layers with many output channels (k_sweep_thread), four lanes per
-// channel otherwise (k_sweep_lanes).
+// channel for layers with many output channels (k_sweep_thread; two lanes per channel
+// with CAE), four lanes per channel otherwise (k_sweep_lanes).
 #include <cuda.h>
 
 #include <algorithm>
+#include <cstdlib>
 
 #include "common.cuh"
 #include "update_tc.cuh"
@@ -171,26 +172,27 @@ __device__ __forceinline__ void cp_async_wait_all() {
 }
 
 // In-block sweep, lane-group form (for layers with few output channels): one block
-// [i0, i0 + bs) for 32 channels of one group.
-// A warp serves 8 channels with 4 lanes each: lane 4 c + q of the warp holds, of
-// channel c, the coordinates 32 b + 8 q + i (i < 8) of every 32-wide sub-block b, so
-// all 32 coordinates of the block stay in registers and every lane has work at every
-// step. At step j = 32 p + t the lane holding coordinate j (slot q = t / 8) rounds it
-// and computes E_j; a shuffle inside the channel's 4 lanes hands E_j to the others,
+// [i0, i0 + bs) for 128 / LPC channels of one group.
+// A warp serves 32 / LPC channels with LPC lanes each: lane LPC c + q of the warp holds,
+// of channel c, the coordinates 32 b + CPL q + i (i < CPL = 32 / LPC) of every 32-wide
+// sub-block b, so all of the block's coordinates stay in registers and every lane has
+// work at every step. At step j = 32 p + t the lane holding coordinate j (slot
+// q = t / CPL) rounds it and computes E_j; a shuffle inside the channel's lanes hands
+// E_j to the others,
 // and each lane applies it to its own coordinates (U's zero lower triangle makes the
 // coordinates at or before j no-ops, so no lane masks). The sub-block in work is
 // always w[0]: the register array shifts by one sub-block after each phase. No block
 // barrier inside the sweep. U[blk, blk] (and P1) is staged once per CTA as its ten
 // 32 x 32 blocks on or above the diagonal.
-template <bool GPTAQ, int GMODE, bool CAE>
-__global__ void __launch_bounds__(128, GPTAQ ? 2 : 4) k_sweep_lanes(
+template <bool GPTAQ, int GMODE, bool CAE, int LPC>
+__global__ void __launch_bounds__(128, (GPTAQ || LPC < 4) ? 2 : 4) k_sweep_lanes(
     float *__restrict__ Wk, int N, int per_group, int K, int i0, int bs,
     const float *__restrict__ U, const float *__restrict__ P1, const float *__restrict__ scale,
     int bits, uint8_t *__restrict__ codes, __nv_bfloat16 *__restrict__ Eh,
     __nv_bfloat16 *__restrict__ El, __nv_bfloat16 *__restrict__ Ph, __nv_bfloat16 *__restrict__ Pl,
     int ldE, int ldG, int erow0, float *__restrict__ loss_acc, int vec, const int32_t *status,
     const SweepGroups sg, const float *__restrict__ W0k) {
-    constexpr int NCH = 32, CLD = 132;
+    constexpr int CPL = 32 / LPC, NCH = 128 / LPC, CLD = 132;   // CPL: a lane's coordinates per sub-block
     if (failed(status)) return;
     extern __shared__ __align__(16) unsigned char smem[];
     float *Us = reinterpret_cast<float *>(smem);                 // [10][32][32]
@@ -205,8 +207,8 @@ __global__ void __launch_bounds__(128, GPTAQ ? 2 : 4) k_sweep_lanes(
     const int n0 = grp * per_group + cta_ch0;
     const int nvalid = min(NCH, per_group - cta_ch0);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int q = lane & 3;
-    const int ch = warp * 8 + (lane >> 2);
+    const int q = lane & (LPC - 1);
+    const int ch = warp * (32 / LPC) + lane / LPC;
     const bool valid = ch < nvalid;
     const int64_t n = (int64_t)n0 + ch;
     const int nsb = (bs + 31) / 32;
@@ -238,40 +240,30 @@ __global__ void __launch_bounds__(128, GPTAQ ? 2 : 4) k_sweep_lanes(
     }
     if (tid < bs) rpiv[tid] = 1.f / __ldg(Ub + (int64_t)tid * K + tid);
 
-    // this lane's coordinates 32 b + 8 q + i of its channel
-    float w[4][8];
+    // a lane's CPL coordinates 32 p + CPL q + i of sub-block p of its channel
+    auto fetch = [&](const float *base, int p, float (&d)[CPL]) {
+        const int c0 = 32 * p + CPL * q;
+        const float *src = base + n * K + i0 + c0;
+        if (valid && (vec & 1) && c0 + CPL <= bs) {
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-        const int c0 = 32 * b + 8 * q;
-        const float *src = Wk + n * K + i0 + c0;
-        if (valid && (vec & 1) && c0 + 8 <= bs) {
-            const float4 x0 = *reinterpret_cast<const float4 *>(src);
-            const float4 x1 = *reinterpret_cast<const float4 *>(src + 4);
-            w[b][0] = x0.x; w[b][1] = x0.y; w[b][2] = x0.z; w[b][3] = x0.w;
-            w[b][4] = x1.x; w[b][5] = x1.y; w[b][6] = x1.z; w[b][7] = x1.w;
+            for (int v = 0; v < CPL / 4; ++v) {
+                const float4 x = *reinterpret_cast<const float4 *>(src + 4 * v);
+                d[4 * v] = x.x; d[4 * v + 1] = x.y; d[4 * v + 2] = x.z; d[4 * v + 3] = x.w;
+            }
         } else {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) w[b][i] = (valid && c0 + i < bs) ? src[i] : 0.f;
-        }
-    }
-    // CAE: this lane's starting weights on the sub-block in work (w0c) and the next (w0n)
-    float w0c[8], w0n[8];
-    auto fetch_w0 = [&](int p, float (&d)[8]) {
-        const int c0 = 32 * p + 8 * q;
-        const float *src = W0k + n * K + i0 + c0;
-        if (valid && (vec & 1) && c0 + 8 <= bs) {
-            const float4 x0 = *reinterpret_cast<const float4 *>(src);
-            const float4 x1 = *reinterpret_cast<const float4 *>(src + 4);
-            d[0] = x0.x; d[1] = x0.y; d[2] = x0.z; d[3] = x0.w;
-            d[4] = x1.x; d[5] = x1.y; d[6] = x1.z; d[7] = x1.w;
-        } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) d[i] = (valid && c0 + i < bs) ? src[i] : 0.f;
+            for (int i = 0; i < CPL; ++i) d[i] = (valid && c0 + i < bs) ? src[i] : 0.f;
         }
     };
+    float w[4][CPL];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) fetch(Wk, b, w[b]);
+    // CAE: this lane's starting weights on the sub-block in work (w0c) and the next (w0n)
+    float w0c[CPL], w0n[CPL];
+    auto fetch_w0 = [&](int p, float (&d)[CPL]) { fetch(W0k, p, d); };
     if (CAE) fetch_w0(0, w0c);
     if (GMODE == 2) {
-        for (int j = q; j < bs; j += 4) {
+        for (int j = q; j < bs; j += LPC) {
             const float sj = valid ? sg.gsc[n * sg.ldg + sg.gsel[i0 + j]] : 1.f;
             sS[j * NCH + ch] = sj;
             sR[j * NCH + ch] = 1.f / sj;
@@ -284,7 +276,7 @@ __global__ void __launch_bounds__(128, GPTAQ ? 2 : 4) k_sweep_lanes(
     float rs = 1.f / s;
     const float zf = (float)(1 << (bits - 1));
     const float cmin = -zf, cmax = (float)((1 << bits) - 1) - zf;
-    const int gsrc = lane & ~3;
+    const int gsrc = lane & ~(LPC - 1);
     float lacc = 0.f;
     uint8_t *crow = Cs + ch * CLD;
     const int64_t ecol = (int64_t)grp * ldG + cta_ch0 + ch;
@@ -301,9 +293,9 @@ __global__ void __launch_bounds__(128, GPTAQ ? 2 : 4) k_sweep_lanes(
             for (int b = 0; b < 4; ++b)
                 if (32 * b < sg.G)
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(w[b][i]));
-            a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
-            a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+                    for (int i = 0; i < CPL; ++i) a = fmaxf(a, fabsf(w[b][i]));
+#pragma unroll
+            for (int x = 1; x < LPC; x <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, x));
             s = a == 0.f ? 1.f : 2.f * a / (cmax - cmin);
             rs = 1.f / s;
             if (valid && q == 0) sg.gsc[n * sg.ldg + (i0 + 32 * p) / sg.G] = s;
@@ -311,7 +303,7 @@ __global__ void __launch_bounds__(128, GPTAQ ? 2 : 4) k_sweep_lanes(
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
             const int j = 32 * p + t;
-            const int oq = t >> 3, oi = t & 7;
+            const int oq = t / CPL, oi = t % CPL;
             const bool live = j < bs;
             const float sj = GMODE == 2 ? sS[j * NCH + ch] : s;
             const float rsj = GMODE == 2 ? sR[j * NCH + ch] : rs;
@@ -343,21 +335,25 @@ __global__ void __launch_bounds__(128, GPTAQ ? 2 : 4) k_sweep_lanes(
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
                 if (b > 0 && p + b >= nsb) break;
-                const float *ur = Us + (bbase + b) * 1024 + t * 32 + 8 * q;
-                const float4 u0 = *reinterpret_cast<const float4 *>(ur);
-                const float4 u1 = *reinterpret_cast<const float4 *>(ur + 4);
-                w[b][0] = fmaf(-e, u0.x, w[b][0]); w[b][1] = fmaf(-e, u0.y, w[b][1]);
-                w[b][2] = fmaf(-e, u0.z, w[b][2]); w[b][3] = fmaf(-e, u0.w, w[b][3]);
-                w[b][4] = fmaf(-e, u1.x, w[b][4]); w[b][5] = fmaf(-e, u1.y, w[b][5]);
-                w[b][6] = fmaf(-e, u1.z, w[b][6]); w[b][7] = fmaf(-e, u1.w, w[b][7]);
+                const float *ur = Us + (bbase + b) * 1024 + t * 32 + CPL * q;
+#pragma unroll
+                for (int c = 0; c < CPL / 4; ++c) {
+                    const float4 u = *reinterpret_cast<const float4 *>(ur + 4 * c);
+                    w[b][4 * c] = fmaf(-e, u.x, w[b][4 * c]);
+                    w[b][4 * c + 1] = fmaf(-e, u.y, w[b][4 * c + 1]);
+                    w[b][4 * c + 2] = fmaf(-e, u.z, w[b][4 * c + 2]);
+                    w[b][4 * c + 3] = fmaf(-e, u.w, w[b][4 * c + 3]);
+                }
                 if (GPTAQ) {
-                    const float *pr = Ps + (bbase + b) * 1024 + t * 32 + 8 * q;
-                    const float4 p0 = *reinterpret_cast<const float4 *>(pr);
-                    const float4 p1 = *reinterpret_cast<const float4 *>(pr + 4);
-                    w[b][0] = fmaf(v, p0.x, w[b][0]); w[b][1] = fmaf(v, p0.y, w[b][1]);
-                    w[b][2] = fmaf(v, p0.z, w[b][2]); w[b][3] = fmaf(v, p0.w, w[b][3]);
-                    w[b][4] = fmaf(v, p1.x, w[b][4]); w[b][5] = fmaf(v, p1.y, w[b][5]);
-                    w[b][6] = fmaf(v, p1.z, w[b][6]); w[b][7] = fmaf(v, p1.w, w[b][7]);
+                    const float *pr = Ps + (bbase + b) * 1024 + t * 32 + CPL * q;
+#pragma unroll
+                    for (int c = 0; c < CPL / 4; ++c) {
+                        const float4 u = *reinterpret_cast<const float4 *>(pr + 4 * c);
+                        w[b][4 * c] = fmaf(v, u.x, w[b][4 * c]);
+                        w[b][4 * c + 1] = fmaf(v, u.y, w[b][4 * c + 1]);
+                        w[b][4 * c + 2] = fmaf(v, u.z, w[b][4 * c + 2]);
+                        w[b][4 * c + 3] = fmaf(v, u.w, w[b][4 * c + 3]);
+                    }
                 }
             }
         }
@@ -365,13 +361,13 @@ __global__ void __launch_bounds__(128, GPTAQ ? 2 : 4) k_sweep_lanes(
 #pragma unroll
         for (int b = 0; b < 3; ++b)
 #pragma unroll
-            for (int i = 0; i < 8; ++i) w[b][i] = w[b + 1][i];
+            for (int i = 0; i < CPL; ++i) w[b][i] = w[b + 1][i];
         if (CAE)
 #pragma unroll
-            for (int i = 0; i < 8; ++i) w0c[i] = w0n[i];
+            for (int i = 0; i < CPL; ++i) w0c[i] = w0n[i];
     }
-    lacc += __shfl_xor_sync(0xffffffffu, lacc, 1);
-    lacc += __shfl_xor_sync(0xffffffffu, lacc, 2);
+#pragma unroll
+    for (int x = 1; x < LPC; x <<= 1) lacc += __shfl_xor_sync(0xffffffffu, lacc, x);
     if (q == 0 && valid) loss_acc[n] += lacc;
     __syncthreads();
     // codes: 16-byte chunks of each channel's block row
@@ -749,9 +745,10 @@ static size_t sweep_thread_smem(bool gptaq, int gmode, bool cae) {
     return sizeof(float) * ((10 * 1024 + 32 * SW_T) * (gptaq ? 2 : 1) + SW_MAXB +
                             (gmode == 2 ? 2 * SW_MAXB * SW_T : 0) + (cae ? 32 * SW_T : 0));
 }
-static size_t sweep_lanes_smem(bool gptaq, int gmode) {
-    return sizeof(float) * (10 * 1024 * (gptaq ? 2 : 1) + 32 * 33 + SW_MAXB +
-                            (gmode == 2 ? 2 * SW_MAXB * 32 : 0));
+static size_t sweep_lanes_smem(bool gptaq, int gmode, int lpc) {
+    const int nch = 128 / lpc;
+    return sizeof(float) * (10 * 1024 * (gptaq ? 2 : 1) + SW_MAXB + (gmode == 2 ? 2 * SW_MAXB * nch : 0)) +
+           (size_t)nch * 132;
 }
 
 typedef void (*SweepKernel)(float *, int, int, int, int, int, const float *, const float *,
@@ -759,16 +756,25 @@ typedef void (*SweepKernel)(float *, int, int, int, int, int, const float *, con
                             __nv_bfloat16 *, __nv_bfloat16 *, int, int, int, float *, int,
                             const int32_t *, const SweepGroups, const float *);
 
+// form 0: one thread per channel; 1: four lanes per channel; 2: two lanes per channel
 #define GPTQ_SWEEP_MODES(K, A, C) {K<A, 0, C>, K<A, 1, C>, K<A, 2, C>}
-static SweepKernel sweep_kernel(bool per_thread, bool gptaq, int gmode, bool cae) {
-    static const SweepKernel tab[2][2][2][3] = {
-        {{GPTQ_SWEEP_MODES(k_sweep_lanes, false, false), GPTQ_SWEEP_MODES(k_sweep_lanes, false, true)},
-         {GPTQ_SWEEP_MODES(k_sweep_lanes, true, false), GPTQ_SWEEP_MODES(k_sweep_lanes, true, true)}},
+#define GPTQ_LANES4(A, C, G) k_sweep_lanes<A, G, C, 4>
+#define GPTQ_LANES2(A, C, G) k_sweep_lanes<A, G, C, 2>
+#define GPTQ_LANE_MODES(L, A, C) {L(A, C, 0), L(A, C, 1), L(A, C, 2)}
+static SweepKernel sweep_kernel(int form, bool gptaq, int gmode, bool cae) {
+    static const SweepKernel tab[3][2][2][3] = {
         {{GPTQ_SWEEP_MODES(k_sweep_thread, false, false), GPTQ_SWEEP_MODES(k_sweep_thread, false, true)},
-         {GPTQ_SWEEP_MODES(k_sweep_thread, true, false), GPTQ_SWEEP_MODES(k_sweep_thread, true, true)}}};
-    return tab[per_thread][gptaq][cae][gmode];
+         {GPTQ_SWEEP_MODES(k_sweep_thread, true, false), GPTQ_SWEEP_MODES(k_sweep_thread, true, true)}},
+        {{GPTQ_LANE_MODES(GPTQ_LANES4, false, false), GPTQ_LANE_MODES(GPTQ_LANES4, false, true)},
+         {GPTQ_LANE_MODES(GPTQ_LANES4, true, false), GPTQ_LANE_MODES(GPTQ_LANES4, true, true)}},
+        {{GPTQ_LANE_MODES(GPTQ_LANES2, false, false), GPTQ_LANE_MODES(GPTQ_LANES2, false, true)},
+         {GPTQ_LANE_MODES(GPTQ_LANES2, true, false), GPTQ_LANE_MODES(GPTQ_LANES2, true, true)}}};
+    return tab[form][gptaq][cae][gmode];
 }
 #undef GPTQ_SWEEP_MODES
+#undef GPTQ_LANES4
+#undef GPTQ_LANES2
+#undef GPTQ_LANE_MODES
 
 // Input-dimension groups and order of one quantisation (G == 0: per-channel scales,
 // natural order).
@@ -899,14 +905,19 @@ static gptq_status quantize_impl(void *W, int wdtype, int N, int K, const float 
     base.neg[0] = 1;
     base.neg[1] = 0;
 
-    // one thread per channel when that still gives every SM two warps; otherwise four
-    // lanes per channel
-    const bool per_thread = (int64_t)N >= 2LL * 148 * 32;
-    const int cta = per_thread ? SW_T : 128;
-    const dim3 grid((per_group + (per_thread ? SW_T : 32) - 1) / (per_thread ? SW_T : 32), groups);
-    SweepKernel kern = sweep_kernel(per_thread, gptaq, gmode, cae != 0);
-    const size_t smem = per_thread ? sweep_thread_smem(gptaq, gmode, cae != 0)
-                                   : sweep_lanes_smem(gptaq, gmode);
+    // one thread per channel when that still gives every SM two warps, two lanes per
+    // channel there instead for CAE (its starting weights then stay in registers: 2.25
+    // against 2.51 ms for a 14336 x 4096 layer on B200, while the plain and GPTAQ sweeps
+    // time the same or slower with two lanes); four lanes per channel for fewer channels.
+    // GPTQ_SWEEP_FORM = 0, 1 or 2 picks the form (comparisons and tests).
+    int form = (int64_t)N >= 2LL * 148 * 32 ? (cae ? 2 : 0) : 1;
+    if (const char *f = getenv("GPTQ_SWEEP_FORM")) form = atoi(f) == 2 ? 2 : atoi(f) == 1 ? 1 : 0;
+    const int cta = form == 0 ? SW_T : 128;
+    const int per_cta = form == 0 ? SW_T : form == 1 ? 32 : 64;
+    const dim3 grid((per_group + per_cta - 1) / per_cta, groups);
+    SweepKernel kern = sweep_kernel(form, gptaq, gmode, cae != 0);
+    const size_t smem = form == 0 ? sweep_thread_smem(gptaq, gmode, cae != 0)
+                                  : sweep_lanes_smem(gptaq, gmode, form == 1 ? 4 : 2);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
         return launch_status();

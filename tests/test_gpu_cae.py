@@ -127,9 +127,13 @@ def test_cae_small_blocks_fp32_dead():
     _check(200, 72, 4, 32, seed=5, gptaq=True, wdtype=torch.float32, dead_cols=(3, 150))
 
 
+@pytest.mark.parametrize("form", [None, "0"])
 @pytest.mark.parametrize("gptaq,K", [(False, 256), (True, 640)])
-def test_cae_thread_sweep(gptaq, K):
-    # many channels: one thread per channel (checked on a sample of channels)
+def test_cae_many_channels(gptaq, K, form, monkeypatch):
+    # many channels: two lanes per channel by default, or one thread per channel
+    # (checked on a sample of channels)
+    if form is not None:
+        monkeypatch.setenv("GPTQ_SWEEP_FORM", form)
     _check(K, 9600, 2, 128, seed=31 + gptaq, gptaq=gptaq, sample=96)
 
 

@@ -118,6 +118,22 @@ def test_ragged_bf16(K, N, M, B, bits):
     _full_check(wl, chunks, synth.weights(wl), label=f"ragged {K}x{N}")
 
 
+@pytest.mark.parametrize("form", ["0", "1", "2"])
+def test_every_sweep_form(form, monkeypatch):
+    # one thread, four lanes or two lanes per channel: each form on its own, on ragged
+    # blocks, plain and GPTAQ
+    monkeypatch.setenv("GPTQ_SWEEP_FORM", form)
+    wl = synth.WORKLOADS["mlp_up"].scaled(K=392, N=200, M=2000, blocksize=128, bits=3,
+                                         chunk=1024)
+    chunks = [synth.tokens_chunk(wl, c) for c in range(synth.num_chunks(wl))]
+    _full_check(wl, chunks, synth.weights(wl), label=f"form {form}")
+    wl = synth.WORKLOADS["gptaq"].scaled(K=256, N=136, M=2048, chunk=1024)
+    n = synth.num_chunks(wl)
+    xq = [synth.tokens_chunk(wl, c) for c in range(n)]
+    xf = [synth.fp_tokens_chunk(wl, c) for c in range(n)]
+    _full_check(wl, xq, synth.weights(wl), gptaq_fp=xf, label=f"gptaq form {form}")
+
+
 def test_rotated_qproj_small():
     wl = synth.WORKLOADS["q_proj"].scaled(K=256, N=256, M=4096)
     _full_check(wl, [synth.tokens_chunk(wl, 0)], synth.weights(wl), label="q_proj")
