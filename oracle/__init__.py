@@ -19,6 +19,7 @@ from .gptq_oracle import (  # noqa: F401
     gram,
     cross_gram,
     dead_and_damp,
+    damped_diagonal,
     is_positive_definite,
     symmetric_scale,
     quantize_codes,

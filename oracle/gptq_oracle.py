@@ -81,13 +81,19 @@ def dead_and_damp(H, percdamp):
     the value chosen does not change the solve.)
     """
     H = np.array(H, dtype=np.float64, copy=True)
-    K = H.shape[0]
-    dead = np.diag(H) == 0.0
-    idx = np.arange(K)
-    H[idx[dead], idx[dead]] = 1.0
-    damp = percdamp * np.mean(np.diag(H))
-    H[idx, idx] += damp
+    d, dead = damped_diagonal(np.diag(H), percdamp)
+    H[np.diag_indices(H.shape[0])] = d
     return H, dead
+
+
+def damped_diagonal(diag, percdamp):
+    """The diagonal of H_d from the diagonal of H alone (dead_and_damp touches nothing
+    else): dead entries set to 1, then percdamp times the mean of the result added to
+    every entry. Returns (diagonal, dead mask)."""
+    d = np.array(diag, dtype=np.float64, copy=True)
+    dead = d == 0.0
+    d[dead] = 1.0
+    return d + percdamp * np.mean(d), dead
 
 
 def is_positive_definite(H):

@@ -199,6 +199,37 @@ def test_U_diagonal_is_free_set_pivot(K):
         assert U[j, j] ** 2 == pytest.approx(P_F[0, 0], rel=1e-10)
 
 
+@pytest.mark.parametrize("K,t", [(9, 4), (16, 1), (16, 15)])
+def test_U_trailing_block_is_factor_of_trailing_block(K, t):
+    # H_d = V V^T with V = U^-1 upper, so the trailing principal block of H_d only sees
+    # the trailing block of V: U[T, T] is the factor of H_d[T, T] alone (the property
+    # the full-size GPU tests sample), and U H_d U^T = I on every row pair
+    _, _, Hd, _ = _random_problem(K, 1, 40 + K + t)
+    U = O.upper_factor(Hd)
+    T = slice(K - t, K)
+    np.testing.assert_allclose(U[T, T], O.upper_factor(Hd[T, T]), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(U @ Hd @ U.T, np.eye(K), atol=1e-10)
+    # a transposed factor fails the identity, and the other upper factor of H_d^-1
+    # (R^-1 with R^T R = H_d, so R^-1 R^-T = H_d^-1) fails the trailing-block property
+    assert not np.allclose(U.T @ Hd @ U, np.eye(K), atol=1e-6)
+    Rinv = np.linalg.inv(np.linalg.cholesky(Hd).T)
+    np.testing.assert_allclose(Rinv @ Rinv.T, np.linalg.inv(Hd), atol=1e-10)
+    assert not np.allclose(Rinv[T, T], O.upper_factor(Hd[T, T]), atol=1e-6)
+
+
+def test_damped_diagonal_is_dead_and_damp_diagonal():
+    _, _, Hd, _ = _random_problem(12, 1, 77)
+    H = Hd.copy()
+    H[3, :] = 0.0
+    H[:, 3] = 0.0
+    full, dead = O.dead_and_damp(H, 0.05)
+    d, dead_d = O.damped_diagonal(np.diag(H), 0.05)
+    np.testing.assert_array_equal(dead, dead_d)
+    np.testing.assert_array_equal(np.diag(full), d)
+    # dead entry: 1 plus the damping of a mean that includes that 1
+    assert d[3] == pytest.approx(1.0 + 0.05 * (np.trace(H) + 1.0) / 12, rel=1e-14)
+
+
 def test_objective_identities():
     X, H, Hd, W = _random_problem(10, 5, 7, M=200)
     s, _ = O.symmetric_scale(W, 2)
