@@ -199,6 +199,16 @@ def time_sum(*a):
     return round(sum(a), 2)
 
 
+def workload_desc(wl, num_chunks):
+    """The workload string of the JSON line's config (both arms)."""
+    return (f"{wl.name}: K={wl.K} N={wl.N} tokens={wl.M} (chunks {num_chunks}x{wl.chunk}) "
+            f"W{wl.bits} blocksize {wl.blocksize} percdamp {wl.percdamp} groups {wl.groups}"
+            + (" gptaq" if wl.gptaq else "") + (" cae" if wl.cae else "")
+            + (f" groupsize {wl.groupsize}" if wl.groupsize else "")
+            + (" act-order" if wl.act_order else "")
+            + (f" first-order beta {wl.first_order}" if wl.first_order else ""))
+
+
 # ----------------------------------------------------------------------------- ours
 
 def run_ours(args, rank, world, local_rank):
@@ -458,12 +468,7 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "strong" if tokens_sharded else "weak",
         "vs_baseline": None, "dtype": "bf16->f32",
         "data": f"synthetic ({wl.stream} bf16 tokens, N(0,{wl.w_sigma}^2) bf16 weights)",
-        "config": {"workload": f"{wl.name}: K={K} N={N} tokens={M} (chunks {nch}x{ch}) W{wl.bits} "
-                               f"blocksize {wl.blocksize} percdamp {wl.percdamp} groups {g}"
-                               + (" gptaq" if wl.gptaq else "") + (" cae" if wl.cae else "")
-                               + (f" groupsize {wl.groupsize}" if wl.groupsize else "")
-                               + (" act-order" if wl.act_order else "")
-                               + (f" first-order beta {wl.first_order}" if wl.first_order else ""),
+        "config": {"workload": workload_desc(wl, nch),
                    "l2": f"inputs larger than L2 (X {Ml * K * 2 / 1e9:.1f} GB per rank)",
                    "cuda_graphs": graph_note,
                    "parallelism": (f"{world} ranks on one layer: token-sharded Gram, NCCL "
@@ -596,8 +601,9 @@ def run_reference(args, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (same recipe, CPU generator)",
-        "config": {"workload": f"{wl.name}: K={wl.K} N={wl.N} tokens={wl.M} W{wl.bits} "
-                               f"blocksize {wl.blocksize} percdamp {wl.percdamp}"},
+        "config": {"workload": workload_desc(wl, synth.num_chunks(wl)),
+                   "parallelism": "rank 0 only: the fp64 CPU oracle on a bounded sample, scaled "
+                                  "to the whole job"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cb["cores"], "kind": "oracle",
                          "sample": cb["sample"]},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
