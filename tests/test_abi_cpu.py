@@ -137,3 +137,49 @@ def test_trust_region_beta_matches_the_oracle(lib):
                              (0.7, 1e-3, 40.0)):
         assert gq.gptq_trust_region_beta(alpha, lq, gamma) == pytest.approx(
             O.trust_region_beta(alpha, lq, gamma), rel=1e-6, abs=1e-7)
+
+
+C_CONSUMER = r"""
+#include <stdio.h>
+#include <string.h>
+#include "gptq.h"
+
+int main(void) {
+    void *fake = (void *)(size_t)(1u << 20);
+    int32_t *status = (int32_t *)fake;
+    size_t ws = gptq_workspace_size(GPTQ_OP_QUANTIZE, 4096, 14336, 1, 128);
+    size_t wsc = gptq_workspace_size(GPTQ_OP_QUANTIZE | GPTQ_WS_CAE, 4096, 14336, 1, 128);
+    gptq_status bad_bits = gptq_quantize_layer(fake, GPTQ_BF16, 8, 16, (const float *)fake, 1, 5,
+                                               128, NULL, 0, NULL, NULL, NULL, (uint8_t *)fake,
+                                               NULL, 0, fake, (size_t)1 << 30, status, NULL);
+    gptq_status empty = gptq_pack_codes((const uint8_t *)fake, 0, 64, 64, 3, (uint32_t *)fake,
+                                        6, NULL);
+    float beta = gptq_trust_region_beta(2.0f, 1.0f, 1.0f);
+    printf("%zu %zu %d %d %.6f %s\n", ws, wsc, (int)bad_bits, (int)empty, beta,
+           gptq_status_string(GPTQ_ERR_NOT_PD));
+    return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_the_library_links(lib, tmp_path):
+    # a C99 consumer: the header compiles as C with warnings as errors, the program links
+    # against the in-tree library and makes host-only calls through the ABI
+    src = tmp_path / "consumer.c"
+    src.write_text(C_CONSUMER)
+    exe = tmp_path / "consumer"
+    libdir = os.path.dirname(gq.LIB_PATH)
+    import subprocess
+    cc = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                         "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                         "-L", libdir, "-l:" + os.path.basename(gq.LIB_PATH),
+                         "-Wl,-rpath," + libdir], capture_output=True, text=True)
+    assert cc.returncode == 0, cc.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0, run.stderr
+    ws, wsc, bad_bits, empty, beta, *msg = run.stdout.split()
+    assert int(ws) == gq.gptq_workspace_size(gq.GPTQ_OP_QUANTIZE, 4096, 14336, 1, 128)
+    assert int(wsc) >= int(ws) + 4096 * 14336 * 4
+    assert int(bad_bits) == gq.GPTQ_ERR_ARG and int(empty) == gq.GPTQ_OK
+    assert float(beta) == pytest.approx(gq.gptq_trust_region_beta(2.0, 1.0, 1.0), rel=1e-6)
+    assert " ".join(msg) == gq.gptq_status_string(gq.GPTQ_ERR_NOT_PD)
