@@ -181,7 +181,7 @@ def oracle_sample(wl, budget_s):
     t_schur = max(t_a - 8 * c_ch, 1e-9)
     t_sweep = t_schur * S_all / S_pre + c_ch * N * L_all / L_pre
     total = t_gram + t_prep + t_sweep
-    cores = torch.get_num_threads()
+    cores = oracle_threads(torch)
     return {
         "seconds_per_step": total,
         "value": K * N / total,
@@ -197,6 +197,43 @@ def oracle_sample(wl, budget_s):
 
 def time_sum(*a):
     return round(sum(a), 2)
+
+
+def oracle_threads(torch):
+    """Threads the oracle's arithmetic runs on: numpy's BLAS pool (its matmuls and
+    inverses), else torch's intra-op pool."""
+    try:
+        import numpy  # noqa: F401  (loads the BLAS the oracle uses)
+        import threadpoolctl
+        pools = [i["num_threads"] for i in threadpoolctl.threadpool_info()
+                 if i.get("user_api") == "blas"]
+        if pools:
+            return max(pools)
+    except Exception:
+        pass
+    return torch.get_num_threads()
+
+
+def host_cpu():
+    """Model name of the host CPU and its logical core count."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "nproc": os.cpu_count()}
+
+
+def cpu_baseline_entry(cb, value):
+    """The JSON line's cpu_baseline object for one oracle sample."""
+    return {"value": value, "unit": UNIT, "cores": cb["cores"], "kind": "oracle",
+            "sample": cb["sample"], **host_cpu(),
+            "stage_seconds": {k: round(v, 3) for k, v in cb["parts_s"].items()},
+            "measured_seconds": cb["measured_s"]}
 
 
 def workload_desc(wl, num_chunks):
@@ -498,8 +535,7 @@ def run_ours(args, rank, world, local_rank):
         line["e2e"] = e2e
     if world == 1 and not args.no_cpu_baseline:
         cb = oracle_sample(wl, args.cpu_sample_seconds)
-        line["cpu_baseline"] = {"value": cb["value"], "unit": UNIT, "cores": cb["cores"],
-                                "kind": "oracle", "sample": cb["sample"]}
+        line["cpu_baseline"] = cpu_baseline_entry(cb, cb["value"])
     return line
 
 
@@ -604,8 +640,7 @@ def run_reference(args, rank, world):
         "config": {"workload": workload_desc(wl, synth.num_chunks(wl)),
                    "parallelism": "rank 0 only: the fp64 CPU oracle on a bounded sample, scaled "
                                   "to the whole job"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cb["cores"], "kind": "oracle",
-                         "sample": cb["sample"]},
+        "cpu_baseline": cpu_baseline_entry(cb, value),
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 

@@ -42,6 +42,10 @@ def test_reference_arm_line():
     assert line["cpu_baseline"]["kind"] == "oracle"
     assert line["cpu_baseline"]["value"] == line["value"]
     assert line["cpu_baseline"]["cores"] >= 1 and line["cpu_baseline"]["sample"]
+    assert line["cpu_baseline"]["nproc"] >= 1
+    assert set(line["cpu_baseline"]["stage_seconds"]) == {"gram", "prepare", "sweep"}
+    assert sum(line["cpu_baseline"]["stage_seconds"].values()) == pytest.approx(
+        line["ms_per_step"] / 1e3, rel=0.05, abs=2e-3)
     assert line["e2e"] == {"value": line["value"], "unit": line["unit"],
                            "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     from post_weight_quantization_solve_b200 import synth
