@@ -82,13 +82,44 @@ def load_library():
     return lib
 
 
-def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+def _device(t, name):
+    """The CUDA device of the call's main tensor (every other tensor must be on it)."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor"
+                         + (f" (got {t.device})" if isinstance(t, torch.Tensor) else ""))
+    return t.device
 
 
-def _stream(stream):
+def _ptr(t, dev=None, name="tensor", rows=False):
+    """Device pointer of `t` for the C ABI, after the layout checks the ABI relies on:
+    a CUDA tensor on the call's device, dense (or, with rows=True, rows that may be
+    padded but whose elements are contiguous). A host pointer would reach the kernels
+    otherwise."""
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor"
+                         + (f" (got {t.device})" if isinstance(t, torch.Tensor) else ""))
+    if dev is not None and t.device != dev:
+        raise ValueError(f"{name} is on {t.device}, the call runs on {dev}")
+    _check_layout(t, name, rows)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _check_layout(t, name, rows=False):
+    """Dense, or (rows=True) contiguous within each row with any row pitch."""
+    if rows:
+        if t.dim() >= 1 and t.numel() > 1 and t.shape[-1] > 1 and t.stride(-1) != 1:
+            raise ValueError(f"{name}: the elements of a row must be contiguous")
+    elif not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _stream(stream, dev=None):
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(dev)
+    elif dev is not None and stream.device != dev:
+        raise ValueError(f"the stream is on {stream.device}, the call runs on {dev}")
     return ctypes.c_void_p(stream.cuda_stream)
 
 
@@ -138,12 +169,16 @@ def gptq_workspace_size(op, K, N=0, g=1, blocksize=0):
 def gptq_accumulate_hessian(H, X, w=None, status=None, stream=None):
     """H[g] += 2 X^T diag(w[g]) X (see include/gptq.h). H: (K,K) or (g,K,K) fp32."""
     lib = load_library()
+    dev = _device(H, "H")
     K = H.shape[-1]
     g = 1 if H.dim() == 2 else H.shape[0]
     M = X.shape[0]
     ldw = 0 if w is None else w.stride(0) if w.dim() == 2 else w.shape[-1]
-    code = lib.gptq_accumulate_hessian(_ptr(H), K, g, _ptr(X), _dtype_code(X), M, X.stride(0),
-                                       _ptr(w), ldw, _ptr(status), _stream(stream))
+    args = (_ptr(H, dev, "H"), K, g, _ptr(X, dev, "X", rows=True), _dtype_code(X), M,
+            X.stride(0), _ptr(w, dev, "w", rows=True), ldw, _ptr(status, dev, "status"),
+            _stream(stream, dev))
+    with torch.cuda.device(dev):
+        code = lib.gptq_accumulate_hessian(*args)
     _check(code, "gptq_accumulate_hessian")
 
 
@@ -152,21 +187,28 @@ def gptaq_accumulate_cross(C, X_fp, X_q, status=None, stream=None):
     lib = load_library()
     if X_fp.stride(0) != X_q.stride(0) or X_fp.dtype != X_q.dtype or X_fp.shape != X_q.shape:
         raise ValueError("X_fp and X_q must share shape, dtype and row stride")
-    code = lib.gptaq_accumulate_cross(_ptr(C), C.shape[-1], _ptr(X_fp), _ptr(X_q),
-                                      _dtype_code(X_q), X_q.shape[0], X_q.stride(0),
-                                      _ptr(status), _stream(stream))
+    dev = _device(C, "C")
+    args = (_ptr(C, dev, "C"), C.shape[-1], _ptr(X_fp, dev, "X_fp", rows=True),
+            _ptr(X_q, dev, "X_q", rows=True), _dtype_code(X_q), X_q.shape[0], X_q.stride(0),
+            _ptr(status, dev, "status"), _stream(stream, dev))
+    with torch.cuda.device(dev):
+        code = lib.gptaq_accumulate_cross(*args)
     _check(code, "gptaq_accumulate_cross")
 
 
 def gptq_prepare(H, percdamp=0.01, dead_out=None, workspace=None, status=None, stream=None):
     """In place: dead fix, damping, H -> U. Returns the status tensor (not synchronised)."""
     lib = load_library()
+    dev = _device(H, "H")
     K = H.shape[-1]
     g = 1 if H.dim() == 2 else H.shape[0]
-    status = new_status(H.device) if status is None else status
-    ws = _workspace(gptq_workspace_size(GPTQ_OP_PREPARE, K, 0, g, 0), H.device, workspace)
-    code = lib.gptq_prepare(_ptr(H), K, g, float(percdamp), _ptr(dead_out), _ptr(ws),
-                            ws.numel() * ws.element_size(), _ptr(status), _stream(stream))
+    status = new_status(dev) if status is None else status
+    ws = _workspace(gptq_workspace_size(GPTQ_OP_PREPARE, K, 0, g, 0), dev, workspace)
+    args = (_ptr(H, dev, "H"), K, g, float(percdamp), _ptr(dead_out, dev, "dead_out"),
+            _ptr(ws, dev, "workspace"), ws.numel() * ws.element_size(),
+            _ptr(status, dev, "status"), _stream(stream, dev))
+    with torch.cuda.device(dev):
+        code = lib.gptq_prepare(*args)
     _check(code, "gptq_prepare")
     return status
 
@@ -175,12 +217,15 @@ def gptq_prepare_noalloc(H, percdamp=0.01, dead_out=None, status=None, stream=No
     """gptq_prepare with the library's fixed device scratch instead of a workspace
     (no allocation anywhere on this path). Returns the status tensor."""
     lib = load_library()
+    dev = _device(H, "H")
     K = H.shape[-1]
     g = 1 if H.dim() == 2 else H.shape[0]
     if status is None:
         raise ValueError("gptq_prepare_noalloc needs a caller-provided status word")
-    code = lib.gptq_prepare_noalloc(_ptr(H), K, g, float(percdamp), _ptr(dead_out),
-                                    _ptr(status), _stream(stream))
+    args = (_ptr(H, dev, "H"), K, g, float(percdamp), _ptr(dead_out, dev, "dead_out"),
+            _ptr(status, dev, "status"), _stream(stream, dev))
+    with torch.cuda.device(dev):
+        code = lib.gptq_prepare_noalloc(*args)
     _check(code, "gptq_prepare_noalloc")
     return status
 
@@ -188,10 +233,13 @@ def gptq_prepare_noalloc(H, percdamp=0.01, dead_out=None, status=None, stream=No
 def gptaq_residual(P1, C, U, workspace=None, stream=None):
     """P1 = [(C U^T) ⊙ strict-upper] U (see include/gptq.h)."""
     lib = load_library()
+    dev = _device(U, "U")
     K = U.shape[-1]
-    ws = _workspace(gptq_workspace_size(GPTQ_OP_RESIDUAL, K, 0, 1, 0), U.device, workspace)
-    code = lib.gptaq_residual(_ptr(P1), _ptr(C), _ptr(U), K, _ptr(ws),
-                              ws.numel() * ws.element_size(), _stream(stream))
+    ws = _workspace(gptq_workspace_size(GPTQ_OP_RESIDUAL, K, 0, 1, 0), dev, workspace)
+    args = (_ptr(P1, dev, "P1"), _ptr(C, dev, "C"), _ptr(U, dev, "U"), K,
+            _ptr(ws, dev, "workspace"), ws.numel() * ws.element_size(), _stream(stream, dev))
+    with torch.cuda.device(dev):
+        code = lib.gptaq_residual(*args)
     _check(code, "gptaq_residual")
 
 
@@ -201,17 +249,21 @@ def gptq_quantize_layer(W, U, bits, blocksize=128, groups=1, P1=None, dead=None,
     """The shared-order sweep (cae: with the compensation-aware error term).
     Returns (codes, status); see include/gptq.h."""
     lib = load_library()
+    dev = _device(W, "W")
     N, K = W.shape
     if codes is None:
-        codes = torch.empty(N, K, dtype=torch.uint8, device=W.device)
-    status = new_status(W.device) if status is None else status
+        codes = torch.empty(N, K, dtype=torch.uint8, device=dev)
+    status = new_status(dev) if status is None else status
     op = GPTQ_OP_QUANTIZE | (GPTQ_WS_CAE if cae else 0)
-    ws = _workspace(gptq_workspace_size(op, K, N, groups, blocksize), W.device, workspace)
-    code = lib.gptq_quantize_layer(_ptr(W), _dtype_code(W), N, K, _ptr(U), groups, bits,
-                                   blocksize, _ptr(P1), int(bool(cae)), _ptr(dead), _ptr(scales_in),
-                                   _ptr(scales_out), _ptr(codes), _ptr(loss), int(write_back),
-                                   _ptr(ws), ws.numel() * ws.element_size(), _ptr(status),
-                                   _stream(stream))
+    ws = _workspace(gptq_workspace_size(op, K, N, groups, blocksize), dev, workspace)
+    args = (_ptr(W, dev, "W"), _dtype_code(W), N, K, _ptr(U, dev, "U"), groups, bits, blocksize,
+            _ptr(P1, dev, "P1"), int(bool(cae)), _ptr(dead, dev, "dead"),
+            _ptr(scales_in, dev, "scales_in"), _ptr(scales_out, dev, "scales_out"),
+            _ptr(codes, dev, "codes"), _ptr(loss, dev, "loss"), int(write_back),
+            _ptr(ws, dev, "workspace"), ws.numel() * ws.element_size(),
+            _ptr(status, dev, "status"), _stream(stream, dev))
+    with torch.cuda.device(dev):
+        code = lib.gptq_quantize_layer(*args)
     _check(code, "gptq_quantize_layer")
     return codes, status
 
@@ -219,21 +271,29 @@ def gptq_quantize_layer(W, U, bits, blocksize=128, groups=1, P1=None, dead=None,
 def gptq_act_order(H, perm=None, stream=None):
     """The act-order processing order of H's input coordinates (int32 [K])."""
     lib = load_library()
+    dev = _device(H, "H")
     K = H.shape[-1]
     if perm is None:
-        perm = torch.empty(K, dtype=torch.int32, device=H.device)
-    _check(lib.gptq_act_order(_ptr(H), K, _ptr(perm), _stream(stream)), "gptq_act_order")
+        perm = torch.empty(K, dtype=torch.int32, device=dev)
+    args = (_ptr(H, dev, "H"), K, _ptr(perm, dev, "perm"), _stream(stream, dev))
+    with torch.cuda.device(dev):
+        code = lib.gptq_act_order(*args)
+    _check(code, "gptq_act_order")
     return perm
 
 
 def gptq_permute_hessian(H, perm, out=None, stream=None):
     """out = H[perm][:, perm] (a new K x K tensor unless `out` is given)."""
     lib = load_library()
+    dev = _device(H, "H")
     K = H.shape[-1]
     if out is None:
-        out = torch.empty_like(H)
-    _check(lib.gptq_permute_hessian(_ptr(out), _ptr(H), K, _ptr(perm), _stream(stream)),
-           "gptq_permute_hessian")
+        out = torch.empty_like(H, memory_format=torch.contiguous_format)
+    args = (_ptr(out, dev, "out"), _ptr(H, dev, "H"), K, _ptr(perm, dev, "perm"),
+            _stream(stream, dev))
+    with torch.cuda.device(dev):
+        code = lib.gptq_permute_hessian(*args)
+    _check(code, "gptq_permute_hessian")
     return out
 
 
@@ -244,24 +304,26 @@ def gptq_quantize_layer_grouped(W, U, bits, blocksize=128, groupsize=128, static
     """The sweep with input-dimension groups and an optional processing order.
     Returns (codes, scales [N][ceil(K / groupsize)], g_idx [K], status); see include/gptq.h."""
     lib = load_library()
+    dev = _device(W, "W")
     N, K = W.shape
     if codes is None:
-        codes = torch.empty(N, K, dtype=torch.uint8, device=W.device)
+        codes = torch.empty(N, K, dtype=torch.uint8, device=dev)
     if scales_out is None:
         shape = (N, (K + groupsize - 1) // groupsize) if groupsize else (N,)
-        scales_out = torch.empty(shape, dtype=torch.float32, device=W.device)
+        scales_out = torch.empty(shape, dtype=torch.float32, device=dev)
     if g_idx is None:
-        g_idx = torch.empty(K, dtype=torch.int32, device=W.device)
-    status = new_status(W.device) if status is None else status
+        g_idx = torch.empty(K, dtype=torch.int32, device=dev)
+    status = new_status(dev) if status is None else status
     op = GPTQ_OP_QUANTIZE_GROUPED | (GPTQ_WS_CAE if cae else 0)
-    ws = _workspace(gptq_workspace_size(op, K, N, 1, blocksize), W.device, workspace)
-    code = lib.gptq_quantize_layer_grouped(_ptr(W), _dtype_code(W), N, K, _ptr(U), bits, blocksize,
-                                           groupsize, int(bool(static_groups)), _ptr(perm),
-                                           _ptr(P1), int(bool(cae)), _ptr(dead), _ptr(scales_out),
-                                           _ptr(g_idx),
-                                           _ptr(codes), _ptr(loss), int(write_back), _ptr(ws),
-                                           ws.numel() * ws.element_size(), _ptr(status),
-                                           _stream(stream))
+    ws = _workspace(gptq_workspace_size(op, K, N, 1, blocksize), dev, workspace)
+    args = (_ptr(W, dev, "W"), _dtype_code(W), N, K, _ptr(U, dev, "U"), bits, blocksize,
+            groupsize, int(bool(static_groups)), _ptr(perm, dev, "perm"), _ptr(P1, dev, "P1"),
+            int(bool(cae)), _ptr(dead, dev, "dead"), _ptr(scales_out, dev, "scales_out"),
+            _ptr(g_idx, dev, "g_idx"), _ptr(codes, dev, "codes"), _ptr(loss, dev, "loss"),
+            int(write_back), _ptr(ws, dev, "workspace"), ws.numel() * ws.element_size(),
+            _ptr(status, dev, "status"), _stream(stream, dev))
+    with torch.cuda.device(dev):
+        code = lib.gptq_quantize_layer_grouped(*args)
     _check(code, "gptq_quantize_layer_grouped")
     return codes, scales_out, g_idx, status
 
@@ -270,23 +332,31 @@ def gptq_pack_codes(codes, bits, words=None, stream=None):
     """codes uint8 [N][K] -> words int32 [N][ceil(K bits / 32)] holding the uint32 bit
     patterns of include/gptq.h's layout (view them with .view(torch.uint32))."""
     lib = load_library()
+    dev = _device(codes, "codes")
     N, K = codes.shape
     nw = (K * bits + 31) // 32
     if words is None:
-        words = torch.empty(N, nw, dtype=torch.int32, device=codes.device)
-    _check(lib.gptq_pack_codes(_ptr(codes), N, K, codes.stride(0), bits, _ptr(words),
-                               words.stride(0), _stream(stream)), "gptq_pack_codes")
+        words = torch.empty(N, nw, dtype=torch.int32, device=dev)
+    args = (_ptr(codes, dev, "codes", rows=True), N, K, codes.stride(0), bits,
+            _ptr(words, dev, "words", rows=True), words.stride(0), _stream(stream, dev))
+    with torch.cuda.device(dev):
+        code = lib.gptq_pack_codes(*args)
+    _check(code, "gptq_pack_codes")
     return words
 
 
 def gptq_unpack_codes(words, bits, K, codes=None, stream=None):
     """The inverse of gptq_pack_codes: words [N][>= ceil(K bits / 32)] -> uint8 [N][K]."""
     lib = load_library()
+    dev = _device(words, "words")
     N = words.shape[0]
     if codes is None:
-        codes = torch.empty(N, K, dtype=torch.uint8, device=words.device)
-    _check(lib.gptq_unpack_codes(_ptr(words), N, K, words.stride(0), bits, _ptr(codes),
-                                 codes.stride(0), _stream(stream)), "gptq_unpack_codes")
+        codes = torch.empty(N, K, dtype=torch.uint8, device=dev)
+    args = (_ptr(words, dev, "words", rows=True), N, K, words.stride(0), bits,
+            _ptr(codes, dev, "codes", rows=True), codes.stride(0), _stream(stream, dev))
+    with torch.cuda.device(dev):
+        code = lib.gptq_unpack_codes(*args)
+    _check(code, "gptq_unpack_codes")
     return codes
 
 
@@ -294,15 +364,17 @@ def gptq_first_order_shift(W, U, G, beta, gamma=None, workspace=None, status=Non
     """W (fp32 [N][K]) <- W - beta G H^-1 in place; gamma (float64 [1]) gets
     sum_n g_n H^-1 g_n^T when given. Returns status; see include/gptq.h."""
     lib = load_library()
+    dev = _device(W, "W")
     if W.dtype != torch.float32:
         raise TypeError("gptq_first_order_shift shifts an fp32 copy of the weights")
     N, K = W.shape
-    status = new_status(W.device) if status is None else status
-    ws = _workspace(gptq_workspace_size(GPTQ_OP_FIRST_ORDER, K, N, 1, 0), W.device, workspace)
-    code = lib.gptq_first_order_shift(_ptr(W), N, K, _ptr(U), _ptr(G), _dtype_code(G),
-                                      ctypes.c_float(beta), _ptr(gamma), _ptr(ws),
-                                      ws.numel() * ws.element_size(), _ptr(status),
-                                      _stream(stream))
+    status = new_status(dev) if status is None else status
+    ws = _workspace(gptq_workspace_size(GPTQ_OP_FIRST_ORDER, K, N, 1, 0), dev, workspace)
+    args = (_ptr(W, dev, "W"), N, K, _ptr(U, dev, "U"), _ptr(G, dev, "G"), _dtype_code(G),
+            ctypes.c_float(beta), _ptr(gamma, dev, "gamma"), _ptr(ws, dev, "workspace"),
+            ws.numel() * ws.element_size(), _ptr(status, dev, "status"), _stream(stream, dev))
+    with torch.cuda.device(dev):
+        code = lib.gptq_first_order_shift(*args)
     _check(code, "gptq_first_order_shift")
     return status
 
@@ -318,7 +390,10 @@ def gptq_selftest_timeout(status=None, stream=None):
     """Run the library's bounded-wait failure path once (about a second): the returned
     status word ends up holding GPTQ_ERR_TIMEOUT; see include/gptq.h."""
     lib = load_library()
-    dev = torch.device("cuda", torch.cuda.current_device())
+    dev = status.device if status is not None else torch.device("cuda", torch.cuda.current_device())
     status = new_status(dev) if status is None else status
-    _check(lib.gptq_selftest_timeout(_ptr(status), _stream(stream)), "gptq_selftest_timeout")
+    args = (_ptr(status, dev, "status"), _stream(stream, dev))
+    with torch.cuda.device(dev):
+        code = lib.gptq_selftest_timeout(*args)
+    _check(code, "gptq_selftest_timeout")
     return status

@@ -7,6 +7,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import post_weight_quantization_solve_b200 as gq
 from post_weight_quantization_solve_b200.build import build
@@ -183,3 +184,43 @@ def test_header_is_plain_c_and_the_library_links(lib, tmp_path):
     assert int(bad_bits) == gq.GPTQ_ERR_ARG and int(empty) == gq.GPTQ_OK
     assert float(beta) == pytest.approx(gq.gptq_trust_region_beta(2.0, 1.0, 1.0), rel=1e-6)
     assert " ".join(msg) == gq.gptq_status_string(gq.GPTQ_ERR_NOT_PD)
+
+
+def test_binding_refuses_host_tensors(lib):
+    # a host pointer must never reach a kernel: every call checks its tensors first
+    W = torch.zeros(8, 16)
+    H = torch.eye(16)
+    X = torch.zeros(32, 16, dtype=torch.bfloat16)
+    codes = torch.zeros(8, 16, dtype=torch.uint8)
+    calls = [
+        lambda: gq.gptq_accumulate_hessian(H, X),
+        lambda: gq.gptaq_accumulate_cross(H, X, X),
+        lambda: gq.gptq_prepare(H),
+        lambda: gq.gptq_prepare_noalloc(H, status=torch.zeros(1, dtype=torch.int32)),
+        lambda: gq.gptaq_residual(H, H, H),
+        lambda: gq.gptq_quantize_layer(W, H, 4, 16),
+        lambda: gq.gptq_act_order(H),
+        lambda: gq.gptq_permute_hessian(H, torch.arange(16, dtype=torch.int32)),
+        lambda: gq.gptq_quantize_layer_grouped(W, H, 4, 16, 16),
+        lambda: gq.gptq_pack_codes(codes, 4),
+        lambda: gq.gptq_unpack_codes(torch.zeros(8, 2, dtype=torch.int32), 4, 16),
+        lambda: gq.gptq_first_order_shift(W, H, W, 0.5),
+    ]
+    for call in calls:
+        with pytest.raises(ValueError, match="must be a CUDA tensor"):
+            call()
+
+
+def test_binding_layout_rules():
+    A = torch.zeros(6, 8)
+    gq._check_layout(A, "A")
+    gq._check_layout(A[1:4], "A")                      # a block of whole rows is dense
+    with pytest.raises(ValueError, match="contiguous"):
+        gq._check_layout(A[:, 1:5], "A")               # padded rows: not dense
+    gq._check_layout(A[:, 1:5], "A", rows=True)        # but fine where a pitch is passed
+    with pytest.raises(ValueError, match="row must be contiguous"):
+        gq._check_layout(A.t(), "A", rows=True)        # a transposed view is refused
+    with pytest.raises(ValueError, match="contiguous"):
+        gq._check_layout(A.t(), "A")
+    gq._check_layout(torch.zeros(0, 8).t(), "A", rows=True)
+    gq._check_layout(torch.zeros(5, 1)[::2], "A", rows=True)
