@@ -224,3 +224,67 @@ def test_binding_layout_rules():
         gq._check_layout(A.t(), "A")
     gq._check_layout(torch.zeros(0, 8).t(), "A", rows=True)
     gq._check_layout(torch.zeros(5, 1)[::2], "A", rows=True)
+
+
+def test_every_wrapper_matches_its_c_signature(lib, monkeypatch):
+    # each wrapper's argument list against the ctypes signature of its entry point: the
+    # count, and every value convertible to its declared type (a fake library records the
+    # calls; the device checks are bypassed so that host tensors stand in for device ones)
+    import contextlib
+
+    calls = {}
+
+    class FakeLib:
+        def __getattr__(self, name):
+            real = getattr(lib, name)
+
+            def fn(*args):
+                assert len(args) == len(real.argtypes), (name, len(args), len(real.argtypes))
+                for a, t in zip(args, real.argtypes):
+                    t.from_param(a)
+                calls[name] = args
+                return 0
+            return fn
+
+    monkeypatch.setattr(gq, "_lib", FakeLib())
+    monkeypatch.setattr(gq, "_device", lambda t, name: t.device)
+    monkeypatch.setattr(gq, "_stream", lambda stream, dev=None: ctypes.c_void_p(0))
+
+    def host_ptr(t, dev=None, name="tensor", rows=False):
+        if t is None:
+            return None
+        gq._check_layout(t, name, rows)
+        return ctypes.c_void_p(t.data_ptr())
+    monkeypatch.setattr(gq, "_ptr", host_ptr)
+    monkeypatch.setattr(torch.cuda, "device", lambda d: contextlib.nullcontext())
+    real_ws = lib.gptq_workspace_size
+    monkeypatch.setattr(gq, "gptq_workspace_size", lambda *a: int(real_ws(*a)))
+
+    K, N = 32, 8
+    H = torch.eye(K)
+    W = torch.zeros(N, K)
+    X = torch.zeros(64, K, dtype=torch.bfloat16)
+    st = torch.zeros(1, dtype=torch.int32)
+    gq.gptq_accumulate_hessian(H, X, status=st)
+    gq.gptq_accumulate_hessian(torch.zeros(2, K, K), X, torch.ones(2, 64), status=st)
+    gq.gptaq_accumulate_cross(H, X, X, status=st)
+    gq.gptq_prepare(H, 0.01, dead_out=torch.zeros(K, dtype=torch.uint8), status=st)
+    gq.gptq_prepare_noalloc(H, 0.01, status=st)
+    gq.gptaq_residual(torch.zeros(K, K), H, H)
+    gq.gptq_quantize_layer(W, H, 3, 16, P1=H, dead=torch.zeros(K, dtype=torch.uint8),
+                           scales_out=torch.zeros(N), loss=torch.zeros(N), write_back=True,
+                           status=st, cae=True)
+    perm = gq.gptq_act_order(H)
+    gq.gptq_permute_hessian(H, perm)
+    gq.gptq_quantize_layer_grouped(W, H, 3, 16, 16, static_groups=True, perm=perm, P1=H,
+                                   status=st, cae=True)
+    words = gq.gptq_pack_codes(torch.zeros(N, K, dtype=torch.uint8), 3)
+    gq.gptq_unpack_codes(words, 3, K)
+    gq.gptq_first_order_shift(W, H, W, 0.5, gamma=torch.zeros(1, dtype=torch.float64),
+                              status=st)
+    gq.gptq_selftest_timeout(status=st)
+    assert set(calls) == set(gq.EXPORTS) - {"gptq_trust_region_beta", "gptq_workspace_size",
+                                            "gptq_kernel_launches", "gptq_status_string"}
+    # the workspace sizes passed are the ones the library asks for
+    assert calls["gptq_quantize_layer"][17] >= int(real_ws(gq.GPTQ_OP_QUANTIZE | gq.GPTQ_WS_CAE,
+                                                           K, N, 1, 16))
