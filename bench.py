@@ -412,18 +412,17 @@ def run_ours(args, rank, world, local_rank):
             l0 = gq.gptq_kernel_launches()
             cap = []
             for fn in parts:
-                gr = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(gr, stream=stream):
+                cap.append(torch.cuda.CUDAGraph())
+                with torch.cuda.graph(cap[-1], stream=stream):
                     fn()
-                cap.append(gr)
             graph_launches = gq.gptq_kernel_launches() - l0   # library kernels in one step
-            graphs = cap
+            graphs, cap = cap, None
             step()                      # one replay before timing
             torch.cuda.synchronize()
             gq.raise_on_status(status, "graph replay")
             graph_note = "on (Gram, prepare and quantize phases each replayed as a CUDA graph)"
         except Exception as e:          # report it and time the eager launches instead
-            graphs = None
+            graphs = cap = None
             graph_note = f"capture failed, eager launches: {type(e).__name__}: {e}"[:200]
             torch.cuda.synchronize()
     if world > 1:
@@ -444,6 +443,9 @@ def run_ours(args, rank, world, local_rank):
     # replays, the kernels captured into one step's graphs times the steps
     launches = (gq.gptq_kernel_launches() - launches0) + (graph_launches * args.steps
                                                           if graphs is not None else 0)
+    # release the graphs now: with the token-sharded Gram they hold NCCL calls, and a
+    # graph holding NCCL work must be gone before the process group is destroyed
+    graphs = None
     if world > 1:
         dist.barrier()
     gq.raise_on_status(status, "timed steps")
