@@ -764,3 +764,21 @@ def test_first_order_gamma_and_trust_region():
         else:
             assert lhs <= alpha * lq + 1e-15
     assert O.trust_region_beta(1.0, 1.0, 0.0) == 1.0
+
+
+def test_planted_mistakes_still_apply():
+    # tests/oracle_mutations.py plants each mistake by replacing a line of the oracle; a
+    # change to the oracle's text must keep every planted mistake applicable (the full
+    # check, which runs these pins once per mistake, is run by hand)
+    import importlib.util
+    import os
+    here = os.path.dirname(os.path.abspath(__file__))
+    spec = importlib.util.spec_from_file_location("oracle_mutations",
+                                                  os.path.join(here, "oracle_mutations.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    src = open(os.path.join(os.path.dirname(here), "oracle", "gptq_oracle.py"),
+               encoding="utf-8").read()
+    assert len(mod.MUTATIONS) >= 50
+    for name, old, new in mod.MUTATIONS:
+        assert old in src and new != old, name
