@@ -111,31 +111,33 @@ def _rank_solve(rank, world, X, W, bits, chunk, groups, weights):
     return H.numpy(), full.numpy(), t.numpy()
 
 
-@pytest.mark.parametrize("groups", [1, 2])
-def test_token_sharded_layer_equals_single_process(groups):
-    rng = np.random.default_rng(3 + groups)
+@pytest.mark.parametrize("groups,world", [(1, 2), (2, 2), (2, 3)])
+def test_token_sharded_layer_equals_single_process(groups, world):
+    # with 3 ranks the token counts differ (the last of the 6 chunks is ragged), the 10
+    # channels split 3/3/4, and rank 1's channels straddle the two 5-channel groups
+    rng = np.random.default_rng(3 + groups + world)
     M, K, N, chunk, bits = 700, 24, 10, 128, 3
     X = rng.standard_normal((M, K)) @ (np.eye(K) + 0.2 * rng.standard_normal((K, K)))
     W = 0.02 * rng.standard_normal((N, K))
     weights = None if groups == 1 else [rng.uniform(0.5, 2.0, M) for _ in range(groups)]
-    out = _run(2, _rank_solve, X, W, bits, chunk, groups, weights)
-    for r in range(2):
+    out = _run(world, _rank_solve, X, W, bits, chunk, groups, weights)
+    for r in range(world):
         assert out[r][0] == "ok", out[r][1]
     H0, codes0, t0 = out[0][1]
-    H1, codes1, t1 = out[1][1]
     for gi in range(groups):
         ref = O.gram(X, None if weights is None else weights[gi])
         np.testing.assert_allclose(H0[gi], ref, rtol=1e-12, atol=1e-9)
-    np.testing.assert_array_equal(H0, H1)          # every rank holds the same statistic
     per = N // groups
     expect = np.zeros((N, K))
     for gi in range(groups):
         expect[gi * per:(gi + 1) * per] = O.solve_layer(
             O.gram(X, None if weights is None else weights[gi]), W[gi * per:(gi + 1) * per],
             bits)["codes"]
-    np.testing.assert_array_equal(codes0, expect)
-    np.testing.assert_array_equal(codes1, expect)
-    np.testing.assert_array_equal(t0, [1.0, 2.0])
+    for r in range(world):
+        Hr, codes_r, t_r = out[r][1]
+        np.testing.assert_array_equal(Hr, H0)      # every rank holds the same statistic
+        np.testing.assert_array_equal(codes_r, expect)
+        np.testing.assert_array_equal(t_r, [world - 1.0, 2.0 * (world - 1)])
 
 
 def _rank_leaves(rank, world):
