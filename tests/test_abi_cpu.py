@@ -288,3 +288,22 @@ def test_every_wrapper_matches_its_c_signature(lib, monkeypatch):
     # the workspace sizes passed are the ones the library asks for
     assert calls["gptq_quantize_layer"][17] >= int(real_ws(gq.GPTQ_OP_QUANTIZE | gq.GPTQ_WS_CAE,
                                                            K, N, 1, 16))
+
+
+@pytest.mark.parametrize("op", [0, 1, 2, 3, 4, 2 | 0x100, 3 | 0x100])
+def test_workspace_sizes_grow_and_stay_aligned(lib, op):
+    # sizes are multiples of 256 bytes, never shrink as the layer grows on the
+    # tensor-core paths (K a multiple of 32; other K take the smaller SIMT workspaces),
+    # and do not overflow at the largest such K the ABI accepts
+    prev = 0
+    for K in (128, 256, 1024, 4096, 14336, 28672, 65504):
+        size = gq.gptq_workspace_size(op, K, 4096, 1, 128)
+        assert size % 256 == 0, (op, K, size)
+        assert size >= prev, (op, K, size, prev)
+        prev = size
+    assert prev >= 4 * 65504 * (65504 if op in (0, 1) else 4096)
+    assert gq.gptq_workspace_size(op, 65535, 4096, 1, 128) % 256 == 0
+    sizes_n = [gq.gptq_workspace_size(op, 4096, N, 1, 128) for N in (1, 100, 4096, 65535)]
+    assert sizes_n == sorted(sizes_n)
+    if op == 0:   # prepare: one more group never costs less
+        assert gq.gptq_workspace_size(0, 4096, 0, 4, 0) > gq.gptq_workspace_size(0, 4096, 0, 2, 0)
