@@ -5,6 +5,7 @@
 from __future__ import annotations
 
 import argparse
+import concurrent.futures
 import glob
 import os
 import subprocess
@@ -31,15 +32,28 @@ def _newer(src, dst, deps):
 def build(force=False, verbose=False, extra=()):
     os.makedirs(OUT, exist_ok=True)
     headers = glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(ROOT, "include", "*.h"))
-    objs = []
+    objs, cmds = [], []
     for src in sorted(glob.glob(os.path.join(CSRC, "*.cu"))):
         obj = os.path.join(OUT, os.path.basename(src) + ".o")
         objs.append(obj)
         if force or _newer(src, obj, headers):
-            cmd = [NVCC, *FLAGS, *extra, "-c", src, "-o", obj]
-            if verbose:
-                print(" ".join(cmd), flush=True)
-            subprocess.run(cmd, check=True)
+            cmds.append([NVCC, *FLAGS, *extra, "-c", src, "-o", obj])
+    # the translation units compile independently: one nvcc per file, several at a time
+    # (the longest file sets the build time)
+    def compile_one(cmd):
+        if verbose:
+            print(" ".join(cmd), flush=True)
+        return subprocess.run(cmd, capture_output=not verbose, text=True)
+    workers = max(1, min(len(cmds), os.cpu_count() or 1, 8))
+    with concurrent.futures.ThreadPoolExecutor(max_workers=workers) as pool:
+        results = list(pool.map(compile_one, cmds))
+    for cmd, r in zip(cmds, results):
+        if r.returncode != 0:
+            if not verbose:
+                sys.stderr.write(r.stdout + r.stderr)
+            raise subprocess.CalledProcessError(r.returncode, cmd)
+        if not verbose and r.stderr.strip():
+            sys.stderr.write(r.stderr)
     if force or any(_newer(o, LIB, []) for o in objs):
         cmd = [NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", *objs, "-o", LIB]
         if verbose:
