@@ -697,9 +697,13 @@ static gptq_status tri_inverse_tc(float *H, int K, const Blocks &bk, float *Tt, 
     if ((s = make_f32_map(&mh[1], Hl, K, K, K, 32, 128)) != GPTQ_OK) return s;
     if ((s = make_f32_map(&mg[0], Gh, K, K, K, 32, 128)) != GPTQ_OK) return s;
     if ((s = make_f32_map(&mg[1], Gl, K, K, K, 32, 128)) != GPTQ_OK) return s;
-    for (int d = (int)levels.size() - 1; d >= 0; --d) {
-        const std::vector<InvNode> &lv = levels[d];
-        if ((int)lv.size() > TC32_MAX_ITEMS) return GPTQ_ERR_ARG;
+    // The nodes of one depth are independent; a depth with more nodes than one launch's
+    // item table (K above 28,672) runs as several rounds of at most TC32_MAX_ITEMS nodes.
+    for (int d = (int)levels.size() - 1; d >= 0; --d)
+    for (size_t c0 = 0; c0 < levels[d].size(); c0 += TC32_MAX_ITEMS) {
+        const std::vector<InvNode> lv(
+            levels[d].begin() + c0,
+            levels[d].begin() + std::min(levels[d].size(), c0 + (size_t)TC32_MAX_ITEMS));
         // T^T of this level: node blocks (b - m) x (m - a) stacked, common pitch
         int pitch = 0, trows = 0;
         std::vector<int> trow0(lv.size());
