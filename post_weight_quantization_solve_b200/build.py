@@ -31,7 +31,8 @@ def _newer(src, dst, deps):
 
 def build(force=False, verbose=False, extra=()):
     os.makedirs(OUT, exist_ok=True)
-    headers = glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(ROOT, "include", "*.h"))
+    headers = (glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) +
+               glob.glob(os.path.join(ROOT, "include", "*.h")))
     objs, cmds = [], []
     for src in sorted(glob.glob(os.path.join(CSRC, "*.cu"))):
         obj = os.path.join(OUT, os.path.basename(src) + ".o")

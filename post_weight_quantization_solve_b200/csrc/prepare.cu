@@ -28,11 +28,10 @@
 #include "common.cuh"
 #include "gemm_simt.cuh"
 #include "gemm_tc32.cuh"
+#include "prepare_plan.h"
 #include "tc_ptx.cuh"
 
 namespace gptq {
-
-constexpr int CH_NB = 128;
 
 __global__ void k_check_finite(const float *A, int64_t count, int32_t *status) {
     int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
@@ -437,38 +436,9 @@ __global__ void k_zero_lower(float *H, int K, const int32_t *status) {
         H[(int64_t)i * K + j] = 0.f;
 }
 
-struct Blocks {
-    int K, T;  // T blocks; block t covers [start(t), start(t+1))
-    int start(int t) const {
-        // blocks are aligned to the bottom-right corner: the first may be short
-        const int first = K - (T - 1) * CH_NB;
-        return t == 0 ? 0 : first + (t - 1) * CH_NB;
-    }
-};
-
-static size_t inverse_scratch_floats(int K) {
-    const int T = (K + CH_NB - 1) / CH_NB;
-    const size_t half = (size_t)((T + 1) / 2) * CH_NB;
-    return half * half;
-}
-
-// Off-diagonal blocks of U = R^-1. The recursion [A B; 0 D]^-1 =
-// [A^-1, -A^-1 B D^-1; 0, D^-1] over block ranges is laid out as a tree; all nodes
-// of one depth are independent and run as one grouped launch per product
-// (deepest first): T = R[a:m, m:b] U[m:b, m:b], then U[a:m, m:b] = -U[a:m, a:m] T.
-struct InvNode {
-    int a, m, b;
-};
-
-static void inv_nodes(const Blocks &bk, int K, int bl, int br, int depth,
-                      std::vector<std::vector<InvNode>> &levels) {
-    if (br - bl <= 1) return;
-    const int mid = (bl + br) / 2;
-    if ((int)levels.size() <= depth) levels.resize(depth + 1);
-    levels[depth].push_back({bk.start(bl), bk.start(mid), br == bk.T ? K : bk.start(br)});
-    inv_nodes(bk, K, bl, mid, depth + 1, levels);
-    inv_nodes(bk, K, mid, br, depth + 1, levels);
-}
+// Off-diagonal blocks of U = R^-1 (the tree of prepare_plan.h): all nodes of one depth
+// are independent and run as grouped launches per product (deepest first):
+// T = R[a:m, m:b] U[m:b, m:b], then U[a:m, m:b] = -U[a:m, a:m] T.
 
 static gptq_status tri_inverse(float *H, int K, int g, const Blocks &bk, float *T,
                                const int32_t *status, cudaStream_t st) {
@@ -700,18 +670,11 @@ static gptq_status tri_inverse_tc(float *H, int K, const Blocks &bk, float *Tt, 
     // The nodes of one depth are independent; a depth with more nodes than one launch's
     // item table (K above 28,672) runs as several rounds of at most TC32_MAX_ITEMS nodes.
     for (int d = (int)levels.size() - 1; d >= 0; --d)
-    for (size_t c0 = 0; c0 < levels[d].size(); c0 += TC32_MAX_ITEMS) {
-        const std::vector<InvNode> lv(
-            levels[d].begin() + c0,
-            levels[d].begin() + std::min(levels[d].size(), c0 + (size_t)TC32_MAX_ITEMS));
-        // T^T of this level: node blocks (b - m) x (m - a) stacked, common pitch
-        int pitch = 0, trows = 0;
-        std::vector<int> trow0(lv.size());
-        for (size_t ni = 0; ni < lv.size(); ++ni) {
-            pitch = std::max(pitch, lv[ni].m - lv[ni].a);
-            trow0[ni] = trows;
-            trows += lv[ni].b - lv[ni].m;
-        }
+    for (const InvRound &round : inv_rounds(levels[d], TC32_MAX_ITEMS)) {
+        const std::vector<InvNode> &lv = round.nodes;
+        // T^T of this round: node blocks (b - m) x (m - a) stacked, common pitch
+        const int pitch = round.pitch, trows = round.trows;
+        const std::vector<int> &trow0 = round.trow0;
         if ((int64_t)trows * pitch > tsz) return GPTQ_ERR_WORKSPACE;
         {   // pairs of the node blocks [a, b) x [a, b) only (normal and transposed)
             static thread_local SplitBlocks sb;

@@ -11,9 +11,14 @@ if ROOT not in sys.path:
 GOLDEN = os.path.join(ROOT, "tests", "golden")
 
 
+@pytest.hookimpl(tryfirst=True)
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: full-size workloads")
+    # scratch files of the tests (tmp_path) stay inside the repository, in a build folder
+    if not config.option.basetemp:
+        os.makedirs(os.path.join(ROOT, "_build"), exist_ok=True)
+        config.option.basetemp = os.path.join(ROOT, "_build", "pytest-tmp")
 
 
 def load_golden(name):
