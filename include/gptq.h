@@ -138,7 +138,11 @@ GPTQ_API gptq_status gptaq_accumulate_cross(float *C, int K, const void *X_fp, c
  * "为什么 Cholesky Factor 不能当作原始逆矩阵": U is upper triangular with
  * U^T U = H^-1; row q of U carries the free-set inverse at q's step.
  * Computed as H = R R^T with R upper (Cholesky of the index-reversed matrix),
- * U = R^-1 (triangular inversion): no explicit H^-1 is formed.
+ * U = R^-1 (triangular inversion): no explicit H^-1 is formed. K a multiple of 32
+ * from 256 up takes the tensor-core path (tf32 x3 products) when the workspace is
+ * the size gptq_workspace_size() reports; other K, or a smaller workspace that
+ * still holds the fp32 SIMT path's scratch (the damped diagonal and one level of
+ * the inverse), take that SIMT path. Both give U to fp32 accuracy.
  *
  *   H        device fp32 [g][K][K] symmetric (the upper triangle is read). On
  *            return it holds U per group: upper triangle U, strict lower zero.
