@@ -288,3 +288,34 @@ def test_grouped_solve_k4096():
         rep = O.replay_row_form(U_ora, W64, s64, wl.bits, c_gpu)
         assert rep["mismatches"] == 0
         assert own_decisions_same(rep, c_gpu.size) >= CODE_SAME
+
+
+def test_prepare_beyond_one_item_table():
+    """K = 28,704: the deepest level of the triangular inverse has more nodes than one
+    launch's item table and runs in two rounds. U is checked as in the 70B test: its
+    trailing block against the oracle's factor of H_d's trailing block, and
+    U H_d U^T = I on sampled rows in fp64."""
+    d = dev()
+    K = 28704
+    g = torch.Generator(device=d).manual_seed(28704)
+    H = torch.zeros(K, K, device=d)
+    for _ in range(2):
+        X = torch.randn(65536, K, device=d, generator=g).to(torch.bfloat16)
+        gq.gptq_accumulate_hessian(H, X)
+        del X
+    U = H.clone()
+    status = gq.gptq_prepare(U, 0.01)
+    gq.raise_on_status(status, "prepare K=28704")
+    diag, _ = O.damped_diagonal(H.diagonal().double().cpu().numpy(), 0.01)
+    t = 1024
+    Hd_t = H[K - t:, K - t:].double().cpu().numpy()
+    Hd_t[np.diag_indices(t)] = diag[K - t:]
+    assert rel_max(U[K - t:, K - t:].double().cpu().numpy(), O.upper_factor(Hd_t)) <= TOL_U
+    Hd = H.double()
+    Hd.diagonal().copy_(torch.as_tensor(diag, device=d))
+    rng = np.random.default_rng(1)
+    r = np.sort(np.union1d(rng.choice(K, 6, replace=False), [0, 127, 128, K // 2, K - 1]))
+    Ur = U[torch.as_tensor(r, device=d)].double()
+    ident = (Ur @ Hd @ Ur.T).cpu().numpy()
+    assert np.abs(ident - np.eye(len(r))).max() <= TOL_IDENT
+    assert torch.count_nonzero(torch.tril(U, diagonal=-1)).item() == 0
