@@ -679,7 +679,7 @@ def unpack_codes(words, bits, K):
 # First-order (gradient) term with a trust-region step
 # --------------------------------------------------------------------------------------
 
-def first_order_obq_sweep(H_d, W, G, beta, bits):
+def first_order_obq_sweep(H_d, W, G, beta, bits, follow=None, band=1e-4):
     """Sequential OBQ on the quadratic model with a first-order term, explicit form.
 
     [G2PTQ] summary: the compensation keeps GPTQ's second-order update and adds the
@@ -697,7 +697,13 @@ def first_order_obq_sweep(H_d, W, G, beta, bits):
     is obq_sweep. PARITY UNPINNED against the pages: no formula or value is printed;
     the pins are internal (reduction to GPTQ, the shifted-start identity, closed forms).
 
-    Returns (codes, W_hat, scales).
+    follow (optional): another run's codes, followed as replay_row_form does. Where
+    they differ from this sweep's decision the step counts as a tie flip when the
+    codes differ by one and |frac(w / s) - 0.5| < band, else as a mismatch, and the
+    sweep continues with the other run's code, so one decision never cascades.
+
+    Returns (codes, W_hat, scales), and with `follow` a fourth item
+    dict(tie_flips, mismatches, worst_tie_distance).
     """
     H_d = np.asarray(H_d, dtype=np.float64)
     W0 = np.asarray(W, dtype=np.float64)
@@ -706,8 +712,22 @@ def first_order_obq_sweep(H_d, W, G, beta, bits):
     w = W0 - beta * np.linalg.solve(H_d, G.T).T
     s, _ = symmetric_scale(w, bits)
     codes = np.zeros((N, K))
+    stats = dict(tie_flips=0, mismatches=0, worst_tie_distance=0.0)
+    Fw = None if follow is None else np.asarray(follow, dtype=np.float64)
     for q in range(K):
         c = quantize_codes(w[:, q], s, bits)
+        if Fw is not None:
+            diff = c != Fw[:, q]
+            if np.any(diff):
+                ratio = w[diff, q] / s[diff]
+                frac_dist = np.abs(np.abs(ratio - np.floor(ratio)) - 0.5)
+                tie = (np.abs(c[diff] - Fw[diff, q]) == 1) & (frac_dist < band)
+                stats["tie_flips"] += int(np.count_nonzero(tie))
+                stats["mismatches"] += int(np.count_nonzero(~tie))
+                if np.any(tie):
+                    stats["worst_tie_distance"] = max(stats["worst_tie_distance"],
+                                                      float(np.max(frac_dist[tie])))
+                c = np.where(diff, Fw[:, q], c)
         w[:, q] = dequantize(c, s, bits)
         codes[:, q] = c
         if q + 1 < K:
@@ -715,6 +735,8 @@ def first_order_obq_sweep(H_d, W, G, beta, bits):
             fx = slice(0, q + 1)
             rhs = beta * G[:, F].T + H_d[F, fx] @ (w[:, fx] - W0[:, fx]).T
             w[:, F] = W0[:, F] - np.linalg.solve(H_d[F, F], rhs).T
+    if Fw is not None:
+        return codes, w, s, stats
     return codes, w, s
 
 

@@ -64,7 +64,9 @@ MUTATIONS = [
     ("first order shift sign", "    return np.asarray(W, dtype=np.float64) - beta * Z, float(np.sum(G * Z))", "    return np.asarray(W, dtype=np.float64) + beta * Z, float(np.sum(G * Z))"),
     ("first order gamma without H^-1", "    return np.asarray(W, dtype=np.float64) - beta * Z, float(np.sum(G * Z))", "    return np.asarray(W, dtype=np.float64) - beta * Z, float(np.sum(G * G))"),
     ("first order sweep drops beta in re-solve", "            rhs = beta * G[:, F].T + H_d[F, fx] @ (w[:, fx] - W0[:, fx]).T", "            rhs = G[:, F].T + H_d[F, fx] @ (w[:, fx] - W0[:, fx]).T"),
-    ("first order sweep scale from W0", "    s, _ = symmetric_scale(w, bits)\n    codes = np.zeros((N, K))\n    for q in range(K):\n        c = quantize_codes(w[:, q], s, bits)", "    s, _ = symmetric_scale(W0, bits)\n    codes = np.zeros((N, K))\n    for q in range(K):\n        c = quantize_codes(w[:, q], s, bits)"),
+    ("first order replay does not follow", "                c = np.where(diff, Fw[:, q], c)\n        w[:, q] = dequantize(c, s, bits)", "                pass\n        w[:, q] = dequantize(c, s, bits)"),
+    ("first order replay tie band ignored", "                tie = (np.abs(c[diff] - Fw[diff, q]) == 1) & (frac_dist < band)", "                tie = np.abs(c[diff] - Fw[diff, q]) == 1"),
+    ("first order sweep scale from W0", "    w = W0 - beta * np.linalg.solve(H_d, G.T).T\n    s, _ = symmetric_scale(w, bits)\n", "    w = W0 - beta * np.linalg.solve(H_d, G.T).T\n    s, _ = symmetric_scale(W0, bits)\n"),
     ("trust region root sign", "    return 1.0 - np.sqrt(1.0 - 2.0 * x)", "    return 1.0 + np.sqrt(1.0 - 2.0 * x) if x < 0 else 1.0 - np.sqrt(1.0 - x)"),
     ("cae p2 without C", "        A = A + np.asarray(C, dtype=np.float64)\n", "        A = A\n"),
     ("cae p2 inclusive mask", "    return np.triu(A @ U.T, k=1) @ U", "    return np.triu(A @ U.T, k=0) @ U"),
@@ -87,9 +89,16 @@ def run_one(workdir, old, new):
         return "not applied"
     with open(path, "w", encoding="utf-8") as f:
         f.write(src.replace(old, new))
+    # the copy is its own pytest root, so the repository's pytest.ini and conftest stay out
+    # of it and the pins import the mutated oracle; the pin that checks the planted
+    # mistakes still apply to the oracle's text is left out, since the copy's text is
+    # changed on purpose
+    with open(os.path.join(case, "pytest.ini"), "w", encoding="utf-8") as f:
+        f.write("[pytest]\n")
     r = subprocess.run([sys.executable, "-m", "pytest", "tests/test_oracle_pins.py", "-x", "-q",
-                        "-p", "no:cacheprovider"], cwd=case, capture_output=True, text=True,
-                       timeout=600)
+                        "-p", "no:cacheprovider", "--rootdir", case, "--deselect",
+                        "tests/test_oracle_pins.py::test_planted_mistakes_still_apply"],
+                       cwd=case, capture_output=True, text=True, timeout=600)
     if r.returncode == 0:
         return "survived"
     failed = [ln for ln in r.stdout.splitlines() if ln.startswith("FAILED")]

@@ -738,6 +738,33 @@ def test_first_order_is_gptq_from_the_shifted_start():
             np.testing.assert_allclose(w_row, w, atol=1e-10)
 
 
+def test_first_order_follow_equals_row_form_replay_from_the_shifted_start():
+    # the explicit first-order sweep's tie-follow mode against replay_row_form (its own
+    # pins) from the shifted start, with planted disagreements: a near tie whose other
+    # code is adopted as a tie flip, and a code two steps away adopted as a mismatch
+    Hd, W, G = _fo_problem(16, 9, 5)
+    beta = 0.8
+    c, w, s = O.first_order_obq_sweep(Hd, W, G, beta, 3)
+    Ws, _ = O.first_order_shift(Hd, W, G, beta)
+    U = O.upper_factor(Hd)
+    # follow its own codes: nothing to count, the same result
+    c2, w2, s2, st = O.first_order_obq_sweep(Hd, W, G, beta, 3, follow=c)
+    assert st["tie_flips"] == 0 and st["mismatches"] == 0
+    np.testing.assert_array_equal(c2, c)
+    np.testing.assert_allclose(w2, w, atol=1e-12)
+    follow = c.copy()
+    follow[2, 5] = c[2, 5] + 2 if c[2, 5] <= 5 else c[2, 5] - 2
+    follow[6, 11] = c[6, 11] + 1 if c[6, 11] < 7 else c[6, 11] - 1
+    for band in (1e-4, 0.6):     # 0.6: every one-apart difference counts as a tie
+        c3, w3, _, st3 = O.first_order_obq_sweep(Hd, W, G, beta, 3, follow=follow, band=band)
+        rep = O.replay_row_form(U, Ws, s, 3, follow, band=band)
+        np.testing.assert_array_equal(c3, rep["codes"])
+        np.testing.assert_allclose(w3, rep["W_hat"], atol=1e-10)
+        assert st3["tie_flips"] == rep["tie_flips"] and st3["mismatches"] == rep["mismatches"]
+        assert c3[2, 5] == follow[2, 5] and c3[6, 11] == follow[6, 11]
+        assert st3["mismatches"] >= 1
+
+
 def test_first_order_diagonal_hessian_is_rtn_of_the_newton_point():
     rng = np.random.default_rng(3)
     K, N = 9, 5
