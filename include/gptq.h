@@ -152,6 +152,11 @@ GPTQ_API gptq_status gptaq_accumulate_cross(float *C, int K, const void *X_fp, c
  *   status   device int32 (see conventions). GPTQ_ERR_NONFINITE for NaN/Inf in H,
  *            GPTQ_ERR_NOT_PD when a pivot p_j <= K * 2^-23 * Hd_jj (Hd the damped
  *            matrix): the pivot is below the factorisation's rounding size.
+ *   Threads: the tensor-core path overlaps steps on a second stream of the library's
+ *   own, with events ordering it against `stream`; that stream and its events are
+ *   kept per (device, caller stream), so calls from several host threads on
+ *   different streams are independent (each with its own workspace). Calls on one
+ *   stream from several threads enqueue one at a time under a lock.
  */
 GPTQ_API gptq_status gptq_prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out,
                          void *ws, size_t ws_bytes, int32_t *status, void *stream);
@@ -163,15 +168,20 @@ GPTQ_API gptq_status gptq_prepare(float *H, int K, int g, float percdamp, uint8_
  * allocate device memory when they need the factor, for example code running
  * inside a host application that owns every device allocation through its own
  * pool and hands plug-ins no workspace, or a latency-critical path that must not
- * take the device-wide synchronisation of cudaMalloc / cudaFree. It computes
- * exactly what gptq_prepare computes, with the same arguments minus the
- * workspace, and allocates nothing: its scratch is a fixed 16 MiB + 64 KiB array
- * in the library's device memory, which every GPU that loads the library holds
- * until the process exits.
+ * take the device-wide synchronisation of cudaMalloc / cudaFree. It takes the same
+ * arguments as gptq_prepare minus the workspace and allocates nothing: its scratch is
+ * a fixed 16 MiB + 64 KiB array in the library's device memory, which every GPU that
+ * loads the library holds until the process exits.
  *
- *   Limit: gptq_workspace_size(GPTQ_OP_PREPARE, K, 0, g, 0) must not exceed that
- *   array (K <= 4096 with g = 1, K <= 2048 with g <= 4); larger sizes return
- *   GPTQ_ERR_ARG before anything is enqueued.
+ *   Path: the array stands in for gptq_prepare's workspace. Where gptq_prepare's full
+ *   workspace fits it (K a multiple of 32 from 256 to 896 with g = 1, to 864 with
+ *   g = 2, to 800 with g = 4) the call takes the tensor-core path with the same
+ *   kernels as gptq_prepare; other sizes take the fp32 SIMT path, whose U agrees with
+ *   gptq_prepare's to fp32 accuracy (not bit for bit).
+ *   Limit: the SIMT path's scratch (the damped diagonal and one level of the
+ *   triangular inverse, g groups) must fit the array: K <= 4096 with g = 1,
+ *   K <= 2048 with g <= 4. Larger sizes return GPTQ_ERR_ARG before anything is
+ *   enqueued.
  *   Set-up: the first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call before
  *   any stream capture.

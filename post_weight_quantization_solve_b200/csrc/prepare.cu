@@ -22,6 +22,7 @@
 
 #include <algorithm>
 #include <cstdlib>
+#include <map>
 #include <mutex>
 #include <vector>
 
@@ -552,37 +553,45 @@ static gptq_status chol_rest_tc(float *H, int K, int j0n, const CUtensorMap (&m)
     return launch_gemm_tc32(m, pr, st);
 }
 
-// Per-device second stream and events for the lookahead (created once).
+// Second stream and events of the lookahead, one set per (device, caller stream),
+// created on first use and kept until exit. Keying on the caller's stream keeps two
+// host threads that enqueue prepare on different streams of one device apart: each
+// has its own side stream and events, so neither can wait on the other's records, and
+// a capture on one stream never pulls in another caller's side-stream work. `mu` is
+// held for a whole enqueue, so calls on the same stream from several threads enqueue
+// one after the other.
 constexpr int LA_MAX_GROUPS = 8;
 struct Lookahead {
+    std::mutex mu;
     cudaStream_t side = nullptr;
     cudaEvent_t fork = nullptr, join = nullptr;
     cudaEvent_t panel[LA_MAX_GROUPS][2], rest[LA_MAX_GROUPS][2];
     bool ok = false;
 };
 
-static Lookahead *lookahead_for_device() {
+static Lookahead *lookahead_for(cudaStream_t caller) {
     static std::mutex mu;
-    static Lookahead la[64];
+    static std::map<std::pair<int, cudaStream_t>, Lookahead *> table;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
     std::lock_guard<std::mutex> lock(mu);
-    Lookahead &L = la[dev];
-    if (!L.ok) {
-        bool good = cudaStreamCreateWithFlags(&L.side, cudaStreamNonBlocking) == cudaSuccess;
-        good = good && cudaEventCreateWithFlags(&L.fork, cudaEventDisableTiming) == cudaSuccess;
-        good = good && cudaEventCreateWithFlags(&L.join, cudaEventDisableTiming) == cudaSuccess;
+    Lookahead *&L = table[{dev, caller}];
+    if (!L) L = new Lookahead();
+    if (!L->ok) {
+        bool good = cudaStreamCreateWithFlags(&L->side, cudaStreamNonBlocking) == cudaSuccess;
+        good = good && cudaEventCreateWithFlags(&L->fork, cudaEventDisableTiming) == cudaSuccess;
+        good = good && cudaEventCreateWithFlags(&L->join, cudaEventDisableTiming) == cudaSuccess;
         for (int gi = 0; gi < LA_MAX_GROUPS && good; ++gi)
             for (int b = 0; b < 2 && good; ++b)
-                good = cudaEventCreateWithFlags(&L.panel[gi][b], cudaEventDisableTiming) == cudaSuccess &&
-                       cudaEventCreateWithFlags(&L.rest[gi][b], cudaEventDisableTiming) == cudaSuccess;
+                good = cudaEventCreateWithFlags(&L->panel[gi][b], cudaEventDisableTiming) == cudaSuccess &&
+                       cudaEventCreateWithFlags(&L->rest[gi][b], cudaEventDisableTiming) == cudaSuccess;
         if (!good) {
             cudaGetLastError();
             return nullptr;
         }
-        L.ok = true;
+        L->ok = true;
     }
-    return &L;
+    return L;
 }
 
 // Trailing sizes below this stay on the SIMT kernels.
@@ -761,8 +770,10 @@ gptq_status prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out, v
     const size_t pair_floats = (size_t)K * CH_NB * 2;
     // the per-(group, parity) pair buffers use the front of the inverse's pair area
     Lookahead *la = (use_tc && g <= LA_MAX_GROUPS && (size_t)g * 2 * pair_floats <= 4 * (size_t)KK)
-                        ? lookahead_for_device()
+                        ? lookahead_for(st)
                         : nullptr;
+    std::unique_lock<std::mutex> la_lock;
+    if (la) la_lock = std::unique_lock<std::mutex>(la->mu);
     bool side_busy = false;         // work issued on the side stream not yet joined
     int rest_of[2] = {-1, -1};      // step whose rest was last recorded in parity slot
     auto join_side = [&]() -> gptq_status {

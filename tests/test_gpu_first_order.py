@@ -2,10 +2,14 @@
 
 The library applies the term as a shifted start W - beta G H^-1 (through U; tf32x3
 tensor-core products for K a multiple of 32 from 256, the fp32 SIMT GEMM otherwise) and then
-runs the ordinary sweep on the shifted fp32 weights; the oracle's explicit per-step
-form equals that reading by its CPU pins. Here: the shift and gamma against the fp64
-solve, then the sweep on the shifted weights by tie-follow replay. The reading itself
-is unpinned against the pages (they print no formula).
+runs the ordinary sweep on the shifted fp32 weights. Here:
+  - the shift and gamma against the same factor in fp64 (the kernel's own error), and
+    against the fp64 solve within a first-order perturbation bound derived per case from
+    U's measured error and the case's own G and H_d (no fixed widening);
+  - the codes of the whole GPU path (shift, then sweep) against the oracle's explicit
+    per-step first-order sweep from its own fp64 start, by tie-follow;
+  - the sweep on the GPU's shifted weights by the row-form replay.
+The reading itself is unpinned against the pages (they print no formula).
 """
 
 import numpy as np
@@ -23,6 +27,25 @@ pytestmark = pytest.mark.gpu
 # the two chained tf32x3 products against the same operands in fp64: the bound of P1,
 # which the residual computes by the same two-product route
 TOL_KERNEL = TOL_P1
+
+
+def shift_bound(U_gpu, U_ora, Hd, G):
+    """First-order perturbation bounds of the shift d = -beta G M (M = H_d^-1 = U^T U) and
+    of gamma = sum_n g_n M g_n^T when M is formed from the GPU's U instead of the exact
+    factor. With eps = ||U_gpu - U_ora||_2 / ||U_ora||_2,
+        ||U_gpu^T U_gpu - M||_2 <= (2 eps + eps^2) ||M||_2,
+    so ||delta d||_F <= (2 eps + eps^2) ||M||_2 beta ||G||_F and
+    |delta gamma| <= (2 eps + eps^2) ||M||_2 ||G||_F^2. Relative to the exact values:
+        d:     (2 eps + eps^2) * ||G||_F ||M||_2 / ||G M||_F      (<= (2 eps + eps^2) kappa(H_d))
+        gamma: (2 eps + eps^2) * ||G||_F^2 ||M||_2 / gamma.
+    Returns (eps, rel_d, rel_gamma)."""
+    eps = np.linalg.norm(U_gpu - U_ora, 2) / np.linalg.norm(U_ora, 2)
+    M = np.linalg.inv(Hd)
+    m2 = np.linalg.norm(M, 2)
+    gf = np.linalg.norm(G)
+    amp = 2 * eps + eps * eps
+    gamma = float(np.sum((G @ M) * G))
+    return eps, amp * gf * m2 / np.linalg.norm(G @ M), amp * gf * gf * m2 / gamma
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -68,12 +91,55 @@ def test_shift_and_gamma_match_oracle(K, N, gdtype, beta):
     # the kernel: the step against the same factor in fp64, beta G (U^T U) and |G U^T|^2
     U64, G64 = _np(U), _np(G)
     T64 = G64 @ U64.T
-    assert rel_max(_np(Ws) - _np(W), -beta * T64 @ U64) <= TOL_KERNEL
-    assert gamma.item() == pytest.approx(float(np.sum(T64 * T64)), rel=TOL_KERNEL)
-    # end to end against the fp64 solve: the step applies U twice, so its bound is U's
-    # tolerance amplified by the conditioning of H (checked here with a 10x margin)
-    assert rel_max(_np(Ws) - _np(W), W_ora - _np(W)) <= 10 * TOL_U
-    assert gamma.item() == pytest.approx(gamma_ora, rel=10 * TOL_U)
+    d_gpu, d_same = _np(Ws) - _np(W), -beta * T64 @ U64
+    gamma_same = float(np.sum(T64 * T64))
+    assert rel_max(d_gpu, d_same) <= TOL_KERNEL
+    kern_f = np.linalg.norm(d_gpu - d_same) / np.linalg.norm(d_same)
+    assert kern_f <= TOL_KERNEL
+    assert gamma.item() == pytest.approx(gamma_same, rel=TOL_KERNEL)
+    # end to end against the fp64 solve: U itself within its tolerance, and the shift and
+    # gamma within the perturbation that U's measured error allows (shift_bound) plus the
+    # kernel's own error on top
+    U_ora = O.upper_factor(Hd)
+    assert rel_max(U64, U_ora) <= TOL_U
+    eps, rel_d, rel_g = shift_bound(U64, U_ora, Hd, G64)
+    d_ora = W_ora - _np(W)
+    bound_d = kern_f * (1 + rel_d) + rel_d
+    assert np.linalg.norm(d_gpu - d_ora) / np.linalg.norm(d_ora) <= bound_d, (eps, rel_d)
+    kern_g = abs(gamma.item() - gamma_same) / gamma_same
+    assert abs(gamma.item() - gamma_ora) / gamma_ora <= kern_g * (1 + rel_g) + rel_g, (eps, rel_g)
+
+
+@pytest.mark.parametrize("K,N,bs,gdtype,beta", [(256, 96, 128, torch.float32, 0.7),
+                                                (192, 130, 32, torch.bfloat16, 1.0),
+                                                (256, 64, 64, torch.bfloat16, 0.35)])
+def test_first_order_codes_match_explicit_oracle_sweep(K, N, bs, gdtype, beta):
+    # the whole GPU path (tf32x3 shift for K = 256, the SIMT shift for K = 192, then the
+    # sweep) against the oracle's explicit per-step solve of the quadratic model from its
+    # own fp64 start and scales (the oracle factors nothing: H_d^-1 g and the re-solves
+    # are np.linalg.solve on the GPU's Gram, upcast)
+    H_in, U, W, G, st = _setup(K, N, 31 + K + N, gdtype)
+    Hd, _ = O.dead_and_damp(H_in, 0.01)
+    Ws = W.clone()
+    gq.gptq_first_order_shift(Ws, U, G, beta, status=st)
+    scales = torch.empty(N, device=dev())
+    Wq = Ws.clone()
+    codes, st = gq.gptq_quantize_layer(Wq, U, 3, bs, scales_out=scales, write_back=True, status=st)
+    gq.raise_on_status(st, "first-order solve")
+    torch.cuda.synchronize()
+    c_gpu = codes.cpu().numpy().astype(np.float64)
+    c_ora, w_ora, s_ora, stats = O.first_order_obq_sweep(Hd, _np(W), _np(G), beta, 3,
+                                                         follow=c_gpu, band=TIE_BAND)
+    assert stats["mismatches"] == 0, stats
+    assert 1.0 - stats["tie_flips"] / c_gpu.size >= CODE_SAME
+    # scales: |amax(a) - amax(b)| <= max |a - b| per channel, plus fp32 rounding
+    Ws_ora, _ = O.first_order_shift(Hd, _np(W), _np(G), beta)
+    amax = np.abs(Ws_ora).max(axis=1)
+    rtol = np.abs(_np(Ws) - Ws_ora).max(axis=1) / amax + 4 * 2.0 ** -24
+    assert np.all(np.abs(_np(scales) - s_ora) <= rtol * s_ora)
+    # write-back on the GPU's grid with the followed codes
+    z = 4.0
+    np.testing.assert_array_equal(_np(Wq), (_np(scales)[:, None] * (c_gpu - z)).astype(np.float32))
 
 
 @pytest.mark.parametrize("K,N,sample", [(392, 200, None), (256, 9600, 64)])

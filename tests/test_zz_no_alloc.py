@@ -23,35 +23,46 @@ from gpu_util import TOL_U, dev, rel_max
 pytestmark = pytest.mark.gpu
 
 
-def _hessian(K, seed, d):
-    wl = synth.WORKLOADS["mlp_up"].scaled(K=K, N=8, M=3 * K, seed=seed)
-    X = synth.tokens_chunk(wl, 0, d).float()
-    return 2.0 * (X.T @ X)          # test input only
+def _hessian(K, seed, d, g=1):
+    Hs = []
+    for gi in range(g):
+        wl = synth.WORKLOADS["mlp_up"].scaled(K=K, N=8, M=3 * K, seed=seed + 101 * gi)
+        X = synth.tokens_chunk(wl, 0, d).float()
+        Hs.append(2.0 * (X.T @ X))          # test input only
+    return Hs[0] if g == 1 else torch.stack(Hs)
 
 
 def _noalloc(lib, H, percdamp, dead, status):
-    return lib.gptq_prepare_noalloc(ctypes.c_void_p(H.data_ptr()), H.shape[-1], 1,
+    g = 1 if H.dim() == 2 else H.shape[0]
+    return lib.gptq_prepare_noalloc(ctypes.c_void_p(H.data_ptr()), H.shape[-1], g,
                                     ctypes.c_float(percdamp), ctypes.c_void_p(dead.data_ptr()),
                                     ctypes.c_void_p(status.data_ptr()),
                                     ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+
+
+# Sizes in an order that would expose stale scratch from the call before: the SIMT path
+# (K = 1000, 4096) and the tensor-core path, where the array also holds the tf32 pairs
+# and the lookahead's panel buffers (K = 512 and 896 with one Hessian, K = 512 with two).
+CASES = [(1000, 1, 11), (512, 1, 14), (4096, 1, 12), (896, 1, 15), (512, 2, 16), (1000, 1, 13),
+         (512, 1, 17)]
 
 
 def test_noalloc_prepare_matches_workspace_prepare():
     build()
     lib = gq.load_library()
     d = dev()
-    for K, seed in [(1000, 11), (4096, 12), (1000, 13)]:
-        H = _hessian(K, seed, d)
+    for K, g, seed in CASES:
+        H = _hessian(K, seed, d, g)
         U_ref = H.clone()
-        dead_ref = torch.empty(K, dtype=torch.uint8, device=d)
+        dead_ref = torch.empty((g, K) if g > 1 else (K,), dtype=torch.uint8, device=d)
         st_ref = gq.gptq_prepare(U_ref, 0.01, dead_out=dead_ref)
         U_new = H.clone()
-        dead_new = torch.full((K,), 7, dtype=torch.uint8, device=d)
+        dead_new = torch.full_like(dead_ref, 7)
         st_new = torch.zeros(1, dtype=torch.int32, device=d)
         assert _noalloc(lib, U_new, 0.01, dead_new, st_new) == gq.GPTQ_OK
         torch.cuda.synchronize()
         assert int(st_ref.item()) == gq.GPTQ_OK and int(st_new.item()) == gq.GPTQ_OK
-        assert rel_max(U_new.double().cpu().numpy(), U_ref.double().cpu().numpy()) <= TOL_U
+        assert rel_max(U_new.double().cpu().numpy(), U_ref.double().cpu().numpy()) <= TOL_U, (K, g)
         assert torch.equal(dead_new, dead_ref)
 
 
