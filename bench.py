@@ -40,6 +40,8 @@ METRIC = "GPTQ layer-solve ms & weights quantized/s (4096×14336, W3); % of TC/H
 # kernel, from an ncu capture of the same 65,536-token launch. Set to None whenever
 # k_gram_tc2 changes until it is captured again.
 GRAM_TRAFFIC_BYTES = 1.588568e9 + 0.504924e9
+GRAM_TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one k_gram_tc2 launch "
+                       "(65,536 tokens, K=4096), profiles/gram_tc2_mlp_up_w3_chunk65536.md")
 UNIT = "weights/s"
 
 
@@ -474,6 +476,31 @@ def run_ours(args, rank, world, local_rank):
     pack_ms = pk0.elapsed_time(pk1) / 10
     pack_bytes = Nl * K + words.numel() * 4
 
+    # one eager solve with the library's kernel timing on (outside the timed steps): the
+    # per-class kernel times of prepare + quantize, and the sweep's dependent-chain latency
+    solve_prof = None
+    if not tokens_sharded and Nl > 0:
+        with torch.cuda.stream(stream):
+            gram_part()
+        torch.cuda.synchronize()
+        gq.gptq_profile_enable(True)
+        with torch.cuda.stream(stream):
+            pe0, pe1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            pe0.record(stream)
+            prepare_part()
+            quantize_part()
+            pe1.record(stream)
+        torch.cuda.synchronize()
+        solve_prof = {k: gq.gptq_profile_read(v) for k, v in
+                      (("sweep", gq.GPTQ_PROF_SWEEP), ("update", gq.GPTQ_PROF_UPDATE),
+                       ("diag", gq.GPTQ_PROF_DIAG), ("tc32", gq.GPTQ_PROF_TC32))}
+        gq.gptq_profile_enable(False)
+        solve_prof["eager_ms"] = pe0.elapsed_time(pe1)
+        out = gq.gptq_chain_latency(torch.zeros(3, device=dev), steps=1 << 16, stream=stream)
+        torch.cuda.synchronize()
+        solve_prof["chain"] = (float(out[0].item()), float(out[1].item()))
+        gq.raise_on_status(status, "profiled solve")
+
     e2e = None
     # through the public API with host buffers: the plain per-channel workloads
     if (not args.no_e2e and g == 1 and not wl.gptaq and not tokens_sharded and not grouped
@@ -496,11 +523,13 @@ def run_ours(args, rank, world, local_rank):
                 "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 4),
                 "traffic": GRAM_TRAFFIC_BYTES if (g == 1 and args.workload == "mlp_up_w3") else None,
+                "traffic_source": GRAM_TRAFFIC_SOURCE,
                 "peak_source": ("MEASURED_PEAKS.json bf16_tflops_sustained (of measured)"
                                 if peaks.get("bf16_tflops_sustained") else "fallback 1.4 PFLOP/s"),
                 "per_launch": f"{ch} tokens x K(K+1) = {flops_launch:.3e} FLOP (symmetric count)",
                 "ms_per_launch": round(gram_launch_ms, 4)}
     weights = K * N * (1 if tokens_sharded else world)
+    solve = solve_summary(wl, solve_prof, prep_ms, quant_ms, peaks, wl.groupsize > 0)
     line = {
         "metric": METRIC, "value": weights / (ms_per_step * 1e-3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -522,6 +551,7 @@ def run_ours(args, rank, world, local_rank):
                       "quantize_includes_first_order_shift": bool(wl.first_order),
                       "prepare_includes_residual": bool(wl.gptaq)},
         "roofline": roofline,
+        "solve": solve,
         "pack": {"kernel": "k_pack (gptq_pack_codes)", "ms": round(pack_ms, 4),
                  "bytes": pack_bytes, "gbs": round(pack_bytes / (pack_ms * 1e-3) / 1e9, 1),
                  "frac_of_hbm": (round(pack_bytes / (pack_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)
@@ -539,6 +569,75 @@ def run_ours(args, rank, world, local_rank):
         cb = oracle_sample(wl, args.cpu_sample_seconds)
         line["cpu_baseline"] = cpu_baseline_entry(cb, cb["value"])
     return line
+
+
+def solve_summary(wl, prof, prep_ms, quant_ms, peaks, input_groups):
+    """The layer solve (prepare + quantize on a resident H: the headline of the metric)
+    with its rooflines, from the timed steps and one profiled eager solve."""
+    K, N = wl.K, wl.N
+    ms = prep_ms + quant_ms
+    hbm = peaks.get("hbm_gbs") or 6650.0
+    tflops = peaks.get("bf16_tflops_sustained") or 1400.0
+    # algorithmic HBM bytes per weight of the solve: W in (bf16), one code byte out, and
+    # U (fp32 K x K) read once, amortised over the N channels
+    bpw = 2.0 + 1.0 + 4.0 * K / N
+    out = {"what": "layer solve: gptq_prepare + gptq_quantize_layer on a resident H (CUDA-graph "
+                   "replay, timed steps)",
+           "ms": ms, "weights_per_s": K * N / (ms * 1e-3),
+           "hbm_roofline": {"bytes_per_weight": round(bpw, 4),
+                            "peak_weights_per_s": hbm * 1e9 / bpw,
+                            "frac": round(K * N / (ms * 1e-3) / (hbm * 1e9 / bpw), 6),
+                            "peak_gbs": hbm, "peak_source": "MEASURED_PEAKS.json hbm_gbs (of measured)"
+                            if peaks.get("hbm_gbs") else "fallback"}}
+    if not prof:
+        return out
+    sweep_ms, sweep_n = prof["sweep"]
+    upd_ms, upd_n = prof["update"]
+    cyc, ns = prof["chain"]
+    tc_sweep = (K % 4 == 0 and not input_groups and
+                os.environ.get("GPTQ_SWEEP_FORM", "3") not in ("0", "1", "2"))
+    S = (256 if wl.gptaq else 512) if tc_sweep else 512
+    # sweep: bytes it must move (fp32 working weights in, codes out, E as a bf16 pair out;
+    # the starting weights in for CAE, the GPTAQ V pair out) against its dependent chain
+    sweep_bytes = N * K * (4 + 1 + 4 + (4 if wl.cae else 0) + (4 if wl.gptaq else 0))
+    chain_ms = K * ns * 1e-6
+    out["sweep"] = {
+        "kernel": ("k_sweep_tc (tensor-core near updates in TMEM)" if tc_sweep
+                   else "k_sweep_thread / k_sweep_lanes"),
+        "ms": round(sweep_ms, 4), "launches": sweep_n,
+        "chain_ns_per_step": round(ns, 3), "chain_cycles_per_step": round(cyc, 2),
+        "chain_bound_ms": round(chain_ms, 4),
+        "frac_of_chain_bound": round(chain_ms / sweep_ms, 4) if sweep_ms else None,
+        "bound": "latency (K dependent rounding steps per channel)",
+        "hbm_bytes": sweep_bytes,
+        "hbm_frac": round(sweep_bytes / (sweep_ms * 1e-3) / (hbm * 1e9), 4) if sweep_ms else None}
+    # far updates: every super-block's E (and GPTAQ's V) against the coordinates after it
+    useful = 0.0
+    for sb0 in range(0, K, S):
+        sb1 = min(K, sb0 + S)
+        useful += 2.0 * N * (sb1 - sb0) * (K - sb1) * (2 if wl.gptaq else 1)
+    if not tc_sweep:     # the SIMT sweeps leave the near updates to the same kernel
+        B = wl.blocksize
+        for sb0 in range(0, K, 512):
+            sb1 = min(K, sb0 + 512)
+            for i0 in range(sb0, sb1, B):
+                i1 = min(i0 + B, sb1)
+                useful += 2.0 * N * (i1 - i0) * (sb1 - i1) * (2 if wl.gptaq else 1)
+    ach = useful / (upd_ms * 1e-3) / 1e12 if upd_ms else None
+    out["update"] = {
+        "kernel": "k_update_tc (bf16x3: three MMAs per product)", "ms": round(upd_ms, 4),
+        "launches": upd_n, "useful_flop": useful,
+        "achieved_tflops_useful": round(ach, 1) if ach else None,
+        "peak_tflops": tflops, "frac_of_sustained": round(ach / tflops, 4) if ach else None,
+        "split_ceiling": "1/3 of peak in useful FLOP (each product is three bf16 MMAs)",
+        "frac_of_split_ceiling": round(3 * ach / tflops, 4) if ach else None}
+    out["prepare_kernels"] = {"diag_ms": round(prof["diag"][0], 4), "diag_launches": prof["diag"][1],
+                              "tc32_ms": round(prof["tc32"][0], 4), "tc32_launches": prof["tc32"][1]}
+    out["profiled_eager_solve_ms"] = round(prof["eager_ms"], 4)
+    out["timing"] = ("sweep / update / factor kernels: CUDA events around each launch on its "
+                     "stream in one eager solve after the timed steps (gptq_profile_*); chain: "
+                     "gptq_chain_latency, one thread, 65536 dependent steps")
+    return out
 
 
 def run_e2e(args, wl, X, W, dev, gq, torch, dist, world):

@@ -397,6 +397,40 @@ GPTQ_API float gptq_trust_region_beta(float alpha, double loss_gptq, double gamm
  */
 GPTQ_API gptq_status gptq_selftest_timeout(int32_t *status, void *stream);
 
+/*
+ * Kernel timing by class -- a benchmark diagnostic (the pages have no counterpart).
+ *
+ * gptq_profile_enable(1) starts a window: from then on the library records a pair of
+ * CUDA events around every launch of the classes below, on the stream that launch
+ * uses (nothing is recorded while a stream is being captured into a CUDA graph);
+ * gptq_profile_enable(0) stops recording. gptq_profile_read synchronises the
+ * window's events of one class and returns their summed elapsed time (ms) and the
+ * number of launches. The events add a little host work per launch; leave profiling
+ * off outside measurements.
+ */
+typedef enum {
+    GPTQ_PROF_SWEEP = 0,     /* in-block sweep kernels of gptq_quantize_layer(_grouped) */
+    GPTQ_PROF_UPDATE = 1,    /* tensor-core lazy (near / far) updates */
+    GPTQ_PROF_DIAG = 2,      /* diagonal-block factor of gptq_prepare */
+    GPTQ_PROF_TC32 = 3,      /* tf32 x3 tensor-core products (factor, inverse, residual, shift) */
+    GPTQ_PROF_KINDS = 4
+} gptq_prof_kind;
+
+GPTQ_API gptq_status gptq_profile_enable(int on);
+GPTQ_API gptq_status gptq_profile_read(int kind, double *ms, int *launches);
+
+/*
+ * gptq_chain_latency -- one thread runs `steps` steps (a multiple of 8, >= 8) of the
+ * sweep's dependent chain for one coordinate: the previous error applied to the
+ * coordinate (FMA), the scale, round-half-even and clamp to the grid, and the
+ * normalised error (FMA, multiply), each step depending on the last. Writes, to the
+ * device buffer `out` (3 floats): SM clock cycles per step, nanoseconds per step, and
+ * a value that keeps the chain live. K steps of this chain bound a sweep over K
+ * coordinates from below, however many channels run in parallel. A diagnostic (the
+ * pages have no counterpart).
+ */
+GPTQ_API gptq_status gptq_chain_latency(float *out, int steps, void *stream);
+
 /* Workspace bytes for an operation (gptq_op); 0 when none is needed. */
 GPTQ_API size_t gptq_workspace_size(int op, int K, int N, int g, int blocksize);
 

@@ -22,6 +22,7 @@ GPTQ_BF16, GPTQ_F32 = 0, 1
 GPTQ_OP_PREPARE, GPTQ_OP_RESIDUAL, GPTQ_OP_QUANTIZE, GPTQ_OP_QUANTIZE_GROUPED = 0, 1, 2, 3
 GPTQ_OP_FIRST_ORDER = 4
 GPTQ_WS_CAE = 0x100
+GPTQ_PROF_SWEEP, GPTQ_PROF_UPDATE, GPTQ_PROF_DIAG, GPTQ_PROF_TC32 = 0, 1, 2, 3
 
 EXPORTS = ("gptq_accumulate_hessian", "gptaq_accumulate_cross", "gptq_prepare",
            "gptq_prepare_noalloc",
@@ -29,7 +30,8 @@ EXPORTS = ("gptq_accumulate_hessian", "gptaq_accumulate_cross", "gptq_prepare",
            "gptq_quantize_layer_grouped", "gptq_pack_codes", "gptq_unpack_codes",
            "gptq_first_order_shift", "gptq_trust_region_beta", "gptq_selftest_timeout",
            "gptq_workspace_size",
-           "gptq_kernel_launches", "gptq_status_string")
+           "gptq_kernel_launches", "gptq_status_string", "gptq_profile_enable",
+           "gptq_profile_read", "gptq_chain_latency")
 
 _lib = None
 
@@ -69,6 +71,9 @@ def load_library():
         "gptq_workspace_size": [I, I, I, I, I],
         "gptq_status_string": [I],
         "gptq_kernel_launches": [],
+        "gptq_profile_enable": [I],
+        "gptq_profile_read": [I, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)],
+        "gptq_chain_latency": [P, I, P],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -384,6 +389,32 @@ def gptq_trust_region_beta(alpha, loss_gptq, gamma):
     return float(load_library().gptq_trust_region_beta(ctypes.c_float(alpha),
                                                         ctypes.c_double(loss_gptq),
                                                         ctypes.c_double(gamma)))
+
+
+def gptq_profile_enable(on):
+    """Start (True) or stop (False) a kernel-timing window (see include/gptq.h)."""
+    _check(load_library().gptq_profile_enable(1 if on else 0), "gptq_profile_enable")
+
+
+def gptq_profile_read(kind):
+    """(summed ms, launches) of one kernel class in the current timing window."""
+    ms, n = ctypes.c_double(0.0), ctypes.c_int(0)
+    _check(load_library().gptq_profile_read(int(kind), ctypes.byref(ms), ctypes.byref(n)),
+           "gptq_profile_read")
+    return ms.value, n.value
+
+
+def gptq_chain_latency(out, steps=65536, stream=None):
+    """One thread times `steps` steps of the sweep's dependent chain: out (3 float32 on
+    the device) receives SM cycles per step, ns per step and a keep-alive value. Returns
+    `out` (not synchronised)."""
+    lib = load_library()
+    dev = _device(out, "out")
+    args = (_ptr(out, dev, "out"), int(steps), _stream(stream, dev))
+    with torch.cuda.device(dev):
+        code = lib.gptq_chain_latency(*args)
+    _check(code, "gptq_chain_latency")
+    return out
 
 
 def gptq_selftest_timeout(status=None, stream=None):

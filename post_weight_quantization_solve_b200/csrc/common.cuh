@@ -57,6 +57,11 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
     return *reinterpret_cast<const float2 *>(&d);
 }
 
+// Timing windows of gptq_profile_enable: events around a launch of one class on its
+// stream (profile.cu). prof_begin returns -1 when nothing is recorded.
+int prof_begin(int kind, cudaStream_t st);
+void prof_end(int rec, cudaStream_t st);
+
 inline bool aligned(const void *p, size_t a) {
     return (reinterpret_cast<uintptr_t>(p) % a) == 0;
 }

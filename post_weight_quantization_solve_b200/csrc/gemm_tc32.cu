@@ -391,8 +391,11 @@ gptq_status launch_gemm_tc32(const CUtensorMap maps[4], Tc32Params &p, cudaStrea
     if (units == 0) return GPTQ_OK;
     const int grid = std::min(units, tc32_sms());
     cudaFuncSetAttribute(k_gemm_tc32, cudaFuncAttributeMaxDynamicSharedMemorySize, G32_SMEM);
+    const int rec = prof_begin(GPTQ_PROF_TC32, st);
     k_gemm_tc32<<<grid, G32_THREADS, G32_SMEM, st>>>(maps[0], maps[1], maps[2], maps[3], p);
-    return launch_status();
+    const gptq_status s = launch_status();
+    prof_end(rec, st);
+    return s;
 }
 
 }  // namespace gptq

@@ -794,11 +794,14 @@ gptq_status prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out, v
             for (int gi = 0; gi < g; ++gi)
                 if (cudaStreamWaitEvent(st, la->rest[gi][(t + 2) & 1], 0) != cudaSuccess)
                     return GPTQ_ERR_CUDA;
+        const int rec = prof_begin(GPTQ_PROF_DIAG, st);
         if (diag_pairs)
             k_chol_diag2<<<g, DG_T, chol_smem, st>>>(H, K, j0, nb, diag_d, tol, status);
         else
             k_chol_diag<<<g, DG_T, chol_smem, st>>>(H, K, j0, nb, diag_d, tol, status);
-        if ((s = launch_status()) != GPTQ_OK) return s;
+        s = launch_status();
+        prof_end(rec, st);
+        if (s != GPTQ_OK) return s;
         if (j0 == 0) break;
         if (use_tc && j0 >= TC_STEP_MIN && nb % 32 == 0) {
             if (la) {

@@ -39,6 +39,7 @@
 #include <cstdlib>
 
 #include "common.cuh"
+#include "sweep_tc.cuh"
 #include "update_tc.cuh"
 
 namespace gptq {
@@ -719,6 +720,7 @@ __global__ void __launch_bounds__(256) k_finalize(T *__restrict__ W, const uint8
 
 constexpr int SUPER = 512;
 
+
 struct QLayout {
     int ldU, ldG, ldE;
     explicit QLayout(int K, int N, int g) {
@@ -738,6 +740,7 @@ size_t quantize_workspace(int K, int N, int g, int blocksize) {
     for (int i = 0; i < 4; ++i) c.take<__nv_bfloat16>((size_t)SUPER * lay.ldE);   // Eh El Ph Pl
     c.take<float>((size_t)N);                               // scale
     c.take<float>((size_t)N);                               // loss_acc
+    c.take<float>((size_t)g * K);                           // 1 / U_jj (tensor-core sweep)
     return round_up(c.off, 256);
 }
 
@@ -817,6 +820,7 @@ static gptq_status quantize_impl(void *W, int wdtype, int N, int K, const float 
     __nv_bfloat16 *Pl = cv.take<__nv_bfloat16>((size_t)SUPER * lay.ldE);
     float *scale = cv.take<float>((size_t)N);
     float *loss_acc = cv.take<float>((size_t)N);
+    float *rp = cv.take<float>((size_t)groups * K);
     const bool grouped = go.G > 0 || go.perm != nullptr;
     const int G = go.G > 0 ? go.G : K;
     const int ng = (K + G - 1) / G;
@@ -905,61 +909,102 @@ static gptq_status quantize_impl(void *W, int wdtype, int N, int K, const float 
     base.neg[0] = 1;
     base.neg[1] = 0;
 
-    // one thread per channel when that still gives every SM two warps, two lanes per
-    // channel there instead for CAE (its starting weights then stay in registers: 2.25
-    // against 2.51 ms for a 14336 x 4096 layer on B200, while the plain and GPTAQ sweeps
-    // time the same or slower with two lanes); four lanes per channel for fewer channels.
-    // GPTQ_SWEEP_FORM = 0, 1 or 2 picks the form (comparisons and tests).
+    // Per-channel scales take the tensor-core sweep (sweep_tc.cu: one launch per
+    // super-block, the near updates accumulated in TMEM) whenever its TMA maps can be
+    // built (K % 4 == 0). Otherwise, and for input groups: one thread per channel when
+    // that still gives every SM two warps, two lanes per channel there instead for CAE
+    // (its starting weights then stay in registers: 2.25 against 2.51 ms for a
+    // 14336 x 4096 layer on B200, while the plain and GPTAQ sweeps time the same or
+    // slower with two lanes); four lanes per channel for fewer channels.
+    // GPTQ_SWEEP_FORM = 0, 1, 2 or 3 picks the form (comparisons and tests; 3 = tensor
+    // core, used only where eligible).
     int form = (int64_t)N >= 2LL * 148 * 32 ? (cae ? 2 : 0) : 1;
-    if (const char *f = getenv("GPTQ_SWEEP_FORM")) form = atoi(f) == 2 ? 2 : atoi(f) == 1 ? 1 : 0;
-    const int cta = form == 0 ? SW_T : 128;
-    const int per_cta = form == 0 ? SW_T : form == 1 ? 32 : 64;
-    const dim3 grid((per_group + per_cta - 1) / per_cta, groups);
-    SweepKernel kern = sweep_kernel(form, gptaq, gmode, cae != 0);
-    const size_t smem = form == 0 ? sweep_thread_smem(gptaq, gmode, cae != 0)
-                                  : sweep_lanes_smem(gptaq, gmode, form == 1 ? 4 : 2);
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-        return launch_status();
-    const int vec = ((K % 4 == 0 && aligned(U, 16) && (!gptaq || aligned(P1, 16))) ? 1 : 0) |
-                    ((K % 16 == 0 && aligned(cp, 16)) ? 2 : 0);
-    SweepGroups sg{G, gsc, ng, gsel};
-    for (int sb0 = 0; sb0 < K; sb0 += SUPER) {
-        const int sb1 = min(K, sb0 + SUPER);
-        for (int i0 = sb0; i0 < sb1; i0 += blocksize) {
-            const int i1 = min(i0 + blocksize, sb1);
-            const int bs = i1 - i0;
-            kern<<<grid, cta, smem, st>>>(Wk, N, per_group, K, i0, bs, U, P1, scale, bits, cp, Eh,
-                                          El, Ph, Pl, lay.ldE, lay.ldG, i0 - sb0, loss_acc, vec,
-                                          status, sg, W0k);
-            s = launch_status();
-            if (s != GPTQ_OK) return s;
-            if (i1 >= sb1) continue;
-            for (int gi = 0; gi < groups; ++gi) {      // near: the rest of the super-block
+    const bool tc_ok = gmode == 0 && sweep_tc_eligible(K, U, P1);
+    if (tc_ok) form = 3;
+    if (const char *f = getenv("GPTQ_SWEEP_FORM")) {
+        const int fv = atoi(f);
+        if (fv >= 0 && fv <= 2) form = fv;
+        else if (fv == 3 && tc_ok) form = 3;
+    }
+    if (form == 3) {
+        static thread_local SweepTcMaps stc_maps;
+        SweepTcMaps *stc = &stc_maps;
+        if ((s = sweep_tc_setup(stc, Wk, W0k, U, P1, Uh, Ul, Qh, Ql, lay.ldU, rp, N, K, groups,
+                                st)) != GPTQ_OK)
+            return s;
+        const int S = sweep_tc_super(gptaq);
+        for (int sb0 = 0; sb0 < K; sb0 += S) {
+            const int sb1 = min(K, sb0 + S);
+            if ((s = sweep_tc_launch(*stc, scale, bits, cp, Eh, El, Ph, Pl, lay.ldE, lay.ldG,
+                                     loss_acc, status, N, per_group, K, groups, sb0, sb1 - sb0,
+                                     gptaq, cae != 0, st)) != GPTQ_OK)
+                return s;
+            if (sb1 >= K) break;
+            for (int gi = 0; gi < groups; ++gi) {      // far: everything after the super-block
                 UpdateParams p = base;
-                p.C = Wk + (int64_t)gi * per_group * K + i1;
-                p.Ncols = sb1 - i1;
-                p.L = bs;
+                p.C = Wk + (int64_t)gi * per_group * K + sb1;
+                p.Ncols = K - sb1;
+                p.L = sb1 - sb0;
                 p.a_x0 = gi * lay.ldG;
-                p.a_y0 = i0 - sb0;
-                p.b_x0 = i1;
-                p.b_y0 = i0;
+                p.a_y0 = 0;
+                p.b_x0 = sb1;
+                p.b_y0 = sb0;
                 const int box = p.L % 64 == 0 ? 64 : 16;
                 if ((s = launch_update_tc(maps[box == 64][gi], p, box, st)) != GPTQ_OK) return s;
             }
         }
-        if (sb1 >= K) break;
-        for (int gi = 0; gi < groups; ++gi) {          // far: everything after the super-block
-            UpdateParams p = base;
-            p.C = Wk + (int64_t)gi * per_group * K + sb1;
-            p.Ncols = K - sb1;
-            p.L = sb1 - sb0;
-            p.a_x0 = gi * lay.ldG;
-            p.a_y0 = 0;
-            p.b_x0 = sb1;
-            p.b_y0 = sb0;
-            const int box = p.L % 64 == 0 ? 64 : 16;
-            if ((s = launch_update_tc(maps[box == 64][gi], p, box, st)) != GPTQ_OK) return s;
+    } else {
+        const int cta = form == 0 ? SW_T : 128;
+        const int per_cta = form == 0 ? SW_T : form == 1 ? 32 : 64;
+        const dim3 grid((per_group + per_cta - 1) / per_cta, groups);
+        SweepKernel kern = sweep_kernel(form, gptaq, gmode, cae != 0);
+        const size_t smem = form == 0 ? sweep_thread_smem(gptaq, gmode, cae != 0)
+                                      : sweep_lanes_smem(gptaq, gmode, form == 1 ? 4 : 2);
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+            return launch_status();
+        const int vec = ((K % 4 == 0 && aligned(U, 16) && (!gptaq || aligned(P1, 16))) ? 1 : 0) |
+                        ((K % 16 == 0 && aligned(cp, 16)) ? 2 : 0);
+        SweepGroups sg{G, gsc, ng, gsel};
+        for (int sb0 = 0; sb0 < K; sb0 += SUPER) {
+            const int sb1 = min(K, sb0 + SUPER);
+            for (int i0 = sb0; i0 < sb1; i0 += blocksize) {
+                const int i1 = min(i0 + blocksize, sb1);
+                const int bs = i1 - i0;
+                const int rec = prof_begin(GPTQ_PROF_SWEEP, st);
+                kern<<<grid, cta, smem, st>>>(Wk, N, per_group, K, i0, bs, U, P1, scale, bits, cp, Eh,
+                                              El, Ph, Pl, lay.ldE, lay.ldG, i0 - sb0, loss_acc, vec,
+                                              status, sg, W0k);
+                s = launch_status();
+                prof_end(rec, st);
+                if (s != GPTQ_OK) return s;
+                if (i1 >= sb1) continue;
+                for (int gi = 0; gi < groups; ++gi) {      // near: the rest of the super-block
+                    UpdateParams p = base;
+                    p.C = Wk + (int64_t)gi * per_group * K + i1;
+                    p.Ncols = sb1 - i1;
+                    p.L = bs;
+                    p.a_x0 = gi * lay.ldG;
+                    p.a_y0 = i0 - sb0;
+                    p.b_x0 = i1;
+                    p.b_y0 = i0;
+                    const int box = p.L % 64 == 0 ? 64 : 16;
+                    if ((s = launch_update_tc(maps[box == 64][gi], p, box, st)) != GPTQ_OK) return s;
+                }
+            }
+            if (sb1 >= K) break;
+            for (int gi = 0; gi < groups; ++gi) {          // far: everything after the super-block
+                UpdateParams p = base;
+                p.C = Wk + (int64_t)gi * per_group * K + sb1;
+                p.Ncols = K - sb1;
+                p.L = sb1 - sb0;
+                p.a_x0 = gi * lay.ldG;
+                p.a_y0 = 0;
+                p.b_x0 = sb1;
+                p.b_y0 = sb0;
+                const int box = p.L % 64 == 0 ? 64 : 16;
+                if ((s = launch_update_tc(maps[box == 64][gi], p, box, st)) != GPTQ_OK) return s;
+            }
         }
     }
     if (grouped) {

@@ -299,8 +299,11 @@ template <int BK, bool TMA_EPI>
 static gptq_status launch_update(const UpdateMaps &maps, const CUtensorMap &cmap,
                                  const UpdateParams &p, int grid, cudaStream_t st) {
     cudaFuncSetAttribute(k_update_tc<BK, TMA_EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, UT_SMEM);
+    const int rec = prof_begin(GPTQ_PROF_UPDATE, st);
     k_update_tc<BK, TMA_EPI><<<grid, UT_THREADS, UT_SMEM, st>>>(maps, cmap, p);
-    return launch_status();
+    const gptq_status s = launch_status();
+    prof_end(rec, st);
+    return s;
 }
 
 // box_rows of the maps must equal the kernel's BK: 64 when L % 64 == 0, else 16.

@@ -86,6 +86,16 @@ def test_host_argument_checks(lib):
     assert lib.gptq_quantize_layer_grouped(fake, 0, 8, 16, fake, 4, 128, 32, 0, None, None, 3,
                                            None, None, None, fake, None, 0, ws, 1 << 30, fake,
                                            None) == gq.GPTQ_ERR_ARG
+    # timing diagnostics: an empty window reads zero; bad kinds and chain lengths refused
+    assert lib.gptq_profile_enable(1) == gq.GPTQ_OK
+    ms, cnt = ctypes.c_double(-1.0), ctypes.c_int(-1)
+    assert lib.gptq_profile_read(gq.GPTQ_PROF_UPDATE, ctypes.byref(ms), ctypes.byref(cnt)) == gq.GPTQ_OK
+    assert ms.value == 0.0 and cnt.value == 0
+    assert lib.gptq_profile_read(4, ctypes.byref(ms), ctypes.byref(cnt)) == gq.GPTQ_ERR_ARG
+    assert lib.gptq_profile_read(0, None, ctypes.byref(cnt)) == gq.GPTQ_ERR_ARG
+    assert lib.gptq_profile_enable(0) == gq.GPTQ_OK
+    assert lib.gptq_chain_latency(fake, 12, None) == gq.GPTQ_ERR_ARG
+    assert lib.gptq_chain_latency(None, 64, None) == gq.GPTQ_ERR_ARG
     # pack / unpack: bits, strides, NULL pointers; N == 0 does nothing
     assert lib.gptq_pack_codes(fake, 4, 64, 64, 5, fake, 64, None) == gq.GPTQ_ERR_ARG
     assert lib.gptq_pack_codes(fake, 4, 64, 63, 4, fake, 8, None) == gq.GPTQ_ERR_ARG
@@ -283,6 +293,9 @@ def test_every_wrapper_matches_its_c_signature(lib, monkeypatch):
     gq.gptq_first_order_shift(W, H, W, 0.5, gamma=torch.zeros(1, dtype=torch.float64),
                               status=st)
     gq.gptq_selftest_timeout(status=st)
+    gq.gptq_chain_latency(torch.zeros(3), steps=64)
+    gq.gptq_profile_enable(True)
+    gq.gptq_profile_read(gq.GPTQ_PROF_SWEEP)
     assert set(calls) == set(gq.EXPORTS) - {"gptq_trust_region_beta", "gptq_workspace_size",
                                             "gptq_kernel_launches", "gptq_status_string"}
     # the workspace sizes passed are the ones the library asks for

@@ -118,9 +118,10 @@ def test_ragged_bf16(K, N, M, B, bits):
     _full_check(wl, chunks, synth.weights(wl), label=f"ragged {K}x{N}")
 
 
-@pytest.mark.parametrize("form", ["0", "1", "2"])
+@pytest.mark.parametrize("form", ["0", "1", "2", "3"])
 def test_every_sweep_form(form, monkeypatch):
-    # one thread, four lanes or two lanes per channel: each form on its own, on ragged
+    # one thread, four lanes or two lanes per channel, or the tensor-core sweep (one
+    # launch per super-block, near updates in TMEM): each form on its own, on ragged
     # blocks, plain and GPTAQ
     monkeypatch.setenv("GPTQ_SWEEP_FORM", form)
     wl = synth.WORKLOADS["mlp_up"].scaled(K=392, N=200, M=2000, blocksize=128, bits=3,
