@@ -933,6 +933,19 @@ static gptq_status quantize_impl(void *W, int wdtype, int N, int K, const float 
                                 st)) != GPTQ_OK)
             return s;
         const int S = sweep_tc_super(gptaq);
+        // the far update reads the sweep's -E (and V) pairs as channel rows with the
+        // super-block's coordinates contiguous ([ldE][512], 64 x 128 boxes) and adds
+        static thread_local UpdateMaps kmaps[8];
+        for (int gi = 0; gi < groups; ++gi) {
+            kmaps[gi] = maps[1][gi];
+            __nv_bfloat16 *a_src[4] = {Eh, El, Ph, Pl};
+            for (int i = 0; i < 4; ++i)
+                if ((s = make_bf16_map(&kmaps[gi].a[i], a_src[i], SUPER, lay.ldE, SUPER, 128)) != GPTQ_OK)
+                    return s;
+        }
+        UpdateParams kbase = base;
+        kbase.a_kmajor = 1;
+        kbase.neg[0] = 0;
         for (int sb0 = 0; sb0 < K; sb0 += S) {
             const int sb1 = min(K, sb0 + S);
             if ((s = sweep_tc_launch(*stc, scale, bits, cp, Eh, El, Ph, Pl, lay.ldE, lay.ldG,
@@ -941,7 +954,7 @@ static gptq_status quantize_impl(void *W, int wdtype, int N, int K, const float 
                 return s;
             if (sb1 >= K) break;
             for (int gi = 0; gi < groups; ++gi) {      // far: everything after the super-block
-                UpdateParams p = base;
+                UpdateParams p = kbase;
                 p.C = Wk + (int64_t)gi * per_group * K + sb1;
                 p.Ncols = K - sb1;
                 p.L = sb1 - sb0;
@@ -949,8 +962,7 @@ static gptq_status quantize_impl(void *W, int wdtype, int N, int K, const float 
                 p.a_y0 = 0;
                 p.b_x0 = sb1;
                 p.b_y0 = sb0;
-                const int box = p.L % 64 == 0 ? 64 : 16;
-                if ((s = launch_update_tc(maps[box == 64][gi], p, box, st)) != GPTQ_OK) return s;
+                if ((s = launch_update_tc(kmaps[gi], p, 64, st)) != GPTQ_OK) return s;
             }
         }
     } else {

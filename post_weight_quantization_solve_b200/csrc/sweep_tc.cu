@@ -15,17 +15,19 @@
 //     lane's 32 columns (tcgen05.ld) and adds them to the weights staged from global
 //     memory, which hold every earlier super-block's far update.
 // The coordinates after the super-block are updated afterwards by the far update
-// (update_tc.cu) from the E (and V) pairs this kernel writes to global memory.
+// (update_tc.cu) from the -E (and V) pairs this kernel writes to global memory, one
+// row per channel with the super-block's coordinates contiguous ([ldE][512]).
 //
 // Products are bf16 x3 splits (hi*hi + hi*lo + lo*hi) of fp32 operands, as in the far
 // update. Operands: A = [-E | V] per channel row, K-major in a 128-byte swizzled tile
 // written by the chain threads; B = rows of U (and P1) as bf16 pairs, MN-major 64-column
 // chunks loaded by TMA. D starts at zero at phase 0 and is summed over the phases.
 //
-// Roles: warps 0-3 run the chain (thread = channel = TMEM lane); thread 0 also issues
-// the MMAs; warp 4 issues the TMA loads (weights, U's diagonal block and 1 / U_jj
-// one phase ahead into double-buffered slots; the B tile once the previous phase's
-// products are done). Every wait is bounded; a timeout sets the status word.
+// Roles: warps 0-3 run the chain (thread = channel = TMEM lane); warp 4 issues the TMA
+// loads (weights, U's diagonal block and 1 / U_jj one phase ahead into double-buffered
+// slots; the B tile once the previous phase's products are done); warp 5 issues the
+// MMAs, so that no chain warp waits for their issue. Every wait is bounded; a timeout
+// sets the status word.
 #include <cuda.h>
 
 #include <algorithm>
@@ -39,13 +41,14 @@ namespace gptq {
 
 namespace {
 constexpr int STC_CH = 128;                 // channels per CTA = TMEM lanes = MMA M
-constexpr int STC_THREADS = 160;            // 4 chain warps + the producer warp
+constexpr int STC_THREADS = 192;            // 4 chain warps, the producer warp, the MMA warp
 constexpr uint32_t STC_TMEM_COLS = 512;
 constexpr int A_TILE = 128 * 128;           // 128 rows x 128 bytes (64 bf16 of k)
 constexpr int B_SPLIT = 32 * 1024;          // one split (hi or lo) of the B tile
 constexpr int W_SLOT = 128 * 128;           // 128 rows x 32 fp32
 constexpr int D_SLOT = 32 * 128;            // 32 x 32 fp32 diagonal block
 constexpr int R_SLOT = 1024;                // 32 fp32 (1 / U_jj), 1 KB aligned slot
+constexpr int ESTRIDE = 512;                // row pitch of the E / V pairs in global memory
 constexpr int OFF_A = 0;                                  // [2 slots][hi, lo]
 constexpr int OFF_B = OFF_A + 4 * A_TILE;                 // [hi, lo]
 constexpr int OFF_W = OFF_B + 2 * B_SPLIT;                // [2 slots]
@@ -177,6 +180,42 @@ __global__ void __launch_bounds__(STC_THREADS, 1)
                 if (nb > 0) tc::mbar_wait(bfull, (nb - 1) & 1, &never);
             }
         }
+    } else if (warp == 5) {
+        if (lane == 0) {
+            // the products of phase q once every chain thread wrote its A row and B landed
+            for (int q = 0; q < nmma; ++q) {
+                if (!tc::mbar_wait(abar, q & 1, abort)) break;
+                if (!tc::mbar_wait(bfull, q & 1, abort)) break;
+                tc::fence_after_sync();
+                const int xb = 64 * ((q + 1) / 2);
+                const int nch = (nend - xb + 63) / 64;
+                const uint32_t a0 = tc::smem_u32(smem + OFF_A + (q & 1) * 2 * A_TILE);
+                const uint32_t b0 = tc::smem_u32(smem + OFF_B);
+                // chunk groups: [0, 1) first (the next phase's columns), then <= 4 at a time
+                for (int c0 = 0; c0 < nch;) {
+                    const int cn = c0 == 0 ? 1 : min(4, nch - c0);
+                    const uint32_t idesc = tc::idesc_bf16_f32(128, 64 * cn, 0, 1, 0);
+                    const uint32_t d = tmem + xb + 64 * c0;
+                    const uint32_t bb = b0 + c0 * CH_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < KP / 16; ++kk) {
+                        const uint64_t ah = tc::desc_sw128(a0 + kk * 32, 16, 1024);
+                        const uint64_t al = tc::desc_sw128(a0 + A_TILE + kk * 32, 16, 1024);
+                        const uint64_t bh = tc::desc_sw128(bb + kk * 2048, CH_BYTES, 1024);
+                        const uint64_t bl = tc::desc_sw128(bb + B_SPLIT + kk * 2048, CH_BYTES, 1024);
+                        tc::mma_bf16(d, ah, bh, idesc, (q > 0 || kk > 0) ? 1u : 0u);
+                        tc::mma_bf16(d, ah, bl, idesc, 1u);
+                        tc::mma_bf16(d, al, bh, idesc, 1u);
+                    }
+                    if (c0 == 0) tc::mma_commit(bar_next);
+                    c0 += cn;
+                }
+                tc::mma_commit(bar_rest);
+            }
+            tc::mma_commit(drain);      // every product is done before TMEM is released
+            volatile int never = 0;
+            tc::mbar_wait(drain, 0, &never);
+        }
     } else {
         const int tid = threadIdx.x;                 // channel row 0..127
         const bool valid = cta_ch0 + tid < p.per_group;
@@ -187,7 +226,6 @@ __global__ void __launch_bounds__(STC_THREADS, 1)
         const float cmin = -zf, cmax = (float)((1 << p.bits) - 1) - zf;
         const int live_end = min(p.S, K - sb0);      // coordinates of this super-block
         const int64_t ecol = (int64_t)grp * p.ldG + cta_ch0 + tid;
-        const int ldE = p.ldE;
         uint8_t *crow = p.codes + n * K + sb0;
         const bool vcodes = valid && p.vcodes;
         const uint32_t arow = (uint32_t)tid * 128;   // this row in the A tiles
@@ -253,19 +291,40 @@ __global__ void __launch_bounds__(STC_THREADS, 1)
                 cw[(t >> 2) & 3] |= (uint32_t)(int)(cf + zf) << (8 * (t & 3));
                 ebuf[t & 7] = -ep;
                 if (GPTAQ) vbuf[t & 7] = vj;
-                // the rest of this phase's coordinates, from the pair holding t + 1
-                const float2 ne = make_float2(-ep, -ep);
-                const float2 vv = make_float2(vj, vj);
+                // the rest of this phase's coordinates. The next one first, alone: its FMA
+                // is the only update the next step's rounding waits for (with GPTAQ the row
+                // term goes in before it, since it does not depend on this step's error).
                 const uint8_t *urow = ud + t * 128;
                 const uint8_t *prow = pd + t * 128;
+                auto uval = [&](const uint8_t *row, int k) {
+                    return *reinterpret_cast<const float *>(row + (((k >> 2) ^ (t & 7)) << 4) + ((k & 3) << 2));
+                };
+                if (t + 1 < 32) {
+                    float &wn = ((t + 1) & 1) ? w[(t + 1) >> 1].y : w[(t + 1) >> 1].x;
+                    if (GPTAQ) wn = fmaf(vj, uval(prow, t + 1), wn);
+                    wn = fmaf(-ep, uval(urow, t + 1), wn);
+                }
+                if ((t & 1) && t + 2 < 32) {      // the other half of the next coordinate's pair
+                    float &wn2 = w[(t + 2) >> 1].y;
+                    if (GPTAQ) wn2 = fmaf(vj, uval(prow, t + 2), wn2);
+                    wn2 = fmaf(-ep, uval(urow, t + 2), wn2);
+                }
+                {
+                    const int p0 = (t & 1) ? (t >> 1) + 2 : (t >> 1) + 1;   // first whole pair
+                    const float2 ne = make_float2(-ep, -ep);
+                    const float2 vv = make_float2(vj, vj);
 #pragma unroll
-                for (int i = (t + 1) / 2; i < 16; ++i) {
-                    const int off = (((i >> 1) ^ (t & 7)) << 4) + ((i & 1) << 3);
-                    const float2 u = *reinterpret_cast<const float2 *>(urow + off);
-                    w[i] = ffma2(ne, u, w[i]);
-                    if (GPTAQ) {
-                        const float2 pp = *reinterpret_cast<const float2 *>(prow + off);
-                        w[i] = ffma2(vv, pp, w[i]);
+                    for (int c = p0 >> 1; c < 8; ++c) {
+                        const int off = (c ^ (t & 7)) << 4;
+                        const float4 u = *reinterpret_cast<const float4 *>(urow + off);
+                        float4 pq;
+                        if (GPTAQ) pq = *reinterpret_cast<const float4 *>(prow + off);
+                        if (2 * c >= p0) {
+                            if (GPTAQ) w[2 * c] = ffma2(vv, make_float2(pq.x, pq.y), w[2 * c]);
+                            w[2 * c] = ffma2(ne, make_float2(u.x, u.y), w[2 * c]);
+                        }
+                        if (GPTAQ) w[2 * c + 1] = ffma2(vv, make_float2(pq.z, pq.w), w[2 * c + 1]);
+                        w[2 * c + 1] = ffma2(ne, make_float2(u.z, u.w), w[2 * c + 1]);
                     }
                 }
                 if ((t & 7) == 7) {
@@ -284,17 +343,10 @@ __global__ void __launch_bounds__(STC_THREADS, 1)
                     }
                     *reinterpret_cast<uint4 *>(ahi + ((c ^ sw) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
                     *reinterpret_cast<uint4 *>(alo + ((c ^ sw) << 4)) = make_uint4(l[0], l[1], l[2], l[3]);
-                    if (valid) {
-                        // E rows hold +E: the negation of the tile's pair is exact
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const int jj = 32 * q + 8 * c + i;
-                            if (jj >= live_end) break;
-                            const uint32_t hw = h[i >> 1] >> (16 * (i & 1));
-                            const uint32_t lw = l[i >> 1] >> (16 * (i & 1));
-                            p.Eh[(int64_t)jj * ldE + ecol] = __ushort_as_bfloat16((unsigned short)(hw ^ 0x8000u));
-                            p.El[(int64_t)jj * ldE + ecol] = __ushort_as_bfloat16((unsigned short)(lw ^ 0x8000u));
-                        }
+                    if (valid) {      // the far update's copy: -E, this channel's row
+                        const int64_t eo = ecol * ESTRIDE + 32 * q + 8 * c;
+                        *reinterpret_cast<uint4 *>(p.Eh + eo) = make_uint4(h[0], h[1], h[2], h[3]);
+                        *reinterpret_cast<uint4 *>(p.El + eo) = make_uint4(l[0], l[1], l[2], l[3]);
                     }
                     if (GPTAQ) {
 #pragma unroll
@@ -309,15 +361,9 @@ __global__ void __launch_bounds__(STC_THREADS, 1)
                         *reinterpret_cast<uint4 *>(ahi + (((4 + c) ^ sw) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
                         *reinterpret_cast<uint4 *>(alo + (((4 + c) ^ sw) << 4)) = make_uint4(l[0], l[1], l[2], l[3]);
                         if (valid) {
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                const int jj = 32 * q + 8 * c + i;
-                                if (jj >= live_end) break;
-                                p.Ph[(int64_t)jj * ldE + ecol] =
-                                    __ushort_as_bfloat16((unsigned short)(h[i >> 1] >> (16 * (i & 1))));
-                                p.Pl[(int64_t)jj * ldE + ecol] =
-                                    __ushort_as_bfloat16((unsigned short)(l[i >> 1] >> (16 * (i & 1))));
-                            }
+                            const int64_t eo = ecol * ESTRIDE + 32 * q + 8 * c;
+                            *reinterpret_cast<uint4 *>(p.Ph + eo) = make_uint4(h[0], h[1], h[2], h[3]);
+                            *reinterpret_cast<uint4 *>(p.Pl + eo) = make_uint4(l[0], l[1], l[2], l[3]);
                         }
                     }
                 }
@@ -339,51 +385,12 @@ __global__ void __launch_bounds__(STC_THREADS, 1)
             tc::fence_async_shared();
             tc::fence_before_sync();
             tc::mbar_arrive(&cfree[slot]);
-            if (q < nmma) {
-                tc::mbar_arrive(abar);
-                if (tid == 0) {
-                    // bounded waits only: a chain thread that gave up never stalls the others
-                    if (!tc::mbar_wait(abar, q & 1, abort)) break;
-                    if (!tc::mbar_wait(bfull, q & 1, abort)) break;
-                    tc::fence_after_sync();
-                    const int xb = 64 * ((q + 1) / 2);
-                    const int nch = (nend - xb + 63) / 64;
-                    const uint32_t a0 = tc::smem_u32(smem + OFF_A + slot * 2 * A_TILE);
-                    const uint32_t b0 = tc::smem_u32(smem + OFF_B);
-                    // chunk groups: [0, 1) first (the next phase's columns), then <= 4 at a time
-                    for (int c0 = 0; c0 < nch;) {
-                        const int cn = c0 == 0 ? 1 : min(4, nch - c0);
-                        const uint32_t idesc = tc::idesc_bf16_f32(128, 64 * cn, 0, 1, 0);
-                        const uint32_t d = tmem + xb + 64 * c0;
-                        const uint32_t bb = b0 + c0 * CH_BYTES;
-#pragma unroll
-                        for (int kk = 0; kk < KP / 16; ++kk) {
-                            const uint64_t ah = tc::desc_sw128(a0 + kk * 32, 16, 1024);
-                            const uint64_t al = tc::desc_sw128(a0 + A_TILE + kk * 32, 16, 1024);
-                            const uint64_t bh = tc::desc_sw128(bb + kk * 2048, CH_BYTES, 1024);
-                            const uint64_t bl = tc::desc_sw128(bb + B_SPLIT + kk * 2048, CH_BYTES, 1024);
-                            tc::mma_bf16(d, ah, bh, idesc, (q > 0 || kk > 0) ? 1u : 0u);
-                            tc::mma_bf16(d, ah, bl, idesc, 1u);
-                            tc::mma_bf16(d, al, bh, idesc, 1u);
-                        }
-                        if (c0 == 0) tc::mma_commit(bar_next);
-                        c0 += cn;
-                    }
-                    tc::mma_commit(bar_rest);
-                }
-            }
+            if (q < nmma) tc::mbar_arrive(abar);
         }
         if (valid) p.loss_acc[n] += lacc;
     }
 
     __syncwarp();
-    __syncthreads();
-    // every product is done before TMEM is released
-    if (threadIdx.x == 0) {
-        tc::mma_commit(drain);
-        volatile int never = 0;
-        tc::mbar_wait(drain, 0, &never);
-    }
     tc::fence_before_sync();
     __syncthreads();
     if (*abort && threadIdx.x == 0) set_status(p.status, GPTQ_ERR_TIMEOUT);

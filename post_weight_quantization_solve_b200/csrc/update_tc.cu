@@ -39,7 +39,7 @@ constexpr int UT_THREADS = 192;
 constexpr uint32_t UT_TMEM_COLS = 512;                // two 256-column accumulators
 }  // namespace
 
-template <int BK, bool TMA_EPI>
+template <int BK, bool TMA_EPI, bool AK>
 __global__ void __launch_bounds__(UT_THREADS, 1)
     k_update_tc(const __grid_constant__ UpdateMaps maps, const __grid_constant__ CUtensorMap cmap,
                 const UpdateParams p) {
@@ -107,8 +107,12 @@ __global__ void __launch_bounds__(UT_THREADS, 1)
                         const CUtensorMap *bm = &maps.b[2 * g + h];
                         uint8_t *a = st + h * A_BYTES;
                         uint8_t *b = st + 2 * A_BYTES + h * B_BYTES;
-                        tc::tma_load_2d(a, am, &full[stage], a_x0 + row0, ay);
-                        tc::tma_load_2d(a + BOX, am, &full[stage], a_x0 + row0 + 64, ay);
+                        if (AK) {       // channel rows with j contiguous: one 64 x 128 box
+                            tc::tma_load_2d(a, am, &full[stage], ay, a_x0 + row0);
+                        } else {
+                            tc::tma_load_2d(a, am, &full[stage], a_x0 + row0, ay);
+                            tc::tma_load_2d(a + BOX, am, &full[stage], a_x0 + row0 + 64, ay);
+                        }
 #pragma unroll
                         for (int q = 0; q < 4; ++q)
                             tc::tma_load_2d(b + q * BOX, bm, &full[stage], b_x0 + col0 + 64 * q, by);
@@ -126,8 +130,8 @@ __global__ void __launch_bounds__(UT_THREADS, 1)
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            const uint32_t idesc_pos = tc::idesc_bf16_f32(UT_BM, UT_BN, 1, 1, 0);
-            const uint32_t idesc_neg = tc::idesc_bf16_f32(UT_BM, UT_BN, 1, 1, 1);
+            const uint32_t idesc_pos = tc::idesc_bf16_f32(UT_BM, UT_BN, AK ? 0 : 1, 1, 0);
+            const uint32_t idesc_neg = tc::idesc_bf16_f32(UT_BM, UT_BN, AK ? 0 : 1, 1, 1);
             const bool neg0 = p.neg[0] != 0, neg1 = p.neg[1] != 0;
             int stage = 0, n = 0, acc = 0;
             uint32_t phase = 0, acc_phase = 0;
@@ -144,8 +148,11 @@ __global__ void __launch_bounds__(UT_THREADS, 1)
                     const uint32_t idesc = (g ? neg1 : neg0) ? idesc_neg : idesc_pos;
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
-                        const uint64_t ah = tc::desc_sw128(s0 + kk * 2048, BOX, 1024);
-                        const uint64_t al = tc::desc_sw128(s0 + A_BYTES + kk * 2048, BOX, 1024);
+                        // A K-major: the k step is 32 bytes inside the 128-byte rows
+                        const uint64_t ah = AK ? tc::desc_sw128(s0 + kk * 32, 16, 1024)
+                                               : tc::desc_sw128(s0 + kk * 2048, BOX, 1024);
+                        const uint64_t al = AK ? tc::desc_sw128(s0 + A_BYTES + kk * 32, 16, 1024)
+                                               : tc::desc_sw128(s0 + A_BYTES + kk * 2048, BOX, 1024);
                         const uint64_t bh = tc::desc_sw128(s0 + 2 * A_BYTES + kk * 2048, BOX, 1024);
                         const uint64_t bl = tc::desc_sw128(s0 + 2 * A_BYTES + B_BYTES + kk * 2048, BOX, 1024);
                         tc::mma_bf16(d, ah, bh, idesc, (it > 0 || kk > 0) ? 1u : 0u);
@@ -295,12 +302,12 @@ static int update_sms() {
     return n > 0 ? n : 148;
 }
 
-template <int BK, bool TMA_EPI>
+template <int BK, bool TMA_EPI, bool AK>
 static gptq_status launch_update(const UpdateMaps &maps, const CUtensorMap &cmap,
                                  const UpdateParams &p, int grid, cudaStream_t st) {
-    cudaFuncSetAttribute(k_update_tc<BK, TMA_EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, UT_SMEM);
+    cudaFuncSetAttribute(k_update_tc<BK, TMA_EPI, AK>, cudaFuncAttributeMaxDynamicSharedMemorySize, UT_SMEM);
     const int rec = prof_begin(GPTQ_PROF_UPDATE, st);
-    k_update_tc<BK, TMA_EPI><<<grid, UT_THREADS, UT_SMEM, st>>>(maps, cmap, p);
+    k_update_tc<BK, TMA_EPI, AK><<<grid, UT_THREADS, UT_SMEM, st>>>(maps, cmap, p);
     const gptq_status s = launch_status();
     prof_end(rec, st);
     return s;
@@ -311,6 +318,7 @@ gptq_status launch_update_tc(const UpdateMaps &maps, const UpdateParams &p, int 
                              cudaStream_t st) {
     if (p.M <= 0 || p.Ncols <= 0 || p.L <= 0) return GPTQ_OK;
     if (p.L % box_rows != 0 || p.ngroups < 1 || p.ngroups > 2) return GPTQ_ERR_ARG;
+    if (p.a_kmajor && box_rows != 64) return GPTQ_ERR_ARG;
     const int tiles = ((p.M + UT_BM - 1) / UT_BM) * ((p.Ncols + UT_BN - 1) / UT_BN);
     const int grid = std::min(tiles, update_sms());
     // bulk reductions need a 16-byte aligned base and row pitch
@@ -318,11 +326,14 @@ gptq_status launch_update_tc(const UpdateMaps &maps, const UpdateParams &p, int 
     const bool tma_epi = (p.ldc % 4 == 0) && aligned(p.C, 16) &&
                          make_out_map(&cmap, p.C, p.Ncols, p.M, p.ldc) == GPTQ_OK;
     if (!tma_epi) memset(&cmap, 0, sizeof(cmap));
+    if (p.a_kmajor)
+        return tma_epi ? launch_update<64, true, true>(maps, cmap, p, grid, st)
+                       : launch_update<64, false, true>(maps, cmap, p, grid, st);
     if (box_rows == 64)
-        return tma_epi ? launch_update<64, true>(maps, cmap, p, grid, st)
-                       : launch_update<64, false>(maps, cmap, p, grid, st);
-    return tma_epi ? launch_update<16, true>(maps, cmap, p, grid, st)
-                   : launch_update<16, false>(maps, cmap, p, grid, st);
+        return tma_epi ? launch_update<64, true, false>(maps, cmap, p, grid, st)
+                       : launch_update<64, false, false>(maps, cmap, p, grid, st);
+    return tma_epi ? launch_update<16, true, false>(maps, cmap, p, grid, st)
+                   : launch_update<16, false, false>(maps, cmap, p, grid, st);
 }
 
 // x -> (hi, lo) with hi = bf16(x), lo = bf16(x - hi); rows x cols fp32 (ld_in) to bf16

@@ -11,7 +11,7 @@ namespace gptq {
 // Product group g uses A operands a[2g] (hi), a[2g+1] (lo) and B operands b[2g],
 // b[2g+1]: group 0 is E with U, group 1 (GPTAQ) the pre-rounding weights with P1.
 struct UpdateMaps {
-    CUtensorMap a[4];   // A operands: [rows j][n], bf16
+    CUtensorMap a[4];   // A operands: [rows j][n] bf16 (a_kmajor: [rows n][j], 64 x 128 boxes)
     CUtensorMap b[4];   // B operands: [rows j][k], bf16
 };
 
@@ -24,6 +24,7 @@ struct UpdateParams {
     int ngroups;            // 1, or 2 with the GPTAQ group
     int neg[2];             // subtract group g's product
     int vec4;               // C rows 16-byte aligned: float4 reductions
+    int a_kmajor;           // A stored with the channel index as rows (k contiguous); L % 64 == 0
     int32_t *status;
 };
 
