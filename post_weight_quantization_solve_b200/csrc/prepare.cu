@@ -34,6 +34,9 @@
 
 namespace gptq {
 
+gptq_status launch_chol_diag_blk(float *H, int K, int g, int j0, int nb, const float *diag_d,
+                                 float tol, int32_t *status, cudaStream_t st);
+
 __global__ void k_check_finite(const float *A, int64_t count, int32_t *status) {
     int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -759,11 +762,14 @@ gptq_status prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out, v
 
     const float tol = (float)K * FLT_EPSILON;
     const int chol_smem = (int)((2 * DG_N * DG_N + 3 * DG_N) * sizeof(float));
-    // two pivots per barrier (GPTQ_DIAG_PAIRS=0 selects one pivot per barrier)
-    const char *pairs_env = getenv("GPTQ_DIAG_PAIRS");
-    const bool diag_pairs = !(pairs_env && pairs_env[0] == '0');
-    cudaFuncSetAttribute(diag_pairs ? k_chol_diag2 : k_chol_diag,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, chol_smem);
+    // diagonal blocks: the blocked factor (16-pivot sub-blocks, diag_blk.cu) by default;
+    // GPTQ_DIAG=pairs or single selects the per-pivot kernels (two pivots or one per
+    // block barrier), kept for comparisons
+    const char *diag_env = getenv("GPTQ_DIAG");
+    const int diag_mode = !diag_env ? 0 : (diag_env[0] == 'p' ? 1 : diag_env[0] == 's' ? 2 : 0);
+    if (diag_mode > 0)
+        cudaFuncSetAttribute(diag_mode == 1 ? k_chol_diag2 : k_chol_diag,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, chol_smem);
     Blocks bk{K, (K + CH_NB - 1) / CH_NB};
     // lookahead on the tensor-core steps (a second stream runs the bulk trailing
     // updates); without it every step runs in order on the caller's stream
@@ -795,11 +801,15 @@ gptq_status prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out, v
                 if (cudaStreamWaitEvent(st, la->rest[gi][(t + 2) & 1], 0) != cudaSuccess)
                     return GPTQ_ERR_CUDA;
         const int rec = prof_begin(GPTQ_PROF_DIAG, st);
-        if (diag_pairs)
-            k_chol_diag2<<<g, DG_T, chol_smem, st>>>(H, K, j0, nb, diag_d, tol, status);
-        else
-            k_chol_diag<<<g, DG_T, chol_smem, st>>>(H, K, j0, nb, diag_d, tol, status);
-        s = launch_status();
+        if (diag_mode == 0) {
+            s = launch_chol_diag_blk(H, K, g, j0, nb, diag_d, tol, status, st);
+        } else {
+            if (diag_mode == 1)
+                k_chol_diag2<<<g, DG_T, chol_smem, st>>>(H, K, j0, nb, diag_d, tol, status);
+            else
+                k_chol_diag<<<g, DG_T, chol_smem, st>>>(H, K, j0, nb, diag_d, tol, status);
+            s = launch_status();
+        }
         prof_end(rec, st);
         if (s != GPTQ_OK) return s;
         if (j0 == 0) break;

@@ -282,3 +282,33 @@ def test_gram_cta_pair_matches_single_cta(K, M, monkeypatch):
         assert rel_max(H, ref) <= TOL_H
         assert np.abs(H - H.T).max() <= 1e-6 * np.abs(ref).max()
     assert rel_max(out["1"], out["0"]) <= 1e-6
+
+
+@pytest.mark.parametrize("form", ["blk", "pairs", "single"])
+@pytest.mark.parametrize("K,g", [(128, 1), (200, 1), (392, 2), (1000, 1)])
+def test_every_diagonal_factor_form(form, K, g, monkeypatch):
+    # the blocked diagonal factor (16-pivot sub-blocks) and the per-pivot kernels (two
+    # pivots or one per block barrier): U against the oracle's factor of the same damped
+    # H, with a short first block (K not a multiple of 128), two Hessians and a dead
+    # coordinate
+    monkeypatch.setenv("GPTQ_DIAG", form)
+    d = dev()
+    gen = torch.Generator(device=d).manual_seed(K + 7 * g)
+    Hs = []
+    for _ in range(g):
+        X = torch.randn(3 * K, K, device=d, generator=gen) @ (
+            torch.eye(K, device=d) + 0.3 * torch.randn(K, K, device=d, generator=gen) / K ** 0.5)
+        X[:, K // 3] = 0.0                       # a dead coordinate
+        Hs.append(2.0 * X.T @ X)
+    H = torch.stack(Hs) if g > 1 else Hs[0]
+    H_in = H.double().cpu().numpy().reshape(g, K, K)
+    U = H.clone()
+    st = gq.gptq_prepare(U, 0.01)
+    gq.raise_on_status(st, f"prepare {form}")
+    torch.cuda.synchronize()
+    U_gpu = U.double().cpu().numpy().reshape(g, K, K)
+    for gi in range(g):
+        Hd, dead = O.dead_and_damp(H_in[gi], 0.01)
+        assert dead[K // 3]
+        assert rel_max(U_gpu[gi], O.upper_factor(Hd)) <= TOL_U, (form, gi)
+        assert np.all(np.tril(U_gpu[gi], -1) == 0.0)
