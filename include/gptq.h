@@ -57,7 +57,9 @@ typedef enum {
     GPTQ_ERR_NONFINITE = 3,  /* NaN or Inf in an input or an intermediate */
     GPTQ_ERR_CUDA = 4,       /* a CUDA launch or API call failed */
     GPTQ_ERR_TIMEOUT = 5,    /* a bounded device wait ran out */
-    GPTQ_ERR_WORKSPACE = 6   /* workspace missing, misaligned or too small */
+    GPTQ_ERR_WORKSPACE = 6,  /* workspace missing, misaligned or too small */
+    GPTQ_ERR_BOUNDS = 7      /* an index check of the GPTQ_DEBUG_BOUNDS build failed (the
+                                access was skipped); see gptq_bounds_report */
 } gptq_status;
 
 typedef enum { GPTQ_BF16 = 0, GPTQ_F32 = 1 } gptq_dtype;
@@ -413,11 +415,59 @@ typedef enum {
     GPTQ_PROF_UPDATE = 1,    /* tensor-core lazy (near / far) updates */
     GPTQ_PROF_DIAG = 2,      /* diagonal-block factor of gptq_prepare */
     GPTQ_PROF_TC32 = 3,      /* tf32 x3 tensor-core products (factor, inverse, residual, shift) */
-    GPTQ_PROF_KINDS = 4
+    GPTQ_PROF_SPLIT = 4,     /* splits of fp32 operands into tf32 / bf16 pairs */
+    GPTQ_PROF_KINDS = 5
 } gptq_prof_kind;
 
 GPTQ_API gptq_status gptq_profile_enable(int on);
 GPTQ_API gptq_status gptq_profile_read(int kind, double *ms, int *launches);
+
+/*
+ * gptq_profile_timeline -- the window's records in launch order: for record i,
+ * kind[i] (a gptq_prof_kind), lane[i] (the stream it ran on, numbered 0, 1, ... in
+ * order of first appearance in the window) and its begin and end times in ms from
+ * the first record's begin event. At most `max` records are written (all arrays
+ * host, `max` entries); *count receives the number of records in the window, which
+ * may exceed `max`. Synchronises the window's events. GPTQ_ERR_ARG on a NULL pointer
+ * or max < 0.
+ */
+GPTQ_API gptq_status gptq_profile_timeline(int max, int *kind, int *lane, double *begin_ms,
+                                           double *end_ms, int *count);
+
+/*
+ * gptq_bounds_report -- records of the index-check build (a debugging aid standing in
+ * for a memory checker; the pages have no counterpart).
+ *
+ * The library built with GPTQ_DEBUG_BOUNDS (libgptq_dbg.so; python -m
+ * post_weight_quantization_solve_b200.build --debug-bounds) checks, in its kernels,
+ * tile origins against the product or block they belong to, TMA box coordinates
+ * against their tensor and the 16-byte rule on the innermost coordinate, and computed
+ * output offsets against the output's extent. A failed check skips the access (never
+ * a trap), counts the failure and stores GPTQ_ERR_BOUNDS in the call's status word.
+ *
+ *   enabled  host int: 1 in the checking build, 0 otherwise (then the rest is zero).
+ *   count    host int: failed checks since the last reset.
+ *   site     host int: the first failure's site: 1 self-test, 2 tf32x3 GEMM tile,
+ *            3 tf32x3 GEMM TMA coordinate, 4 tf32x3 GEMM output element, 5 tf32x3
+ *            GEMM pair element, 6 Gram load box, 7 Gram reduction box, 8 sweep load
+ *            box, 9 sweep output offset, 10 lazy-update load box, 11 lazy-update
+ *            output element, 12 diagonal block; 0 when count is 0.
+ *   index    host int64: the first failure's offset or coordinate.
+ *   reset    non-zero: clear the records after reading them.
+ * Synchronises the device (reads device records). GPTQ_ERR_ARG on a NULL pointer,
+ * GPTQ_ERR_CUDA when a record cannot be read.
+ */
+GPTQ_API gptq_status gptq_bounds_report(int *enabled, int *count, int *site, int64_t *index,
+                                        int reset);
+
+/*
+ * gptq_bounds_selftest -- checking build only: one thread runs one check that always
+ * fails (site 1; no memory is accessed), so that a test sees the record and the
+ * status word change. Other builds return GPTQ_ERR_ARG and enqueue nothing.
+ *
+ *   status  device int32 (required): receives GPTQ_ERR_BOUNDS.
+ */
+GPTQ_API gptq_status gptq_bounds_selftest(int32_t *status, void *stream);
 
 /*
  * gptq_chain_latency -- one thread runs `steps` steps (a multiple of 8, >= 8) of the

@@ -14,15 +14,17 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libgptq.so")
+# GPTQ_LIBRARY selects another build of the library (the index-checking
+# libgptq_dbg.so of `build --debug-bounds`); by default the package's libgptq.so
+LIB_PATH = os.environ.get("GPTQ_LIBRARY") or os.path.join(_HERE, "libgptq.so")
 
 GPTQ_OK, GPTQ_ERR_ARG, GPTQ_ERR_NOT_PD, GPTQ_ERR_NONFINITE = 0, 1, 2, 3
-GPTQ_ERR_CUDA, GPTQ_ERR_TIMEOUT, GPTQ_ERR_WORKSPACE = 4, 5, 6
+GPTQ_ERR_CUDA, GPTQ_ERR_TIMEOUT, GPTQ_ERR_WORKSPACE, GPTQ_ERR_BOUNDS = 4, 5, 6, 7
 GPTQ_BF16, GPTQ_F32 = 0, 1
 GPTQ_OP_PREPARE, GPTQ_OP_RESIDUAL, GPTQ_OP_QUANTIZE, GPTQ_OP_QUANTIZE_GROUPED = 0, 1, 2, 3
 GPTQ_OP_FIRST_ORDER = 4
 GPTQ_WS_CAE = 0x100
-GPTQ_PROF_SWEEP, GPTQ_PROF_UPDATE, GPTQ_PROF_DIAG, GPTQ_PROF_TC32 = 0, 1, 2, 3
+GPTQ_PROF_SWEEP, GPTQ_PROF_UPDATE, GPTQ_PROF_DIAG, GPTQ_PROF_TC32, GPTQ_PROF_SPLIT = 0, 1, 2, 3, 4
 
 EXPORTS = ("gptq_accumulate_hessian", "gptaq_accumulate_cross", "gptq_prepare",
            "gptq_prepare_noalloc",
@@ -31,7 +33,8 @@ EXPORTS = ("gptq_accumulate_hessian", "gptaq_accumulate_cross", "gptq_prepare",
            "gptq_first_order_shift", "gptq_trust_region_beta", "gptq_selftest_timeout",
            "gptq_workspace_size",
            "gptq_kernel_launches", "gptq_status_string", "gptq_profile_enable",
-           "gptq_profile_read", "gptq_chain_latency")
+           "gptq_profile_read", "gptq_profile_timeline", "gptq_chain_latency",
+           "gptq_bounds_report", "gptq_bounds_selftest")
 
 _lib = None
 
@@ -73,6 +76,12 @@ def load_library():
         "gptq_kernel_launches": [],
         "gptq_profile_enable": [I],
         "gptq_profile_read": [I, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)],
+        "gptq_bounds_report": [ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int),
+                               ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int64), I],
+        "gptq_bounds_selftest": [P, P],
+        "gptq_profile_timeline": [I, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int),
+                                  ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double),
+                                  ctypes.POINTER(ctypes.c_int)],
         "gptq_chain_latency": [P, I, P],
     }
     for name, args in sig.items():
@@ -404,6 +413,19 @@ def gptq_profile_read(kind):
     return ms.value, n.value
 
 
+def gptq_profile_timeline(max_records=4096):
+    """The timing window's records in launch order: a list of (kind, lane, begin_ms,
+    end_ms), lane numbering the streams in order of first use, times from the first
+    record's begin (see include/gptq.h)."""
+    n = max(0, int(max_records))
+    kind, lane = (ctypes.c_int * max(n, 1))(), (ctypes.c_int * max(n, 1))()
+    t0, t1 = (ctypes.c_double * max(n, 1))(), (ctypes.c_double * max(n, 1))()
+    count = ctypes.c_int(0)
+    _check(load_library().gptq_profile_timeline(n, kind, lane, t0, t1, ctypes.byref(count)),
+           "gptq_profile_timeline")
+    return [(kind[i], lane[i], t0[i], t1[i]) for i in range(min(n, count.value))]
+
+
 def gptq_chain_latency(out, steps=65536, stream=None):
     """One thread times `steps` steps of the sweep's dependent chain: out (3 float32 on
     the device) receives SM cycles per step, ns per step and a keep-alive value. Returns
@@ -415,6 +437,30 @@ def gptq_chain_latency(out, steps=65536, stream=None):
         code = lib.gptq_chain_latency(*args)
     _check(code, "gptq_chain_latency")
     return out
+
+
+def gptq_bounds_report(reset=False):
+    """Records of the index-checking build: (enabled, failed checks, first site, first
+    index); enabled is False for the normal build (see include/gptq.h)."""
+    en, cnt, site = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    idx = ctypes.c_int64(0)
+    _check(load_library().gptq_bounds_report(ctypes.byref(en), ctypes.byref(cnt), ctypes.byref(site),
+                                             ctypes.byref(idx), 1 if reset else 0),
+           "gptq_bounds_report")
+    return bool(en.value), cnt.value, site.value, idx.value
+
+
+def gptq_bounds_selftest(status=None, stream=None):
+    """Index-checking build only: one check that always fails (no access), so the
+    returned status word ends up holding GPTQ_ERR_BOUNDS."""
+    lib = load_library()
+    dev = status.device if status is not None else torch.device("cuda", torch.cuda.current_device())
+    status = new_status(dev) if status is None else status
+    args = (_ptr(status, dev, "status"), _stream(stream, dev))
+    with torch.cuda.device(dev):
+        code = lib.gptq_bounds_selftest(*args)
+    _check(code, "gptq_bounds_selftest")
+    return status
 
 
 def gptq_selftest_timeout(status=None, stream=None):

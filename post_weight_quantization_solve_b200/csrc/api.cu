@@ -4,6 +4,10 @@
 
 #include <cmath>
 
+#include <mutex>
+#include <vector>
+
+#include "bounds.cuh"
 #include "common.cuh"
 #include "tc_ptx.cuh"
 
@@ -78,6 +82,27 @@ __global__ void k_selftest_timeout(int32_t *status) {
     __syncthreads();
     if (threadIdx.x == 0 && !tc::mbar_wait(&bar, 0, &abort_flag)) set_status(status, GPTQ_ERR_TIMEOUT);
 }
+
+#ifdef GPTQ_DEBUG_BOUNDS
+// Readers of the translation units' check records, registered at load time.
+static std::mutex &bounds_mu() {
+    static std::mutex mu;
+    return mu;
+}
+static std::vector<BoundsReader> &bounds_readers() {
+    static std::vector<BoundsReader> v;
+    return v;
+}
+void gptq::bounds_register(BoundsReader fn) {
+    std::lock_guard<std::mutex> lock(bounds_mu());
+    bounds_readers().push_back(fn);
+}
+
+// One check that always fails; no memory is accessed.
+__global__ void k_bounds_selftest(int32_t *status, int never) {
+    if (threadIdx.x == 0) (void)GQ_IN_BOUNDS(status, never != 0, BS_SELFTEST, -1);
+}
+#endif
 
 static bool stream_ok(int xdtype, const void *X, int64_t ldx, int K) {
     if (ldx < K) return false;
@@ -296,8 +321,48 @@ const char *gptq_status_string(int status) {
         case GPTQ_ERR_CUDA: return "CUDA launch or API error";
         case GPTQ_ERR_TIMEOUT: return "bounded device wait ran out";
         case GPTQ_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case GPTQ_ERR_BOUNDS: return "an index check failed (the access was skipped)";
         default: return "unknown status";
     }
+}
+
+gptq_status gptq_bounds_report(int *enabled, int *count, int *site, int64_t *index, int reset) {
+    if (!enabled || !count || !site || !index) return GPTQ_ERR_ARG;
+    *enabled = 0;
+    *count = 0;
+    *site = 0;
+    *index = 0;
+#ifdef GPTQ_DEBUG_BOUNDS
+    *enabled = 1;
+    if (cudaDeviceSynchronize() != cudaSuccess) {
+        cudaGetLastError();
+        return GPTQ_ERR_CUDA;
+    }
+    std::lock_guard<std::mutex> lock(bounds_mu());
+    for (BoundsReader fn : bounds_readers()) {
+        BoundsRecord r{0, 0, 0};
+        if (!fn(&r, reset != 0)) return GPTQ_ERR_CUDA;
+        if (r.count > 0 && *count == 0) {
+            *site = r.site;
+            *index = r.index;
+        }
+        *count += r.count;
+    }
+#else
+    (void)reset;
+#endif
+    return GPTQ_OK;
+}
+
+gptq_status gptq_bounds_selftest(int32_t *status, void *stream) {
+    if (!status) return GPTQ_ERR_ARG;
+#ifdef GPTQ_DEBUG_BOUNDS
+    k_bounds_selftest<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(status, 0);
+    return launch_status();
+#else
+    (void)stream;
+    return GPTQ_ERR_ARG;
+#endif
 }
 
 }  // extern "C"

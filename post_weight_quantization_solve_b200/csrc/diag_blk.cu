@@ -24,6 +24,7 @@
 // refuse a pivot p_j <= tol * Hd_jj.
 #include <float.h>
 
+#include "bounds.cuh"
 #include "common.cuh"
 
 namespace gptq {
@@ -54,7 +55,12 @@ __global__ void __launch_bounds__(DB_T, 1) k_chol_diag_blk(float *H, int K, int 
     __shared__ __align__(16) float rowb[32 * DB_SB];   // pivot rows of S (0-15) and V (16-31)
     const int tid = threadIdx.x;
     // one reading of the status word for the whole CTA
-    if (tid == 0) *skip = failed(status) ? 1 : 0;
+    if (tid == 0) {
+        *skip = failed(status) ? 1 : 0;
+        // the block lies inside H (nothing of it is read or written otherwise)
+        if (!GQ_IN_BOUNDS(status, j0 >= 0 && nb >= 1 && nb <= DB_N && j0 + nb <= K, BS_DIAG, j0))
+            *skip = 1;
+    }
     __syncthreads();
     if (*skip) return;
     const int g = blockIdx.x;

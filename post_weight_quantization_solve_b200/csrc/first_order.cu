@@ -84,6 +84,7 @@ static gptq_status first_order_tc(float *W, int N, int K, const float *U, const 
     if (cudaMemsetAsync(T, 0, sizeof(float) * (size_t)NK, st) != cudaSuccess) return GPTQ_ERR_CUDA;
     p = Tc32Params{};
     p.C = T; p.alpha = 1.f; p.accumulate = 1; p.b_lower = 1; p.status = status;
+    p.c_extent = NK;
     p.nitems = 1;
     p.item[0].m = N; p.item[0].n = K; p.item[0].k = K;
     p.item[0].c_off = 0; p.item[0].ldc = K;
@@ -99,6 +100,7 @@ static gptq_status first_order_tc(float *W, int N, int K, const float *U, const 
     if ((s = make_f32_map(&m[3], Vl, K, K, K, 32, 128)) != GPTQ_OK) return s;
     p = Tc32Params{};
     p.C = W; p.alpha = -beta; p.accumulate = 1; p.b_upper = 1; p.status = status;
+    p.c_extent = NK;
     p.nitems = 1;
     p.item[0].m = N; p.item[0].n = K; p.item[0].k = K;
     p.item[0].c_off = 0; p.item[0].ldc = K;

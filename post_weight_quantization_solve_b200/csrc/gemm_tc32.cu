@@ -21,6 +21,7 @@
 #include <algorithm>
 #include <vector>
 
+#include "bounds.cuh"
 #include "common.cuh"
 #include "gemm_tc32.cuh"
 #include "tc_ptx.cuh"
@@ -57,7 +58,7 @@ __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64
 // bank; reading it through a reference inside loops that store to global memory
 // makes every access a reload).
 struct G32Unit {
-    int i0, j0, k0, k1;
+    int i0, j0, k0, k1, kmax;
     int m, n, ldc, parts;
     int a_x0, a_y0, b_x0, b_y0;
     int64_t c_off;
@@ -82,9 +83,14 @@ __device__ __forceinline__ bool g32_unit(const Tc32Params &p, int u, G32Unit &w)
     const int steps = ke > kb ? (ke - kb) / G32_BK : 0;
     w.k0 = kb + (int)((int64_t)steps * part / I.parts) * G32_BK;
     w.k1 = kb + (int)((int64_t)steps * (part + 1) / I.parts) * G32_BK;
-    w.m = I.m; w.n = I.n; w.ldc = I.ldc; w.parts = I.parts;
+    w.m = I.m; w.n = I.n; w.ldc = I.ldc; w.parts = I.parts; w.kmax = I.k;
     w.a_x0 = I.a_x0; w.a_y0 = I.a_y0; w.b_x0 = I.b_x0; w.b_y0 = I.b_y0;
     w.c_off = I.c_off;
+    // every role decodes the same units, so a unit that fails is skipped by all three
+    if (!GQ_IN_BOUNDS(p.status, it < p.nitems && w.i0 < w.m && w.j0 < w.n && w.k0 >= 0 &&
+                                    w.k0 <= w.k1 && w.k1 <= w.kmax,
+                      BS_TC32_TILE, u))
+        return false;
     return !(p.upper_tiles && w.i0 > w.j0 + G32_BN - 1);
 }
 
@@ -135,6 +141,13 @@ __global__ void __launch_bounds__(G32_THREADS, 1)
                 G32Unit w;
                 if (!g32_unit(p, u, w)) continue;
                 for (int k = w.k0; k < w.k1; k += G32_BK) {
+                    // fp32 boxes: the innermost coordinate on a 16-byte boundary
+                    if (!GQ_IN_BOUNDS(p.status, ((w.a_x0 + k) & 3) == 0 && ((w.b_x0 + k) & 3) == 0 &&
+                                                    w.a_x0 + k >= 0 && w.b_x0 + k >= 0,
+                                      BS_TC32_TMA, w.a_x0 + k)) {
+                        *abort = 1;
+                        break;
+                    }
                     if (!tc::mbar_wait(&empty[stage], phase ^ 1, abort)) break;
                     tc::mbar_arrive_expect_tx(&full[stage], G32_STAGE);
                     uint8_t *st = smem + stage * G32_STAGE;
@@ -213,6 +226,11 @@ __global__ void __launch_bounds__(G32_THREADS, 1)
             const bool rvalid = row < w.m;
             float *crow = cbase + (int64_t)row * w.ldc;
             const bool v4 = ((w.ldc | (int)(w.c_off & 3)) & 3) == 0 && vec_c;
+            float *const phi = reduce ? nullptr : p.pair_hi;
+            float *const plo = p.pair_lo;
+            const int64_t pld = p.pair_ld;
+            const bool pv4 = phi && (pld & 3) == 0 &&
+                             ((reinterpret_cast<uintptr_t>(phi) | reinterpret_cast<uintptr_t>(plo)) & 15) == 0;
 #pragma unroll 1
             for (int c = 0; c < G32_BN / 32; ++c) {
                 uint32_t v[32];
@@ -220,6 +238,10 @@ __global__ void __launch_bounds__(G32_THREADS, 1)
                 tc::tmem_ld_wait();
                 const int col0 = w.j0 + c * 32;
                 if (!rvalid || col0 >= w.n) continue;
+                if (!GQ_IN_BOUNDS(p.status, p.c_extent == 0 || (w.c_off + (int64_t)row * w.ldc + col0 >= 0 &&
+                                                                w.c_off + (int64_t)row * w.ldc + min(col0 + 32, w.n) <= p.c_extent),
+                                  BS_TC32_C, w.c_off + (int64_t)row * w.ldc + col0))
+                    continue;
                 float x[32];
 #pragma unroll
                 for (int q = 0; q < 32; ++q) {
@@ -242,6 +264,35 @@ __global__ void __launch_bounds__(G32_THREADS, 1)
                         if (col0 + q >= w.n) break;
                         if (reduce) atomicAdd(crow + col0 + q, x[q]);
                         else crow[col0 + q] = x[q];
+                    }
+                }
+                if (phi && GQ_IN_BOUNDS(p.status, p.pair_extent == 0 || ((int64_t)row * pld + min(col0 + 32, w.n) <= p.pair_extent),
+                                        BS_TC32_PAIR, (int64_t)row * pld + col0)) {
+                    // the stored values' tf32 pairs, as split_tf32 forms them
+                    float *hrow = phi + (int64_t)row * pld + col0, *lrow = plo + (int64_t)row * pld + col0;
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) {
+                        uint32_t b;
+                        asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(b) : "f"(x[q]));
+                        v[q] = b;
+                        x[q] -= __uint_as_float(b);
+                    }
+                    if (pv4 && col0 + 32 <= w.n) {
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            reinterpret_cast<float4 *>(hrow)[q] =
+                                make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                            __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+                            reinterpret_cast<float4 *>(lrow)[q] =
+                                make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) {
+                            if (col0 + q >= w.n) break;
+                            hrow[q] = __uint_as_float(v[q]);
+                            lrow[q] = x[q];
+                        }
                     }
                 }
             }
@@ -319,13 +370,54 @@ __global__ void k_split_tf32(const float *__restrict__ in, int64_t ld_in, int co
     }
 }
 
+// The same split, four columns per thread (16-byte loads and stores), the matrix
+// flattened to rows x cols/4 units so that narrow column blocks still fill the grid;
+// batched over blockIdx.y.
+__global__ void k_split_tf32_v4(const float *__restrict__ in, int64_t ld_in, uint32_t c4,
+                                uint32_t units, float *__restrict__ hi, float *__restrict__ lo,
+                                int64_t ld_out, int64_t batch_in, int64_t batch_out) {
+    in += blockIdx.y * batch_in;
+    hi += blockIdx.y * batch_out;
+    lo += blockIdx.y * batch_out;
+    for (uint32_t u = blockIdx.x * blockDim.x + threadIdx.x; u < units; u += gridDim.x * blockDim.x) {
+        const uint32_t r = u / c4, c = (u - r * c4) * 4;
+        const float4 x = *reinterpret_cast<const float4 *>(in + r * ld_in + c);
+        float4 h, l;
+        uint32_t b;
+        asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(b) : "f"(x.x));
+        h.x = __uint_as_float(b);
+        asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(b) : "f"(x.y));
+        h.y = __uint_as_float(b);
+        asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(b) : "f"(x.z));
+        h.z = __uint_as_float(b);
+        asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(b) : "f"(x.w));
+        h.w = __uint_as_float(b);
+        l = make_float4(x.x - h.x, x.y - h.y, x.z - h.z, x.w - h.w);
+        *reinterpret_cast<float4 *>(hi + r * ld_out + c) = h;
+        *reinterpret_cast<float4 *>(lo + r * ld_out + c) = l;
+    }
+}
+
 gptq_status split_tf32(const float *in, int64_t ld_in, int rows, int cols, float *hi, float *lo,
                        int64_t ld_out, int batch, int64_t batch_in, int64_t batch_out,
                        cudaStream_t st) {
     if (rows <= 0 || cols <= 0) return GPTQ_OK;
-    const int bx = (int)std::min<int64_t>(8, (cols + 255) / 256);
-    k_split_tf32<<<dim3(bx, rows, batch), 256, 0, st>>>(in, ld_in, cols, hi, lo, ld_out, batch_in,
-                                                        batch_out);
+    const int rec = prof_begin(GPTQ_PROF_SPLIT, st);
+    const int64_t units = (int64_t)rows * (cols / 4);
+    const bool vec = cols % 4 == 0 && ld_in % 4 == 0 && ld_out % 4 == 0 && batch_in % 4 == 0 &&
+                     batch_out % 4 == 0 && aligned(in, 16) && aligned(hi, 16) && aligned(lo, 16) &&
+                     units < (int64_t)1 << 31 && batch <= 65535;
+    if (vec) {
+        const int bx = (int)std::min<int64_t>((units + 255) / 256, 148 * 8);
+        k_split_tf32_v4<<<dim3(bx, batch), 256, 0, st>>>(in, ld_in, (uint32_t)(cols / 4),
+                                                         (uint32_t)units, hi, lo, ld_out, batch_in,
+                                                         batch_out);
+    } else {
+        const int bx = (int)std::min<int64_t>(8, (cols + 255) / 256);
+        k_split_tf32<<<dim3(bx, rows, batch), 256, 0, st>>>(in, ld_in, cols, hi, lo, ld_out,
+                                                            batch_in, batch_out);
+    }
+    prof_end(rec, st);
     return launch_status();
 }
 
@@ -361,12 +453,14 @@ gptq_status split_tf32_t(const float *in, int64_t ld_in, int rows, int cols, flo
                          int64_t ld_out, int batch, int64_t batch_in, int64_t batch_out,
                          cudaStream_t st) {
     if (rows <= 0 || cols <= 0) return GPTQ_OK;
+    const int rec = prof_begin(GPTQ_PROF_SPLIT, st);
     k_split_tf32_t<<<dim3((cols + 31) / 32, (rows + 31) / 32, batch), dim3(32, 8), 0, st>>>(
         in, ld_in, rows, cols, hi, lo, ld_out, batch_in, batch_out);
+    prof_end(rec, st);
     return launch_status();
 }
 
-static int tc32_sms() {
+int tc32_sms() {
     int dev = 0, n = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -389,7 +483,9 @@ gptq_status launch_gemm_tc32(const CUtensorMap maps[4], Tc32Params &p, cudaStrea
     }
     p.units = units;
     if (units == 0) return GPTQ_OK;
-    const int grid = std::min(units, tc32_sms());
+    if (p.pair_hi && (p.nitems != 1 || p.accumulate || p.item[0].parts != 1 || !p.pair_lo))
+        return GPTQ_ERR_ARG;
+    const int grid = std::min(units, p.max_grid > 0 ? std::min(p.max_grid, tc32_sms()) : tc32_sms());
     cudaFuncSetAttribute(k_gemm_tc32, cudaFuncAttributeMaxDynamicSharedMemorySize, G32_SMEM);
     const int rec = prof_begin(GPTQ_PROF_TC32, st);
     k_gemm_tc32<<<grid, G32_THREADS, G32_SMEM, st>>>(maps[0], maps[1], maps[2], maps[3], p);

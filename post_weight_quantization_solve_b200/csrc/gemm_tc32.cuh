@@ -27,6 +27,14 @@ struct Tc32Params {
     int a_lower;            // A(i,k) == 0 for k > i: the k range ends at the row tile
     int b_lower;            // B(k,j) == 0 for k < j: the k range starts at the column tile
     int nitems, units;
+    int max_grid;           // > 0: at most this many CTAs (leaves SMs to other streams)
+    // Optional (one item, overwrite mode, unsplit inner range): the stored values also
+    // as tf32 pairs, element (i, j) of the item at pair_hi / pair_lo[i * pair_ld + j].
+    float *pair_hi, *pair_lo;
+    int64_t pair_ld;
+    // Elements addressable from C and from each pair array (0: not given); the
+    // index-checking build skips any store beyond them.
+    int64_t c_extent, pair_extent;
     int32_t *status;
     Tc32Item item[TC32_MAX_ITEMS];
 };
@@ -41,5 +49,6 @@ gptq_status split_tf32_t(const float *in, int64_t ld_in, int rows, int cols, flo
                          int64_t ld_out, int batch, int64_t batch_in, int64_t batch_out,
                          cudaStream_t st);
 gptq_status launch_gemm_tc32(const CUtensorMap maps[4], Tc32Params &p, cudaStream_t st);
+int tc32_sms();
 
 }  // namespace gptq

@@ -27,6 +27,7 @@
 #include <algorithm>
 #include <cstdlib>
 
+#include "bounds.cuh"
 #include "common.cuh"
 #include "tc_ptx.cuh"
 
@@ -122,6 +123,13 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
                 int ti, tj, k0, k1;
                 gt_unit(p, u, ti, tj, k0, k1);
                 for (int k = k0; k < k1; ++k) {
+                    // bf16 boxes: feature origins on 16-byte boundaries, token step inside the chunk
+                    if (!GQ_IN_BOUNDS(p.status, k >= 0 && k < p.S && ti >= 0 && tj >= 0 && ti * GT_BM < p.K &&
+                                                    tj * GT_BN < p.K && ((ti * GT_BM) & 7) == 0 && ((tj * GT_BN) & 7) == 0,
+                                      BS_GRAM_TMA, (long long)k * GT_BK)) {
+                        *abort = 1;
+                        break;
+                    }
                     if (!tc::mbar_wait(&empty[stage], phase ^ 1, abort)) break;
                     tc::mbar_arrive_expect_tx(&full[stage], GT_STAGE);
                     uint8_t *a = smem + stage * GT_STAGE;
@@ -192,7 +200,9 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
         auto stage_out = [&](int x, int y) {
             tc::fence_async_shared();
             __syncwarp();
-            if (lane == 0) {
+            // a reduction box starts inside H, its column on a 16-byte boundary
+            if (lane == 0 && GQ_IN_BOUNDS(p.status, x >= 0 && y >= 0 && x < p.K && y < p.K && (x & 3) == 0,
+                                          BS_GRAM_RED, (long long)y * p.K + x)) {
                 tc::tma_reduce_add_2d(&hmap, buf, x, y);
                 tc::bulk_commit();
                 tc::bulk_wait_read<0>();    // buf is free again
@@ -361,6 +371,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(G2_THREADS, 1)
                 const int ra = ti * 2 * G2_BM + (int)rank * G2_BM;   // this CTA's A rows
                 const int cb = tj * G2_BN + (int)rank * (G2_BN / 2);  // this CTA's B columns
                 for (int k = k0; k < k1; ++k) {
+                    if (!GQ_IN_BOUNDS(p.status, k >= 0 && k < p.S && ra >= 0 && cb >= 0 && ra < p.K + G2_BM &&
+                                                    cb < p.K + G2_BN && (ra & 7) == 0 && (cb & 7) == 0,
+                                      BS_GRAM_TMA, (long long)k * G2_BK)) {
+                        *abort = 1;
+                        break;
+                    }
                     if (!tc::mbar_wait(&empty[stage], phase ^ 1, abort)) break;
                     if (rank == 0) tc::mbar_arrive_expect_tx(&full[stage], 2 * G2_STAGE);
                     const uint32_t fb = tc::mapa_shared(tc::smem_u32(&full[stage]), 0);
@@ -440,7 +456,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(G2_THREADS, 1)
         auto stage_out = [&](int x, int y) {
             tc::fence_async_shared();
             __syncwarp();
-            if (lane == 0) {
+            if (lane == 0 && GQ_IN_BOUNDS(p.status, x >= 0 && y >= 0 && x < p.K && y < p.K && (x & 3) == 0,
+                                          BS_GRAM_RED, (long long)y * p.K + x)) {
                 tc::tma_reduce_add_2d(&hmap, buf, x, y);
                 tc::bulk_commit();
                 tc::bulk_wait_read<0>();

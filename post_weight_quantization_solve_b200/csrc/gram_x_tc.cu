@@ -25,6 +25,7 @@
 
 #include <algorithm>
 
+#include "bounds.cuh"
 #include "common.cuh"
 #include "tc_ptx.cuh"
 
@@ -131,6 +132,14 @@ __global__ void __launch_bounds__(GX_THREADS, 1)
                 int grp, ti, tj, k0, k1;
                 gx_unit(p, u, grp, ti, tj, k0, k1);
                 for (int k = k0; k < k1; ++k) {
+                    // bf16 boxes: feature origins on 16-byte boundaries, token step inside the chunk
+                    if (!GQ_IN_BOUNDS(p.status, grp >= 0 && grp < p.groups && k >= 0 && k < p.S && ti >= 0 &&
+                                                    tj >= 0 && ti * GX_BM < p.K && tj * GX_BN < p.K &&
+                                                    ((ti * GX_BM) & 7) == 0 && ((tj * GX_BN) & 7) == 0,
+                                      BS_GRAM_TMA, (long long)k * GX_BK)) {
+                        *abort = 1;
+                        break;
+                    }
                     if (!tc::mbar_wait(&empty[stage], phase ^ 1, abort)) break;
                     tc::mbar_arrive_expect_tx(&full[stage], src_bytes);
                     uint8_t *st = smem + stage * GX_STAGE;
@@ -260,7 +269,10 @@ __global__ void __launch_bounds__(GX_THREADS, 1)
         auto stage_out = [&](int x, int y) {
             tc::fence_async_shared();
             __syncwarp();
-            if (lane == 0) {
+            // a reduction box starts inside the stack of H_g, its column on a 16-byte boundary
+            if (lane == 0 && GQ_IN_BOUNDS(p.status, x >= 0 && y >= 0 && x < p.K && y < p.groups * p.K &&
+                                                        (x & 3) == 0,
+                                          BS_GRAM_RED, (long long)y * p.K + x)) {
                 tc::tma_reduce_add_2d(&hmap, buf, x, y);
                 tc::bulk_commit();
                 tc::bulk_wait_read<0>();    // buf is free again

@@ -531,9 +531,12 @@ static gptq_status chol_panel_strip_tc(float *H, int K, int j0, int j1, int j0n,
     pp.item[0].m = j0; pp.item[0].n = nb; pp.item[0].k = nb;
     pp.item[0].a_x0 = 0; pp.item[0].a_y0 = 0; pp.item[0].b_x0 = 0; pp.item[0].b_y0 = j0;
     pp.item[0].c_off = j0; pp.item[0].ldc = K;
+    // the epilogue also writes the tf32 pairs of the new panel R over the front rows
+    // (0..j0) of the block's pairs: each row tile is read (as A) and written by the
+    // same unit, and the U_JJ rows read as B lie behind them
+    pp.pair_hi = Ch; pp.pair_lo = Cl; pp.pair_ld = nb;
+    pp.c_extent = (int64_t)K * K; pp.pair_extent = (int64_t)j1 * nb;
     if ((s = launch_gemm_tc32(m, pp, st)) != GPTQ_OK) return s;
-    // pairs of the new panel R (rows 0..j0 of the block, overwriting the front)
-    if ((s = split_tf32(H + j0, K, j0, nb, Ch, Cl, nb, 1, 0, 0, st)) != GPTQ_OK) return s;
     // strip: every row above j0 against the rows of J' (entries below the diagonal of
     // H[J', J'] are updated too; nothing reads them)
     ps = Tc32Params{};
@@ -541,11 +544,12 @@ static gptq_status chol_panel_strip_tc(float *H, int K, int j0, int j1, int j0n,
     ps.item[0].m = j0; ps.item[0].n = j0 - j0n; ps.item[0].k = nb;
     ps.item[0].a_x0 = 0; ps.item[0].a_y0 = 0; ps.item[0].b_x0 = 0; ps.item[0].b_y0 = j0n;
     ps.item[0].c_off = j0n; ps.item[0].ldc = K;
+    ps.c_extent = (int64_t)K * K;
     return launch_gemm_tc32(m, ps, st);
 }
 
 static gptq_status chol_rest_tc(float *H, int K, int j0n, const CUtensorMap (&m)[4],
-                                int32_t *status, cudaStream_t st, int nb) {
+                                int32_t *status, cudaStream_t st, int nb, int max_grid) {
     if (j0n <= 0) return GPTQ_OK;
     static thread_local Tc32Params pr;
     pr = Tc32Params{};
@@ -553,6 +557,8 @@ static gptq_status chol_rest_tc(float *H, int K, int j0n, const CUtensorMap (&m)
     pr.nitems = 1;
     pr.item[0].m = j0n; pr.item[0].n = j0n; pr.item[0].k = nb;
     pr.item[0].c_off = 0; pr.item[0].ldc = K;
+    pr.max_grid = max_grid;
+    pr.c_extent = (int64_t)K * K;
     return launch_gemm_tc32(m, pr, st);
 }
 
@@ -705,6 +711,7 @@ static gptq_status tri_inverse_tc(float *H, int K, const Blocks &bk, float *Tt, 
         // T^T = (U_bb^T)(R_ab^T): A rows j of H^T at column m, B^T rows i of H at column m
         p1 = Tc32Params{};
         p1.C = Tt; p1.alpha = 1.f; p1.accumulate = 1; p1.a_lower = 1; p1.status = status;
+        p1.c_extent = (int64_t)trows * pitch;
         p1.nitems = (int)lv.size();
         for (size_t ni = 0; ni < lv.size(); ++ni) {
             const InvNode &nd = lv[ni];
@@ -724,6 +731,7 @@ static gptq_status tri_inverse_tc(float *H, int K, const Blocks &bk, float *Tt, 
         // U_ab = -U_aa T into zeroed blocks of H: A rows of H at column a, B^T rows of T^T
         p2 = Tc32Params{};
         p2.C = H; p2.alpha = -1.f; p2.accumulate = 1; p2.a_upper = 1; p2.status = status;
+        p2.c_extent = KK;
         p2.nitems = (int)lv.size();
         int maxm = 0, maxn = 0;
         for (size_t ni = 0; ni < lv.size(); ++ni) {
@@ -831,7 +839,8 @@ gptq_status prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out, v
                     if (cudaEventRecord(la->panel[gi][t & 1], st) != cudaSuccess ||
                         cudaStreamWaitEvent(la->side, la->panel[gi][t & 1], 0) != cudaSuccess)
                         return GPTQ_ERR_CUDA;
-                    if ((s = chol_rest_tc(Hg, K, j0n, m, status, la->side, nb)) != GPTQ_OK) return s;
+                    if ((s = chol_rest_tc(Hg, K, j0n, m, status, la->side, nb, 0)) != GPTQ_OK)
+                        return s;
                     if (cudaEventRecord(la->rest[gi][t & 1], la->side) != cudaSuccess)
                         return GPTQ_ERR_CUDA;
                 }
@@ -844,7 +853,7 @@ gptq_status prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out, v
                 const int j0n = bk.start(t - 1);
                 if ((s = chol_panel_strip_tc(Hg, K, j0, j1, j0n, ex, status, st, m)) != GPTQ_OK)
                     return s;
-                if ((s = chol_rest_tc(Hg, K, j0n, m, status, st, nb)) != GPTQ_OK) return s;
+                if ((s = chol_rest_tc(Hg, K, j0n, m, status, st, nb, 0)) != GPTQ_OK) return s;
             }
             continue;
         }

@@ -13,7 +13,7 @@ namespace gptq {
 
 namespace {
 struct ProfRecord {
-    int kind;
+    int kind, lane;
     cudaEvent_t a, b;
 };
 std::mutex g_prof_mu;
@@ -21,6 +21,14 @@ bool g_prof_on = false;
 std::vector<ProfRecord> g_prof;          // records of this profiling window
 std::vector<cudaEvent_t> g_prof_pool;    // events to reuse
 size_t g_prof_used = 0;
+std::vector<cudaStream_t> g_prof_lanes;  // streams of this window, in order of first use
+
+int lane_of(cudaStream_t st) {
+    for (size_t i = 0; i < g_prof_lanes.size(); ++i)
+        if (g_prof_lanes[i] == st) return (int)i;
+    g_prof_lanes.push_back(st);
+    return (int)g_prof_lanes.size() - 1;
+}
 
 cudaEvent_t pool_event() {
     if (g_prof_used < g_prof_pool.size()) return g_prof_pool[g_prof_used++];
@@ -48,7 +56,7 @@ int prof_begin(int kind, cudaStream_t st) {
         cudaGetLastError();
         return -1;
     }
-    g_prof.push_back({kind, a, b});
+    g_prof.push_back({kind, lane_of(st), a, b});
     return (int)g_prof.size() - 1;
 }
 
@@ -97,6 +105,7 @@ gptq_status gptq_profile_enable(int on) {
     g_prof_on = on != 0;
     if (g_prof_on) {          // a new window: earlier records are dropped
         g_prof.clear();
+        g_prof_lanes.clear();
         g_prof_used = 0;
     }
     return GPTQ_OK;
@@ -119,6 +128,28 @@ gptq_status gptq_profile_read(int kind, double *ms, int *launches) {
     }
     *ms = total;
     *launches = count;
+    return GPTQ_OK;
+}
+
+gptq_status gptq_profile_timeline(int max, int *kind, int *lane, double *begin_ms, double *end_ms,
+                                  int *count) {
+    if (max < 0 || !kind || !lane || !begin_ms || !end_ms || !count) return GPTQ_ERR_ARG;
+    std::lock_guard<std::mutex> lock(g_prof_mu);
+    *count = (int)g_prof.size();
+    for (int i = 0; i < (int)g_prof.size() && i < max; ++i) {
+        const ProfRecord &r = g_prof[i];
+        float t0 = 0.f, t1 = 0.f;
+        if (r.kind >= 0 && (cudaEventSynchronize(r.b) != cudaSuccess ||
+            cudaEventElapsedTime(&t0, g_prof[0].a, r.a) != cudaSuccess ||
+            cudaEventElapsedTime(&t1, g_prof[0].a, r.b) != cudaSuccess)) {
+            cudaGetLastError();
+            return GPTQ_ERR_CUDA;
+        }
+        kind[i] = r.kind;
+        lane[i] = r.lane;
+        begin_ms[i] = t0;
+        end_ms[i] = t1;
+    }
     return GPTQ_OK;
 }
 

@@ -956,6 +956,7 @@ static gptq_status quantize_impl(void *W, int wdtype, int N, int K, const float 
             for (int gi = 0; gi < groups; ++gi) {      // far: everything after the super-block
                 UpdateParams p = kbase;
                 p.C = Wk + (int64_t)gi * per_group * K + sb1;
+                p.c_extent = (int64_t)N * K - (p.C - Wk);
                 p.Ncols = K - sb1;
                 p.L = sb1 - sb0;
                 p.a_x0 = gi * lay.ldG;
@@ -994,6 +995,7 @@ static gptq_status quantize_impl(void *W, int wdtype, int N, int K, const float 
                 for (int gi = 0; gi < groups; ++gi) {      // near: the rest of the super-block
                     UpdateParams p = base;
                     p.C = Wk + (int64_t)gi * per_group * K + i1;
+                    p.c_extent = (int64_t)N * K - (p.C - Wk);
                     p.Ncols = sb1 - i1;
                     p.L = bs;
                     p.a_x0 = gi * lay.ldG;
@@ -1008,6 +1010,7 @@ static gptq_status quantize_impl(void *W, int wdtype, int N, int K, const float 
             for (int gi = 0; gi < groups; ++gi) {          // far: everything after the super-block
                 UpdateParams p = base;
                 p.C = Wk + (int64_t)gi * per_group * K + sb1;
+                p.c_extent = (int64_t)N * K - (p.C - Wk);
                 p.Ncols = K - sb1;
                 p.L = sb1 - sb0;
                 p.a_x0 = gi * lay.ldG;

@@ -38,6 +38,7 @@ static gptq_status residual_tc(float *P1, const float *C, const float *U, int K,
     cudaMemsetAsync(T, 0, sizeof(float) * (size_t)KK, st);
     p = Tc32Params{};
     p.C = T; p.alpha = 1.f; p.accumulate = 1; p.upper_tiles = 1; p.mask_strict_upper = 1;
+    p.c_extent = KK;
     p.nitems = 1;
     p.item[0].m = K; p.item[0].n = K; p.item[0].k = K;
     p.item[0].c_off = 0; p.item[0].ldc = K;
@@ -47,6 +48,7 @@ static gptq_status residual_tc(float *P1, const float *C, const float *U, int K,
     cudaMemsetAsync(P1, 0, sizeof(float) * (size_t)KK, st);
     p = Tc32Params{};
     p.C = P1; p.alpha = 1.f; p.accumulate = 1; p.a_upper = 1; p.b_upper = 1;
+    p.c_extent = KK;
     p.nitems = 1;
     p.item[0].m = K; p.item[0].n = K; p.item[0].k = K;
     p.item[0].c_off = 0; p.item[0].ldc = K;

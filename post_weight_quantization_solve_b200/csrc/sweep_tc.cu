@@ -32,6 +32,7 @@
 
 #include <algorithm>
 
+#include "bounds.cuh"
 #include "common.cuh"
 #include "sweep_tc.cuh"
 #include "tc_ptx.cuh"
@@ -133,8 +134,14 @@ __global__ void __launch_bounds__(STC_THREADS, 1)
                 uint32_t bytes = W_SLOT + D_SLOT + 128;
                 if (CAE) bytes += W_SLOT;
                 if (GPTAQ) bytes += D_SLOT;
-                tc::mbar_arrive_expect_tx(&cfull[s], bytes);
                 const int x = sb0 + 32 * q;
+                // fp32 boxes: the coordinate on a 16-byte boundary, inside W and U
+                if (!GQ_IN_BOUNDS(p.status, x >= 0 && x < K && (x & 3) == 0 && n0 < p.N,
+                                  BS_SWEEP_TMA, x)) {
+                    *abort = 1;
+                    return;
+                }
+                tc::mbar_arrive_expect_tx(&cfull[s], bytes);
                 tc::tma_load_2d(smem + OFF_W + s * W_SLOT, &maps.w, &cfull[s], x, n0);
                 if (CAE) tc::tma_load_2d(smem + OFF_W0 + s * W_SLOT, &maps.w0, &cfull[s], x, n0);
                 tc::tma_load_2d(smem + OFF_UD + s * D_SLOT, &maps.ud, &cfull[s], x, grp * K + x);
@@ -146,8 +153,16 @@ __global__ void __launch_bounds__(STC_THREADS, 1)
             auto issue_b = [&](int q) {
                 const int xb = 64 * ((q + 1) / 2);
                 const int nch = (nend - xb + 63) / 64;
-                tc::mbar_arrive_expect_tx(bfull, 2 * nch * CH_BYTES);
                 const int y = sb0 + 32 * q;
+                // bf16 boxes: columns on 16-byte boundaries, from inside the super-block's
+                // span of U; rows of U inside the factor
+                if (!GQ_IN_BOUNDS(p.status, y >= 0 && y < K && ((sb0 + xb) & 7) == 0 &&
+                                                sb0 + xb + 64 * (nch - 1) < K + 64,
+                                  BS_SWEEP_TMA, (long long)y * K + sb0 + xb)) {
+                    *abort = 1;
+                    return;
+                }
+                tc::mbar_arrive_expect_tx(bfull, 2 * nch * CH_BYTES);
                 for (int c = 0; c < nch; ++c) {
                     const int x = sb0 + xb + 64 * c;
                     uint8_t *dh = smem + OFF_B + c * CH_BYTES;
@@ -343,7 +358,9 @@ __global__ void __launch_bounds__(STC_THREADS, 1)
                     }
                     *reinterpret_cast<uint4 *>(ahi + ((c ^ sw) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
                     *reinterpret_cast<uint4 *>(alo + ((c ^ sw) << 4)) = make_uint4(l[0], l[1], l[2], l[3]);
-                    if (valid) {      // the far update's copy: -E, this channel's row
+                    if (valid && GQ_IN_BOUNDS(p.status, ecol * ESTRIDE + 32 * q + 8 * c + 8 <= (int64_t)p.ldE * ESTRIDE,
+                                              BS_SWEEP_OUT, ecol * ESTRIDE + 32 * q + 8 * c)) {
+                        // the far update's copy: -E, this channel's row
                         const int64_t eo = ecol * ESTRIDE + 32 * q + 8 * c;
                         *reinterpret_cast<uint4 *>(p.Eh + eo) = make_uint4(h[0], h[1], h[2], h[3]);
                         *reinterpret_cast<uint4 *>(p.El + eo) = make_uint4(l[0], l[1], l[2], l[3]);
@@ -360,7 +377,8 @@ __global__ void __launch_bounds__(STC_THREADS, 1)
                         }
                         *reinterpret_cast<uint4 *>(ahi + (((4 + c) ^ sw) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
                         *reinterpret_cast<uint4 *>(alo + (((4 + c) ^ sw) << 4)) = make_uint4(l[0], l[1], l[2], l[3]);
-                        if (valid) {
+                        if (valid && GQ_IN_BOUNDS(p.status, ecol * ESTRIDE + 32 * q + 8 * c + 8 <= (int64_t)p.ldE * ESTRIDE,
+                                                  BS_SWEEP_OUT, ecol * ESTRIDE + 32 * q + 8 * c)) {
                             const int64_t eo = ecol * ESTRIDE + 32 * q + 8 * c;
                             *reinterpret_cast<uint4 *>(p.Ph + eo) = make_uint4(h[0], h[1], h[2], h[3]);
                             *reinterpret_cast<uint4 *>(p.Pl + eo) = make_uint4(l[0], l[1], l[2], l[3]);
@@ -369,7 +387,9 @@ __global__ void __launch_bounds__(STC_THREADS, 1)
                 }
                 if ((t & 15) == 15 && valid) {
                     const int c16 = 32 * q + (t & 16);        // 16 codes of this channel
-                    if (c16 < live_end) {
+                    if (c16 < live_end &&
+                        GQ_IN_BOUNDS(p.status, n < p.N && sb0 + min(c16 + 16, live_end) <= K,
+                                     BS_SWEEP_OUT, n * K + sb0 + c16)) {
                         if (vcodes && c16 + 16 <= live_end) {
                             *reinterpret_cast<uint4 *>(crow + c16) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
                         } else {

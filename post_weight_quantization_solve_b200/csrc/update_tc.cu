@@ -24,6 +24,7 @@
 
 #include <algorithm>
 
+#include "bounds.cuh"
 #include "common.cuh"
 #include "tc_ptx.cuh"
 #include "update_tc.cuh"
@@ -97,10 +98,19 @@ __global__ void __launch_bounds__(UT_THREADS, 1)
                 const int row0 = (tile % nm) * UT_BM, col0 = (tile / nm) * UT_BN;
                 for (int it = 0; it < per_tile; ++it) {
                     const int g = it / ksteps, ks = it - g * ksteps;
+                    const int ay = a_y0 + ks * BK, by = b_y0 + ks * BK;
+                    // bf16 boxes: innermost coordinates on 16-byte boundaries, the inner
+                    // step and the tile inside the product
+                    if (!GQ_IN_BOUNDS(p.status, g < p.ngroups && ks * BK < p.L && row0 < p.M && col0 < p.Ncols &&
+                                                    ay >= 0 && by >= 0 && ((AK ? ay : a_x0 + row0) & 7) == 0 &&
+                                                    ((b_x0 + col0) & 7) == 0,
+                                      BS_UPDATE_TMA, AK ? ay : a_x0 + row0)) {
+                        *abort = 1;
+                        break;
+                    }
                     if (!tc::mbar_wait(&empty[stage], phase ^ 1, abort)) break;
                     tc::mbar_arrive_expect_tx(&full[stage], STAGE);
                     uint8_t *st = smem + stage * STAGE;
-                    const int ay = a_y0 + ks * BK, by = b_y0 + ks * BK;
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {       // hi, lo
                         const CUtensorMap *am = &maps.a[2 * g + h];
@@ -203,13 +213,18 @@ __global__ void __launch_bounds__(UT_THREADS, 1)
                             make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
                     tc::fence_async_shared();
                     __syncwarp();
-                    if (lane == 0) {
+                    if (lane == 0 && GQ_IN_BOUNDS(p.status, cb >= 0 && cb < Ncols && (cb & 3) == 0 &&
+                                                                row0 + quad * 32 < M,
+                                                  BS_UPDATE_C, (int64_t)(row0 + quad * 32) * ldc + cb)) {
                         tc::tma_reduce_add_2d(&cmap, buf, cb, row0 + quad * 32);
                         tc::bulk_commit();
                     }
                     ++nbuf;
                 } else {
                     if (r >= M || cb >= Ncols) continue;
+                    if (!GQ_IN_BOUNDS(p.status, p.c_extent == 0 || (int64_t)r * ldc + min(cb + 32, Ncols) <= p.c_extent,
+                                      BS_UPDATE_C, (int64_t)r * ldc + cb))
+                        continue;
                     float *crow = C + (int64_t)r * ldc;
                     if (vec4 && cb + 32 <= Ncols) {
 #pragma unroll
@@ -388,8 +403,10 @@ gptq_status split_bf16(const float *in, int64_t ld_in, int rows, int cols, __nv_
                         ? 1
                         : 0;
     const int bx = (int)std::min<int64_t>(vec ? 2 : 8, (ld_out + 255) / 256);
+    const int rec = prof_begin(GPTQ_PROF_SPLIT, st);
     k_split_bf16<<<dim3(bx, rows, batch), 256, 0, st>>>(in, ld_in, cols, hi, lo, ld_out, batch_in,
                                                         batch_out, vec);
+    prof_end(rec, st);
     return launch_status();
 }
 

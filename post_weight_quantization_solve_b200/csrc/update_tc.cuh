@@ -25,6 +25,7 @@ struct UpdateParams {
     int neg[2];             // subtract group g's product
     int vec4;               // C rows 16-byte aligned: float4 reductions
     int a_kmajor;           // A stored with the channel index as rows (k contiguous); L % 64 == 0
+    int64_t c_extent;       // elements addressable from C (0: not given; index-checking build)
     int32_t *status;
 };
 

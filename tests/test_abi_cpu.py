@@ -34,7 +34,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for code in range(7):
+    for code in range(8):
         assert gq.gptq_status_string(code) not in ("", "unknown status")
     assert gq.gptq_status_string(99) == "unknown status"
 
@@ -91,10 +91,25 @@ def test_host_argument_checks(lib):
     ms, cnt = ctypes.c_double(-1.0), ctypes.c_int(-1)
     assert lib.gptq_profile_read(gq.GPTQ_PROF_UPDATE, ctypes.byref(ms), ctypes.byref(cnt)) == gq.GPTQ_OK
     assert ms.value == 0.0 and cnt.value == 0
-    assert lib.gptq_profile_read(4, ctypes.byref(ms), ctypes.byref(cnt)) == gq.GPTQ_ERR_ARG
+    assert lib.gptq_profile_read(5, ctypes.byref(ms), ctypes.byref(cnt)) == gq.GPTQ_ERR_ARG
     assert lib.gptq_profile_read(0, None, ctypes.byref(cnt)) == gq.GPTQ_ERR_ARG
+    ki, la = (ctypes.c_int * 2)(), (ctypes.c_int * 2)()
+    t0, t1 = (ctypes.c_double * 2)(), (ctypes.c_double * 2)()
+    assert lib.gptq_profile_timeline(2, ki, la, t0, t1, ctypes.byref(cnt)) == gq.GPTQ_OK
+    assert cnt.value == 0
+    assert lib.gptq_profile_timeline(-1, ki, la, t0, t1, ctypes.byref(cnt)) == gq.GPTQ_ERR_ARG
+    assert lib.gptq_profile_timeline(2, ki, la, t0, None, ctypes.byref(cnt)) == gq.GPTQ_ERR_ARG
     assert lib.gptq_profile_enable(0) == gq.GPTQ_OK
     assert lib.gptq_chain_latency(fake, 12, None) == gq.GPTQ_ERR_ARG
+    # index-check records: the normal build has none and no self-test
+    en, cnt, site, idx = ctypes.c_int(-1), ctypes.c_int(-1), ctypes.c_int(-1), ctypes.c_int64(-1)
+    assert lib.gptq_bounds_report(ctypes.byref(en), ctypes.byref(cnt), ctypes.byref(site),
+                                  ctypes.byref(idx), 1) == gq.GPTQ_OK
+    assert (en.value, cnt.value, site.value, idx.value) == (0, 0, 0, 0)
+    assert lib.gptq_bounds_report(None, ctypes.byref(cnt), ctypes.byref(site), ctypes.byref(idx),
+                                  0) == gq.GPTQ_ERR_ARG
+    assert lib.gptq_bounds_selftest(fake, None) == gq.GPTQ_ERR_ARG
+    assert lib.gptq_bounds_selftest(None, None) == gq.GPTQ_ERR_ARG
     assert lib.gptq_chain_latency(None, 64, None) == gq.GPTQ_ERR_ARG
     # pack / unpack: bits, strides, NULL pointers; N == 0 does nothing
     assert lib.gptq_pack_codes(fake, 4, 64, 64, 5, fake, 64, None) == gq.GPTQ_ERR_ARG
@@ -133,6 +148,17 @@ def test_host_argument_checks(lib):
     assert lib.gptaq_accumulate_cross(fake, 16, fake, fake, gq.GPTQ_BF16, 0, 16,
                                       None, None) == gq.GPTQ_OK
     assert lib.gptaq_residual(fake, fake, fake, 16, ws, 8, None) == gq.GPTQ_ERR_WORKSPACE
+
+
+def test_checking_build_exports_the_same_entry_points(lib):
+    # the GPTQ_DEBUG_BOUNDS variant builds and loads beside the normal library, with the
+    # same C ABI (it differs only inside the kernels)
+    from post_weight_quantization_solve_b200.build import LIB_DBG
+
+    dbg = ctypes.CDLL(build(debug_bounds=True))
+    assert os.path.samefile(LIB_DBG, dbg._name)
+    for name in header_entry_points():
+        assert hasattr(dbg, name), name
 
 
 def test_product_path_fails_loudly_without_library(monkeypatch, tmp_path):
@@ -296,6 +322,9 @@ def test_every_wrapper_matches_its_c_signature(lib, monkeypatch):
     gq.gptq_chain_latency(torch.zeros(3), steps=64)
     gq.gptq_profile_enable(True)
     gq.gptq_profile_read(gq.GPTQ_PROF_SWEEP)
+    gq.gptq_profile_timeline(8)
+    gq.gptq_bounds_report(reset=True)
+    gq.gptq_bounds_selftest(status=st)
     assert set(calls) == set(gq.EXPORTS) - {"gptq_trust_region_beta", "gptq_workspace_size",
                                             "gptq_kernel_launches", "gptq_status_string"}
     # the workspace sizes passed are the ones the library asks for
