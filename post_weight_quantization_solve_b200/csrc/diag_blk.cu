@@ -9,8 +9,9 @@
 //
 // The 128 pivots run as eight sub-blocks of 16, from the last:
 //   (A) one warp factors the sub-block S_bb = L_bb D_b L_bb^T and forms V_bb = L_bb^-1:
-//       lanes 0-15 hold the rows of S_bb, lanes 16-31 the rows of V_bb, and each pivot's
-//       row reaches the other lanes by shuffles (no block barrier per pivot);
+//       lanes 0-15 hold the rows of S_bb, lanes 16-31 the rows of V_bb, four pivots per
+//       step, each step's pivot rows published in shared memory (no block barrier per
+//       pivot);
 //   (A') the sub-block's rows of V over the later columns: V_b,later = V_bb X, where X
 //       holds what the later sub-blocks' eliminations left there;
 //   (B) the panel above the sub-block: P = S_ab V_bb^T and L_ab = P D_b^-1;
@@ -18,10 +19,13 @@
 //       sub-block (upper triangle);
 //   (D) the rows before the sub-block of V: V_a,c -= L_ab V_b,c for the columns c from
 //       the sub-block on (right-looking elimination of L^-1).
-// A, then A' with B, then C with D, each separated by one block barrier: three per
-// sub-block instead of one per pivot (pair). The products run from shared memory in
-// 4 x 4 register tiles. The pivot test is the same as the per-pivot kernels':
-// refuse a pivot p_j <= tol * Hd_jj.
+// Two block barriers per sub-block: one warp's A runs beside the previous sub-block's
+// C and D on six other warps, then A' and B. The products run from shared memory in
+// 4 x 4 register tiles. The block arrives in two groups of asynchronous copies (the
+// last sub-block's rows first, the rest during its factor), and the eighth warp, which
+// shares the factoring warp's scheduler and takes no tiles, writes each sub-block's
+// rows of U as soon as they are final. The pivot test is the same as the per-pivot
+// kernels': refuse a pivot p_j <= tol * Hd_jj.
 #include <float.h>
 
 #include "bounds.cuh"
@@ -73,14 +77,22 @@ __global__ void __launch_bounds__(DB_T, 1) k_chol_diag_blk(float *H, int K, int 
     const bool vec = nb == DB_N && K % 4 == 0 && j0 % 4 == 0 &&
                      (reinterpret_cast<uintptr_t>(H) & 15) == 0;
     if (vec) {
-#pragma unroll 4
-        for (int it = 0; it < DB_N * DB_N / 4 / DB_T; ++it) {
-            const int id = tid + DB_T * it, r = id >> 5, c4 = (id & 31) * 4;
+        // two groups of copies: the last sub-block's rows (all the first factor step
+        // reads), then the rest, which lands while that step runs
+        auto copy = [&](int id) {
+            const int r = id >> 5, c4 = (id & 31) * 4;
             const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(S + r * DB_LD + c4));
             asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst),
                          "l"(H + (int64_t)(j0 + r) * K + j0 + c4)
                          : "memory");
-        }
+        };
+        constexpr int LAST = (DB_N - DB_SB) * DB_N / 4;      // first copy of the last rows
+#pragma unroll
+        for (int it = 0; it < DB_SB * DB_N / 4 / DB_T; ++it) copy(LAST + tid + DB_T * it);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+#pragma unroll 4
+        for (int it = 0; it < LAST / DB_T; ++it) copy(tid + DB_T * it);
+        asm volatile("cp.async.commit_group;" ::: "memory");
     } else {
         for (int idx = tid; idx < DB_N * DB_N; idx += DB_T) {
             const int r = idx >> 7, c = idx & 127;
@@ -94,7 +106,7 @@ __global__ void __launch_bounds__(DB_T, 1) k_chol_diag_blk(float *H, int K, int 
             make_float4(r == c4 ? 1.f : 0.f, r == c4 + 1 ? 1.f : 0.f, r == c4 + 2 ? 1.f : 0.f,
                         r == c4 + 3 ? 1.f : 0.f);
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");
+    asm volatile("cp.async.wait_group 1;" ::: "memory");   // this thread's last-rows copies
     if (tid < DB_N) dref[tid] = tid < nb ? diag_d[j0 + tid] : 1.f;
     __syncthreads();
 
@@ -221,7 +233,9 @@ __global__ void __launch_bounds__(DB_T, 1) k_chol_diag_blk(float *H, int K, int 
         #pragma unroll
                         for (int t = 3; t >= 0; --t) {
                             d[t] = P[t][t];
-                            r[t] = __frcp_rn(fmaxf(d[t], FLT_MIN));
+                            // the pivot's reciprocal (hardware approximation, ~1 ulp): it only
+                            // scales multipliers whose rounding is of the same order
+                            asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r[t]) : "f"(fmaxf(d[t], FLT_MIN)));
         #pragma unroll
                             for (int q = 0; q < t; ++q) m[q][t] = P[q][t] * r[t];
         #pragma unroll
@@ -287,8 +301,30 @@ __global__ void __launch_bounds__(DB_T, 1) k_chol_diag_blk(float *H, int K, int 
                     if (tid < DB_SB && o + tid < nb && !(dd[o + tid] > tol * dref[o + tid]))
                         set_status(status, GPTQ_ERR_NOT_PD);
                 }
+                // this warp's share of the block's other rows (the first factor step reads
+                // only the last sub-block's; the tiles start from the next iteration)
+                asm volatile("cp.async.wait_group 0;" ::: "memory");
+            } else if (tid < 128 || tid >= 160) {
+                // the tiles on six warps: warp 4 shares warp 0's scheduler and stays off them
+                asm volatile("cp.async.wait_group 0;" ::: "memory");
+                const int wi = tid < 128 ? tid - 32 : tid - 64;
+                for (int u = wi; u < nCo + nD; u += DB_T - 64) tile(u < nCo ? u : u + 10);
             } else {
-                for (int u = tid - 32; u < nCo + nD; u += DB_T - 32) tile(u < nCo ? u : u + 10);
+                asm volatile("cp.async.wait_group 0;" ::: "memory");
+                // warp 4: sub-block b + 1's rows of U are final (nothing after its step
+                // writes them): U = D^-1/2 V, zero below the diagonal, written out now
+                if (vec && b + 1 < DB_N / DB_SB) {
+                    const int lane = tid - 128;
+#pragma unroll 4
+                    for (int it = 0; it < DB_SB * DB_N / 4 / 32; ++it) {
+                        const int id = lane + 32 * it, r = op + (id >> 5), c4 = (id & 31) * 4;
+                        const float4 v = *reinterpret_cast<const float4 *>(V + r * DB_LD + c4);
+                        const float sc = 1.f / sqrtf(fmaxf(dd[r], FLT_MIN));
+                        *reinterpret_cast<float4 *>(H + (int64_t)(j0 + r) * K + j0 + c4) =
+                            make_float4(c4 >= r ? v.x * sc : 0.f, c4 + 1 >= r ? v.y * sc : 0.f,
+                                        c4 + 2 >= r ? v.z * sc : 0.f, c4 + 3 >= r ? v.w * sc : 0.f);
+                    }
+                }
             }
         }
         __syncthreads();
@@ -343,9 +379,9 @@ __global__ void __launch_bounds__(DB_T, 1) k_chol_diag_blk(float *H, int K, int 
     // U_JJ = D^-1/2 V (zero below the diagonal)
     if (tid < DB_N) dref[tid] = 1.f / sqrtf(fmaxf(dd[tid], FLT_MIN));
     __syncthreads();
-    if (vec) {
-#pragma unroll 4
-        for (int it = 0; it < DB_N * DB_N / 4 / DB_T; ++it) {
+    if (vec) {      // rows 16 .. 127 were written during the later iterations
+#pragma unroll
+        for (int it = 0; it < DB_SB * DB_N / 4 / DB_T; ++it) {
             const int id = tid + DB_T * it, r = id >> 5, c4 = (id & 31) * 4;
             const float4 v = *reinterpret_cast<const float4 *>(V + r * DB_LD + c4);
             const float sc = dref[r];
