@@ -28,6 +28,8 @@
 // kernels': refuse a pivot p_j <= tol * Hd_jj.
 #include <float.h>
 
+#include <algorithm>
+
 #include "bounds.cuh"
 #include "common.cuh"
 
@@ -44,9 +46,48 @@ constexpr size_t diag_blk_smem() {
     return sizeof(float) * (2 * DB_N * DB_LD + 2 * DB_SB * DB_LD + 3 * DB_N + 4);
 }
 
+// x -> its tf32 pair (hi = x rounded to tf32, lo = x - hi), as the tf32x3 products read it.
+__device__ __forceinline__ void tf32_pair(float x, float &hi, float &lo) {
+    uint32_t b;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(b) : "f"(x));
+    hi = __uint_as_float(b);
+    lo = x - hi;
+}
+
+__device__ __forceinline__ void store_pair4(float *hi, float *lo, float4 v) {
+    float4 h, l;
+    tf32_pair(v.x, h.x, l.x);
+    tf32_pair(v.y, h.y, l.y);
+    tf32_pair(v.z, h.z, l.z);
+    tf32_pair(v.w, h.w, l.w);
+    *reinterpret_cast<float4 *>(hi) = h;
+    *reinterpret_cast<float4 *>(lo) = l;
+}
+
+// Grid: g factor CTAs, then (with pairs) g * nsplit CTAs that write the tf32 pairs of
+// the column block's rows above the diagonal block, H[0:j0, J], for the step's panel
+// product. pairs: per group (stride pstride floats) hi rows then lo rows (at
+// (j0 + nb) * nb), row pitch nb; the factor CTA adds U_JJ's rows j0 .. j0 + nb.
 __global__ void __launch_bounds__(DB_T, 1) k_chol_diag_blk(float *H, int K, int j0, int nb,
                                                           const float *diag_d, float tol,
-                                                          int32_t *status) {
+                                                          int32_t *status, float *pairs,
+                                                          int64_t pstride, int nsplit) {
+    if (pairs && (int)blockIdx.x >= (int)gridDim.x / (1 + nsplit)) {
+        // a pair-split CTA: rows [r0, r1) of H[0:j0, J] of one group
+        const int id = (int)blockIdx.x - (int)gridDim.x / (1 + nsplit);
+        const int gi = id / nsplit, part = id - gi * nsplit;
+        if (failed(status)) return;
+        const int r0 = (int)((int64_t)j0 * part / nsplit), r1 = (int)((int64_t)j0 * (part + 1) / nsplit);
+        const float *Hg = H + (int64_t)gi * K * K;
+        float *ph = pairs + gi * pstride, *pl = ph + (int64_t)(j0 + nb) * nb;
+        const int c4n = nb / 4;
+        for (int idx = threadIdx.x; idx < (r1 - r0) * c4n; idx += DB_T) {
+            const int r = r0 + idx / c4n, c = (idx % c4n) * 4;
+            const float4 v = *reinterpret_cast<const float4 *>(Hg + (int64_t)r * K + j0 + c);
+            store_pair4(ph + (int64_t)r * nb + c, pl + (int64_t)r * nb + c, v);
+        }
+        return;
+    }
     extern __shared__ __align__(16) float sm[];
     float *S = sm;                          // [128][LD] the block, upper triangle
     float *V = S + DB_N * DB_LD;            // [128][LD] V = L^-1 (unit upper)
@@ -70,6 +111,9 @@ __global__ void __launch_bounds__(DB_T, 1) k_chol_diag_blk(float *H, int K, int 
     const int g = blockIdx.x;
     H += (int64_t)g * K * K;
     diag_d += (int64_t)g * K;
+    // this group's pair rows of U_JJ (rows j0 .. j0 + nb of the column block's pairs)
+    float *ph = pairs ? pairs + g * pstride : nullptr;
+    float *pl = pairs ? ph + (int64_t)(j0 + nb) * nb : nullptr;
 
     // S = the block as stored; only its upper triangle is ever read (the lower one may
     // hold stale values). Beyond nb: the identity. V = I. A full block arrives as
@@ -116,6 +160,9 @@ __global__ void __launch_bounds__(DB_T, 1) k_chol_diag_blk(float *H, int K, int 
     // factor thus overlaps the bulk of the previous step's updates.
     for (int b = DB_N / DB_SB - 1; b >= 0; --b) {
         const int o = DB_SB * b;                 // first coordinate of sub-block b
+        // the step's panel product (launched as a programmatic dependent) may start its
+        // set-up during the last sub-block; it waits for this grid's end before reading
+        if (b == 0) asm volatile("griddepcontrol.launch_dependents;");
         {
             const int op = o + DB_SB;            // step b + 1 (none for the last sub-block)
             const int T = b + 1 < DB_N / DB_SB ? op / 4 : 0;
@@ -320,9 +367,11 @@ __global__ void __launch_bounds__(DB_T, 1) k_chol_diag_blk(float *H, int K, int 
                         const int id = lane + 32 * it, r = op + (id >> 5), c4 = (id & 31) * 4;
                         const float4 v = *reinterpret_cast<const float4 *>(V + r * DB_LD + c4);
                         const float sc = 1.f / sqrtf(fmaxf(dd[r], FLT_MIN));
-                        *reinterpret_cast<float4 *>(H + (int64_t)(j0 + r) * K + j0 + c4) =
+                        const float4 u =
                             make_float4(c4 >= r ? v.x * sc : 0.f, c4 + 1 >= r ? v.y * sc : 0.f,
                                         c4 + 2 >= r ? v.z * sc : 0.f, c4 + 3 >= r ? v.w * sc : 0.f);
+                        *reinterpret_cast<float4 *>(H + (int64_t)(j0 + r) * K + j0 + c4) = u;
+                        if (ph) store_pair4(ph + (int64_t)(j0 + r) * DB_N + c4, pl + (int64_t)(j0 + r) * DB_N + c4, u);
                     }
                 }
             }
@@ -385,26 +434,37 @@ __global__ void __launch_bounds__(DB_T, 1) k_chol_diag_blk(float *H, int K, int 
             const int id = tid + DB_T * it, r = id >> 5, c4 = (id & 31) * 4;
             const float4 v = *reinterpret_cast<const float4 *>(V + r * DB_LD + c4);
             const float sc = dref[r];
-            *reinterpret_cast<float4 *>(H + (int64_t)(j0 + r) * K + j0 + c4) =
-                make_float4(c4 >= r ? v.x * sc : 0.f, c4 + 1 >= r ? v.y * sc : 0.f,
-                            c4 + 2 >= r ? v.z * sc : 0.f, c4 + 3 >= r ? v.w * sc : 0.f);
+            const float4 u = make_float4(c4 >= r ? v.x * sc : 0.f, c4 + 1 >= r ? v.y * sc : 0.f,
+                                         c4 + 2 >= r ? v.z * sc : 0.f, c4 + 3 >= r ? v.w * sc : 0.f);
+            *reinterpret_cast<float4 *>(H + (int64_t)(j0 + r) * K + j0 + c4) = u;
+            if (ph) store_pair4(ph + (int64_t)(j0 + r) * DB_N + c4, pl + (int64_t)(j0 + r) * DB_N + c4, u);
         }
     } else {
         for (int idx = tid; idx < nb * nb; idx += DB_T) {
             const int r = idx / nb, c = idx - r * nb;
-            H[(int64_t)(j0 + r) * K + j0 + c] = c >= r ? V[r * DB_LD + c] * dref[r] : 0.f;
+            const float u = c >= r ? V[r * DB_LD + c] * dref[r] : 0.f;
+            H[(int64_t)(j0 + r) * K + j0 + c] = u;
+            if (ph) tf32_pair(u, ph[(int64_t)(j0 + r) * nb + c], pl[(int64_t)(j0 + r) * nb + c]);
         }
     }
 }
 
 gptq_status launch_chol_diag_blk(float *H, int K, int g, int j0, int nb, const float *diag_d,
-                                 float tol, int32_t *status, cudaStream_t st) {
+                                 float tol, int32_t *status, cudaStream_t st, float *pairs,
+                                 int64_t pstride) {
     if (nb < 1 || nb > DB_N) return GPTQ_ERR_ARG;
+    // the pairs are written with 16-byte stores over rows of nb = 128 floats
+    if (pairs && (nb != DB_N || K % 4 != 0 || j0 % 4 != 0 || pstride % 4 != 0 ||
+                  (reinterpret_cast<uintptr_t>(pairs) & 15) != 0 || (reinterpret_cast<uintptr_t>(H) & 15) != 0))
+        return GPTQ_ERR_ARG;
     const int smem = (int)diag_blk_smem();
     if (cudaFuncSetAttribute(k_chol_diag_blk, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
         cudaSuccess)
         return launch_status();
-    k_chol_diag_blk<<<g, DB_T, smem, st>>>(H, K, j0, nb, diag_d, tol, status);
+    // about 128 rows (64 KB of H) per split CTA
+    const int nsplit = pairs ? std::max(1, std::min(64, (j0 + 127) / 128)) : 0;
+    k_chol_diag_blk<<<g * (1 + nsplit), DB_T, smem, st>>>(H, K, j0, nb, diag_d, tol, status, pairs,
+                                                          pstride, nsplit);
     return launch_status();
 }
 

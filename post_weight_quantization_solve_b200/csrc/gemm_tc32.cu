@@ -132,6 +132,11 @@ __global__ void __launch_bounds__(G32_THREADS, 1)
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    // Launched as a programmatic dependent (Tc32Params::pdl), the set-up above overlaps
+    // the previous kernel's tail; nothing global is read or written before this wait,
+    // which returns once that kernel has finished and its writes are visible (at once
+    // for an ordinary launch).
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     if (warp == 0) {
         if (lane == 0) {
@@ -207,6 +212,8 @@ __global__ void __launch_bounds__(G32_THREADS, 1)
         }
     } else {
         const int quad = warp & 3;
+        // a dependent launch may start its set-up now (it waits for this grid's end)
+        asm volatile("griddepcontrol.launch_dependents;");
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
@@ -488,7 +495,23 @@ gptq_status launch_gemm_tc32(const CUtensorMap maps[4], Tc32Params &p, cudaStrea
     const int grid = std::min(units, p.max_grid > 0 ? std::min(p.max_grid, tc32_sms()) : tc32_sms());
     cudaFuncSetAttribute(k_gemm_tc32, cudaFuncAttributeMaxDynamicSharedMemorySize, G32_SMEM);
     const int rec = prof_begin(GPTQ_PROF_TC32, st);
-    k_gemm_tc32<<<grid, G32_THREADS, G32_SMEM, st>>>(maps[0], maps[1], maps[2], maps[3], p);
+    if (p.pdl) {
+        // programmatic dependent launch: the kernel's set-up may overlap the previous
+        // kernel on the stream; its griddepcontrol.wait orders every global access
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(G32_THREADS);
+        cfg.dynamicSmemBytes = G32_SMEM;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cudaLaunchKernelEx(&cfg, k_gemm_tc32, maps[0], maps[1], maps[2], maps[3], p);
+    } else {
+        k_gemm_tc32<<<grid, G32_THREADS, G32_SMEM, st>>>(maps[0], maps[1], maps[2], maps[3], p);
+    }
     const gptq_status s = launch_status();
     prof_end(rec, st);
     return s;

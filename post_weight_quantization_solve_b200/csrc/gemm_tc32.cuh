@@ -28,6 +28,7 @@ struct Tc32Params {
     int b_lower;            // B(k,j) == 0 for k < j: the k range starts at the column tile
     int nitems, units;
     int max_grid;           // > 0: at most this many CTAs (leaves SMs to other streams)
+    int pdl;                // launch as a programmatic dependent of the stream's previous kernel
     // Optional (one item, overwrite mode, unsplit inner range): the stored values also
     // as tf32 pairs, element (i, j) of the item at pair_hi / pair_lo[i * pair_ld + j].
     float *pair_hi, *pair_lo;

@@ -35,7 +35,8 @@
 namespace gptq {
 
 gptq_status launch_chol_diag_blk(float *H, int K, int g, int j0, int nb, const float *diag_d,
-                                 float tol, int32_t *status, cudaStream_t st);
+                                 float tol, int32_t *status, cudaStream_t st, float *pairs,
+                                 int64_t pstride);
 
 __global__ void k_check_finite(const float *A, int64_t count, int32_t *status) {
     int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
@@ -517,12 +518,15 @@ static size_t tc_extra_floats(int K) {
 // per-(group, step parity) buffer so that a rest still reading them is not
 // overwritten by the next step.
 static gptq_status chol_panel_strip_tc(float *H, int K, int j0, int j1, int j0n, float *buf,
-                                       int32_t *status, cudaStream_t st, CUtensorMap (&m)[4]) {
+                                       int32_t *status, cudaStream_t st, CUtensorMap (&m)[4],
+                                       bool pairs_ready) {
     const int nb = j1 - j0;
     float *Ch = buf, *Cl = Ch + (size_t)j1 * nb;
     static thread_local Tc32Params pp, ps;
     gptq_status s;
-    if ((s = split_tf32(H + j0, K, j1, nb, Ch, Cl, nb, 1, 0, 0, st)) != GPTQ_OK) return s;
+    // the column block's pairs (rows 0 .. j1), unless the diagonal factor's launch wrote them
+    if (!pairs_ready && (s = split_tf32(H + j0, K, j1, nb, Ch, Cl, nb, 1, 0, 0, st)) != GPTQ_OK)
+        return s;
     if ((s = make_f32_map(&m[0], Ch, nb, j1, nb, 32, 128)) != GPTQ_OK) return s;
     if ((s = make_f32_map(&m[1], Cl, nb, j1, nb, 32, 128)) != GPTQ_OK) return s;
     m[2] = m[0]; m[3] = m[1];
@@ -535,6 +539,7 @@ static gptq_status chol_panel_strip_tc(float *H, int K, int j0, int j1, int j0n,
     // (0..j0) of the block's pairs: each row tile is read (as A) and written by the
     // same unit, and the U_JJ rows read as B lie behind them
     pp.pair_hi = Ch; pp.pair_lo = Cl; pp.pair_ld = nb;
+    pp.pdl = 1;         // its set-up overlaps the end of the kernel before it
     pp.c_extent = (int64_t)K * K; pp.pair_extent = (int64_t)j1 * nb;
     if ((s = launch_gemm_tc32(m, pp, st)) != GPTQ_OK) return s;
     // strip: every row above j0 against the rows of J' (entries below the diagonal of
@@ -545,6 +550,7 @@ static gptq_status chol_panel_strip_tc(float *H, int K, int j0, int j1, int j0n,
     ps.item[0].a_x0 = 0; ps.item[0].a_y0 = 0; ps.item[0].b_x0 = 0; ps.item[0].b_y0 = j0n;
     ps.item[0].c_off = j0n; ps.item[0].ldc = K;
     ps.c_extent = (int64_t)K * K;
+    ps.pdl = 1;
     return launch_gemm_tc32(m, ps, st);
 }
 
@@ -808,9 +814,16 @@ gptq_status prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out, v
             for (int gi = 0; gi < g; ++gi)
                 if (cudaStreamWaitEvent(st, la->rest[gi][(t + 2) & 1], 0) != cudaSuccess)
                     return GPTQ_ERR_CUDA;
+        // with the lookahead's per-group pair buffers, the factor's launch also writes the
+        // tf32 pairs of the column block that the step's panel product reads
+        const bool tc_step = use_tc && j0 >= TC_STEP_MIN && nb % 32 == 0;
+        const bool fused_pairs =
+            la && tc_step && diag_mode == 0 && nb == CH_NB && K % 4 == 0 && aligned(H, 16);
         const int rec = prof_begin(GPTQ_PROF_DIAG, st);
         if (diag_mode == 0) {
-            s = launch_chol_diag_blk(H, K, g, j0, nb, diag_d, tol, status, st);
+            s = launch_chol_diag_blk(H, K, g, j0, nb, diag_d, tol, status, st,
+                                     fused_pairs ? ex + (size_t)(t & 1) * pair_floats : nullptr,
+                                     (int64_t)(2 * pair_floats));
         } else {
             if (diag_mode == 1)
                 k_chol_diag2<<<g, DG_T, chol_smem, st>>>(H, K, j0, nb, diag_d, tol, status);
@@ -821,7 +834,7 @@ gptq_status prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out, v
         prof_end(rec, st);
         if (s != GPTQ_OK) return s;
         if (j0 == 0) break;
-        if (use_tc && j0 >= TC_STEP_MIN && nb % 32 == 0) {
+        if (tc_step) {
             if (la) {
                 const int j0n = bk.start(t - 1);
                 if (!side_busy) {
@@ -834,7 +847,8 @@ gptq_status prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out, v
                     float *Hg = H + (int64_t)gi * KK;
                     float *buf = ex + (size_t)(gi * 2 + (t & 1)) * pair_floats;
                     CUtensorMap m[4];
-                    if ((s = chol_panel_strip_tc(Hg, K, j0, j1, j0n, buf, status, st, m)) != GPTQ_OK)
+                    if ((s = chol_panel_strip_tc(Hg, K, j0, j1, j0n, buf, status, st, m, fused_pairs)) !=
+                        GPTQ_OK)
                         return s;
                     if (cudaEventRecord(la->panel[gi][t & 1], st) != cudaSuccess ||
                         cudaStreamWaitEvent(la->side, la->panel[gi][t & 1], 0) != cudaSuccess)
@@ -851,7 +865,7 @@ gptq_status prepare(float *H, int K, int g, float percdamp, uint8_t *dead_out, v
                 float *Hg = H + (int64_t)gi * KK;
                 CUtensorMap m[4];
                 const int j0n = bk.start(t - 1);
-                if ((s = chol_panel_strip_tc(Hg, K, j0, j1, j0n, ex, status, st, m)) != GPTQ_OK)
+                if ((s = chol_panel_strip_tc(Hg, K, j0, j1, j0n, ex, status, st, m, false)) != GPTQ_OK)
                     return s;
                 if ((s = chol_rest_tc(Hg, K, j0n, m, status, st, nb, 0)) != GPTQ_OK) return s;
             }
