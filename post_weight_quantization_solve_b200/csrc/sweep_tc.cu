@@ -124,6 +124,11 @@ __global__ void __launch_bounds__(STC_THREADS, 1)
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    // set-up done: wait for the previous kernel on the stream (when launched as its
+    // programmatic dependent; at once otherwise) before any global access, and let the
+    // next kernel start its own set-up
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
 
     if (warp == 4) {
         if (lane == 0) {
@@ -524,7 +529,19 @@ gptq_status sweep_tc_launch(const SweepTcMaps &maps, const float *scale, int bit
         cudaSuccess)
         return launch_status();
     const int rec = prof_begin(GPTQ_PROF_SWEEP, st);
-    kern<<<grid, STC_THREADS, STC_SMEM, st>>>(maps, p);
+    // a programmatic dependent of the previous kernel on the stream (the far update):
+    // its set-up overlaps that kernel's end; griddepcontrol.wait orders its accesses
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(STC_THREADS);
+    cfg.dynamicSmemBytes = STC_SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, kern, maps, p);
     const gptq_status s = launch_status();
     prof_end(rec, st);
     return s;

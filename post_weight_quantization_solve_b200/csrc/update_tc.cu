@@ -88,6 +88,11 @@ __global__ void __launch_bounds__(UT_THREADS, 1)
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    // set-up done: wait for the previous kernel on the stream (when launched as its
+    // programmatic dependent; at once otherwise) before any global access, and let the
+    // next kernel start its own set-up
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
 
     if (warp == 0) {
         if (lane == 0) {
@@ -322,7 +327,19 @@ static gptq_status launch_update(const UpdateMaps &maps, const CUtensorMap &cmap
                                  const UpdateParams &p, int grid, cudaStream_t st) {
     cudaFuncSetAttribute(k_update_tc<BK, TMA_EPI, AK>, cudaFuncAttributeMaxDynamicSharedMemorySize, UT_SMEM);
     const int rec = prof_begin(GPTQ_PROF_UPDATE, st);
-    k_update_tc<BK, TMA_EPI, AK><<<grid, UT_THREADS, UT_SMEM, st>>>(maps, cmap, p);
+    // a programmatic dependent of the previous kernel on the stream (a sweep): its set-up
+    // overlaps that kernel's end; griddepcontrol.wait orders its accesses
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(UT_THREADS);
+    cfg.dynamicSmemBytes = UT_SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, k_update_tc<BK, TMA_EPI, AK>, maps, cmap, p);
     const gptq_status s = launch_status();
     prof_end(rec, st);
     return s;
