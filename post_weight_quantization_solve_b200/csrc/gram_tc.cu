@@ -114,6 +114,11 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    // set-up done: wait for the previous kernel on the stream (when launched as its
+    // programmatic dependent; at once otherwise) before any global access, and let the
+    // next kernel start its own set-up
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
 
     if (warp == 0) {
         if (lane == 0) {
@@ -356,6 +361,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(G2_THREADS, 1)
     tc::cluster_sync();             // both CTAs' barriers exist before any remote use
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    // set-up done: wait for the previous kernel on the stream (when launched as its
+    // programmatic dependent; at once otherwise) before any global access, and let the
+    // next kernel start its own set-up
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
     // an earlier failure skips the work; both CTAs take the even CTA's reading of the
     // status, so the pair always agrees and meets at the final cluster barrier
     const int units =
@@ -627,10 +637,35 @@ gptq_status gram_tc(float *H, int K, int g, const void *X, int64_t M, int64_t ld
     }
     if (pair) {
         cudaFuncSetAttribute(k_gram_tc2, cudaFuncAttributeMaxDynamicSharedMemorySize, G2_SMEM);
-        k_gram_tc2<<<grid, G2_THREADS, G2_SMEM, st>>>(tmap, hmap, p);
+        // programmatic dependents: a chunk's launch sets up while the previous one ends
+        {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(G2_THREADS);
+        cfg.dynamicSmemBytes = G2_SMEM;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cudaLaunchKernelEx(&cfg, k_gram_tc2, tmap, hmap, p);
+    }
     } else {
         cudaFuncSetAttribute(k_gram_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, GT_SMEM);
-        k_gram_tc<<<grid, GT_THREADS, GT_SMEM, st>>>(tmap, hmap, p);
+        {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(GT_THREADS);
+        cfg.dynamicSmemBytes = GT_SMEM;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cudaLaunchKernelEx(&cfg, k_gram_tc, tmap, hmap, p);
+    }
     }
     gptq_status s = launch_status();
     if (s != GPTQ_OK) return s;

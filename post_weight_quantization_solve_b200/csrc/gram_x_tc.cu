@@ -123,6 +123,11 @@ __global__ void __launch_bounds__(GX_THREADS, 1)
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    // set-up done: wait for the previous kernel on the stream (when launched as its
+    // programmatic dependent; at once otherwise) before any global access, and let the
+    // next kernel start its own set-up
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
 
     if (warp == 0) {
         if (lane == 0) {
@@ -422,7 +427,19 @@ gptq_status gram_x_tc(float *H, int K, int g, const void *X, const void *X2, int
     CUtensorMap hmap;
     if ((s = make_f32_map(&hmap, H, K, (int64_t)p.groups * K, K, 32, 32)) != GPTQ_OK) return s;
     cudaFuncSetAttribute(k_gram_x_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, GX_SMEM);
-    k_gram_x_tc<<<grid, GX_THREADS, GX_SMEM, st>>>(ma0, ma1, mb, hmap, p);
+    {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(GX_THREADS);
+        cfg.dynamicSmemBytes = GX_SMEM;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cudaLaunchKernelEx(&cfg, k_gram_x_tc, ma0, ma1, mb, hmap, p);
+    }
     if ((s = launch_status()) != GPTQ_OK) return s;
     *used = true;
     return GPTQ_OK;
