@@ -168,7 +168,10 @@ def test_grouped70b_fullsize():
         (H_d = V V^T with V = U^-1 upper couples that block to nothing else);
       - U H_d U^T = I on sampled row pairs, in fp64;
     and sampled channels of every group are replayed by the oracle's sweep on the
-    GPU's U (upcast), which pins the sweep given U."""
+    GPU's U (upcast), which pins the sweep given U. The result's reconstruction error on
+    those channels, 1/2 D^T H_d D with D = W - W_hat in fp64, equals the loss the sweep
+    reports (1/2 sum E^2 along the trajectory: the two agree for the sequential optimal
+    compensation), and their summed error is below round-to-nearest's on the same grid."""
     wl = synth.WORKLOADS["grouped70b"]
     d = dev()
     K, N, g = wl.K, wl.N, wl.groups
@@ -202,9 +205,11 @@ def test_grouped70b_fullsize():
     dead = torch.empty(g, K, dtype=torch.uint8, device=d)
     status = gq.gptq_prepare(U, wl.percdamp, dead_out=dead, status=status)
     scales = torch.empty(N, device=d)
+    loss = torch.empty(N, device=d)
     Wq = W.clone()
     codes, status = gq.gptq_quantize_layer(Wq, U, wl.bits, wl.blocksize, groups=g, dead=dead,
-                                           scales_out=scales, write_back=True, status=status)
+                                           scales_out=scales, loss=loss, write_back=True,
+                                           status=status)
     gq.raise_on_status(status, "grouped70b")
     torch.cuda.synchronize()
     assert not dead.any().item()
@@ -224,11 +229,24 @@ def test_grouped70b_fullsize():
         r = np.sort(np.union1d(rng.choice(K, 6, replace=False), [0, K // 2, K - 1]))
         Ur = U[gi][torch.as_tensor(r, device=d)].double()
         ident = (Ur @ Hd @ Ur.T).cpu().numpy()
-        del Hd
         assert np.abs(ident - np.eye(len(r))).max() <= TOL_IDENT, np.abs(ident - np.eye(len(r))).max()
         # sampled channels of the group, replayed on the GPU's factor
         ch = gi * per + np.sort(rng.choice(per, 6, replace=False))
         sel = torch.as_tensor(ch, device=d)
+        # reconstruction error of those channels (fp64 on the device): the reported loss,
+        # and against round-to-nearest on the same scales
+        W0 = W[sel].double()
+        sc = scales[sel].double()[:, None]
+        z = 2.0 ** (wl.bits - 1)
+        Dq = W0 - sc * (codes[sel].double() - z)        # the exact grid values, not bf16
+        err_q = 0.5 * ((Dq @ Hd) * Dq).sum(1)
+        Dr = W0 - sc * (torch.clamp(torch.round(W0 / sc), -z, z - 1))
+        err_rtn = 0.5 * ((Dr @ Hd) * Dr).sum(1)
+        del Hd
+        # the same bound as the parity suite's check of this identity (fp32 loss, U to 1e-4)
+        np.testing.assert_allclose(loss[sel].double().cpu().numpy(), err_q.cpu().numpy(),
+                                   rtol=2e-3, atol=0)
+        assert err_q.sum().item() < err_rtn.sum().item(), (err_q.sum().item(), err_rtn.sum().item())
         W64 = W[sel].double().cpu().numpy()
         s64 = scales[sel].double().cpu().numpy()
         np.testing.assert_allclose(s64, O.symmetric_scale(W64, wl.bits)[0], rtol=2e-7)
