@@ -39,7 +39,7 @@ METRIC = "GPTQ layer-solve ms & weights quantized/s (4096×14336, W3); % of TC/H
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the dominant
 # kernel, from an ncu capture of the same 65,536-token launch. Set to None whenever
 # k_gram_tc2 changes until it is captured again.
-GRAM_TRAFFIC_BYTES = 1.588568e9 + 0.504924e9
+GRAM_TRAFFIC_BYTES = 1.568243e9 + 0.498444e9
 GRAM_TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one k_gram_tc2 launch "
                        "(65,536 tokens, K=4096), profiles/gram_tc2_mlp_up_w3_chunk65536.md")
 UNIT = "weights/s"
