@@ -217,6 +217,14 @@ __global__ void __launch_bounds__(GX_THREADS, 1)
             const float *wg = p.w ? p.w + (int64_t)grp * p.ldw : nullptr;
             bool ok = true;
             for (int k = k0; k < k1; ++k) {
+                // this stage's token weights (two distinct tokens per thread), requested
+                // before the wait so that their latency overlaps it
+                float swr[4];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int64_t m = (int64_t)k * GX_BK + (((t + 128 * r) * 16) % GX_BOX) / 128;
+                    swr[r] = (wg && m < p.M) ? wg[m] : 0.f;     // rows past M are zero-filled
+                }
                 if (!tc::mbar_wait(&full[stage], phase, abort)) { ok = false; break; }
                 uint8_t *st = smem + stage * GX_STAGE;
                 const uint4 *s0 = reinterpret_cast<const uint4 *>(st);
@@ -226,9 +234,7 @@ __global__ void __launch_bounds__(GX_THREADS, 1)
                 // 8 KB tile = 512 16-byte units; 4 per thread
 #pragma unroll
                 for (int r = 0; r < 4; ++r) {
-                    const int unit = t + 128 * r;
-                    const int byte = unit * 16;
-                    const int token = (byte % GX_BOX) / 128;      // row inside the box
+                    const int unit = t + 128 * r;    // its token (box row): ((16 unit) % box) / 128
                     const uint4 xa = s0[unit];
                     const __nv_bfloat16 *xv = reinterpret_cast<const __nv_bfloat16 *>(&xa);
                     float a[8];
@@ -238,18 +244,21 @@ __global__ void __launch_bounds__(GX_THREADS, 1)
 #pragma unroll
                         for (int e = 0; e < 8; ++e) a[e] = __bfloat162float(xv[e]) - __bfloat162float(qv[e]);
                     } else {
-                        const int64_t m = (int64_t)k * GX_BK + token;
-                        const float sw = (m < p.M) ? wg[m] : 0.f;   // rows past M are zero-filled
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) a[e] = sw * __bfloat162float(xv[e]);
+                        for (int e = 0; e < 8; ++e) a[e] = swr[r] * __bfloat162float(xv[e]);
                     }
+                    // hi = bf16(a), lo = bf16(a - hi), two values per conversion (the
+                    // one-value conversions saturated the conversion pipe)
                     uint4 ho, lo;
-                    __nv_bfloat16 *hv = reinterpret_cast<__nv_bfloat16 *>(&ho);
-                    __nv_bfloat16 *lv = reinterpret_cast<__nv_bfloat16 *>(&lo);
+                    uint32_t *hw = reinterpret_cast<uint32_t *>(&ho);
+                    uint32_t *lw = reinterpret_cast<uint32_t *>(&lo);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        hv[e] = __float2bfloat16_rn(a[e]);
-                        lv[e] = __float2bfloat16_rn(a[e] - __bfloat162float(hv[e]));
+                    for (int e = 0; e < 4; ++e) {
+                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(a[2 * e], a[2 * e + 1]);
+                        const float2 hf = __bfloat1622float2(h2);
+                        const __nv_bfloat162 l2 = __floats2bfloat162_rn(a[2 * e] - hf.x, a[2 * e + 1] - hf.y);
+                        hw[e] = *reinterpret_cast<const uint32_t *>(&h2);
+                        lw[e] = *reinterpret_cast<const uint32_t *>(&l2);
                     }
                     dhi[unit] = ho;
                     dlo[unit] = lo;
