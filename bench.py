@@ -706,8 +706,10 @@ def run_e2e(args, wl, X, W, dev, gq, torch, dist, world):
     d2h = codes_h.numel() + scales_h.numel() * 4
     return {"value": K * N * world / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            # the copies bound this step: the rate the host-to-device stream achieved
+            "h2d_gbs": h2d / (ms * 1e-3) / 1e9,
             "note": "token stream + W from pinned host each step (copy stream, double-buffered), "
-                    "codes + scales back"}
+                    "codes + scales back; bound by the host-to-device copy of the stream"}
 
 
 def load_peaks():
