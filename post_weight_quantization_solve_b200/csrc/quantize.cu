@@ -737,7 +737,9 @@ size_t quantize_workspace(int K, int N, int g, int blocksize) {
     c.take<float>((size_t)N * K);                           // Wk
     for (int i = 0; i < 2; ++i) c.take<__nv_bfloat16>((size_t)g * K * lay.ldU);   // Uh, Ul
     for (int i = 0; i < 2; ++i) c.take<__nv_bfloat16>((size_t)K * lay.ldU);       // Qh, Ql
-    for (int i = 0; i < 4; ++i) c.take<__nv_bfloat16>((size_t)SUPER * lay.ldE);   // Eh El Ph Pl
+    // Eh El Ph Pl: [SUPER][ldE] for the SIMT sweeps, [ldE][two super-blocks] for the
+    // tensor-core sweep
+    for (int i = 0; i < 4; ++i) c.take<__nv_bfloat16>((size_t)SWEEP_TC_ESTRIDE * lay.ldE);
     c.take<float>((size_t)N);                               // scale
     c.take<float>((size_t)N);                               // loss_acc
     c.take<float>((size_t)g * K);                           // 1 / U_jj (tensor-core sweep)
@@ -814,10 +816,10 @@ static gptq_status quantize_impl(void *W, int wdtype, int N, int K, const float 
     __nv_bfloat16 *Ul = cv.take<__nv_bfloat16>((size_t)groups * K * lay.ldU);
     __nv_bfloat16 *Qh = cv.take<__nv_bfloat16>((size_t)K * lay.ldU);
     __nv_bfloat16 *Ql = cv.take<__nv_bfloat16>((size_t)K * lay.ldU);
-    __nv_bfloat16 *Eh = cv.take<__nv_bfloat16>((size_t)SUPER * lay.ldE);
-    __nv_bfloat16 *El = cv.take<__nv_bfloat16>((size_t)SUPER * lay.ldE);
-    __nv_bfloat16 *Ph = cv.take<__nv_bfloat16>((size_t)SUPER * lay.ldE);
-    __nv_bfloat16 *Pl = cv.take<__nv_bfloat16>((size_t)SUPER * lay.ldE);
+    __nv_bfloat16 *Eh = cv.take<__nv_bfloat16>((size_t)SWEEP_TC_ESTRIDE * lay.ldE);
+    __nv_bfloat16 *El = cv.take<__nv_bfloat16>((size_t)SWEEP_TC_ESTRIDE * lay.ldE);
+    __nv_bfloat16 *Ph = cv.take<__nv_bfloat16>((size_t)SWEEP_TC_ESTRIDE * lay.ldE);
+    __nv_bfloat16 *Pl = cv.take<__nv_bfloat16>((size_t)SWEEP_TC_ESTRIDE * lay.ldE);
     float *scale = cv.take<float>((size_t)N);
     float *loss_acc = cv.take<float>((size_t)N);
     float *rp = cv.take<float>((size_t)groups * K);
@@ -933,36 +935,43 @@ static gptq_status quantize_impl(void *W, int wdtype, int N, int K, const float 
                                 st)) != GPTQ_OK)
             return s;
         const int S = sweep_tc_super(gptaq);
-        // the far update reads the sweep's -E (and V) pairs as channel rows with the
-        // super-block's coordinates contiguous ([ldE][512], 64 x 128 boxes) and adds
+        // the far update reads the sweep's -E (and V) pairs as channel rows with two
+        // super-blocks' coordinates contiguous ([ldE][2 x 512], 64 x 128 boxes) and adds
         static thread_local UpdateMaps kmaps[8];
         for (int gi = 0; gi < groups; ++gi) {
             kmaps[gi] = maps[1][gi];
             __nv_bfloat16 *a_src[4] = {Eh, El, Ph, Pl};
             for (int i = 0; i < 4; ++i)
-                if ((s = make_bf16_map(&kmaps[gi].a[i], a_src[i], SUPER, lay.ldE, SUPER, 128)) != GPTQ_OK)
+                if ((s = make_bf16_map(&kmaps[gi].a[i], a_src[i], SWEEP_TC_ESTRIDE, lay.ldE,
+                                       SWEEP_TC_ESTRIDE, 128)) != GPTQ_OK)
                     return s;
         }
         UpdateParams kbase = base;
         kbase.a_kmajor = 1;
         kbase.neg[0] = 0;
-        for (int sb0 = 0; sb0 < K; sb0 += S) {
+        // Far updates by pairs of super-blocks: after an even super-block only the next
+        // super-block's columns take its errors (the next sweep needs them); after the odd
+        // one, everything after the pair takes both super-blocks' errors as one product
+        // of inner length 2S, so the rest of W is read and written once per pair.
+        int idx = 0;
+        for (int sb0 = 0; sb0 < K; sb0 += S, ++idx) {
             const int sb1 = min(K, sb0 + S);
             if ((s = sweep_tc_launch(*stc, scale, bits, cp, Eh, El, Ph, Pl, lay.ldE, lay.ldG,
                                      loss_acc, status, N, per_group, K, groups, sb0, sb1 - sb0,
-                                     gptaq, cae != 0, st)) != GPTQ_OK)
+                                     (idx & 1) * S, gptaq, cae != 0, st)) != GPTQ_OK)
                 return s;
             if (sb1 >= K) break;
-            for (int gi = 0; gi < groups; ++gi) {      // far: everything after the super-block
+            const bool odd = (idx & 1) != 0;
+            for (int gi = 0; gi < groups; ++gi) {
                 UpdateParams p = kbase;
                 p.C = Wk + (int64_t)gi * per_group * K + sb1;
                 p.c_extent = (int64_t)N * K - (p.C - Wk);
-                p.Ncols = K - sb1;
-                p.L = sb1 - sb0;
+                p.Ncols = odd ? K - sb1 : min(K, sb1 + S) - sb1;
+                p.L = odd ? 2 * S : S;            // every super-block before the last is full
                 p.a_x0 = gi * lay.ldG;
                 p.a_y0 = 0;
                 p.b_x0 = sb1;
-                p.b_y0 = sb0;
+                p.b_y0 = odd ? sb0 - S : sb0;
                 if ((s = launch_update_tc(kmaps[gi], p, 64, st)) != GPTQ_OK) return s;
             }
         }

@@ -49,7 +49,9 @@ constexpr int B_SPLIT = 32 * 1024;          // one split (hi or lo) of the B til
 constexpr int W_SLOT = 128 * 128;           // 128 rows x 32 fp32
 constexpr int D_SLOT = 32 * 128;            // 32 x 32 fp32 diagonal block
 constexpr int R_SLOT = 1024;                // 32 fp32 (1 / U_jj), 1 KB aligned slot
-constexpr int ESTRIDE = 512;                // row pitch of the E / V pairs in global memory
+// row pitch of the E / V pairs in global memory: two super-blocks side by side, so that
+// the far update can take the errors of two consecutive super-blocks as one product
+constexpr int ESTRIDE = 1024;
 constexpr int OFF_A = 0;                                  // [2 slots][hi, lo]
 constexpr int OFF_B = OFF_A + 4 * A_TILE;                 // [hi, lo]
 constexpr int OFF_W = OFF_B + 2 * B_SPLIT;                // [2 slots]
@@ -71,6 +73,7 @@ struct SweepTcParams {
     int N, per_group, K, bits;
     int ldE, ldG;
     int sb0, S;             // super-block origin and length
+    int eoff;               // column of this super-block's errors in the E / V rows
     int vcodes;             // code rows 16-byte aligned (K % 16 == 0)
 };
 
@@ -363,10 +366,10 @@ __global__ void __launch_bounds__(STC_THREADS, 1)
                     }
                     *reinterpret_cast<uint4 *>(ahi + ((c ^ sw) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
                     *reinterpret_cast<uint4 *>(alo + ((c ^ sw) << 4)) = make_uint4(l[0], l[1], l[2], l[3]);
-                    if (valid && GQ_IN_BOUNDS(p.status, ecol * ESTRIDE + 32 * q + 8 * c + 8 <= (int64_t)p.ldE * ESTRIDE,
-                                              BS_SWEEP_OUT, ecol * ESTRIDE + 32 * q + 8 * c)) {
+                    if (valid && GQ_IN_BOUNDS(p.status, ecol * ESTRIDE + p.eoff + 32 * q + 8 * c + 8 <= (int64_t)p.ldE * ESTRIDE,
+                                              BS_SWEEP_OUT, ecol * ESTRIDE + p.eoff + 32 * q + 8 * c)) {
                         // the far update's copy: -E, this channel's row
-                        const int64_t eo = ecol * ESTRIDE + 32 * q + 8 * c;
+                        const int64_t eo = ecol * ESTRIDE + p.eoff + 32 * q + 8 * c;
                         *reinterpret_cast<uint4 *>(p.Eh + eo) = make_uint4(h[0], h[1], h[2], h[3]);
                         *reinterpret_cast<uint4 *>(p.El + eo) = make_uint4(l[0], l[1], l[2], l[3]);
                     }
@@ -382,9 +385,9 @@ __global__ void __launch_bounds__(STC_THREADS, 1)
                         }
                         *reinterpret_cast<uint4 *>(ahi + (((4 + c) ^ sw) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
                         *reinterpret_cast<uint4 *>(alo + (((4 + c) ^ sw) << 4)) = make_uint4(l[0], l[1], l[2], l[3]);
-                        if (valid && GQ_IN_BOUNDS(p.status, ecol * ESTRIDE + 32 * q + 8 * c + 8 <= (int64_t)p.ldE * ESTRIDE,
-                                                  BS_SWEEP_OUT, ecol * ESTRIDE + 32 * q + 8 * c)) {
-                            const int64_t eo = ecol * ESTRIDE + 32 * q + 8 * c;
+                        if (valid && GQ_IN_BOUNDS(p.status, ecol * ESTRIDE + p.eoff + 32 * q + 8 * c + 8 <= (int64_t)p.ldE * ESTRIDE,
+                                                  BS_SWEEP_OUT, ecol * ESTRIDE + p.eoff + 32 * q + 8 * c)) {
+                            const int64_t eo = ecol * ESTRIDE + p.eoff + 32 * q + 8 * c;
                             *reinterpret_cast<uint4 *>(p.Ph + eo) = make_uint4(h[0], h[1], h[2], h[3]);
                             *reinterpret_cast<uint4 *>(p.Pl + eo) = make_uint4(l[0], l[1], l[2], l[3]);
                         }
@@ -507,10 +510,11 @@ gptq_status sweep_tc_setup(SweepTcMaps *maps, float *Wk, const float *W0k, const
 gptq_status sweep_tc_launch(const SweepTcMaps &maps, const float *scale, int bits, uint8_t *codes,
                             __nv_bfloat16 *Eh, __nv_bfloat16 *El, __nv_bfloat16 *Ph,
                             __nv_bfloat16 *Pl, int ldE, int ldG, float *loss_acc, int32_t *status,
-                            int N, int per_group, int K, int groups, int sb0, int S, bool gptaq,
-                            bool cae, cudaStream_t st) {
+                            int N, int per_group, int K, int groups, int sb0, int S, int eoff,
+                            bool gptaq, bool cae, cudaStream_t st) {
     // the B tile holds at most 8 (plain) or 4 (GPTAQ, twice as deep) 64-column chunks
     if (S < 1 || S > sweep_tc_super(gptaq) || sb0 % 64 != 0 || sb0 + S > K) return GPTQ_ERR_ARG;
+    if (eoff < 0 || eoff % 32 != 0 || eoff + 32 * ((S + 31) / 32) > ESTRIDE) return GPTQ_ERR_ARG;
     SweepTcParams p;
     p.scale = scale;
     p.codes = codes;
@@ -520,6 +524,7 @@ gptq_status sweep_tc_launch(const SweepTcMaps &maps, const float *scale, int bit
     p.N = N; p.per_group = per_group; p.K = K; p.bits = bits;
     p.ldE = ldE; p.ldG = ldG;
     p.sb0 = sb0; p.S = S;
+    p.eoff = eoff;
     p.vcodes = (K % 16 == 0 && aligned(codes, 16)) ? 1 : 0;
     const dim3 grid((per_group + STC_CH - 1) / STC_CH, groups);
     typedef void (*Kern)(const SweepTcMaps, const SweepTcParams);

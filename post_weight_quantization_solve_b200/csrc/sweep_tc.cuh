@@ -27,11 +27,13 @@ gptq_status sweep_tc_setup(SweepTcMaps *maps, float *Wk, const float *W0k, const
                            const __nv_bfloat16 *Qh, const __nv_bfloat16 *Ql, int ldU, float *rp,
                            int N, int K, int g, cudaStream_t st);
 // One super-block [sb0, sb0 + S) for every channel: codes, loss, and the E (and V) pairs
-// of the super-block for the far update.
+// of the super-block for the far update, at columns [eoff, eoff + S) of the channel rows.
 gptq_status sweep_tc_launch(const SweepTcMaps &maps, const float *scale, int bits, uint8_t *codes,
                             __nv_bfloat16 *Eh, __nv_bfloat16 *El, __nv_bfloat16 *Ph,
                             __nv_bfloat16 *Pl, int ldE, int ldG, float *loss_acc, int32_t *status,
-                            int N, int per_group, int K, int groups, int sb0, int S, bool gptaq,
-                            bool cae, cudaStream_t st);
+                            int N, int per_group, int K, int groups, int sb0, int S, int eoff,
+                            bool gptaq, bool cae, cudaStream_t st);
+// Row pitch of the E / V pair rows the sweep writes (elements): two super-blocks.
+constexpr int SWEEP_TC_ESTRIDE = 1024;
 
 }  // namespace gptq
