@@ -40,6 +40,7 @@
 
 #include "common.cuh"
 #include "sweep_tc.cuh"
+#include "update_plan.h"
 #include "update_tc.cuh"
 
 namespace gptq {
@@ -949,30 +950,32 @@ static gptq_status quantize_impl(void *W, int wdtype, int N, int K, const float 
         UpdateParams kbase = base;
         kbase.a_kmajor = 1;
         kbase.neg[0] = 0;
-        // Far updates by pairs of super-blocks: after an even super-block only the next
-        // super-block's columns take its errors (the next sweep needs them); after the odd
-        // one, everything after the pair takes both super-blocks' errors as one product
-        // of inner length 2S, so the rest of W is read and written once per pair.
-        int idx = 0;
-        for (int sb0 = 0; sb0 < K; sb0 += S, ++idx) {
+        // Far updates by pairs of super-blocks (update_plan.h): after an even super-block
+        // only the next super-block's columns take its errors (the next sweep needs them);
+        // after the odd one, everything after the pair takes both super-blocks' errors as
+        // one product of inner length 2S, so the rest of W is read and written once per pair.
+        const std::vector<FarUpdate> plan = far_update_plan(K, S);
+        size_t next = 0;
+        for (int idx = 0, sb0 = 0; sb0 < K; sb0 += S, ++idx) {
             const int sb1 = min(K, sb0 + S);
             if ((s = sweep_tc_launch(*stc, scale, bits, cp, Eh, El, Ph, Pl, lay.ldE, lay.ldG,
                                      loss_acc, status, N, per_group, K, groups, sb0, sb1 - sb0,
-                                     (idx & 1) * S, gptaq, cae != 0, st)) != GPTQ_OK)
+                                     sweep_error_column(idx, S), gptaq, cae != 0, st)) != GPTQ_OK)
                 return s;
-            if (sb1 >= K) break;
-            const bool odd = (idx & 1) != 0;
-            for (int gi = 0; gi < groups; ++gi) {
-                UpdateParams p = kbase;
-                p.C = Wk + (int64_t)gi * per_group * K + sb1;
-                p.c_extent = (int64_t)N * K - (p.C - Wk);
-                p.Ncols = odd ? K - sb1 : min(K, sb1 + S) - sb1;
-                p.L = odd ? 2 * S : S;            // every super-block before the last is full
-                p.a_x0 = gi * lay.ldG;
-                p.a_y0 = 0;
-                p.b_x0 = sb1;
-                p.b_y0 = odd ? sb0 - S : sb0;
-                if ((s = launch_update_tc(kmaps[gi], p, 64, st)) != GPTQ_OK) return s;
+            for (; next < plan.size() && plan[next].after == idx; ++next) {
+                const FarUpdate &u = plan[next];
+                for (int gi = 0; gi < groups; ++gi) {
+                    UpdateParams p = kbase;
+                    p.C = Wk + (int64_t)gi * per_group * K + u.col0;
+                    p.c_extent = (int64_t)N * K - (p.C - Wk);
+                    p.Ncols = u.col1 - u.col0;
+                    p.L = u.k1 - u.k0;
+                    p.a_x0 = gi * lay.ldG;
+                    p.a_y0 = 0;                   // E column of coordinate k0
+                    p.b_x0 = u.col0;
+                    p.b_y0 = u.k0;
+                    if ((s = launch_update_tc(kmaps[gi], p, 64, st)) != GPTQ_OK) return s;
+                }
             }
         }
     } else {
