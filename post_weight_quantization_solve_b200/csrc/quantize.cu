@@ -19,15 +19,18 @@
 // After each block the rest of its super-block is updated ("near" update); after
 // each super-block the coordinates beyond it ("far" update, inner length S). Both
 // are tensor-core products (update_tc.cu); the blocking changes only the order of
-// the work, and the far traffic drops by S / B.
+// the work, and the far traffic drops by S / B. The tensor-core sweep (sweep_tc.cu)
+// keeps the near updates in TMEM and runs the far updates by pairs of super-blocks
+// (update_plan.h: inner length 2S after every second super-block).
 //
 // Layout on the device:
 //   Wk        fp32 [N][K] working weights (dead coordinates zeroed)
-//   Eh, El    bf16 [S][ldE] normalised errors of the super-block as hi + lo pairs,
-//             row j - sb0, column grp * ldG + local channel (channel fastest, so the
-//             sweep's stores coalesce; the update reads it as an MN-major operand)
-//   Ph, Pl    bf16 [S][ldE] pre-rounding weights (GPTAQ; with CAE the starting
-//             weights), same layout
+//   Eh, El    bf16 normalised errors as hi + lo pairs. SIMT sweeps: [S][ldE], row
+//             j - sb0, column grp * ldG + local channel (channel fastest, so their stores
+//             coalesce; the update reads it as an MN-major operand). Tensor-core sweep:
+//             [ldE][1024], a channel's row holding two super-blocks (columns 0 and S),
+//             read by the update as a K-major operand.
+//   Ph, Pl    pre-rounding weights (GPTAQ; with CAE the starting weights), same layouts
 //   W0k       fp32 [N][K] starting weights w^(0) (CAE only)
 //   Uh, Ul    bf16 [g][K][ldU] U as hi + lo pairs;  Qh, Ql  the same for P1
 // The sweep keeps each channel's block coordinates in registers: one thread per
