@@ -557,7 +557,9 @@ def run_ours(args, rank, world, local_rank):
                  "frac_of_hbm": (round(pack_bytes / (pack_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)
                                  if peaks.get("hbm_gbs") else None),
                  "note": "codes N x K bytes in + packed words out, 10 launches after the timed "
-                         "steps, not part of the step"},
+                         "steps, not part of the step; issued back to back from Python, so the "
+                         "host's launch rate can bound this figure (the kernel alone: "
+                         "profiles/pack_mlp_up_w3_N14336_K4096.md)"},
         "gpu_launches": int(launches),
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                    "reasons": clocks["reasons"]},
